@@ -1,0 +1,678 @@
+/*
+ * sq_oracle.c -- plain, slow, scalar CPU oracle for the SquareQ W4 linear
+ * layer.  TEST INFRASTRUCTURE ONLY: the parity tests, the smoke check and the
+ * bench's CPU-baseline leg call it; the product (libsq, the CUDA path) never
+ * links, imports or executes anything here, and this file shares no code,
+ * header, table or constant with it.
+ *
+ * What it computes (SquareQ README, section "SquareQ v3 -- W4 (Hadamard-256 +
+ * low-rank + int4 / NVFP4)"):
+ *
+ *     W = lora_up . lora_down^T + inverse_H256( dequant( residual ) )
+ *
+ * with a block-diagonal normalised Hadamard-256 over the input dim
+ * ("Rotation" paragraph), an int4 group-32 codec with MSE-swept scale
+ * fractions or an NVFP4 codec (e2m1 codes, ue4m3 block-16 scales in the
+ * cuBLASLt tiled layout, fp32 per-tensor global scale) ("Residual codecs"
+ * paragraph), and a rank-32 bf16 low-rank branch ("Low-rank branch").
+ *
+ * Arithmetic rules (the pages fix none of them; these are the readings that
+ * make bit-exact parity well defined):
+ *   - fp32 values are IEEE binary32, one round-to-nearest-even per operation,
+ *     and no contraction into FMA (build with -ffp-contract=off, no
+ *     -ffast-math) except where fmaf() is written;
+ *   - every narrowing conversion (bf16, fp16, ue4m3, e2m1) is round to nearest,
+ *     ties to even, through one routine, round_to_grid(), written from the
+ *     formats' definitions;
+ *   - forward outputs are evaluated in fp64 on the exact decoded operands.
+ *
+ * OpenMP only spreads independent rows / groups over threads; each output is
+ * still computed by one thread in the order written here.
+ */
+#include <math.h>
+#include <stdint.h>
+#include <string.h>
+#include <stdlib.h>
+#ifdef _OPENMP
+#include <omp.h>
+#endif
+
+int or_num_threads(void)
+{
+#ifdef _OPENMP
+    return omp_get_max_threads();
+#else
+    return 1;
+#endif
+}
+
+/* ------------------------------------------------------------------------ */
+/* Rounding to a small floating-point grid                                   */
+/* ------------------------------------------------------------------------ */
+
+/*
+ * Round a non-negative finite value a to the nearest value of a binary
+ * floating-point grid with `mant_bits` fraction bits whose smallest normal
+ * exponent is `emin` (below 2^emin the spacing is fixed at 2^(emin-mant_bits),
+ * i.e. gradual underflow).  Ties go to the even multiple of the spacing, which
+ * is the value whose last fraction bit is 0.  No upper limit is applied here.
+ * The input is a float widened to double, so a / spacing is exact.
+ */
+static double round_to_grid(double a, int mant_bits, int emin)
+{
+    int E;
+    if (a == 0.0)
+        return 0.0;
+    if (a < ldexp(1.0, emin)) {
+        E = emin;
+    } else {
+        int ex;
+        (void)frexp(a, &ex);     /* a = m * 2^ex, m in [0.5, 1) */
+        E = ex - 1;              /* 2^E <= a < 2^(E+1) */
+    }
+    double spacing = ldexp(1.0, E - mant_bits);
+    return nearbyint(a / spacing) * spacing;   /* default mode: ties to even */
+}
+
+/* exponent E with 2^E <= v < 2^(E+1), for v > 0 */
+static int floor_log2(double v)
+{
+    int ex;
+    (void)frexp(v, &ex);
+    return ex - 1;
+}
+
+/* bf16: 7 fraction bits, fp32's exponent range (emin = -126). */
+uint16_t or_f32_to_bf16(float v)
+{
+    uint32_t bits;
+    memcpy(&bits, &v, 4);
+    uint16_t sign = (uint16_t)((bits >> 16) & 0x8000u);
+    if (isnan(v))
+        return (uint16_t)(sign | 0x7FC0u);
+    if (isinf(v))
+        return (uint16_t)(sign | 0x7F80u);
+    double r = round_to_grid(fabs((double)v), 7, -126);
+    if (r >= ldexp(1.0, 128))
+        return (uint16_t)(sign | 0x7F80u);            /* overflow -> inf */
+    float rf = (float)r;                               /* exact: r is on the bf16 grid */
+    uint32_t rb;
+    memcpy(&rb, &rf, 4);
+    return (uint16_t)(sign | (rb >> 16));
+}
+
+float or_bf16_to_f32(uint16_t h)
+{
+    uint32_t bits = (uint32_t)h << 16;
+    float v;
+    memcpy(&v, &bits, 4);
+    return v;
+}
+
+/* IEEE binary16: 10 fraction bits, emin = -14, largest finite 65504. */
+uint16_t or_f32_to_f16(float v)
+{
+    uint16_t sign = signbit(v) ? 0x8000u : 0u;
+    if (isnan(v))
+        return (uint16_t)(sign | 0x7E00u);
+    if (isinf(v))
+        return (uint16_t)(sign | 0x7C00u);
+    double r = round_to_grid(fabs((double)v), 10, -14);
+    if (r > 65504.0)
+        return (uint16_t)(sign | 0x7C00u);            /* overflow -> inf */
+    if (r == 0.0)
+        return sign;
+    if (r < ldexp(1.0, -14))                           /* subnormal: r = m * 2^-24 */
+        return (uint16_t)(sign | (uint16_t)(r / ldexp(1.0, -24)));
+    int E = floor_log2(r);
+    uint32_t mant = (uint32_t)(r / ldexp(1.0, E - 10)) - 1024u;
+    return (uint16_t)(sign | ((uint32_t)(E + 15) << 10) | mant);
+}
+
+float or_f16_to_f32(uint16_t h)
+{
+    int sign = (h >> 15) & 1;
+    int e = (h >> 10) & 31;
+    int m = h & 1023;
+    double v;
+    if (e == 0)
+        v = ldexp((double)m, -24);
+    else if (e == 31)
+        v = m ? NAN : INFINITY;
+    else
+        v = ldexp(1024.0 + m, e - 15 - 10);
+    return (float)(sign ? -v : v);
+}
+
+/*
+ * Unsigned e4m3 ("ue4m3") block scale: 4 exponent bits (bias 7), 3 fraction
+ * bits, smallest normal 2^-6, spacing 2^-9 below it, largest finite 448
+ * (code 0x7E; 0x7F is NaN).  Conversion is round-to-nearest-even with
+ * saturation to 448 ("satfinite").  The input must be >= 0 or NaN.
+ */
+uint8_t or_f32_to_ue4m3(float v)
+{
+    if (isnan(v))
+        return 0x7Fu;
+    if (!(v > 0.0f))
+        return 0x00u;
+    double r = isinf(v) ? 448.0 : round_to_grid((double)v, 3, -6);
+    if (r > 448.0)
+        r = 448.0;
+    if (r == 0.0)
+        return 0x00u;
+    if (r < ldexp(1.0, -6))
+        return (uint8_t)(r / ldexp(1.0, -9));        /* codes 1..7 */
+    int E = floor_log2(r);
+    uint32_t mant = (uint32_t)(r / ldexp(1.0, E - 3)) - 8u;
+    return (uint8_t)(((uint32_t)(E + 7) << 3) | mant);
+}
+
+float or_ue4m3_to_f32(uint8_t c)
+{
+    int e = (c >> 3) & 15;
+    int m = c & 7;
+    if (c == 0x7F || c == 0xFF)
+        return NAN;
+    if (e == 0)
+        return (float)ldexp((double)m, -9);
+    return (float)ldexp(8.0 + m, e - 7 - 3);
+}
+
+/*
+ * e2m1 (FP4): sign bit, 2 exponent bits (bias 1), 1 fraction bit.
+ * Magnitudes {0, 0.5, 1, 1.5, 2, 3, 4, 6} for codes 0..7.  Conversion is
+ * round-to-nearest-even with saturation to 6; the sign bit is kept, so a
+ * negative value that rounds to zero gives code 0x8.
+ */
+uint8_t or_f32_to_e2m1(float v)
+{
+    static const double grid[8] = {0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0};
+    uint8_t sign = signbit(v) ? 0x8u : 0x0u;
+    double a = fabs((double)v);
+    double r = isinf(v) ? 6.0 : round_to_grid(a, 1, 0);
+    if (r > 6.0)
+        r = 6.0;
+    for (uint8_t c = 0; c < 8; c++)
+        if (grid[c] == r)
+            return (uint8_t)(sign | c);
+    return (uint8_t)(sign | 0x7u);   /* unreachable for finite inputs */
+}
+
+float or_e2m1_to_f32(uint8_t c)
+{
+    static const float mag[8] = {0.0f, 0.5f, 1.0f, 1.5f, 2.0f, 3.0f, 4.0f, 6.0f};
+    float v = mag[c & 7];
+    return (c & 8) ? -v : v;
+}
+
+/* ------------------------------------------------------------------------ */
+/* O1, O2: block-diagonal normalised Hadamard-256 over the input dim         */
+/* ------------------------------------------------------------------------ */
+
+/*
+ * In-place normalised Hadamard transform of 256 values (SquareQ README,
+ * "Rotation" paragraph: block-diagonal normalised Hadamard-256).  Reading:
+ * Sylvester ordering, H[i][j] = (-1)^popcount(i & j) / 16, evaluated as
+ * radix-2 butterflies with strides 1, 2, 4, ..., 128 (each butterfly writes
+ * a+b to the lower and a-b to the upper index), then a scale by 1/16, which
+ * is exact in binary.  H is symmetric and orthogonal, so it is its own
+ * inverse: the same routine serves as inverse_H256.
+ */
+void or_fwht256(float *v)
+{
+    for (int h = 1; h < 256; h <<= 1) {
+        for (int j = 0; j < 256; j++) {
+            if ((j & h) == 0) {
+                float a = v[j];
+                float b = v[j + h];
+                v[j] = a + b;
+                v[j + h] = a - b;
+            }
+        }
+    }
+    for (int j = 0; j < 256; j++)
+        v[j] = v[j] * 0.0625f;
+}
+
+/* Rotate every 256-wide block of every row of a [rows, K] fp32 matrix. */
+void or_rotate_rows_f32(const float *in, int64_t rows, int64_t K, float *out)
+{
+#pragma omp parallel for schedule(static)
+    for (int64_t r = 0; r < rows; r++) {
+        for (int64_t b = 0; b < K; b += 256) {
+            float v[256];
+            for (int i = 0; i < 256; i++)
+                v[i] = in[r * K + b + i];
+            or_fwht256(v);
+            for (int i = 0; i < 256; i++)
+                out[r * K + b + i] = v[i];
+        }
+    }
+}
+
+/* Same for a bf16 matrix (bit patterns); bf16 widens to fp32 exactly. */
+void or_rotate_rows_bf16(const uint16_t *in, int64_t rows, int64_t K, float *out)
+{
+#pragma omp parallel for schedule(static)
+    for (int64_t r = 0; r < rows; r++) {
+        for (int64_t b = 0; b < K; b += 256) {
+            float v[256];
+            for (int i = 0; i < 256; i++)
+                v[i] = or_bf16_to_f32(in[r * K + b + i]);
+            or_fwht256(v);
+            for (int i = 0; i < 256; i++)
+                out[r * K + b + i] = v[i];
+        }
+    }
+}
+
+/* ------------------------------------------------------------------------ */
+/* O3: int4 group-32 codec with an MSE-swept scale fraction                  */
+/* ------------------------------------------------------------------------ */
+
+/*
+ * Fraction j of the sweep: f_j = (50 + 2 j) / 100, j = 0..25, correctly
+ * rounded to fp32 (IEEE division of two exact values).
+ */
+float or_int4_fraction(int j)
+{
+    return (float)(50 + 2 * j) / 100.0f;
+}
+
+/*
+ * One group of 32 rotated residual values (SquareQ README, "Residual codecs":
+ * int4 group-32 scales with MSE-swept fractions).  For each fraction f_j the
+ * scale is s = fp16(RN(RN(f_j * a) / 7)), a = max|r_i|, and the codes are
+ * q_i = clamp(rint_even(RN(r_i * RN(1/s))), -7, 7); the group's squared error
+ * sum_i RN((r_i - q_i s)^2) is accumulated by an xor butterfly over the 32
+ * lanes (strides 16, 8, 4, 2, 1; lane 0's value is the result).  A scale that
+ * rounds to 0 gives q = 0 and error r_i.  The smallest error wins; on a tie the
+ * smaller fraction wins.  Outputs: 32 codes in [-7, 7], the fp16 scale bits,
+ * the winning j.
+ */
+void or_int4_group32(const float *r, int8_t *q_out, uint16_t *s_out, uint8_t *j_out)
+{
+    float a = 0.0f;
+    for (int i = 0; i < 32; i++) {
+        float m = fabsf(r[i]);
+        if (m > a)
+            a = m;
+    }
+    float best = INFINITY;
+    int best_j = -1;
+    for (int j = 0; j < 26; j++) {
+        float f = or_int4_fraction(j);
+        float fa = f * a;
+        float s7 = fa / 7.0f;
+        uint16_t sh = or_f32_to_f16(s7);
+        float s = or_f16_to_f32(sh);
+        int8_t q[32];
+        float p[32];
+        if (s == 0.0f) {
+            for (int i = 0; i < 32; i++) {
+                q[i] = 0;
+                p[i] = r[i] * r[i];
+            }
+        } else {
+            float inv = 1.0f / s;
+            for (int i = 0; i < 32; i++) {
+                float v = r[i] * inv;
+                float rq = nearbyintf(v);
+                if (rq > 7.0f)
+                    rq = 7.0f;
+                if (rq < -7.0f)
+                    rq = -7.0f;
+                q[i] = (int8_t)rq;
+                float qs = rq * s;              /* exact: <= 14 significant bits */
+                float e = r[i] - qs;
+                p[i] = e * e;
+            }
+        }
+        for (int d = 16; d >= 1; d >>= 1) {
+            float nxt[32];
+            for (int i = 0; i < 32; i++)
+                nxt[i] = p[i] + p[i ^ d];
+            memcpy(p, nxt, sizeof(p));
+        }
+        float mse = p[0];
+        if (best_j < 0 || mse < best) {
+            best = mse;
+            best_j = j;
+            memcpy(q_out, q, 32);
+            *s_out = sh;
+        }
+    }
+    *j_out = (uint8_t)best_j;
+}
+
+/*
+ * int4 builder: rotate R [N, K] fp32 row-blockwise, then run the group codec
+ * on every 32 consecutive rotated values of a row.  codes [N, K/2]: element
+ * 2k in the low nibble, 4-bit two's complement; scales [N, K/32] fp16 bits;
+ * frac [N, K/32] winning j (may be NULL).
+ */
+void or_build_int4(const float *R, int64_t N, int64_t K,
+                   uint8_t *codes, uint16_t *scales, uint8_t *frac)
+{
+#pragma omp parallel for schedule(static)
+    for (int64_t n = 0; n < N; n++) {
+        for (int64_t b = 0; b < K; b += 256) {
+            float v[256];
+            for (int i = 0; i < 256; i++)
+                v[i] = R[n * K + b + i];
+            or_fwht256(v);
+            for (int g = 0; g < 8; g++) {
+                int8_t q[32];
+                uint16_t s;
+                uint8_t j;
+                or_int4_group32(v + 32 * g, q, &s, &j);
+                int64_t gi = n * (K / 32) + (b / 32) + g;
+                scales[gi] = s;
+                if (frac)
+                    frac[gi] = j;
+                for (int i = 0; i < 32; i += 2) {
+                    uint8_t lo = (uint8_t)q[i] & 0xFu;
+                    uint8_t hi = (uint8_t)q[i + 1] & 0xFu;
+                    codes[n * (K / 2) + (b + 32 * g + i) / 2] = (uint8_t)(lo | (hi << 4));
+                }
+            }
+        }
+    }
+}
+
+/* ------------------------------------------------------------------------ */
+/* O4, O5: NVFP4 codec and the tiled scale-factor layout                     */
+/* ------------------------------------------------------------------------ */
+
+/*
+ * Byte offset of scale (row r, scale column c) in the tiled layout, C = K/16
+ * scale columns per row (a multiple of 4).  The pages name "the cuBLASLt tiled
+ * layout" without printing it; this is the publicly documented 1D
+ * block-scaling layout: 128-row x 4-column tiles of 512 bytes, tiles ordered
+ * along the scale columns first, and inside a tile row r%32 picks a 16-byte
+ * line, (r%128)/32 a 4-byte word in it and c%4 the byte.
+ */
+int64_t or_sf_offset(int64_t r, int64_t c, int64_t C)
+{
+    return ((r / 128) * (C / 4) + c / 4) * 512 + (r % 32) * 16 + ((r % 128) / 32) * 4 + (c % 4);
+}
+
+/* bytes of a tiled scale buffer for `rows` rows of K elements */
+int64_t or_sf_bytes(int64_t rows, int64_t K)
+{
+    return ((rows + 127) / 128) * 128 * (K / 16);
+}
+
+/* Global scale g = RN(A / (6 * 448)) from the rotated tensor's absmax A. */
+float or_nvfp4_global_scale(float A)
+{
+    return A / 2688.0f;
+}
+
+/*
+ * One block of 16 rotated values with global scale g (SquareQ README,
+ * "Residual codecs": e2m1 + ue4m3 block-16 scales + per-tensor global scale).
+ * b = max|r|, sf = ue4m3(RN(b / RN(6 g))); with den = RN(value(sf) * g) the
+ * codes are e2m1(RN(r_i * RN(1/den))).  sf == 0 or g == 0 gives all-zero
+ * codes.  codes8 gets 8 bytes, element 2k in the low nibble.
+ */
+void or_nvfp4_block16(const float *r, float g, uint8_t *codes8, uint8_t *sf_out)
+{
+    float b = 0.0f;
+    for (int i = 0; i < 16; i++) {
+        float m = fabsf(r[i]);
+        if (m > b)
+            b = m;
+    }
+    uint8_t sf = 0;
+    uint8_t c[16];
+    memset(c, 0, sizeof(c));
+    if (g != 0.0f) {
+        float sixg = 6.0f * g;
+        float ratio = b / sixg;
+        sf = or_f32_to_ue4m3(ratio);
+        if (sf != 0) {
+            float dec = or_ue4m3_to_f32(sf);
+            float den = dec * g;
+            float inv = 1.0f / den;
+            for (int i = 0; i < 16; i++)
+                c[i] = or_f32_to_e2m1(r[i] * inv);
+        }
+    }
+    for (int i = 0; i < 8; i++)
+        codes8[i] = (uint8_t)(c[2 * i] | (c[2 * i + 1] << 4));
+    *sf_out = sf;
+}
+
+/*
+ * Quantise an already rotated [rows, K] fp32 matrix with global scale g.
+ * codes [rows, K/2]; sf_tiled gets or_sf_bytes(rows, K) bytes in the tiled
+ * layout, padding rows zero.
+ */
+void or_nvfp4_quant_rotated(const float *rot, int64_t rows, int64_t K, float g,
+                            uint8_t *codes, uint8_t *sf_tiled)
+{
+    int64_t C = K / 16;
+    memset(sf_tiled, 0, (size_t)or_sf_bytes(rows, K));
+#pragma omp parallel for schedule(static)
+    for (int64_t r = 0; r < rows; r++) {
+        for (int64_t c = 0; c < C; c++) {
+            uint8_t sf;
+            or_nvfp4_block16(rot + r * K + 16 * c, g, codes + r * (K / 2) + 8 * c, &sf);
+            sf_tiled[or_sf_offset(r, c, C)] = sf;
+        }
+    }
+}
+
+static float absmax_f32(const float *v, int64_t n)
+{
+    float a = 0.0f;
+    for (int64_t i = 0; i < n; i++) {
+        float m = fabsf(v[i]);
+        if (m > a)
+            a = m;
+    }
+    return a;
+}
+
+/*
+ * NVFP4 builder: rotate R, A = max|rotated R|, g_w = RN(A / 2688), then the
+ * block codec.  `rot_scratch` holds N*K floats (caller-owned).
+ */
+void or_build_nvfp4(const float *R, int64_t N, int64_t K, float *rot_scratch,
+                    uint8_t *codes, uint8_t *sf_tiled, float *g_out)
+{
+    or_rotate_rows_f32(R, N, K, rot_scratch);
+    float A = absmax_f32(rot_scratch, N * K);
+    float g = or_nvfp4_global_scale(A);
+    or_nvfp4_quant_rotated(rot_scratch, N, K, g, codes, sf_tiled);
+    *g_out = g;
+}
+
+/*
+ * O6 activation quantisation: rotate x [M, K] bf16, g_x = RN(max|xr| / 2688)
+ * unless `static_g` is set (then *g_inout is used as given), block codec, and
+ * the low-rank input t[m, r] = sum_k x[m, k] * lora_down[k, r] in fp64
+ * (lora_down [K, 32] bf16; t may be NULL).  `rot_scratch` holds M*K floats.
+ */
+void or_act_quant_nvfp4(const uint16_t *x, int64_t M, int64_t K, int static_g,
+                        float *g_inout, float *rot_scratch,
+                        uint8_t *codes, uint8_t *sf_tiled,
+                        const uint16_t *lora_down, double *t)
+{
+    or_rotate_rows_bf16(x, M, K, rot_scratch);
+    float g = *g_inout;
+    if (!static_g)
+        g = or_nvfp4_global_scale(absmax_f32(rot_scratch, M * K));
+    or_nvfp4_quant_rotated(rot_scratch, M, K, g, codes, sf_tiled);
+    *g_inout = g;
+    if (t) {
+#pragma omp parallel for schedule(static)
+        for (int64_t m = 0; m < M; m++) {
+            for (int rr = 0; rr < 32; rr++) {
+                double acc = 0.0;
+                for (int64_t k = 0; k < K; k++)
+                    acc += (double)or_bf16_to_f32(x[m * K + k]) *
+                           (double)or_bf16_to_f32(lora_down[k * 32 + rr]);
+                t[m * 32 + rr] = acc;
+            }
+        }
+    }
+}
+
+/* ------------------------------------------------------------------------ */
+/* O7, O8: forward y = x . W^T                                              */
+/* ------------------------------------------------------------------------ */
+
+/*
+ * Since W = U D^T + H(deq(Q)) and H is symmetric, y = x W^T =
+ * H(x) deq(Q)^T + (x D) U^T: the rotation moves onto the activation
+ * (SquareQ README, "Op-level parity of the full FP4 forward": rotate, block
+ * quant, tiled scales, GEMM, epilogue).
+ *
+ * NVFP4 forward, fp64 on the exact decoded operands:
+ *   y[m,n] = g_x g_w sum_k e2m1(xc[m,k]) sf_x(m,k/16) e2m1(wc[n,k]) sf_w(n,k/16)
+ *            + sum_r t[m,r] U[n,r]
+ * Only the rows listed in `rows` (n_rows of them) are evaluated; y is
+ * [n_rows, N].  t is [M, 32] fp64 (or NULL for no low-rank term), U [N, 32]
+ * bf16 bits.
+ */
+void or_linear_fwd_nvfp4(const uint8_t *xc, const uint8_t *xsf, float g_x,
+                         const uint8_t *wc, const uint8_t *wsf, float g_w,
+                         const double *t, const uint16_t *U,
+                         int64_t M, int64_t N, int64_t K,
+                         const int64_t *rows, int64_t n_rows, double *y)
+{
+    int64_t C = K / 16;
+    (void)M;
+    /* decoded activation rows, e2m1 * sf (exact in fp64) */
+    double *xd = (double *)malloc((size_t)(n_rows * K) * sizeof(double));
+    for (int64_t i = 0; i < n_rows; i++) {
+        int64_t m = rows[i];
+        for (int64_t k = 0; k < K; k++) {
+            uint8_t byte = xc[m * (K / 2) + k / 2];
+            uint8_t code = (k & 1) ? (byte >> 4) : (byte & 0xF);
+            xd[i * K + k] = (double)or_e2m1_to_f32(code) *
+                            (double)or_ue4m3_to_f32(xsf[or_sf_offset(m, k / 16, C)]);
+        }
+    }
+#pragma omp parallel for schedule(static)
+    for (int64_t n = 0; n < N; n++) {
+        double *wd = (double *)malloc((size_t)K * sizeof(double));
+        for (int64_t k = 0; k < K; k++) {
+            uint8_t byte = wc[n * (K / 2) + k / 2];
+            uint8_t code = (k & 1) ? (byte >> 4) : (byte & 0xF);
+            wd[k] = (double)or_e2m1_to_f32(code) *
+                    (double)or_ue4m3_to_f32(wsf[or_sf_offset(n, k / 16, C)]);
+        }
+        for (int64_t i = 0; i < n_rows; i++) {
+            int64_t m = rows[i];
+            double acc = 0.0;
+            for (int64_t k = 0; k < K; k++)
+                acc += xd[i * K + k] * wd[k];
+            double out = (double)g_x * (double)g_w * acc;
+            if (t)
+                for (int r = 0; r < 32; r++)
+                    out += t[m * 32 + r] * (double)or_bf16_to_f32(U[n * 32 + r]);
+            y[i * N + n] = out;
+        }
+        free(wd);
+    }
+    free(xd);
+}
+
+/*
+ * int4 forward ("dequant-first"), fp64 on the exact operands:
+ *   xb = bf16(H(x)),  wb[n,k] = bf16(q[n,k] * s[n,k/32]),
+ *   y[m,n] = sum_k xb wb + sum_r t[m,r] U[n,r].
+ * xrot is the fp32 rotated x [M, K]; codes/scales as or_build_int4 writes.
+ */
+void or_linear_fwd_int4(const float *xrot, const uint8_t *codes, const uint16_t *scales,
+                        const double *t, const uint16_t *U,
+                        int64_t M, int64_t N, int64_t K,
+                        const int64_t *rows, int64_t n_rows, double *y)
+{
+    (void)M;
+    double *xb = (double *)malloc((size_t)(n_rows * K) * sizeof(double));
+    for (int64_t i = 0; i < n_rows; i++)
+        for (int64_t k = 0; k < K; k++)
+            xb[i * K + k] = (double)or_bf16_to_f32(or_f32_to_bf16(xrot[rows[i] * K + k]));
+#pragma omp parallel for schedule(static)
+    for (int64_t n = 0; n < N; n++) {
+        double *wb = (double *)malloc((size_t)K * sizeof(double));
+        for (int64_t k = 0; k < K; k++) {
+            uint8_t byte = codes[n * (K / 2) + k / 2];
+            int nib = (k & 1) ? (byte >> 4) : (byte & 0xF);
+            int q = nib >= 8 ? nib - 16 : nib;
+            float s = or_f16_to_f32(scales[n * (K / 32) + k / 32]);
+            float d = (float)q * s;                     /* exact */
+            wb[k] = (double)or_bf16_to_f32(or_f32_to_bf16(d));
+        }
+        for (int64_t i = 0; i < n_rows; i++) {
+            int64_t m = rows[i];
+            double acc = 0.0;
+            for (int64_t k = 0; k < K; k++)
+                acc += xb[i * K + k] * wb[k];
+            if (t)
+                for (int r = 0; r < 32; r++)
+                    acc += t[m * 32 + r] * (double)or_bf16_to_f32(U[n * 32 + r]);
+            y[i * N + n] = acc;
+        }
+        free(wb);
+    }
+    free(xb);
+}
+
+/* ------------------------------------------------------------------------ */
+/* O9: bf16 reconstruct of W from the payload                                */
+/* ------------------------------------------------------------------------ */
+
+/*
+ * W[n,k] = bf16( RN( L[n,k] + h[n,k] ) ) (SquareQ README, "the bwd-side bf16
+ * reconstruct from the same payload"), where
+ *   d = q * s (int4, exact) or RN(RN(e2m1 * value(sf)) * g_w) (NVFP4),
+ *   h = inverse_H256 of d over each 256-block of the row (= the same FWHT),
+ *   L = fmaf chain over r = 0..31 of U[n,r] * D[k,r], starting from 0.
+ * residual_only drops L: W = bf16(h).
+ * fmt: 1 = int4 g32 (scales fp16 [N, K/32]), 2 = NVFP4 (sf tiled, g_w).
+ */
+void or_reconstruct_bf16(int fmt, const uint8_t *codes, const void *scales, float g_w,
+                         const uint16_t *U, const uint16_t *D,
+                         int64_t N, int64_t K, int residual_only, uint16_t *W)
+{
+    int64_t C = K / 16;
+#pragma omp parallel for schedule(static)
+    for (int64_t n = 0; n < N; n++) {
+        for (int64_t b = 0; b < K; b += 256) {
+            float v[256];
+            for (int i = 0; i < 256; i++) {
+                int64_t k = b + i;
+                uint8_t byte = codes[n * (K / 2) + k / 2];
+                uint8_t nib = (k & 1) ? (byte >> 4) : (byte & 0xF);
+                if (fmt == 1) {
+                    int q = nib >= 8 ? (int)nib - 16 : (int)nib;
+                    float s = or_f16_to_f32(((const uint16_t *)scales)[n * (K / 32) + k / 32]);
+                    v[i] = (float)q * s;
+                } else {
+                    float dec = or_ue4m3_to_f32(((const uint8_t *)scales)[or_sf_offset(n, k / 16, C)]);
+                    float e = or_e2m1_to_f32(nib);
+                    float ed = e * dec;
+                    v[i] = ed * g_w;
+                }
+            }
+            or_fwht256(v);
+            for (int i = 0; i < 256; i++) {
+                int64_t k = b + i;
+                float out = v[i];
+                if (!residual_only) {
+                    float L = 0.0f;
+                    for (int r = 0; r < 32; r++)
+                        L = fmaf(or_bf16_to_f32(U[n * 32 + r]), or_bf16_to_f32(D[k * 32 + r]), L);
+                    out = L + v[i];
+                }
+                W[n * K + k] = or_f32_to_bf16(out);
+            }
+        }
+    }
+}
