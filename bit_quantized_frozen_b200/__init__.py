@@ -1,0 +1,241 @@
+"""Python binding of libsq, the SquareQ W4 quantized linear layer for B200 (sm_100a).
+
+Thin ctypes marshalling over the C ABI declared in ``include/sq.h``: every
+function below has the same name as its C entry point, takes torch tensors
+(device memory, contiguous) and passes their pointers, sizes and the current
+CUDA stream.  All arithmetic runs in the library's CUDA kernels; there is no
+CPU or PyTorch fallback -- if ``libsq.so`` is missing or the device is not
+sm_100, the calls raise.
+
+The layer (SquareQ README, section "SquareQ v3 -- W4"):
+    W = lora_up @ lora_down^T + inverse_H256(dequant(residual))
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from dataclasses import dataclass
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libsq.so")
+
+SQ_OK = 0
+SQ_FMT_INT4_G32 = 1
+SQ_FMT_NVFP4 = 2
+SQ_OP_BUILD_INT4 = 1
+SQ_OP_BUILD_NVFP4 = 2
+SQ_OP_ACT_QUANT_NVFP4 = 3
+SQ_OP_LINEAR_FWD_NVFP4 = 4
+SQ_OP_LINEAR_FWD_INT4 = 5
+SQ_OP_RECONSTRUCT = 6
+SQ_ACT_STATIC_SCALE = 0x1
+SQ_RECON_RESIDUAL_ONLY = 0x2
+RANK = 32
+
+EXPORTED = [
+    "sq_status_str", "sq_abi_version", "sq_last_error_detail", "sq_sf_bytes", "sq_workspace_bytes",
+    "sq_build_int4", "sq_build_nvfp4", "sq_act_quant_nvfp4", "sq_linear_fwd", "sq_reconstruct_bf16",
+    "sq_check_device_status",
+]
+
+
+class SqError(RuntimeError):
+    def __init__(self, fn: str, status: int, detail: str = ""):
+        self.status = status
+        msg = f"{fn} failed: {status_str(status)} ({status})"
+        if detail:
+            msg += f": {detail}"
+        super().__init__(msg)
+
+
+class sq_weight(ctypes.Structure):
+    _fields_ = [
+        ("fmt", ctypes.c_int32),
+        ("N", ctypes.c_int64),
+        ("K", ctypes.c_int64),
+        ("codes", ctypes.c_void_p),
+        ("scales", ctypes.c_void_p),
+        ("g_w", ctypes.c_void_p),
+        ("lora_up", ctypes.c_void_p),
+        ("lora_down", ctypes.c_void_p),
+    ]
+
+
+_P = ctypes.c_void_p
+_I64 = ctypes.c_int64
+_SIGS = {
+    "sq_status_str": ([ctypes.c_int], ctypes.c_char_p),
+    "sq_abi_version": ([], ctypes.c_int),
+    "sq_last_error_detail": ([], ctypes.c_char_p),
+    "sq_sf_bytes": ([_I64, _I64], ctypes.c_size_t),
+    "sq_workspace_bytes": ([ctypes.c_int, _I64, _I64, _I64], ctypes.c_size_t),
+    "sq_build_int4": ([_P, _I64, _I64, ctypes.c_int32, _P, _P, _P, _P], ctypes.c_int),
+    "sq_build_nvfp4": ([_P, _I64, _I64, _P, _P, _P, _P, ctypes.c_size_t, _P], ctypes.c_int),
+    "sq_act_quant_nvfp4": ([_P, _I64, _I64, _P, _P, _P, _P, _P, ctypes.c_uint32, _P, ctypes.c_size_t, _P],
+                           ctypes.c_int),
+    "sq_linear_fwd": ([ctypes.POINTER(sq_weight), _P, _I64, _P, _P, ctypes.c_uint32, _P, ctypes.c_size_t, _P],
+                      ctypes.c_int),
+    "sq_reconstruct_bf16": ([ctypes.POINTER(sq_weight), _P, ctypes.c_uint32, _P], ctypes.c_int),
+    "sq_check_device_status": ([_P, _P], ctypes.c_int),
+}
+_lib = None
+
+
+def lib() -> ctypes.CDLL:
+    """Load libsq.so (raises if it has not been built)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(f"libsq.so not found at {LIB_PATH}; build it with "
+                               "`python -m bit_quantized_frozen_b200.build`")
+        L = ctypes.CDLL(LIB_PATH)
+        for name, (args, res) in _SIGS.items():
+            fn = getattr(L, name)
+            fn.argtypes = args
+            fn.restype = res
+        _lib = L
+    return _lib
+
+
+def status_str(status: int) -> str:
+    return lib().sq_status_str(int(status)).decode()
+
+
+def _check(fn: str, status: int):
+    if status != SQ_OK:
+        raise SqError(fn, status, lib().sq_last_error_detail().decode())
+
+
+def _ptr(t) -> int | None:
+    if t is None:
+        return None
+    if isinstance(t, int):
+        return t
+    if not t.is_cuda:
+        raise ValueError("expected a CUDA tensor")
+    if not t.is_contiguous():
+        raise ValueError("expected a contiguous tensor")
+    return t.data_ptr()
+
+
+def _stream(stream) -> int | None:
+    if stream is None:
+        return torch.cuda.current_stream().cuda_stream
+    if isinstance(stream, int):
+        return stream
+    return stream.cuda_stream
+
+
+def _numel_bytes(t) -> int:
+    return t.numel() * t.element_size()
+
+
+# ---- C entry points ----------------------------------------------------------
+
+def sq_abi_version() -> int:
+    return lib().sq_abi_version()
+
+
+def sq_sf_bytes(rows: int, K: int) -> int:
+    return lib().sq_sf_bytes(rows, K)
+
+
+def sq_workspace_bytes(op: int, M: int, N: int, K: int) -> int:
+    return lib().sq_workspace_bytes(op, M, N, K)
+
+
+def sq_build_int4(R, codes, scales, frac_idx=None, group: int = 32, stream=None):
+    N, K = R.shape
+    _check("sq_build_int4", lib().sq_build_int4(_ptr(R), N, K, group, _ptr(codes), _ptr(scales), _ptr(frac_idx),
+                                                _stream(stream)))
+
+
+def sq_build_nvfp4(R, codes, sf_tiled, g_w, ws, stream=None):
+    N, K = R.shape
+    _check("sq_build_nvfp4", lib().sq_build_nvfp4(_ptr(R), N, K, _ptr(codes), _ptr(sf_tiled), _ptr(g_w), _ptr(ws),
+                                                  _numel_bytes(ws), _stream(stream)))
+
+
+def sq_act_quant_nvfp4(x, codes, sf_tiled, g_x, lora_down=None, t=None, flags: int = 0, ws=None, stream=None):
+    M, K = x.shape
+    _check("sq_act_quant_nvfp4",
+           lib().sq_act_quant_nvfp4(_ptr(x), M, K, _ptr(codes), _ptr(sf_tiled), _ptr(g_x), _ptr(lora_down), _ptr(t),
+                                    flags, _ptr(ws), 0 if ws is None else _numel_bytes(ws), _stream(stream)))
+
+
+def sq_linear_fwd(w: "Weight", x, y, g_x=None, flags: int = 0, ws=None, stream=None):
+    M = x.shape[0]
+    cw = w.as_c()
+    _check("sq_linear_fwd", lib().sq_linear_fwd(ctypes.byref(cw), _ptr(x), M, _ptr(y), _ptr(g_x), flags, _ptr(ws),
+                                                0 if ws is None else _numel_bytes(ws), _stream(stream)))
+
+
+def sq_reconstruct_bf16(w: "Weight", W_out, flags: int = 0, stream=None):
+    cw = w.as_c()
+    _check("sq_reconstruct_bf16", lib().sq_reconstruct_bf16(ctypes.byref(cw), _ptr(W_out), flags, _stream(stream)))
+
+
+def sq_check_device_status(ws, stream=None):
+    _check("sq_check_device_status", lib().sq_check_device_status(_ptr(ws), _stream(stream)))
+
+
+# ---- a built weight and allocating helpers (torch provides the memory) --------
+
+@dataclass
+class Weight:
+    fmt: int
+    N: int
+    K: int
+    codes: torch.Tensor                  # uint8 [N, K/2]
+    scales: torch.Tensor                 # int4: float16 [N, K/32]; NVFP4: uint8 tiled
+    g_w: torch.Tensor | None = None      # float32 [1] (NVFP4)
+    lora_up: torch.Tensor | None = None  # bf16 [N, 32]
+    lora_down: torch.Tensor | None = None  # bf16 [K, 32]
+    frac_idx: torch.Tensor | None = None  # uint8 [N, K/32] (int4)
+
+    def as_c(self) -> sq_weight:
+        return sq_weight(self.fmt, self.N, self.K, _ptr(self.codes), _ptr(self.scales), _ptr(self.g_w),
+                         _ptr(self.lora_up), _ptr(self.lora_down))
+
+
+def workspace(op: int, M: int, N: int, K: int, device=None) -> torch.Tensor:
+    n = max(sq_workspace_bytes(op, M, N, K), 256)
+    return torch.empty(n, dtype=torch.uint8, device=device or "cuda")
+
+
+def build_int4(R: torch.Tensor, lora_up=None, lora_down=None, stream=None) -> Weight:
+    N, K = R.shape
+    dev = R.device
+    codes = torch.empty((N, K // 2), dtype=torch.uint8, device=dev)
+    scales = torch.empty((N, K // 32), dtype=torch.float16, device=dev)
+    frac = torch.empty((N, K // 32), dtype=torch.uint8, device=dev)
+    sq_build_int4(R, codes, scales, frac, stream=stream)
+    return Weight(SQ_FMT_INT4_G32, N, K, codes, scales, None, lora_up, lora_down, frac)
+
+
+def build_nvfp4(R: torch.Tensor, lora_up=None, lora_down=None, ws=None, stream=None) -> Weight:
+    N, K = R.shape
+    dev = R.device
+    codes = torch.empty((N, K // 2), dtype=torch.uint8, device=dev)
+    sf = torch.empty(sq_sf_bytes(N, K), dtype=torch.uint8, device=dev)
+    g = torch.empty(1, dtype=torch.float32, device=dev)
+    ws = ws if ws is not None else workspace(SQ_OP_BUILD_NVFP4, 0, N, K, dev)
+    sq_build_nvfp4(R, codes, sf, g, ws, stream=stream)
+    return Weight(SQ_FMT_NVFP4, N, K, codes, sf, g, lora_up, lora_down)
+
+
+def linear_fwd(w: Weight, x: torch.Tensor, ws=None, g_x=None, flags: int = 0, stream=None) -> torch.Tensor:
+    M = x.shape[0]
+    y = torch.empty((M, w.N), dtype=torch.float32, device=x.device)
+    op = SQ_OP_LINEAR_FWD_NVFP4 if w.fmt == SQ_FMT_NVFP4 else SQ_OP_LINEAR_FWD_INT4
+    ws = ws if ws is not None else workspace(op, M, w.N, w.K, x.device)
+    sq_linear_fwd(w, x, y, g_x=g_x, flags=flags, ws=ws, stream=stream)
+    return y
+
+
+def reconstruct_bf16(w: Weight, residual_only: bool = False, stream=None) -> torch.Tensor:
+    W = torch.empty((w.N, w.K), dtype=torch.bfloat16, device=w.codes.device)
+    sq_reconstruct_bf16(w, W, SQ_RECON_RESIDUAL_ONLY if residual_only else 0, stream=stream)
+    return W

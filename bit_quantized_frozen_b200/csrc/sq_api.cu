@@ -1,0 +1,398 @@
+// sq_api.cu -- the C ABI of libsq (include/sq.h): host-side validation,
+// workspace carving and the launch sequence of each operation.  Nothing here
+// allocates, synchronises or copies to the host (except the explicit status
+// read-back); every error is returned as an sq_status before any launch.
+#include <cuda_runtime.h>
+
+#include <cstdio>
+#include <cstring>
+
+#include "sq.h"
+#include "sq_kernels.h"
+
+namespace {
+
+constexpr int kMaxDevices = 64;
+int g_sms[kMaxDevices];          // 0 = not yet queried
+int g_cc_ok[kMaxDevices];        // 0 unknown, 1 sm_100, -1 other
+
+thread_local char g_detail[256] = "";
+
+void set_detail(const char *what, cudaError_t e)
+{
+    snprintf(g_detail, sizeof(g_detail), "%s: %s", what, cudaGetErrorString(e));
+}
+
+// current device must be compute capability 10.0 (the sm_100a code this library carries)
+sq_status check_device(int *sms)
+{
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) {
+        set_detail("cudaGetDevice", e);
+        return SQ_ERR_DEVICE;
+    }
+    if (dev < 0 || dev >= kMaxDevices)
+        return SQ_ERR_DEVICE;
+    if (g_cc_ok[dev] == 0) {
+        int major = 0, minor = 0, n = 0;
+        if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+            cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess ||
+            cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+            return SQ_ERR_DEVICE;
+        g_sms[dev] = n;
+        g_cc_ok[dev] = (major == 10 && minor == 0) ? 1 : -1;
+    }
+    if (g_cc_ok[dev] != 1) {
+        snprintf(g_detail, sizeof(g_detail), "device %d is not compute capability 10.0", dev);
+        return SQ_ERR_DEVICE;
+    }
+    *sms = g_sms[dev];
+    return SQ_OK;
+}
+
+bool aligned(const void *p, uintptr_t a)
+{
+    return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0;
+}
+
+size_t round_up(size_t v, size_t a)
+{
+    return (v + a - 1) / a * a;
+}
+
+constexpr int64_t kMaxM = int64_t(1) << 24;
+constexpr int64_t kMaxN = int64_t(1) << 20;
+constexpr int64_t kMaxK = int64_t(1) << 17;
+
+bool shape_ok_nk(int64_t N, int64_t K)
+{
+    return N >= 128 && N % 128 == 0 && N <= kMaxN && K >= 256 && K % 256 == 0 && K <= kMaxK;
+}
+
+bool shape_ok_mk(int64_t M, int64_t K)
+{
+    return M >= 1 && M <= kMaxM && K >= 256 && K % 256 == 0 && K <= kMaxK;
+}
+
+// workspace layout ----------------------------------------------------------
+// [0, 256): header -- u32 status, u32 amax, f32 g_x scratch
+constexpr size_t kHeader = 256;
+constexpr size_t kAlign = 1024;
+
+struct FwdLayout {
+    size_t a = 0, a_sf = 0, b = 0, tsplit = 0, udup = 0, dt = 0, total = 0;
+};
+
+FwdLayout fwd_layout(int fmt, int64_t M, int64_t N, int64_t K)
+{
+    FwdLayout L;
+    size_t off = kHeader;
+    auto take = [&](size_t bytes) {
+        off = round_up(off, kAlign);
+        size_t at = off;
+        off += bytes;
+        return at;
+    };
+    if (fmt == SQ_FMT_NVFP4) {
+        L.a = take((size_t)M * (size_t)K / 2);
+        L.a_sf = take(sq_sf_bytes(M, K));
+    } else {
+        L.a = take((size_t)M * (size_t)K * 2);
+        L.b = take((size_t)N * (size_t)K * 2);
+    }
+    L.tsplit = take((size_t)M * 64 * 2);
+    L.udup = take((size_t)N * 64 * 2);
+    L.dt = take((size_t)K * 32 * 2);
+    L.total = round_up(off, kAlign);
+    return L;
+}
+
+uint8_t *ws_at(void *ws, size_t off)
+{
+    return reinterpret_cast<uint8_t *>(ws) + off;
+}
+
+#define SQ_CUDA(call, what)                     \
+    do {                                        \
+        cudaError_t e_ = (call);                \
+        if (e_ != cudaSuccess) {                \
+            set_detail(what, e_);               \
+            return SQ_ERR_CUDA;                 \
+        }                                       \
+    } while (0)
+
+sq_status check_weight(const sq_weight *w)
+{
+    if (!w || !w->codes || !w->scales)
+        return SQ_ERR_NULL;
+    if (w->fmt != SQ_FMT_INT4_G32 && w->fmt != SQ_FMT_NVFP4)
+        return SQ_ERR_ARG;
+    if (w->fmt == SQ_FMT_NVFP4 && !w->g_w)
+        return SQ_ERR_NULL;
+    if (!shape_ok_nk(w->N, w->K))
+        return SQ_ERR_SHAPE;
+    if (!aligned(w->codes, 16) || !aligned(w->scales, 16) || !aligned(w->g_w, 4) ||
+        !aligned(w->lora_up, 16) || !aligned(w->lora_down, 16))
+        return SQ_ERR_ALIGN;
+    return SQ_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char *sq_status_str(int status)
+{
+    switch (status) {
+    case SQ_OK: return "ok";
+    case SQ_ERR_NULL: return "null pointer";
+    case SQ_ERR_SHAPE: return "unsupported shape";
+    case SQ_ERR_ALIGN: return "misaligned pointer";
+    case SQ_ERR_WORKSPACE: return "workspace too small";
+    case SQ_ERR_DEVICE: return "device is not sm_100";
+    case SQ_ERR_CUDA: return "CUDA error";
+    case SQ_ERR_ARG: return "bad argument";
+    case SQ_ERR_TIMEOUT: return "kernel wait timed out";
+    default: return "unknown status";
+    }
+}
+
+int sq_abi_version(void)
+{
+    return 1;
+}
+
+const char *sq_last_error_detail(void)
+{
+    return g_detail;
+}
+
+size_t sq_sf_bytes(int64_t rows, int64_t K)
+{
+    if (rows < 0 || K < 0)
+        return 0;
+    return (size_t)((rows + 127) / 128 * 128) * (size_t)(K / 16);
+}
+
+size_t sq_workspace_bytes(int op, int64_t M, int64_t N, int64_t K)
+{
+    if (M < 0 || N < 0 || K < 0)
+        return 0;
+    switch (op) {
+    case SQ_OP_BUILD_INT4:
+    case SQ_OP_RECONSTRUCT:
+        return kHeader;
+    case SQ_OP_BUILD_NVFP4:
+        return kHeader;
+    case SQ_OP_ACT_QUANT_NVFP4:
+        return round_up(kHeader, kAlign) + round_up((size_t)K * 32 * 2, kAlign);
+    case SQ_OP_LINEAR_FWD_NVFP4:
+        return fwd_layout(SQ_FMT_NVFP4, M, N, K).total;
+    case SQ_OP_LINEAR_FWD_INT4:
+        return fwd_layout(SQ_FMT_INT4_G32, M, N, K).total;
+    default:
+        return 0;
+    }
+}
+
+sq_status sq_build_int4(const float *R, int64_t N, int64_t K, int32_t group, uint8_t *codes, uint16_t *scales,
+                        uint8_t *frac_idx, void *stream)
+{
+    if (!R || !codes || !scales)
+        return SQ_ERR_NULL;
+    if (group != 32 || !shape_ok_nk(N, K))
+        return SQ_ERR_SHAPE;
+    if (!aligned(R, 16) || !aligned(codes, 16) || !aligned(scales, 16) || !aligned(frac_idx, 16))
+        return SQ_ERR_ALIGN;
+    int sms = 0;
+    sq_status st = check_device(&sms);
+    if (st != SQ_OK)
+        return st;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    SQ_CUDA(sq::launch_int4_build(R, N, K, codes, scales, frac_idx, sms, s), "int4 build");
+    return SQ_OK;
+}
+
+sq_status sq_build_nvfp4(const float *R, int64_t N, int64_t K, uint8_t *codes, uint8_t *sf_tiled, float *g_w,
+                         void *ws, size_t ws_bytes, void *stream)
+{
+    if (!R || !codes || !sf_tiled || !g_w || !ws)
+        return SQ_ERR_NULL;
+    if (!shape_ok_nk(N, K))
+        return SQ_ERR_SHAPE;
+    if (!aligned(R, 16) || !aligned(codes, 16) || !aligned(sf_tiled, 16) || !aligned(g_w, 4) || !aligned(ws, 256))
+        return SQ_ERR_ALIGN;
+    if (ws_bytes < sq_workspace_bytes(SQ_OP_BUILD_NVFP4, 0, N, K))
+        return SQ_ERR_WORKSPACE;
+    int sms = 0;
+    sq_status st = check_device(&sms);
+    if (st != SQ_OK)
+        return st;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    uint32_t *amax = reinterpret_cast<uint32_t *>(ws_at(ws, 4));
+    SQ_CUDA(cudaMemsetAsync(amax, 0, 4, s), "memset");
+    SQ_CUDA(sq::launch_absmax_rot_f32(R, N, K, amax, sms, s), "absmax");
+    SQ_CUDA(sq::launch_nvfp4_quant_f32(R, N, K, amax, nullptr, g_w, codes, sf_tiled, sms, s), "nvfp4 quant");
+    return SQ_OK;
+}
+
+sq_status sq_act_quant_nvfp4(const uint16_t *x, int64_t M, int64_t K, uint8_t *codes, uint8_t *sf_tiled,
+                             float *g_x, const uint16_t *lora_down, float *t, uint32_t flags, void *ws,
+                             size_t ws_bytes, void *stream)
+{
+    if (!x || !codes || !sf_tiled || !g_x || !ws)
+        return SQ_ERR_NULL;
+    if (flags & ~SQ_ACT_STATIC_SCALE)
+        return SQ_ERR_ARG;
+    if (!shape_ok_mk(M, K))
+        return SQ_ERR_SHAPE;
+    if (!aligned(x, 16) || !aligned(codes, 16) || !aligned(sf_tiled, 16) || !aligned(g_x, 4) ||
+        !aligned(lora_down, 16) || !aligned(t, 16) || !aligned(ws, 256))
+        return SQ_ERR_ALIGN;
+    if (ws_bytes < sq_workspace_bytes(SQ_OP_ACT_QUANT_NVFP4, M, 0, K))
+        return SQ_ERR_WORKSPACE;
+    int sms = 0;
+    sq_status st = check_device(&sms);
+    if (st != SQ_OK)
+        return st;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    const bool stat = (flags & SQ_ACT_STATIC_SCALE) != 0;
+    uint32_t *amax = reinterpret_cast<uint32_t *>(ws_at(ws, 4));
+    if (!stat) {
+        SQ_CUDA(cudaMemsetAsync(amax, 0, 4, s), "memset");
+        SQ_CUDA(sq::launch_absmax_rot_bf16(x, M, K, amax, sms, s), "absmax");
+    }
+    SQ_CUDA(sq::launch_nvfp4_quant_bf16(x, M, K, amax, stat ? g_x : nullptr, stat ? nullptr : g_x, codes, sf_tiled,
+                                        sms, s),
+            "nvfp4 quant");
+    if (lora_down && t) {
+        uint16_t *dt = reinterpret_cast<uint16_t *>(ws_at(ws, round_up(kHeader, kAlign)));
+        SQ_CUDA(sq::launch_lora_prep(nullptr, 0, lora_down, K, nullptr, dt, sms, s), "lora prep");
+        SQ_CUDA(sq::launch_lowrank_t(x, M, K, dt, nullptr, nullptr, t, nullptr, s), "lowrank t");
+    }
+    return SQ_OK;
+}
+
+sq_status sq_linear_fwd(const sq_weight *w, const uint16_t *x, int64_t M, float *y, float *g_x, uint32_t flags,
+                        void *ws, size_t ws_bytes, void *stream)
+{
+    sq_status st = check_weight(w);
+    if (st != SQ_OK)
+        return st;
+    if (!x || !y || !ws)
+        return SQ_ERR_NULL;
+    if (flags & ~SQ_ACT_STATIC_SCALE)
+        return SQ_ERR_ARG;
+    const bool stat = (flags & SQ_ACT_STATIC_SCALE) != 0;
+    if (stat && (!g_x || w->fmt != SQ_FMT_NVFP4))
+        return stat && !g_x ? SQ_ERR_NULL : SQ_ERR_ARG;
+    const int64_t N = w->N, K = w->K;
+    if (!shape_ok_mk(M, K))
+        return SQ_ERR_SHAPE;
+    if (!aligned(x, 16) || !aligned(y, 16) || !aligned(g_x, 4) || !aligned(ws, 256))
+        return SQ_ERR_ALIGN;
+    const FwdLayout L = fwd_layout(w->fmt, M, N, K);
+    if (ws_bytes < L.total)
+        return SQ_ERR_WORKSPACE;
+    int sms = 0;
+    st = check_device(&sms);
+    if (st != SQ_OK)
+        return st;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    const bool lora = w->lora_up && w->lora_down;
+    uint16_t *tsplit = lora ? reinterpret_cast<uint16_t *>(ws_at(ws, L.tsplit)) : nullptr;
+    uint16_t *udup = lora ? reinterpret_cast<uint16_t *>(ws_at(ws, L.udup)) : nullptr;
+    uint16_t *dt = reinterpret_cast<uint16_t *>(ws_at(ws, L.dt));
+    uint32_t *status = reinterpret_cast<uint32_t *>(ws_at(ws, 0));
+    sq::GemmLaunch g;
+    memset(&g, 0, sizeof(g));
+    g.M = M;
+    g.N = N;
+    g.K = K;
+    g.y = y;
+    g.status = status;
+    g.tsplit = tsplit;
+    g.udup = udup;
+    if (w->fmt == SQ_FMT_NVFP4) {
+        uint32_t *amax = reinterpret_cast<uint32_t *>(ws_at(ws, 4));
+        float *gx = g_x ? g_x : reinterpret_cast<float *>(ws_at(ws, 8));
+        uint8_t *xc = ws_at(ws, L.a);
+        uint8_t *xsf = ws_at(ws, L.a_sf);
+        SQ_CUDA(cudaMemsetAsync(status, 0, 8, s), "memset");   // status word + absmax
+        if (!stat)
+            SQ_CUDA(sq::launch_absmax_rot_bf16(x, M, K, amax, sms, s), "absmax");
+        SQ_CUDA(sq::launch_nvfp4_quant_bf16(x, M, K, amax, stat ? gx : nullptr, stat ? nullptr : gx, xc, xsf, sms,
+                                            s),
+                "nvfp4 act quant");
+        if (lora) {
+            SQ_CUDA(sq::launch_lora_prep(w->lora_up, N, w->lora_down, K, udup, dt, sms, s), "lora prep");
+            SQ_CUDA(sq::launch_lowrank_t(x, M, K, dt, gx, w->g_w, nullptr, tsplit, s), "lowrank t");
+        }
+        g.fp4 = 1;
+        g.a = xc;
+        g.b = w->codes;
+        g.sfa = xsf;
+        g.sfb = reinterpret_cast<const uint8_t *>(w->scales);
+        g.g_x = gx;
+        g.g_w = w->g_w;
+    } else {
+        SQ_CUDA(cudaMemsetAsync(status, 0, 4, s), "memset");
+        uint16_t *xb = reinterpret_cast<uint16_t *>(ws_at(ws, L.a));
+        uint16_t *wb = reinterpret_cast<uint16_t *>(ws_at(ws, L.b));
+        SQ_CUDA(sq::launch_rotate_bf16(x, M, K, xb, sms, s), "rotate x");
+        SQ_CUDA(sq::launch_dequant_int4(w->codes, reinterpret_cast<const uint16_t *>(w->scales), N, K, wb, sms, s),
+                "dequant");
+        if (lora) {
+            SQ_CUDA(sq::launch_lora_prep(w->lora_up, N, w->lora_down, K, udup, dt, sms, s), "lora prep");
+            SQ_CUDA(sq::launch_lowrank_t(x, M, K, dt, nullptr, nullptr, nullptr, tsplit, s), "lowrank t");
+        }
+        g.fp4 = 0;
+        g.a = xb;
+        g.b = wb;
+    }
+    SQ_CUDA(sq::launch_gemm(g, sms, s), "gemm");
+    return SQ_OK;
+}
+
+sq_status sq_reconstruct_bf16(const sq_weight *w, uint16_t *W_out, uint32_t flags, void *stream)
+{
+    sq_status st = check_weight(w);
+    if (st != SQ_OK)
+        return st;
+    if (!W_out)
+        return SQ_ERR_NULL;
+    if (flags & ~SQ_RECON_RESIDUAL_ONLY)
+        return SQ_ERR_ARG;
+    if (!aligned(W_out, 16))
+        return SQ_ERR_ALIGN;
+    int sms = 0;
+    st = check_device(&sms);
+    if (st != SQ_OK)
+        return st;
+    const int with_lowrank = (!(flags & SQ_RECON_RESIDUAL_ONLY) && w->lora_up && w->lora_down) ? 1 : 0;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    SQ_CUDA(sq::launch_reconstruct(w->fmt, w->codes, w->scales, w->g_w, w->lora_up, w->lora_down, w->N, w->K,
+                                   with_lowrank, W_out, s),
+            "reconstruct");
+    return SQ_OK;
+}
+
+sq_status sq_check_device_status(void *ws, void *stream)
+{
+    if (!ws)
+        return SQ_ERR_NULL;
+    if (!aligned(ws, 256))
+        return SQ_ERR_ALIGN;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    uint32_t word = 0;
+    SQ_CUDA(cudaMemcpyAsync(&word, ws, 4, cudaMemcpyDeviceToHost, s), "status read");
+    SQ_CUDA(cudaStreamSynchronize(s), "status sync");
+    if (word != 0) {
+        SQ_CUDA(cudaMemsetAsync(ws, 0, 4, s), "status clear");
+        return SQ_ERR_TIMEOUT;
+    }
+    return SQ_OK;
+}
+
+}  // extern "C"

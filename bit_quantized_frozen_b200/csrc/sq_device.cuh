@@ -1,0 +1,146 @@
+// sq_device.cuh -- device helpers shared by the libsq kernels (sm_100a).
+//
+// Rounding discipline: every fp32 operation that feeds an integer or packed
+// output uses the explicit round-to-nearest intrinsics (__fadd_rn, __fmul_rn,
+// __fdiv_rn, __frcp_rn, ...), so the compiler cannot contract or reorder it,
+// and the result is the IEEE result of the operation sequence stated in sq.h.
+#pragma once
+
+#include <cstdint>
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+
+namespace sq {
+
+constexpr int kRank = 32;          // low-rank branch rank
+constexpr int kHad = 256;          // Hadamard block size over K
+constexpr int kSfBlock = 16;       // NVFP4 values per ue4m3 scale
+constexpr int kGroup = 32;         // int4 values per fp16 scale
+constexpr int kFracCount = 26;     // int4 scale fractions 0.50, 0.52, ..., 1.00
+
+// device status word bits (first word of every workspace)
+constexpr uint32_t kStatusTimeout = 1u;
+
+// ---------------------------------------------------------------------------
+// Hadamard-256 over one warp.
+//
+// Layout: lane l holds v[0..3] = elements 4l..4l+3 and v[4..7] = elements
+// 128+4l..128+4l+3 of the 256-block, so a warp's loads are contiguous.
+// Butterfly stride h pairs element j with j+h when (j & h) == 0; the lower
+// element becomes a+b and the upper a-b (a = lower, b = upper), strides in the
+// order 1, 2, 4, ..., 128, then a scale by 1/16 (exact).  Strides 1 and 2 and
+// 128 pair values inside a lane; strides 4..64 pair lane l with lane l^(h/4).
+// Every butterfly has the same two operands whichever lane computes it, so
+// the result equals the sequential radix-2 transform bit for bit.
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ void fwht256_warp(float (&v)[8], int lane)
+{
+#pragma unroll
+    for (int half = 0; half < 8; half += 4) {
+        float a0 = v[half + 0], a1 = v[half + 1], a2 = v[half + 2], a3 = v[half + 3];
+        // h = 1
+        float b0 = __fadd_rn(a0, a1), b1 = __fsub_rn(a0, a1);
+        float b2 = __fadd_rn(a2, a3), b3 = __fsub_rn(a2, a3);
+        // h = 2
+        v[half + 0] = __fadd_rn(b0, b2);
+        v[half + 2] = __fsub_rn(b0, b2);
+        v[half + 1] = __fadd_rn(b1, b3);
+        v[half + 3] = __fsub_rn(b1, b3);
+    }
+#pragma unroll
+    for (int x = 1; x <= 16; x <<= 1) {          // h = 4x
+        const bool lower = (lane & x) == 0;
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            float p = __shfl_xor_sync(0xffffffffu, v[i], x);
+            v[i] = lower ? __fadd_rn(v[i], p) : __fsub_rn(p, v[i]);
+        }
+    }
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {                // h = 128
+        float a = v[i], b = v[i + 4];
+        v[i] = __fadd_rn(a, b);
+        v[i + 4] = __fsub_rn(a, b);
+    }
+#pragma unroll
+    for (int i = 0; i < 8; ++i)
+        v[i] = __fmul_rn(v[i], 0.0625f);
+}
+
+// ---------------------------------------------------------------------------
+// Narrowing conversions (PTX cvt, round-to-nearest-even, satfinite).
+// ---------------------------------------------------------------------------
+
+// ue4m3 code of a non-negative value (e4m3 with sign 0; saturates at 448).
+__device__ __forceinline__ uint32_t to_ue4m3(float v)
+{
+    uint16_t packed;   // upper byte <- first source, lower byte <- second source
+    asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(packed) : "f"(0.0f), "f"(v));
+    return (uint32_t)packed & 0xFFu;
+}
+
+// value of a ue4m3 code (exact through fp16)
+__device__ __forceinline__ float ue4m3_value(uint32_t code)
+{
+    uint32_t h2;
+    uint16_t in = (uint16_t)(code & 0xFFu);
+    asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(h2) : "h"(in));
+    return __half2float(__ushort_as_half((unsigned short)(h2 & 0xFFFFu)));
+}
+
+// e2m1 magnitude codes of two non-negative values, packed lo | hi << 4.
+__device__ __forceinline__ uint32_t to_e2m1x2_mag(float lo, float hi)
+{
+    uint32_t out;
+    asm("{\n\t.reg .b8 t;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 t, %1, %2;\n\t"
+        "cvt.u32.u8 %0, t;\n\t}"
+        : "=r"(out) : "f"(hi), "f"(lo));
+    return out;
+}
+
+// e2m1 codes of two values with their sign bits kept (negative -> bit 3 set,
+// including values that round to zero), packed lo | hi << 4.
+__device__ __forceinline__ uint32_t to_e2m1x2(float lo, float hi)
+{
+    uint32_t mag = to_e2m1x2_mag(fabsf(lo), fabsf(hi));
+    uint32_t s = ((__float_as_uint(lo) >> 31) << 3) | ((__float_as_uint(hi) >> 31) << 7);
+    return mag | s;
+}
+
+// values of two e2m1 codes held in one byte (low nibble first), exact
+__device__ __forceinline__ float2 e2m1x2_value(uint32_t byte)
+{
+    uint32_t h2;
+    uint16_t in = (uint16_t)(byte & 0xFFu);
+    asm("{\n\t.reg .b8 t;\n\t"
+        "cvt.u8.u16 t, %1;\n\t"
+        "cvt.rn.f16x2.e2m1x2 %0, t;\n\t}"
+        : "=r"(h2) : "h"(in));
+    __half2 h = *reinterpret_cast<__half2 *>(&h2);
+    return __half22float2(h);
+}
+
+__device__ __forceinline__ float bf16_bits_to_f32(uint32_t bits16)
+{
+    return __uint_as_float(bits16 << 16);
+}
+
+__device__ __forceinline__ uint32_t f32_to_bf16_bits(float v)
+{
+    return (uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(v));
+}
+
+// tiled scale-factor byte offset, C = K/16 scale columns
+__device__ __forceinline__ int64_t sf_offset(int64_t r, int64_t c, int64_t C)
+{
+    return ((r >> 7) * (C >> 2) + (c >> 2)) * 512 + (r & 31) * 16 + ((r & 127) >> 5) * 4 + (c & 3);
+}
+
+// non-negative float max through its bit pattern (for atomicMax on u32)
+__device__ __forceinline__ void atomic_max_nonneg(uint32_t *addr, float v)
+{
+    atomicMax(addr, __float_as_uint(v));
+}
+
+}  // namespace sq

@@ -1,0 +1,413 @@
+// sq_gemm.cu -- persistent, warp-specialised tcgen05 GEMM of the W4 forward:
+//
+//   y[M, N] = beta * ( A B^T + Tsplit Udup^T )            (fp32 out)
+//
+//   NVFP4 path: A = e2m1 activation codes [M, K/2] with ue4m3 block-16 scales,
+//               B = e2m1 weight codes [N, K/2] with ue4m3 scales (tiled layout),
+//               block-scaled MMA (kind::mxf4nvf4.block16), beta = g_x * g_w.
+//   int4 path:  A = bf16(H x) [M, K], B = bf16(q s) [N, K], kind::f16, beta = 1.
+//   Low-rank:   Tsplit [M, 64] = [hi | lo] bf16 split of t / beta, Udup [N, 64]
+//               = [U | U]; one extra kind::f16 K-step into the same accumulator
+//               adds (t / beta) U^T, so the epilogue only scales by beta.
+//
+// (SquareQ README, "Op-level parity of the full FP4 forward": block-scaled
+// GEMM + epilogue; "Residual codecs": int4 "dequant-first".)
+//
+// CTA tile 128 x 256, one CTA per SM, 192 threads:
+//   warps 0-3  epilogue: tcgen05.ld of their 32 accumulator lanes, scale,
+//              128B-swizzled staging in shared memory, TMA store;
+//   warp 4     TMA producer (tiles of A, B, the scale factors, the low-rank
+//              operands) into a ring of shared-memory stages;
+//   warp 5     tensor-memory allocator and the single MMA-issuing thread.
+// Tensor memory (512 columns): two accumulator slots at columns 0 and 192
+// that overlap in columns 192..255, and the scale factors at 448..495.  The
+// epilogue reads the overlapping 64 columns of a tile first and then releases
+// the MMA thread, which starts the next tile while the other 192 columns
+// drain -- accumulator double buffering in 448 columns.
+#include <cuda.h>
+
+#include "sq_device.cuh"
+#include "sq_kernels.h"
+#include "sq_ptx.cuh"
+
+namespace sq {
+
+constexpr int BM = 128;
+constexpr int BN = 256;
+constexpr int kRowBytes = 128;                 // every stage holds 128-byte rows (one swizzle atom)
+constexpr int kABytes = BM * kRowBytes;        // 16 KB
+constexpr int kBBytes = BN * kRowBytes;        // 32 KB
+constexpr int kSfaBytes = 4 * 512;             // 4 scale chunks of 128 rows x 4 scales
+constexpr int kSfbBytes = 2 * kSfaBytes;       // 256 rows
+constexpr int kEpiWarps = 4;
+constexpr int kThreads = 192;
+constexpr int kStagingBytes = 32 * 128;        // one warp's 32 rows x 32 fp32
+constexpr uint32_t kTmemCols = 512;
+constexpr uint32_t kAccSlot1 = 192;
+constexpr uint32_t kSfaCol = 448;
+constexpr uint32_t kSfbCol = 464;
+
+// instruction descriptors: M = 128, N = 256, K-major A and B
+constexpr uint32_t kIdescBf16 = (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(BN >> 3) << 17) |
+                                ((uint32_t)(BM >> 4) << 24);           // f32 accum, bf16 x bf16
+constexpr uint32_t kIdescNvfp4 = (1u << 7) | (1u << 10) | ((uint32_t)(BN >> 3) << 17) |
+                                 ((uint32_t)(BM >> 4) << 24);          // e2m1 x e2m1, ue4m3 scales
+
+template <bool FP4>
+struct GemmCfg {
+    static constexpr int kStages = FP4 ? 3 : 4;
+    static constexpr int kStageBytes = kABytes + kBBytes + (FP4 ? kSfaBytes + kSfbBytes : 0);
+    static constexpr int kKPerStage = FP4 ? 256 : 64;            // K values per stage
+    static constexpr int kStagingOff = kStages * kStageBytes;
+    static constexpr int kBarOff = kStagingOff + kEpiWarps * 2 * kStagingBytes;
+    static constexpr int kSmemBytes = kBarOff + 256 + 1024;      // barriers + 1 KB alignment slack
+};
+
+struct GemmArgs {
+    const uint8_t *sfa;      // NVFP4: tiled activation scales
+    const uint8_t *sfb;      // NVFP4: tiled weight scales
+    const float *g_x;        // NVFP4: activation global scale (device)
+    const float *g_w;        // NVFP4: weight global scale (device)
+    uint32_t *status;        // device status word
+    int M, N, K;
+    int lora;                // 1: add the low-rank K-step
+};
+
+template <bool FP4>
+__global__ void __launch_bounds__(kThreads, 1)
+    sq_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                   const __grid_constant__ CUtensorMap tmT, const __grid_constant__ CUtensorMap tmU,
+                   const __grid_constant__ CUtensorMap tmY, const GemmArgs args)
+{
+    using Cfg = GemmCfg<FP4>;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint64_t *bars = reinterpret_cast<uint64_t *>(smem + Cfg::kBarOff);
+    // barrier slots: full[s], empty[s], acc_full[2], acc_empty, drain
+    const uint32_t bar_full = smem_u32(bars);
+    const uint32_t bar_empty = smem_u32(bars + Cfg::kStages);
+    const uint32_t bar_acc_full = smem_u32(bars + 2 * Cfg::kStages);
+    const uint32_t bar_acc_empty = smem_u32(bars + 2 * Cfg::kStages + 2);
+    const uint32_t bar_drain = smem_u32(bars + 2 * Cfg::kStages + 3);
+    uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(bars + 2 * Cfg::kStages + 4);
+    volatile uint32_t *abort_flag = tmem_holder + 1;
+
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < Cfg::kStages; ++s) {
+            mbar_init(bar_full + 8 * s, 1);
+            mbar_init(bar_empty + 8 * s, 1);
+        }
+        mbar_init(bar_acc_full, 1);
+        mbar_init(bar_acc_full + 8, 1);
+        mbar_init(bar_acc_empty, kEpiWarps);
+        mbar_init(bar_drain, 1);
+        *abort_flag = 0u;
+        fence_mbar_init();
+    }
+    if (warp == 5) {
+        tmem_alloc(smem_u32(tmem_holder), kTmemCols);
+        tmem_relinquish();
+    }
+    if (warp == 4 && lane == 0) {
+        prefetch_tmap(&tmA);
+        prefetch_tmap(&tmB);
+        prefetch_tmap(&tmT);
+        prefetch_tmap(&tmU);
+        prefetch_tmap(&tmY);
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem_base = *tmem_holder;
+
+    const int m_tiles = (args.M + BM - 1) / BM;
+    const int n_tiles = (args.N + BN - 1) / BN;
+    const int tiles = m_tiles * n_tiles;
+    const int k_stages = args.K / Cfg::kKPerStage;
+    const int stages_per_tile = k_stages + (args.lora ? 1 : 0);
+    const int sf_chunks_per_row_tile = args.K / 64;          // 512-byte chunks per 128-row tile
+
+    if (warp == 4) {
+        // ------------------------------------------------------------ producer
+        if (lane == 0) {
+            int stage = 0;
+            uint32_t phase = 0;
+            bool ok = true;
+            for (int tile = blockIdx.x; tile < tiles && ok; tile += gridDim.x) {
+                const int mt = tile % m_tiles, nt = tile / m_tiles;
+                const int m0 = mt * BM, n0 = nt * BN;
+                const bool sfb_hi = (n0 + 128) < args.N;
+                for (int ks = 0; ks < stages_per_tile; ++ks) {
+                    if (!mbar_wait(bar_empty + 8 * stage, phase ^ 1u, abort_flag, args.status)) {
+                        ok = false;
+                        break;
+                    }
+                    uint8_t *sbase = smem + stage * Cfg::kStageBytes;
+                    const uint32_t fb = bar_full + 8 * stage;
+                    const uint32_t sA = smem_u32(sbase), sB = smem_u32(sbase + kABytes);
+                    if (args.lora && ks == 0) {
+                        mbar_arrive_expect_tx(fb, kABytes + kBBytes);
+                        tma_load_2d(sA, &tmT, 0, m0, fb);
+                        tma_load_2d(sB, &tmU, 0, n0, fb);
+                    } else {
+                        const int kk = ks - (args.lora ? 1 : 0);
+                        if (FP4) {
+                            const uint32_t bytes = kABytes + kBBytes + kSfaBytes + (sfb_hi ? kSfbBytes : kSfaBytes);
+                            mbar_arrive_expect_tx(fb, bytes);
+                            tma_load_2d(sA, &tmA, kk * kRowBytes, m0, fb);
+                            tma_load_2d(sB, &tmB, kk * kRowBytes, n0, fb);
+                            const uint32_t sSfa = smem_u32(sbase + kABytes + kBBytes);
+                            const uint32_t sSfb = sSfa + kSfaBytes;
+                            const int64_t chunk = (int64_t)kk * 4;
+                            bulk_load(sSfa, args.sfa + ((int64_t)mt * sf_chunks_per_row_tile + chunk) * 512,
+                                      kSfaBytes, fb);
+                            bulk_load(sSfb, args.sfb + ((int64_t)(2 * nt) * sf_chunks_per_row_tile + chunk) * 512,
+                                      kSfaBytes, fb);
+                            if (sfb_hi)
+                                bulk_load(sSfb + kSfaBytes,
+                                          args.sfb + ((int64_t)(2 * nt + 1) * sf_chunks_per_row_tile + chunk) * 512,
+                                          kSfaBytes, fb);
+                        } else {
+                            mbar_arrive_expect_tx(fb, kABytes + kBBytes);
+                            tma_load_2d(sA, &tmA, kk * 64, m0, fb);
+                            tma_load_2d(sB, &tmB, kk * 64, n0, fb);
+                        }
+                    }
+                    if (++stage == Cfg::kStages) {
+                        stage = 0;
+                        phase ^= 1u;
+                    }
+                }
+            }
+            // let every load that was issued land (and be consumed) before the CTA exits
+            for (int s = 0; s < Cfg::kStages; ++s) {
+                (void)mbar_wait(bar_empty + 8 * stage, phase ^ 1u, abort_flag, args.status);
+                if (++stage == Cfg::kStages) {
+                    stage = 0;
+                    phase ^= 1u;
+                }
+            }
+        }
+        __syncwarp();
+    } else if (warp == 5) {
+        // ------------------------------------------------------------ MMA issuer
+        if (lane == 0) {
+            int stage = 0;
+            uint32_t phase = 0;
+            int count = 0;
+            bool ok = true;
+            for (int tile = blockIdx.x; tile < tiles && ok; tile += gridDim.x, ++count) {
+                const uint32_t acc = tmem_base + ((count & 1) ? kAccSlot1 : 0u);
+                if (count > 0 && !mbar_wait(bar_acc_empty, (uint32_t)((count - 1) & 1), abort_flag, args.status))
+                    break;
+                tc_fence_after();
+                for (int ks = 0; ks < stages_per_tile; ++ks) {
+                    if (!mbar_wait(bar_full + 8 * stage, phase, abort_flag, args.status)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    uint8_t *sbase = smem + stage * Cfg::kStageBytes;
+                    const uint32_t sA = smem_u32(sbase), sB = smem_u32(sbase + kABytes);
+                    if (args.lora && ks == 0) {
+#pragma unroll
+                        for (int k = 0; k < 4; ++k)
+                            mma_bf16(acc, sdesc_sw128(sA + 32 * k), sdesc_sw128(sB + 32 * k), kIdescBf16,
+                                     k > 0 ? 1u : 0u);
+                    } else if (FP4) {
+                        const uint32_t sSfa = sA + kABytes + kBBytes;
+                        const uint32_t sSfb = sSfa + kSfaBytes;
+#pragma unroll
+                        for (int k = 0; k < 4; ++k) {
+                            tmem_cp_32x128b_x4(tmem_base + kSfaCol + 4 * k, sdesc_sf(sSfa + 512 * k));
+                            tmem_cp_32x128b_x4(tmem_base + kSfbCol + 8 * k, sdesc_sf(sSfb + 512 * k));
+                            tmem_cp_32x128b_x4(tmem_base + kSfbCol + 8 * k + 4, sdesc_sf(sSfb + kSfaBytes + 512 * k));
+                        }
+#pragma unroll
+                        for (int k = 0; k < 4; ++k)
+                            mma_nvfp4(acc, sdesc_sw128(sA + 32 * k), sdesc_sw128(sB + 32 * k), kIdescNvfp4,
+                                      tmem_base + kSfaCol + 4 * k, tmem_base + kSfbCol + 8 * k,
+                                      (ks > 0 || k > 0) ? 1u : 0u);
+                    } else {
+#pragma unroll
+                        for (int k = 0; k < 4; ++k)
+                            mma_bf16(acc, sdesc_sw128(sA + 32 * k), sdesc_sw128(sB + 32 * k), kIdescBf16,
+                                     (ks > 0 || k > 0) ? 1u : 0u);
+                    }
+                    tc_commit(bar_empty + 8 * stage);
+                    if (++stage == Cfg::kStages) {
+                        stage = 0;
+                        phase ^= 1u;
+                    }
+                }
+                if (ok)
+                    tc_commit(bar_acc_full + 8 * (count & 1));
+            }
+            // all issued MMAs must finish before tensor memory is released
+            tc_commit(bar_drain);
+            (void)mbar_wait(bar_drain, 0, abort_flag, args.status);
+        }
+        __syncwarp();
+    } else {
+        // ------------------------------------------------------------ epilogue
+        float beta = 1.0f;
+        if (FP4) {
+            const float b = __fmul_rn(*args.g_x, *args.g_w);
+            beta = b == 0.0f ? 1.0f : b;
+        }
+        uint8_t *staging = smem + Cfg::kStagingOff + warp * 2 * kStagingBytes;
+        int sb = 0;
+        int count = 0;
+        for (int tile = blockIdx.x; tile < tiles; tile += gridDim.x, ++count) {
+            const int mt = tile % m_tiles, nt = tile / m_tiles;
+            const int m0 = mt * BM, n0 = nt * BN;
+            const int slot = count & 1;
+            bool ok = true;
+            if (lane == 0)
+                ok = mbar_wait(bar_acc_full + 8 * slot, (uint32_t)((count >> 1) & 1), abort_flag, args.status);
+            ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+            if (!ok)
+                break;
+            tc_fence_after();
+            const uint32_t acc = tmem_base + ((uint32_t)(32 * warp) << 16) + (slot ? kAccSlot1 : 0u);
+#pragma unroll 1
+            for (int ci = 0; ci < 8; ++ci) {
+                const int c = slot ? ci : ((ci + 6) & 7);   // overlapping columns first
+                uint32_t r[32];
+                tmem_ld_32cols(acc + 32 * c, r);
+                tmem_wait_ld();
+                if (ci == 1) {
+                    tc_fence_before();
+                    __syncwarp();
+                    if (lane == 0)
+                        mbar_arrive(bar_acc_empty);
+                }
+                // staging buffer sb is free once at most one store group is pending
+                if (lane == 0)
+                    bulk_wait_group_read1();
+                __syncwarp();
+                uint8_t *buf = staging + sb * kStagingBytes;
+#pragma unroll
+                for (int j = 0; j < 8; ++j) {
+                    float4 o;
+                    o.x = __fmul_rn(__uint_as_float(r[4 * j + 0]), beta);
+                    o.y = __fmul_rn(__uint_as_float(r[4 * j + 1]), beta);
+                    o.z = __fmul_rn(__uint_as_float(r[4 * j + 2]), beta);
+                    o.w = __fmul_rn(__uint_as_float(r[4 * j + 3]), beta);
+                    *reinterpret_cast<float4 *>(buf + lane * 128 + ((j ^ (lane & 7)) << 4)) = o;
+                }
+                fence_proxy_async_smem();
+                __syncwarp();
+                if (lane == 0) {
+                    tma_store_2d(&tmY, smem_u32(buf), n0 + 32 * c, m0 + 32 * warp);
+                    bulk_commit_group();
+                }
+                sb ^= 1;
+            }
+        }
+        if (lane == 0)
+            bulk_wait_group_all();
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    if (warp == 5)
+        tmem_dealloc(tmem_base, kTmemCols);
+}
+
+// ---------------------------------------------------------------------------
+// host side: tensor maps and launch
+// ---------------------------------------------------------------------------
+typedef CUresult (*PFN_encodeTiled)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,
+                                    const cuuint64_t *, const cuuint32_t *, const cuuint32_t *,
+                                    CUtensorMapInterleave, CUtensorMapSwizzle, CUtensorMapL2promotion,
+                                    CUtensorMapFloatOOBfill);
+
+static PFN_encodeTiled encode_fn()
+{
+    static PFN_encodeTiled fn = nullptr;
+    if (!fn) {
+        void *p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_encodeTiled>(p);
+    }
+    return fn;
+}
+
+// 2D row-major tensor [rows, inner] of `esize`-byte elements, box [box_rows, box_inner]
+static bool make_tmap(CUtensorMap *m, CUtensorMapDataType dt, int esize, const void *base, uint64_t inner,
+                      uint64_t rows, uint32_t box_inner, uint32_t box_rows, CUtensorMapSwizzle sw)
+{
+    PFN_encodeTiled fn = encode_fn();
+    if (!fn)
+        return false;
+    cuuint64_t dims[2] = {inner, rows};
+    cuuint64_t strides[1] = {inner * (uint64_t)esize};
+    cuuint32_t box[2] = {box_inner, box_rows};
+    cuuint32_t estr[2] = {1, 1};
+    CUresult r = fn(m, dt, 2, const_cast<void *>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, sw,
+                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
+cudaError_t launch_gemm(const GemmLaunch &g, int sms, cudaStream_t stream)
+{
+    CUtensorMap tA, tB, tT, tU, tY;
+    const bool fp4 = g.fp4 != 0;
+    bool ok = true;
+    if (fp4) {
+        ok &= make_tmap(&tA, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, g.a, (uint64_t)g.K / 2, (uint64_t)g.M, 128, BM,
+                        CU_TENSOR_MAP_SWIZZLE_128B);
+        ok &= make_tmap(&tB, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, g.b, (uint64_t)g.K / 2, (uint64_t)g.N, 128, BN,
+                        CU_TENSOR_MAP_SWIZZLE_128B);
+    } else {
+        ok &= make_tmap(&tA, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, g.a, (uint64_t)g.K, (uint64_t)g.M, 64, BM,
+                        CU_TENSOR_MAP_SWIZZLE_128B);
+        ok &= make_tmap(&tB, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, g.b, (uint64_t)g.K, (uint64_t)g.N, 64, BN,
+                        CU_TENSOR_MAP_SWIZZLE_128B);
+    }
+    const bool lora = g.tsplit && g.udup;
+    // without a low-rank step the maps below are never used; point them at A/B
+    ok &= make_tmap(&tT, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, lora ? (const void *)g.tsplit : g.a, 64,
+                    (uint64_t)g.M, 64, BM, CU_TENSOR_MAP_SWIZZLE_128B);
+    ok &= make_tmap(&tU, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, lora ? (const void *)g.udup : g.b, 64,
+                    (uint64_t)g.N, 64, BN, CU_TENSOR_MAP_SWIZZLE_128B);
+    ok &= make_tmap(&tY, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, g.y, (uint64_t)g.N, (uint64_t)g.M, 32, 32,
+                    CU_TENSOR_MAP_SWIZZLE_128B);
+    if (!ok)
+        return cudaErrorInvalidValue;
+    GemmArgs a;
+    a.sfa = g.sfa;
+    a.sfb = g.sfb;
+    a.g_x = g.g_x;
+    a.g_w = g.g_w;
+    a.status = g.status;
+    a.M = (int)g.M;
+    a.N = (int)g.N;
+    a.K = (int)g.K;
+    a.lora = lora ? 1 : 0;
+    const int tiles = (int)(((g.M + BM - 1) / BM) * ((g.N + BN - 1) / BN));
+    const int grid = tiles < sms ? tiles : sms;
+    if (fp4) {
+        const int smem = GemmCfg<true>::kSmemBytes;
+        cudaError_t e = cudaFuncSetAttribute(sq_gemm_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+        if (e != cudaSuccess)
+            return e;
+        sq_gemm_kernel<true><<<grid, kThreads, smem, stream>>>(tA, tB, tT, tU, tY, a);
+    } else {
+        const int smem = GemmCfg<false>::kSmemBytes;
+        cudaError_t e = cudaFuncSetAttribute(sq_gemm_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+        if (e != cudaSuccess)
+            return e;
+        sq_gemm_kernel<false><<<grid, kThreads, smem, stream>>>(tA, tB, tT, tU, tY, a);
+    }
+    return cudaGetLastError();
+}
+
+}  // namespace sq

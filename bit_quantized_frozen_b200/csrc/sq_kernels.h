@@ -1,0 +1,50 @@
+// sq_kernels.h -- internal launchers of libsq (not part of the C ABI).
+#pragma once
+
+#include <cstdint>
+#include <cuda_runtime.h>
+
+namespace sq {
+
+cudaError_t launch_absmax_rot_f32(const float *in, int64_t rows, int64_t K, uint32_t *amax, int sms,
+                                  cudaStream_t s);
+cudaError_t launch_absmax_rot_bf16(const uint16_t *in, int64_t rows, int64_t K, uint32_t *amax, int sms,
+                                   cudaStream_t s);
+cudaError_t launch_nvfp4_quant_f32(const float *in, int64_t rows, int64_t K, const uint32_t *amax,
+                                   const float *g_static, float *g_out, uint8_t *codes, uint8_t *sf, int sms,
+                                   cudaStream_t s);
+cudaError_t launch_nvfp4_quant_bf16(const uint16_t *in, int64_t rows, int64_t K, const uint32_t *amax,
+                                    const float *g_static, float *g_out, uint8_t *codes, uint8_t *sf, int sms,
+                                    cudaStream_t s);
+cudaError_t launch_int4_build(const float *R, int64_t N, int64_t K, uint8_t *codes, uint16_t *scales,
+                              uint8_t *frac, int sms, cudaStream_t s);
+cudaError_t launch_rotate_bf16(const uint16_t *x, int64_t M, int64_t K, uint16_t *xb, int sms, cudaStream_t s);
+cudaError_t launch_dequant_int4(const uint8_t *codes, const uint16_t *scales, int64_t N, int64_t K, uint16_t *wb,
+                                int sms, cudaStream_t s);
+cudaError_t launch_lora_prep(const uint16_t *U, int64_t N, const uint16_t *D, int64_t K, uint16_t *udup,
+                             uint16_t *dt, int sms, cudaStream_t s);
+cudaError_t launch_lowrank_t(const uint16_t *x, int64_t M, int64_t K, const uint16_t *dt, const float *g_x,
+                             const float *g_w, float *t_out, uint16_t *tsplit, cudaStream_t s);
+cudaError_t launch_reconstruct(int fmt, const uint8_t *codes, const void *scales, const float *g_w,
+                               const uint16_t *U, const uint16_t *D, int64_t N, int64_t K, int with_lowrank,
+                               uint16_t *W, cudaStream_t s);
+
+// forward GEMM y = beta (A B^T + tsplit udup^T), see sq_gemm.cu
+struct GemmLaunch {
+    int fp4;                 // 1: NVFP4 codes + tiled scales, 0: bf16 operands
+    const void *a;           // [M, K/2] u8 or [M, K] bf16
+    const void *b;           // [N, K/2] u8 or [N, K] bf16
+    const uint8_t *sfa;      // NVFP4 scales of a (tiled)
+    const uint8_t *sfb;      // NVFP4 scales of b (tiled)
+    const float *g_x;        // NVFP4: device scalars, beta = g_x * g_w
+    const float *g_w;
+    const uint16_t *tsplit;  // [M, 64] bf16 or NULL (no low-rank step)
+    const uint16_t *udup;    // [N, 64] bf16 or NULL
+    float *y;                // [M, N] fp32
+    uint32_t *status;        // device status word
+    int64_t M, N, K;
+};
+
+cudaError_t launch_gemm(const GemmLaunch &g, int sms, cudaStream_t stream);
+
+}  // namespace sq

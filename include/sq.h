@@ -1,0 +1,223 @@
+/*
+ * sq.h -- C ABI of libsq, the SquareQ W4 quantized linear layer on NVIDIA B200
+ * (sm_100a).
+ *
+ * The layer (SquareQ README, section "SquareQ v3 -- W4 (Hadamard-256 +
+ * low-rank + int4 / NVFP4)"):
+ *
+ *     W = lora_up . lora_down^T + inverse_H256( dequant( residual ) )
+ *
+ * H256 is the block-diagonal normalised Sylvester Hadamard matrix of order 256
+ * over the input dimension K ("Rotation" paragraph); it is symmetric and
+ * orthogonal, so inverse_H256 = H256.  The residual is stored either as int4
+ * with fp16 group-32 scales chosen by an MSE sweep over scale fractions, or as
+ * NVFP4 (e2m1 codes, ue4m3 scales per 16 values in the tiled scale layout, one
+ * fp32 global scale) ("Residual codecs" paragraph).  lora_up / lora_down are
+ * the rank-32 bf16 low-rank branch ("Low-rank branch" paragraph).
+ *
+ * Conventions for every entry point:
+ *   - Pointers marked "device" must point to device memory of the current
+ *     device; the library never allocates, frees, copies to the host or
+ *     synchronises.  Work is enqueued on `stream` (a cudaStream_t passed as
+ *     void*, NULL = legacy default stream) and runs asynchronously.
+ *   - Matrices are row-major and densely packed.  bf16 and fp16 values are
+ *     passed as their 16-bit patterns (uint16_t).
+ *   - Arguments are validated on the host before anything is enqueued; a
+ *     failed check returns a status and enqueues nothing.  A CUDA launch error
+ *     returns SQ_ERR_CUDA.  There is no fallback path: a device other than
+ *     compute capability 10.0 returns SQ_ERR_DEVICE.
+ *   - Shapes: K % 256 == 0 (the rotation's block size), N % 128 == 0, M >= 1.
+ *     All device pointers must be 16-byte aligned, workspaces 256-byte aligned.
+ *   - Rounding: every narrowing conversion is round-to-nearest-even; fp32
+ *     arithmetic follows the order stated for each operation, so integer and
+ *     packed outputs are reproducible bit for bit.
+ *   - Caller-owned workspace: its size comes from sq_workspace_bytes().  It
+ *     must not be shared by calls that may run concurrently.
+ */
+#ifndef SQ_H
+#define SQ_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define SQ_API __attribute__((visibility("default")))
+#else
+#define SQ_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    SQ_OK = 0,
+    SQ_ERR_NULL = 1,       /* a required pointer is NULL                          */
+    SQ_ERR_SHAPE = 2,      /* K % 256, N % 128, M < 1, group != 32, or too large  */
+    SQ_ERR_ALIGN = 3,      /* pointer not 16-byte (workspace: 256-byte) aligned   */
+    SQ_ERR_WORKSPACE = 4,  /* workspace smaller than sq_workspace_bytes()         */
+    SQ_ERR_DEVICE = 5,     /* current device is not sm_100 (B200 class)          */
+    SQ_ERR_CUDA = 6,       /* a CUDA call or launch failed                        */
+    SQ_ERR_ARG = 7,        /* bad enum / flag value                               */
+    SQ_ERR_TIMEOUT = 8     /* a kernel gave up a bounded wait (device status word) */
+} sq_status;
+
+typedef enum {
+    SQ_FMT_INT4_G32 = 1,   /* int4 codes [N, K/2], fp16 scales [N, K/32]          */
+    SQ_FMT_NVFP4 = 2       /* e2m1 codes [N, K/2], ue4m3 tiled scales, fp32 g_w   */
+} sq_format;
+
+/* operations for sq_workspace_bytes() */
+typedef enum {
+    SQ_OP_BUILD_INT4 = 1,
+    SQ_OP_BUILD_NVFP4 = 2,
+    SQ_OP_ACT_QUANT_NVFP4 = 3,
+    SQ_OP_LINEAR_FWD_NVFP4 = 4,
+    SQ_OP_LINEAR_FWD_INT4 = 5,
+    SQ_OP_RECONSTRUCT = 6
+} sq_op;
+
+/* flags */
+#define SQ_ACT_STATIC_SCALE    0x1u  /* sq_act_quant_nvfp4 / sq_linear_fwd: *g_x is an input */
+#define SQ_RECON_RESIDUAL_ONLY 0x2u  /* sq_reconstruct_bf16: drop the low-rank term        */
+
+/*
+ * A built weight.  All pointers are device pointers owned by the caller.
+ *   fmt        SQ_FMT_INT4_G32 or SQ_FMT_NVFP4
+ *   N, K       output / input features
+ *   codes      [N, K/2] uint8, value 2k in the low nibble of byte k
+ *              (int4: 4-bit two's complement in [-7, 7]; NVFP4: e2m1)
+ *   scales     int4: fp16 bits [N, K/32]; NVFP4: ue4m3 bytes in the tiled
+ *              layout, sq_sf_bytes(N, K) bytes
+ *   g_w        NVFP4 only: 1 float, the per-tensor global scale
+ *   lora_up    bf16 [N, 32], or NULL for no low-rank branch
+ *   lora_down  bf16 [K, 32], or NULL for no low-rank branch
+ */
+typedef struct {
+    int32_t fmt;
+    int64_t N;
+    int64_t K;
+    const uint8_t *codes;
+    const void *scales;
+    const float *g_w;
+    const uint16_t *lora_up;
+    const uint16_t *lora_down;
+} sq_weight;
+
+/* Human-readable name of a status code (static string). */
+SQ_API const char *sq_status_str(int status);
+
+/* ABI version, currently 1. */
+SQ_API int sq_abi_version(void);
+
+/*
+ * Text of the last failing CUDA call or device check made by this thread
+ * inside libsq (static thread-local buffer; "" if none).
+ */
+SQ_API const char *sq_last_error_detail(void);
+
+/*
+ * Bytes of a tiled NVFP4 scale buffer for `rows` rows of K values:
+ * ceil(rows/128)*128 * K/16.  The layout is the public cuBLAS / tcgen05
+ * 1D block-scaling layout: 512-byte tiles of 128 rows x 4 scales; scale
+ * (r, c), C = K/16, sits at byte
+ *   ((r/128)*(C/4) + c/4)*512 + (r%32)*16 + ((r%128)/32)*4 + c%4.
+ * Rows past `rows` up to the next multiple of 128 hold 0.
+ */
+SQ_API size_t sq_sf_bytes(int64_t rows, int64_t K);
+
+/* Workspace bytes an operation needs for the given shape (M unused for builds). */
+SQ_API size_t sq_workspace_bytes(int op, int64_t M, int64_t N, int64_t K);
+
+/*
+ * int4 group-32 builder (SquareQ README, "Residual codecs": int4 group-32
+ * scales with MSE-swept fractions).  For each row of R [N, K] fp32 (device):
+ * rotate every 256-block with H256, then for each group of 32 rotated values
+ * r_i with a = max|r_i| try the fractions f_j = (50 + 2j)/100, j = 0..25:
+ *   s_j = fp16(RN(RN(f_j a) / 7)),  q_i = clamp(rint(RN(r_i RN(1/s_j))), -7, 7),
+ *   error_j = sum over an xor butterfly (strides 16,8,4,2,1) of RN((r_i - q_i s_j)^2)
+ * (a scale of 0 gives q = 0 and error r_i^2); keep the smallest error, the
+ * smaller j on ties.  Outputs (device): codes [N, K/2], scales fp16 bits
+ * [N, K/32], frac_idx [N, K/32] winning j (may be NULL).  group must be 32.
+ * Rotated values must stay below 458000 in magnitude (fp16 scale range).
+ */
+SQ_API sq_status sq_build_int4(const float *R, int64_t N, int64_t K, int32_t group,
+                        uint8_t *codes, uint16_t *scales, uint8_t *frac_idx,
+                        void *stream);
+
+/*
+ * NVFP4 builder (SquareQ README, "Residual codecs": e2m1 + ue4m3 block-16
+ * scales in the tiled layout + per-tensor global scale).  Pass 1 rotates R
+ * [N, K] fp32 (device) and takes A = max|H R|; g_w = RN(A / 2688), i.e.
+ * A / (6 * 448).  Pass 2 rotates again and, per 16 values with b = max|r|:
+ *   sf = ue4m3(RN(b / RN(6 g_w))),  code_i = e2m1(RN(r_i RN(1 / RN(value(sf) g_w))))
+ * (sf == 0 or g_w == 0 gives zero codes; negative values rounding to 0 keep
+ * the sign bit, code 0x8).  Outputs (device): codes [N, K/2], sf_tiled
+ * (sq_sf_bytes(N, K) bytes), g_w (1 float).  ws: sq_workspace_bytes(
+ * SQ_OP_BUILD_NVFP4, 0, N, K) bytes of device scratch (holds the absmax).
+ */
+SQ_API sq_status sq_build_nvfp4(const float *R, int64_t N, int64_t K,
+                         uint8_t *codes, uint8_t *sf_tiled, float *g_w,
+                         void *ws, size_t ws_bytes, void *stream);
+
+/*
+ * Activation quantisation, the prologue of the NVFP4 forward (SquareQ README,
+ * "Op-level parity of the full FP4 forward": H256-rotate + block-quant + tiled
+ * scales).  x [M, K] bf16 (device) is rotated; g_x = RN(max|H x| / 2688)
+ * unless SQ_ACT_STATIC_SCALE is set, in which case *g_x (device) is read as
+ * given.  Then the same block-16 step as sq_build_nvfp4 with g_x.  Outputs
+ * (device): codes [M, K/2], sf_tiled (sq_sf_bytes(M, K) bytes, padding rows
+ * 0), g_x (written unless static).  If lora_down (bf16 [K, 32]) and t are
+ * both non-NULL, also t[m, r] = sum_k x[m, k] lora_down[k, r] as fp32 [M, 32]
+ * (the low-rank input; fp32 accumulation, order unspecified).
+ */
+SQ_API sq_status sq_act_quant_nvfp4(const uint16_t *x, int64_t M, int64_t K,
+                             uint8_t *codes, uint8_t *sf_tiled, float *g_x,
+                             const uint16_t *lora_down, float *t, uint32_t flags,
+                             void *ws, size_t ws_bytes, void *stream);
+
+/*
+ * Forward y = x W^T, y [M, N] fp32 (device), x [M, K] bf16 (device).
+ * Because H is symmetric, x W^T = H(x) deq(Q)^T + (x lora_down) lora_up^T.
+ *   NVFP4: the activation prologue above, then a block-scaled e2m1 x e2m1
+ *          tensor-core GEMM (tcgen05, fp32 accumulation in tensor memory),
+ *          y = g_x g_w acc + t lora_up^T.
+ *   int4:  "dequant-first": xb = bf16(H x), wb = bf16(q s), y = xb wb^T +
+ *          t lora_up^T on bf16 tensor cores (fp32 accumulation).
+ * The low-rank term is accumulated on the tensor cores in the same
+ * accumulator.  Accuracy: max|y - y_exact| / max|y_exact| <= 2e-3 against the
+ * exact result on the same quantised operands.  flags: SQ_ACT_STATIC_SCALE
+ * (NVFP4; *g_x is then an input, g_x must be non-NULL).  g_x (device, may be
+ * NULL unless static) receives the activation global scale.  ws:
+ * sq_workspace_bytes(SQ_OP_LINEAR_FWD_NVFP4 or _INT4, M, N, K) bytes.
+ */
+SQ_API sq_status sq_linear_fwd(const sq_weight *w, const uint16_t *x, int64_t M, float *y,
+                        float *g_x, uint32_t flags, void *ws, size_t ws_bytes,
+                        void *stream);
+
+/*
+ * bf16 reconstruct of W for the backward pass (SquareQ README: "the bwd-side
+ * bf16 reconstruct from the same payload").  For each element
+ *   d = q s (int4) or RN(RN(e2m1 value(sf)) g_w) (NVFP4),
+ *   h = H256 applied to each 256-block of d along K,
+ *   L = fmaf(U[n,31], D[k,31], ... fmaf(U[n,0], D[k,0], 0)),
+ *   W[n, k] = bf16(RN(L + h))          (bf16(h) with SQ_RECON_RESIDUAL_ONLY
+ *                                       or NULL low-rank pointers).
+ * W_out: [N, K] bf16 (device).
+ */
+SQ_API sq_status sq_reconstruct_bf16(const sq_weight *w, uint16_t *W_out, uint32_t flags,
+                              void *stream);
+
+/*
+ * Read back and clear the device status word that a forward kernel sets when
+ * it gives up a bounded wait (SQ_ERR_TIMEOUT); ws is the workspace of the
+ * sq_linear_fwd call to check (each such call clears the word when it
+ * starts).  This call synchronises `stream` and copies 4 bytes to the host.
+ */
+SQ_API sq_status sq_check_device_status(void *ws, void *stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SQ_H */

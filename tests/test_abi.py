@@ -1,0 +1,130 @@
+"""Host-side tests of the C ABI (no GPU needed): the library loads, exports
+every entry point that include/sq.h declares, computes its size helpers, and
+rejects bad arguments with the documented status before touching the device.
+Fault injection happens on the host only (NULL, misaligned and mis-shaped
+arguments, an undersized workspace, a missing device)."""
+import ctypes
+import os
+import re
+
+import pytest
+import torch
+
+import bit_quantized_frozen_b200 as sq
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "sq.h")
+
+SQ_ERR_NULL, SQ_ERR_SHAPE, SQ_ERR_ALIGN, SQ_ERR_WORKSPACE, SQ_ERR_DEVICE, SQ_ERR_ARG = 1, 2, 3, 4, 5, 7
+
+# fake, never dereferenced device addresses: validation fails before any CUDA call
+A = 0x7F0000000000
+MIS = A + 8
+
+
+def header_functions():
+    text = open(HEADER).read()
+    return sorted(set(re.findall(r"^SQ_API[^;(]*?\b(sq_\w+)\s*\(", text, re.M)))
+
+
+def test_header_declares_the_five_operations():
+    names = header_functions()
+    for op in ["sq_build_int4", "sq_build_nvfp4", "sq_act_quant_nvfp4", "sq_linear_fwd", "sq_reconstruct_bf16"]:
+        assert op in names
+
+
+def test_library_exports_every_declared_symbol():
+    L = ctypes.CDLL(sq.LIB_PATH)
+    for name in header_functions():
+        assert hasattr(L, name), name
+    assert sorted(sq.EXPORTED) == header_functions()
+
+
+def test_size_helpers():
+    assert sq.sq_abi_version() == 1
+    assert sq.sq_sf_bytes(1, 256) == 128 * 16
+    assert sq.sq_sf_bytes(128, 512) == 128 * 32
+    assert sq.sq_sf_bytes(129, 512) == 256 * 32
+    assert sq.sq_sf_bytes(4480, 6144) == 4480 * 384
+    assert sq.sq_workspace_bytes(sq.SQ_OP_BUILD_NVFP4, 0, 256, 512) >= 8
+    ws = sq.sq_workspace_bytes(sq.SQ_OP_LINEAR_FWD_NVFP4, 64, 256, 512)
+    assert ws >= 64 * 256 + sq.sq_sf_bytes(64, 512) + 64 * 128 + 256 * 128 + 512 * 64
+    wsi = sq.sq_workspace_bytes(sq.SQ_OP_LINEAR_FWD_INT4, 64, 256, 512)
+    assert wsi >= 64 * 512 * 2 + 256 * 512 * 2
+    assert sq.sq_workspace_bytes(99, 1, 1, 1) == 0
+    assert sq.status_str(0) == "ok"
+    assert sq.status_str(2) == "unsupported shape"
+
+
+def _int4(R=A, N=256, K=512, group=32, codes=A, scales=A, frac=None):
+    return sq.lib().sq_build_int4(R, N, K, group, codes, scales, frac, None)
+
+
+def test_build_int4_validation():
+    assert _int4(R=None) == SQ_ERR_NULL
+    assert _int4(codes=None) == SQ_ERR_NULL
+    assert _int4(K=300) == SQ_ERR_SHAPE
+    assert _int4(N=100) == SQ_ERR_SHAPE
+    assert _int4(group=64) == SQ_ERR_SHAPE
+    assert _int4(R=MIS) == SQ_ERR_ALIGN
+    assert _int4(frac=MIS) == SQ_ERR_ALIGN
+
+
+def test_build_nvfp4_validation():
+    L = sq.lib()
+    assert L.sq_build_nvfp4(A, 256, 512, A, A, A, None, 256, None) == SQ_ERR_NULL
+    assert L.sq_build_nvfp4(A, 256, 250, A, A, A, A, 256, None) == SQ_ERR_SHAPE
+    assert L.sq_build_nvfp4(A, 256, 512, A, A, A, A + 16, 256, None) == SQ_ERR_ALIGN
+    assert L.sq_build_nvfp4(A, 256, 512, A, A, A, A, 4, None) == SQ_ERR_WORKSPACE
+
+
+def test_act_quant_validation():
+    L = sq.lib()
+    big = 1 << 30
+    assert L.sq_act_quant_nvfp4(None, 4, 512, A, A, A, None, None, 0, A, big, None) == SQ_ERR_NULL
+    assert L.sq_act_quant_nvfp4(A, 0, 512, A, A, A, None, None, 0, A, big, None) == SQ_ERR_SHAPE
+    assert L.sq_act_quant_nvfp4(A, 4, 512, A, A, A, None, None, 0x80, A, big, None) == SQ_ERR_ARG
+    assert L.sq_act_quant_nvfp4(A, 4, 512, A, A, A, None, MIS, 0, A, big, None) == SQ_ERR_ALIGN
+    assert L.sq_act_quant_nvfp4(A, 4, 512, A, A, A, None, None, 0, A, 16, None) == SQ_ERR_WORKSPACE
+
+
+def _w(fmt=sq.SQ_FMT_NVFP4, N=256, K=512, codes=A, scales=A, g_w=A, U=A, D=A):
+    return sq.sq_weight(fmt, N, K, codes, scales, g_w, U, D)
+
+
+def test_linear_fwd_validation():
+    L = sq.lib()
+    big = 1 << 34
+    fwd = lambda w, x=A, M=8, y=A, gx=None, fl=0, ws=A, wsb=big: L.sq_linear_fwd(
+        ctypes.byref(w), x, M, y, gx, fl, ws, wsb, None)
+    assert fwd(_w(codes=None)) == SQ_ERR_NULL
+    assert fwd(_w(g_w=None)) == SQ_ERR_NULL
+    assert fwd(_w(fmt=7)) == SQ_ERR_ARG
+    assert fwd(_w(N=192)) == SQ_ERR_SHAPE
+    assert fwd(_w(), M=0) == SQ_ERR_SHAPE
+    assert fwd(_w(), y=MIS) == SQ_ERR_ALIGN
+    assert fwd(_w(), ws=A + 64) == SQ_ERR_ALIGN
+    assert fwd(_w(), wsb=100) == SQ_ERR_WORKSPACE
+    assert fwd(_w(), fl=sq.SQ_ACT_STATIC_SCALE) == SQ_ERR_NULL          # static scale needs g_x
+    assert fwd(_w(fmt=sq.SQ_FMT_INT4_G32, g_w=None), gx=A, fl=sq.SQ_ACT_STATIC_SCALE) == SQ_ERR_ARG
+    assert fwd(_w(), fl=0x40) == SQ_ERR_ARG
+
+
+def test_reconstruct_validation():
+    L = sq.lib()
+    assert L.sq_reconstruct_bf16(ctypes.byref(_w()), None, 0, None) == SQ_ERR_NULL
+    assert L.sq_reconstruct_bf16(ctypes.byref(_w()), MIS, 0, None) == SQ_ERR_ALIGN
+    assert L.sq_reconstruct_bf16(ctypes.byref(_w()), A, 0x10, None) == SQ_ERR_ARG
+    assert L.sq_reconstruct_bf16(ctypes.byref(_w(U=MIS)), A, 0, None) == SQ_ERR_ALIGN
+
+
+@pytest.mark.skipif(torch.cuda.is_available(), reason="checks the no-device path")
+def test_valid_call_without_device_reports_device_error():
+    assert _int4() == SQ_ERR_DEVICE
+    assert sq.lib().sq_reconstruct_bf16(ctypes.byref(_w()), A, 0, None) == SQ_ERR_DEVICE
+
+
+def test_binding_raises_with_status():
+    with pytest.raises(sq.SqError) as e:
+        sq._check("sq_build_int4", SQ_ERR_SHAPE)
+    assert e.value.status == SQ_ERR_SHAPE
