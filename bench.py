@@ -1,0 +1,500 @@
+#!/usr/bin/env python
+"""Benchmark of the SquareQ W4 linear layer hot path on B200.
+
+One step = one pass of the whole hot path over one synthetic layer of the
+chosen shape (default the headline 4480 x 16384 x 6144, M x N x K):
+  sq_build_int4, sq_build_nvfp4, sq_linear_fwd (NVFP4, incl. the activation
+  prologue), sq_linear_fwd (int4), sq_reconstruct_bf16 (both payloads).
+Every op is timed with CUDA events on the launching stream after an L2 flush
+(a 256 MB write outside the op's events); the NVFP4 forward is the headline
+metric (TFLOP/s = 2 M N K / time of the whole sq_linear_fwd call).  The GEMM
+kernel alone is timed with events recorded around its launch inside the
+library (sq_set_gemm_events) for the roofline line.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
+
+With N > 1 (launched by torch.distributed.run) every rank runs an independent
+replica (the layer does not shard; no collective on the data path) and the
+device time is the max over ranks.  --impl reference times the CPU oracle on a
+bounded sample of the same workload on rank 0.
+"""
+from __future__ import annotations
+
+import argparse
+import datetime
+import hashlib
+import json
+import os
+import re
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import synth_inputs as si  # noqa: E402
+
+METRIC = "W4 linear fwd TFLOP/s & % FP4/BF16 tensor peak; quantize/reconstruct GB/s % HBM"
+HEADLINE = "large_4480x6144x16384"
+# SquareQ README, NVFP4 vs bf16 table: 4480 x 16384 x 6144 fp4 GEMM 1074 us on an
+# RTX 5080 (sm_120, cuBLASLt), i.e. 2*4480*16384*6144 / 1074e-6 = 840.3 TFLOP/s.
+PAGES_FP4_TFLOPS = {"large_4480x6144x16384": 2 * 4480 * 16384 * 6144 / 1074e-6 / 1e12}
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+FP4_PER_BF16 = 4.0        # nominal dense FP4 / BF16 tensor ratio (9 / 2.25 PFLOP/s)
+FLUSH_BYTES = 256 << 20   # > 126 MB L2
+
+
+def parse():
+    p = argparse.ArgumentParser()
+    p.add_argument("--gpus", type=int, default=1)
+    p.add_argument("--steps", type=int, default=50)
+    p.add_argument("--warmup", type=int, default=5)
+    p.add_argument("--impl", default="sq", choices=["sq", "reference"])
+    p.add_argument("--config", default=HEADLINE, choices=sorted(si.CONFIGS))
+    p.add_argument("--no-cpu-baseline", action="store_true")
+    p.add_argument("--no-e2e", action="store_true")
+    p.add_argument("--no-clocks", action="store_true")
+    return p.parse_args()
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            d = json.load(f)
+        return {k: float(d[k]) for k in ("hbm_gbs", "bf16_tflops", "bf16_tflops_sustained")}, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+# ---------------------------------------------------------------------------
+# per-op algorithmic work (bytes per element of the [N,K] or [M,K] operand)
+# ---------------------------------------------------------------------------
+
+def op_work(M, N, K):
+    NK, MK = N * K, M * K
+    return {
+        "build_int4": ("GB/s", NK * (4 + 0.5 + 2 / 32 + 1 / 32)),
+        "build_nvfp4": ("GB/s", NK * (4 + 0.5 + 1 / 16)),
+        "fwd_nvfp4": ("TFLOP/s", 2.0 * M * N * K),
+        "fwd_int4": ("TFLOP/s", 2.0 * M * N * K),
+        "reconstruct_nvfp4": ("GB/s", NK * (0.5 + 1 / 16 + 2)),
+        "reconstruct_int4": ("GB/s", NK * (0.5 + 2 / 32 + 2)),
+        "gemm_nvfp4": ("TFLOP/s", 2.0 * M * N * K),
+        "gemm_int4": ("TFLOP/s", 2.0 * M * N * K),
+    }
+
+
+LAUNCHES_PER_STEP = {   # our kernels per op (memsets excluded)
+    "build_int4": 1, "build_nvfp4": 2, "fwd_nvfp4": 5, "fwd_int4": 5,
+    "reconstruct_nvfp4": 1, "reconstruct_int4": 1,
+}
+
+
+# ---------------------------------------------------------------------------
+# clocks during the timed region
+# ---------------------------------------------------------------------------
+
+class ClockSampler:
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.hw_slowdown,"
+              "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+              "clocks_event_reasons.sw_power_cap,utilization.gpu")
+
+    def __init__(self, gpu_index: int):
+        self.idx = gpu_index
+        self.proc = None
+        self.lines = []
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.idx), f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "100"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.thread = threading.Thread(target=self._read, daemon=True)
+            self.thread.start()
+        except OSError:
+            self.proc = None
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        time.sleep(0.15)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        rows = []
+        for ln in self.lines:
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) < 8:
+                continue
+            try:
+                rows.append((float(parts[0]), float(parts[1]), parts[3:7], float(parts[7])))
+            except ValueError:
+                continue
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
+        loaded = [r for r in rows if r[3] > 0] or rows
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in loaded for i, v in enumerate(r[2]) if v.lower() == "active"})
+        return {"sm_mhz": statistics.median(r[0] for r in loaded), "sm_max_mhz": max(r[1] for r in rows),
+                "reasons": reasons, "samples": len(rows), "samples_under_load": len([r for r in rows if r[3] > 0])}
+
+
+def physical_gpu_index(local_rank: int) -> int:
+    vis = os.environ.get("CUDA_VISIBLE_DEVICES", "")
+    if vis:
+        ids = [v.strip() for v in vis.split(",") if v.strip()]
+        if local_rank < len(ids) and ids[local_rank].isdigit():
+            return int(ids[local_rank])
+    return local_rank
+
+
+# ---------------------------------------------------------------------------
+# roofline traffic from the committed ncu summary (null once the kernel changed)
+# ---------------------------------------------------------------------------
+
+GEMM_SOURCES = ["bit_quantized_frozen_b200/csrc/sq_gemm.cu", "bit_quantized_frozen_b200/csrc/sq_ptx.cuh"]
+
+
+def gemm_source_hash() -> str:
+    h = hashlib.sha256()
+    for rel in GEMM_SOURCES:
+        with open(os.path.join(ROOT, rel), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def profiled_traffic(config: str):
+    """dram bytes per launch of the NVFP4 GEMM from profiles/, scaled to `config`."""
+    path = os.path.join(ROOT, "profiles", "gemm_nvfp4_ncu.md")
+    if not os.path.exists(path):
+        return None, "no ncu summary"
+    text = open(path).read()
+    m_hash = re.search(r"kernel_source_sha256:\s*([0-9a-f]+)", text)
+    if not m_hash or m_hash.group(1) != gemm_source_hash():
+        return None, "kernel changed since the ncu capture"
+    m = re.search(rf"traffic_bytes_per_launch\[{re.escape(config)}\]:\s*([0-9.eE+]+)", text)
+    if not m:
+        return None, "no capture for this workload"
+    return float(m.group(1)), "ncu"
+
+
+# ---------------------------------------------------------------------------
+# CPU oracle on a bounded sample of the workload
+# ---------------------------------------------------------------------------
+
+def cpu_sample(d, M_s: int, N_s: int):
+    """Run the oracle's whole pipeline on rows [0, N_s) of R and [0, M_s) of x.
+    Returns per-op seconds."""
+    import oracle
+    oracle.build()
+    R = np.ascontiguousarray(d["R"][:N_s])
+    x = np.ascontiguousarray(d["x"][:M_s])
+    U = np.ascontiguousarray(d["U"][:N_s])
+    D = d["D"]
+    K = R.shape[1]
+    t = {}
+    t0 = time.perf_counter()
+    c4, s4, _ = oracle.build_int4(R)
+    t["build_int4"] = time.perf_counter() - t0
+    t0 = time.perf_counter()
+    wc, wsf, gw = oracle.build_nvfp4(R)
+    t["build_nvfp4"] = time.perf_counter() - t0
+    t0 = time.perf_counter()
+    xc, xsf, gx, tt = oracle.act_quant_nvfp4(x, D)
+    oracle.linear_fwd_nvfp4(xc, xsf, gx, wc, wsf, gw, tt, U, M_s, N_s, K)
+    t["fwd_nvfp4"] = time.perf_counter() - t0
+    t0 = time.perf_counter()
+    xr = oracle.rotate_rows_bf16(x)
+    _, _, _, tt2 = oracle.act_quant_nvfp4(x, D)
+    oracle.linear_fwd_int4(xr, c4, s4, tt2, U, M_s, N_s, K)
+    t["fwd_int4"] = time.perf_counter() - t0
+    t0 = time.perf_counter()
+    oracle.reconstruct_bf16(2, wc, wsf, gw, U, D, N_s, K)
+    t["reconstruct_nvfp4"] = time.perf_counter() - t0
+    t0 = time.perf_counter()
+    oracle.reconstruct_bf16(1, c4, s4, 0.0, U, D, N_s, K)
+    t["reconstruct_int4"] = time.perf_counter() - t0
+    return t, oracle.num_threads()
+
+
+REF_SAMPLE = (64, 2048)    # reference arm, per step: M_s rows of x, N_s rows of R (all K)
+CPU_SAMPLE = (128, 4096)   # one-off CPU baseline of the GPU arm
+
+
+def cpu_sample_desc(cfg, M_s, N_s):
+    return (f"oracle pipeline on x rows 0..{M_s - 1} and R rows 0..{N_s - 1} (all K={cfg.K}) of the "
+            f"{cfg.M}x{cfg.N}x{cfg.K} workload; metric = 2*{M_s}*{N_s}*{cfg.K} / oracle NVFP4-forward time")
+
+
+def run_reference(args, cfg, d):
+    M_s, N_s = REF_SAMPLE
+    flops = 2.0 * M_s * N_s * cfg.K
+    for _ in range(args.warmup):
+        cpu_sample(d, M_s, N_s)
+    times = []
+    cores = 1
+    t_start = time.perf_counter()
+    for _ in range(args.steps):
+        t, cores = cpu_sample(d, M_s, N_s)
+        times.append(t)
+    wall = time.perf_counter() - t_start
+    fwd = statistics.mean(t["fwd_nvfp4"] for t in times)
+    value = flops / fwd / 1e12
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": wall / max(args.steps, 1) * 1e3,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "f64 (oracle, exact decoded operands)", "data": "synthetic (seeded)",
+        "config": workload_config(cfg, args),
+        "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
+                         "sample": cpu_sample_desc(cfg, M_s, N_s)},
+        "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+        "ops_s": {k: statistics.mean(t[k] for t in times) for k in times[0]},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def workload_config(cfg, args):
+    return {
+        "workload": f"SquareQ W4 linear {cfg.M}x{cfg.N}x{cfg.K} (M tokens x N out x K in), rank 32, "
+                    f"seed {cfg.seed}, {cfg.dist} residual" + (f", {cfg.hot_channels} hot channels"
+                                                              if cfg.hot_channels else ""),
+        "name": cfg.name, "M": cfg.M, "N": cfg.N, "K": cfg.K, "rank": 32,
+        "codecs": ["nvfp4 (e2m1, ue4m3 block-16, fp32 global)", "int4 group-32 MSE-swept"],
+        "l2": "flushed (256 MB write) before every op, outside its events",
+        "parallelism": f"replicas x{args.gpus}",
+    }
+
+
+# ---------------------------------------------------------------------------
+# the CUDA path
+# ---------------------------------------------------------------------------
+
+def run_sq(args, cfg, d, rank, world, local_rank):
+    import torch
+    import bit_quantized_frozen_b200 as sq
+
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    M, N, K = cfg.M, cfg.N, cfg.K
+    to_bf16 = lambda a: torch.from_numpy(a.view(np.int16)).to(dev).view(torch.bfloat16)
+    R = torch.from_numpy(d["R"]).to(dev)
+    x = to_bf16(d["x"])
+    U = to_bf16(d["U"])
+    D = to_bf16(d["D"])
+
+    # outputs and workspaces, allocated once
+    i4 = sq.Weight(sq.SQ_FMT_INT4_G32, N, K, torch.empty((N, K // 2), dtype=torch.uint8, device=dev),
+                   torch.empty((N, K // 32), dtype=torch.float16, device=dev), None, U, D,
+                   torch.empty((N, K // 32), dtype=torch.uint8, device=dev))
+    nv = sq.Weight(sq.SQ_FMT_NVFP4, N, K, torch.empty((N, K // 2), dtype=torch.uint8, device=dev),
+                   torch.empty(sq.sq_sf_bytes(N, K), dtype=torch.uint8, device=dev),
+                   torch.empty(1, dtype=torch.float32, device=dev), U, D)
+    ws_b = sq.workspace(sq.SQ_OP_BUILD_NVFP4, 0, N, K, dev)
+    ws_nv = sq.workspace(sq.SQ_OP_LINEAR_FWD_NVFP4, M, N, K, dev)
+    ws_i4 = sq.workspace(sq.SQ_OP_LINEAR_FWD_INT4, M, N, K, dev)
+    g_x = torch.empty(1, dtype=torch.float32, device=dev)
+    y_nv = torch.empty((M, N), dtype=torch.float32, device=dev)
+    y_i4 = torch.empty((M, N), dtype=torch.float32, device=dev)
+    W = torch.empty((N, K), dtype=torch.bfloat16, device=dev)
+    flush = torch.empty(FLUSH_BYTES // 4, dtype=torch.int32, device=dev)
+
+    ops = [
+        ("build_int4", lambda: sq.sq_build_int4(R, i4.codes, i4.scales, i4.frac_idx)),
+        ("build_nvfp4", lambda: sq.sq_build_nvfp4(R, nv.codes, nv.scales, nv.g_w, ws_b)),
+        ("fwd_nvfp4", lambda: sq.sq_linear_fwd(nv, x, y_nv, g_x=g_x, ws=ws_nv)),
+        ("fwd_int4", lambda: sq.sq_linear_fwd(i4, x, y_i4, ws=ws_i4)),
+        ("reconstruct_nvfp4", lambda: sq.sq_reconstruct_bf16(nv, W)),
+        ("reconstruct_int4", lambda: sq.sq_reconstruct_bf16(i4, W)),
+    ]
+    names = [n for n, _ in ops]
+    gemm_of = {"fwd_nvfp4": "gemm_nvfp4", "fwd_int4": "gemm_int4"}
+
+    def run_step(evs):
+        for name, fn in ops:
+            flush.fill_(1)
+            if evs is None:
+                fn()
+                continue
+            a, b = evs[name]
+            if name in gemm_of:
+                ga, gb = evs[gemm_of[name]]
+                sq.sq_set_gemm_events(ga, gb)
+            a.record()
+            fn()
+            b.record()
+            if name in gemm_of:
+                sq.sq_set_gemm_events(None, None)
+
+    for _ in range(args.warmup):
+        run_step(None)
+    torch.cuda.synchronize()
+    sq.sq_check_device_status(ws_nv)
+    sq.sq_check_device_status(ws_i4)
+
+    keys = names + list(gemm_of.values())
+    evs = [{k: (torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for k in keys}
+           for _ in range(args.steps)]
+    outer = (torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+    sampler = None
+    if rank == 0 and not args.no_clocks:
+        sampler = ClockSampler(physical_gpu_index(local_rank))
+        sampler.start()
+        time.sleep(0.3)
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+    outer[0].record()
+    for s in range(args.steps):
+        run_step(evs[s])
+    outer[1].record()
+    torch.cuda.synchronize()
+    if world > 1:
+        torch.distributed.barrier()
+    clocks = sampler.stop() if sampler else None
+    sq.sq_check_device_status(ws_nv)
+    sq.sq_check_device_status(ws_i4)
+
+    per_op = {k: statistics.mean(e[k][0].elapsed_time(e[k][1]) for e in evs) for k in keys}   # ms
+    outer_ms = outer[0].elapsed_time(outer[1]) / max(args.steps, 1)
+    if world > 1:
+        t = torch.tensor([per_op[k] for k in keys] + [outer_ms], dtype=torch.float64, device=dev)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        vals = t.tolist()
+        per_op = dict(zip(keys, vals[:-1]))
+        outer_ms = vals[-1]
+
+    # end to end through the C ABI with host buffers: H2D of x, forward, D2H of y
+    e2e = None
+    if not args.no_e2e:
+        x_host = torch.from_numpy(d["x"].view(np.int16)).view(torch.bfloat16).pin_memory()
+        y_host = torch.empty((M, N), dtype=torch.float32).pin_memory()
+        x_dev = torch.empty_like(x)
+        reps = 3
+        for _ in range(1):
+            x_dev.copy_(x_host, non_blocking=True)
+            sq.sq_linear_fwd(nv, x_dev, y_nv, g_x=g_x, ws=ws_nv)
+            y_host.copy_(y_nv, non_blocking=True)
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for _ in range(reps):
+            x_dev.copy_(x_host, non_blocking=True)
+            sq.sq_linear_fwd(nv, x_dev, y_nv, g_x=g_x, ws=ws_nv)
+            y_host.copy_(y_nv, non_blocking=True)
+        e1.record()
+        torch.cuda.synchronize()
+        e2e_ms = e0.elapsed_time(e1) / reps
+        if world > 1:
+            t = torch.tensor([e2e_ms], dtype=torch.float64, device=dev)
+            torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+            e2e_ms = t.item()
+        e2e = {"value": world * 2.0 * M * N * K / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
+               "h2d_bytes_per_step": int(M * K * 2), "d2h_bytes_per_step": int(M * N * 4),
+               "ms_per_step": e2e_ms, "path": "pinned x -> device, sq_linear_fwd (NVFP4), y -> pinned host"}
+    return per_op, outer_ms, clocks, e2e
+
+
+def summarise(args, cfg, per_op, outer_ms, clocks, e2e, world, cpu):
+    peaks, peak_src = load_peaks()
+    fp4_peak = peaks["bf16_tflops"] * FP4_PER_BF16
+    M, N, K = cfg.M, cfg.N, cfg.K
+    work = op_work(M, N, K)
+    ops = {}
+    for k, ms in per_op.items():
+        unit, amount = work[k]
+        rate = amount / (ms * 1e-3) / (1e12 if unit == "TFLOP/s" else 1e9)
+        if unit == "GB/s":
+            frac, peak = rate / peaks["hbm_gbs"], "hbm"
+        else:
+            peak_v = fp4_peak if "nvfp4" in k else peaks["bf16_tflops"]
+            frac, peak = rate / peak_v, "fp4 tensor" if "nvfp4" in k else "bf16 tensor"
+        ops[k] = {"ms": ms, unit: rate, "frac": frac, "of": f"{peak} ({peak_src})"}
+    fwd_tflops = 2.0 * M * N * K / (per_op["fwd_nvfp4"] * 1e-3) / 1e12
+    gemm_tflops = 2.0 * M * N * K / (per_op["gemm_nvfp4"] * 1e-3) / 1e12
+    traffic, traffic_src = profiled_traffic(cfg.name)
+    step_ms = sum(per_op[k] for k in LAUNCHES_PER_STEP)
+    base = PAGES_FP4_TFLOPS.get(cfg.name)
+    line = {
+        "metric": METRIC,
+        "value": world * fwd_tflops,
+        "unit": "TFLOP/s",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": step_ms,
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": (world * fwd_tflops / base) if base else None,
+        "vs_baseline_note": ("pages' RTX 5080 (sm_120) cuBLASLt fp4 GEMM-only time for this shape; "
+                             "context, not a target") if base else None,
+        "dtype": "e2m1 x e2m1 with ue4m3 block-16 scales -> fp32 (NVFP4 headline); bf16 x bf16 -> fp32 (int4 path)",
+        "data": "synthetic (seeded numpy; shapes/distributions of the pages' model layers)",
+        "config": workload_config(cfg, args),
+        "roofline": {
+            "kernel": "sq_gemm_kernel<NVFP4> (tcgen05 block-scaled GEMM + low-rank step + epilogue)",
+            "bound": "tensor",
+            "achieved": gemm_tflops,
+            "peak": fp4_peak,
+            "unit": "TFLOP/s",
+            "frac": gemm_tflops / fp4_peak,
+            "peak_source": f"{peak_src} bf16 burst {peaks['bf16_tflops']} TFLOP/s x {FP4_PER_BF16} (nominal fp4/bf16)",
+            "traffic": traffic,
+            "traffic_source": traffic_src,
+            "algorithmic": f"2*M*N*K = {2.0 * M * N * K:.4g} flop per launch",
+        },
+        "ops": ops,
+        "ms_per_step_with_flushes": outer_ms,
+        "gpu_launches": sum(LAUNCHES_PER_STEP.values()) * args.steps,
+        "clocks": clocks,
+        "e2e": e2e,
+        "cpu_baseline": cpu,
+    }
+    return line
+
+
+def main():
+    args = parse()
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    cfg = si.CONFIGS[args.config]
+    if args.impl == "reference":
+        if rank != 0:
+            return
+        d = si.make_config(cfg.name)
+        run_reference(args, cfg, d)
+        return
+    import torch
+    if world > 1:
+        torch.cuda.set_device(local_rank)
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                             device_id=torch.device("cuda", local_rank))
+    d = si.make_config(cfg.name)
+    per_op, outer_ms, clocks, e2e = run_sq(args, cfg, d, rank, world, local_rank)
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        M_s, N_s = CPU_SAMPLE
+        t, cores = cpu_sample(d, M_s, N_s)
+        cpu = {"value": 2.0 * M_s * N_s * cfg.K / t["fwd_nvfp4"] / 1e12, "unit": "TFLOP/s", "cores": cores,
+               "kind": "oracle", "sample": cpu_sample_desc(cfg, M_s, N_s), "ops_s": t}
+    if rank == 0:
+        print(json.dumps(summarise(args, cfg, per_op, outer_ms, clocks, e2e, world, cpu)), flush=True)
+    if world > 1:
+        torch.distributed.barrier()
+        torch.distributed.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -37,7 +37,7 @@ RANK = 32
 EXPORTED = [
     "sq_status_str", "sq_abi_version", "sq_last_error_detail", "sq_sf_bytes", "sq_workspace_bytes",
     "sq_build_int4", "sq_build_nvfp4", "sq_act_quant_nvfp4", "sq_linear_fwd", "sq_reconstruct_bf16",
-    "sq_check_device_status",
+    "sq_check_device_status", "sq_set_gemm_events",
 ]
 
 
@@ -79,6 +79,7 @@ _SIGS = {
                       ctypes.c_int),
     "sq_reconstruct_bf16": ([ctypes.POINTER(sq_weight), _P, ctypes.c_uint32, _P], ctypes.c_int),
     "sq_check_device_status": ([_P, _P], ctypes.c_int),
+    "sq_set_gemm_events": ([_P, _P], ctypes.c_int),
 }
 _lib = None
 
@@ -179,6 +180,18 @@ def sq_reconstruct_bf16(w: "Weight", W_out, flags: int = 0, stream=None):
 
 def sq_check_device_status(ws, stream=None):
     _check("sq_check_device_status", lib().sq_check_device_status(_ptr(ws), _stream(stream)))
+
+
+def sq_set_gemm_events(start_event=None, stop_event=None):
+    """Record these torch.cuda.Event objects around the GEMM launch of later
+    sq_linear_fwd calls on this thread (None, None turns it off)."""
+    def handle(ev):
+        if ev is None:
+            return None
+        if ev.cuda_event == 0:          # torch creates the CUDA event lazily
+            ev.record()
+        return ev.cuda_event
+    _check("sq_set_gemm_events", lib().sq_set_gemm_events(handle(start_event), handle(stop_event)))
 
 
 # ---- a built weight and allocating helpers (torch provides the memory) --------

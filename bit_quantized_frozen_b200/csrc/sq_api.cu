@@ -17,6 +17,8 @@ int g_sms[kMaxDevices];          // 0 = not yet queried
 int g_cc_ok[kMaxDevices];        // 0 unknown, 1 sm_100, -1 other
 
 thread_local char g_detail[256] = "";
+thread_local cudaEvent_t g_gemm_ev0 = nullptr;   // sq_set_gemm_events
+thread_local cudaEvent_t g_gemm_ev1 = nullptr;
 
 void set_detail(const char *what, cudaError_t e)
 {
@@ -351,7 +353,11 @@ sq_status sq_linear_fwd(const sq_weight *w, const uint16_t *x, int64_t M, float 
         g.a = xb;
         g.b = wb;
     }
+    if (g_gemm_ev0)
+        SQ_CUDA(cudaEventRecord(g_gemm_ev0, s), "event record");
     SQ_CUDA(sq::launch_gemm(g, sms, s), "gemm");
+    if (g_gemm_ev1)
+        SQ_CUDA(cudaEventRecord(g_gemm_ev1, s), "event record");
     return SQ_OK;
 }
 
@@ -375,6 +381,15 @@ sq_status sq_reconstruct_bf16(const sq_weight *w, uint16_t *W_out, uint32_t flag
     SQ_CUDA(sq::launch_reconstruct(w->fmt, w->codes, w->scales, w->g_w, w->lora_up, w->lora_down, w->N, w->K,
                                    with_lowrank, W_out, s),
             "reconstruct");
+    return SQ_OK;
+}
+
+sq_status sq_set_gemm_events(void *start_event, void *stop_event)
+{
+    if ((start_event == nullptr) != (stop_event == nullptr))
+        return SQ_ERR_NULL;
+    g_gemm_ev0 = reinterpret_cast<cudaEvent_t>(start_event);
+    g_gemm_ev1 = reinterpret_cast<cudaEvent_t>(stop_event);
     return SQ_OK;
 }
 

@@ -34,10 +34,11 @@ namespace sq {
 
 constexpr int BM = 128;
 constexpr int BN = 256;
-constexpr int kRowBytes = 128;                 // every stage holds 128-byte rows (one swizzle atom)
-constexpr int kABytes = BM * kRowBytes;        // 16 KB
-constexpr int kBBytes = BN * kRowBytes;        // 32 KB
-constexpr int kSfaBytes = 4 * 512;             // 4 scale chunks of 128 rows x 4 scales
+constexpr int kRowBytes = 64;                  // every stage holds 64-byte rows (64B swizzle atom)
+constexpr int kABytes = BM * kRowBytes;        // 8 KB
+constexpr int kBBytes = BN * kRowBytes;        // 16 KB
+constexpr int kMmaPerStage = 2;                // two MMAs of 32 bytes of K each
+constexpr int kSfaBytes = kMmaPerStage * 512;  // one 512-byte scale chunk (128 rows x 4 scales) per MMA
 constexpr int kSfbBytes = 2 * kSfaBytes;       // 256 rows
 constexpr int kEpiWarps = 4;
 constexpr int kThreads = 192;
@@ -55,9 +56,9 @@ constexpr uint32_t kIdescNvfp4 = (1u << 7) | (1u << 10) | ((uint32_t)(BN >> 3) <
 
 template <bool FP4>
 struct GemmCfg {
-    static constexpr int kStages = FP4 ? 3 : 4;
+    static constexpr int kStages = FP4 ? 7 : 8;
     static constexpr int kStageBytes = kABytes + kBBytes + (FP4 ? kSfaBytes + kSfbBytes : 0);
-    static constexpr int kKPerStage = FP4 ? 256 : 64;            // K values per stage
+    static constexpr int kKPerStage = FP4 ? 128 : 32;            // K values per stage
     static constexpr int kStagingOff = kStages * kStageBytes;
     static constexpr int kBarOff = kStagingOff + kEpiWarps * 2 * kStagingBytes;
     static constexpr int kSmemBytes = kBarOff + 256 + 1024;      // barriers + 1 KB alignment slack
@@ -127,7 +128,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int n_tiles = (args.N + BN - 1) / BN;
     const int tiles = m_tiles * n_tiles;
     const int k_stages = args.K / Cfg::kKPerStage;
-    const int stages_per_tile = k_stages + (args.lora ? 1 : 0);
+    const int lora_stages = args.lora ? 2 : 0;                // [t_hi | U], then [t_lo | U]
+    const int stages_per_tile = k_stages + lora_stages;
     const int sf_chunks_per_row_tile = args.K / 64;          // 512-byte chunks per 128-row tile
 
     if (warp == 4) {
@@ -148,12 +150,12 @@ __global__ void __launch_bounds__(kThreads, 1)
                     uint8_t *sbase = smem + stage * Cfg::kStageBytes;
                     const uint32_t fb = bar_full + 8 * stage;
                     const uint32_t sA = smem_u32(sbase), sB = smem_u32(sbase + kABytes);
-                    if (args.lora && ks == 0) {
+                    if (ks < lora_stages) {
                         mbar_arrive_expect_tx(fb, kABytes + kBBytes);
-                        tma_load_2d(sA, &tmT, 0, m0, fb);
-                        tma_load_2d(sB, &tmU, 0, n0, fb);
+                        tma_load_2d(sA, &tmT, 32 * ks, m0, fb);
+                        tma_load_2d(sB, &tmU, 32 * ks, n0, fb);
                     } else {
-                        const int kk = ks - (args.lora ? 1 : 0);
+                        const int kk = ks - lora_stages;
                         if (FP4) {
                             const uint32_t bytes = kABytes + kBBytes + kSfaBytes + (sfb_hi ? kSfbBytes : kSfaBytes);
                             mbar_arrive_expect_tx(fb, bytes);
@@ -161,7 +163,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                             tma_load_2d(sB, &tmB, kk * kRowBytes, n0, fb);
                             const uint32_t sSfa = smem_u32(sbase + kABytes + kBBytes);
                             const uint32_t sSfb = sSfa + kSfaBytes;
-                            const int64_t chunk = (int64_t)kk * 4;
+                            const int64_t chunk = (int64_t)kk * kMmaPerStage;
                             bulk_load(sSfa, args.sfa + ((int64_t)mt * sf_chunks_per_row_tile + chunk) * 512,
                                       kSfaBytes, fb);
                             bulk_load(sSfb, args.sfb + ((int64_t)(2 * nt) * sf_chunks_per_row_tile + chunk) * 512,
@@ -172,8 +174,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                                           kSfaBytes, fb);
                         } else {
                             mbar_arrive_expect_tx(fb, kABytes + kBBytes);
-                            tma_load_2d(sA, &tmA, kk * 64, m0, fb);
-                            tma_load_2d(sB, &tmB, kk * 64, n0, fb);
+                            tma_load_2d(sA, &tmA, kk * 32, m0, fb);
+                            tma_load_2d(sB, &tmB, kk * 32, n0, fb);
                         }
                     }
                     if (++stage == Cfg::kStages) {
@@ -212,29 +214,29 @@ __global__ void __launch_bounds__(kThreads, 1)
                     tc_fence_after();
                     uint8_t *sbase = smem + stage * Cfg::kStageBytes;
                     const uint32_t sA = smem_u32(sbase), sB = smem_u32(sbase + kABytes);
-                    if (args.lora && ks == 0) {
+                    if (ks < lora_stages) {
 #pragma unroll
-                        for (int k = 0; k < 4; ++k)
-                            mma_bf16(acc, sdesc_sw128(sA + 32 * k), sdesc_sw128(sB + 32 * k), kIdescBf16,
-                                     k > 0 ? 1u : 0u);
+                        for (int k = 0; k < kMmaPerStage; ++k)
+                            mma_bf16(acc, sdesc_sw64(sA + 32 * k), sdesc_sw64(sB + 32 * k), kIdescBf16,
+                                     (ks > 0 || k > 0) ? 1u : 0u);
                     } else if (FP4) {
                         const uint32_t sSfa = sA + kABytes + kBBytes;
                         const uint32_t sSfb = sSfa + kSfaBytes;
 #pragma unroll
-                        for (int k = 0; k < 4; ++k) {
+                        for (int k = 0; k < kMmaPerStage; ++k) {
                             tmem_cp_32x128b_x4(tmem_base + kSfaCol + 4 * k, sdesc_sf(sSfa + 512 * k));
                             tmem_cp_32x128b_x4(tmem_base + kSfbCol + 8 * k, sdesc_sf(sSfb + 512 * k));
                             tmem_cp_32x128b_x4(tmem_base + kSfbCol + 8 * k + 4, sdesc_sf(sSfb + kSfaBytes + 512 * k));
                         }
 #pragma unroll
-                        for (int k = 0; k < 4; ++k)
-                            mma_nvfp4(acc, sdesc_sw128(sA + 32 * k), sdesc_sw128(sB + 32 * k), kIdescNvfp4,
+                        for (int k = 0; k < kMmaPerStage; ++k)
+                            mma_nvfp4(acc, sdesc_sw64(sA + 32 * k), sdesc_sw64(sB + 32 * k), kIdescNvfp4,
                                       tmem_base + kSfaCol + 4 * k, tmem_base + kSfbCol + 8 * k,
                                       (ks > 0 || k > 0) ? 1u : 0u);
                     } else {
 #pragma unroll
-                        for (int k = 0; k < 4; ++k)
-                            mma_bf16(acc, sdesc_sw128(sA + 32 * k), sdesc_sw128(sB + 32 * k), kIdescBf16,
+                        for (int k = 0; k < kMmaPerStage; ++k)
+                            mma_bf16(acc, sdesc_sw64(sA + 32 * k), sdesc_sw64(sB + 32 * k), kIdescBf16,
                                      (ks > 0 || k > 0) ? 1u : 0u);
                     }
                     tc_commit(bar_empty + 8 * stage);
@@ -362,22 +364,22 @@ cudaError_t launch_gemm(const GemmLaunch &g, int sms, cudaStream_t stream)
     const bool fp4 = g.fp4 != 0;
     bool ok = true;
     if (fp4) {
-        ok &= make_tmap(&tA, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, g.a, (uint64_t)g.K / 2, (uint64_t)g.M, 128, BM,
-                        CU_TENSOR_MAP_SWIZZLE_128B);
-        ok &= make_tmap(&tB, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, g.b, (uint64_t)g.K / 2, (uint64_t)g.N, 128, BN,
-                        CU_TENSOR_MAP_SWIZZLE_128B);
+        ok &= make_tmap(&tA, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, g.a, (uint64_t)g.K / 2, (uint64_t)g.M, kRowBytes, BM,
+                        CU_TENSOR_MAP_SWIZZLE_64B);
+        ok &= make_tmap(&tB, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, g.b, (uint64_t)g.K / 2, (uint64_t)g.N, kRowBytes, BN,
+                        CU_TENSOR_MAP_SWIZZLE_64B);
     } else {
-        ok &= make_tmap(&tA, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, g.a, (uint64_t)g.K, (uint64_t)g.M, 64, BM,
-                        CU_TENSOR_MAP_SWIZZLE_128B);
-        ok &= make_tmap(&tB, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, g.b, (uint64_t)g.K, (uint64_t)g.N, 64, BN,
-                        CU_TENSOR_MAP_SWIZZLE_128B);
+        ok &= make_tmap(&tA, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, g.a, (uint64_t)g.K, (uint64_t)g.M, kRowBytes / 2,
+                        BM, CU_TENSOR_MAP_SWIZZLE_64B);
+        ok &= make_tmap(&tB, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, g.b, (uint64_t)g.K, (uint64_t)g.N, kRowBytes / 2,
+                        BN, CU_TENSOR_MAP_SWIZZLE_64B);
     }
     const bool lora = g.tsplit && g.udup;
     // without a low-rank step the maps below are never used; point them at A/B
     ok &= make_tmap(&tT, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, lora ? (const void *)g.tsplit : g.a, 64,
-                    (uint64_t)g.M, 64, BM, CU_TENSOR_MAP_SWIZZLE_128B);
+                    (uint64_t)g.M, kRowBytes / 2, BM, CU_TENSOR_MAP_SWIZZLE_64B);
     ok &= make_tmap(&tU, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, lora ? (const void *)g.udup : g.b, 64,
-                    (uint64_t)g.N, 64, BN, CU_TENSOR_MAP_SWIZZLE_128B);
+                    (uint64_t)g.N, kRowBytes / 2, BN, CU_TENSOR_MAP_SWIZZLE_64B);
     ok &= make_tmap(&tY, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, g.y, (uint64_t)g.N, (uint64_t)g.M, 32, 32,
                     CU_TENSOR_MAP_SWIZZLE_128B);
     if (!ok)

@@ -213,6 +213,13 @@ __device__ __forceinline__ uint64_t sdesc_sw128(uint32_t saddr)
            ((uint64_t)1u << 46) | ((uint64_t)2u << 61);
 }
 
+// same, 64-byte swizzle: rows of 64 bytes, 8-row groups 512 bytes apart
+__device__ __forceinline__ uint64_t sdesc_sw64(uint32_t saddr)
+{
+    return (uint64_t)((saddr & 0x3FFFFu) >> 4) | ((uint64_t)1u << 16) | ((uint64_t)(512u >> 4) << 32) |
+           ((uint64_t)1u << 46) | ((uint64_t)4u << 61);
+}
+
 // shared-memory descriptor of a 32-row x 16-byte block (no swizzle, rows
 // contiguous, 8-row groups 128 bytes apart), the source of tcgen05.cp 32x128b
 __device__ __forceinline__ uint64_t sdesc_sf(uint32_t saddr)

@@ -209,6 +209,16 @@ SQ_API sq_status sq_reconstruct_bf16(const sq_weight *w, uint16_t *W_out, uint32
                               void *stream);
 
 /*
+ * Optional instrumentation for timing the tensor-core GEMM on its own: when
+ * both handles are non-NULL, every later sq_linear_fwd call made by this host
+ * thread records start_event immediately before and stop_event immediately
+ * after its GEMM launch, on the call's stream.  The handles are cudaEvent_t
+ * values passed as void*, created and owned by the caller; (NULL, NULL) turns
+ * recording off.  No work is added or skipped.
+ */
+SQ_API sq_status sq_set_gemm_events(void *start_event, void *stop_event);
+
+/*
  * Read back and clear the device status word that a forward kernel sets when
  * it gives up a bounded wait (SQ_ERR_TIMEOUT); ws is the workspace of the
  * sq_linear_fwd call to check (each such call clears the word when it
