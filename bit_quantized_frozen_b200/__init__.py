@@ -19,7 +19,7 @@ from dataclasses import dataclass
 import torch
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(_HERE, "libsq.so")
+LIB_PATH = os.environ.get("SQ_LIBSQ_PATH") or os.path.join(_HERE, "libsq.so")
 
 SQ_OK = 0
 SQ_FMT_INT4_G32 = 1

@@ -13,17 +13,20 @@
 // (SquareQ README, "Op-level parity of the full FP4 forward": block-scaled
 // GEMM + epilogue; "Residual codecs": int4 "dequant-first".)
 //
-// CTA tile 128 x 256, one CTA per SM, 192 threads:
+// CTA tile 128 x 256, one CTA per SM, 6 warps (+4 scale warps on the NVFP4 path):
 //   warps 0-3  epilogue: tcgen05.ld of their 32 accumulator lanes, scale,
 //              128B-swizzled staging in shared memory, TMA store;
 //   warp 4     TMA producer (tiles of A, B, the scale factors, the low-rank
 //              operands) into a ring of shared-memory stages;
-//   warp 5     tensor-memory allocator and the single MMA-issuing thread.
-// Tensor memory (512 columns): two accumulator slots at columns 0 and 192
-// that overlap in columns 192..255, and the scale factors at 448..495.  The
-// epilogue reads the overlapping 64 columns of a tile first and then releases
-// the MMA thread, which starts the next tile while the other 192 columns
-// drain -- accumulator double buffering in 448 columns.
+//   warp 5     tensor-memory allocator and the single MMA-issuing thread;
+//   warps 6-9  (NVFP4) move each MMA's ue4m3 scale factors from shared memory
+//              into tensor memory with tcgen05.st, one 32-lane sub-partition
+//              per warp, so the tensor pipe spends no cycles on copies.
+// Tensor memory (512 columns): two accumulator slots at columns 0 and 128
+// that overlap in columns 128..255, and two 48-column scale-factor buffers at
+// 384..479 (NVFP4).  The epilogue reads the overlapping 128 columns of a tile
+// first and then releases the MMA thread, which starts the next tile while
+// the other 128 columns drain -- accumulator double buffering in 384 columns.
 #include <cuda.h>
 
 #include "sq_device.cuh"
@@ -34,19 +37,20 @@ namespace sq {
 
 constexpr int BM = 128;
 constexpr int BN = 256;
-constexpr int kRowBytes = 64;                  // every stage holds 64-byte rows (64B swizzle atom)
-constexpr int kABytes = BM * kRowBytes;        // 8 KB
-constexpr int kBBytes = BN * kRowBytes;        // 16 KB
-constexpr int kMmaPerStage = 2;                // two MMAs of 32 bytes of K each
-constexpr int kSfaBytes = kMmaPerStage * 512;  // one 512-byte scale chunk (128 rows x 4 scales) per MMA
+constexpr int kRowBytes = 128;                 // every stage holds 128-byte rows (one swizzle atom)
+constexpr int kABytes = BM * kRowBytes;        // 16 KB
+constexpr int kBBytes = BN * kRowBytes;        // 32 KB
+constexpr int kMmaPerStage = 4;                // K = 64 (fp4) or 16 (bf16) per MMA, 32 bytes of the row each
+constexpr int kSfaBytes = kMmaPerStage * 512;  // one 512-byte chunk (128 rows x 4 scales) per MMA
 constexpr int kSfbBytes = 2 * kSfaBytes;       // 256 rows
 constexpr int kEpiWarps = 4;
-constexpr int kThreads = 192;
 constexpr int kStagingBytes = 32 * 128;        // one warp's 32 rows x 32 fp32
 constexpr uint32_t kTmemCols = 512;
-constexpr uint32_t kAccSlot1 = 192;
-constexpr uint32_t kSfaCol = 448;
-constexpr uint32_t kSfbCol = 464;
+constexpr uint32_t kAccSlot1 = 128;            // accumulator slots [0, 256) and [128, 384)
+constexpr int kOverlapChunks = 4;              // 32-column chunks shared by the two slots
+constexpr uint32_t kSfCol = 384;               // two scale-factor buffers of 48 columns, one stage each
+constexpr uint32_t kSfBufCols = 48;            // SFB for MMA k at +8k (256 rows), SFA at +32+4k (128 rows)
+constexpr uint32_t kSfBufs = 2;
 
 // instruction descriptors: M = 128, N = 256, K-major A and B
 constexpr uint32_t kIdescBf16 = (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(BN >> 3) << 17) |
@@ -56,12 +60,15 @@ constexpr uint32_t kIdescNvfp4 = (1u << 7) | (1u << 10) | ((uint32_t)(BN >> 3) <
 
 template <bool FP4>
 struct GemmCfg {
-    static constexpr int kStages = FP4 ? 7 : 8;
+    static constexpr int kStages = FP4 ? 3 : 4;
+    static constexpr int kScaleWarps = FP4 ? 4 : 0;              // warps 6..9 fill the scale-factor ring
+    static constexpr int kThreads = 32 * (6 + kScaleWarps);
     static constexpr int kStageBytes = kABytes + kBBytes + (FP4 ? kSfaBytes + kSfbBytes : 0);
-    static constexpr int kKPerStage = FP4 ? 128 : 32;            // K values per stage
+    static constexpr int kKPerStage = FP4 ? 256 : 64;            // K values per stage
     static constexpr int kStagingOff = kStages * kStageBytes;
     static constexpr int kBarOff = kStagingOff + kEpiWarps * 2 * kStagingBytes;
-    static constexpr int kSmemBytes = kBarOff + 256 + 1024;      // barriers + 1 KB alignment slack
+    static constexpr int kNumBars = 2 * kStages + 4 + (FP4 ? 2 * kSfBufs : 0);
+    static constexpr int kSmemBytes = kBarOff + 8 * kNumBars + 16 + 1024;   // + holder, flag, alignment
 };
 
 struct GemmArgs {
@@ -71,11 +78,48 @@ struct GemmArgs {
     const float *g_w;        // NVFP4: weight global scale (device)
     uint32_t *status;        // device status word
     int M, N, K;
-    int lora;                // 1: add the low-rank K-step
+    int lora;                // 1: add the low-rank K-steps
 };
 
+// warp-uniform bounded wait: lane 0 polls, the verdict is broadcast
+__device__ __forceinline__ bool warp_wait(uint32_t bar, uint32_t parity, volatile uint32_t *abort_flag,
+                                          uint32_t *status, int lane)
+{
+    int ok = 1;
+    if (lane == 0)
+        ok = mbar_wait(bar, parity, abort_flag, status) ? 1 : 0;
+    return __shfl_sync(0xffffffffu, ok, 0) != 0;
+}
+
+// scale one 32-row x 32-column accumulator chunk and TMA-store it through a
+// 128B-swizzled staging buffer (two per warp, used alternately)
+__device__ __forceinline__ void store_chunk(const uint32_t (&r)[32], float beta, uint8_t *staging, int sb, int lane,
+                                            const CUtensorMap *tmY, int x, int y)
+{
+    // staging buffer sb is free once at most one store group is pending
+    if (lane == 0)
+        bulk_wait_group_read1();
+    __syncwarp();
+    uint8_t *buf = staging + sb * kStagingBytes;
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+        float4 o;
+        o.x = __fmul_rn(__uint_as_float(r[4 * j + 0]), beta);
+        o.y = __fmul_rn(__uint_as_float(r[4 * j + 1]), beta);
+        o.z = __fmul_rn(__uint_as_float(r[4 * j + 2]), beta);
+        o.w = __fmul_rn(__uint_as_float(r[4 * j + 3]), beta);
+        *reinterpret_cast<float4 *>(buf + lane * 128 + ((j ^ (lane & 7)) << 4)) = o;
+    }
+    fence_proxy_async_smem();
+    __syncwarp();
+    if (lane == 0) {
+        tma_store_2d(tmY, smem_u32(buf), x, y);
+        bulk_commit_group();
+    }
+}
+
 template <bool FP4>
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(GemmCfg<FP4>::kThreads, 1)
     sq_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                    const __grid_constant__ CUtensorMap tmT, const __grid_constant__ CUtensorMap tmU,
                    const __grid_constant__ CUtensorMap tmY, const GemmArgs args)
@@ -84,13 +128,15 @@ __global__ void __launch_bounds__(kThreads, 1)
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint64_t *bars = reinterpret_cast<uint64_t *>(smem + Cfg::kBarOff);
-    // barrier slots: full[s], empty[s], acc_full[2], acc_empty, drain
+    // barriers: full[s], empty[s], acc_full[2], acc_empty, drain, sf_full[r], sf_empty[r]
     const uint32_t bar_full = smem_u32(bars);
     const uint32_t bar_empty = smem_u32(bars + Cfg::kStages);
     const uint32_t bar_acc_full = smem_u32(bars + 2 * Cfg::kStages);
     const uint32_t bar_acc_empty = smem_u32(bars + 2 * Cfg::kStages + 2);
     const uint32_t bar_drain = smem_u32(bars + 2 * Cfg::kStages + 3);
-    uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(bars + 2 * Cfg::kStages + 4);
+    const uint32_t bar_sf_full = smem_u32(bars + 2 * Cfg::kStages + 4);
+    const uint32_t bar_sf_empty = bar_sf_full + 8 * kSfBufs;
+    uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(bars + Cfg::kNumBars);
     volatile uint32_t *abort_flag = tmem_holder + 1;
 
     const int warp = threadIdx.x >> 5;
@@ -99,12 +145,18 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (threadIdx.x == 0) {
         for (int s = 0; s < Cfg::kStages; ++s) {
             mbar_init(bar_full + 8 * s, 1);
-            mbar_init(bar_empty + 8 * s, 1);
+            mbar_init(bar_empty + 8 * s, 1 + Cfg::kScaleWarps);   // MMA commit + scale warps done reading
         }
         mbar_init(bar_acc_full, 1);
         mbar_init(bar_acc_full + 8, 1);
         mbar_init(bar_acc_empty, kEpiWarps);
         mbar_init(bar_drain, 1);
+        if (FP4) {
+            for (uint32_t r = 0; r < kSfBufs; ++r) {
+                mbar_init(bar_sf_full + 8 * r, Cfg::kScaleWarps);
+                mbar_init(bar_sf_empty + 8 * r, 1);
+            }
+        }
         *abort_flag = 0u;
         fence_mbar_init();
     }
@@ -128,7 +180,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int n_tiles = (args.N + BN - 1) / BN;
     const int tiles = m_tiles * n_tiles;
     const int k_stages = args.K / Cfg::kKPerStage;
-    const int lora_stages = args.lora ? 2 : 0;                // [t_hi | U], then [t_lo | U]
+    const int lora_stages = args.lora ? 1 : 0;                // [t_hi | t_lo] x [U | U]
     const int stages_per_tile = k_stages + lora_stages;
     const int sf_chunks_per_row_tile = args.K / 64;          // 512-byte chunks per 128-row tile
 
@@ -152,8 +204,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                     const uint32_t sA = smem_u32(sbase), sB = smem_u32(sbase + kABytes);
                     if (ks < lora_stages) {
                         mbar_arrive_expect_tx(fb, kABytes + kBBytes);
-                        tma_load_2d(sA, &tmT, 32 * ks, m0, fb);
-                        tma_load_2d(sB, &tmU, 32 * ks, n0, fb);
+                        tma_load_2d(sA, &tmT, 0, m0, fb);
+                        tma_load_2d(sB, &tmU, 0, n0, fb);
                     } else {
                         const int kk = ks - lora_stages;
                         if (FP4) {
@@ -174,8 +226,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                                           kSfaBytes, fb);
                         } else {
                             mbar_arrive_expect_tx(fb, kABytes + kBBytes);
-                            tma_load_2d(sA, &tmA, kk * 32, m0, fb);
-                            tma_load_2d(sB, &tmB, kk * 32, n0, fb);
+                            tma_load_2d(sA, &tmA, kk * 64, m0, fb);
+                            tma_load_2d(sB, &tmB, kk * 64, n0, fb);
                         }
                     }
                     if (++stage == Cfg::kStages) {
@@ -200,13 +252,14 @@ __global__ void __launch_bounds__(kThreads, 1)
             int stage = 0;
             uint32_t phase = 0;
             int count = 0;
+            uint32_t sfbuf = 0, sfphase = 0;
             bool ok = true;
             for (int tile = blockIdx.x; tile < tiles && ok; tile += gridDim.x, ++count) {
                 const uint32_t acc = tmem_base + ((count & 1) ? kAccSlot1 : 0u);
                 if (count > 0 && !mbar_wait(bar_acc_empty, (uint32_t)((count - 1) & 1), abort_flag, args.status))
                     break;
                 tc_fence_after();
-                for (int ks = 0; ks < stages_per_tile; ++ks) {
+                for (int ks = 0; ks < stages_per_tile && ok; ++ks) {
                     if (!mbar_wait(bar_full + 8 * stage, phase, abort_flag, args.status)) {
                         ok = false;
                         break;
@@ -217,26 +270,30 @@ __global__ void __launch_bounds__(kThreads, 1)
                     if (ks < lora_stages) {
 #pragma unroll
                         for (int k = 0; k < kMmaPerStage; ++k)
-                            mma_bf16(acc, sdesc_sw64(sA + 32 * k), sdesc_sw64(sB + 32 * k), kIdescBf16,
-                                     (ks > 0 || k > 0) ? 1u : 0u);
+                            mma_bf16(acc, sdesc_sw128(sA + 32 * k), sdesc_sw128(sB + 32 * k), kIdescBf16,
+                                     k > 0 ? 1u : 0u);
                     } else if (FP4) {
-                        const uint32_t sSfa = sA + kABytes + kBBytes;
-                        const uint32_t sSfb = sSfa + kSfaBytes;
-#pragma unroll
-                        for (int k = 0; k < kMmaPerStage; ++k) {
-                            tmem_cp_32x128b_x4(tmem_base + kSfaCol + 4 * k, sdesc_sf(sSfa + 512 * k));
-                            tmem_cp_32x128b_x4(tmem_base + kSfbCol + 8 * k, sdesc_sf(sSfb + 512 * k));
-                            tmem_cp_32x128b_x4(tmem_base + kSfbCol + 8 * k + 4, sdesc_sf(sSfb + kSfaBytes + 512 * k));
+                        // this stage's scale factors were put in tensor-memory buffer `sfb` by the
+                        // scale warps; the buffer is handed back when these MMAs complete
+                        if (!mbar_wait(bar_sf_full + 8 * sfbuf, sfphase, abort_flag, args.status)) {
+                            ok = false;
+                            break;
                         }
+                        tc_fence_after();
+                        const uint32_t sf = tmem_base + kSfCol + kSfBufCols * sfbuf;
 #pragma unroll
                         for (int k = 0; k < kMmaPerStage; ++k)
-                            mma_nvfp4(acc, sdesc_sw64(sA + 32 * k), sdesc_sw64(sB + 32 * k), kIdescNvfp4,
-                                      tmem_base + kSfaCol + 4 * k, tmem_base + kSfbCol + 8 * k,
-                                      (ks > 0 || k > 0) ? 1u : 0u);
+                            mma_nvfp4(acc, sdesc_sw128(sA + 32 * k), sdesc_sw128(sB + 32 * k), kIdescNvfp4,
+                                      sf + 32 + 4 * k, sf + 8 * k, (ks > 0 || k > 0) ? 1u : 0u);
+                        tc_commit(bar_sf_empty + 8 * sfbuf);
+                        if (++sfbuf == kSfBufs) {
+                            sfbuf = 0;
+                            sfphase ^= 1u;
+                        }
                     } else {
 #pragma unroll
                         for (int k = 0; k < kMmaPerStage; ++k)
-                            mma_bf16(acc, sdesc_sw64(sA + 32 * k), sdesc_sw64(sB + 32 * k), kIdescBf16,
+                            mma_bf16(acc, sdesc_sw128(sA + 32 * k), sdesc_sw128(sB + 32 * k), kIdescBf16,
                                      (ks > 0 || k > 0) ? 1u : 0u);
                     }
                     tc_commit(bar_empty + 8 * stage);
@@ -253,6 +310,70 @@ __global__ void __launch_bounds__(kThreads, 1)
             (void)mbar_wait(bar_drain, 0, abort_flag, args.status);
         }
         __syncwarp();
+    } else if (warp >= 6) {
+        // ------------------------------------------------------------ scale warps (NVFP4)
+        // Warp w owns tensor-memory lanes 32*(w%4)..+31.  For each stage it copies
+        // line `lane` of the four SFA chunks (rows 32*j + lane, j = 0..3) into 4
+        // columns per MMA, and line `lane` of the eight SFB chunks (rows
+        // 128*h + 32*j + lane) into 8 columns per MMA -- the layout that
+        // tcgen05.cp .32x128b.warpx4 produces -- with one store round per stage.
+        const uint32_t lane_base = (uint32_t)(32 * (warp & 3)) << 16;
+        int stage = 0;
+        uint32_t phase = 0;
+        uint32_t sfbuf = 0, sfphase = 0;
+        bool ok = true;
+        for (int tile = blockIdx.x; tile < tiles && ok; tile += gridDim.x) {
+            for (int ks = 0; ks < stages_per_tile && ok; ++ks) {
+                if (!warp_wait(bar_full + 8 * stage, phase, abort_flag, args.status, lane)) {
+                    ok = false;
+                    break;
+                }
+                uint4 sfa[kMmaPerStage], sfb0[kMmaPerStage], sfb1[kMmaPerStage];
+                const bool scaled = ks >= lora_stages;
+                if (scaled) {
+                    const uint8_t *sSfa = smem + stage * Cfg::kStageBytes + kABytes + kBBytes;
+                    const uint8_t *sSfb = sSfa + kSfaBytes;
+#pragma unroll
+                    for (int k = 0; k < kMmaPerStage; ++k) {
+                        sfa[k] = *reinterpret_cast<const uint4 *>(sSfa + 512 * k + 16 * lane);
+                        sfb0[k] = *reinterpret_cast<const uint4 *>(sSfb + 512 * k + 16 * lane);
+                        sfb1[k] = *reinterpret_cast<const uint4 *>(sSfb + kSfaBytes + 512 * k + 16 * lane);
+                    }
+                }
+                __syncwarp();
+                if (lane == 0)
+                    mbar_arrive(bar_empty + 8 * stage);
+                if (scaled) {
+                    if (!warp_wait(bar_sf_empty + 8 * sfbuf, sfphase ^ 1u, abort_flag, args.status, lane)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    const uint32_t sf = tmem_base + lane_base + kSfCol + kSfBufCols * sfbuf;
+#pragma unroll
+                    for (int k = 0; k < kMmaPerStage; ++k) {
+                        const uint32_t a4[4] = {sfa[k].x, sfa[k].y, sfa[k].z, sfa[k].w};
+                        const uint32_t b8[8] = {sfb0[k].x, sfb0[k].y, sfb0[k].z, sfb0[k].w,
+                                                sfb1[k].x, sfb1[k].y, sfb1[k].z, sfb1[k].w};
+                        tmem_st_8cols(sf + 8 * k, b8);
+                        tmem_st_4cols(sf + 32 + 4 * k, a4);
+                    }
+                    tmem_wait_st();
+                    tc_fence_before();
+                    __syncwarp();
+                    if (lane == 0)
+                        mbar_arrive(bar_sf_full + 8 * sfbuf);
+                    if (++sfbuf == kSfBufs) {
+                        sfbuf = 0;
+                        sfphase ^= 1u;
+                    }
+                }
+                if (++stage == Cfg::kStages) {
+                    stage = 0;
+                    phase ^= 1u;
+                }
+            }
+        }
     } else {
         // ------------------------------------------------------------ epilogue
         float beta = 1.0f;
@@ -267,51 +388,40 @@ __global__ void __launch_bounds__(kThreads, 1)
             const int mt = tile % m_tiles, nt = tile / m_tiles;
             const int m0 = mt * BM, n0 = nt * BN;
             const int slot = count & 1;
-            bool ok = true;
-            if (lane == 0)
-                ok = mbar_wait(bar_acc_full + 8 * slot, (uint32_t)((count >> 1) & 1), abort_flag, args.status);
-            ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
-            if (!ok)
+            if (!warp_wait(bar_acc_full + 8 * slot, (uint32_t)((count >> 1) & 1), abort_flag, args.status, lane))
                 break;
             tc_fence_after();
             const uint32_t acc = tmem_base + ((uint32_t)(32 * warp) << 16) + (slot ? kAccSlot1 : 0u);
-#pragma unroll 1
-            for (int ci = 0; ci < 8; ++ci) {
-                const int c = slot ? ci : ((ci + 6) & 7);   // overlapping columns first
-                uint32_t r[32];
-                tmem_ld_32cols(acc + 32 * c, r);
-                tmem_wait_ld();
-                if (ci == 1) {
-                    tc_fence_before();
-                    __syncwarp();
-                    if (lane == 0)
-                        mbar_arrive(bar_acc_empty);
-                }
-                // staging buffer sb is free once at most one store group is pending
-                if (lane == 0)
-                    bulk_wait_group_read1();
-                __syncwarp();
-                uint8_t *buf = staging + sb * kStagingBytes;
+            // the chunks this slot shares with the other one are read first, in one
+            // batch, so the MMA thread can start the next tile as early as possible
+            const int first = slot ? 0 : 8 - kOverlapChunks;
+            uint32_t r[kOverlapChunks][32];
 #pragma unroll
-                for (int j = 0; j < 8; ++j) {
-                    float4 o;
-                    o.x = __fmul_rn(__uint_as_float(r[4 * j + 0]), beta);
-                    o.y = __fmul_rn(__uint_as_float(r[4 * j + 1]), beta);
-                    o.z = __fmul_rn(__uint_as_float(r[4 * j + 2]), beta);
-                    o.w = __fmul_rn(__uint_as_float(r[4 * j + 3]), beta);
-                    *reinterpret_cast<float4 *>(buf + lane * 128 + ((j ^ (lane & 7)) << 4)) = o;
-                }
-                fence_proxy_async_smem();
-                __syncwarp();
-                if (lane == 0) {
-                    tma_store_2d(&tmY, smem_u32(buf), n0 + 32 * c, m0 + 32 * warp);
-                    bulk_commit_group();
-                }
+            for (int q = 0; q < kOverlapChunks; ++q)
+                tmem_ld_32cols(acc + 32 * (first + q), r[q]);
+            tmem_wait_ld();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0)
+                mbar_arrive(bar_acc_empty);
+#pragma unroll
+            for (int q = 0; q < kOverlapChunks; ++q) {
+                store_chunk(r[q], beta, staging, sb, lane, &tmY, n0 + 32 * (first + q), m0 + 32 * warp);
+                sb ^= 1;
+            }
+#pragma unroll 1
+            for (int q = kOverlapChunks; q < 8; ++q) {
+                const int c = (first + q) & 7;
+                uint32_t rr[32];
+                tmem_ld_32cols(acc + 32 * c, rr);
+                tmem_wait_ld();
+                store_chunk(rr, beta, staging, sb, lane, &tmY, n0 + 32 * c, m0 + 32 * warp);
                 sb ^= 1;
             }
         }
         if (lane == 0)
             bulk_wait_group_all();
+        __syncwarp();
     }
 
     tc_fence_before();
@@ -364,22 +474,22 @@ cudaError_t launch_gemm(const GemmLaunch &g, int sms, cudaStream_t stream)
     const bool fp4 = g.fp4 != 0;
     bool ok = true;
     if (fp4) {
-        ok &= make_tmap(&tA, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, g.a, (uint64_t)g.K / 2, (uint64_t)g.M, kRowBytes, BM,
-                        CU_TENSOR_MAP_SWIZZLE_64B);
-        ok &= make_tmap(&tB, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, g.b, (uint64_t)g.K / 2, (uint64_t)g.N, kRowBytes, BN,
-                        CU_TENSOR_MAP_SWIZZLE_64B);
+        ok &= make_tmap(&tA, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, g.a, (uint64_t)g.K / 2, (uint64_t)g.M, 128, BM,
+                        CU_TENSOR_MAP_SWIZZLE_128B);
+        ok &= make_tmap(&tB, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, g.b, (uint64_t)g.K / 2, (uint64_t)g.N, 128, BN,
+                        CU_TENSOR_MAP_SWIZZLE_128B);
     } else {
-        ok &= make_tmap(&tA, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, g.a, (uint64_t)g.K, (uint64_t)g.M, kRowBytes / 2,
-                        BM, CU_TENSOR_MAP_SWIZZLE_64B);
-        ok &= make_tmap(&tB, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, g.b, (uint64_t)g.K, (uint64_t)g.N, kRowBytes / 2,
-                        BN, CU_TENSOR_MAP_SWIZZLE_64B);
+        ok &= make_tmap(&tA, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, g.a, (uint64_t)g.K, (uint64_t)g.M, 64, BM,
+                        CU_TENSOR_MAP_SWIZZLE_128B);
+        ok &= make_tmap(&tB, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, g.b, (uint64_t)g.K, (uint64_t)g.N, 64, BN,
+                        CU_TENSOR_MAP_SWIZZLE_128B);
     }
     const bool lora = g.tsplit && g.udup;
     // without a low-rank step the maps below are never used; point them at A/B
     ok &= make_tmap(&tT, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, lora ? (const void *)g.tsplit : g.a, 64,
-                    (uint64_t)g.M, kRowBytes / 2, BM, CU_TENSOR_MAP_SWIZZLE_64B);
+                    (uint64_t)g.M, 64, BM, CU_TENSOR_MAP_SWIZZLE_128B);
     ok &= make_tmap(&tU, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, lora ? (const void *)g.udup : g.b, 64,
-                    (uint64_t)g.N, kRowBytes / 2, BN, CU_TENSOR_MAP_SWIZZLE_64B);
+                    (uint64_t)g.N, 64, BN, CU_TENSOR_MAP_SWIZZLE_128B);
     ok &= make_tmap(&tY, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, g.y, (uint64_t)g.N, (uint64_t)g.M, 32, 32,
                     CU_TENSOR_MAP_SWIZZLE_128B);
     if (!ok)
@@ -401,13 +511,13 @@ cudaError_t launch_gemm(const GemmLaunch &g, int sms, cudaStream_t stream)
         cudaError_t e = cudaFuncSetAttribute(sq_gemm_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
         if (e != cudaSuccess)
             return e;
-        sq_gemm_kernel<true><<<grid, kThreads, smem, stream>>>(tA, tB, tT, tU, tY, a);
+        sq_gemm_kernel<true><<<grid, GemmCfg<true>::kThreads, smem, stream>>>(tA, tB, tT, tU, tY, a);
     } else {
         const int smem = GemmCfg<false>::kSmemBytes;
         cudaError_t e = cudaFuncSetAttribute(sq_gemm_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
         if (e != cudaSuccess)
             return e;
-        sq_gemm_kernel<false><<<grid, kThreads, smem, stream>>>(tA, tB, tT, tU, tY, a);
+        sq_gemm_kernel<false><<<grid, GemmCfg<false>::kThreads, smem, stream>>>(tA, tB, tT, tU, tY, a);
     }
     return cudaGetLastError();
 }
