@@ -83,7 +83,7 @@ constexpr size_t kHeader = 256;
 constexpr size_t kAlign = 1024;
 
 struct FwdLayout {
-    size_t a = 0, a_sf = 0, b = 0, tsplit = 0, udup = 0, dt = 0, total = 0;
+    size_t a = 0, a_sf = 0, b = 0, t32 = 0, tsplit = 0, udup = 0, total = 0;
 };
 
 FwdLayout fwd_layout(int fmt, int64_t M, int64_t N, int64_t K)
@@ -103,9 +103,9 @@ FwdLayout fwd_layout(int fmt, int64_t M, int64_t N, int64_t K)
         L.a = take((size_t)M * (size_t)K * 2);
         L.b = take((size_t)N * (size_t)K * 2);
     }
+    L.t32 = take((size_t)M * 32 * 4);
     L.tsplit = take((size_t)M * 64 * 2);
     L.udup = take((size_t)N * 64 * 2);
-    L.dt = take((size_t)K * 32 * 2);
     L.total = round_up(off, kAlign);
     return L;
 }
@@ -188,7 +188,7 @@ size_t sq_workspace_bytes(int op, int64_t M, int64_t N, int64_t K)
     case SQ_OP_BUILD_NVFP4:
         return kHeader;
     case SQ_OP_ACT_QUANT_NVFP4:
-        return round_up(kHeader, kAlign) + round_up((size_t)K * 32 * 2, kAlign);
+        return kHeader;
     case SQ_OP_LINEAR_FWD_NVFP4:
         return fwd_layout(SQ_FMT_NVFP4, M, N, K).total;
     case SQ_OP_LINEAR_FWD_INT4:
@@ -260,19 +260,15 @@ sq_status sq_act_quant_nvfp4(const uint16_t *x, int64_t M, int64_t K, uint8_t *c
         return st;
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     const bool stat = (flags & SQ_ACT_STATIC_SCALE) != 0;
+    const bool with_t = lora_down && t;
     uint32_t *amax = reinterpret_cast<uint32_t *>(ws_at(ws, 4));
-    if (!stat) {
-        SQ_CUDA(cudaMemsetAsync(amax, 0, 4, s), "memset");
-        SQ_CUDA(sq::launch_absmax_rot_bf16(x, M, K, amax, sms, s), "absmax");
-    }
+    SQ_CUDA(cudaMemsetAsync(ws, 0, 8, s), "memset");          // status word + absmax
+    if (!stat || with_t)
+        SQ_CUDA(sq::launch_act_pass1(x, M, K, lora_down, stat ? nullptr : amax, with_t ? t : nullptr, s),
+                "activation pass 1");
     SQ_CUDA(sq::launch_nvfp4_quant_bf16(x, M, K, amax, stat ? g_x : nullptr, stat ? nullptr : g_x, codes, sf_tiled,
                                         sms, s),
             "nvfp4 quant");
-    if (lora_down && t) {
-        uint16_t *dt = reinterpret_cast<uint16_t *>(ws_at(ws, round_up(kHeader, kAlign)));
-        SQ_CUDA(sq::launch_lora_prep(nullptr, 0, lora_down, K, nullptr, dt, sms, s), "lora prep");
-        SQ_CUDA(sq::launch_lowrank_t(x, M, K, dt, nullptr, nullptr, t, nullptr, s), "lowrank t");
-    }
     return SQ_OK;
 }
 
@@ -305,8 +301,9 @@ sq_status sq_linear_fwd(const sq_weight *w, const uint16_t *x, int64_t M, float 
     const bool lora = w->lora_up && w->lora_down;
     uint16_t *tsplit = lora ? reinterpret_cast<uint16_t *>(ws_at(ws, L.tsplit)) : nullptr;
     uint16_t *udup = lora ? reinterpret_cast<uint16_t *>(ws_at(ws, L.udup)) : nullptr;
-    uint16_t *dt = reinterpret_cast<uint16_t *>(ws_at(ws, L.dt));
+    float *t32 = lora ? reinterpret_cast<float *>(ws_at(ws, L.t32)) : nullptr;
     uint32_t *status = reinterpret_cast<uint32_t *>(ws_at(ws, 0));
+    uint32_t *amax = reinterpret_cast<uint32_t *>(ws_at(ws, 4));
     sq::GemmLaunch g;
     memset(&g, 0, sizeof(g));
     g.M = M;
@@ -316,21 +313,20 @@ sq_status sq_linear_fwd(const sq_weight *w, const uint16_t *x, int64_t M, float 
     g.status = status;
     g.tsplit = tsplit;
     g.udup = udup;
+    SQ_CUDA(cudaMemsetAsync(status, 0, 8, s), "memset");   // status word + absmax
     if (w->fmt == SQ_FMT_NVFP4) {
-        uint32_t *amax = reinterpret_cast<uint32_t *>(ws_at(ws, 4));
         float *gx = g_x ? g_x : reinterpret_cast<float *>(ws_at(ws, 8));
         uint8_t *xc = ws_at(ws, L.a);
         uint8_t *xsf = ws_at(ws, L.a_sf);
-        SQ_CUDA(cudaMemsetAsync(status, 0, 8, s), "memset");   // status word + absmax
-        if (!stat)
-            SQ_CUDA(sq::launch_absmax_rot_bf16(x, M, K, amax, sms, s), "absmax");
+        // one read of x for the absmax and the low-rank input, one for the quantisation
+        if (!stat || lora)
+            SQ_CUDA(sq::launch_act_pass1(x, M, K, w->lora_down, stat ? nullptr : amax, t32, s), "activation pass 1");
         SQ_CUDA(sq::launch_nvfp4_quant_bf16(x, M, K, amax, stat ? gx : nullptr, stat ? nullptr : gx, xc, xsf, sms,
                                             s),
                 "nvfp4 act quant");
-        if (lora) {
-            SQ_CUDA(sq::launch_lora_prep(w->lora_up, N, w->lora_down, K, udup, dt, sms, s), "lora prep");
-            SQ_CUDA(sq::launch_lowrank_t(x, M, K, dt, gx, w->g_w, nullptr, tsplit, s), "lowrank t");
-        }
+        if (lora)
+            SQ_CUDA(sq::launch_lowrank_finish(t32, M, gx, w->g_w, tsplit, w->lora_up, N, udup, sms, s),
+                    "low-rank operands");
         g.fp4 = 1;
         g.a = xc;
         g.b = w->codes;
@@ -339,15 +335,15 @@ sq_status sq_linear_fwd(const sq_weight *w, const uint16_t *x, int64_t M, float 
         g.g_x = gx;
         g.g_w = w->g_w;
     } else {
-        SQ_CUDA(cudaMemsetAsync(status, 0, 4, s), "memset");
         uint16_t *xb = reinterpret_cast<uint16_t *>(ws_at(ws, L.a));
         uint16_t *wb = reinterpret_cast<uint16_t *>(ws_at(ws, L.b));
         SQ_CUDA(sq::launch_rotate_bf16(x, M, K, xb, sms, s), "rotate x");
         SQ_CUDA(sq::launch_dequant_int4(w->codes, reinterpret_cast<const uint16_t *>(w->scales), N, K, wb, sms, s),
                 "dequant");
         if (lora) {
-            SQ_CUDA(sq::launch_lora_prep(w->lora_up, N, w->lora_down, K, udup, dt, sms, s), "lora prep");
-            SQ_CUDA(sq::launch_lowrank_t(x, M, K, dt, nullptr, nullptr, nullptr, tsplit, s), "lowrank t");
+            SQ_CUDA(sq::launch_act_pass1(x, M, K, w->lora_down, nullptr, t32, s), "low-rank input");
+            SQ_CUDA(sq::launch_lowrank_finish(t32, M, nullptr, nullptr, tsplit, w->lora_up, N, udup, sms, s),
+                    "low-rank operands");
         }
         g.fp4 = 0;
         g.a = xb;

@@ -68,6 +68,64 @@ __device__ __forceinline__ void fwht256_warp(float (&v)[8], int lane)
 }
 
 // ---------------------------------------------------------------------------
+// Hadamard-256 over 8 lanes.
+//
+// Layout: lane q = lane % 8 of an aligned group of 8 lanes holds v[0..31] =
+// elements 32q..32q+31 of one 256-block (a warp holds 4 blocks).  Strides
+// 1..16 pair values inside a lane, strides 32, 64, 128 pair lane q with lane
+// q ^ 1, q ^ 2, q ^ 4.  Same butterflies, same operands, same order of
+// strides as the sequential transform, so the result is identical bit for bit.
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ void fwht256_l32(float (&v)[32], int lane)
+{
+#pragma unroll
+    for (int h = 1; h < 32; h <<= 1)
+#pragma unroll
+        for (int i = 0; i < 32; ++i)
+            if ((i & h) == 0) {
+                const float a = v[i], b = v[i + h];
+                v[i] = __fadd_rn(a, b);
+                v[i + h] = __fsub_rn(a, b);
+            }
+#pragma unroll
+    for (int x = 1; x <= 4; x <<= 1) {          // h = 32x
+        const bool lower = (lane & x) == 0;
+#pragma unroll
+        for (int i = 0; i < 32; ++i) {
+            const float p = __shfl_xor_sync(0xffffffffu, v[i], x);
+            v[i] = lower ? __fadd_rn(v[i], p) : __fsub_rn(p, v[i]);
+        }
+    }
+#pragma unroll
+    for (int i = 0; i < 32; ++i)
+        v[i] = __fmul_rn(v[i], 0.0625f);
+}
+
+// 32 consecutive values into registers (fp32 source or bf16 bit patterns)
+__device__ __forceinline__ void load32(const float *p, float (&v)[32])
+{
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+        const float4 a = __ldg(reinterpret_cast<const float4 *>(p) + i);
+        v[4 * i] = a.x; v[4 * i + 1] = a.y; v[4 * i + 2] = a.z; v[4 * i + 3] = a.w;
+    }
+}
+
+__device__ __forceinline__ void load32(const uint16_t *p, float (&v)[32])
+{
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const uint4 a = __ldg(reinterpret_cast<const uint4 *>(p) + i);
+        const uint32_t w[4] = {a.x, a.y, a.z, a.w};
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            v[8 * i + 2 * j] = __uint_as_float(w[j] << 16);
+            v[8 * i + 2 * j + 1] = __uint_as_float(w[j] & 0xFFFF0000u);
+        }
+    }
+}
+
+// ---------------------------------------------------------------------------
 // Narrowing conversions (PTX cvt, round-to-nearest-even, satfinite).
 // ---------------------------------------------------------------------------
 

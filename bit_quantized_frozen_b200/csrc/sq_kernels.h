@@ -21,10 +21,11 @@ cudaError_t launch_int4_build(const float *R, int64_t N, int64_t K, uint8_t *cod
 cudaError_t launch_rotate_bf16(const uint16_t *x, int64_t M, int64_t K, uint16_t *xb, int sms, cudaStream_t s);
 cudaError_t launch_dequant_int4(const uint8_t *codes, const uint16_t *scales, int64_t N, int64_t K, uint16_t *wb,
                                 int sms, cudaStream_t s);
-cudaError_t launch_lora_prep(const uint16_t *U, int64_t N, const uint16_t *D, int64_t K, uint16_t *udup,
-                             uint16_t *dt, int sms, cudaStream_t s);
-cudaError_t launch_lowrank_t(const uint16_t *x, int64_t M, int64_t K, const uint16_t *dt, const float *g_x,
-                             const float *g_w, float *t_out, uint16_t *tsplit, cudaStream_t s);
+cudaError_t launch_act_pass1(const uint16_t *x, int64_t M, int64_t K, const uint16_t *D, uint32_t *amax,
+                             float *t32, cudaStream_t s);
+cudaError_t launch_lowrank_finish(const float *t32, int64_t M, const float *g_x, const float *g_w,
+                                  uint16_t *tsplit, const uint16_t *U, int64_t N, uint16_t *udup, int sms,
+                                  cudaStream_t s);
 cudaError_t launch_reconstruct(int fmt, const uint8_t *codes, const void *scales, const float *g_w,
                                const uint16_t *U, const uint16_t *D, int64_t N, int64_t K, int with_lowrank,
                                uint16_t *W, cudaStream_t s);

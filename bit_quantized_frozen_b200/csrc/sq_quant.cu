@@ -14,45 +14,45 @@
 namespace sq {
 
 // ---------------------------------------------------------------------------
-// loading one 256-block into the warp layout of fwht256_warp
+// Warp tasks over 256-blocks.  A warp takes 4 consecutive blocks of the
+// row-major matrix (flat block index 4*task + lane/8); lane q = lane % 8 holds
+// values 32q..32q+31 of its block (the layout of fwht256_l32).  Blocks past the
+// end are processed as zeros and never stored, so every lane joins the
+// shuffles of the transform.
 // ---------------------------------------------------------------------------
-__device__ __forceinline__ void load_block(const float *p, int lane, float (&v)[8])
+template <typename T>
+__device__ __forceinline__ void load_block_l32(const T *base, int64_t block, bool valid, int lane, float (&v)[32])
 {
-    float4 a = __ldg(reinterpret_cast<const float4 *>(p + 4 * lane));
-    float4 b = __ldg(reinterpret_cast<const float4 *>(p + 128 + 4 * lane));
-    v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w;
-    v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
-}
-
-__device__ __forceinline__ void load_block(const uint16_t *p, int lane, float (&v)[8])
-{
-    uint2 a = __ldg(reinterpret_cast<const uint2 *>(p + 4 * lane));
-    uint2 b = __ldg(reinterpret_cast<const uint2 *>(p + 128 + 4 * lane));
-    v[0] = bf16_bits_to_f32(a.x & 0xFFFFu); v[1] = bf16_bits_to_f32(a.x >> 16);
-    v[2] = bf16_bits_to_f32(a.y & 0xFFFFu); v[3] = bf16_bits_to_f32(a.y >> 16);
-    v[4] = bf16_bits_to_f32(b.x & 0xFFFFu); v[5] = bf16_bits_to_f32(b.x >> 16);
-    v[6] = bf16_bits_to_f32(b.y & 0xFFFFu); v[7] = bf16_bits_to_f32(b.y >> 16);
+    if (valid) {
+        load32(base + block * kHad + 32 * (lane & 7), v);
+    } else {
+#pragma unroll
+        for (int i = 0; i < 32; ++i)
+            v[i] = 0.0f;
+    }
 }
 
 // ---------------------------------------------------------------------------
-// pass 1: A = max |H in| over a [rows, K] matrix, folded into *amax (u32 bits)
+// pass 1 of the NVFP4 builder: A = max |H R| over a [rows, K] matrix, folded
+// into *amax (u32 bits of a non-negative float)
 // ---------------------------------------------------------------------------
 template <typename T>
 __global__ void __launch_bounds__(256) absmax_rot_kernel(const T *__restrict__ in, int64_t rows,
                                                          int64_t K, uint32_t *__restrict__ amax)
 {
     const int lane = threadIdx.x & 31;
+    const int64_t blocks = rows * (K / kHad);
+    const int64_t tasks = (blocks + 3) / 4;
     const int64_t warps_total = (int64_t)gridDim.x * (blockDim.x >> 5);
-    const int64_t kb_per_row = K / kHad;
-    const int64_t tasks = rows * kb_per_row;
     float m = 0.0f;
     for (int64_t task = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); task < tasks;
          task += warps_total) {
-        float v[8];
-        load_block(in + task * kHad, lane, v);
-        fwht256_warp(v, lane);
+        const int64_t b = 4 * task + (lane >> 3);
+        float v[32];
+        load_block_l32(in, b, b < blocks, lane, v);
+        fwht256_l32(v, lane);
 #pragma unroll
-        for (int i = 0; i < 8; ++i)
+        for (int i = 0; i < 32; ++i)
             m = fmaxf(m, fabsf(v[i]));
     }
 #pragma unroll
@@ -71,11 +71,12 @@ __global__ void __launch_bounds__(256) absmax_rot_kernel(const T *__restrict__ i
 }
 
 // ---------------------------------------------------------------------------
-// pass 2: NVFP4 block quantisation of H in with global scale g.
-// rows_pad >= rows (a multiple of 128): rows past `rows` are zero, and only
-// their scale bytes are written (as 0), which fills the tiled layout's padding.
-// g comes from *g_static when non-NULL, else RN(A / 2688) from *amax, and is
-// stored to *g_out (when non-NULL) by thread 0 of block 0.
+// NVFP4 block quantisation of H in with global scale g.  rows_pad >= rows (a
+// multiple of 128): rows past `rows` are zero and only their scale bytes are
+// written (as 0), which fills the tiled layout's padding.  g comes from
+// *g_static when non-NULL, else RN(A / 2688) from *amax, and is stored to
+// *g_out (when non-NULL) by thread 0 of block 0.  Each lane owns two whole
+// 16-value blocks, so block maxima and scales need no shuffles.
 // ---------------------------------------------------------------------------
 template <typename T>
 __global__ void __launch_bounds__(256) nvfp4_quant_kernel(const T *__restrict__ in, int64_t rows,
@@ -87,73 +88,69 @@ __global__ void __launch_bounds__(256) nvfp4_quant_kernel(const T *__restrict__ 
                                                           uint8_t *__restrict__ sf)
 {
     const int lane = threadIdx.x & 31;
+    const int q = lane & 7;
     const float g = g_static ? *g_static : __fdiv_rn(__uint_as_float(*amax), 2688.0f);
     if (g_out && blockIdx.x == 0 && threadIdx.x == 0)
         *g_out = g;
     const float sixg = __fmul_rn(6.0f, g);
-    const int64_t warps_total = (int64_t)gridDim.x * (blockDim.x >> 5);
     const int64_t kb_per_row = K / kHad;
     const int64_t C = K / kSfBlock;
-    const int64_t tasks = rows_pad * kb_per_row;
+    const int64_t blocks = rows_pad * kb_per_row;
+    const int64_t tasks = (blocks + 3) / 4;
+    const int64_t warps_total = (int64_t)gridDim.x * (blockDim.x >> 5);
     for (int64_t task = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); task < tasks;
          task += warps_total) {
-        const int64_t row = task / kb_per_row;
-        const int64_t kb = task - row * kb_per_row;
-        float v[8];
-        const bool valid = row < rows;
-        if (valid) {
-            load_block(in + row * K + kb * kHad, lane, v);
-            fwht256_warp(v, lane);
-        } else {
-#pragma unroll
-            for (int i = 0; i < 8; ++i)
-                v[i] = 0.0f;
-        }
-        uint32_t packed[2];
+        const int64_t b = 4 * task + (lane >> 3);
+        const int64_t row = b / kb_per_row;
+        const int64_t kb = b - row * kb_per_row;
+        const bool in_range = b < blocks;
+        float v[32];
+        load_block_l32(in, row * kb_per_row + kb, in_range && row < rows, lane, v);
+        fwht256_l32(v, lane);
+        if (!in_range)
+            continue;
+        uint32_t word[4];
         uint32_t sfc[2];
 #pragma unroll
         for (int h = 0; h < 2; ++h) {
-            // block of 16 = 4 lanes x 4 values
-            float b = fmaxf(fmaxf(fabsf(v[4 * h]), fabsf(v[4 * h + 1])),
-                            fmaxf(fabsf(v[4 * h + 2]), fabsf(v[4 * h + 3])));
-            b = fmaxf(b, __shfl_xor_sync(0xffffffffu, b, 1));
-            b = fmaxf(b, __shfl_xor_sync(0xffffffffu, b, 2));
+            float bmax = 0.0f;
+#pragma unroll
+            for (int i = 0; i < 16; ++i)
+                bmax = fmaxf(bmax, fabsf(v[16 * h + i]));
             uint32_t code = 0;
-            uint32_t pk = 0;
+            uint32_t w0 = 0, w1 = 0;
             if (g != 0.0f) {
-                code = to_ue4m3(__fdiv_rn(b, sixg));
+                code = to_ue4m3(__fdiv_rn(bmax, sixg));
                 if (code != 0) {
-                    const float den = __fmul_rn(ue4m3_value(code), g);
-                    const float inv = __frcp_rn(den);
-                    pk = to_e2m1x2(__fmul_rn(v[4 * h], inv), __fmul_rn(v[4 * h + 1], inv)) |
-                         (to_e2m1x2(__fmul_rn(v[4 * h + 2], inv), __fmul_rn(v[4 * h + 3], inv)) << 8);
+                    const float inv = __frcp_rn(__fmul_rn(ue4m3_value(code), g));
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) {
+                        w0 |= to_e2m1x2(__fmul_rn(v[16 * h + 2 * i], inv), __fmul_rn(v[16 * h + 2 * i + 1], inv))
+                              << (8 * i);
+                        w1 |= to_e2m1x2(__fmul_rn(v[16 * h + 8 + 2 * i], inv),
+                                        __fmul_rn(v[16 * h + 8 + 2 * i + 1], inv))
+                              << (8 * i);
+                    }
                 }
             }
-            packed[h] = pk;
+            word[2 * h] = w0;
+            word[2 * h + 1] = w1;
             sfc[h] = code;
         }
-        if (valid) {
-            uint16_t *cp = reinterpret_cast<uint16_t *>(codes + row * (K / 2) + kb * (kHad / 2));
-            cp[lane] = (uint16_t)packed[0];
-            cp[32 + lane] = (uint16_t)packed[1];   // bytes 64..127 of the block
-        }
-        if ((lane & 3) == 0) {
-            const int64_t c0 = kb * (kHad / kSfBlock) + (lane >> 2);
-            sf[sf_offset(row, c0, C)] = (uint8_t)sfc[0];
-            sf[sf_offset(row, c0 + 8, C)] = (uint8_t)sfc[1];
-        }
+        if (row < rows)
+            *reinterpret_cast<uint4 *>(codes + row * (K / 2) + kb * (kHad / 2) + 16 * q) =
+                make_uint4(word[0], word[1], word[2], word[3]);
+        // scale columns 2q, 2q+1 of the block are adjacent bytes of the tiled layout
+        *reinterpret_cast<uint16_t *>(sf + sf_offset(row, kb * (kHad / kSfBlock) + 2 * q, C)) =
+            (uint16_t)(sfc[0] | (sfc[1] << 8));
     }
 }
 
 // ---------------------------------------------------------------------------
-// int4 group-32 builder.  A warp takes 4 consecutive 256-blocks (1024 values,
-// 32 groups), rotates them, stages them in shared memory and then each lane
-// sweeps one whole group of 32 in registers.
-// Staging layout: group G, float4 w of the group sits in slot G*8 + (w ^ (G&7))
-// so both the rotated writes and the per-group reads are conflict free.
+// int4 group-32 builder.  With the 8-lane Hadamard layout every lane holds one
+// whole group of 32 rotated values and sweeps the 26 scale fractions in
+// registers; a warp covers 32 consecutive groups.
 // ---------------------------------------------------------------------------
-constexpr int kInt4Warps = 8;
-
 __device__ __forceinline__ float group_sq_error(const float (&r)[32], float s, float inv)
 {
     float p[32];
@@ -178,81 +175,62 @@ __device__ __forceinline__ float group_sq_error(const float (&r)[32], float s, f
     return p[0];
 }
 
-__global__ void __launch_bounds__(kInt4Warps * 32) int4_build_kernel(const float *__restrict__ R,
-                                                                     int64_t N, int64_t K,
-                                                                     uint8_t *__restrict__ codes,
-                                                                     uint16_t *__restrict__ scales,
-                                                                     uint8_t *__restrict__ frac)
+__global__ void __launch_bounds__(256, 2) int4_build_kernel(const float *__restrict__ R, int64_t N, int64_t K,
+                                                         uint8_t *__restrict__ codes,
+                                                         uint16_t *__restrict__ scales,
+                                                         uint8_t *__restrict__ frac)
 {
-    __shared__ __align__(16) float4 stage[kInt4Warps][256];
     const int lane = threadIdx.x & 31;
-    const int wid = threadIdx.x >> 5;
     const int64_t blocks = N * K / kHad;
     const int64_t tasks = (blocks + 3) / 4;
-    const int64_t warps_total = (int64_t)gridDim.x * kInt4Warps;
-    float4 *st = stage[wid];
-    for (int64_t task = (int64_t)blockIdx.x * kInt4Warps + wid; task < tasks; task += warps_total) {
-        const int64_t b0 = task * 4;
-        const int nb = (int)(blocks - b0 < 4 ? blocks - b0 : 4);
-        for (int b = 0; b < nb; ++b) {
-            float v[8];
-            load_block(R + (b0 + b) * kHad, lane, v);
-            fwht256_warp(v, lane);
-            const int G0 = 8 * b + (lane >> 3);
-            const int G1 = G0 + 4;
-            const int w = lane & 7;
-            st[G0 * 8 + (w ^ (G0 & 7))] = make_float4(v[0], v[1], v[2], v[3]);
-            st[G1 * 8 + (w ^ (G1 & 7))] = make_float4(v[4], v[5], v[6], v[7]);
-        }
-        __syncwarp();
-        const int G = lane;
-        if (G < nb * 8) {
-            float r[32];
+    const int64_t warps_total = (int64_t)gridDim.x * (blockDim.x >> 5);
+    for (int64_t task = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); task < tasks;
+         task += warps_total) {
+        const int64_t b = 4 * task + (lane >> 3);
+        const bool valid = b < blocks;
+        float r[32];
+        load_block_l32(R, b, valid, lane, r);
+        fwht256_l32(r, lane);
+        if (!valid)
+            continue;
+        float a = 0.0f;
 #pragma unroll
-            for (int w = 0; w < 8; ++w) {
-                float4 q4 = st[G * 8 + (w ^ (G & 7))];
-                r[4 * w] = q4.x; r[4 * w + 1] = q4.y; r[4 * w + 2] = q4.z; r[4 * w + 3] = q4.w;
-            }
-            float a = 0.0f;
-#pragma unroll
-            for (int i = 0; i < 32; ++i)
-                a = fmaxf(a, fabsf(r[i]));
-            float best = 0.0f, best_s = 0.0f;
-            uint16_t best_h = 0;
-            int best_j = 0;
+        for (int i = 0; i < 32; ++i)
+            a = fmaxf(a, fabsf(r[i]));
+        float best = 0.0f, best_s = 0.0f;
+        uint16_t best_h = 0;
+        int best_j = 0;
 #pragma unroll 1
-            for (int j = 0; j < kFracCount; ++j) {
-                const float f = __fdiv_rn((float)(50 + 2 * j), 100.0f);
-                const __half hs = __float2half_rn(__fdiv_rn(__fmul_rn(f, a), 7.0f));
-                const float s = __half2float(hs);
-                const float inv = s == 0.0f ? 0.0f : __frcp_rn(s);
-                const float mse = group_sq_error(r, s, inv);
-                if (j == 0 || mse < best) {
-                    best = mse;
-                    best_j = j;
-                    best_s = s;
-                    best_h = __half_as_ushort(hs);
-                }
+        for (int j = 0; j < kFracCount; ++j) {
+            const float f = __fdiv_rn((float)(50 + 2 * j), 100.0f);
+            const __half hs = __float2half_rn(__fdiv_rn(__fmul_rn(f, a), 7.0f));
+            const float s = __half2float(hs);
+            const float inv = s == 0.0f ? 0.0f : __frcp_rn(s);
+            const float mse = group_sq_error(r, s, inv);
+            if (j == 0 || mse < best) {
+                best = mse;
+                best_j = j;
+                best_s = s;
+                best_h = __half_as_ushort(hs);
             }
-            // codes for the winning scale (same arithmetic as in the sweep)
-            const float inv = best_s == 0.0f ? 0.0f : __frcp_rn(best_s);
-            uint32_t word[4] = {0u, 0u, 0u, 0u};
-#pragma unroll
-            for (int i = 0; i < 32; ++i) {
-                int q = 0;
-                if (best_s != 0.0f) {
-                    float qf = rintf(__fmul_rn(r[i], inv));
-                    q = (int)fminf(fmaxf(qf, -7.0f), 7.0f);
-                }
-                word[i >> 3] |= ((uint32_t)q & 0xFu) << (4 * (i & 7));
-            }
-            const int64_t gidx = b0 * 8 + G;     // flat group index
-            reinterpret_cast<uint4 *>(codes)[gidx] = make_uint4(word[0], word[1], word[2], word[3]);
-            scales[gidx] = best_h;
-            if (frac)
-                frac[gidx] = (uint8_t)best_j;
         }
-        __syncwarp();
+        // codes for the winning scale (same arithmetic as in the sweep)
+        const float inv = best_s == 0.0f ? 0.0f : __frcp_rn(best_s);
+        uint32_t word[4] = {0u, 0u, 0u, 0u};
+#pragma unroll
+        for (int i = 0; i < 32; ++i) {
+            int q = 0;
+            if (best_s != 0.0f) {
+                float qf = rintf(__fmul_rn(r[i], inv));
+                q = (int)fminf(fmaxf(qf, -7.0f), 7.0f);
+            }
+            word[i >> 3] |= ((uint32_t)q & 0xFu) << (4 * (i & 7));
+        }
+        const int64_t gidx = 32 * task + lane;     // flat group index
+        reinterpret_cast<uint4 *>(codes)[gidx] = make_uint4(word[0], word[1], word[2], word[3]);
+        scales[gidx] = best_h;
+        if (frac)
+            frac[gidx] = (uint8_t)best_j;
     }
 }
 
@@ -263,21 +241,27 @@ __global__ void __launch_bounds__(256) rotate_bf16_kernel(const uint16_t *__rest
                                                           int64_t K, uint16_t *__restrict__ xb)
 {
     const int lane = threadIdx.x & 31;
+    const int64_t blocks = M * (K / kHad);
+    const int64_t tasks = (blocks + 3) / 4;
     const int64_t warps_total = (int64_t)gridDim.x * (blockDim.x >> 5);
-    const int64_t tasks = M * (K / kHad);
     for (int64_t task = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); task < tasks;
          task += warps_total) {
-        float v[8];
-        load_block(x + task * kHad, lane, v);
-        fwht256_warp(v, lane);
-        uint2 lo, hi;
-        lo.x = f32_to_bf16_bits(v[0]) | (f32_to_bf16_bits(v[1]) << 16);
-        lo.y = f32_to_bf16_bits(v[2]) | (f32_to_bf16_bits(v[3]) << 16);
-        hi.x = f32_to_bf16_bits(v[4]) | (f32_to_bf16_bits(v[5]) << 16);
-        hi.y = f32_to_bf16_bits(v[6]) | (f32_to_bf16_bits(v[7]) << 16);
-        uint16_t *o = xb + task * kHad;
-        *reinterpret_cast<uint2 *>(o + 4 * lane) = lo;
-        *reinterpret_cast<uint2 *>(o + 128 + 4 * lane) = hi;
+        const int64_t b = 4 * task + (lane >> 3);
+        const bool valid = b < blocks;
+        float v[32];
+        load_block_l32(x, b, valid, lane, v);
+        fwht256_l32(v, lane);
+        if (!valid)
+            continue;
+        uint4 *o = reinterpret_cast<uint4 *>(xb + b * kHad + 32 * (lane & 7));
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            uint32_t w[4];
+#pragma unroll
+            for (int j = 0; j < 4; ++j)
+                w[j] = f32_to_bf16_bits(v[8 * i + 2 * j]) | (f32_to_bf16_bits(v[8 * i + 2 * j + 1]) << 16);
+            o[i] = make_uint4(w[0], w[1], w[2], w[3]);
+        }
     }
 }
 
@@ -306,39 +290,54 @@ __global__ void __launch_bounds__(256) dequant_int4_kernel(const uint32_t *__res
 }
 
 // ---------------------------------------------------------------------------
-// low-rank operand preparation: udup[n] = [U[n, 0:32] | U[n, 0:32]] (bf16
-// [N, 64], the B operand of the low-rank MMA step) and dt = lora_down^T
-// (bf16 [32, K], for contiguous fragment loads).
+// Activation pass 1: one read of x for two results.
+//   amax (optional): max |H x| over the whole tensor (the activation global
+//                    scale's input), from the 8-lane Hadamard transform;
+//   t32 (optional):  t = x . lora_down, fp32 [M, 32], on mma.sync bf16 tensor
+//                    cores (fp32 accumulation; each CTA sums its partials in a
+//                    fixed order, so t is deterministic).
+// A CTA owns 16 rows and walks K in 256-column chunks; the x chunk (16 x 256)
+// and the lora_down chunk (256 x 32) are staged in shared memory by cp.async,
+// double buffered.  Warps 0-3 transform rows 4w..4w+3, warps 4-7 run k-steps
+// 4(w-4)..4(w-4)+3 of the chunk for all 32 outputs.
+// x tile: 16-byte chunk c of row r sits at c ^ ((c >> 2) & 7) ^ (r & 7), which
+// keeps both the transform's per-row reads and ldmatrix conflict free; D tile:
+// chunk c of k-row k sits at c ^ ((k >> 1) & 3).
 // ---------------------------------------------------------------------------
-__global__ void __launch_bounds__(256) lora_prep_kernel(const uint16_t *__restrict__ U, int64_t N,
-                                                        const uint16_t *__restrict__ D, int64_t K,
-                                                        uint16_t *__restrict__ udup,
-                                                        uint16_t *__restrict__ dt)
+constexpr int kP1Rows = 16;
+constexpr int kP1XBytes = kP1Rows * kHad * 2;      // 8 KB
+constexpr int kP1DBytes = kHad * kRank * 2;        // 16 KB
+constexpr int kP1BufBytes = kP1XBytes + kP1DBytes;
+constexpr int kP1Smem = 2 * kP1BufBytes;           // 48 KB
+
+__device__ __forceinline__ void cp_async16(uint32_t dst, const void *src, uint32_t src_bytes)
 {
-    const int64_t nU = udup ? N * 64 : 0;
-    const int64_t nD = dt ? K * 32 : 0;
-    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < nU + nD;
-         i += (int64_t)gridDim.x * blockDim.x) {
-        if (i < nU) {
-            const int64_t n = i >> 6;
-            udup[i] = U[n * 32 + (i & 31)];
-        } else {
-            const int64_t j = i - nU;          // j = r * K + k
-            const int64_t r = j / K;
-            const int64_t k = j - r * K;
-            dt[j] = D[k * 32 + r];
-        }
-    }
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "r"(src_bytes) : "memory");
 }
 
-// ---------------------------------------------------------------------------
-// low-rank input t = x . lora_down (fp32 accumulation) on mma.sync bf16.
-// A CTA takes 16 rows; its 8 warps split K and their partial [16, 32] tiles
-// are summed in a fixed order.  Output either fp32 t [M, 32], or the split
-// form used by the forward's low-rank MMA step: with beta = g_x g_w (1 when
-// either is NULL or the product is 0), tt = t / beta, hi = bf16(tt),
-// lo = bf16(tt - hi), tsplit[m] = [hi[0:32] | lo[0:32]] (bf16 [M, 64]).
-// ---------------------------------------------------------------------------
+__device__ __forceinline__ void cp_async_commit()
+{
+    asm volatile("cp.async.commit_group;" ::: "memory");
+}
+
+template <int N>
+__device__ __forceinline__ void cp_async_wait()
+{
+    asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
+}
+
+__device__ __forceinline__ void ldmatrix_x4(uint32_t addr, uint32_t (&r)[4])
+{
+    asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]) : "r"(addr));
+}
+
+__device__ __forceinline__ void ldmatrix_x4_trans(uint32_t addr, uint32_t (&r)[4])
+{
+    asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]) : "r"(addr));
+}
+
 __device__ __forceinline__ void mma_bf16_16816(float (&c)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1)
 {
     asm volatile("mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 "
@@ -347,77 +346,193 @@ __device__ __forceinline__ void mma_bf16_16816(float (&c)[4], const uint32_t (&a
                  : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
 }
 
-__global__ void __launch_bounds__(256) lowrank_t_kernel(const uint16_t *__restrict__ x, int64_t M, int64_t K,
-                                                        const uint16_t *__restrict__ dt,
-                                                        const float *__restrict__ g_x,
-                                                        const float *__restrict__ g_w,
-                                                        float *__restrict__ t_out,
-                                                        uint16_t *__restrict__ tsplit)
+__device__ __forceinline__ uint32_t p1_xoff(int r, int c)
 {
-    __shared__ float part[8][16][33];
-    const int lane = threadIdx.x & 31;
-    const int wid = threadIdx.x >> 5;
-    const int gq = lane >> 2;       // groupID
-    const int tq = lane & 3;        // thread in group
-    const int64_t m0 = (int64_t)blockIdx.x * 16;
-    const int64_t kslice = K / 8;
-    const int64_t kbeg = wid * kslice;
-    const int64_t r0 = m0 + gq, r1 = m0 + gq + 8;
-    const uint32_t *x0 = reinterpret_cast<const uint32_t *>(x + (r0 < M ? r0 : 0) * K);
-    const uint32_t *x1 = reinterpret_cast<const uint32_t *>(x + (r1 < M ? r1 : 0) * K);
-    const uint32_t mask0 = r0 < M ? 0xffffffffu : 0u;
-    const uint32_t mask1 = r1 < M ? 0xffffffffu : 0u;
-    float c[4][4];
+    return (uint32_t)(r * 512 + 16 * (c ^ ((c >> 2) & 7) ^ (r & 7)));
+}
+
+__device__ __forceinline__ uint32_t p1_doff(int k, int c)
+{
+    return (uint32_t)(k * 64 + 16 * (c ^ ((k >> 1) & 3)));
+}
+
+__global__ void __launch_bounds__(256) act_pass1_kernel(const uint16_t *__restrict__ x, int64_t M, int64_t K,
+                                                        const uint16_t *__restrict__ D,
+                                                        uint32_t *__restrict__ amax, float *__restrict__ t32)
+{
+    extern __shared__ __align__(128) uint8_t p1_smem[];
+    const int tid = threadIdx.x;
+    const int lane = tid & 31;
+    const int warp = tid >> 5;
+    const int64_t m0 = (int64_t)blockIdx.x * kP1Rows;
+    const int nkb = (int)(K / kHad);
+    const uint32_t sbase = (uint32_t)__cvta_generic_to_shared(p1_smem);
+
+    auto issue = [&](int kb, int buf) {
+        const uint32_t xs = sbase + buf * kP1BufBytes;
+        const uint32_t ds = xs + kP1XBytes;
+#pragma unroll
+        for (int i = 0; i < 2; ++i) {                 // x: 16 rows x 32 chunks
+            const int e = tid + 256 * i;
+            const int r = e >> 5, c = e & 31;
+            const int64_t row = m0 + r;
+            const bool ok = row < M;
+            const uint16_t *src = x + (ok ? row : 0) * K + (int64_t)kb * kHad + 8 * c;
+            cp_async16(xs + p1_xoff(r, c), src, ok ? 16u : 0u);
+        }
+        if (t32) {
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {             // D: 256 k-rows x 4 chunks
+                const int e = tid + 256 * i;
+                const int k = e >> 2, c = e & 3;
+                cp_async16(ds + p1_doff(k, c), D + ((int64_t)kb * kHad + k) * kRank + 8 * c, 16u);
+            }
+        }
+        cp_async_commit();
+    };
+
+    float m = 0.0f;
+    float acc[4][4];
 #pragma unroll
     for (int nt = 0; nt < 4; ++nt)
 #pragma unroll
         for (int i = 0; i < 4; ++i)
-            c[nt][i] = 0.0f;
-    for (int64_t k0 = kbeg; k0 < kbeg + kslice; k0 += 16) {
-        const int64_t ka = (k0 + 2 * tq) >> 1;      // 32-bit word index
-        uint32_t a[4];
-        a[0] = __ldg(x0 + ka) & mask0;
-        a[1] = __ldg(x1 + ka) & mask1;
-        a[2] = __ldg(x0 + ka + 4) & mask0;
-        a[3] = __ldg(x1 + ka + 4) & mask1;
+            acc[nt][i] = 0.0f;
+
+    issue(0, 0);
+    for (int kb = 0; kb < nkb; ++kb) {
+        const int buf = kb & 1;
+        if (kb + 1 < nkb) {
+            issue(kb + 1, buf ^ 1);
+            cp_async_wait<1>();
+        } else {
+            cp_async_wait<0>();
+        }
+        __syncthreads();
+        const uint32_t xs = sbase + buf * kP1BufBytes;
+        const uint32_t ds = xs + kP1XBytes;
+        if (warp < 4) {
+            if (amax) {
+                const int r = 4 * warp + (lane >> 3);
+                const int q = lane & 7;
+                float v[32];
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    const uint4 a = *reinterpret_cast<const uint4 *>(p1_smem + (p1_xoff(r, 4 * q + i) +
+                                                                                 buf * kP1BufBytes));
+                    const uint32_t w[4] = {a.x, a.y, a.z, a.w};
+#pragma unroll
+                    for (int j = 0; j < 4; ++j) {
+                        v[8 * i + 2 * j] = __uint_as_float(w[j] << 16);
+                        v[8 * i + 2 * j + 1] = __uint_as_float(w[j] & 0xFFFF0000u);
+                    }
+                }
+                fwht256_l32(v, lane);
+#pragma unroll
+                for (int i = 0; i < 32; ++i)
+                    m = fmaxf(m, fabsf(v[i]));
+            }
+        } else if (t32) {
+            const int w4 = warp - 4;
+#pragma unroll
+            for (int s = 0; s < 4; ++s) {
+                const int ks = 4 * w4 + s;            // k-step: columns 16ks..16ks+15 of the chunk
+                // A 16x16: matrices (rows 0-7 | 8-15) x (k 0-7 | 8-15); lane provides row (lane & 15)
+                uint32_t a[4];
+                const int ar = lane & 15;
+                const int ac = 2 * ks + (lane >> 4);
+                ldmatrix_x4(xs + p1_xoff(ar, ac), a);
+                // B: (k 0-7 | 8-15) x (n-tile pair), transposed load of row-major D
+#pragma unroll
+                for (int np = 0; np < 2; ++np) {
+                    uint32_t b[4];
+                    const int bk = 16 * ks + (lane & 7) + 8 * ((lane >> 3) & 1);
+                    const int bc = 2 * np + (lane >> 4);
+                    ldmatrix_x4_trans(ds + p1_doff(bk, bc), b);
+                    mma_bf16_16816(acc[2 * np], a, b[0], b[1]);
+                    mma_bf16_16816(acc[2 * np + 1], a, b[2], b[3]);
+                }
+            }
+        }
+        __syncthreads();
+    }
+
+    if (amax) {
+#pragma unroll
+        for (int xx = 16; xx >= 1; xx >>= 1)
+            m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, xx));
+    }
+    // partial t tiles of warps 4-7 and the absmax reduce through the (now idle) smem
+    float *part = reinterpret_cast<float *>(p1_smem);          // [4][16][33]
+    float *wmax = part + 4 * 16 * 33;                           // [8]
+    if (warp >= 4 && t32) {
+        const int w4 = warp - 4;
+        const int g = lane >> 2, tq = lane & 3;
 #pragma unroll
         for (int nt = 0; nt < 4; ++nt) {
-            const uint32_t *drow = reinterpret_cast<const uint32_t *>(dt + (int64_t)(8 * nt + gq) * K);
-            const uint32_t b0 = __ldg(drow + ka);
-            const uint32_t b1 = __ldg(drow + ka + 4);
-            mma_bf16_16816(c[nt], a, b0, b1);
+            part[(w4 * 16 + g) * 33 + 8 * nt + 2 * tq] = acc[nt][0];
+            part[(w4 * 16 + g) * 33 + 8 * nt + 2 * tq + 1] = acc[nt][1];
+            part[(w4 * 16 + g + 8) * 33 + 8 * nt + 2 * tq] = acc[nt][2];
+            part[(w4 * 16 + g + 8) * 33 + 8 * nt + 2 * tq + 1] = acc[nt][3];
         }
     }
-#pragma unroll
-    for (int nt = 0; nt < 4; ++nt) {
-        part[wid][gq][8 * nt + 2 * tq] = c[nt][0];
-        part[wid][gq][8 * nt + 2 * tq + 1] = c[nt][1];
-        part[wid][gq + 8][8 * nt + 2 * tq] = c[nt][2];
-        part[wid][gq + 8][8 * nt + 2 * tq + 1] = c[nt][3];
-    }
+    if (lane == 0)
+        wmax[warp] = m;
     __syncthreads();
+    if (amax && tid == 0) {
+        float b = 0.0f;
+        for (int w = 0; w < 4; ++w)
+            b = fmaxf(b, wmax[w]);
+        atomic_max_nonneg(amax, b);
+    }
+    if (t32) {
+        for (int e = tid; e < kP1Rows * kRank; e += 256) {
+            const int r = e >> 5, col = e & 31;
+            if (m0 + r >= M)
+                continue;
+            float v = 0.0f;
+#pragma unroll
+            for (int w = 0; w < 4; ++w)
+                v = __fadd_rn(v, part[(w * 16 + r) * 33 + col]);
+            t32[(m0 + r) * kRank + col] = v;
+        }
+    }
+}
+
+// ---------------------------------------------------------------------------
+// low-rank operands of the forward's extra MMA step.  With beta = g_x g_w (1
+// when either pointer is NULL or the product is 0): tt = t / beta,
+// tsplit[m] = [bf16(tt) | bf16(tt - bf16(tt))] (bf16 [M, 64]), and
+// udup[n] = [U[n] | U[n]] (bf16 [N, 64]).
+// ---------------------------------------------------------------------------
+__global__ void __launch_bounds__(256) lowrank_finish_kernel(const float *__restrict__ t32, int64_t M,
+                                                             const float *__restrict__ g_x,
+                                                             const float *__restrict__ g_w,
+                                                             uint16_t *__restrict__ tsplit,
+                                                             const uint16_t *__restrict__ U, int64_t N,
+                                                             uint16_t *__restrict__ udup)
+{
     float beta = 1.0f;
     if (g_x && g_w) {
         const float b = __fmul_rn(*g_x, *g_w);
         beta = b == 0.0f ? 1.0f : b;
     }
-    for (int e = threadIdx.x; e < 16 * 32; e += blockDim.x) {
-        const int row = e >> 5, col = e & 31;
-        const int64_t m = m0 + row;
-        if (m >= M)
-            continue;
-        float s = 0.0f;
-#pragma unroll
-        for (int w = 0; w < 8; ++w)
-            s = __fadd_rn(s, part[w][row][col]);
-        if (t_out)
-            t_out[m * 32 + col] = s;
-        if (tsplit) {
-            const float tt = __fdiv_rn(s, beta);
+    const int64_t nT = M * kRank, nU = N * kRank;
+    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < nT + nU;
+         i += (int64_t)gridDim.x * blockDim.x) {
+        if (i < nT) {
+            const int64_t m = i >> 5, col = i & 31;
+            const float tt = __fdiv_rn(t32[i], beta);
             const uint32_t hi = f32_to_bf16_bits(tt);
             const uint32_t lo = f32_to_bf16_bits(__fsub_rn(tt, bf16_bits_to_f32(hi)));
             tsplit[m * 64 + col] = (uint16_t)hi;
             tsplit[m * 64 + 32 + col] = (uint16_t)lo;
+        } else {
+            const int64_t j = i - nT;
+            const int64_t n = j >> 5, col = j & 31;
+            const uint16_t u = U[j];
+            udup[n * 64 + col] = u;
+            udup[n * 64 + 32 + col] = u;
         }
     }
 }
@@ -540,14 +655,15 @@ static int grid_for(int64_t warp_tasks, int warps_per_block, int sms, int ctas_p
 cudaError_t launch_absmax_rot_f32(const float *in, int64_t rows, int64_t K, uint32_t *amax, int sms,
                                   cudaStream_t s)
 {
-    absmax_rot_kernel<float><<<grid_for(rows * (K / kHad), 8, sms, 8), 256, 0, s>>>(in, rows, K, amax);
+    absmax_rot_kernel<float><<<grid_for((rows * (K / kHad) + 3) / 4, 8, sms, 8), 256, 0, s>>>(in, rows, K, amax);
     return cudaGetLastError();
 }
 
 cudaError_t launch_absmax_rot_bf16(const uint16_t *in, int64_t rows, int64_t K, uint32_t *amax, int sms,
                                    cudaStream_t s)
 {
-    absmax_rot_kernel<uint16_t><<<grid_for(rows * (K / kHad), 8, sms, 8), 256, 0, s>>>(in, rows, K, amax);
+    absmax_rot_kernel<uint16_t><<<grid_for((rows * (K / kHad) + 3) / 4, 8, sms, 8), 256, 0, s>>>(in, rows, K,
+                                                                                                   amax);
     return cudaGetLastError();
 }
 
@@ -556,7 +672,7 @@ cudaError_t launch_nvfp4_quant_f32(const float *in, int64_t rows, int64_t K, con
                                    int sms, cudaStream_t s)
 {
     const int64_t rows_pad = (rows + 127) / 128 * 128;
-    nvfp4_quant_kernel<float><<<grid_for(rows_pad * (K / kHad), 8, sms, 8), 256, 0, s>>>(
+    nvfp4_quant_kernel<float><<<grid_for((rows_pad * (K / kHad) + 3) / 4, 8, sms, 8), 256, 0, s>>>(
         in, rows, rows_pad, K, amax, g_static, g_out, codes, sf);
     return cudaGetLastError();
 }
@@ -566,7 +682,7 @@ cudaError_t launch_nvfp4_quant_bf16(const uint16_t *in, int64_t rows, int64_t K,
                                     int sms, cudaStream_t s)
 {
     const int64_t rows_pad = (rows + 127) / 128 * 128;
-    nvfp4_quant_kernel<uint16_t><<<grid_for(rows_pad * (K / kHad), 8, sms, 8), 256, 0, s>>>(
+    nvfp4_quant_kernel<uint16_t><<<grid_for((rows_pad * (K / kHad) + 3) / 4, 8, sms, 8), 256, 0, s>>>(
         in, rows, rows_pad, K, amax, g_static, g_out, codes, sf);
     return cudaGetLastError();
 }
@@ -575,14 +691,13 @@ cudaError_t launch_int4_build(const float *R, int64_t N, int64_t K, uint8_t *cod
                               uint8_t *frac, int sms, cudaStream_t s)
 {
     const int64_t tasks = (N * K / kHad + 3) / 4;
-    int4_build_kernel<<<grid_for(tasks, kInt4Warps, sms, 4), kInt4Warps * 32, 0, s>>>(R, N, K, codes,
-                                                                                      scales, frac);
+    int4_build_kernel<<<grid_for(tasks, 8, sms, 4), 256, 0, s>>>(R, N, K, codes, scales, frac);
     return cudaGetLastError();
 }
 
 cudaError_t launch_rotate_bf16(const uint16_t *x, int64_t M, int64_t K, uint16_t *xb, int sms, cudaStream_t s)
 {
-    rotate_bf16_kernel<<<grid_for(M * (K / kHad), 8, sms, 8), 256, 0, s>>>(x, M, K, xb);
+    rotate_bf16_kernel<<<grid_for((M * (K / kHad) + 3) / 4, 8, sms, 8), 256, 0, s>>>(x, M, K, xb);
     return cudaGetLastError();
 }
 
@@ -595,19 +710,20 @@ cudaError_t launch_dequant_int4(const uint8_t *codes, const uint16_t *scales, in
     return cudaGetLastError();
 }
 
-cudaError_t launch_lora_prep(const uint16_t *U, int64_t N, const uint16_t *D, int64_t K, uint16_t *udup,
-                             uint16_t *dt, int sms, cudaStream_t s)
+cudaError_t launch_act_pass1(const uint16_t *x, int64_t M, int64_t K, const uint16_t *D, uint32_t *amax,
+                             float *t32, cudaStream_t s)
 {
-    const int64_t total = (udup ? N * 64 : 0) + (dt ? K * 32 : 0);
-    lora_prep_kernel<<<grid_for(total, 256, sms, 4), 256, 0, s>>>(U, N, D, K, udup, dt);
+    const int64_t grid = (M + kP1Rows - 1) / kP1Rows;
+    act_pass1_kernel<<<(unsigned)grid, 256, kP1Smem, s>>>(x, M, K, D, amax, t32);
     return cudaGetLastError();
 }
 
-cudaError_t launch_lowrank_t(const uint16_t *x, int64_t M, int64_t K, const uint16_t *dt, const float *g_x,
-                             const float *g_w, float *t_out, uint16_t *tsplit, cudaStream_t s)
+cudaError_t launch_lowrank_finish(const float *t32, int64_t M, const float *g_x, const float *g_w,
+                                  uint16_t *tsplit, const uint16_t *U, int64_t N, uint16_t *udup, int sms,
+                                  cudaStream_t s)
 {
-    const int64_t grid = (M + 15) / 16;
-    lowrank_t_kernel<<<(unsigned)grid, 256, 0, s>>>(x, M, K, dt, g_x, g_w, t_out, tsplit);
+    lowrank_finish_kernel<<<grid_for((M + N) * kRank, 256, sms, 4), 256, 0, s>>>(t32, M, g_x, g_w, tsplit, U, N,
+                                                                                  udup);
     return cudaGetLastError();
 }
 

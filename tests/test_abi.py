@@ -48,7 +48,8 @@ def test_size_helpers():
     assert sq.sq_sf_bytes(4480, 6144) == 4480 * 384
     assert sq.sq_workspace_bytes(sq.SQ_OP_BUILD_NVFP4, 0, 256, 512) >= 8
     ws = sq.sq_workspace_bytes(sq.SQ_OP_LINEAR_FWD_NVFP4, 64, 256, 512)
-    assert ws >= 64 * 256 + sq.sq_sf_bytes(64, 512) + 64 * 128 + 256 * 128 + 512 * 64
+    # activation codes + scales, fp32 t, [t_hi | t_lo], [U | U]
+    assert ws >= 64 * 256 + sq.sq_sf_bytes(64, 512) + 64 * 32 * 4 + 64 * 128 + 256 * 128
     wsi = sq.sq_workspace_bytes(sq.SQ_OP_LINEAR_FWD_INT4, 64, 256, 512)
     assert wsi >= 64 * 512 * 2 + 256 * 512 * 2
     assert sq.sq_workspace_bytes(99, 1, 1, 1) == 0
