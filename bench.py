@@ -40,10 +40,10 @@ sys.path.insert(0, ROOT)
 import synth_inputs as si  # noqa: E402
 
 METRIC = "W4 linear fwd TFLOP/s & % FP4/BF16 tensor peak; quantize/reconstruct GB/s % HBM"
-HEADLINE = "large_4480x6144x16384"
+HEADLINE = "large_4480x16384x6144"
 # SquareQ README, NVFP4 vs bf16 table: 4480 x 16384 x 6144 fp4 GEMM 1074 us on an
 # RTX 5080 (sm_120, cuBLASLt), i.e. 2*4480*16384*6144 / 1074e-6 = 840.3 TFLOP/s.
-PAGES_FP4_TFLOPS = {"large_4480x6144x16384": 2 * 4480 * 16384 * 6144 / 1074e-6 / 1e12}
+PAGES_FP4_TFLOPS = {"large_4480x16384x6144": 2 * 4480 * 16384 * 6144 / 1074e-6 / 1e12}
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 FP4_PER_BF16 = 4.0        # nominal dense FP4 / BF16 tensor ratio (9 / 2.25 PFLOP/s)
 FLUSH_BYTES = 256 << 20   # > 126 MB L2

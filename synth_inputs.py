@@ -42,13 +42,14 @@ class Config:
     hot_channels: int = 0
 
 
+# names give M x N x K (tokens x out x in), the order of the pages' GEMM table
 CONFIGS = {
-    "tiny_64x512x256": Config("tiny_64x512x256", 64, 512, 256, 0, "normal"),
+    "tiny_64x256x512": Config("tiny_64x256x512", 64, 512, 256, 0, "normal"),
     "proj_1536x3072x3072": Config("proj_1536x3072x3072", 1536, 3072, 3072, 1, "normal"),
-    "qkv_1536x3072x9216": Config("qkv_1536x3072x9216", 1536, 3072, 9216, 2, "normal", 4),
+    "qkv_1536x9216x3072": Config("qkv_1536x9216x3072", 1536, 3072, 9216, 2, "normal", 4),
     "large_4480x6144x6144": Config("large_4480x6144x6144", 4480, 6144, 6144, 3, "student"),
-    "large_4480x6144x16384": Config("large_4480x6144x16384", 4480, 6144, 16384, 3, "student"),
-    "down_4480x16384x6144": Config("down_4480x16384x6144", 4480, 16384, 6144, 4, "student"),
+    "large_4480x16384x6144": Config("large_4480x16384x6144", 4480, 6144, 16384, 3, "student"),
+    "down_4480x6144x16384": Config("down_4480x6144x16384", 4480, 16384, 6144, 4, "student"),
 }
 
 # the builder stack: 28 residual weights of the down-projection shape

@@ -20,9 +20,9 @@ from sqcase import FWD_TOL, bf16_dev, bits16, first_mismatch, host, norm_err, to
 
 pytestmark = pytest.mark.gpu
 
-FULL = ["tiny_64x512x256"]
-SAMPLED = ["proj_1536x3072x3072", "qkv_1536x3072x9216"]
-LARGE = ["large_4480x6144x6144", "large_4480x6144x16384", "down_4480x16384x6144"]
+FULL = ["tiny_64x256x512"]
+SAMPLED = ["proj_1536x3072x3072", "qkv_1536x9216x3072"]
+LARGE = ["large_4480x6144x6144", "large_4480x16384x6144", "down_4480x6144x16384"]
 
 
 @pytest.fixture(scope="module")
