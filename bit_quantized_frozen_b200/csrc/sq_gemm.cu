@@ -453,8 +453,8 @@ static PFN_encodeTiled encode_fn()
 }
 
 // 2D row-major tensor [rows, inner] of `esize`-byte elements, box [box_rows, box_inner]
-static bool make_tmap(CUtensorMap *m, CUtensorMapDataType dt, int esize, const void *base, uint64_t inner,
-                      uint64_t rows, uint32_t box_inner, uint32_t box_rows, CUtensorMapSwizzle sw)
+bool make_tmap(CUtensorMap *m, CUtensorMapDataType dt, int esize, const void *base, uint64_t inner,
+               uint64_t rows, uint32_t box_inner, uint32_t box_rows, CUtensorMapSwizzle sw)
 {
     PFN_encodeTiled fn = encode_fn();
     if (!fn)

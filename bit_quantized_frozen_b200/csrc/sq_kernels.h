@@ -2,6 +2,7 @@
 #pragma once
 
 #include <cstdint>
+#include <cuda.h>
 #include <cuda_runtime.h>
 
 namespace sq {
@@ -47,5 +48,9 @@ struct GemmLaunch {
 };
 
 cudaError_t launch_gemm(const GemmLaunch &g, int sms, cudaStream_t stream);
+
+// 2D row-major tensor map [rows, inner] of esize-byte elements, box [box_rows, box_inner]
+bool make_tmap(CUtensorMap *m, CUtensorMapDataType dt, int esize, const void *base, uint64_t inner,
+               uint64_t rows, uint32_t box_inner, uint32_t box_rows, CUtensorMapSwizzle sw);
 
 }  // namespace sq

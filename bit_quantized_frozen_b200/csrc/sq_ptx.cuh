@@ -70,7 +70,8 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatil
                 return false;
             if (global_ns() - t0 > kWaitLimitNs) {
                 *abort_flag = 1u;
-                atomicOr(status, 1u);
+                if (status)
+                    atomicOr(status, 1u);
                 return false;
             }
         }

@@ -10,82 +10,159 @@
 // operation by operation in include/sq.h.
 #include "sq_kernels.h"
 #include "sq_device.cuh"
+#include "sq_ptx.cuh"
 
 namespace sq {
 
 // ---------------------------------------------------------------------------
-// Warp tasks over 256-blocks.  A warp takes 4 consecutive blocks of the
-// row-major matrix (flat block index 4*task + lane/8); lane q = lane % 8 holds
-// values 32q..32q+31 of its block (the layout of fwht256_l32).  Blocks past the
-// end are processed as zeros and never stored, so every lane joins the
-// shuffles of the transform.
+// Block streamer.  The input ([rows, K], K % 256 == 0) is viewed as a 2-D
+// tensor of 32-value rows; a producer warp (warp 8) TMA-loads chunks of 256
+// such rows (32 Hadamard blocks) into a ring of shared-memory stages, with the
+// 128-byte (fp32) or 64-byte (bf16) swizzle so that eight consumer warps can
+// each read their own 32-value row conflict free.  Consumer warp w, lane L
+// gets row 32w + L of the chunk: block 4w + L/8, values 32(L%8)..+31 -- the
+// layout of fwht256_l32.  Rows past the tensor are zero-filled by the TMA.
 // ---------------------------------------------------------------------------
+constexpr int kStreamConsumers = 8;
+constexpr int kStreamThreads = 32 * (kStreamConsumers + 1);
+
 template <typename T>
-__device__ __forceinline__ void load_block_l32(const T *base, int64_t block, bool valid, int lane, float (&v)[32])
+struct StreamCfg {
+    static constexpr int kStages = sizeof(T) == 4 ? 3 : 4;
+    static constexpr int kChunkBytes = 32 * kHad * (int)sizeof(T);            // 32 blocks
+    static constexpr int kSmem = kStages * kChunkBytes + 2 * kStages * 8 + 16 + 1024;
+};
+
+template <typename T>
+__device__ __forceinline__ void read_row(const uint8_t *buf, int row, float (&v)[32])
 {
-    if (valid) {
-        load32(base + block * kHad + 32 * (lane & 7), v);
-    } else {
+    if (sizeof(T) == 4) {          // 128-byte rows, chunk i at i ^ (row & 7)
 #pragma unroll
-        for (int i = 0; i < 32; ++i)
-            v[i] = 0.0f;
+        for (int i = 0; i < 8; ++i) {
+            const float4 a = *reinterpret_cast<const float4 *>(buf + row * 128 + 16 * (i ^ (row & 7)));
+            v[4 * i] = a.x; v[4 * i + 1] = a.y; v[4 * i + 2] = a.z; v[4 * i + 3] = a.w;
+        }
+    } else {                       // 64-byte rows, chunk i at i ^ ((row >> 1) & 3)
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            const uint4 a = *reinterpret_cast<const uint4 *>(buf + row * 64 + 16 * (i ^ ((row >> 1) & 3)));
+            const uint32_t w[4] = {a.x, a.y, a.z, a.w};
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                v[8 * i + 2 * j] = __uint_as_float(w[j] << 16);
+                v[8 * i + 2 * j + 1] = __uint_as_float(w[j] & 0xFFFF0000u);
+            }
+        }
     }
 }
 
+// Runs f(block, v, valid) on every 256-block of the stream, one call per lane
+// per chunk in consumer warps (all 32 lanes of a warp call f together, so f
+// may shuffle).  total_blocks may exceed the tensor (zero blocks).
+template <typename T, typename F>
+__device__ __forceinline__ void stream_blocks(const CUtensorMap *tm, int64_t total_blocks, uint32_t *status, F &&f)
+{
+    using Cfg = StreamCfg<T>;
+    extern __shared__ uint8_t stream_smem_raw[];
+    uint8_t *smem =
+        reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(stream_smem_raw) + 1023) & ~uintptr_t(1023));
+    uint64_t *bars = reinterpret_cast<uint64_t *>(smem + Cfg::kStages * Cfg::kChunkBytes);
+    const uint32_t full = smem_u32(bars), empty = smem_u32(bars + Cfg::kStages);
+    volatile uint32_t *abort_flag = reinterpret_cast<uint32_t *>(bars + 2 * Cfg::kStages);
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    if (threadIdx.x == 0) {
+        for (int st = 0; st < Cfg::kStages; ++st) {
+            mbar_init(full + 8 * st, 1);
+            mbar_init(empty + 8 * st, kStreamConsumers);
+        }
+        *abort_flag = 0u;
+        fence_mbar_init();
+    }
+    __syncthreads();
+    const int64_t chunks = (total_blocks + 31) / 32;
+    if (warp == kStreamConsumers) {
+        if (lane == 0) {
+            prefetch_tmap(tm);
+            int it = 0;
+            for (int64_t c = blockIdx.x; c < chunks; c += gridDim.x, ++it) {
+                const int st = it % Cfg::kStages;
+                const uint32_t ph = (uint32_t)(it / Cfg::kStages) & 1u;
+                if (!mbar_wait(empty + 8 * st, ph ^ 1u, abort_flag, status))
+                    break;
+                mbar_arrive_expect_tx(full + 8 * st, Cfg::kChunkBytes);
+                tma_load_2d(smem_u32(smem + st * Cfg::kChunkBytes), tm, 0, (int32_t)(c * 256), full + 8 * st);
+            }
+        }
+        __syncwarp();
+    } else {
+        int it = 0;
+        for (int64_t c = blockIdx.x; c < chunks; c += gridDim.x, ++it) {
+            const int st = it % Cfg::kStages;
+            const uint32_t ph = (uint32_t)(it / Cfg::kStages) & 1u;
+            int ok = 1;
+            if (lane == 0)
+                ok = mbar_wait(full + 8 * st, ph, abort_flag, status) ? 1 : 0;
+            if (__shfl_sync(0xffffffffu, ok, 0) == 0)
+                break;
+            float v[32];
+            read_row<T>(smem + st * Cfg::kChunkBytes, 32 * warp + lane, v);
+            __syncwarp();
+            if (lane == 0)
+                mbar_arrive(empty + 8 * st);
+            const int64_t block = 32 * c + 4 * warp + (lane >> 3);
+            f(block, v, block < total_blocks);
+        }
+    }
+    __syncthreads();
+}
+
 // ---------------------------------------------------------------------------
-// pass 1 of the NVFP4 builder: A = max |H R| over a [rows, K] matrix, folded
+// pass 1 of the NVFP4 builder: A = max |H in| over a [rows, K] matrix, folded
 // into *amax (u32 bits of a non-negative float)
 // ---------------------------------------------------------------------------
 template <typename T>
-__global__ void __launch_bounds__(256) absmax_rot_kernel(const T *__restrict__ in, int64_t rows,
-                                                         int64_t K, uint32_t *__restrict__ amax)
+__global__ void __launch_bounds__(kStreamThreads) absmax_rot_kernel(const __grid_constant__ CUtensorMap tm,
+                                                                    int64_t blocks, uint32_t *__restrict__ amax)
 {
     const int lane = threadIdx.x & 31;
-    const int64_t blocks = rows * (K / kHad);
-    const int64_t tasks = (blocks + 3) / 4;
-    const int64_t warps_total = (int64_t)gridDim.x * (blockDim.x >> 5);
     float m = 0.0f;
-    for (int64_t task = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); task < tasks;
-         task += warps_total) {
-        const int64_t b = 4 * task + (lane >> 3);
-        float v[32];
-        load_block_l32(in, b, b < blocks, lane, v);
+    stream_blocks<T>(&tm, blocks, nullptr, [&](int64_t, float (&v)[32], bool) {
         fwht256_l32(v, lane);
 #pragma unroll
         for (int i = 0; i < 32; ++i)
             m = fmaxf(m, fabsf(v[i]));
-    }
+    });
 #pragma unroll
     for (int x = 16; x >= 1; x >>= 1)
         m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, x));
-    __shared__ float wmax[32];
+    __shared__ float wmax[kStreamConsumers + 1];
     if (lane == 0)
         wmax[threadIdx.x >> 5] = m;
     __syncthreads();
     if (threadIdx.x == 0) {
         float b = 0.0f;
-        for (int w = 0; w < (int)(blockDim.x >> 5); ++w)
+        for (int w = 0; w < kStreamConsumers; ++w)
             b = fmaxf(b, wmax[w]);
         atomic_max_nonneg(amax, b);
     }
 }
 
 // ---------------------------------------------------------------------------
-// NVFP4 block quantisation of H in with global scale g.  rows_pad >= rows (a
-// multiple of 128): rows past `rows` are zero and only their scale bytes are
-// written (as 0), which fills the tiled layout's padding.  g comes from
+// NVFP4 block quantisation of H in with global scale g, over rows_pad rows
+// (a multiple of 128): rows past `rows` are zero and only their scale bytes
+// are written (as 0), which fills the tiled layout's padding.  g comes from
 // *g_static when non-NULL, else RN(A / 2688) from *amax, and is stored to
 // *g_out (when non-NULL) by thread 0 of block 0.  Each lane owns two whole
 // 16-value blocks, so block maxima and scales need no shuffles.
 // ---------------------------------------------------------------------------
 template <typename T>
-__global__ void __launch_bounds__(256) nvfp4_quant_kernel(const T *__restrict__ in, int64_t rows,
-                                                          int64_t rows_pad, int64_t K,
-                                                          const uint32_t *__restrict__ amax,
-                                                          const float *__restrict__ g_static,
-                                                          float *__restrict__ g_out,
-                                                          uint8_t *__restrict__ codes,
-                                                          uint8_t *__restrict__ sf)
+__global__ void __launch_bounds__(kStreamThreads) nvfp4_quant_kernel(const __grid_constant__ CUtensorMap tm,
+                                                                     int64_t rows, int64_t rows_pad, int64_t K,
+                                                                     const uint32_t *__restrict__ amax,
+                                                                     const float *__restrict__ g_static,
+                                                                     float *__restrict__ g_out,
+                                                                     uint8_t *__restrict__ codes,
+                                                                     uint8_t *__restrict__ sf)
 {
     const int lane = threadIdx.x & 31;
     const int q = lane & 7;
@@ -95,20 +172,12 @@ __global__ void __launch_bounds__(256) nvfp4_quant_kernel(const T *__restrict__ 
     const float sixg = __fmul_rn(6.0f, g);
     const int64_t kb_per_row = K / kHad;
     const int64_t C = K / kSfBlock;
-    const int64_t blocks = rows_pad * kb_per_row;
-    const int64_t tasks = (blocks + 3) / 4;
-    const int64_t warps_total = (int64_t)gridDim.x * (blockDim.x >> 5);
-    for (int64_t task = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); task < tasks;
-         task += warps_total) {
-        const int64_t b = 4 * task + (lane >> 3);
+    stream_blocks<T>(&tm, rows_pad * kb_per_row, nullptr, [&](int64_t b, float (&v)[32], bool valid) {
+        fwht256_l32(v, lane);
+        if (!valid)
+            return;
         const int64_t row = b / kb_per_row;
         const int64_t kb = b - row * kb_per_row;
-        const bool in_range = b < blocks;
-        float v[32];
-        load_block_l32(in, row * kb_per_row + kb, in_range && row < rows, lane, v);
-        fwht256_l32(v, lane);
-        if (!in_range)
-            continue;
         uint32_t word[4];
         uint32_t sfc[2];
 #pragma unroll
@@ -143,13 +212,13 @@ __global__ void __launch_bounds__(256) nvfp4_quant_kernel(const T *__restrict__ 
         // scale columns 2q, 2q+1 of the block are adjacent bytes of the tiled layout
         *reinterpret_cast<uint16_t *>(sf + sf_offset(row, kb * (kHad / kSfBlock) + 2 * q, C)) =
             (uint16_t)(sfc[0] | (sfc[1] << 8));
-    }
+    });
 }
 
 // ---------------------------------------------------------------------------
 // int4 group-32 builder.  With the 8-lane Hadamard layout every lane holds one
 // whole group of 32 rotated values and sweeps the 26 scale fractions in
-// registers; a warp covers 32 consecutive groups.
+// registers (group index = 8 * block + lane % 8).
 // ---------------------------------------------------------------------------
 __device__ __forceinline__ float group_sq_error(const float (&r)[32], float s, float inv)
 {
@@ -175,24 +244,16 @@ __device__ __forceinline__ float group_sq_error(const float (&r)[32], float s, f
     return p[0];
 }
 
-__global__ void __launch_bounds__(256, 2) int4_build_kernel(const float *__restrict__ R, int64_t N, int64_t K,
-                                                         uint8_t *__restrict__ codes,
-                                                         uint16_t *__restrict__ scales,
-                                                         uint8_t *__restrict__ frac)
+__global__ void __launch_bounds__(kStreamThreads) int4_build_kernel(const __grid_constant__ CUtensorMap tm,
+                                                                    int64_t blocks, uint8_t *__restrict__ codes,
+                                                                    uint16_t *__restrict__ scales,
+                                                                    uint8_t *__restrict__ frac)
 {
     const int lane = threadIdx.x & 31;
-    const int64_t blocks = N * K / kHad;
-    const int64_t tasks = (blocks + 3) / 4;
-    const int64_t warps_total = (int64_t)gridDim.x * (blockDim.x >> 5);
-    for (int64_t task = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); task < tasks;
-         task += warps_total) {
-        const int64_t b = 4 * task + (lane >> 3);
-        const bool valid = b < blocks;
-        float r[32];
-        load_block_l32(R, b, valid, lane, r);
+    stream_blocks<float>(&tm, blocks, nullptr, [&](int64_t b, float (&r)[32], bool valid) {
         fwht256_l32(r, lane);
         if (!valid)
-            continue;
+            return;
         float a = 0.0f;
 #pragma unroll
         for (int i = 0; i < 32; ++i)
@@ -226,33 +287,25 @@ __global__ void __launch_bounds__(256, 2) int4_build_kernel(const float *__restr
             }
             word[i >> 3] |= ((uint32_t)q & 0xFu) << (4 * (i & 7));
         }
-        const int64_t gidx = 32 * task + lane;     // flat group index
+        const int64_t gidx = 8 * b + (lane & 7);     // flat group index
         reinterpret_cast<uint4 *>(codes)[gidx] = make_uint4(word[0], word[1], word[2], word[3]);
         scales[gidx] = best_h;
         if (frac)
             frac[gidx] = (uint8_t)best_j;
-    }
+    });
 }
 
 // ---------------------------------------------------------------------------
 // int4 forward prologue: xb = bf16(H x), [M, K]
 // ---------------------------------------------------------------------------
-__global__ void __launch_bounds__(256) rotate_bf16_kernel(const uint16_t *__restrict__ x, int64_t M,
-                                                          int64_t K, uint16_t *__restrict__ xb)
+__global__ void __launch_bounds__(kStreamThreads) rotate_bf16_kernel(const __grid_constant__ CUtensorMap tm,
+                                                                     int64_t blocks, uint16_t *__restrict__ xb)
 {
     const int lane = threadIdx.x & 31;
-    const int64_t blocks = M * (K / kHad);
-    const int64_t tasks = (blocks + 3) / 4;
-    const int64_t warps_total = (int64_t)gridDim.x * (blockDim.x >> 5);
-    for (int64_t task = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); task < tasks;
-         task += warps_total) {
-        const int64_t b = 4 * task + (lane >> 3);
-        const bool valid = b < blocks;
-        float v[32];
-        load_block_l32(x, b, valid, lane, v);
+    stream_blocks<uint16_t>(&tm, blocks, nullptr, [&](int64_t b, float (&v)[32], bool valid) {
         fwht256_l32(v, lane);
         if (!valid)
-            continue;
+            return;
         uint4 *o = reinterpret_cast<uint4 *>(xb + b * kHad + 32 * (lane & 7));
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
@@ -262,7 +315,7 @@ __global__ void __launch_bounds__(256) rotate_bf16_kernel(const uint16_t *__rest
                 w[j] = f32_to_bf16_bits(v[8 * i + 2 * j]) | (f32_to_bf16_bits(v[8 * i + 2 * j + 1]) << 16);
             o[i] = make_uint4(w[0], w[1], w[2], w[3]);
         }
-    }
+    });
 }
 
 // ---------------------------------------------------------------------------
@@ -652,52 +705,109 @@ static int grid_for(int64_t warp_tasks, int warps_per_block, int sms, int ctas_p
     return (int)(want < 1 ? 1 : want);
 }
 
-cudaError_t launch_absmax_rot_f32(const float *in, int64_t rows, int64_t K, uint32_t *amax, int sms,
-                                  cudaStream_t s)
+// streamer launch: tensor map over `in` as [rows * K / 32, 32], persistent grid
+template <typename T>
+static bool stream_map(CUtensorMap *tm, const T *in, int64_t rows, int64_t K)
 {
-    absmax_rot_kernel<float><<<grid_for((rows * (K / kHad) + 3) / 4, 8, sms, 8), 256, 0, s>>>(in, rows, K, amax);
+    const bool f32 = sizeof(T) == 4;
+    return make_tmap(tm, f32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, (int)sizeof(T), in,
+                     32, (uint64_t)(rows * K / 32), 32, 256, f32 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B);
+}
+
+template <typename T, typename Kern>
+static cudaError_t stream_attr(Kern k)
+{
+    return cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, StreamCfg<T>::kSmem);
+}
+
+static int stream_grid(int64_t blocks, int sms, int per_sm)
+{
+    const int64_t chunks = (blocks + 31) / 32;
+    const int64_t cap = (int64_t)sms * per_sm;
+    return (int)(chunks < 1 ? 1 : (chunks < cap ? chunks : cap));
+}
+
+template <typename T>
+static cudaError_t launch_absmax_rot(const T *in, int64_t rows, int64_t K, uint32_t *amax, int sms, cudaStream_t s)
+{
+    CUtensorMap tm;
+    if (!stream_map(&tm, in, rows, K))
+        return cudaErrorInvalidValue;
+    cudaError_t e = stream_attr<T>(absmax_rot_kernel<T>);
+    if (e != cudaSuccess)
+        return e;
+    const int64_t blocks = rows * (K / kHad);
+    absmax_rot_kernel<T><<<stream_grid(blocks, sms, sizeof(T) == 4 ? 2 : 3), kStreamThreads, StreamCfg<T>::kSmem, s>>>(
+        tm, blocks, amax);
     return cudaGetLastError();
+}
+
+template <typename T>
+static cudaError_t launch_nvfp4_quant(const T *in, int64_t rows, int64_t K, const uint32_t *amax, const float *g_static,
+                                      float *g_out, uint8_t *codes, uint8_t *sf, int sms, cudaStream_t s)
+{
+    CUtensorMap tm;
+    if (!stream_map(&tm, in, rows, K))
+        return cudaErrorInvalidValue;
+    cudaError_t e = stream_attr<T>(nvfp4_quant_kernel<T>);
+    if (e != cudaSuccess)
+        return e;
+    const int64_t rows_pad = (rows + 127) / 128 * 128;
+    nvfp4_quant_kernel<T><<<stream_grid(rows_pad * (K / kHad), sms, sizeof(T) == 4 ? 2 : 3), kStreamThreads,
+                            StreamCfg<T>::kSmem, s>>>(tm, rows, rows_pad, K, amax, g_static, g_out, codes, sf);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_absmax_rot_f32(const float *in, int64_t rows, int64_t K, uint32_t *amax, int sms, cudaStream_t s)
+{
+    return launch_absmax_rot(in, rows, K, amax, sms, s);
 }
 
 cudaError_t launch_absmax_rot_bf16(const uint16_t *in, int64_t rows, int64_t K, uint32_t *amax, int sms,
                                    cudaStream_t s)
 {
-    absmax_rot_kernel<uint16_t><<<grid_for((rows * (K / kHad) + 3) / 4, 8, sms, 8), 256, 0, s>>>(in, rows, K,
-                                                                                                   amax);
-    return cudaGetLastError();
+    return launch_absmax_rot(in, rows, K, amax, sms, s);
 }
 
 cudaError_t launch_nvfp4_quant_f32(const float *in, int64_t rows, int64_t K, const uint32_t *amax,
-                                   const float *g_static, float *g_out, uint8_t *codes, uint8_t *sf,
-                                   int sms, cudaStream_t s)
+                                   const float *g_static, float *g_out, uint8_t *codes, uint8_t *sf, int sms,
+                                   cudaStream_t s)
 {
-    const int64_t rows_pad = (rows + 127) / 128 * 128;
-    nvfp4_quant_kernel<float><<<grid_for((rows_pad * (K / kHad) + 3) / 4, 8, sms, 8), 256, 0, s>>>(
-        in, rows, rows_pad, K, amax, g_static, g_out, codes, sf);
-    return cudaGetLastError();
+    return launch_nvfp4_quant(in, rows, K, amax, g_static, g_out, codes, sf, sms, s);
 }
 
 cudaError_t launch_nvfp4_quant_bf16(const uint16_t *in, int64_t rows, int64_t K, const uint32_t *amax,
-                                    const float *g_static, float *g_out, uint8_t *codes, uint8_t *sf,
-                                    int sms, cudaStream_t s)
+                                    const float *g_static, float *g_out, uint8_t *codes, uint8_t *sf, int sms,
+                                    cudaStream_t s)
 {
-    const int64_t rows_pad = (rows + 127) / 128 * 128;
-    nvfp4_quant_kernel<uint16_t><<<grid_for((rows_pad * (K / kHad) + 3) / 4, 8, sms, 8), 256, 0, s>>>(
-        in, rows, rows_pad, K, amax, g_static, g_out, codes, sf);
-    return cudaGetLastError();
+    return launch_nvfp4_quant(in, rows, K, amax, g_static, g_out, codes, sf, sms, s);
 }
 
 cudaError_t launch_int4_build(const float *R, int64_t N, int64_t K, uint8_t *codes, uint16_t *scales,
                               uint8_t *frac, int sms, cudaStream_t s)
 {
-    const int64_t tasks = (N * K / kHad + 3) / 4;
-    int4_build_kernel<<<grid_for(tasks, 8, sms, 4), 256, 0, s>>>(R, N, K, codes, scales, frac);
+    CUtensorMap tm;
+    if (!stream_map(&tm, R, N, K))
+        return cudaErrorInvalidValue;
+    cudaError_t e = stream_attr<float>(int4_build_kernel);
+    if (e != cudaSuccess)
+        return e;
+    const int64_t blocks = N * K / kHad;
+    int4_build_kernel<<<stream_grid(blocks, sms, 2), kStreamThreads, StreamCfg<float>::kSmem, s>>>(tm, blocks, codes,
+                                                                                                   scales, frac);
     return cudaGetLastError();
 }
 
 cudaError_t launch_rotate_bf16(const uint16_t *x, int64_t M, int64_t K, uint16_t *xb, int sms, cudaStream_t s)
 {
-    rotate_bf16_kernel<<<grid_for((M * (K / kHad) + 3) / 4, 8, sms, 8), 256, 0, s>>>(x, M, K, xb);
+    CUtensorMap tm;
+    if (!stream_map(&tm, x, M, K))
+        return cudaErrorInvalidValue;
+    cudaError_t e = stream_attr<uint16_t>(rotate_bf16_kernel);
+    if (e != cudaSuccess)
+        return e;
+    const int64_t blocks = M * (K / kHad);
+    rotate_bf16_kernel<<<stream_grid(blocks, sms, 3), kStreamThreads, StreamCfg<uint16_t>::kSmem, s>>>(tm, blocks, xb);
     return cudaGetLastError();
 }
 
