@@ -49,11 +49,11 @@ __device__ __forceinline__ void fwht256_warp(float (&v)[8], int lane)
     }
 #pragma unroll
     for (int x = 1; x <= 16; x <<= 1) {          // h = 4x
-        const bool lower = (lane & x) == 0;
+        const float sg = (lane & x) == 0 ? 1.0f : -1.0f;
 #pragma unroll
         for (int i = 0; i < 8; ++i) {
-            float p = __shfl_xor_sync(0xffffffffu, v[i], x);
-            v[i] = lower ? __fadd_rn(v[i], p) : __fsub_rn(p, v[i]);
+            const float p = __shfl_xor_sync(0xffffffffu, v[i], x);
+            v[i] = __fmaf_rn(sg, v[i], p);
         }
     }
 #pragma unroll
@@ -89,11 +89,12 @@ __device__ __forceinline__ void fwht256_l32(float (&v)[32], int lane)
             }
 #pragma unroll
     for (int x = 1; x <= 4; x <<= 1) {          // h = 32x
-        const bool lower = (lane & x) == 0;
+        // lower lane: p + v, upper lane: p - v, as one fma with +-1 (same single rounding)
+        const float sg = (lane & x) == 0 ? 1.0f : -1.0f;
 #pragma unroll
         for (int i = 0; i < 32; ++i) {
             const float p = __shfl_xor_sync(0xffffffffu, v[i], x);
-            v[i] = lower ? __fadd_rn(v[i], p) : __fsub_rn(p, v[i]);
+            v[i] = __fmaf_rn(sg, v[i], p);
         }
     }
 #pragma unroll

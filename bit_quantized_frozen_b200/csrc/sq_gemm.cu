@@ -35,24 +35,26 @@
 
 namespace sq {
 
-constexpr int BM = 128;
+constexpr int BM = 256;                        // cluster tile: two CTAs x 128 rows
 constexpr int BN = 256;
+constexpr int kRowsPerCta = 128;
 constexpr int kRowBytes = 128;                 // every stage holds 128-byte rows (one swizzle atom)
-constexpr int kABytes = BM * kRowBytes;        // 16 KB
-constexpr int kBBytes = BN * kRowBytes;        // 32 KB
+constexpr int kABytes = kRowsPerCta * kRowBytes;   // 16 KB: this CTA's 128 rows of A
+constexpr int kBBytes = 128 * kRowBytes;           // 16 KB: this CTA's half (128 rows) of B
 constexpr int kMmaPerStage = 4;                // K = 64 (fp4) or 16 (bf16) per MMA, 32 bytes of the row each
 constexpr int kSfaBytes = kMmaPerStage * 512;  // one 512-byte chunk (128 rows x 4 scales) per MMA
-constexpr int kSfbBytes = 2 * kSfaBytes;       // 256 rows
+constexpr int kSfbBytes = 2 * kSfaBytes;       // both 128-row halves of B (every CTA needs all 256)
 constexpr int kEpiWarps = 4;
 constexpr int kStagingBytes = 32 * 128;        // one warp's 32 rows x 32 fp32
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kAccSlot1 = 128;            // accumulator slots [0, 256) and [128, 384)
 constexpr int kOverlapChunks = 4;              // 32-column chunks shared by the two slots
-constexpr uint32_t kSfCol = 384;               // two scale-factor buffers of 48 columns, one stage each
-constexpr uint32_t kSfBufCols = 48;            // SFB for MMA k at +8k (256 rows), SFA at +32+4k (128 rows)
-constexpr uint32_t kSfBufs = 2;
+constexpr uint32_t kSfCol = 384;               // ring of five scale-factor buffers, two MMAs each
+constexpr int kMmaPerSfBuf = 2;
+constexpr uint32_t kSfBufCols = 24;            // SFB for MMA k at +8k (256 rows), SFA at +16+4k (128 rows)
+constexpr uint32_t kSfBufs = 5;
 
-// instruction descriptors: M = 128, N = 256, K-major A and B
+// instruction descriptors: M = 256 (the CTA pair), N = 256, K-major A and B
 constexpr uint32_t kIdescBf16 = (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(BN >> 3) << 17) |
                                 ((uint32_t)(BM >> 4) << 24);           // f32 accum, bf16 x bf16
 constexpr uint32_t kIdescNvfp4 = (1u << 7) | (1u << 10) | ((uint32_t)(BN >> 3) << 17) |
@@ -60,14 +62,15 @@ constexpr uint32_t kIdescNvfp4 = (1u << 7) | (1u << 10) | ((uint32_t)(BN >> 3) <
 
 template <bool FP4>
 struct GemmCfg {
-    static constexpr int kStages = FP4 ? 3 : 4;
-    static constexpr int kScaleWarps = FP4 ? 4 : 0;              // warps 6..9 fill the scale-factor ring
+    static constexpr int kStages = FP4 ? 5 : 6;
+    static constexpr int kScaleWarps = FP4 ? 4 : 0;              // warps 6..9 fill the scale-factor buffers
     static constexpr int kThreads = 32 * (6 + kScaleWarps);
     static constexpr int kStageBytes = kABytes + kBBytes + (FP4 ? kSfaBytes + kSfbBytes : 0);
     static constexpr int kKPerStage = FP4 ? 256 : 64;            // K values per stage
     static constexpr int kStagingOff = kStages * kStageBytes;
     static constexpr int kBarOff = kStagingOff + kEpiWarps * 2 * kStagingBytes;
-    static constexpr int kNumBars = 2 * kStages + 4 + (FP4 ? 2 * kSfBufs : 0);
+    // full[s], empty[s], sfdata[s], acc_full[2], acc_empty, drain, sf_full[b], sf_empty[b]
+    static constexpr int kNumBars = 3 * kStages + 4 + 2 * kSfBufs;
     static constexpr int kSmemBytes = kBarOff + 8 * kNumBars + 16 + 1024;   // + holder, flag, alignment
 };
 
@@ -78,16 +81,25 @@ struct GemmArgs {
     const float *g_w;        // NVFP4: weight global scale (device)
     uint32_t *status;        // device status word
     int M, N, K;
-    int lora;                // 1: add the low-rank K-steps
+    int lora;                // 1: add the low-rank K-step
 };
 
-// warp-uniform bounded wait: lane 0 polls, the verdict is broadcast
+// warp-uniform bounded wait on a local barrier: lane 0 polls, the verdict is broadcast
 __device__ __forceinline__ bool warp_wait(uint32_t bar, uint32_t parity, volatile uint32_t *abort_flag,
                                           uint32_t *status, int lane)
 {
     int ok = 1;
     if (lane == 0)
         ok = mbar_wait(bar, parity, abort_flag, status) ? 1 : 0;
+    return __shfl_sync(0xffffffffu, ok, 0) != 0;
+}
+
+__device__ __forceinline__ bool warp_wait_cluster(uint32_t bar, uint32_t parity, volatile uint32_t *abort_flag,
+                                                  uint32_t *status, int lane)
+{
+    int ok = 1;
+    if (lane == 0)
+        ok = mbar_wait_cluster(bar, parity, abort_flag, status) ? 1 : 0;
     return __shfl_sync(0xffffffffu, ok, 0) != 0;
 }
 
@@ -119,7 +131,7 @@ __device__ __forceinline__ void store_chunk(const uint32_t (&r)[32], float beta,
 }
 
 template <bool FP4>
-__global__ void __launch_bounds__(GemmCfg<FP4>::kThreads, 1)
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(GemmCfg<FP4>::kThreads, 1)
     sq_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                    const __grid_constant__ CUtensorMap tmT, const __grid_constant__ CUtensorMap tmU,
                    const __grid_constant__ CUtensorMap tmY, const GemmArgs args)
@@ -128,41 +140,42 @@ __global__ void __launch_bounds__(GemmCfg<FP4>::kThreads, 1)
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint64_t *bars = reinterpret_cast<uint64_t *>(smem + Cfg::kBarOff);
-    // barriers: full[s], empty[s], acc_full[2], acc_empty, drain, sf_full[r], sf_empty[r]
-    const uint32_t bar_full = smem_u32(bars);
-    const uint32_t bar_empty = smem_u32(bars + Cfg::kStages);
-    const uint32_t bar_acc_full = smem_u32(bars + 2 * Cfg::kStages);
-    const uint32_t bar_acc_empty = smem_u32(bars + 2 * Cfg::kStages + 2);
-    const uint32_t bar_drain = smem_u32(bars + 2 * Cfg::kStages + 3);
-    const uint32_t bar_sf_full = smem_u32(bars + 2 * Cfg::kStages + 4);
-    const uint32_t bar_sf_empty = bar_sf_full + 8 * kSfBufs;
+    const uint32_t bar_full = smem_u32(bars);                          // leader: A/B of both CTAs landed
+    const uint32_t bar_empty = bar_full + 8 * Cfg::kStages;            // each CTA: its stage may be refilled
+    const uint32_t bar_sfdata = bar_empty + 8 * Cfg::kStages;          // each CTA: its scale tiles landed
+    const uint32_t bar_acc_full = bar_sfdata + 8 * Cfg::kStages;       // each CTA: accumulator ready
+    const uint32_t bar_acc_empty = bar_acc_full + 16;                  // leader: overlap drained in both CTAs
+    const uint32_t bar_drain = bar_acc_empty + 8;                      // leader: every MMA finished
+    const uint32_t bar_sf_full = bar_drain + 8;                        // leader: both CTAs' scales stored
+    const uint32_t bar_sf_empty = bar_sf_full + 8 * kSfBufs;           // each CTA: scale buffer free
     uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(bars + Cfg::kNumBars);
     volatile uint32_t *abort_flag = tmem_holder + 1;
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
+    const uint32_t rank = cluster_ctarank();      // 0 = leader (issues the pair's MMAs)
+    const bool leader = rank == 0;
 
     if (threadIdx.x == 0) {
-        for (int s = 0; s < Cfg::kStages; ++s) {
-            mbar_init(bar_full + 8 * s, 1);
-            mbar_init(bar_empty + 8 * s, 1 + Cfg::kScaleWarps);   // MMA commit + scale warps done reading
+        for (int st = 0; st < Cfg::kStages; ++st) {
+            mbar_init(bar_full + 8 * st, 1);                             // leader's expect_tx (both CTAs' bytes)
+            mbar_init(bar_empty + 8 * st, 1 + Cfg::kScaleWarps);        // MMA commit + scale warps
+            mbar_init(bar_sfdata + 8 * st, 1);
         }
         mbar_init(bar_acc_full, 1);
         mbar_init(bar_acc_full + 8, 1);
-        mbar_init(bar_acc_empty, kEpiWarps);
+        mbar_init(bar_acc_empty, 2 * kEpiWarps);
         mbar_init(bar_drain, 1);
-        if (FP4) {
-            for (uint32_t r = 0; r < kSfBufs; ++r) {
-                mbar_init(bar_sf_full + 8 * r, Cfg::kScaleWarps);
-                mbar_init(bar_sf_empty + 8 * r, 1);
-            }
+        for (uint32_t b = 0; b < kSfBufs; ++b) {
+            mbar_init(bar_sf_full + 8 * b, 2 * Cfg::kScaleWarps);
+            mbar_init(bar_sf_empty + 8 * b, 1);
         }
         *abort_flag = 0u;
         fence_mbar_init();
     }
     if (warp == 5) {
-        tmem_alloc(smem_u32(tmem_holder), kTmemCols);
-        tmem_relinquish();
+        tmem_alloc2(smem_u32(tmem_holder), kTmemCols);
+        tmem_relinquish2();
     }
     if (warp == 4 && lane == 0) {
         prefetch_tmap(&tmA);
@@ -172,62 +185,72 @@ __global__ void __launch_bounds__(GemmCfg<FP4>::kThreads, 1)
         prefetch_tmap(&tmY);
     }
     tc_fence_before();
-    __syncthreads();
+    cluster_sync();                               // barriers of both CTAs initialised, TMEM allocated
     tc_fence_after();
     const uint32_t tmem_base = *tmem_holder;
 
     const int m_tiles = (args.M + BM - 1) / BM;
     const int n_tiles = (args.N + BN - 1) / BN;
     const int tiles = m_tiles * n_tiles;
+    const int cluster_id = blockIdx.x >> 1;
+    const int clusters = gridDim.x >> 1;
     const int k_stages = args.K / Cfg::kKPerStage;
     const int lora_stages = args.lora ? 1 : 0;                // [t_hi | t_lo] x [U | U]
     const int stages_per_tile = k_stages + lora_stages;
     const int sf_chunks_per_row_tile = args.K / 64;          // 512-byte chunks per 128-row tile
+    const int m_rows_pad = (args.M + 127) / 128 * 128;
 
     if (warp == 4) {
-        // ------------------------------------------------------------ producer
+        // ------------------------------------------------------------ producer (both CTAs)
         if (lane == 0) {
             int stage = 0;
             uint32_t phase = 0;
             bool ok = true;
-            for (int tile = blockIdx.x; tile < tiles && ok; tile += gridDim.x) {
+            for (int tile = cluster_id; tile < tiles && ok; tile += clusters) {
                 const int mt = tile % m_tiles, nt = tile / m_tiles;
-                const int m0 = mt * BM, n0 = nt * BN;
-                const bool sfb_hi = (n0 + 128) < args.N;
+                const int m0 = mt * BM + (int)rank * kRowsPerCta;         // this CTA's rows of A / y
+                const int nh = nt * BN + (int)rank * 128;                 // this CTA's half of B
+                const bool sfa_ok = m0 < m_rows_pad;
+                const bool sfb_hi = (nt * BN + 128) < args.N;
                 for (int ks = 0; ks < stages_per_tile; ++ks) {
                     if (!mbar_wait(bar_empty + 8 * stage, phase ^ 1u, abort_flag, args.status)) {
                         ok = false;
                         break;
                     }
                     uint8_t *sbase = smem + stage * Cfg::kStageBytes;
-                    const uint32_t fb = bar_full + 8 * stage;
+                    const uint32_t fb = bar_full + 8 * stage;            // counted on the leader's copy
                     const uint32_t sA = smem_u32(sbase), sB = smem_u32(sbase + kABytes);
+                    const uint32_t sd = bar_sfdata + 8 * stage;
+                    if (leader)
+                        mbar_arrive_expect_tx(fb, 2 * (kABytes + kBBytes));
                     if (ks < lora_stages) {
-                        mbar_arrive_expect_tx(fb, kABytes + kBBytes);
-                        tma_load_2d(sA, &tmT, 0, m0, fb);
-                        tma_load_2d(sB, &tmU, 0, n0, fb);
+                        tma_load_2d_pair(sA, &tmT, 0, m0, fb);
+                        tma_load_2d_pair(sB, &tmU, 0, nh, fb);
+                        if (FP4)
+                            mbar_arrive(sd);                              // keeps the scale warps in step
                     } else {
                         const int kk = ks - lora_stages;
                         if (FP4) {
-                            const uint32_t bytes = kABytes + kBBytes + kSfaBytes + (sfb_hi ? kSfbBytes : kSfaBytes);
-                            mbar_arrive_expect_tx(fb, bytes);
-                            tma_load_2d(sA, &tmA, kk * kRowBytes, m0, fb);
-                            tma_load_2d(sB, &tmB, kk * kRowBytes, n0, fb);
+                            tma_load_2d_pair(sA, &tmA, kk * kRowBytes, m0, fb);
+                            tma_load_2d_pair(sB, &tmB, kk * kRowBytes, nh, fb);
                             const uint32_t sSfa = smem_u32(sbase + kABytes + kBBytes);
                             const uint32_t sSfb = sSfa + kSfaBytes;
                             const int64_t chunk = (int64_t)kk * kMmaPerStage;
-                            bulk_load(sSfa, args.sfa + ((int64_t)mt * sf_chunks_per_row_tile + chunk) * 512,
-                                      kSfaBytes, fb);
+                            const uint32_t sf_bytes = (sfa_ok ? kSfaBytes : 0) + (sfb_hi ? kSfbBytes : kSfaBytes);
+                            mbar_arrive_expect_tx(sd, sf_bytes);
+                            if (sfa_ok)
+                                bulk_load(sSfa,
+                                          args.sfa + ((int64_t)(m0 / 128) * sf_chunks_per_row_tile + chunk) * 512,
+                                          kSfaBytes, sd);
                             bulk_load(sSfb, args.sfb + ((int64_t)(2 * nt) * sf_chunks_per_row_tile + chunk) * 512,
-                                      kSfaBytes, fb);
+                                      kSfaBytes, sd);
                             if (sfb_hi)
                                 bulk_load(sSfb + kSfaBytes,
                                           args.sfb + ((int64_t)(2 * nt + 1) * sf_chunks_per_row_tile + chunk) * 512,
-                                          kSfaBytes, fb);
+                                          kSfaBytes, sd);
                         } else {
-                            mbar_arrive_expect_tx(fb, kABytes + kBBytes);
-                            tma_load_2d(sA, &tmA, kk * 64, m0, fb);
-                            tma_load_2d(sB, &tmB, kk * 64, n0, fb);
+                            tma_load_2d_pair(sA, &tmA, kk * 64, m0, fb);
+                            tma_load_2d_pair(sB, &tmB, kk * 64, nh, fb);
                         }
                     }
                     if (++stage == Cfg::kStages) {
@@ -237,7 +260,7 @@ __global__ void __launch_bounds__(GemmCfg<FP4>::kThreads, 1)
                 }
             }
             // let every load that was issued land (and be consumed) before the CTA exits
-            for (int s = 0; s < Cfg::kStages; ++s) {
+            for (int st = 0; st < Cfg::kStages; ++st) {
                 (void)mbar_wait(bar_empty + 8 * stage, phase ^ 1u, abort_flag, args.status);
                 if (++stage == Cfg::kStages) {
                     stage = 0;
@@ -247,20 +270,21 @@ __global__ void __launch_bounds__(GemmCfg<FP4>::kThreads, 1)
         }
         __syncwarp();
     } else if (warp == 5) {
-        // ------------------------------------------------------------ MMA issuer
-        if (lane == 0) {
+        // ------------------------------------------------------------ MMA issuer (leader)
+        if (leader && lane == 0) {
             int stage = 0;
             uint32_t phase = 0;
             int count = 0;
             uint32_t sfbuf = 0, sfphase = 0;
             bool ok = true;
-            for (int tile = blockIdx.x; tile < tiles && ok; tile += gridDim.x, ++count) {
+            for (int tile = cluster_id; tile < tiles && ok; tile += clusters, ++count) {
                 const uint32_t acc = tmem_base + ((count & 1) ? kAccSlot1 : 0u);
-                if (count > 0 && !mbar_wait(bar_acc_empty, (uint32_t)((count - 1) & 1), abort_flag, args.status))
+                if (count > 0 &&
+                    !mbar_wait_cluster(bar_acc_empty, (uint32_t)((count - 1) & 1), abort_flag, args.status))
                     break;
                 tc_fence_after();
                 for (int ks = 0; ks < stages_per_tile && ok; ++ks) {
-                    if (!mbar_wait(bar_full + 8 * stage, phase, abort_flag, args.status)) {
+                    if (!mbar_wait_cluster(bar_full + 8 * stage, phase, abort_flag, args.status)) {
                         ok = false;
                         break;
                     }
@@ -270,61 +294,68 @@ __global__ void __launch_bounds__(GemmCfg<FP4>::kThreads, 1)
                     if (ks < lora_stages) {
 #pragma unroll
                         for (int k = 0; k < kMmaPerStage; ++k)
-                            mma_bf16(acc, sdesc_sw128(sA + 32 * k), sdesc_sw128(sB + 32 * k), kIdescBf16,
-                                     k > 0 ? 1u : 0u);
+                            mma2_bf16(acc, sdesc_sw128(sA + 32 * k), sdesc_sw128(sB + 32 * k), kIdescBf16,
+                                      k > 0 ? 1u : 0u);
                     } else if (FP4) {
-                        // this stage's scale factors were put in tensor-memory buffer `sfb` by the
-                        // scale warps; the buffer is handed back when these MMAs complete
-                        if (!mbar_wait(bar_sf_full + 8 * sfbuf, sfphase, abort_flag, args.status)) {
-                            ok = false;
-                            break;
-                        }
-                        tc_fence_after();
-                        const uint32_t sf = tmem_base + kSfCol + kSfBufCols * sfbuf;
+                        // the scale factors of each pair of MMAs sit in the next tensor-memory
+                        // buffer of the ring, in both CTAs
+                        for (int h = 0; h < kMmaPerStage / kMmaPerSfBuf; ++h) {
+                            if (!mbar_wait_cluster(bar_sf_full + 8 * sfbuf, sfphase, abort_flag, args.status)) {
+                                ok = false;
+                                break;
+                            }
+                            tc_fence_after();
+                            const uint32_t sf = tmem_base + kSfCol + kSfBufCols * sfbuf;
 #pragma unroll
-                        for (int k = 0; k < kMmaPerStage; ++k)
-                            mma_nvfp4(acc, sdesc_sw128(sA + 32 * k), sdesc_sw128(sB + 32 * k), kIdescNvfp4,
-                                      sf + 32 + 4 * k, sf + 8 * k, (ks > 0 || k > 0) ? 1u : 0u);
-                        tc_commit(bar_sf_empty + 8 * sfbuf);
-                        if (++sfbuf == kSfBufs) {
-                            sfbuf = 0;
-                            sfphase ^= 1u;
+                            for (int kk = 0; kk < kMmaPerSfBuf; ++kk) {
+                                const int k = kMmaPerSfBuf * h + kk;
+                                mma2_nvfp4(acc, sdesc_sw128(sA + 32 * k), sdesc_sw128(sB + 32 * k), kIdescNvfp4,
+                                           sf + 16 + 4 * kk, sf + 8 * kk, (ks > 0 || k > 0) ? 1u : 0u);
+                            }
+                            tc_commit2_both(bar_sf_empty + 8 * sfbuf);
+                            if (++sfbuf == kSfBufs) {
+                                sfbuf = 0;
+                                sfphase ^= 1u;
+                            }
                         }
+                        if (!ok)
+                            break;
                     } else {
 #pragma unroll
                         for (int k = 0; k < kMmaPerStage; ++k)
-                            mma_bf16(acc, sdesc_sw128(sA + 32 * k), sdesc_sw128(sB + 32 * k), kIdescBf16,
-                                     (ks > 0 || k > 0) ? 1u : 0u);
+                            mma2_bf16(acc, sdesc_sw128(sA + 32 * k), sdesc_sw128(sB + 32 * k), kIdescBf16,
+                                      (ks > 0 || k > 0) ? 1u : 0u);
                     }
-                    tc_commit(bar_empty + 8 * stage);
+                    tc_commit2_both(bar_empty + 8 * stage);
                     if (++stage == Cfg::kStages) {
                         stage = 0;
                         phase ^= 1u;
                     }
                 }
                 if (ok)
-                    tc_commit(bar_acc_full + 8 * (count & 1));
+                    tc_commit2_both(bar_acc_full + 8 * (count & 1));
             }
             // all issued MMAs must finish before tensor memory is released
-            tc_commit(bar_drain);
+            tc_commit2_local(bar_drain);
             (void)mbar_wait(bar_drain, 0, abort_flag, args.status);
         }
         __syncwarp();
     } else if (warp >= 6) {
-        // ------------------------------------------------------------ scale warps (NVFP4)
-        // Warp w owns tensor-memory lanes 32*(w%4)..+31.  For each stage it copies
-        // line `lane` of the four SFA chunks (rows 32*j + lane, j = 0..3) into 4
-        // columns per MMA, and line `lane` of the eight SFB chunks (rows
-        // 128*h + 32*j + lane) into 8 columns per MMA -- the layout that
-        // tcgen05.cp .32x128b.warpx4 produces -- with one store round per stage.
+        // ------------------------------------------------------------ scale warps (NVFP4, both CTAs)
+        // Warp w owns tensor-memory lanes 32*(w%4)..+31 of its CTA.  For each stage it
+        // copies line `lane` of the four SFA chunks (this CTA's rows 32*j + lane) into 4
+        // columns per MMA, and line `lane` of the eight SFB chunks (rows 128*h + 32*j +
+        // lane) into 8 columns per MMA -- the layout tcgen05.cp .32x128b.warpx4 would
+        // produce -- with one store round per stage, then tells the leader.
         const uint32_t lane_base = (uint32_t)(32 * (warp & 3)) << 16;
+        const uint32_t sf_full_leader = mapa_shared(bar_sf_full, 0);
         int stage = 0;
         uint32_t phase = 0;
         uint32_t sfbuf = 0, sfphase = 0;
         bool ok = true;
-        for (int tile = blockIdx.x; tile < tiles && ok; tile += gridDim.x) {
+        for (int tile = cluster_id; tile < tiles && ok; tile += clusters) {
             for (int ks = 0; ks < stages_per_tile && ok; ++ks) {
-                if (!warp_wait(bar_full + 8 * stage, phase, abort_flag, args.status, lane)) {
+                if (!warp_wait(bar_sfdata + 8 * stage, phase, abort_flag, args.status, lane)) {
                     ok = false;
                     break;
                 }
@@ -344,28 +375,32 @@ __global__ void __launch_bounds__(GemmCfg<FP4>::kThreads, 1)
                 if (lane == 0)
                     mbar_arrive(bar_empty + 8 * stage);
                 if (scaled) {
-                    if (!warp_wait(bar_sf_empty + 8 * sfbuf, sfphase ^ 1u, abort_flag, args.status, lane)) {
-                        ok = false;
-                        break;
-                    }
-                    tc_fence_after();
-                    const uint32_t sf = tmem_base + lane_base + kSfCol + kSfBufCols * sfbuf;
 #pragma unroll
-                    for (int k = 0; k < kMmaPerStage; ++k) {
-                        const uint32_t a4[4] = {sfa[k].x, sfa[k].y, sfa[k].z, sfa[k].w};
-                        const uint32_t b8[8] = {sfb0[k].x, sfb0[k].y, sfb0[k].z, sfb0[k].w,
-                                                sfb1[k].x, sfb1[k].y, sfb1[k].z, sfb1[k].w};
-                        tmem_st_8cols(sf + 8 * k, b8);
-                        tmem_st_4cols(sf + 32 + 4 * k, a4);
-                    }
-                    tmem_wait_st();
-                    tc_fence_before();
-                    __syncwarp();
-                    if (lane == 0)
-                        mbar_arrive(bar_sf_full + 8 * sfbuf);
-                    if (++sfbuf == kSfBufs) {
-                        sfbuf = 0;
-                        sfphase ^= 1u;
+                    for (int h = 0; h < kMmaPerStage / kMmaPerSfBuf; ++h) {
+                        if (!warp_wait(bar_sf_empty + 8 * sfbuf, sfphase ^ 1u, abort_flag, args.status, lane)) {
+                            ok = false;
+                            break;
+                        }
+                        tc_fence_after();
+                        const uint32_t sf = tmem_base + lane_base + kSfCol + kSfBufCols * sfbuf;
+#pragma unroll
+                        for (int kk = 0; kk < kMmaPerSfBuf; ++kk) {
+                            const int k = kMmaPerSfBuf * h + kk;
+                            const uint32_t a4[4] = {sfa[k].x, sfa[k].y, sfa[k].z, sfa[k].w};
+                            const uint32_t b8[8] = {sfb0[k].x, sfb0[k].y, sfb0[k].z, sfb0[k].w,
+                                                    sfb1[k].x, sfb1[k].y, sfb1[k].z, sfb1[k].w};
+                            tmem_st_8cols(sf + 8 * kk, b8);
+                            tmem_st_4cols(sf + 16 + 4 * kk, a4);
+                        }
+                        tmem_wait_st();
+                        tc_fence_before();
+                        __syncwarp();
+                        if (lane == 0)
+                            mbar_arrive_cluster(sf_full_leader + 8 * sfbuf);
+                        if (++sfbuf == kSfBufs) {
+                            sfbuf = 0;
+                            sfphase ^= 1u;
+                        }
                     }
                 }
                 if (++stage == Cfg::kStages) {
@@ -375,25 +410,28 @@ __global__ void __launch_bounds__(GemmCfg<FP4>::kThreads, 1)
             }
         }
     } else {
-        // ------------------------------------------------------------ epilogue
+        // ------------------------------------------------------------ epilogue (both CTAs)
         float beta = 1.0f;
         if (FP4) {
             const float b = __fmul_rn(*args.g_x, *args.g_w);
             beta = b == 0.0f ? 1.0f : b;
         }
+        const uint32_t acc_empty_leader = mapa_shared(bar_acc_empty, 0);
         uint8_t *staging = smem + Cfg::kStagingOff + warp * 2 * kStagingBytes;
         int sb = 0;
         int count = 0;
-        for (int tile = blockIdx.x; tile < tiles; tile += gridDim.x, ++count) {
+        for (int tile = cluster_id; tile < tiles; tile += clusters, ++count) {
             const int mt = tile % m_tiles, nt = tile / m_tiles;
-            const int m0 = mt * BM, n0 = nt * BN;
+            const int m0 = mt * BM + (int)rank * kRowsPerCta;
+            const int n0 = nt * BN;
             const int slot = count & 1;
             if (!warp_wait(bar_acc_full + 8 * slot, (uint32_t)((count >> 1) & 1), abort_flag, args.status, lane))
                 break;
             tc_fence_after();
             const uint32_t acc = tmem_base + ((uint32_t)(32 * warp) << 16) + (slot ? kAccSlot1 : 0u);
+            const bool rows_live = m0 + 32 * warp < args.M;       // skip stores wholly below the matrix
             // the chunks this slot shares with the other one are read first, in one
-            // batch, so the MMA thread can start the next tile as early as possible
+            // batch, so the leader can start the next tile as early as possible
             const int first = slot ? 0 : 8 - kOverlapChunks;
             uint32_t r[kOverlapChunks][32];
 #pragma unroll
@@ -403,11 +441,13 @@ __global__ void __launch_bounds__(GemmCfg<FP4>::kThreads, 1)
             tc_fence_before();
             __syncwarp();
             if (lane == 0)
-                mbar_arrive(bar_acc_empty);
+                mbar_arrive_cluster(acc_empty_leader);
+            if (rows_live) {
 #pragma unroll
-            for (int q = 0; q < kOverlapChunks; ++q) {
-                store_chunk(r[q], beta, staging, sb, lane, &tmY, n0 + 32 * (first + q), m0 + 32 * warp);
-                sb ^= 1;
+                for (int q = 0; q < kOverlapChunks; ++q) {
+                    store_chunk(r[q], beta, staging, sb, lane, &tmY, n0 + 32 * (first + q), m0 + 32 * warp);
+                    sb ^= 1;
+                }
             }
 #pragma unroll 1
             for (int q = kOverlapChunks; q < 8; ++q) {
@@ -415,8 +455,10 @@ __global__ void __launch_bounds__(GemmCfg<FP4>::kThreads, 1)
                 uint32_t rr[32];
                 tmem_ld_32cols(acc + 32 * c, rr);
                 tmem_wait_ld();
-                store_chunk(rr, beta, staging, sb, lane, &tmY, n0 + 32 * c, m0 + 32 * warp);
-                sb ^= 1;
+                if (rows_live) {
+                    store_chunk(rr, beta, staging, sb, lane, &tmY, n0 + 32 * c, m0 + 32 * warp);
+                    sb ^= 1;
+                }
             }
         }
         if (lane == 0)
@@ -425,10 +467,10 @@ __global__ void __launch_bounds__(GemmCfg<FP4>::kThreads, 1)
     }
 
     tc_fence_before();
-    __syncthreads();
+    cluster_sync();                               // no CTA leaves while its peer may still signal it
     tc_fence_after();
     if (warp == 5)
-        tmem_dealloc(tmem_base, kTmemCols);
+        tmem_dealloc2(tmem_base, kTmemCols);
 }
 
 // ---------------------------------------------------------------------------
@@ -474,22 +516,22 @@ cudaError_t launch_gemm(const GemmLaunch &g, int sms, cudaStream_t stream)
     const bool fp4 = g.fp4 != 0;
     bool ok = true;
     if (fp4) {
-        ok &= make_tmap(&tA, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, g.a, (uint64_t)g.K / 2, (uint64_t)g.M, 128, BM,
+        ok &= make_tmap(&tA, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, g.a, (uint64_t)g.K / 2, (uint64_t)g.M, 128, 128,
                         CU_TENSOR_MAP_SWIZZLE_128B);
-        ok &= make_tmap(&tB, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, g.b, (uint64_t)g.K / 2, (uint64_t)g.N, 128, BN,
+        ok &= make_tmap(&tB, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, g.b, (uint64_t)g.K / 2, (uint64_t)g.N, 128, 128,
                         CU_TENSOR_MAP_SWIZZLE_128B);
     } else {
-        ok &= make_tmap(&tA, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, g.a, (uint64_t)g.K, (uint64_t)g.M, 64, BM,
+        ok &= make_tmap(&tA, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, g.a, (uint64_t)g.K, (uint64_t)g.M, 64, 128,
                         CU_TENSOR_MAP_SWIZZLE_128B);
-        ok &= make_tmap(&tB, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, g.b, (uint64_t)g.K, (uint64_t)g.N, 64, BN,
+        ok &= make_tmap(&tB, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, g.b, (uint64_t)g.K, (uint64_t)g.N, 64, 128,
                         CU_TENSOR_MAP_SWIZZLE_128B);
     }
     const bool lora = g.tsplit && g.udup;
     // without a low-rank step the maps below are never used; point them at A/B
     ok &= make_tmap(&tT, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, lora ? (const void *)g.tsplit : g.a, 64,
-                    (uint64_t)g.M, 64, BM, CU_TENSOR_MAP_SWIZZLE_128B);
+                    (uint64_t)g.M, 64, 128, CU_TENSOR_MAP_SWIZZLE_128B);
     ok &= make_tmap(&tU, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, lora ? (const void *)g.udup : g.b, 64,
-                    (uint64_t)g.N, 64, BN, CU_TENSOR_MAP_SWIZZLE_128B);
+                    (uint64_t)g.N, 64, 128, CU_TENSOR_MAP_SWIZZLE_128B);
     ok &= make_tmap(&tY, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, g.y, (uint64_t)g.N, (uint64_t)g.M, 32, 32,
                     CU_TENSOR_MAP_SWIZZLE_128B);
     if (!ok)
@@ -505,7 +547,28 @@ cudaError_t launch_gemm(const GemmLaunch &g, int sms, cudaStream_t stream)
     a.K = (int)g.K;
     a.lora = lora ? 1 : 0;
     const int tiles = (int)(((g.M + BM - 1) / BM) * ((g.N + BN - 1) / BN));
-    const int grid = tiles < sms ? tiles : sms;
+    // persistent grid: as many CTA pairs as can be resident at once (not every SM
+    // can pair up inside its GPC), each walking the tile list
+    int pairs = sms / 2;
+    {
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = dim3(2 * pairs);
+        cfg.blockDim = dim3(fp4 ? GemmCfg<true>::kThreads : GemmCfg<false>::kThreads);
+        cfg.dynamicSmemBytes = fp4 ? GemmCfg<true>::kSmemBytes : GemmCfg<false>::kSmemBytes;
+        int resident = 0;
+        cudaError_t e = fp4 ? cudaFuncSetAttribute(sq_gemm_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                                   GemmCfg<true>::kSmemBytes)
+                            : cudaFuncSetAttribute(sq_gemm_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                                   GemmCfg<false>::kSmemBytes);
+        if (e != cudaSuccess)
+            return e;
+        e = fp4 ? cudaOccupancyMaxActiveClusters(&resident, sq_gemm_kernel<true>, &cfg)
+                : cudaOccupancyMaxActiveClusters(&resident, sq_gemm_kernel<false>, &cfg);
+        if (e == cudaSuccess && resident > 0 && resident < pairs)
+            pairs = resident;
+        (void)cudaGetLastError();
+    }
+    const int grid = 2 * (tiles < pairs ? tiles : pairs);        // clusters of two CTAs
     if (fp4) {
         const int smem = GemmCfg<true>::kSmemBytes;
         cudaError_t e = cudaFuncSetAttribute(sq_gemm_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
