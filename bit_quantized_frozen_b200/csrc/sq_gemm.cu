@@ -22,11 +22,11 @@
 //   warps 6-9  (NVFP4) move each MMA's ue4m3 scale factors from shared memory
 //              into tensor memory with tcgen05.st, one 32-lane sub-partition
 //              per warp, so the tensor pipe spends no cycles on copies.
-// Tensor memory (512 columns): two accumulator slots at columns 0 and 128
-// that overlap in columns 128..255, and two 48-column scale-factor buffers at
-// 384..479 (NVFP4).  The epilogue reads the overlapping 128 columns of a tile
+// Tensor memory (512 columns): two accumulator slots at columns 0 and 96
+// that overlap in columns 96..255, and three 48-column scale-factor buffers at
+// 352..495 (NVFP4).  The epilogue reads the overlapping 160 columns of a tile
 // first and then releases the MMA thread, which starts the next tile while
-// the other 128 columns drain -- accumulator double buffering in 384 columns.
+// the other 96 columns drain -- accumulator double buffering in 352 columns.
 #include <cuda.h>
 
 #include "sq_device.cuh"
@@ -47,12 +47,12 @@ constexpr int kSfbBytes = 2 * kSfaBytes;       // both 128-row halves of B (ever
 constexpr int kEpiWarps = 4;
 constexpr int kStagingBytes = 32 * 128;        // one warp's 32 rows x 32 fp32
 constexpr uint32_t kTmemCols = 512;
-constexpr uint32_t kAccSlot1 = 128;            // accumulator slots [0, 256) and [128, 384)
-constexpr int kOverlapChunks = 4;              // 32-column chunks shared by the two slots
-constexpr uint32_t kSfCol = 384;               // ring of five scale-factor buffers, two MMAs each
-constexpr int kMmaPerSfBuf = 2;
-constexpr uint32_t kSfBufCols = 24;            // SFB for MMA k at +8k (256 rows), SFA at +16+4k (128 rows)
-constexpr uint32_t kSfBufs = 5;
+constexpr uint32_t kAccSlot1 = 96;             // accumulator slots [0, 256) and [96, 352)
+constexpr int kOverlapChunks = 5;              // 32-column chunks shared by the two slots
+constexpr uint32_t kSfCol = 352;               // ring of three scale-factor buffers, one stage (4 MMAs) each
+constexpr int kMmaPerSfBuf = 4;
+constexpr uint32_t kSfBufCols = 48;            // SFB for MMA k at +8k (256 rows), SFA at +32+4k (128 rows)
+constexpr uint32_t kSfBufs = 3;
 
 // instruction descriptors: M = 256 (the CTA pair), N = 256, K-major A and B
 constexpr uint32_t kIdescBf16 = (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(BN >> 3) << 17) |
@@ -69,8 +69,8 @@ struct GemmCfg {
     static constexpr int kKPerStage = FP4 ? 256 : 64;            // K values per stage
     static constexpr int kStagingOff = kStages * kStageBytes;
     static constexpr int kBarOff = kStagingOff + kEpiWarps * 2 * kStagingBytes;
-    // full[s], empty[s], sfdata[s], acc_full[2], acc_empty, drain, sf_full[b], sf_empty[b]
-    static constexpr int kNumBars = 3 * kStages + 4 + 2 * kSfBufs;
+    // full[s], empty[s], sfdata[s], acc_full[2], acc_empty, drain
+    static constexpr int kNumBars = 3 * kStages + 4;
     static constexpr int kSmemBytes = kBarOff + 8 * kNumBars + 16 + 1024;   // + holder, flag, alignment
 };
 
@@ -140,14 +140,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(GemmCfg<FP4>::kThrea
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint64_t *bars = reinterpret_cast<uint64_t *>(smem + Cfg::kBarOff);
-    const uint32_t bar_full = smem_u32(bars);                          // leader: A/B of both CTAs landed
+    const uint32_t bar_full = smem_u32(bars);                          // leader: both CTAs' stage ready
     const uint32_t bar_empty = bar_full + 8 * Cfg::kStages;            // each CTA: its stage may be refilled
     const uint32_t bar_sfdata = bar_empty + 8 * Cfg::kStages;          // each CTA: its scale tiles landed
     const uint32_t bar_acc_full = bar_sfdata + 8 * Cfg::kStages;       // each CTA: accumulator ready
     const uint32_t bar_acc_empty = bar_acc_full + 16;                  // leader: overlap drained in both CTAs
     const uint32_t bar_drain = bar_acc_empty + 8;                      // leader: every MMA finished
-    const uint32_t bar_sf_full = bar_drain + 8;                        // leader: both CTAs' scales stored
-    const uint32_t bar_sf_empty = bar_sf_full + 8 * kSfBufs;           // each CTA: scale buffer free
     uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(bars + Cfg::kNumBars);
     volatile uint32_t *abort_flag = tmem_holder + 1;
 
@@ -158,7 +156,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(GemmCfg<FP4>::kThrea
 
     if (threadIdx.x == 0) {
         for (int st = 0; st < Cfg::kStages; ++st) {
-            mbar_init(bar_full + 8 * st, 1);                             // leader's expect_tx (both CTAs' bytes)
+            // leader's expect_tx (both CTAs' bytes) + every scale warp of both CTAs
+            mbar_init(bar_full + 8 * st, 1 + 2 * Cfg::kScaleWarps);
             mbar_init(bar_empty + 8 * st, 1 + Cfg::kScaleWarps);        // MMA commit + scale warps
             mbar_init(bar_sfdata + 8 * st, 1);
         }
@@ -166,10 +165,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(GemmCfg<FP4>::kThrea
         mbar_init(bar_acc_full + 8, 1);
         mbar_init(bar_acc_empty, 2 * kEpiWarps);
         mbar_init(bar_drain, 1);
-        for (uint32_t b = 0; b < kSfBufs; ++b) {
-            mbar_init(bar_sf_full + 8 * b, 2 * Cfg::kScaleWarps);
-            mbar_init(bar_sf_empty + 8 * b, 1);
-        }
         *abort_flag = 0u;
         fence_mbar_init();
     }
@@ -271,65 +266,62 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(GemmCfg<FP4>::kThrea
         __syncwarp();
     } else if (warp == 5) {
         // ------------------------------------------------------------ MMA issuer (leader)
+        // One thread issues every MMA of the pair, so its per-stage work is kept to a
+        // few adds: shared-memory descriptors are built once and advanced by the
+        // stage offset (the start-address field holds address / 16).
         if (leader && lane == 0) {
+            const uint32_t s0 = smem_u32(smem);
+            const uint64_t dA0 = sdesc_sw128(s0);                      // stage 0, A, k = 0
+            const uint64_t dB0 = sdesc_sw128(s0 + kABytes);
+            constexpr uint32_t kStage16 = Cfg::kStageBytes >> 4;
             int stage = 0;
+            uint32_t off16 = 0;
             uint32_t phase = 0;
             int count = 0;
-            uint32_t sfbuf = 0, sfphase = 0;
+            uint32_t sfbuf = 0;
+            uint32_t sf = tmem_base + kSfCol;
             bool ok = true;
             for (int tile = cluster_id; tile < tiles && ok; tile += clusters, ++count) {
                 const uint32_t acc = tmem_base + ((count & 1) ? kAccSlot1 : 0u);
                 if (count > 0 &&
                     !mbar_wait_cluster(bar_acc_empty, (uint32_t)((count - 1) & 1), abort_flag, args.status))
                     break;
-                tc_fence_after();
-                for (int ks = 0; ks < stages_per_tile && ok; ++ks) {
+                for (int ks = 0; ks < stages_per_tile; ++ks) {
                     if (!mbar_wait_cluster(bar_full + 8 * stage, phase, abort_flag, args.status)) {
                         ok = false;
                         break;
                     }
                     tc_fence_after();
-                    uint8_t *sbase = smem + stage * Cfg::kStageBytes;
-                    const uint32_t sA = smem_u32(sbase), sB = smem_u32(sbase + kABytes);
+                    const uint64_t a = dA0 + off16, b = dB0 + off16;
                     if (ks < lora_stages) {
 #pragma unroll
                         for (int k = 0; k < kMmaPerStage; ++k)
-                            mma2_bf16(acc, sdesc_sw128(sA + 32 * k), sdesc_sw128(sB + 32 * k), kIdescBf16,
-                                      k > 0 ? 1u : 0u);
+                            mma2_bf16(acc, a + 2 * k, b + 2 * k, kIdescBf16, k > 0 ? 1u : 0u);
                     } else if (FP4) {
-                        // the scale factors of each pair of MMAs sit in the next tensor-memory
-                        // buffer of the ring, in both CTAs
-                        for (int h = 0; h < kMmaPerStage / kMmaPerSfBuf; ++h) {
-                            if (!mbar_wait_cluster(bar_sf_full + 8 * sfbuf, sfphase, abort_flag, args.status)) {
-                                ok = false;
-                                break;
-                            }
-                            tc_fence_after();
-                            const uint32_t sf = tmem_base + kSfCol + kSfBufCols * sfbuf;
+                        // the scale factors of stage g sit in tensor-memory buffer g % 3 of both
+                        // CTAs; full[] above already counted the scale warps that stored them
 #pragma unroll
-                            for (int kk = 0; kk < kMmaPerSfBuf; ++kk) {
-                                const int k = kMmaPerSfBuf * h + kk;
-                                mma2_nvfp4(acc, sdesc_sw128(sA + 32 * k), sdesc_sw128(sB + 32 * k), kIdescNvfp4,
-                                           sf + 16 + 4 * kk, sf + 8 * kk, (ks > 0 || k > 0) ? 1u : 0u);
-                            }
-                            tc_commit2_both(bar_sf_empty + 8 * sfbuf);
-                            if (++sfbuf == kSfBufs) {
-                                sfbuf = 0;
-                                sfphase ^= 1u;
-                            }
-                        }
-                        if (!ok)
-                            break;
+                        for (int k = 0; k < kMmaPerStage; ++k)
+                            mma2_nvfp4(acc, a + 2 * k, b + 2 * k, kIdescNvfp4, sf + 32 + 4 * k, sf + 8 * k,
+                                       (ks > 0 || k > 0) ? 1u : 0u);
                     } else {
 #pragma unroll
                         for (int k = 0; k < kMmaPerStage; ++k)
-                            mma2_bf16(acc, sdesc_sw128(sA + 32 * k), sdesc_sw128(sB + 32 * k), kIdescBf16,
-                                      (ks > 0 || k > 0) ? 1u : 0u);
+                            mma2_bf16(acc, a + 2 * k, b + 2 * k, kIdescBf16, (ks > 0 || k > 0) ? 1u : 0u);
                     }
                     tc_commit2_both(bar_empty + 8 * stage);
                     if (++stage == Cfg::kStages) {
                         stage = 0;
+                        off16 = 0;
                         phase ^= 1u;
+                    } else {
+                        off16 += kStage16;
+                    }
+                    if (++sfbuf == kSfBufs) {             // scale buffer of the next stage
+                        sfbuf = 0;
+                        sf = tmem_base + kSfCol;
+                    } else {
+                        sf += kSfBufCols;
                     }
                 }
                 if (ok)
@@ -342,19 +334,24 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(GemmCfg<FP4>::kThrea
         __syncwarp();
     } else if (warp >= 6) {
         // ------------------------------------------------------------ scale warps (NVFP4, both CTAs)
-        // Warp w owns tensor-memory lanes 32*(w%4)..+31 of its CTA.  For each stage it
+        // Warp w owns tensor-memory lanes 32*(w%4)..+31 of its CTA.  For stage g it
         // copies line `lane` of the four SFA chunks (this CTA's rows 32*j + lane) into 4
-        // columns per MMA, and line `lane` of the eight SFB chunks (rows 128*h + 32*j +
+        // columns per MMA and line `lane` of the eight SFB chunks (rows 128*h + 32*j +
         // lane) into 8 columns per MMA -- the layout tcgen05.cp .32x128b.warpx4 would
-        // produce -- with one store round per stage, then tells the leader.
+        // produce -- in buffer g % 3, with one store round, and then arrives on the
+        // leader's full[] barrier of the stage.  Buffer g % 3 is free once the MMAs of
+        // stage g - 3 are done, i.e. once that stage's empty[] barrier completed.
         const uint32_t lane_base = (uint32_t)(32 * (warp & 3)) << 16;
-        const uint32_t sf_full_leader = mapa_shared(bar_sf_full, 0);
+        const uint32_t full_leader = mapa_shared(bar_full, 0);
         int stage = 0;
         uint32_t phase = 0;
-        uint32_t sfbuf = 0, sfphase = 0;
+        int lstage = 0;                 // ring position and phase of stage g - 3
+        uint32_t lphase = 0;
+        uint32_t sfbuf = 0;
+        int g = 0;
         bool ok = true;
         for (int tile = cluster_id; tile < tiles && ok; tile += clusters) {
-            for (int ks = 0; ks < stages_per_tile && ok; ++ks) {
+            for (int ks = 0; ks < stages_per_tile && ok; ++ks, ++g) {
                 if (!warp_wait(bar_sfdata + 8 * stage, phase, abort_flag, args.status, lane)) {
                     ok = false;
                     break;
@@ -374,35 +371,35 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(GemmCfg<FP4>::kThrea
                 __syncwarp();
                 if (lane == 0)
                     mbar_arrive(bar_empty + 8 * stage);
-                if (scaled) {
-#pragma unroll
-                    for (int h = 0; h < kMmaPerStage / kMmaPerSfBuf; ++h) {
-                        if (!warp_wait(bar_sf_empty + 8 * sfbuf, sfphase ^ 1u, abort_flag, args.status, lane)) {
-                            ok = false;
-                            break;
-                        }
-                        tc_fence_after();
-                        const uint32_t sf = tmem_base + lane_base + kSfCol + kSfBufCols * sfbuf;
-#pragma unroll
-                        for (int kk = 0; kk < kMmaPerSfBuf; ++kk) {
-                            const int k = kMmaPerSfBuf * h + kk;
-                            const uint32_t a4[4] = {sfa[k].x, sfa[k].y, sfa[k].z, sfa[k].w};
-                            const uint32_t b8[8] = {sfb0[k].x, sfb0[k].y, sfb0[k].z, sfb0[k].w,
-                                                    sfb1[k].x, sfb1[k].y, sfb1[k].z, sfb1[k].w};
-                            tmem_st_8cols(sf + 8 * kk, b8);
-                            tmem_st_4cols(sf + 16 + 4 * kk, a4);
-                        }
-                        tmem_wait_st();
-                        tc_fence_before();
-                        __syncwarp();
-                        if (lane == 0)
-                            mbar_arrive_cluster(sf_full_leader + 8 * sfbuf);
-                        if (++sfbuf == kSfBufs) {
-                            sfbuf = 0;
-                            sfphase ^= 1u;
-                        }
+                if (g >= (int)kSfBufs) {
+                    if (scaled && !warp_wait(bar_empty + 8 * lstage, lphase, abort_flag, args.status, lane)) {
+                        ok = false;
+                        break;
+                    }
+                    if (++lstage == Cfg::kStages) {
+                        lstage = 0;
+                        lphase ^= 1u;
                     }
                 }
+                if (scaled) {
+                    tc_fence_after();
+                    const uint32_t sf = tmem_base + lane_base + kSfCol + kSfBufCols * sfbuf;
+#pragma unroll
+                    for (int k = 0; k < kMmaPerStage; ++k) {
+                        const uint32_t a4[4] = {sfa[k].x, sfa[k].y, sfa[k].z, sfa[k].w};
+                        const uint32_t b8[8] = {sfb0[k].x, sfb0[k].y, sfb0[k].z, sfb0[k].w,
+                                                sfb1[k].x, sfb1[k].y, sfb1[k].z, sfb1[k].w};
+                        tmem_st_8cols(sf + 8 * k, b8);
+                        tmem_st_4cols(sf + 32 + 4 * k, a4);
+                    }
+                    tmem_wait_st();
+                    tc_fence_before();
+                }
+                __syncwarp();
+                if (lane == 0)
+                    mbar_arrive_cluster(full_leader + 8 * stage);
+                if (++sfbuf == kSfBufs)
+                    sfbuf = 0;
                 if (++stage == Cfg::kStages) {
                     stage = 0;
                     phase ^= 1u;
@@ -432,7 +429,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(GemmCfg<FP4>::kThrea
             const bool rows_live = m0 + 32 * warp < args.M;       // skip stores wholly below the matrix
             // the chunks this slot shares with the other one are read first, in one
             // batch, so the leader can start the next tile as early as possible
-            const int first = slot ? 0 : 8 - kOverlapChunks;
+            const int first = slot ? 0 : 8 - kOverlapChunks;   // slot 0 shares its last 5 chunks
             uint32_t r[kOverlapChunks][32];
 #pragma unroll
             for (int q = 0; q < kOverlapChunks; ++q)
