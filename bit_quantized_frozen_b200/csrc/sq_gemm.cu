@@ -545,11 +545,17 @@ cudaError_t launch_gemm(const GemmLaunch &g, int sms, cudaStream_t stream)
     a.lora = lora ? 1 : 0;
     const int tiles = (int)(((g.M + BM - 1) / BM) * ((g.N + BN - 1) / BN));
     // persistent grid: as many CTA pairs as can be resident at once (not every SM
-    // can pair up inside its GPC), each walking the tile list
-    int pairs = sms / 2;
-    {
+    // can pair up inside its GPC), each walking the tile list; queried once per
+    // device and kernel, together with the shared-memory opt-in
+    constexpr int kMaxDev = 64;
+    static int resident_pairs[2][kMaxDev];
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDev)
+        return cudaErrorInvalidDevice;
+    int &pairs_cached = resident_pairs[fp4 ? 1 : 0][dev];
+    if (pairs_cached == 0) {
         cudaLaunchConfig_t cfg = {};
-        cfg.gridDim = dim3(2 * pairs);
+        cfg.gridDim = dim3(2 * (sms / 2));
         cfg.blockDim = dim3(fp4 ? GemmCfg<true>::kThreads : GemmCfg<false>::kThreads);
         cfg.dynamicSmemBytes = fp4 ? GemmCfg<true>::kSmemBytes : GemmCfg<false>::kSmemBytes;
         int resident = 0;
@@ -561,24 +567,17 @@ cudaError_t launch_gemm(const GemmLaunch &g, int sms, cudaStream_t stream)
             return e;
         e = fp4 ? cudaOccupancyMaxActiveClusters(&resident, sq_gemm_kernel<true>, &cfg)
                 : cudaOccupancyMaxActiveClusters(&resident, sq_gemm_kernel<false>, &cfg);
-        if (e == cudaSuccess && resident > 0 && resident < pairs)
-            pairs = resident;
         (void)cudaGetLastError();
+        pairs_cached = (e == cudaSuccess && resident > 0 && resident < sms / 2) ? resident : sms / 2;
     }
+    const int pairs = pairs_cached;
     const int grid = 2 * (tiles < pairs ? tiles : pairs);        // clusters of two CTAs
-    if (fp4) {
-        const int smem = GemmCfg<true>::kSmemBytes;
-        cudaError_t e = cudaFuncSetAttribute(sq_gemm_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-        if (e != cudaSuccess)
-            return e;
-        sq_gemm_kernel<true><<<grid, GemmCfg<true>::kThreads, smem, stream>>>(tA, tB, tT, tU, tY, a);
-    } else {
-        const int smem = GemmCfg<false>::kSmemBytes;
-        cudaError_t e = cudaFuncSetAttribute(sq_gemm_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-        if (e != cudaSuccess)
-            return e;
-        sq_gemm_kernel<false><<<grid, GemmCfg<false>::kThreads, smem, stream>>>(tA, tB, tT, tU, tY, a);
-    }
+    if (fp4)
+        sq_gemm_kernel<true><<<grid, GemmCfg<true>::kThreads, GemmCfg<true>::kSmemBytes, stream>>>(
+            tA, tB, tT, tU, tY, a);
+    else
+        sq_gemm_kernel<false><<<grid, GemmCfg<false>::kThreads, GemmCfg<false>::kSmemBytes, stream>>>(
+            tA, tB, tT, tU, tY, a);
     return cudaGetLastError();
 }
 

@@ -714,10 +714,21 @@ static bool stream_map(CUtensorMap *tm, const T *in, int64_t rows, int64_t K)
                      32, (uint64_t)(rows * K / 32), 32, 256, f32 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B);
 }
 
+// shared-memory opt-in, once per device and kernel
 template <typename T, typename Kern>
 static cudaError_t stream_attr(Kern k)
 {
-    return cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, StreamCfg<T>::kSmem);
+    constexpr int kMaxDev = 64;
+    static bool done[kMaxDev];
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDev)
+        return cudaErrorInvalidDevice;
+    if (done[dev])
+        return cudaSuccess;
+    cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, StreamCfg<T>::kSmem);
+    if (e == cudaSuccess)
+        done[dev] = true;
+    return e;
 }
 
 static int stream_grid(int64_t blocks, int sms, int per_sm)
