@@ -375,7 +375,7 @@ sq_status sq_reconstruct_bf16(const sq_weight *w, uint16_t *W_out, uint32_t flag
     const int with_lowrank = (!(flags & SQ_RECON_RESIDUAL_ONLY) && w->lora_up && w->lora_down) ? 1 : 0;
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     SQ_CUDA(sq::launch_reconstruct(w->fmt, w->codes, w->scales, w->g_w, w->lora_up, w->lora_down, w->N, w->K,
-                                   with_lowrank, W_out, s),
+                                   with_lowrank, W_out, sms, s),
             "reconstruct");
     return SQ_OK;
 }

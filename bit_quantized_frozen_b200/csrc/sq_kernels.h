@@ -29,7 +29,7 @@ cudaError_t launch_lowrank_finish(const float *t32, int64_t M, const float *g_x,
                                   cudaStream_t s);
 cudaError_t launch_reconstruct(int fmt, const uint8_t *codes, const void *scales, const float *g_w,
                                const uint16_t *U, const uint16_t *D, int64_t N, int64_t K, int with_lowrank,
-                               uint16_t *W, cudaStream_t s);
+                               uint16_t *W, int sms, cudaStream_t s);
 
 // forward GEMM y = beta (A B^T + tsplit udup^T), see sq_gemm.cu
 struct GemmLaunch {

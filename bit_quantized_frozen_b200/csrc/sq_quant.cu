@@ -591,106 +591,261 @@ __global__ void __launch_bounds__(256) lowrank_finish_kernel(const float *__rest
 }
 
 // ---------------------------------------------------------------------------
-// bf16 reconstruct.  CTA = (256-column block kb, 128-row chunk); lora_down for
-// the block is staged transposed in shared memory as fp32, each warp walks 16
-// rows: d from the payload, H256 over the block, the rank-32 fma chain, bf16.
+// bf16 reconstruct.  Tile = one 256-column block kb x 64 rows.  Persistent
+// CTAs of 256 threads walk a contiguous range of tiles (kb-major), staging the
+// next tile's codes, scales and lora_up rows in shared memory by cp.async
+// while the current one is computed, and keeping lora_down for the current kb
+// in registers.
+// Phase 1: each lane decodes 32 payload values of a row (one int4 group, or
+//   two NVFP4 blocks), runs the 8-lane Hadamard transform and writes h into a
+//   shared fp32 tile (float4 f of a row stored at f ^ (f >> 3) -- conflict free
+//   for both phases).
+// Phase 2: thread t owns columns 2(t%128), 2(t%128)+1 and rows 32(t/128)..+31.
+//   lora_down for its two columns stays in registers; lora_up rows are
+//   broadcast from shared memory; each output's rank-32 fmaf chain runs in
+//   order r = 0..31 from 0, two columns at a time with fma.rn.f32x2 (two
+//   independent fmaf, bit-identical to the scalar chain); W = bf16(RN(L + h)).
 // ---------------------------------------------------------------------------
-constexpr int kReconRows = 128;
-constexpr int kDtPitch = 260;   // floats per staged row (16-byte aligned, fewer bank conflicts)
+constexpr int kRecRows = 64;
+constexpr int kRecCodeBytes = kRecRows * kHad / 2;        // 8 KB
+constexpr int kRecScaleBytes = kRecRows * 16;             // 1 KB (8 fp16 or 16 ue4m3 per row)
+constexpr int kRecUBytes = kRecRows * kRank * 2;          // 4 KB
+constexpr int kRecStageBytes = kRecCodeBytes + kRecScaleBytes + kRecUBytes;
+constexpr int kRecHBytes = kRecRows * kHad * 4;           // 64 KB
+constexpr int kRecUsBytes = kRecRows * kRank * 8;         // 16 KB
+constexpr int kRecSmemLowrank = kRecHBytes + kRecUsBytes + 2 * kRecStageBytes;   // 106 KB
+constexpr int kRecSmemResidual = 2 * kRecStageBytes;
 
-__global__ void __launch_bounds__(256) reconstruct_kernel(int fmt, const uint8_t *__restrict__ codes,
-                                                          const void *__restrict__ scales,
-                                                          const float *__restrict__ g_w,
-                                                          const uint16_t *__restrict__ U,
-                                                          const uint16_t *__restrict__ D, int64_t N,
-                                                          int64_t K, int with_lowrank,
-                                                          uint16_t *__restrict__ W)
+__device__ __forceinline__ uint64_t pack2(float lo, float hi)
 {
-    extern __shared__ __align__(16) float dts[];   // [32][kDtPitch]
-    const int lane = threadIdx.x & 31;
-    const int wid = threadIdx.x >> 5;
-    const int64_t kb = blockIdx.x;
-    const int64_t C = K / kSfBlock;
-    if (with_lowrank) {
-        const uint16_t *Dk = D + kb * kHad * kRank;
-        for (int i = threadIdx.x; i < kHad * kRank; i += blockDim.x)
-            dts[(i & 31) * kDtPitch + (i >> 5)] = bf16_bits_to_f32(Dk[i]);
+    uint64_t r;
+    asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+    return r;
+}
+
+__device__ __forceinline__ void unpack2(uint64_t v, float &lo, float &hi)
+{
+    asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+}
+
+// acc = fma(a, b, acc) on two fp32 lanes, each rounded once
+__device__ __forceinline__ void fma2(uint64_t &acc, uint64_t a, uint64_t b)
+{
+    asm("fma.rn.f32x2 %0, %1, %2, %0;" : "+l"(acc) : "l"(a), "l"(b));
+}
+
+__device__ __forceinline__ void cp_async4(uint32_t dst, const void *src, uint32_t src_bytes)
+{
+    asm volatile("cp.async.ca.shared.global [%0], [%1], 4, %2;" ::"r"(dst), "l"(src), "r"(src_bytes) : "memory");
+}
+
+// Stage tile (kb, rows n0..n0+63) into one buffer: codes [64][128 B], scales
+// [64][16 B] (int4: the 8 fp16 group scales; NVFP4: the 16 ue4m3 block scales,
+// gathered from the tiled layout 4 bytes at a time), lora_up [64][64 B].
+// Rows past N are zero filled.
+template <int FMT, bool LOWRANK>
+__device__ __forceinline__ void rec_stage(uint32_t buf, const uint8_t *codes, const void *scales, const uint16_t *U,
+                                          int64_t N, int64_t K, int64_t kb, int64_t n0, int tid)
+{
+#pragma unroll
+    for (int i = 0; i < 2; ++i) {
+        const int e = tid + 256 * i;
+        const int r = e >> 3, c = e & 7;
+        const int64_t n = n0 + r;
+        const uint8_t *src = n < N ? codes + n * (K / 2) + kb * (kHad / 2) + 16 * c : codes;
+        cp_async16(buf + r * 128 + 16 * c, src, n < N ? 16u : 0u);
     }
-    __syncthreads();
-    const float g = fmt == 2 ? *g_w : 0.0f;
-    const int64_t n_end_c = (int64_t)(blockIdx.y + 1) * kReconRows;
-    const int64_t n_end = N < n_end_c ? N : n_end_c;
-    for (int64_t n = (int64_t)blockIdx.y * kReconRows + wid; n < n_end; n += 8) {
-        const uint8_t *crow = codes + n * (K / 2) + kb * (kHad / 2);
-        const uint32_t c0 = *reinterpret_cast<const uint16_t *>(crow + 2 * lane);
-        const uint32_t c1 = *reinterpret_cast<const uint16_t *>(crow + 64 + 2 * lane);
-        float v[8];
-        if (fmt == 1) {
-            const uint16_t *srow = reinterpret_cast<const uint16_t *>(scales) + n * (K / kGroup) + kb * 8;
-            const float s0 = __half2float(__ushort_as_half(srow[lane >> 3]));
-            const float s1 = __half2float(__ushort_as_half(srow[4 + (lane >> 3)]));
-#pragma unroll
-            for (int i = 0; i < 4; ++i) {
-                int q0 = (int)((c0 >> (4 * i)) & 0xFu);
-                int q1 = (int)((c1 >> (4 * i)) & 0xFu);
-                q0 = q0 >= 8 ? q0 - 16 : q0;
-                q1 = q1 >= 8 ? q1 - 16 : q1;
-                v[i] = __fmul_rn((float)q0, s0);
-                v[4 + i] = __fmul_rn((float)q1, s1);
-            }
-        } else {
-            const uint8_t *sf = reinterpret_cast<const uint8_t *>(scales);
-            const int64_t cc = kb * (kHad / kSfBlock) + (lane >> 2);
-            const float d0 = ue4m3_value(sf[sf_offset(n, cc, C)]);
-            const float d1 = ue4m3_value(sf[sf_offset(n, cc + 8, C)]);
-            const float2 e00 = e2m1x2_value(c0 & 0xFFu), e01 = e2m1x2_value(c0 >> 8);
-            const float2 e10 = e2m1x2_value(c1 & 0xFFu), e11 = e2m1x2_value(c1 >> 8);
-            const float e[8] = {e00.x, e00.y, e01.x, e01.y, e10.x, e10.y, e11.x, e11.y};
-#pragma unroll
-            for (int i = 0; i < 8; ++i)
-                v[i] = __fmul_rn(__fmul_rn(e[i], i < 4 ? d0 : d1), g);
+    const uint32_t sbuf = buf + kRecCodeBytes;
+    if (FMT == 1) {
+        if (tid < kRecRows) {
+            const int64_t n = n0 + tid;
+            const uint8_t *src = n < N ? reinterpret_cast<const uint8_t *>(scales) + (n * (K / kGroup) + kb * 8) * 2
+                                       : reinterpret_cast<const uint8_t *>(scales);
+            cp_async16(sbuf + 16 * tid, src, n < N ? 16u : 0u);
         }
-        fwht256_warp(v, lane);
-        if (with_lowrank) {
-            float u[kRank];
-            const uint4 *up = reinterpret_cast<const uint4 *>(U + n * kRank);
+    } else {
+        const int r = tid >> 2, j = tid & 3;
+        const int64_t n = n0 + r;
+        const uint8_t *src = n < N ? reinterpret_cast<const uint8_t *>(scales) +
+                                         sf_offset(n, kb * (kHad / kSfBlock) + 4 * j, K / kSfBlock)
+                                   : reinterpret_cast<const uint8_t *>(scales);
+        cp_async4(sbuf + 16 * r + 4 * j, src, n < N ? 4u : 0u);
+    }
+    if (LOWRANK) {
+        const int r = tid >> 2, c = tid & 3;
+        const int64_t n = n0 + r;
+        const uint16_t *src = n < N ? U + n * kRank + 8 * c : U;
+        cp_async16(buf + kRecCodeBytes + kRecScaleBytes + r * 64 + 16 * c, src, n < N ? 16u : 0u);
+    }
+}
+
+// 32 payload values of staged row r, group q (values 32q..32q+31 of the block)
+template <int FMT>
+__device__ __forceinline__ void rec_decode(const uint8_t *stage, int r, int q, float g, float (&v)[32])
+{
+    const uint4 c = *reinterpret_cast<const uint4 *>(stage + r * 128 + 16 * q);
+    const uint32_t w[4] = {c.x, c.y, c.z, c.w};
+    const uint8_t *sc = stage + kRecCodeBytes + 16 * r;
+    if (FMT == 1) {
+        const float s = __half2float(*reinterpret_cast<const __half *>(sc + 2 * q));
 #pragma unroll
-            for (int q = 0; q < 4; ++q) {
-                const uint4 w = __ldg(up + q);
-                const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
+        for (int i = 0; i < 32; ++i) {
+            int qq = (int)((w[i >> 3] >> (4 * (i & 7))) & 0xFu);
+            qq = qq >= 8 ? qq - 16 : qq;
+            v[i] = __fmul_rn((float)qq, s);
+        }
+    } else {
+        const uint32_t sf2 = *reinterpret_cast<const uint16_t *>(sc + 2 * q);
+        const float d0 = ue4m3_value(sf2 & 0xFFu), d1 = ue4m3_value(sf2 >> 8);
 #pragma unroll
-                for (int p = 0; p < 4; ++p) {
-                    u[8 * q + 2 * p] = bf16_bits_to_f32(ww[p] & 0xFFFFu);
-                    u[8 * q + 2 * p + 1] = bf16_bits_to_f32(ww[p] >> 16);
+        for (int b = 0; b < 16; ++b) {
+            const float2 e = e2m1x2_value((w[b >> 2] >> (8 * (b & 3))) & 0xFFu);
+            const float d = b < 8 ? d0 : d1;
+            v[2 * b] = __fmul_rn(__fmul_rn(e.x, d), g);
+            v[2 * b + 1] = __fmul_rn(__fmul_rn(e.y, d), g);
+        }
+    }
+}
+
+template <int FMT, bool LOWRANK>
+__global__ void __launch_bounds__(256, 2) reconstruct_kernel(const uint8_t *__restrict__ codes,
+                                                             const void *__restrict__ scales,
+                                                             const float *__restrict__ g_w,
+                                                             const uint16_t *__restrict__ U,
+                                                             const uint16_t *__restrict__ D, int64_t N, int64_t K,
+                                                             uint16_t *__restrict__ W)
+{
+    extern __shared__ __align__(128) uint8_t rec_smem[];
+    float *h = reinterpret_cast<float *>(rec_smem);                                // [64][256] swizzled
+    uint64_t *us = reinterpret_cast<uint64_t *>(rec_smem + kRecHBytes);            // [64][32] (u, u)
+    uint8_t *stage0 = rec_smem + (LOWRANK ? kRecHBytes + kRecUsBytes : 0);
+    const int tid = threadIdx.x;
+    const int lane = tid & 31, warp = tid >> 5;
+    const float g = FMT == 2 ? *g_w : 0.0f;
+    const int64_t NT = (N + kRecRows - 1) / kRecRows;
+    const int64_t T = (K / kHad) * NT;
+    const int64_t t_begin = T * blockIdx.x / gridDim.x;
+    const int64_t t_end = T * (blockIdx.x + 1) / gridDim.x;
+    if (t_begin >= t_end)
+        return;
+    const uint32_t sbase = smem_u32(stage0);
+    rec_stage<FMT, LOWRANK>(sbase, codes, scales, U, N, K, t_begin / NT, (t_begin % NT) * kRecRows, tid);
+    cp_async_commit();
+
+    const int cp = tid & 127;                        // phase 2: column pair
+    const int rbase = 32 * (tid >> 7);
+    const int f = cp >> 1;                           // float4 of h holding columns 2cp, 2cp+1
+    const int fo = 2 * (cp & 1);
+    uint64_t d2[kRank];
+    int64_t cur_kb = -1;
+
+#pragma unroll 1
+    for (int64_t t = t_begin, i = 0; t < t_end; ++t, ++i) {
+        const int buf = (int)(i & 1);
+        if (t + 1 < t_end)
+            rec_stage<FMT, LOWRANK>(sbase + (buf ^ 1) * kRecStageBytes, codes, scales, U, N, K, (t + 1) / NT,
+                                    ((t + 1) % NT) * kRecRows, tid);
+        cp_async_commit();
+        cp_async_wait<1>();
+        __syncthreads();                             // tile t staged; previous tile's phase 2 done
+        const int64_t kb = t / NT;
+        const int64_t n0 = (t % NT) * kRecRows;
+        const uint8_t *st = stage0 + buf * kRecStageBytes;
+
+        // phase 1: h = H(d)
+#pragma unroll 1
+        for (int pass = 0; pass < 2; ++pass) {
+            const int r = 32 * pass + 4 * warp + (lane >> 3);
+            const int q = lane & 7;
+            float v[32];
+            rec_decode<FMT>(st, r, q, g, v);
+            fwht256_l32(v, lane);
+            if (!LOWRANK) {                          // residual only: straight to W
+                const int64_t n = n0 + r;
+                if (n < N) {
+                    uint4 *o = reinterpret_cast<uint4 *>(W + n * K + kb * kHad + 32 * q);
+#pragma unroll
+                    for (int k = 0; k < 4; ++k) {
+                        uint32_t ww[4];
+#pragma unroll
+                        for (int j = 0; j < 4; ++j)
+                            ww[j] = f32_to_bf16_bits(v[8 * k + 2 * j]) |
+                                    (f32_to_bf16_bits(v[8 * k + 2 * j + 1]) << 16);
+                        o[k] = make_uint4(ww[0], ww[1], ww[2], ww[3]);
+                    }
+                }
+            } else {
+                float4 *row = reinterpret_cast<float4 *>(h + r * kHad);
+#pragma unroll
+                for (int k = 0; k < 8; ++k) {
+                    const int ff = 8 * q + k;
+                    row[ff ^ (ff >> 3)] = make_float4(v[4 * k], v[4 * k + 1], v[4 * k + 2], v[4 * k + 3]);
                 }
             }
-            float L[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+        }
+        if (!LOWRANK) {
+            __syncthreads();                         // stage buffer free before the next prefetch lands
+            continue;
+        }
+        {
+            const uint16_t *ust = reinterpret_cast<const uint16_t *>(st + kRecCodeBytes + kRecScaleBytes);
 #pragma unroll
-            for (int r = 0; r < kRank; ++r) {
-                const float4 a = *reinterpret_cast<const float4 *>(dts + r * kDtPitch + 4 * lane);
-                const float4 b = *reinterpret_cast<const float4 *>(dts + r * kDtPitch + 128 + 4 * lane);
-                L[0] = __fmaf_rn(u[r], a.x, L[0]);
-                L[1] = __fmaf_rn(u[r], a.y, L[1]);
-                L[2] = __fmaf_rn(u[r], a.z, L[2]);
-                L[3] = __fmaf_rn(u[r], a.w, L[3]);
-                L[4] = __fmaf_rn(u[r], b.x, L[4]);
-                L[5] = __fmaf_rn(u[r], b.y, L[5]);
-                L[6] = __fmaf_rn(u[r], b.z, L[6]);
-                L[7] = __fmaf_rn(u[r], b.w, L[7]);
+            for (int j = 0; j < kRecRows * kRank / 256; ++j) {
+                const float u = bf16_bits_to_f32(ust[tid + 256 * j]);
+                us[tid + 256 * j] = pack2(u, u);
+            }
+        }
+        if (kb != cur_kb) {                          // lora_down of this thread's two columns
+            cur_kb = kb;
+            const int64_t k0 = kb * kHad + 2 * cp;
+            const uint4 *dr0 = reinterpret_cast<const uint4 *>(D + k0 * kRank);
+            const uint4 *dr1 = reinterpret_cast<const uint4 *>(D + (k0 + 1) * kRank);
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+                const uint4 a = __ldg(dr0 + k), b = __ldg(dr1 + k);
+                const uint32_t wa[4] = {a.x, a.y, a.z, a.w}, wb[4] = {b.x, b.y, b.z, b.w};
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                    d2[8 * k + 2 * j] = pack2(bf16_bits_to_f32(wa[j] & 0xFFFFu), bf16_bits_to_f32(wb[j] & 0xFFFFu));
+                    d2[8 * k + 2 * j + 1] = pack2(bf16_bits_to_f32(wa[j] >> 16), bf16_bits_to_f32(wb[j] >> 16));
+                }
+            }
+        }
+        __syncthreads();                             // h and us complete
+
+        // phase 2
+        const int64_t k0 = kb * kHad + 2 * cp;
+#pragma unroll 1
+        for (int r0 = rbase; r0 < rbase + 32; r0 += 4) {
+            uint64_t acc[4] = {0ull, 0ull, 0ull, 0ull};
+#pragma unroll
+            for (int rr = 0; rr < kRank; rr += 2) {
+                ulonglong2 u2[4];
+#pragma unroll
+                for (int j = 0; j < 4; ++j)
+                    u2[j] = *reinterpret_cast<const ulonglong2 *>(us + (r0 + j) * kRank + rr);
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                    fma2(acc[j], u2[j].x, d2[rr]);
+                    fma2(acc[j], u2[j].y, d2[rr + 1]);
+                }
             }
 #pragma unroll
-            for (int i = 0; i < 8; ++i)
-                v[i] = __fadd_rn(L[i], v[i]);
+            for (int j = 0; j < 4; ++j) {
+                const int r = r0 + j;
+                const int64_t n = n0 + r;
+                if (n >= N)
+                    continue;
+                const float2 hv = *reinterpret_cast<const float2 *>(h + r * kHad + 4 * (f ^ (f >> 3)) + fo);
+                float L0, L1;
+                unpack2(acc[j], L0, L1);
+                const uint32_t o = f32_to_bf16_bits(__fadd_rn(L0, hv.x)) |
+                                   (f32_to_bf16_bits(__fadd_rn(L1, hv.y)) << 16);
+                *reinterpret_cast<uint32_t *>(W + n * K + k0) = o;
+            }
         }
-        uint2 lo, hi;
-        lo.x = f32_to_bf16_bits(v[0]) | (f32_to_bf16_bits(v[1]) << 16);
-        lo.y = f32_to_bf16_bits(v[2]) | (f32_to_bf16_bits(v[3]) << 16);
-        hi.x = f32_to_bf16_bits(v[4]) | (f32_to_bf16_bits(v[5]) << 16);
-        hi.y = f32_to_bf16_bits(v[6]) | (f32_to_bf16_bits(v[7]) << 16);
-        uint16_t *o = W + n * K + kb * kHad;
-        *reinterpret_cast<uint2 *>(o + 4 * lane) = lo;
-        *reinterpret_cast<uint2 *>(o + 128 + 4 * lane) = hi;
     }
+    cp_async_wait<0>();
 }
 
 // ---------------------------------------------------------------------------
@@ -850,12 +1005,37 @@ cudaError_t launch_lowrank_finish(const float *t32, int64_t M, const float *g_x,
 
 cudaError_t launch_reconstruct(int fmt, const uint8_t *codes, const void *scales, const float *g_w,
                                const uint16_t *U, const uint16_t *D, int64_t N, int64_t K, int with_lowrank,
-                               uint16_t *W, cudaStream_t s)
+                               uint16_t *W, int sms, cudaStream_t s)
 {
-    // 32 x 260 floats = 33,280 bytes of dynamic shared memory: under the 48 KB default
-    const int smem = with_lowrank ? kRank * kDtPitch * (int)sizeof(float) : 0;
-    dim3 grid((unsigned)(K / kHad), (unsigned)((N + kReconRows - 1) / kReconRows));
-    reconstruct_kernel<<<grid, 256, smem, s>>>(fmt, codes, scales, g_w, U, D, N, K, with_lowrank, W);
+    constexpr int kMaxDev = 64;
+    static bool attr_done[kMaxDev];
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDev)
+        return cudaErrorInvalidDevice;
+    if (!attr_done[dev]) {
+        cudaError_t e = cudaFuncSetAttribute(reconstruct_kernel<1, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             kRecSmemLowrank);
+        if (e == cudaSuccess)
+            e = cudaFuncSetAttribute(reconstruct_kernel<2, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                     kRecSmemLowrank);
+        if (e != cudaSuccess)
+            return e;
+        attr_done[dev] = true;
+    }
+    const int64_t tiles = (K / kHad) * ((N + kRecRows - 1) / kRecRows);
+    const unsigned grid = (unsigned)(tiles < 2LL * sms ? tiles : 2LL * sms);
+    const int smem = with_lowrank ? kRecSmemLowrank : kRecSmemResidual;
+    if (fmt == 2) {
+        if (with_lowrank)
+            reconstruct_kernel<2, true><<<grid, 256, smem, s>>>(codes, scales, g_w, U, D, N, K, W);
+        else
+            reconstruct_kernel<2, false><<<grid, 256, smem, s>>>(codes, scales, g_w, U, D, N, K, W);
+    } else {
+        if (with_lowrank)
+            reconstruct_kernel<1, true><<<grid, 256, smem, s>>>(codes, scales, g_w, U, D, N, K, W);
+        else
+            reconstruct_kernel<1, false><<<grid, 256, smem, s>>>(codes, scales, g_w, U, D, N, K, W);
+    }
     return cudaGetLastError();
 }
 
