@@ -612,8 +612,8 @@ constexpr int kRecScaleBytes = kRecRows * 16;             // 1 KB (8 fp16 or 16 
 constexpr int kRecUBytes = kRecRows * kRank * 2;          // 4 KB
 constexpr int kRecStageBytes = kRecCodeBytes + kRecScaleBytes + kRecUBytes;
 constexpr int kRecHBytes = kRecRows * kHad * 4;           // 64 KB
-constexpr int kRecUsBytes = kRecRows * kRank * 8;         // 16 KB
-constexpr int kRecSmemLowrank = kRecHBytes + kRecUsBytes + 2 * kRecStageBytes;   // 106 KB
+constexpr int kRecUsBytes = kRecRows * kRank * 4;         // 8 KB
+constexpr int kRecSmemLowrank = kRecHBytes + kRecUsBytes + 2 * kRecStageBytes;   // 98 KB
 constexpr int kRecSmemResidual = 2 * kRecStageBytes;
 
 __device__ __forceinline__ uint64_t pack2(float lo, float hi)
@@ -717,7 +717,7 @@ __global__ void __launch_bounds__(256, 2) reconstruct_kernel(const uint8_t *__re
 {
     extern __shared__ __align__(128) uint8_t rec_smem[];
     float *h = reinterpret_cast<float *>(rec_smem);                                // [64][256] swizzled
-    uint64_t *us = reinterpret_cast<uint64_t *>(rec_smem + kRecHBytes);            // [64][32] (u, u)
+    float *us = reinterpret_cast<float *>(rec_smem + kRecHBytes);                  // [64][32] lora_up, fp32
     uint8_t *stage0 = rec_smem + (LOWRANK ? kRecHBytes + kRecUsBytes : 0);
     const int tid = threadIdx.x;
     const int lane = tid & 31, warp = tid >> 5;
@@ -791,8 +791,7 @@ __global__ void __launch_bounds__(256, 2) reconstruct_kernel(const uint8_t *__re
             const uint16_t *ust = reinterpret_cast<const uint16_t *>(st + kRecCodeBytes + kRecScaleBytes);
 #pragma unroll
             for (int j = 0; j < kRecRows * kRank / 256; ++j) {
-                const float u = bf16_bits_to_f32(ust[tid + 256 * j]);
-                us[tid + 256 * j] = pack2(u, u);
+                us[tid + 256 * j] = bf16_bits_to_f32(ust[tid + 256 * j]);
             }
         }
         if (kb != cur_kb) {                          // lora_down of this thread's two columns
@@ -819,15 +818,17 @@ __global__ void __launch_bounds__(256, 2) reconstruct_kernel(const uint8_t *__re
         for (int r0 = rbase; r0 < rbase + 32; r0 += 4) {
             uint64_t acc[4] = {0ull, 0ull, 0ull, 0ull};
 #pragma unroll
-            for (int rr = 0; rr < kRank; rr += 2) {
-                ulonglong2 u2[4];
+            for (int rr = 0; rr < kRank; rr += 4) {
+                float4 u4[4];
 #pragma unroll
                 for (int j = 0; j < 4; ++j)
-                    u2[j] = *reinterpret_cast<const ulonglong2 *>(us + (r0 + j) * kRank + rr);
+                    u4[j] = *reinterpret_cast<const float4 *>(us + (r0 + j) * kRank + rr);
 #pragma unroll
                 for (int j = 0; j < 4; ++j) {
-                    fma2(acc[j], u2[j].x, d2[rr]);
-                    fma2(acc[j], u2[j].y, d2[rr + 1]);
+                    fma2(acc[j], pack2(u4[j].x, u4[j].x), d2[rr]);
+                    fma2(acc[j], pack2(u4[j].y, u4[j].y), d2[rr + 1]);
+                    fma2(acc[j], pack2(u4[j].z, u4[j].z), d2[rr + 2]);
+                    fma2(acc[j], pack2(u4[j].w, u4[j].w), d2[rr + 3]);
                 }
             }
 #pragma unroll
