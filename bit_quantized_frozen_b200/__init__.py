@@ -37,7 +37,7 @@ RANK = 32
 EXPORTED = [
     "sq_status_str", "sq_abi_version", "sq_last_error_detail", "sq_sf_bytes", "sq_workspace_bytes",
     "sq_build_int4", "sq_build_nvfp4", "sq_act_quant_nvfp4", "sq_linear_fwd", "sq_reconstruct_bf16",
-    "sq_check_device_status", "sq_set_gemm_events",
+    "sq_check_device_status", "sq_set_gemm_events", "sq_linear_fwd_noalloc",
 ]
 
 
@@ -77,6 +77,8 @@ _SIGS = {
                            ctypes.c_int),
     "sq_linear_fwd": ([ctypes.POINTER(sq_weight), _P, _I64, _P, _P, ctypes.c_uint32, _P, ctypes.c_size_t, _P],
                       ctypes.c_int),
+    "sq_linear_fwd_noalloc": ([ctypes.POINTER(sq_weight), _P, _I64, _P, _P, ctypes.c_uint32,
+                               ctypes.POINTER(ctypes.c_void_p), _P], ctypes.c_int),
     "sq_reconstruct_bf16": ([ctypes.POINTER(sq_weight), _P, ctypes.c_uint32, _P], ctypes.c_int),
     "sq_check_device_status": ([_P, _P], ctypes.c_int),
     "sq_set_gemm_events": ([_P, _P], ctypes.c_int),
@@ -171,6 +173,17 @@ def sq_linear_fwd(w: "Weight", x, y, g_x=None, flags: int = 0, ws=None, stream=N
     cw = w.as_c()
     _check("sq_linear_fwd", lib().sq_linear_fwd(ctypes.byref(cw), _ptr(x), M, _ptr(y), _ptr(g_x), flags, _ptr(ws),
                                                 0 if ws is None else _numel_bytes(ws), _stream(stream)))
+
+
+def sq_linear_fwd_noalloc(w: "Weight", x, y, g_x=None, flags: int = 0, stream=None) -> int:
+    """sq_linear_fwd on libsq's static per-device scratch (no workspace);
+    returns the scratch's device address (for sq_check_device_status)."""
+    M = x.shape[0]
+    cw = w.as_c()
+    scratch = ctypes.c_void_p()
+    _check("sq_linear_fwd_noalloc", lib().sq_linear_fwd_noalloc(ctypes.byref(cw), _ptr(x), M, _ptr(y), _ptr(g_x),
+                                                                flags, ctypes.byref(scratch), _stream(stream)))
+    return scratch.value
 
 
 def sq_reconstruct_bf16(w: "Weight", W_out, flags: int = 0, stream=None):

@@ -4,11 +4,14 @@
 // read-back); every error is returned as an sq_status before any launch.
 #include <cuda_runtime.h>
 
+#include <atomic>
 #include <cstdio>
 #include <cstring>
 
 #include "sq.h"
 #include "sq_kernels.h"
+
+static __device__ __align__(256) uint8_t g_noalloc_scratch[size_t(32) << 20];
 
 namespace {
 
@@ -123,6 +126,14 @@ uint8_t *ws_at(void *ws, size_t off)
             return SQ_ERR_CUDA;                 \
         }                                       \
     } while (0)
+
+// Static scratch of sq_linear_fwd_noalloc --------------------------------------
+// A fixed 32 MiB forward workspace that lives in the module's own device
+// memory (one copy per device, created when the module's device code is
+// loaded, released with the context), so that the call needs no allocation.
+// Its device address is looked up once per device, with that device current.
+constexpr size_t kNoAllocScratchBytes = size_t(32) << 20;
+std::atomic<void *> g_noalloc_scratch_ptr[kMaxDevices];
 
 sq_status check_weight(const sq_weight *w)
 {
@@ -355,6 +366,42 @@ sq_status sq_linear_fwd(const sq_weight *w, const uint16_t *x, int64_t M, float 
     if (g_gemm_ev1)
         SQ_CUDA(cudaEventRecord(g_gemm_ev1, s), "event record");
     return SQ_OK;
+}
+
+sq_status sq_linear_fwd_noalloc(const sq_weight *w, const uint16_t *x, int64_t M, float *y, float *g_x,
+                                uint32_t flags, void **scratch_out, void *stream)
+{
+    static_assert(sizeof(g_noalloc_scratch) == kNoAllocScratchBytes, "scratch size");
+    if (scratch_out)
+        *scratch_out = nullptr;
+    sq_status st = check_weight(w);
+    if (st != SQ_OK)
+        return st;
+    if (!shape_ok_mk(M, w->K))
+        return SQ_ERR_SHAPE;
+    const int op = w->fmt == SQ_FMT_NVFP4 ? SQ_OP_LINEAR_FWD_NVFP4 : SQ_OP_LINEAR_FWD_INT4;
+    const size_t need = sq_workspace_bytes(op, M, w->N, w->K);
+    if (need > kNoAllocScratchBytes) {
+        snprintf(g_detail, sizeof(g_detail),
+                 "sq_linear_fwd_noalloc: M=%lld N=%lld K=%lld needs %zu bytes of scratch, the static scratch "
+                 "holds %zu; use sq_linear_fwd with a caller workspace",
+                 (long long)M, (long long)w->N, (long long)w->K, need, kNoAllocScratchBytes);
+        return SQ_ERR_WORKSPACE;
+    }
+    int sms = 0;
+    st = check_device(&sms);
+    if (st != SQ_OK)
+        return st;
+    int dev = 0;
+    SQ_CUDA(cudaGetDevice(&dev), "cudaGetDevice");
+    void *scratch = g_noalloc_scratch_ptr[dev].load(std::memory_order_acquire);
+    if (!scratch) {                  // first call on this device: look the scratch up (device is current)
+        SQ_CUDA(cudaGetSymbolAddress(&scratch, g_noalloc_scratch), "cudaGetSymbolAddress(static scratch)");
+        g_noalloc_scratch_ptr[dev].store(scratch, std::memory_order_release);
+    }
+    if (scratch_out)
+        *scratch_out = scratch;
+    return sq_linear_fwd(w, x, M, y, g_x, flags, scratch, kNoAllocScratchBytes, stream);
 }
 
 sq_status sq_reconstruct_bf16(const sq_weight *w, uint16_t *W_out, uint32_t flags, void *stream)

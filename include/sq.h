@@ -196,6 +196,40 @@ SQ_API sq_status sq_linear_fwd(const sq_weight *w, const uint16_t *x, int64_t M,
                         void *stream);
 
 /*
+ * sq_linear_fwd without a caller workspace.  The SquareQ pages have no
+ * counterpart of this call: it is a library convenience for callers that
+ * cannot allocate device memory at the point of the forward -- plain C hosts
+ * without a device allocator of their own, and latency-critical loops where
+ * cudaMalloc (which may synchronise the device, and may fail under memory
+ * pressure) is not allowed.  Nothing is allocated: the workspace is a fixed
+ * 32 MiB scratch array in libsq's own device memory, one per device.
+ *
+ * Same arguments, results and accuracy as sq_linear_fwd, minus (ws,
+ * ws_bytes).  scratch_out (host, may be NULL) receives the device address of
+ * the scratch this call used; pass it to sq_check_device_status to read the
+ * call's device status word.
+ *
+ * Limit: sq_workspace_bytes(SQ_OP_LINEAR_FWD_NVFP4 or _INT4, M, N, K) must
+ * be at most 33554432 (32 MiB); larger shapes return SQ_ERR_WORKSPACE before
+ * any work, with the sizes in sq_last_error_detail().  (NVFP4 at N = 16384,
+ * K = 6144 fits M up to 8462 rows; the int4 forward, which keeps a bf16 copy
+ * of W in the workspace, fits N x K up to about 16 M values, e.g. M = 1536
+ * at N = K = 3072.)
+ *
+ * The first call on each device looks up the scratch's address
+ * (cudaGetSymbolAddress, with that device current), which may load libsq's
+ * device code; make that first call before any stream capture.  Nothing has
+ * to start at zero: each call clears the status word and the absmax
+ * accumulator at the start of its own stream work, like sq_linear_fwd.
+ *
+ * All calls on a device share the one scratch: calls that may overlap on the
+ * device (different streams without an event between them, or several host
+ * threads) race on it and give wrong results.  Order them on one stream.
+ */
+SQ_API sq_status sq_linear_fwd_noalloc(const sq_weight *w, const uint16_t *x, int64_t M, float *y,
+                                       float *g_x, uint32_t flags, void **scratch_out, void *stream);
+
+/*
  * bf16 reconstruct of W for the backward pass (SquareQ README: "the bwd-side
  * bf16 reconstruct from the same payload").  For each element
  *   d = q s (int4) or RN(RN(e2m1 value(sf)) g_w) (NVFP4),
