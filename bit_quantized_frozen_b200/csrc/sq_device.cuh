@@ -68,6 +68,51 @@ __device__ __forceinline__ void fwht256_warp(float (&v)[8], int lane)
 }
 
 // ---------------------------------------------------------------------------
+// Two fp32 lanes in one 64-bit register (sm_100 packed arithmetic).  Each lane
+// of add / sub / mul / fma .rn.f32x2 is rounded once, exactly like the scalar
+// instruction, so packed and scalar code give identical bits.
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ uint64_t f2_pack(float lo, float hi)
+{
+    uint64_t r;
+    asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+    return r;
+}
+
+__device__ __forceinline__ void f2_unpack(uint64_t v, float &lo, float &hi)
+{
+    asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+}
+
+__device__ __forceinline__ uint64_t f2_add(uint64_t a, uint64_t b)
+{
+    uint64_t r;
+    asm("add.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+    return r;
+}
+
+__device__ __forceinline__ uint64_t f2_sub(uint64_t a, uint64_t b)
+{
+    uint64_t r;
+    asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+    return r;
+}
+
+__device__ __forceinline__ uint64_t f2_mul(uint64_t a, uint64_t b)
+{
+    uint64_t r;
+    asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+    return r;
+}
+
+__device__ __forceinline__ uint64_t f2_fma(uint64_t a, uint64_t b, uint64_t c)
+{
+    uint64_t r;
+    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(r) : "l"(a), "l"(b), "l"(c));
+    return r;
+}
+
+// ---------------------------------------------------------------------------
 // Hadamard-256 over 8 lanes.
 //
 // Layout: lane q = lane % 8 of an aligned group of 8 lanes holds v[0..31] =
@@ -75,31 +120,53 @@ __device__ __forceinline__ void fwht256_warp(float (&v)[8], int lane)
 // 1..16 pair values inside a lane, strides 32, 64, 128 pair lane q with lane
 // q ^ 1, q ^ 2, q ^ 4.  Same butterflies, same operands, same order of
 // strides as the sequential transform, so the result is identical bit for bit.
+// Strides >= 2 run on packed pairs (v[2j], v[2j+1]).  With SCALE = false the
+// final multiply by 1/16 is left to the caller (exact: a power of two).
 // ---------------------------------------------------------------------------
+template <bool SCALE = true>
 __device__ __forceinline__ void fwht256_l32(float (&v)[32], int lane)
 {
 #pragma unroll
-    for (int h = 1; h < 32; h <<= 1)
+    for (int j = 0; j < 16; ++j) {               // stride 1, inside each pair
+        const float a = v[2 * j], b = v[2 * j + 1];
+        v[2 * j] = __fadd_rn(a, b);
+        v[2 * j + 1] = __fsub_rn(a, b);
+    }
+    uint64_t p[16];
 #pragma unroll
-        for (int i = 0; i < 32; ++i)
-            if ((i & h) == 0) {
-                const float a = v[i], b = v[i + h];
-                v[i] = __fadd_rn(a, b);
-                v[i + h] = __fsub_rn(a, b);
+    for (int j = 0; j < 16; ++j)
+        p[j] = f2_pack(v[2 * j], v[2 * j + 1]);
+#pragma unroll
+    for (int hp = 1; hp < 16; hp <<= 1)          // strides 2, 4, 8, 16 = pair strides 1..8
+#pragma unroll
+        for (int j = 0; j < 16; ++j)
+            if ((j & hp) == 0) {
+                const uint64_t a = p[j], b = p[j + hp];
+                p[j] = f2_add(a, b);
+                p[j + hp] = f2_sub(a, b);
             }
 #pragma unroll
-    for (int x = 1; x <= 4; x <<= 1) {          // h = 32x
+    for (int x = 1; x <= 4; x <<= 1) {          // strides 32x, across lanes
         // lower lane: p + v, upper lane: p - v, as one fma with +-1 (same single rounding)
         const float sg = (lane & x) == 0 ? 1.0f : -1.0f;
+        const uint64_t sg2 = f2_pack(sg, sg);
 #pragma unroll
-        for (int i = 0; i < 32; ++i) {
-            const float p = __shfl_xor_sync(0xffffffffu, v[i], x);
-            v[i] = __fmaf_rn(sg, v[i], p);
+        for (int j = 0; j < 16; ++j) {
+            float lo, hi;
+            f2_unpack(p[j], lo, hi);
+            const uint64_t o = f2_pack(__shfl_xor_sync(0xffffffffu, lo, x), __shfl_xor_sync(0xffffffffu, hi, x));
+            p[j] = f2_fma(sg2, p[j], o);
         }
     }
+    if (SCALE) {
+        const uint64_t sc = f2_pack(0.0625f, 0.0625f);
 #pragma unroll
-    for (int i = 0; i < 32; ++i)
-        v[i] = __fmul_rn(v[i], 0.0625f);
+        for (int j = 0; j < 16; ++j)
+            p[j] = f2_mul(p[j], sc);
+    }
+#pragma unroll
+    for (int j = 0; j < 16; ++j)
+        f2_unpack(p[j], v[2 * j], v[2 * j + 1]);
 }
 
 // 32 consecutive values into registers (fp32 source or bf16 bit patterns)
@@ -159,12 +226,24 @@ __device__ __forceinline__ uint32_t to_e2m1x2_mag(float lo, float hi)
 }
 
 // e2m1 codes of two values with their sign bits kept (negative -> bit 3 set,
-// including values that round to zero), packed lo | hi << 4.
+// including values that round to zero), packed lo | hi << 4.  The signed
+// conversion keeps the sign of a negative value that rounds to zero (checked
+// against the magnitude conversion plus explicit sign bits).
 __device__ __forceinline__ uint32_t to_e2m1x2(float lo, float hi)
 {
-    uint32_t mag = to_e2m1x2_mag(fabsf(lo), fabsf(hi));
-    uint32_t s = ((__float_as_uint(lo) >> 31) << 3) | ((__float_as_uint(hi) >> 31) << 7);
-    return mag | s;
+    return to_e2m1x2_mag(lo, hi);
+}
+
+// e2m1 codes of four values, packed a | b << 4 | c << 8 | d << 12
+__device__ __forceinline__ uint32_t to_e2m1x4(float a, float b, float c, float d)
+{
+    uint16_t out;
+    asm("{\n\t.reg .b8 t0, t1;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 t0, %2, %1;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 t1, %4, %3;\n\t"
+        "mov.b16 %0, {t0, t1};\n\t}"
+        : "=h"(out) : "f"(a), "f"(b), "f"(c), "f"(d));
+    return out;
 }
 
 // values of two e2m1 codes held in one byte (low nibble first), exact

@@ -127,11 +127,13 @@ __global__ void __launch_bounds__(kStreamThreads) absmax_rot_kernel(const __grid
     const int lane = threadIdx.x & 31;
     float m = 0.0f;
     stream_blocks<T>(&tm, blocks, nullptr, [&](int64_t, float (&v)[32], bool) {
-        fwht256_l32(v, lane);
+        fwht256_l32<false>(v, lane);
 #pragma unroll
         for (int i = 0; i < 32; ++i)
             m = fmaxf(m, fabsf(v[i]));
     });
+    // max |v / 16| == (max |v|) / 16 bit for bit: rounding is monotonic
+    m = __fmul_rn(m, 0.0625f);
 #pragma unroll
     for (int x = 16; x >= 1; x >>= 1)
         m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, x));
@@ -172,11 +174,12 @@ __global__ void __launch_bounds__(kStreamThreads) nvfp4_quant_kernel(const __gri
     const float sixg = __fmul_rn(6.0f, g);
     const int64_t kb_per_row = K / kHad;
     const int64_t C = K / kSfBlock;
+    const bool idx32 = rows_pad * kb_per_row <= (int64_t)UINT32_MAX;
     stream_blocks<T>(&tm, rows_pad * kb_per_row, nullptr, [&](int64_t b, float (&v)[32], bool valid) {
         fwht256_l32(v, lane);
         if (!valid)
             return;
-        const int64_t row = b / kb_per_row;
+        const int64_t row = idx32 ? (int64_t)((uint32_t)b / (uint32_t)kb_per_row) : b / kb_per_row;
         const int64_t kb = b - row * kb_per_row;
         uint32_t word[4];
         uint32_t sfc[2];
@@ -192,14 +195,14 @@ __global__ void __launch_bounds__(kStreamThreads) nvfp4_quant_kernel(const __gri
                 code = to_ue4m3(__fdiv_rn(bmax, sixg));
                 if (code != 0) {
                     const float inv = __frcp_rn(__fmul_rn(ue4m3_value(code), g));
+                    const uint64_t inv2 = f2_pack(inv, inv);
+                    float s[16];
 #pragma unroll
-                    for (int i = 0; i < 4; ++i) {
-                        w0 |= to_e2m1x2(__fmul_rn(v[16 * h + 2 * i], inv), __fmul_rn(v[16 * h + 2 * i + 1], inv))
-                              << (8 * i);
-                        w1 |= to_e2m1x2(__fmul_rn(v[16 * h + 8 + 2 * i], inv),
-                                        __fmul_rn(v[16 * h + 8 + 2 * i + 1], inv))
-                              << (8 * i);
-                    }
+                    for (int i = 0; i < 8; ++i)
+                        f2_unpack(f2_mul(f2_pack(v[16 * h + 2 * i], v[16 * h + 2 * i + 1]), inv2), s[2 * i],
+                                  s[2 * i + 1]);
+                    w0 = to_e2m1x4(s[0], s[1], s[2], s[3]) | (to_e2m1x4(s[4], s[5], s[6], s[7]) << 16);
+                    w1 = to_e2m1x4(s[8], s[9], s[10], s[11]) | (to_e2m1x4(s[12], s[13], s[14], s[15]) << 16);
                 }
             }
             word[2 * h] = w0;
@@ -347,21 +350,25 @@ __global__ void __launch_bounds__(256) dequant_int4_kernel(const uint32_t *__res
 //   amax (optional): max |H x| over the whole tensor (the activation global
 //                    scale's input), from the 8-lane Hadamard transform;
 //   t32 (optional):  t = x . lora_down, fp32 [M, 32], on mma.sync bf16 tensor
-//                    cores (fp32 accumulation; each CTA sums its partials in a
-//                    fixed order, so t is deterministic).
-// A CTA owns 16 rows and walks K in 256-column chunks; the x chunk (16 x 256)
-// and the lora_down chunk (256 x 32) are staged in shared memory by cp.async,
-// double buffered.  Warps 0-3 transform rows 4w..4w+3, warps 4-7 run k-steps
-// 4(w-4)..4(w-4)+3 of the chunk for all 32 outputs.
+//                    cores (fp32 accumulation, summed in a fixed order, so t
+//                    is deterministic for a given shape and SM count).
+// A CTA owns 32 rows and a range of 256-column chunks; when there are few row
+// tiles, K is split over a cluster of `split` CTAs (one per range) whose
+// partial t tiles are summed in rank order by rank 0 through distributed
+// shared memory.  The x chunk (32 x 256) and the lora_down chunk (256 x 32)
+// are staged by cp.async in a 3-deep ring.  Every warp transforms 4 rows and
+// runs 4 of the chunk's 16 k-steps for one 16-row half of the tile.
 // x tile: 16-byte chunk c of row r sits at c ^ ((c >> 2) & 7) ^ (r & 7), which
 // keeps both the transform's per-row reads and ldmatrix conflict free; D tile:
 // chunk c of k-row k sits at c ^ ((k >> 1) & 3).
 // ---------------------------------------------------------------------------
-constexpr int kP1Rows = 16;
-constexpr int kP1XBytes = kP1Rows * kHad * 2;      // 8 KB
+constexpr int kP1Rows = 32;
+constexpr int kP1XBytes = kP1Rows * kHad * 2;      // 16 KB
 constexpr int kP1DBytes = kHad * kRank * 2;        // 16 KB
 constexpr int kP1BufBytes = kP1XBytes + kP1DBytes;
-constexpr int kP1Smem = 2 * kP1BufBytes;           // 48 KB
+constexpr int kP1Stages = 3;
+constexpr int kP1Smem = kP1Stages * kP1BufBytes;   // 96 KB
+constexpr int kP1MaxSplit = 8;
 
 __device__ __forceinline__ void cp_async16(uint32_t dst, const void *src, uint32_t src_bytes)
 {
@@ -409,23 +416,34 @@ __device__ __forceinline__ uint32_t p1_doff(int k, int c)
     return (uint32_t)(k * 64 + 16 * (c ^ ((k >> 1) & 3)));
 }
 
-__global__ void __launch_bounds__(256) act_pass1_kernel(const uint16_t *__restrict__ x, int64_t M, int64_t K,
-                                                        const uint16_t *__restrict__ D,
-                                                        uint32_t *__restrict__ amax, float *__restrict__ t32)
+__device__ __forceinline__ float ld_shared_cluster_f32(uint32_t addr)
+{
+    float v;
+    asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(v) : "r"(addr) : "memory");
+    return v;
+}
+
+__global__ void __launch_bounds__(256, 2) act_pass1_kernel(const uint16_t *__restrict__ x, int64_t M, int64_t K,
+                                                           const uint16_t *__restrict__ D,
+                                                           uint32_t *__restrict__ amax, float *__restrict__ t32,
+                                                           int split)
 {
     extern __shared__ __align__(128) uint8_t p1_smem[];
     const int tid = threadIdx.x;
     const int lane = tid & 31;
     const int warp = tid >> 5;
-    const int64_t m0 = (int64_t)blockIdx.x * kP1Rows;
+    const int j = (int)(blockIdx.x % (unsigned)split);       // cluster rank (clusters run along x)
+    const int64_t m0 = (int64_t)(blockIdx.x / (unsigned)split) * kP1Rows;
     const int nkb = (int)(K / kHad);
+    const int kb0 = (int)((int64_t)j * nkb / split);
+    const int nch = (int)((int64_t)(j + 1) * nkb / split) - kb0;
     const uint32_t sbase = (uint32_t)__cvta_generic_to_shared(p1_smem);
 
     auto issue = [&](int kb, int buf) {
         const uint32_t xs = sbase + buf * kP1BufBytes;
         const uint32_t ds = xs + kP1XBytes;
 #pragma unroll
-        for (int i = 0; i < 2; ++i) {                 // x: 16 rows x 32 chunks
+        for (int i = 0; i < 4; ++i) {                 // x: 32 rows x 32 chunks
             const int e = tid + 256 * i;
             const int r = e >> 5, c = e & 31;
             const int64_t row = m0 + r;
@@ -441,7 +459,6 @@ __global__ void __launch_bounds__(256) act_pass1_kernel(const uint16_t *__restri
                 cp_async16(ds + p1_doff(k, c), D + ((int64_t)kb * kHad + k) * kRank + 8 * c, 16u);
             }
         }
-        cp_async_commit();
     };
 
     float m = 0.0f;
@@ -452,81 +469,82 @@ __global__ void __launch_bounds__(256) act_pass1_kernel(const uint16_t *__restri
         for (int i = 0; i < 4; ++i)
             acc[nt][i] = 0.0f;
 
-    issue(0, 0);
-    for (int kb = 0; kb < nkb; ++kb) {
-        const int buf = kb & 1;
-        if (kb + 1 < nkb) {
-            issue(kb + 1, buf ^ 1);
-            cp_async_wait<1>();
-        } else {
-            cp_async_wait<0>();
-        }
-        __syncthreads();
+#pragma unroll
+    for (int c = 0; c < kP1Stages - 1; ++c) {
+        if (c < nch)
+            issue(kb0 + c, c);
+        cp_async_commit();                            // (possibly empty) group c
+    }
+    const int mt = warp >> 2;                         // MMA: rows 16mt..16mt+15
+#pragma unroll 1
+    for (int c = 0; c < nch; ++c) {
+        cp_async_wait<kP1Stages - 2>();               // chunk c has landed (this thread's copies)
+        __syncthreads();                              // ... everyone's; stage of chunk c-1 is free
+        if (c + kP1Stages - 1 < nch)
+            issue(kb0 + c + kP1Stages - 1, (c + kP1Stages - 1) % kP1Stages);
+        cp_async_commit();
+        const int buf = c % kP1Stages;
         const uint32_t xs = sbase + buf * kP1BufBytes;
         const uint32_t ds = xs + kP1XBytes;
-        if (warp < 4) {
-            if (amax) {
-                const int r = 4 * warp + (lane >> 3);
-                const int q = lane & 7;
-                float v[32];
+        if (amax) {
+            const int r = 4 * warp + (lane >> 3);
+            const int q = lane & 7;
+            float v[32];
 #pragma unroll
-                for (int i = 0; i < 4; ++i) {
-                    const uint4 a = *reinterpret_cast<const uint4 *>(p1_smem + (p1_xoff(r, 4 * q + i) +
-                                                                                 buf * kP1BufBytes));
-                    const uint32_t w[4] = {a.x, a.y, a.z, a.w};
+            for (int i = 0; i < 4; ++i) {
+                const uint4 a = *reinterpret_cast<const uint4 *>(p1_smem + (p1_xoff(r, 4 * q + i) +
+                                                                             buf * kP1BufBytes));
+                const uint32_t w[4] = {a.x, a.y, a.z, a.w};
 #pragma unroll
-                    for (int j = 0; j < 4; ++j) {
-                        v[8 * i + 2 * j] = __uint_as_float(w[j] << 16);
-                        v[8 * i + 2 * j + 1] = __uint_as_float(w[j] & 0xFFFF0000u);
-                    }
+                for (int jj = 0; jj < 4; ++jj) {
+                    v[8 * i + 2 * jj] = __uint_as_float(w[jj] << 16);
+                    v[8 * i + 2 * jj + 1] = __uint_as_float(w[jj] & 0xFFFF0000u);
                 }
-                fwht256_l32(v, lane);
-#pragma unroll
-                for (int i = 0; i < 32; ++i)
-                    m = fmaxf(m, fabsf(v[i]));
             }
-        } else if (t32) {
-            const int w4 = warp - 4;
+            fwht256_l32<false>(v, lane);
 #pragma unroll
-            for (int s = 0; s < 4; ++s) {
-                const int ks = 4 * w4 + s;            // k-step: columns 16ks..16ks+15 of the chunk
+            for (int i = 0; i < 32; ++i)
+                m = fmaxf(m, fabsf(v[i]));
+        }
+        if (t32) {
+#pragma unroll
+            for (int ss = 0; ss < 4; ++ss) {
+                const int ks = 4 * (warp & 3) + ss;   // k-step: columns 16ks..16ks+15 of the chunk
                 // A 16x16: matrices (rows 0-7 | 8-15) x (k 0-7 | 8-15); lane provides row (lane & 15)
                 uint32_t a[4];
-                const int ar = lane & 15;
-                const int ac = 2 * ks + (lane >> 4);
-                ldmatrix_x4(xs + p1_xoff(ar, ac), a);
+                ldmatrix_x4(xs + p1_xoff(16 * mt + (lane & 15), 2 * ks + (lane >> 4)), a);
                 // B: (k 0-7 | 8-15) x (n-tile pair), transposed load of row-major D
 #pragma unroll
                 for (int np = 0; np < 2; ++np) {
                     uint32_t b[4];
                     const int bk = 16 * ks + (lane & 7) + 8 * ((lane >> 3) & 1);
-                    const int bc = 2 * np + (lane >> 4);
-                    ldmatrix_x4_trans(ds + p1_doff(bk, bc), b);
+                    ldmatrix_x4_trans(ds + p1_doff(bk, 2 * np + (lane >> 4)), b);
                     mma_bf16_16816(acc[2 * np], a, b[0], b[1]);
                     mma_bf16_16816(acc[2 * np + 1], a, b[2], b[3]);
                 }
             }
         }
-        __syncthreads();
     }
+    cp_async_wait<0>();
+    __syncthreads();                                  // ring idle: reuse it below
 
     if (amax) {
+        m = __fmul_rn(m, 0.0625f);                    // the transform's 1/16, once (exact for a max)
 #pragma unroll
         for (int xx = 16; xx >= 1; xx >>= 1)
             m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, xx));
     }
-    // partial t tiles of warps 4-7 and the absmax reduce through the (now idle) smem
-    float *part = reinterpret_cast<float *>(p1_smem);          // [4][16][33]
-    float *wmax = part + 4 * 16 * 33;                           // [8]
-    if (warp >= 4 && t32) {
-        const int w4 = warp - 4;
+    float *part = reinterpret_cast<float *>(p1_smem);          // [8 warps][16][33]
+    float *tcta = part + 8 * 16 * 33;                           // [32][32] this CTA's t tile
+    float *wmax = tcta + kP1Rows * kRank;                       // [8]
+    if (t32) {
         const int g = lane >> 2, tq = lane & 3;
 #pragma unroll
         for (int nt = 0; nt < 4; ++nt) {
-            part[(w4 * 16 + g) * 33 + 8 * nt + 2 * tq] = acc[nt][0];
-            part[(w4 * 16 + g) * 33 + 8 * nt + 2 * tq + 1] = acc[nt][1];
-            part[(w4 * 16 + g + 8) * 33 + 8 * nt + 2 * tq] = acc[nt][2];
-            part[(w4 * 16 + g + 8) * 33 + 8 * nt + 2 * tq + 1] = acc[nt][3];
+            part[(warp * 16 + g) * 33 + 8 * nt + 2 * tq] = acc[nt][0];
+            part[(warp * 16 + g) * 33 + 8 * nt + 2 * tq + 1] = acc[nt][1];
+            part[(warp * 16 + g + 8) * 33 + 8 * nt + 2 * tq] = acc[nt][2];
+            part[(warp * 16 + g + 8) * 33 + 8 * nt + 2 * tq + 1] = acc[nt][3];
         }
     }
     if (lane == 0)
@@ -534,22 +552,38 @@ __global__ void __launch_bounds__(256) act_pass1_kernel(const uint16_t *__restri
     __syncthreads();
     if (amax && tid == 0) {
         float b = 0.0f;
-        for (int w = 0; w < 4; ++w)
+        for (int w = 0; w < 8; ++w)
             b = fmaxf(b, wmax[w]);
         atomic_max_nonneg(amax, b);
     }
-    if (t32) {
-        for (int e = tid; e < kP1Rows * kRank; e += 256) {
-            const int r = e >> 5, col = e & 31;
-            if (m0 + r >= M)
-                continue;
-            float v = 0.0f;
+    if (!t32)
+        return;
+    for (int e = tid; e < kP1Rows * kRank; e += 256) {          // k-step partials, fixed order
+        const int r = e >> 5, col = e & 31;
+        const int h = r >> 4, rr = r & 15;
+        float v = 0.0f;
 #pragma unroll
-            for (int w = 0; w < 4; ++w)
-                v = __fadd_rn(v, part[(w * 16 + r) * 33 + col]);
-            t32[(m0 + r) * kRank + col] = v;
+        for (int w = 0; w < 4; ++w)
+            v = __fadd_rn(v, part[((4 * h + w) * 16 + rr) * 33 + col]);
+        tcta[e] = v;
+    }
+    if (split > 1)
+        cluster_sync();                               // every rank's tile is complete
+    else
+        __syncthreads();
+    if (j == 0) {
+        const uint32_t tl = (uint32_t)__cvta_generic_to_shared(tcta);
+        for (int e = tid; e < kP1Rows * kRank; e += 256) {
+            const int64_t row = m0 + (e >> 5);
+            float v = tcta[e];
+            for (int rk = 1; rk < split; ++rk)
+                v = __fadd_rn(v, ld_shared_cluster_f32(mapa_shared(tl + 4 * e, (uint32_t)rk)));
+            if (row < M)
+                t32[row * kRank + (e & 31)] = v;
         }
     }
+    if (split > 1)
+        cluster_sync();                               // ranks > 0 keep their tiles until rank 0 is done
 }
 
 // ---------------------------------------------------------------------------
@@ -988,11 +1022,43 @@ cudaError_t launch_dequant_int4(const uint8_t *codes, const uint16_t *scales, in
 }
 
 cudaError_t launch_act_pass1(const uint16_t *x, int64_t M, int64_t K, const uint16_t *D, uint32_t *amax,
-                             float *t32, cudaStream_t s)
+                             float *t32, int sms, cudaStream_t s)
 {
-    const int64_t grid = (M + kP1Rows - 1) / kP1Rows;
-    act_pass1_kernel<<<(unsigned)grid, 256, kP1Smem, s>>>(x, M, K, D, amax, t32);
-    return cudaGetLastError();
+    constexpr int kMaxDev = 64;
+    static bool attr_done[kMaxDev];
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDev)
+        return cudaErrorInvalidDevice;
+    if (!attr_done[dev]) {
+        cudaError_t e = cudaFuncSetAttribute(act_pass1_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kP1Smem);
+        if (e != cudaSuccess)
+            return e;
+        attr_done[dev] = true;
+    }
+    const int64_t tiles = (M + kP1Rows - 1) / kP1Rows;
+    const int nkb = (int)(K / kHad);
+    int64_t split = (2LL * sms) / tiles;              // two CTAs per SM
+    split = split < 1 ? 1 : split;
+    split = split > kP1MaxSplit ? kP1MaxSplit : split;
+    split = split > nkb ? nkb : split;
+    const unsigned grid = (unsigned)(tiles * split);
+    if (split == 1) {
+        act_pass1_kernel<<<grid, 256, kP1Smem, s>>>(x, M, K, D, amax, t32, 1);
+        return cudaGetLastError();
+    }
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(grid);
+    cfg.blockDim = dim3(256);
+    cfg.dynamicSmemBytes = kP1Smem;
+    cfg.stream = s;
+    cudaLaunchAttribute at[1];
+    at[0].id = cudaLaunchAttributeClusterDimension;
+    at[0].val.clusterDim.x = (unsigned)split;
+    at[0].val.clusterDim.y = 1;
+    at[0].val.clusterDim.z = 1;
+    cfg.attrs = at;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, act_pass1_kernel, x, M, K, D, amax, t32, (int)split);
 }
 
 cudaError_t launch_lowrank_finish(const float *t32, int64_t M, const float *g_x, const float *g_w,
