@@ -278,7 +278,7 @@ sq_status sq_act_quant_nvfp4(const uint16_t *x, int64_t M, int64_t K, uint8_t *c
         SQ_CUDA(sq::launch_act_pass1(x, M, K, lora_down, stat ? nullptr : amax, with_t ? t : nullptr, sms, s),
                 "activation pass 1");
     SQ_CUDA(sq::launch_nvfp4_quant_bf16(x, M, K, amax, stat ? g_x : nullptr, stat ? nullptr : g_x, codes, sf_tiled,
-                                        sms, s),
+                                        sq::LowrankOut{}, sms, s),
             "nvfp4 quant");
     return SQ_OK;
 }
@@ -332,12 +332,19 @@ sq_status sq_linear_fwd(const sq_weight *w, const uint16_t *x, int64_t M, float 
         // one read of x for the absmax and the low-rank input, one for the quantisation
         if (!stat || lora)
             SQ_CUDA(sq::launch_act_pass1(x, M, K, w->lora_down, stat ? nullptr : amax, t32, sms, s), "activation pass 1");
-        SQ_CUDA(sq::launch_nvfp4_quant_bf16(x, M, K, amax, stat ? gx : nullptr, stat ? nullptr : gx, xc, xsf, sms,
-                                            s),
-                "nvfp4 act quant");
-        if (lora)
-            SQ_CUDA(sq::launch_lowrank_finish(t32, M, gx, w->g_w, tsplit, w->lora_up, N, udup, sms, s),
-                    "low-rank operands");
+        // the quantisation also writes the low-rank operands (g_x is known by then)
+        sq::LowrankOut lr;
+        if (lora) {
+            lr.t32 = t32;
+            lr.g_w = w->g_w;
+            lr.tsplit = tsplit;
+            lr.U = w->lora_up;
+            lr.N = N;
+            lr.udup = udup;
+        }
+        SQ_CUDA(sq::launch_nvfp4_quant_bf16(x, M, K, amax, stat ? gx : nullptr, stat ? nullptr : gx, xc, xsf, lr,
+                                            sms, s),
+                "nvfp4 act quant + low-rank operands");
         g.fp4 = 1;
         g.a = xc;
         g.b = w->codes;

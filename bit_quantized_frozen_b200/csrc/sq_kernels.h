@@ -7,6 +7,17 @@
 
 namespace sq {
 
+// low-rank operands of the NVFP4 forward, written by the activation quant
+// kernel after its blocks (t32 == nullptr: nothing to write)
+struct LowrankOut {
+    const float *t32 = nullptr;      // [M, 32] fp32, t = x lora_down
+    const float *g_w = nullptr;      // weight global scale (beta = g_x g_w)
+    uint16_t *tsplit = nullptr;      // [M, 64] bf16
+    const uint16_t *U = nullptr;     // lora_up [N, 32] bf16
+    int64_t N = 0;
+    uint16_t *udup = nullptr;        // [N, 64] bf16
+};
+
 cudaError_t launch_absmax_rot_f32(const float *in, int64_t rows, int64_t K, uint32_t *amax, int sms,
                                   cudaStream_t s);
 cudaError_t launch_absmax_rot_bf16(const uint16_t *in, int64_t rows, int64_t K, uint32_t *amax, int sms,
@@ -15,8 +26,8 @@ cudaError_t launch_nvfp4_quant_f32(const float *in, int64_t rows, int64_t K, con
                                    const float *g_static, float *g_out, uint8_t *codes, uint8_t *sf, int sms,
                                    cudaStream_t s);
 cudaError_t launch_nvfp4_quant_bf16(const uint16_t *in, int64_t rows, int64_t K, const uint32_t *amax,
-                                    const float *g_static, float *g_out, uint8_t *codes, uint8_t *sf, int sms,
-                                    cudaStream_t s);
+                                    const float *g_static, float *g_out, uint8_t *codes, uint8_t *sf,
+                                    const LowrankOut &lr, int sms, cudaStream_t s);
 cudaError_t launch_int4_build(const float *R, int64_t N, int64_t K, uint8_t *codes, uint16_t *scales,
                               uint8_t *frac, int sms, cudaStream_t s);
 cudaError_t launch_rotate_bf16(const uint16_t *x, int64_t M, int64_t K, uint16_t *xb, int sms, cudaStream_t s);

@@ -58,9 +58,16 @@ __device__ __forceinline__ void read_row(const uint8_t *buf, int row, float (&v)
 
 // Runs f(block, v, valid) on every 256-block of the stream, one call per lane
 // per chunk in consumer warps (all 32 lanes of a warp call f together, so f
-// may shuffle).  total_blocks may exceed the tensor (zero blocks).
-template <typename T, typename F>
-__device__ __forceinline__ void stream_blocks(const CUtensorMap *tm, int64_t total_blocks, uint32_t *status, F &&f)
+// may shuffle).  total_blocks may exceed the tensor (zero blocks).  pre(c) is
+// run once by every consumer thread c (0 .. 32 * consumers - 1) before its
+// first chunk, while the first loads are in flight.
+struct NoPrologue {
+    __device__ void operator()(int) const {}
+};
+
+template <typename T, typename F, typename P = NoPrologue>
+__device__ __forceinline__ void stream_blocks(const CUtensorMap *tm, int64_t total_blocks, uint32_t *status, F &&f,
+                                              P &&pre = P())
 {
     using Cfg = StreamCfg<T>;
     extern __shared__ uint8_t stream_smem_raw[];
@@ -95,6 +102,7 @@ __device__ __forceinline__ void stream_blocks(const CUtensorMap *tm, int64_t tot
         }
         __syncwarp();
     } else {
+        pre(threadIdx.x);
         int it = 0;
         for (int64_t c = blockIdx.x; c < chunks; c += gridDim.x, ++it) {
             const int st = it % Cfg::kStages;
@@ -150,6 +158,49 @@ __global__ void __launch_bounds__(kStreamThreads) absmax_rot_kernel(const __grid
 }
 
 // ---------------------------------------------------------------------------
+// low-rank operands of the forward's extra MMA step.  With beta = g_x g_w (1
+// when either scale is absent or the product is 0): tt = t / beta,
+// tsplit[m] = [bf16(tt) | bf16(tt - bf16(tt))] (bf16 [M, 64]), and
+// udup[n] = [U[n] | U[n]] (bf16 [N, 64]).
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ float lowrank_beta(float g_x, const float *g_w)
+{
+    if (!g_w)
+        return 1.0f;
+    const float b = __fmul_rn(g_x, *g_w);
+    return b == 0.0f ? 1.0f : b;
+}
+
+// unit i < M*8: t[m, 4c..4c+3] -> both halves of tsplit[m] (m = i/8, c = i%8);
+// unit i >= M*8: 16-byte chunk c of U[n] -> both halves of udup[n] (n, c from i - M*8)
+__device__ __forceinline__ void lowrank_unit(int64_t i, int64_t nT, const float *__restrict__ t32, float beta,
+                                             uint16_t *__restrict__ tsplit, const uint16_t *__restrict__ U,
+                                             uint16_t *__restrict__ udup)
+{
+    if (i < nT) {
+        const int64_t m = i >> 3, c = i & 7;
+        const float4 t4 = *reinterpret_cast<const float4 *>(t32 + m * kRank + 4 * c);
+        const float tv[4] = {t4.x, t4.y, t4.z, t4.w};
+        uint32_t hi[4], lo[4];
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+            const float tt = __fdiv_rn(tv[k], beta);
+            hi[k] = f32_to_bf16_bits(tt);
+            lo[k] = f32_to_bf16_bits(__fsub_rn(tt, bf16_bits_to_f32(hi[k])));
+        }
+        *reinterpret_cast<uint2 *>(tsplit + m * 64 + 4 * c) = make_uint2(hi[0] | (hi[1] << 16), hi[2] | (hi[3] << 16));
+        *reinterpret_cast<uint2 *>(tsplit + m * 64 + 32 + 4 * c) =
+            make_uint2(lo[0] | (lo[1] << 16), lo[2] | (lo[3] << 16));
+    } else {
+        const int64_t j = i - nT;
+        const int64_t n = j >> 2, c = j & 3;
+        const uint4 u = *reinterpret_cast<const uint4 *>(U + n * kRank + 8 * c);
+        *reinterpret_cast<uint4 *>(udup + n * 64 + 8 * c) = u;
+        *reinterpret_cast<uint4 *>(udup + n * 64 + 32 + 8 * c) = u;
+    }
+}
+
+// ---------------------------------------------------------------------------
 // NVFP4 block quantisation of H in with global scale g, over rows_pad rows
 // (a multiple of 128): rows past `rows` are zero and only their scale bytes
 // are written (as 0), which fills the tiled layout's padding.  g comes from
@@ -164,7 +215,7 @@ __global__ void __launch_bounds__(kStreamThreads) nvfp4_quant_kernel(const __gri
                                                                      const float *__restrict__ g_static,
                                                                      float *__restrict__ g_out,
                                                                      uint8_t *__restrict__ codes,
-                                                                     uint8_t *__restrict__ sf)
+                                                                     uint8_t *__restrict__ sf, LowrankOut lr)
 {
     const int lane = threadIdx.x & 31;
     const int q = lane & 7;
@@ -175,6 +226,16 @@ __global__ void __launch_bounds__(kStreamThreads) nvfp4_quant_kernel(const __gri
     const int64_t kb_per_row = K / kHad;
     const int64_t C = K / kSfBlock;
     const bool idx32 = rows_pad * kb_per_row <= (int64_t)UINT32_MAX;
+    // the forward's low-rank operands (g is final here), done while the first chunks load
+    auto lowrank = [&](int c) {
+        if (!lr.t32)
+            return;
+        const float beta = lowrank_beta(g, lr.g_w);
+        const int64_t nT = rows * 8, total = nT + lr.N * 4;
+        const int64_t stride = (int64_t)gridDim.x * (32 * kStreamConsumers);
+        for (int64_t i = (int64_t)blockIdx.x * (32 * kStreamConsumers) + c; i < total; i += stride)
+            lowrank_unit(i, nT, lr.t32, beta, lr.tsplit, lr.U, lr.udup);
+    };
     stream_blocks<T>(&tm, rows_pad * kb_per_row, nullptr, [&](int64_t b, float (&v)[32], bool valid) {
         fwht256_l32(v, lane);
         if (!valid)
@@ -215,7 +276,7 @@ __global__ void __launch_bounds__(kStreamThreads) nvfp4_quant_kernel(const __gri
         // scale columns 2q, 2q+1 of the block are adjacent bytes of the tiled layout
         *reinterpret_cast<uint16_t *>(sf + sf_offset(row, kb * (kHad / kSfBlock) + 2 * q, C)) =
             (uint16_t)(sfc[0] | (sfc[1] << 8));
-    });
+    }, lowrank);
 }
 
 // ---------------------------------------------------------------------------
@@ -587,10 +648,8 @@ __global__ void __launch_bounds__(256, 2) act_pass1_kernel(const uint16_t *__res
 }
 
 // ---------------------------------------------------------------------------
-// low-rank operands of the forward's extra MMA step.  With beta = g_x g_w (1
-// when either pointer is NULL or the product is 0): tt = t / beta,
-// tsplit[m] = [bf16(tt) | bf16(tt - bf16(tt))] (bf16 [M, 64]), and
-// udup[n] = [U[n] | U[n]] (bf16 [N, 64]).
+// low-rank operands as a kernel of their own (the int4 forward; see
+// lowrank_unit).  g_x NULL means beta = 1.
 // ---------------------------------------------------------------------------
 __global__ void __launch_bounds__(256) lowrank_finish_kernel(const float *__restrict__ t32, int64_t M,
                                                              const float *__restrict__ g_x,
@@ -599,29 +658,11 @@ __global__ void __launch_bounds__(256) lowrank_finish_kernel(const float *__rest
                                                              const uint16_t *__restrict__ U, int64_t N,
                                                              uint16_t *__restrict__ udup)
 {
-    float beta = 1.0f;
-    if (g_x && g_w) {
-        const float b = __fmul_rn(*g_x, *g_w);
-        beta = b == 0.0f ? 1.0f : b;
-    }
-    const int64_t nT = M * kRank, nU = N * kRank;
-    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < nT + nU;
-         i += (int64_t)gridDim.x * blockDim.x) {
-        if (i < nT) {
-            const int64_t m = i >> 5, col = i & 31;
-            const float tt = __fdiv_rn(t32[i], beta);
-            const uint32_t hi = f32_to_bf16_bits(tt);
-            const uint32_t lo = f32_to_bf16_bits(__fsub_rn(tt, bf16_bits_to_f32(hi)));
-            tsplit[m * 64 + col] = (uint16_t)hi;
-            tsplit[m * 64 + 32 + col] = (uint16_t)lo;
-        } else {
-            const int64_t j = i - nT;
-            const int64_t n = j >> 5, col = j & 31;
-            const uint16_t u = U[j];
-            udup[n * 64 + col] = u;
-            udup[n * 64 + 32 + col] = u;
-        }
-    }
+    const float beta = g_x ? lowrank_beta(*g_x, g_w) : 1.0f;
+    const int64_t nT = M * 8;
+    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < nT + N * 4;
+         i += (int64_t)gridDim.x * blockDim.x)
+        lowrank_unit(i, nT, t32, beta, tsplit, U, udup);
 }
 
 // ---------------------------------------------------------------------------
@@ -945,7 +986,8 @@ static cudaError_t launch_absmax_rot(const T *in, int64_t rows, int64_t K, uint3
 
 template <typename T>
 static cudaError_t launch_nvfp4_quant(const T *in, int64_t rows, int64_t K, const uint32_t *amax, const float *g_static,
-                                      float *g_out, uint8_t *codes, uint8_t *sf, int sms, cudaStream_t s)
+                                      float *g_out, uint8_t *codes, uint8_t *sf, const LowrankOut &lr, int sms,
+                                      cudaStream_t s)
 {
     CUtensorMap tm;
     if (!stream_map(&tm, in, rows, K))
@@ -955,7 +997,7 @@ static cudaError_t launch_nvfp4_quant(const T *in, int64_t rows, int64_t K, cons
         return e;
     const int64_t rows_pad = (rows + 127) / 128 * 128;
     nvfp4_quant_kernel<T><<<stream_grid(rows_pad * (K / kHad), sms, sizeof(T) == 4 ? 2 : 3), kStreamThreads,
-                            StreamCfg<T>::kSmem, s>>>(tm, rows, rows_pad, K, amax, g_static, g_out, codes, sf);
+                            StreamCfg<T>::kSmem, s>>>(tm, rows, rows_pad, K, amax, g_static, g_out, codes, sf, lr);
     return cudaGetLastError();
 }
 
@@ -974,14 +1016,14 @@ cudaError_t launch_nvfp4_quant_f32(const float *in, int64_t rows, int64_t K, con
                                    const float *g_static, float *g_out, uint8_t *codes, uint8_t *sf, int sms,
                                    cudaStream_t s)
 {
-    return launch_nvfp4_quant(in, rows, K, amax, g_static, g_out, codes, sf, sms, s);
+    return launch_nvfp4_quant(in, rows, K, amax, g_static, g_out, codes, sf, LowrankOut{}, sms, s);
 }
 
 cudaError_t launch_nvfp4_quant_bf16(const uint16_t *in, int64_t rows, int64_t K, const uint32_t *amax,
-                                    const float *g_static, float *g_out, uint8_t *codes, uint8_t *sf, int sms,
-                                    cudaStream_t s)
+                                    const float *g_static, float *g_out, uint8_t *codes, uint8_t *sf,
+                                    const LowrankOut &lr, int sms, cudaStream_t s)
 {
-    return launch_nvfp4_quant(in, rows, K, amax, g_static, g_out, codes, sf, sms, s);
+    return launch_nvfp4_quant(in, rows, K, amax, g_static, g_out, codes, sf, lr, sms, s);
 }
 
 cudaError_t launch_int4_build(const float *R, int64_t N, int64_t K, uint8_t *codes, uint16_t *scales,
@@ -1065,7 +1107,7 @@ cudaError_t launch_lowrank_finish(const float *t32, int64_t M, const float *g_x,
                                   uint16_t *tsplit, const uint16_t *U, int64_t N, uint16_t *udup, int sms,
                                   cudaStream_t s)
 {
-    lowrank_finish_kernel<<<grid_for((M + N) * kRank, 256, sms, 4), 256, 0, s>>>(t32, M, g_x, g_w, tsplit, U, N,
+    lowrank_finish_kernel<<<grid_for(M * 8 + N * 4, 256, sms, 4), 256, 0, s>>>(t32, M, g_x, g_w, tsplit, U, N,
                                                                                   udup);
     return cudaGetLastError();
 }
