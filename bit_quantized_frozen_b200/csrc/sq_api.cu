@@ -275,7 +275,8 @@ sq_status sq_act_quant_nvfp4(const uint16_t *x, int64_t M, int64_t K, uint8_t *c
     uint32_t *amax = reinterpret_cast<uint32_t *>(ws_at(ws, 4));
     SQ_CUDA(cudaMemsetAsync(ws, 0, 8, s), "memset");          // status word + absmax
     if (!stat || with_t)
-        SQ_CUDA(sq::launch_act_pass1(x, M, K, lora_down, stat ? nullptr : amax, with_t ? t : nullptr, sms, s),
+        SQ_CUDA(sq::launch_act_pass1(x, M, K, lora_down, stat ? nullptr : amax, with_t ? t : nullptr,
+                                             reinterpret_cast<uint32_t *>(ws), sms, s),
                 "activation pass 1");
     SQ_CUDA(sq::launch_nvfp4_quant_bf16(x, M, K, amax, stat ? g_x : nullptr, stat ? nullptr : g_x, codes, sf_tiled,
                                         sq::LowrankOut{}, sms, s),
@@ -331,7 +332,8 @@ sq_status sq_linear_fwd(const sq_weight *w, const uint16_t *x, int64_t M, float 
         uint8_t *xsf = ws_at(ws, L.a_sf);
         // one read of x for the absmax and the low-rank input, one for the quantisation
         if (!stat || lora)
-            SQ_CUDA(sq::launch_act_pass1(x, M, K, w->lora_down, stat ? nullptr : amax, t32, sms, s), "activation pass 1");
+            SQ_CUDA(sq::launch_act_pass1(x, M, K, w->lora_down, stat ? nullptr : amax, t32, status, sms, s),
+                    "activation pass 1");
         // the quantisation also writes the low-rank operands (g_x is known by then)
         sq::LowrankOut lr;
         if (lora) {
@@ -359,7 +361,7 @@ sq_status sq_linear_fwd(const sq_weight *w, const uint16_t *x, int64_t M, float 
         SQ_CUDA(sq::launch_dequant_int4(w->codes, reinterpret_cast<const uint16_t *>(w->scales), N, K, wb, sms, s),
                 "dequant");
         if (lora) {
-            SQ_CUDA(sq::launch_act_pass1(x, M, K, w->lora_down, nullptr, t32, sms, s), "low-rank input");
+            SQ_CUDA(sq::launch_act_pass1(x, M, K, w->lora_down, nullptr, t32, status, sms, s), "low-rank input");
             SQ_CUDA(sq::launch_lowrank_finish(t32, M, nullptr, nullptr, tsplit, w->lora_up, N, udup, sms, s),
                     "low-rank operands");
         }

@@ -34,7 +34,7 @@ cudaError_t launch_rotate_bf16(const uint16_t *x, int64_t M, int64_t K, uint16_t
 cudaError_t launch_dequant_int4(const uint8_t *codes, const uint16_t *scales, int64_t N, int64_t K, uint16_t *wb,
                                 int sms, cudaStream_t s);
 cudaError_t launch_act_pass1(const uint16_t *x, int64_t M, int64_t K, const uint16_t *D, uint32_t *amax,
-                             float *t32, int sms, cudaStream_t s);
+                             float *t32, uint32_t *status, int sms, cudaStream_t s);
 cudaError_t launch_lowrank_finish(const float *t32, int64_t M, const float *g_x, const float *g_w,
                                   uint16_t *tsplit, const uint16_t *U, int64_t N, uint16_t *udup, int sms,
                                   cudaStream_t s);

@@ -416,19 +416,20 @@ __global__ void __launch_bounds__(256) dequant_int4_kernel(const uint32_t *__res
 // A CTA owns 32 rows and a range of 256-column chunks; when there are few row
 // tiles, K is split over a cluster of `split` CTAs (one per range) whose
 // partial t tiles are summed in rank order by rank 0 through distributed
-// shared memory.  The x chunk (32 x 256) and the lora_down chunk (256 x 32)
-// are staged by cp.async in a 3-deep ring.  Every warp transforms 4 rows and
-// runs 4 of the chunk's 16 k-steps for one 16-row half of the tile.
-// x tile: 16-byte chunk c of row r sits at c ^ ((c >> 2) & 7) ^ (r & 7), which
-// keeps both the transform's per-row reads and ldmatrix conflict free; D tile:
-// chunk c of k-row k sits at c ^ ((k >> 1) & 3).
+// shared memory.  One producer warp streams each chunk -- the x tile (32 x 256,
+// four TMA boxes of 64 columns, 128-byte swizzle) and the lora_down tile
+// (256 x 32, one box, 64-byte swizzle) -- into a 3-deep ring with mbarriers;
+// every consumer warp transforms 4 rows and runs 4 of the chunk's 16 k-steps
+// for one 16-row half of the tile, then releases the stage on its own.
 // ---------------------------------------------------------------------------
 constexpr int kP1Rows = 32;
 constexpr int kP1XBytes = kP1Rows * kHad * 2;      // 16 KB
 constexpr int kP1DBytes = kHad * kRank * 2;        // 16 KB
 constexpr int kP1BufBytes = kP1XBytes + kP1DBytes;
 constexpr int kP1Stages = 3;
-constexpr int kP1Smem = kP1Stages * kP1BufBytes;   // 96 KB
+constexpr int kP1Consumers = 8;
+constexpr int kP1Threads = 32 * (kP1Consumers + 1);
+constexpr int kP1Smem = kP1Stages * kP1BufBytes + 1024 + 256;   // ring, 1 KB alignment, barriers
 constexpr int kP1MaxSplit = 8;
 
 __device__ __forceinline__ void cp_async16(uint32_t dst, const void *src, uint32_t src_bytes)
@@ -467,11 +468,13 @@ __device__ __forceinline__ void mma_bf16_16816(float (&c)[4], const uint32_t (&a
                  : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
 }
 
+// x stage: 16-byte chunk c (0..31) of row r -- box c / 8, 128-byte swizzle
 __device__ __forceinline__ uint32_t p1_xoff(int r, int c)
 {
-    return (uint32_t)(r * 512 + 16 * (c ^ ((c >> 2) & 7) ^ (r & 7)));
+    return (uint32_t)((c >> 3) * 4096 + r * 128 + 16 * ((c & 7) ^ (r & 7)));
 }
 
+// lora_down stage: 16-byte chunk c (0..3) of k-row k -- 64-byte swizzle
 __device__ __forceinline__ uint32_t p1_doff(int k, int c)
 {
     return (uint32_t)(k * 64 + 16 * (c ^ ((k >> 1) & 3)));
@@ -484,12 +487,18 @@ __device__ __forceinline__ float ld_shared_cluster_f32(uint32_t addr)
     return v;
 }
 
-__global__ void __launch_bounds__(256, 2) act_pass1_kernel(const uint16_t *__restrict__ x, int64_t M, int64_t K,
-                                                           const uint16_t *__restrict__ D,
-                                                           uint32_t *__restrict__ amax, float *__restrict__ t32,
-                                                           int split)
+__global__ void __launch_bounds__(kP1Threads, 2) act_pass1_kernel(const __grid_constant__ CUtensorMap tmx,
+                                                                  const __grid_constant__ CUtensorMap tmd,
+                                                                  int64_t M, int64_t K, uint32_t *__restrict__ amax,
+                                                                  float *__restrict__ t32, int split,
+                                                                  uint32_t *__restrict__ status)
 {
-    extern __shared__ __align__(128) uint8_t p1_smem[];
+    extern __shared__ uint8_t p1_raw[];
+    uint8_t *p1_smem =
+        reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(p1_raw) + 1023) & ~uintptr_t(1023));
+    uint64_t *bars = reinterpret_cast<uint64_t *>(p1_smem + kP1Stages * kP1BufBytes);
+    const uint32_t full = smem_u32(bars), empty = smem_u32(bars + kP1Stages);
+    volatile uint32_t *abort_flag = reinterpret_cast<uint32_t *>(bars + 2 * kP1Stages);
     const int tid = threadIdx.x;
     const int lane = tid & 31;
     const int warp = tid >> 5;
@@ -498,29 +507,16 @@ __global__ void __launch_bounds__(256, 2) act_pass1_kernel(const uint16_t *__res
     const int nkb = (int)(K / kHad);
     const int kb0 = (int)((int64_t)j * nkb / split);
     const int nch = (int)((int64_t)(j + 1) * nkb / split) - kb0;
-    const uint32_t sbase = (uint32_t)__cvta_generic_to_shared(p1_smem);
-
-    auto issue = [&](int kb, int buf) {
-        const uint32_t xs = sbase + buf * kP1BufBytes;
-        const uint32_t ds = xs + kP1XBytes;
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {                 // x: 32 rows x 32 chunks
-            const int e = tid + 256 * i;
-            const int r = e >> 5, c = e & 31;
-            const int64_t row = m0 + r;
-            const bool ok = row < M;
-            const uint16_t *src = x + (ok ? row : 0) * K + (int64_t)kb * kHad + 8 * c;
-            cp_async16(xs + p1_xoff(r, c), src, ok ? 16u : 0u);
+    const uint32_t sbase = smem_u32(p1_smem);
+    if (tid == 0) {
+        for (int st = 0; st < kP1Stages; ++st) {
+            mbar_init(full + 8 * st, 1);
+            mbar_init(empty + 8 * st, kP1Consumers);
         }
-        if (t32) {
-#pragma unroll
-            for (int i = 0; i < 4; ++i) {             // D: 256 k-rows x 4 chunks
-                const int e = tid + 256 * i;
-                const int k = e >> 2, c = e & 3;
-                cp_async16(ds + p1_doff(k, c), D + ((int64_t)kb * kHad + k) * kRank + 8 * c, 16u);
-            }
-        }
-    };
+        *abort_flag = 0u;
+        fence_mbar_init();
+    }
+    __syncthreads();
 
     float m = 0.0f;
     float acc[4][4];
@@ -530,63 +526,94 @@ __global__ void __launch_bounds__(256, 2) act_pass1_kernel(const uint16_t *__res
         for (int i = 0; i < 4; ++i)
             acc[nt][i] = 0.0f;
 
+    if (warp == kP1Consumers) {                       // producer
+        if (lane == 0) {
+            prefetch_tmap(&tmx);
+            if (t32)
+                prefetch_tmap(&tmd);
+            for (int c = 0; c < nch; ++c) {
+                const int st = c % kP1Stages;
+                const uint32_t ph = (uint32_t)(c / kP1Stages) & 1u;
+                if (!mbar_wait(empty + 8 * st, ph ^ 1u, abort_flag, status))
+                    break;
+                mbar_arrive_expect_tx(full + 8 * st, t32 ? kP1BufBytes : kP1XBytes);
+                const uint32_t xs = sbase + st * kP1BufBytes;
+                const int kb = kb0 + c;
 #pragma unroll
-    for (int c = 0; c < kP1Stages - 1; ++c) {
-        if (c < nch)
-            issue(kb0 + c, c);
-        cp_async_commit();                            // (possibly empty) group c
-    }
-    const int mt = warp >> 2;                         // MMA: rows 16mt..16mt+15
-#pragma unroll 1
-    for (int c = 0; c < nch; ++c) {
-        cp_async_wait<kP1Stages - 2>();               // chunk c has landed (this thread's copies)
-        __syncthreads();                              // ... everyone's; stage of chunk c-1 is free
-        if (c + kP1Stages - 1 < nch)
-            issue(kb0 + c + kP1Stages - 1, (c + kP1Stages - 1) % kP1Stages);
-        cp_async_commit();
-        const int buf = c % kP1Stages;
-        const uint32_t xs = sbase + buf * kP1BufBytes;
-        const uint32_t ds = xs + kP1XBytes;
-        if (amax) {
-            const int r = 4 * warp + (lane >> 3);
-            const int q = lane & 7;
-            float v[32];
-#pragma unroll
-            for (int i = 0; i < 4; ++i) {
-                const uint4 a = *reinterpret_cast<const uint4 *>(p1_smem + (p1_xoff(r, 4 * q + i) +
-                                                                             buf * kP1BufBytes));
-                const uint32_t w[4] = {a.x, a.y, a.z, a.w};
-#pragma unroll
-                for (int jj = 0; jj < 4; ++jj) {
-                    v[8 * i + 2 * jj] = __uint_as_float(w[jj] << 16);
-                    v[8 * i + 2 * jj + 1] = __uint_as_float(w[jj] & 0xFFFF0000u);
-                }
-            }
-            fwht256_l32<false>(v, lane);
-#pragma unroll
-            for (int i = 0; i < 32; ++i)
-                m = fmaxf(m, fabsf(v[i]));
-        }
-        if (t32) {
-#pragma unroll
-            for (int ss = 0; ss < 4; ++ss) {
-                const int ks = 4 * (warp & 3) + ss;   // k-step: columns 16ks..16ks+15 of the chunk
-                // A 16x16: matrices (rows 0-7 | 8-15) x (k 0-7 | 8-15); lane provides row (lane & 15)
-                uint32_t a[4];
-                ldmatrix_x4(xs + p1_xoff(16 * mt + (lane & 15), 2 * ks + (lane >> 4)), a);
-                // B: (k 0-7 | 8-15) x (n-tile pair), transposed load of row-major D
-#pragma unroll
-                for (int np = 0; np < 2; ++np) {
-                    uint32_t b[4];
-                    const int bk = 16 * ks + (lane & 7) + 8 * ((lane >> 3) & 1);
-                    ldmatrix_x4_trans(ds + p1_doff(bk, 2 * np + (lane >> 4)), b);
-                    mma_bf16_16816(acc[2 * np], a, b[0], b[1]);
-                    mma_bf16_16816(acc[2 * np + 1], a, b[2], b[3]);
-                }
+                for (int b = 0; b < 4; ++b)
+                    tma_load_2d(xs + 4096 * b, &tmx, kb * kHad + 64 * b, (int32_t)m0, full + 8 * st);
+                if (t32)
+                    tma_load_2d(xs + kP1XBytes, &tmd, 0, kb * kHad, full + 8 * st);
             }
         }
+        __syncwarp();
+    } else {
+        const int mt = warp >> 2;                     // MMA: rows 16mt..16mt+15
+        for (int c = 0; c < nch; ++c) {
+            const int st = c % kP1Stages;
+            const uint32_t ph = (uint32_t)(c / kP1Stages) & 1u;
+            int ok = 1;
+            if (lane == 0)
+                ok = mbar_wait(full + 8 * st, ph, abort_flag, status) ? 1 : 0;
+            if (__shfl_sync(0xffffffffu, ok, 0) == 0)
+                break;
+            const uint32_t xs = sbase + st * kP1BufBytes;
+            const uint32_t ds = xs + kP1XBytes;
+            if (amax) {
+                const int r = 4 * warp + (lane >> 3);
+                const int q = lane & 7;
+                const int sb = q >> 1;                // box of this lane's 32 values
+                // read chunk (i + sb) & 3 of the lane's four at step i (the 8 lanes of a
+                // row then hit 8 different banks), then rotate back by sb
+                const uint8_t *rowp = p1_smem + st * kP1BufBytes + sb * 4096 + r * 128;
+                uint4 tmp[4], rot[4], ch[4];
+#pragma unroll
+                for (int i = 0; i < 4; ++i)
+                    tmp[i] = *reinterpret_cast<const uint4 *>(rowp + 16 * ((4 * (q & 1) + ((i + sb) & 3)) ^ (r & 7)));
+#pragma unroll
+                for (int i = 0; i < 4; ++i)
+                    rot[i] = (sb & 1) ? tmp[(i + 3) & 3] : tmp[i];
+#pragma unroll
+                for (int i = 0; i < 4; ++i)
+                    ch[i] = (sb & 2) ? rot[(i + 2) & 3] : rot[i];
+                float v[32];
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    const uint32_t w[4] = {ch[i].x, ch[i].y, ch[i].z, ch[i].w};
+#pragma unroll
+                    for (int jj = 0; jj < 4; ++jj) {
+                        v[8 * i + 2 * jj] = __uint_as_float(w[jj] << 16);
+                        v[8 * i + 2 * jj + 1] = __uint_as_float(w[jj] & 0xFFFF0000u);
+                    }
+                }
+                fwht256_l32<false>(v, lane);
+#pragma unroll
+                for (int i = 0; i < 32; ++i)
+                    m = fmaxf(m, fabsf(v[i]));
+            }
+            if (t32) {
+#pragma unroll
+                for (int ss = 0; ss < 4; ++ss) {
+                    const int ks = 4 * (warp & 3) + ss;   // k-step: columns 16ks..16ks+15 of the chunk
+                    // A 16x16: matrices (rows 0-7 | 8-15) x (k 0-7 | 8-15); lane provides row (lane & 15)
+                    uint32_t a[4];
+                    ldmatrix_x4(xs + p1_xoff(16 * mt + (lane & 15), 2 * ks + (lane >> 4)), a);
+                    // B: (k 0-7 | 8-15) x (n-tile pair), transposed load of row-major D
+#pragma unroll
+                    for (int np = 0; np < 2; ++np) {
+                        uint32_t b[4];
+                        const int bk = 16 * ks + (lane & 7) + 8 * ((lane >> 3) & 1);
+                        ldmatrix_x4_trans(ds + p1_doff(bk, 2 * np + (lane >> 4)), b);
+                        mma_bf16_16816(acc[2 * np], a, b[0], b[1]);
+                        mma_bf16_16816(acc[2 * np + 1], a, b[2], b[3]);
+                    }
+                }
+            }
+            __syncwarp();
+            if (lane == 0)
+                mbar_arrive(empty + 8 * st);
+        }
     }
-    cp_async_wait<0>();
     __syncthreads();                                  // ring idle: reuse it below
 
     if (amax) {
@@ -597,8 +624,8 @@ __global__ void __launch_bounds__(256, 2) act_pass1_kernel(const uint16_t *__res
     }
     float *part = reinterpret_cast<float *>(p1_smem);          // [8 warps][16][33]
     float *tcta = part + 8 * 16 * 33;                           // [32][32] this CTA's t tile
-    float *wmax = tcta + kP1Rows * kRank;                       // [8]
-    if (t32) {
+    float *wmax = tcta + kP1Rows * kRank;                       // [9]
+    if (t32 && warp < kP1Consumers) {
         const int g = lane >> 2, tq = lane & 3;
 #pragma unroll
         for (int nt = 0; nt < 4; ++nt) {
@@ -613,13 +640,13 @@ __global__ void __launch_bounds__(256, 2) act_pass1_kernel(const uint16_t *__res
     __syncthreads();
     if (amax && tid == 0) {
         float b = 0.0f;
-        for (int w = 0; w < 8; ++w)
+        for (int w = 0; w < kP1Consumers; ++w)
             b = fmaxf(b, wmax[w]);
         atomic_max_nonneg(amax, b);
     }
     if (!t32)
         return;
-    for (int e = tid; e < kP1Rows * kRank; e += 256) {          // k-step partials, fixed order
+    for (int e = tid; e < kP1Rows * kRank; e += kP1Threads) {   // k-step partials, fixed order
         const int r = e >> 5, col = e & 31;
         const int h = r >> 4, rr = r & 15;
         float v = 0.0f;
@@ -634,7 +661,7 @@ __global__ void __launch_bounds__(256, 2) act_pass1_kernel(const uint16_t *__res
         __syncthreads();
     if (j == 0) {
         const uint32_t tl = (uint32_t)__cvta_generic_to_shared(tcta);
-        for (int e = tid; e < kP1Rows * kRank; e += 256) {
+        for (int e = tid; e < kP1Rows * kRank; e += kP1Threads) {
             const int64_t row = m0 + (e >> 5);
             float v = tcta[e];
             for (int rk = 1; rk < split; ++rk)
@@ -1064,7 +1091,7 @@ cudaError_t launch_dequant_int4(const uint8_t *codes, const uint16_t *scales, in
 }
 
 cudaError_t launch_act_pass1(const uint16_t *x, int64_t M, int64_t K, const uint16_t *D, uint32_t *amax,
-                             float *t32, int sms, cudaStream_t s)
+                             float *t32, uint32_t *status, int sms, cudaStream_t s)
 {
     constexpr int kMaxDev = 64;
     static bool attr_done[kMaxDev];
@@ -1077,6 +1104,14 @@ cudaError_t launch_act_pass1(const uint16_t *x, int64_t M, int64_t K, const uint
             return e;
         attr_done[dev] = true;
     }
+    CUtensorMap tmx, tmd;
+    memset(&tmd, 0, sizeof(tmd));
+    if (!make_tmap(&tmx, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, x, (uint64_t)K, (uint64_t)M, 64, kP1Rows,
+                   CU_TENSOR_MAP_SWIZZLE_128B))
+        return cudaErrorInvalidValue;
+    if (t32 && !make_tmap(&tmd, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, D, (uint64_t)kRank, (uint64_t)K, kRank, kHad,
+                          CU_TENSOR_MAP_SWIZZLE_64B))
+        return cudaErrorInvalidValue;
     const int64_t tiles = (M + kP1Rows - 1) / kP1Rows;
     const int nkb = (int)(K / kHad);
     int64_t split = (2LL * sms) / tiles;              // two CTAs per SM
@@ -1085,12 +1120,12 @@ cudaError_t launch_act_pass1(const uint16_t *x, int64_t M, int64_t K, const uint
     split = split > nkb ? nkb : split;
     const unsigned grid = (unsigned)(tiles * split);
     if (split == 1) {
-        act_pass1_kernel<<<grid, 256, kP1Smem, s>>>(x, M, K, D, amax, t32, 1);
+        act_pass1_kernel<<<grid, kP1Threads, kP1Smem, s>>>(tmx, tmd, M, K, amax, t32, 1, status);
         return cudaGetLastError();
     }
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(grid);
-    cfg.blockDim = dim3(256);
+    cfg.blockDim = dim3(kP1Threads);
     cfg.dynamicSmemBytes = kP1Smem;
     cfg.stream = s;
     cudaLaunchAttribute at[1];
@@ -1100,7 +1135,7 @@ cudaError_t launch_act_pass1(const uint16_t *x, int64_t M, int64_t K, const uint
     at[0].val.clusterDim.z = 1;
     cfg.attrs = at;
     cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, act_pass1_kernel, x, M, K, D, amax, t32, (int)split);
+    return cudaLaunchKernelEx(&cfg, act_pass1_kernel, tmx, tmd, M, K, amax, t32, (int)split, status);
 }
 
 cudaError_t launch_lowrank_finish(const float *t32, int64_t M, const float *g_x, const float *g_w,
