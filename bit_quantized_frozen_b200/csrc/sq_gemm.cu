@@ -22,11 +22,14 @@
 //   warps 6-9  (NVFP4) move each MMA's ue4m3 scale factors from shared memory
 //              into tensor memory with tcgen05.st, one 32-lane sub-partition
 //              per warp, so the tensor pipe spends no cycles on copies.
-// Tensor memory (512 columns): two accumulator slots at columns 0 and 96
-// that overlap in columns 96..255, and three 48-column scale-factor buffers at
-// 352..495 (NVFP4).  The epilogue reads the overlapping 160 columns of a tile
-// first and then releases the MMA thread, which starts the next tile while
-// the other 96 columns drain -- accumulator double buffering in 352 columns.
+// Tensor memory (512 columns): two accumulator slots at columns 0 and 64
+// that overlap in columns 64..255, and four 48-column scale-factor buffers at
+// 320..511 (NVFP4: four stages of scale factors between the scale warps and
+// the MMAs that read them).  The epilogue takes the overlapping 192 columns
+// of a tile first -- four chunks into registers, two of them parked in its
+// staging buffers, then the last two -- and releases the MMA thread, which
+// starts the next tile while the rest drains: accumulator double buffering
+// in 320 columns.
 #include <cuda.h>
 
 #include "sq_device.cuh"
@@ -47,12 +50,11 @@ constexpr int kSfbBytes = 2 * kSfaBytes;       // both 128-row halves of B (ever
 constexpr int kEpiWarps = 4;
 constexpr int kStagingBytes = 32 * 128;        // one warp's 32 rows x 32 fp32
 constexpr uint32_t kTmemCols = 512;
-constexpr uint32_t kAccSlot1 = 96;             // accumulator slots [0, 256) and [96, 352)
-constexpr int kOverlapChunks = 5;              // 32-column chunks shared by the two slots
-constexpr uint32_t kSfCol = 352;               // ring of three scale-factor buffers, one stage (4 MMAs) each
-constexpr int kMmaPerSfBuf = 4;
+constexpr uint32_t kAccSlot1 = 64;             // accumulator slots [0, 256) and [64, 320)
+constexpr int kOverlapChunks = 6;              // 32-column chunks shared by the two slots
+constexpr uint32_t kSfCol = 320;               // ring of four scale-factor buffers, one stage (4 MMAs) each
 constexpr uint32_t kSfBufCols = 48;            // SFB for MMA k at +8k (256 rows), SFA at +32+4k (128 rows)
-constexpr uint32_t kSfBufs = 3;
+constexpr uint32_t kSfBufs = 4;
 
 // instruction descriptors: M = 256 (the CTA pair), N = 256, K-major A and B
 constexpr uint32_t kIdescBf16 = (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(BN >> 3) << 17) |
@@ -103,15 +105,10 @@ __device__ __forceinline__ bool warp_wait_cluster(uint32_t bar, uint32_t parity,
     return __shfl_sync(0xffffffffu, ok, 0) != 0;
 }
 
-// scale one 32-row x 32-column accumulator chunk and TMA-store it through a
-// 128B-swizzled staging buffer (two per warp, used alternately)
-__device__ __forceinline__ void store_chunk(const uint32_t (&r)[32], float beta, uint8_t *staging, int sb, int lane,
-                                            const CUtensorMap *tmY, int x, int y)
+// scale one 32-row x 32-column accumulator chunk into 128B-swizzled staging
+// buffer sb of the warp (the caller made sure the buffer is free)
+__device__ __forceinline__ void stage_chunk(const uint32_t (&r)[32], float beta, uint8_t *staging, int sb, int lane)
 {
-    // staging buffer sb is free once at most one store group is pending
-    if (lane == 0)
-        bulk_wait_group_read1();
-    __syncwarp();
     uint8_t *buf = staging + sb * kStagingBytes;
 #pragma unroll
     for (int j = 0; j < 8; ++j) {
@@ -122,12 +119,28 @@ __device__ __forceinline__ void store_chunk(const uint32_t (&r)[32], float beta,
         o.w = __fmul_rn(__uint_as_float(r[4 * j + 3]), beta);
         *reinterpret_cast<float4 *>(buf + lane * 128 + ((j ^ (lane & 7)) << 4)) = o;
     }
+}
+
+// TMA-store staging buffer sb (written by the whole warp) to y at (x, y)
+__device__ __forceinline__ void issue_store(uint8_t *staging, int sb, int lane, const CUtensorMap *tmY, int x, int y)
+{
     fence_proxy_async_smem();
     __syncwarp();
     if (lane == 0) {
-        tma_store_2d(tmY, smem_u32(buf), x, y);
+        tma_store_2d(tmY, smem_u32(staging + sb * kStagingBytes), x, y);
         bulk_commit_group();
     }
+}
+
+// stage + store a chunk through buffer sb, once at most one earlier store is pending
+__device__ __forceinline__ void store_chunk(const uint32_t (&r)[32], float beta, uint8_t *staging, int sb, int lane,
+                                            const CUtensorMap *tmY, int x, int y)
+{
+    if (lane == 0)
+        bulk_wait_group_read1();
+    __syncwarp();
+    stage_chunk(r, beta, staging, sb, lane);
+    issue_store(staging, sb, lane, tmY, x, y);
 }
 
 template <bool FP4>
@@ -415,7 +428,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(GemmCfg<FP4>::kThrea
         }
         const uint32_t acc_empty_leader = mapa_shared(bar_acc_empty, 0);
         uint8_t *staging = smem + Cfg::kStagingOff + warp * 2 * kStagingBytes;
-        int sb = 0;
         int count = 0;
         for (int tile = cluster_id; tile < tiles; tile += clusters, ++count) {
             const int mt = tile % m_tiles, nt = tile / m_tiles;
@@ -427,35 +439,44 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(GemmCfg<FP4>::kThrea
             tc_fence_after();
             const uint32_t acc = tmem_base + ((uint32_t)(32 * warp) << 16) + (slot ? kAccSlot1 : 0u);
             const bool rows_live = m0 + 32 * warp < args.M;       // skip stores wholly below the matrix
-            // the chunks this slot shares with the other one are read first, in one
-            // batch, so the leader can start the next tile as early as possible
-            const int first = slot ? 0 : 8 - kOverlapChunks;   // slot 0 shares its last 5 chunks
-            uint32_t r[kOverlapChunks][32];
-#pragma unroll
-            for (int q = 0; q < kOverlapChunks; ++q)
-                tmem_ld_32cols(acc + 32 * (first + q), r[q]);
+            // The six chunks this slot shares with the other one leave tensor memory
+            // first: four into registers, two of those parked in the (now free)
+            // staging buffers, then the last two; then the leader may start the next
+            // tile.  Chunk q of the tile is column block (first + q) % 8.
+            const int first = slot ? 0 : 8 - kOverlapChunks;   // slot 0 shares its last 6 chunks
+            const int ytop = m0 + 32 * warp;
+            if (lane == 0)
+                bulk_wait_group_read0();                       // both staging buffers free
+            __syncwarp();
+            uint32_t r0[32], r1[32], r2[32], r3[32];
+            tmem_ld_32cols(acc + 32 * ((first + 0) & 7), r0);
+            tmem_ld_32cols(acc + 32 * ((first + 1) & 7), r1);
+            tmem_ld_32cols(acc + 32 * ((first + 2) & 7), r2);
+            tmem_ld_32cols(acc + 32 * ((first + 3) & 7), r3);
+            tmem_wait_ld();
+            stage_chunk(r0, beta, staging, 0, lane);
+            stage_chunk(r1, beta, staging, 1, lane);
+            tmem_ld_32cols(acc + 32 * ((first + 4) & 7), r0);
+            tmem_ld_32cols(acc + 32 * ((first + 5) & 7), r1);
             tmem_wait_ld();
             tc_fence_before();
             __syncwarp();
             if (lane == 0)
                 mbar_arrive_cluster(acc_empty_leader);
             if (rows_live) {
-#pragma unroll
-                for (int q = 0; q < kOverlapChunks; ++q) {
-                    store_chunk(r[q], beta, staging, sb, lane, &tmY, n0 + 32 * (first + q), m0 + 32 * warp);
-                    sb ^= 1;
-                }
+                issue_store(staging, 0, lane, &tmY, n0 + 32 * ((first + 0) & 7), ytop);
+                issue_store(staging, 1, lane, &tmY, n0 + 32 * ((first + 1) & 7), ytop);
+                store_chunk(r2, beta, staging, 0, lane, &tmY, n0 + 32 * ((first + 2) & 7), ytop);
+                store_chunk(r3, beta, staging, 1, lane, &tmY, n0 + 32 * ((first + 3) & 7), ytop);
+                store_chunk(r0, beta, staging, 0, lane, &tmY, n0 + 32 * ((first + 4) & 7), ytop);
+                store_chunk(r1, beta, staging, 1, lane, &tmY, n0 + 32 * ((first + 5) & 7), ytop);
             }
-#pragma unroll 1
-            for (int q = kOverlapChunks; q < 8; ++q) {
-                const int c = (first + q) & 7;
-                uint32_t rr[32];
-                tmem_ld_32cols(acc + 32 * c, rr);
-                tmem_wait_ld();
-                if (rows_live) {
-                    store_chunk(rr, beta, staging, sb, lane, &tmY, n0 + 32 * c, m0 + 32 * warp);
-                    sb ^= 1;
-                }
+            tmem_ld_32cols(acc + 32 * ((first + 6) & 7), r2);
+            tmem_ld_32cols(acc + 32 * ((first + 7) & 7), r3);
+            tmem_wait_ld();
+            if (rows_live) {
+                store_chunk(r2, beta, staging, 0, lane, &tmY, n0 + 32 * ((first + 6) & 7), ytop);
+                store_chunk(r3, beta, staging, 1, lane, &tmY, n0 + 32 * ((first + 7) & 7), ytop);
             }
         }
         if (lane == 0)

@@ -181,6 +181,12 @@ __device__ __forceinline__ void bulk_commit_group()
     asm volatile("cp.async.bulk.commit_group;" ::: "memory");
 }
 
+// every committed bulk store group has finished reading shared memory
+__device__ __forceinline__ void bulk_wait_group_read0()
+{
+    asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
+}
+
 __device__ __forceinline__ void bulk_wait_group_read1()
 {
     asm volatile("cp.async.bulk.wait_group.read 1;" ::: "memory");
