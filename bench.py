@@ -176,7 +176,7 @@ def gemm_source_hash() -> str:
 
 def profiled_traffic(config: str):
     """dram bytes per launch of the NVFP4 GEMM from profiles/, scaled to `config`."""
-    path = os.path.join(ROOT, "profiles", "gemm_nvfp4_ncu.md")
+    path = os.path.join(ROOT, "profiles", "gemm_nvfp4_4480x16384x6144.md")
     if not os.path.exists(path):
         return None, "no ncu summary"
     text = open(path).read()
