@@ -196,6 +196,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(GemmCfg<FP4>::kThrea
     cluster_sync();                               // barriers of both CTAs initialised, TMEM allocated
     tc_fence_after();
     const uint32_t tmem_base = *tmem_holder;
+    grid_dep_wait();                              // operands written by the preceding kernels are visible
 
     const int m_tiles = (args.M + BM - 1) / BM;
     const int n_tiles = (args.N + BN - 1) / BN;
@@ -593,13 +594,21 @@ cudaError_t launch_gemm(const GemmLaunch &g, int sms, cudaStream_t stream)
     }
     const int pairs = pairs_cached;
     const int grid = 2 * (tiles < pairs ? tiles : pairs);        // clusters of two CTAs
+    // dependent launch: the set-up (barriers, tensor memory, descriptor prefetch) overlaps
+    // the end of the preceding kernel; the kernel waits for its results before loading
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)grid);
+    cfg.blockDim = dim3(fp4 ? GemmCfg<true>::kThreads : GemmCfg<false>::kThreads);
+    cfg.dynamicSmemBytes = fp4 ? GemmCfg<true>::kSmemBytes : GemmCfg<false>::kSmemBytes;
+    cfg.stream = stream;
+    cudaLaunchAttribute at[1];
+    at[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    at[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = at;
+    cfg.numAttrs = 1;
     if (fp4)
-        sq_gemm_kernel<true><<<grid, GemmCfg<true>::kThreads, GemmCfg<true>::kSmemBytes, stream>>>(
-            tA, tB, tT, tU, tY, a);
-    else
-        sq_gemm_kernel<false><<<grid, GemmCfg<false>::kThreads, GemmCfg<false>::kSmemBytes, stream>>>(
-            tA, tB, tT, tU, tY, a);
-    return cudaGetLastError();
+        return cudaLaunchKernelEx(&cfg, sq_gemm_kernel<true>, tA, tB, tT, tU, tY, a);
+    return cudaLaunchKernelEx(&cfg, sq_gemm_kernel<false>, tA, tB, tT, tU, tY, a);
 }
 
 }  // namespace sq

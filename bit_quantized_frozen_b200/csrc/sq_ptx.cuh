@@ -78,6 +78,21 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatil
     }
 }
 
+// ---- programmatic dependent launch ---------------------------------------------
+// Wait until the preceding grid of the stream has completed and its writes are
+// visible (returns at once when the launch was not a dependent launch).
+__device__ __forceinline__ void grid_dep_wait()
+{
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+}
+
+// Let the next grid of the stream, if launched as a dependent launch, start its
+// CTAs now (it still waits for this grid's results with grid_dep_wait).
+__device__ __forceinline__ void grid_dep_launch()
+{
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
 // ---- clusters ------------------------------------------------------------------
 __device__ __forceinline__ uint32_t cluster_ctarank()
 {

@@ -133,6 +133,7 @@ __global__ void __launch_bounds__(kStreamThreads) absmax_rot_kernel(const __grid
                                                                     int64_t blocks, uint32_t *__restrict__ amax)
 {
     const int lane = threadIdx.x & 31;
+    grid_dep_launch();                              // the quantisation pass may start loading
     float m = 0.0f;
     stream_blocks<T>(&tm, blocks, nullptr, [&](int64_t, float (&v)[32], bool) {
         fwht256_l32<false>(v, lane);
@@ -219,15 +220,20 @@ __global__ void __launch_bounds__(kStreamThreads) nvfp4_quant_kernel(const __gri
 {
     const int lane = threadIdx.x & 31;
     const int q = lane & 7;
-    const float g = g_static ? *g_static : __fdiv_rn(__uint_as_float(*amax), 2688.0f);
-    if (g_out && blockIdx.x == 0 && threadIdx.x == 0)
-        *g_out = g;
-    const float sixg = __fmul_rn(6.0f, g);
+    grid_dep_launch();
+    // amax (and t) come from the preceding pass: the consumers wait for it before
+    // their first block, the producer starts streaming at once
+    float g = 0.0f, sixg = 0.0f;
     const int64_t kb_per_row = K / kHad;
     const int64_t C = K / kSfBlock;
     const bool idx32 = rows_pad * kb_per_row <= (int64_t)UINT32_MAX;
     // the forward's low-rank operands (g is final here), done while the first chunks load
     auto lowrank = [&](int c) {
+        grid_dep_wait();
+        g = g_static ? *g_static : __fdiv_rn(__uint_as_float(*amax), 2688.0f);
+        sixg = __fmul_rn(6.0f, g);
+        if (g_out && blockIdx.x == 0 && c == 0)
+            *g_out = g;
         if (!lr.t32)
             return;
         const float beta = lowrank_beta(g, lr.g_w);
@@ -517,6 +523,7 @@ __global__ void __launch_bounds__(kP1Threads, 2) act_pass1_kernel(const __grid_c
         fence_mbar_init();
     }
     __syncthreads();
+    grid_dep_launch();                                // the quantisation pass may start loading x
 
     float m = 0.0f;
     float acc[4][4];
@@ -1023,9 +1030,19 @@ static cudaError_t launch_nvfp4_quant(const T *in, int64_t rows, int64_t K, cons
     if (e != cudaSuccess)
         return e;
     const int64_t rows_pad = (rows + 127) / 128 * 128;
-    nvfp4_quant_kernel<T><<<stream_grid(rows_pad * (K / kHad), sms, sizeof(T) == 4 ? 2 : 3), kStreamThreads,
-                            StreamCfg<T>::kSmem, s>>>(tm, rows, rows_pad, K, amax, g_static, g_out, codes, sf, lr);
-    return cudaGetLastError();
+    // dependent launch: the CTAs start (and stream x) while the absmax pass drains
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)stream_grid(rows_pad * (K / kHad), sms, sizeof(T) == 4 ? 2 : 3));
+    cfg.blockDim = dim3(kStreamThreads);
+    cfg.dynamicSmemBytes = StreamCfg<T>::kSmem;
+    cfg.stream = s;
+    cudaLaunchAttribute at[1];
+    at[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    at[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = at;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, nvfp4_quant_kernel<T>, tm, rows, rows_pad, K, amax, g_static, g_out, codes, sf,
+                              lr);
 }
 
 cudaError_t launch_absmax_rot_f32(const float *in, int64_t rows, int64_t K, uint32_t *amax, int sms, cudaStream_t s)
