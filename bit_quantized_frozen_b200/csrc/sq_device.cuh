@@ -169,6 +169,72 @@ __device__ __forceinline__ void fwht256_l32(float (&v)[32], int lane)
         f2_unpack(p[j], v[2 * j], v[2 * j + 1]);
 }
 
+// ---------------------------------------------------------------------------
+// Hadamard-256 over 8 lanes, strided layout, without the final 1/16.
+//
+// Lane q = lane % 8 of an aligned group of 8 lanes holds v[8b + j] = element
+// 64b + 8q + j of one 256-block (b = 0..3, j = 0..7): every 16-byte piece of a
+// row it reads is a different bank slot for the 8 lanes.  Strides 1, 2, 4 pair
+// values inside a lane, strides 8, 16, 32 pair lane q with q ^ 1, q ^ 2, q ^ 4,
+// strides 64, 128 pair values inside a lane again: the sequential order of
+// strides with the same operands, so every element is identical bit for bit to
+// the sequential transform (before its 1/16).
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ void fwht256_l32s_unscaled(float (&v)[32], int lane)
+{
+#pragma unroll
+    for (int j = 0; j < 16; ++j) {               // stride 1, inside each pair
+        const float a = v[2 * j], b = v[2 * j + 1];
+        v[2 * j] = __fadd_rn(a, b);
+        v[2 * j + 1] = __fsub_rn(a, b);
+    }
+    uint64_t p[16];                              // p[4b + j/2] = (v[8b + j], v[8b + j + 1]), j even
+#pragma unroll
+    for (int j = 0; j < 16; ++j)
+        p[j] = f2_pack(v[2 * j], v[2 * j + 1]);
+#pragma unroll
+    for (int hp = 1; hp <= 2; hp <<= 1)          // strides 2, 4
+#pragma unroll
+        for (int j = 0; j < 16; ++j)
+            if ((j & hp) == 0) {
+                const uint64_t a = p[j], b = p[j + hp];
+                p[j] = f2_add(a, b);
+                p[j + hp] = f2_sub(a, b);
+            }
+#pragma unroll
+    for (int x = 1; x <= 4; x <<= 1) {           // strides 8, 16, 32, across lanes
+        const float sg = (lane & x) == 0 ? 1.0f : -1.0f;
+        const uint64_t sg2 = f2_pack(sg, sg);
+#pragma unroll
+        for (int j = 0; j < 16; ++j) {
+            float lo, hi;
+            f2_unpack(p[j], lo, hi);
+            const uint64_t o = f2_pack(__shfl_xor_sync(0xffffffffu, lo, x), __shfl_xor_sync(0xffffffffu, hi, x));
+            p[j] = f2_fma(sg2, p[j], o);
+        }
+    }
+#pragma unroll
+    for (int hp = 4; hp <= 8; hp <<= 1)          // strides 64, 128
+#pragma unroll
+        for (int j = 0; j < 16; ++j)
+            if ((j & hp) == 0) {
+                const uint64_t a = p[j], b = p[j + hp];
+                p[j] = f2_add(a, b);
+                p[j + hp] = f2_sub(a, b);
+            }
+#pragma unroll
+    for (int j = 0; j < 16; ++j)
+        f2_unpack(p[j], v[2 * j], v[2 * j + 1]);
+}
+
+// max(a, b, c) in one instruction (sm_100)
+__device__ __forceinline__ float fmax3(float a, float b, float c)
+{
+    float r;
+    asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+    return r;
+}
+
 // 32 consecutive values into registers (fp32 source or bf16 bit patterns)
 __device__ __forceinline__ void load32(const float *p, float (&v)[32])
 {

@@ -138,8 +138,8 @@ __global__ void __launch_bounds__(kStreamThreads) absmax_rot_kernel(const __grid
     stream_blocks<T>(&tm, blocks, nullptr, [&](int64_t, float (&v)[32], bool) {
         fwht256_l32<false>(v, lane);
 #pragma unroll
-        for (int i = 0; i < 32; ++i)
-            m = fmaxf(m, fabsf(v[i]));
+        for (int i = 0; i < 32; i += 2)
+            m = fmax3(m, fabsf(v[i]), fabsf(v[i + 1]));
     });
     // max |v / 16| == (max |v|) / 16 bit for bit: rounding is monotonic
     m = __fmul_rn(m, 0.0625f);
@@ -567,36 +567,26 @@ __global__ void __launch_bounds__(kP1Threads, 2) act_pass1_kernel(const __grid_c
             const uint32_t xs = sbase + st * kP1BufBytes;
             const uint32_t ds = xs + kP1XBytes;
             if (amax) {
+                // lane q of row r takes 16 bytes (8 values, columns 64b + 8q..) of each of the
+                // four boxes: the 8 lanes of a row read 8 different bank slots
                 const int r = 4 * warp + (lane >> 3);
                 const int q = lane & 7;
-                const int sb = q >> 1;                // box of this lane's 32 values
-                // read chunk (i + sb) & 3 of the lane's four at step i (the 8 lanes of a
-                // row then hit 8 different banks), then rotate back by sb
-                const uint8_t *rowp = p1_smem + st * kP1BufBytes + sb * 4096 + r * 128;
-                uint4 tmp[4], rot[4], ch[4];
-#pragma unroll
-                for (int i = 0; i < 4; ++i)
-                    tmp[i] = *reinterpret_cast<const uint4 *>(rowp + 16 * ((4 * (q & 1) + ((i + sb) & 3)) ^ (r & 7)));
-#pragma unroll
-                for (int i = 0; i < 4; ++i)
-                    rot[i] = (sb & 1) ? tmp[(i + 3) & 3] : tmp[i];
-#pragma unroll
-                for (int i = 0; i < 4; ++i)
-                    ch[i] = (sb & 2) ? rot[(i + 2) & 3] : rot[i];
+                const uint8_t *rowp = p1_smem + st * kP1BufBytes + r * 128 + 16 * (q ^ (r & 7));
                 float v[32];
 #pragma unroll
-                for (int i = 0; i < 4; ++i) {
-                    const uint32_t w[4] = {ch[i].x, ch[i].y, ch[i].z, ch[i].w};
+                for (int b = 0; b < 4; ++b) {
+                    const uint4 a = *reinterpret_cast<const uint4 *>(rowp + 4096 * b);
+                    const uint32_t w[4] = {a.x, a.y, a.z, a.w};
 #pragma unroll
                     for (int jj = 0; jj < 4; ++jj) {
-                        v[8 * i + 2 * jj] = __uint_as_float(w[jj] << 16);
-                        v[8 * i + 2 * jj + 1] = __uint_as_float(w[jj] & 0xFFFF0000u);
+                        v[8 * b + 2 * jj] = __uint_as_float(w[jj] << 16);
+                        v[8 * b + 2 * jj + 1] = __uint_as_float(w[jj] & 0xFFFF0000u);
                     }
                 }
-                fwht256_l32<false>(v, lane);
+                fwht256_l32s_unscaled(v, lane);
 #pragma unroll
-                for (int i = 0; i < 32; ++i)
-                    m = fmaxf(m, fabsf(v[i]));
+                for (int i = 0; i < 32; i += 2)
+                    m = fmax3(m, fabsf(v[i]), fabsf(v[i + 1]));
             }
             if (t32) {
 #pragma unroll
