@@ -434,7 +434,7 @@ constexpr int kP1DBytes = kHad * kRank * 2;        // 16 KB
 constexpr int kP1BufBytes = kP1XBytes + kP1DBytes;
 constexpr int kP1Stages = 3;
 constexpr int kP1Consumers = 8;
-constexpr int kP1Threads = 32 * (kP1Consumers + 1);
+constexpr int kP1Threads = 32 * (kP1Consumers + 2);   // + TMA producer warp + MMA warp
 constexpr int kP1Smem = kP1Stages * kP1BufBytes + 1024 + 256;   // ring, 1 KB alignment, barriers
 constexpr int kP1MaxSplit = 8;
 
@@ -493,6 +493,19 @@ __device__ __forceinline__ float ld_shared_cluster_f32(uint32_t addr)
     return v;
 }
 
+// t = x . lora_down on the tensor cores: one thread issues, per chunk, 16 MMAs
+// (M = 128, N = 32, K = 16, bf16 -> fp32 in tensor memory).  A is the x stage
+// (K-major, 128B swizzle); only rows 0..31 are the tile's, the MMA's other 96
+// rows read the rest of the stage and their results are never read.  B is the
+// lora_down stage, N-major (32 values of a k-row are one 64-byte swizzled row).
+constexpr uint32_t kP1Idesc = (1u << 4) | (1u << 7) | (1u << 10) | (1u << 16) | ((uint32_t)(kRank >> 3) << 17) |
+                              ((uint32_t)(128 >> 4) << 24);
+__device__ __forceinline__ uint64_t p1_bdesc(uint32_t saddr)
+{
+    return (uint64_t)((saddr & 0x3FFFFu) >> 4) | ((uint64_t)1u << 16) | ((uint64_t)(512u >> 4) << 32) |
+           ((uint64_t)1u << 46) | ((uint64_t)4u << 61);
+}
+
 __global__ void __launch_bounds__(kP1Threads, 2) act_pass1_kernel(const __grid_constant__ CUtensorMap tmx,
                                                                   const __grid_constant__ CUtensorMap tmd,
                                                                   int64_t M, int64_t K, uint32_t *__restrict__ amax,
@@ -504,7 +517,9 @@ __global__ void __launch_bounds__(kP1Threads, 2) act_pass1_kernel(const __grid_c
         reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(p1_raw) + 1023) & ~uintptr_t(1023));
     uint64_t *bars = reinterpret_cast<uint64_t *>(p1_smem + kP1Stages * kP1BufBytes);
     const uint32_t full = smem_u32(bars), empty = smem_u32(bars + kP1Stages);
-    volatile uint32_t *abort_flag = reinterpret_cast<uint32_t *>(bars + 2 * kP1Stages);
+    const uint32_t done = smem_u32(bars + 2 * kP1Stages);                  // every MMA finished
+    uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(bars + 2 * kP1Stages + 1);
+    volatile uint32_t *abort_flag = tmem_holder + 1;
     const int tid = threadIdx.x;
     const int lane = tid & 31;
     const int warp = tid >> 5;
@@ -517,23 +532,24 @@ __global__ void __launch_bounds__(kP1Threads, 2) act_pass1_kernel(const __grid_c
     if (tid == 0) {
         for (int st = 0; st < kP1Stages; ++st) {
             mbar_init(full + 8 * st, 1);
-            mbar_init(empty + 8 * st, kP1Consumers);
+            mbar_init(empty + 8 * st, (amax ? kP1Consumers : 0) + (t32 ? 1 : 0));
         }
+        mbar_init(done, 1);
         *abort_flag = 0u;
         fence_mbar_init();
     }
+    if (t32 && warp == kP1Consumers + 1) {
+        tmem_alloc(smem_u32(tmem_holder), 32);
+        tmem_relinquish();
+    }
+    tc_fence_before();
     __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem_base = t32 ? *tmem_holder : 0u;
     grid_dep_launch();                                // the quantisation pass may start loading x
 
     float m = 0.0f;
-    float acc[4][4];
-#pragma unroll
-    for (int nt = 0; nt < 4; ++nt)
-#pragma unroll
-        for (int i = 0; i < 4; ++i)
-            acc[nt][i] = 0.0f;
-
-    if (warp == kP1Consumers) {                       // producer
+    if (warp == kP1Consumers) {                       // TMA producer
         if (lane == 0) {
             prefetch_tmap(&tmx);
             if (t32)
@@ -554,8 +570,29 @@ __global__ void __launch_bounds__(kP1Threads, 2) act_pass1_kernel(const __grid_c
             }
         }
         __syncwarp();
-    } else {
-        const int mt = warp >> 2;                     // MMA: rows 16mt..16mt+15
+    } else if (warp == kP1Consumers + 1) {            // MMA issuer: t
+        if (t32 && lane == 0) {
+            bool ok = true;
+            for (int c = 0; c < nch && ok; ++c) {
+                const int st = c % kP1Stages;
+                const uint32_t ph = (uint32_t)(c / kP1Stages) & 1u;
+                if (!mbar_wait(full + 8 * st, ph, abort_flag, status)) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+                const uint32_t xs = sbase + st * kP1BufBytes;
+                const uint64_t da = sdesc_sw128(xs), db = p1_bdesc(xs + kP1XBytes);
+#pragma unroll
+                for (int ks = 0; ks < 16; ++ks)           // k-step: columns 16ks..16ks+15 of the chunk
+                    mma_bf16(tmem_base, da + (uint64_t)((ks >> 2) * 256 + (ks & 3) * 2),
+                             db + (uint64_t)(ks * 64), kP1Idesc, (c > 0 || ks > 0) ? 1u : 0u);
+                tc_commit(empty + 8 * st);
+            }
+            tc_commit(done);
+        }
+        __syncwarp();
+    } else if (amax) {                                // consumers: Hadamard absmax
         for (int c = 0; c < nch; ++c) {
             const int st = c % kP1Stages;
             const uint32_t ph = (uint32_t)(c / kP1Stages) & 1u;
@@ -564,54 +601,54 @@ __global__ void __launch_bounds__(kP1Threads, 2) act_pass1_kernel(const __grid_c
                 ok = mbar_wait(full + 8 * st, ph, abort_flag, status) ? 1 : 0;
             if (__shfl_sync(0xffffffffu, ok, 0) == 0)
                 break;
-            const uint32_t xs = sbase + st * kP1BufBytes;
-            const uint32_t ds = xs + kP1XBytes;
-            if (amax) {
-                // lane q of row r takes 16 bytes (8 values, columns 64b + 8q..) of each of the
-                // four boxes: the 8 lanes of a row read 8 different bank slots
-                const int r = 4 * warp + (lane >> 3);
-                const int q = lane & 7;
-                const uint8_t *rowp = p1_smem + st * kP1BufBytes + r * 128 + 16 * (q ^ (r & 7));
-                float v[32];
+            // lane q of row r takes 16 bytes (8 values, columns 64b + 8q..) of each of the
+            // four boxes: the 8 lanes of a row read 8 different bank slots
+            const int r = 4 * warp + (lane >> 3);
+            const int q = lane & 7;
+            const uint8_t *rowp = p1_smem + st * kP1BufBytes + r * 128 + 16 * (q ^ (r & 7));
+            float v[32];
 #pragma unroll
-                for (int b = 0; b < 4; ++b) {
-                    const uint4 a = *reinterpret_cast<const uint4 *>(rowp + 4096 * b);
-                    const uint32_t w[4] = {a.x, a.y, a.z, a.w};
+            for (int b = 0; b < 4; ++b) {
+                const uint4 a = *reinterpret_cast<const uint4 *>(rowp + 4096 * b);
+                const uint32_t w[4] = {a.x, a.y, a.z, a.w};
 #pragma unroll
-                    for (int jj = 0; jj < 4; ++jj) {
-                        v[8 * b + 2 * jj] = __uint_as_float(w[jj] << 16);
-                        v[8 * b + 2 * jj + 1] = __uint_as_float(w[jj] & 0xFFFF0000u);
-                    }
-                }
-                fwht256_l32s_unscaled(v, lane);
-#pragma unroll
-                for (int i = 0; i < 32; i += 2)
-                    m = fmax3(m, fabsf(v[i]), fabsf(v[i + 1]));
-            }
-            if (t32) {
-#pragma unroll
-                for (int ss = 0; ss < 4; ++ss) {
-                    const int ks = 4 * (warp & 3) + ss;   // k-step: columns 16ks..16ks+15 of the chunk
-                    // A 16x16: matrices (rows 0-7 | 8-15) x (k 0-7 | 8-15); lane provides row (lane & 15)
-                    uint32_t a[4];
-                    ldmatrix_x4(xs + p1_xoff(16 * mt + (lane & 15), 2 * ks + (lane >> 4)), a);
-                    // B: (k 0-7 | 8-15) x (n-tile pair), transposed load of row-major D
-#pragma unroll
-                    for (int np = 0; np < 2; ++np) {
-                        uint32_t b[4];
-                        const int bk = 16 * ks + (lane & 7) + 8 * ((lane >> 3) & 1);
-                        ldmatrix_x4_trans(ds + p1_doff(bk, 2 * np + (lane >> 4)), b);
-                        mma_bf16_16816(acc[2 * np], a, b[0], b[1]);
-                        mma_bf16_16816(acc[2 * np + 1], a, b[2], b[3]);
-                    }
+                for (int jj = 0; jj < 4; ++jj) {
+                    v[8 * b + 2 * jj] = __uint_as_float(w[jj] << 16);
+                    v[8 * b + 2 * jj + 1] = __uint_as_float(w[jj] & 0xFFFF0000u);
                 }
             }
             __syncwarp();
             if (lane == 0)
-                mbar_arrive(empty + 8 * st);
+                mbar_arrive(empty + 8 * st);              // the stage's x is in registers
+            fwht256_l32s_unscaled(v, lane);
+#pragma unroll
+            for (int i = 0; i < 32; i += 2)
+                m = fmax3(m, fabsf(v[i]), fabsf(v[i + 1]));
         }
     }
-    __syncthreads();                                  // ring idle: reuse it below
+    __syncthreads();                                  // every role's loop is done
+
+    // t rows 0..31 of this CTA: tensor-memory lanes 0..31, read by warp 0 once every MMA finished
+    uint32_t tr[32];
+    if (t32 && warp == 0) {
+        int ok = 1;
+        if (lane == 0)
+            ok = mbar_wait(done, 0, abort_flag, status) ? 1 : 0;
+        ok = __shfl_sync(0xffffffffu, ok, 0);
+        tc_fence_after();
+        if (ok) {
+            tmem_ld_32cols(tmem_base, tr);
+            tmem_wait_ld();
+        } else {
+#pragma unroll
+            for (int i = 0; i < 32; ++i)
+                tr[i] = 0u;
+        }
+        tc_fence_before();
+    }
+    __syncthreads();                                  // ring idle and tensor memory read
+    if (t32 && warp == kP1Consumers + 1)
+        tmem_dealloc(tmem_base, 32);
 
     if (amax) {
         m = __fmul_rn(m, 0.0625f);                    // the transform's 1/16, once (exact for a max)
@@ -619,18 +656,14 @@ __global__ void __launch_bounds__(kP1Threads, 2) act_pass1_kernel(const __grid_c
         for (int xx = 16; xx >= 1; xx >>= 1)
             m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, xx));
     }
-    float *part = reinterpret_cast<float *>(p1_smem);          // [8 warps][16][33]
-    float *tcta = part + 8 * 16 * 33;                           // [32][32] this CTA's t tile
-    float *wmax = tcta + kP1Rows * kRank;                       // [9]
-    if (t32 && warp < kP1Consumers) {
-        const int g = lane >> 2, tq = lane & 3;
+    float *tcta = reinterpret_cast<float *>(p1_smem);          // [32][32] this CTA's t tile
+    float *wmax = tcta + kP1Rows * kRank;                       // [10]
+    if (t32 && warp == 0) {
 #pragma unroll
-        for (int nt = 0; nt < 4; ++nt) {
-            part[(warp * 16 + g) * 33 + 8 * nt + 2 * tq] = acc[nt][0];
-            part[(warp * 16 + g) * 33 + 8 * nt + 2 * tq + 1] = acc[nt][1];
-            part[(warp * 16 + g + 8) * 33 + 8 * nt + 2 * tq] = acc[nt][2];
-            part[(warp * 16 + g + 8) * 33 + 8 * nt + 2 * tq + 1] = acc[nt][3];
-        }
+        for (int i = 0; i < 32; i += 4)                  // once per CTA: bank conflicts do not matter
+            *reinterpret_cast<float4 *>(tcta + lane * kRank + i) =
+                make_float4(__uint_as_float(tr[i]), __uint_as_float(tr[i + 1]), __uint_as_float(tr[i + 2]),
+                            __uint_as_float(tr[i + 3]));
     }
     if (lane == 0)
         wmax[warp] = m;
@@ -643,19 +676,8 @@ __global__ void __launch_bounds__(kP1Threads, 2) act_pass1_kernel(const __grid_c
     }
     if (!t32)
         return;
-    for (int e = tid; e < kP1Rows * kRank; e += kP1Threads) {   // k-step partials, fixed order
-        const int r = e >> 5, col = e & 31;
-        const int h = r >> 4, rr = r & 15;
-        float v = 0.0f;
-#pragma unroll
-        for (int w = 0; w < 4; ++w)
-            v = __fadd_rn(v, part[((4 * h + w) * 16 + rr) * 33 + col]);
-        tcta[e] = v;
-    }
     if (split > 1)
         cluster_sync();                               // every rank's tile is complete
-    else
-        __syncthreads();
     if (j == 0) {
         const uint32_t tl = (uint32_t)__cvta_generic_to_shared(tcta);
         for (int e = tid; e < kP1Rows * kRank; e += kP1Threads) {
