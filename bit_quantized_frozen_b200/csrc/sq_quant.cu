@@ -290,31 +290,53 @@ __global__ void __launch_bounds__(kStreamThreads) nvfp4_quant_kernel(const __gri
 // whole group of 32 rotated values and sweeps the 26 scale fractions in
 // registers (group index = 8 * block + lane % 8).
 // ---------------------------------------------------------------------------
-__device__ __forceinline__ float group_sq_error(const float (&r)[32], float s, float inv)
+// sum of RN((r_i - q_i s)^2) over the group, as lane 0 of an xor butterfly over
+// strides 16, 8, 4, 2, 1; rp holds the 32 rotated values as pairs (r_2j, r_2j+1).
+// q = clamp(rint(r inv), -7, 7): |r inv| <= 14, so adding and subtracting
+// 1.5 * 2^23 rounds to the nearest integer, ties to even, exactly like rint (and
+// on the FMA pipe, not the conversion unit).  q s is exact (<= 14 significant
+// bits), so fma(-q, s, r) rounds like r - q s.
+__device__ __forceinline__ float group_sq_error(const uint64_t (&rp)[16], float s, float inv)
 {
-    float p[32];
+    uint64_t p[16];
+    if (s == 0.0f) {                                   // q = 0: error r^2
 #pragma unroll
-    for (int i = 0; i < 32; ++i) {
-        float e;
-        if (s == 0.0f) {
-            e = r[i];
-        } else {
-            float q = rintf(__fmul_rn(r[i], inv));
-            q = fminf(fmaxf(q, -7.0f), 7.0f);
-            e = __fsub_rn(r[i], __fmul_rn(q, s));   // q*s is exact
+        for (int j = 0; j < 16; ++j)
+            p[j] = f2_mul(rp[j], rp[j]);
+    } else {
+        constexpr float kRound = 12582912.0f;          // 1.5 * 2^23
+        const uint64_t inv2 = f2_pack(inv, inv), nsn = f2_pack(-s, -s);
+        const uint64_t rnd = f2_pack(kRound, kRound);
+#pragma unroll
+        for (int j = 0; j < 16; ++j) {
+            float t0, t1;
+            f2_unpack(f2_add(f2_mul(rp[j], inv2), rnd), t0, t1);
+            t0 = fminf(fmaxf(t0, kRound - 7.0f), kRound + 7.0f);
+            t1 = fminf(fmaxf(t1, kRound - 7.0f), kRound + 7.0f);
+            const uint64_t q = f2_sub(f2_pack(t0, t1), rnd);
+            const uint64_t e = f2_fma(q, nsn, rp[j]);
+            p[j] = f2_mul(e, e);
         }
-        p[i] = __fmul_rn(e, e);
     }
-    // lane 0 of an xor butterfly over strides 16, 8, 4, 2, 1
+    // strides 16, 8, 4, 2 are pair strides 8, 4, 2, 1; stride 1 adds the two halves of pair 0
 #pragma unroll
-    for (int d = 16; d >= 1; d >>= 1)
+    for (int d = 8; d >= 1; d >>= 1)
 #pragma unroll
-        for (int i = 0; i < d; ++i)
-            p[i] = __fadd_rn(p[i], p[i + d]);
-    return p[0];
+        for (int j = 0; j < d; ++j)
+            p[j] = f2_add(p[j], p[j + d]);
+    float lo, hi;
+    f2_unpack(p[0], lo, hi);
+    return __fadd_rn(lo, hi);
 }
 
-__global__ void __launch_bounds__(kStreamThreads) int4_build_kernel(const __grid_constant__ CUtensorMap tm,
+// the swept scale fractions RN((50 + 2j) / 100), j = 0..25 (folded at compile time, IEEE rounding)
+__constant__ float kFrac[26] = {
+    50.0f / 100, 52.0f / 100, 54.0f / 100, 56.0f / 100, 58.0f / 100, 60.0f / 100, 62.0f / 100,
+    64.0f / 100, 66.0f / 100, 68.0f / 100, 70.0f / 100, 72.0f / 100, 74.0f / 100, 76.0f / 100,
+    78.0f / 100, 80.0f / 100, 82.0f / 100, 84.0f / 100, 86.0f / 100, 88.0f / 100, 90.0f / 100,
+    92.0f / 100, 94.0f / 100, 96.0f / 100, 98.0f / 100, 100.0f / 100};
+
+__global__ void __launch_bounds__(kStreamThreads, 2) int4_build_kernel(const __grid_constant__ CUtensorMap tm,
                                                                     int64_t blocks, uint8_t *__restrict__ codes,
                                                                     uint16_t *__restrict__ scales,
                                                                     uint8_t *__restrict__ frac)
@@ -326,18 +348,22 @@ __global__ void __launch_bounds__(kStreamThreads) int4_build_kernel(const __grid
             return;
         float a = 0.0f;
 #pragma unroll
-        for (int i = 0; i < 32; ++i)
-            a = fmaxf(a, fabsf(r[i]));
+        for (int i = 0; i < 32; i += 2)
+            a = fmax3(a, fabsf(r[i]), fabsf(r[i + 1]));
+        uint64_t rp[16];
+#pragma unroll
+        for (int j = 0; j < 16; ++j)
+            rp[j] = f2_pack(r[2 * j], r[2 * j + 1]);
         float best = 0.0f, best_s = 0.0f;
         uint16_t best_h = 0;
         int best_j = 0;
 #pragma unroll 1
         for (int j = 0; j < kFracCount; ++j) {
-            const float f = __fdiv_rn((float)(50 + 2 * j), 100.0f);
+            const float f = kFrac[j];
             const __half hs = __float2half_rn(__fdiv_rn(__fmul_rn(f, a), 7.0f));
             const float s = __half2float(hs);
             const float inv = s == 0.0f ? 0.0f : __frcp_rn(s);
-            const float mse = group_sq_error(r, s, inv);
+            const float mse = group_sq_error(rp, s, inv);
             if (j == 0 || mse < best) {
                 best = mse;
                 best_j = j;
@@ -349,13 +375,15 @@ __global__ void __launch_bounds__(kStreamThreads) int4_build_kernel(const __grid
         const float inv = best_s == 0.0f ? 0.0f : __frcp_rn(best_s);
         uint32_t word[4] = {0u, 0u, 0u, 0u};
 #pragma unroll
-        for (int i = 0; i < 32; ++i) {
-            int q = 0;
+        for (int i = 0; i < 32; i += 2) {
+            float r0, r1;
+            f2_unpack(rp[i >> 1], r0, r1);
+            int q0 = 0, q1 = 0;
             if (best_s != 0.0f) {
-                float qf = rintf(__fmul_rn(r[i], inv));
-                q = (int)fminf(fmaxf(qf, -7.0f), 7.0f);
+                q0 = (int)fminf(fmaxf(rintf(__fmul_rn(r0, inv)), -7.0f), 7.0f);
+                q1 = (int)fminf(fmaxf(rintf(__fmul_rn(r1, inv)), -7.0f), 7.0f);
             }
-            word[i >> 3] |= ((uint32_t)q & 0xFu) << (4 * (i & 7));
+            word[i >> 3] |= (((uint32_t)q0 & 0xFu) | (((uint32_t)q1 & 0xFu) << 4)) << (4 * (i & 7));
         }
         const int64_t gidx = 8 * b + (lane & 7);     // flat group index
         reinterpret_cast<uint4 *>(codes)[gidx] = make_uint4(word[0], word[1], word[2], word[3]);
