@@ -265,6 +265,17 @@ def run_reference(args, cfg, d):
     print(json.dumps(line), flush=True)
 
 
+def max_over_ranks(values, world, device):
+    """Element-wise max over the ranks of per-rank timings (every multi-GPU time is the
+    slowest rank's); identity for one rank."""
+    if world <= 1:
+        return list(values)
+    import torch
+    t = torch.tensor(list(values), dtype=torch.float64, device=device)
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return t.tolist()
+
+
 def workload_config(cfg, args):
     return {
         "workload": f"SquareQ W4 linear {cfg.M}x{cfg.N}x{cfg.K} (M tokens x N out x K in), rank 32, "
@@ -376,12 +387,9 @@ def run_sq(args, cfg, d, rank, world, local_rank):
                                  for e in (even if k in gemm_of.values() else odd if k in gemm_of else evs))
               for k in keys}   # ms
     outer_ms = outer[0].elapsed_time(outer[1]) / max(args.steps, 1)
-    if world > 1:
-        t = torch.tensor([per_op[k] for k in keys] + [outer_ms], dtype=torch.float64, device=dev)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        vals = t.tolist()
-        per_op = dict(zip(keys, vals[:-1]))
-        outer_ms = vals[-1]
+    vals = max_over_ranks([per_op[k] for k in keys] + [outer_ms], world, dev)
+    per_op = dict(zip(keys, vals[:-1]))
+    outer_ms = vals[-1]
 
     # end to end through the C ABI with host buffers: H2D of x, forward, D2H of y.
     # Steps are independent, so step i+1's upload and forward run on one stream while
@@ -422,11 +430,7 @@ def run_sq(args, cfg, d, rank, world, local_rank):
         s_main.wait_stream(s_d2h)
         e1.record(s_main)
         torch.cuda.synchronize()
-        e2e_ms = e0.elapsed_time(e1) / reps
-        if world > 1:
-            t = torch.tensor([e2e_ms], dtype=torch.float64, device=dev)
-            torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-            e2e_ms = t.item()
+        e2e_ms = max_over_ranks([e0.elapsed_time(e1) / reps], world, dev)[0]
         e2e = {"value": world * 2.0 * M * N * K / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
                "h2d_bytes_per_step": int(M * K * 2), "d2h_bytes_per_step": int(M * N * 4),
                "ms_per_step": e2e_ms,
