@@ -254,8 +254,8 @@ __global__ void __launch_bounds__(kStreamThreads) nvfp4_quant_kernel(const __gri
         for (int h = 0; h < 2; ++h) {
             float bmax = 0.0f;
 #pragma unroll
-            for (int i = 0; i < 16; ++i)
-                bmax = fmaxf(bmax, fabsf(v[16 * h + i]));
+            for (int i = 0; i < 16; i += 2)
+                bmax = fmax3(bmax, fabsf(v[16 * h + i]), fabsf(v[16 * h + i + 1]));
             uint32_t code = 0;
             uint32_t w0 = 0, w1 = 0;
             if (g != 0.0f) {
@@ -857,7 +857,7 @@ __device__ __forceinline__ void rec_decode(const uint8_t *stage, int r, int q, f
 }
 
 template <int FMT, bool LOWRANK>
-__global__ void __launch_bounds__(256, 2) reconstruct_kernel(const uint8_t *__restrict__ codes,
+__global__ void __launch_bounds__(256, LOWRANK ? 2 : 3) reconstruct_kernel(const uint8_t *__restrict__ codes,
                                                              const void *__restrict__ scales,
                                                              const float *__restrict__ g_w,
                                                              const uint16_t *__restrict__ U,
@@ -1224,7 +1224,8 @@ cudaError_t launch_reconstruct(int fmt, const uint8_t *codes, const void *scales
         attr_done[dev] = true;
     }
     const int64_t tiles = (K / kHad) * ((N + kRecRows - 1) / kRecRows);
-    const unsigned grid = (unsigned)(tiles < 2LL * sms ? tiles : 2LL * sms);
+    const int64_t per_sm = with_lowrank ? 2 : 3;            // resident CTAs per SM (registers, shared memory)
+    const unsigned grid = (unsigned)(tiles < per_sm * sms ? tiles : per_sm * sms);
     const int smem = with_lowrank ? kRecSmemLowrank : kRecSmemResidual;
     if (fmt == 2) {
         if (with_lowrank)
