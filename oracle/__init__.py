@@ -56,6 +56,9 @@ _SIGS = {
     "or_int4_fraction": ([ctypes.c_int], _F),
     "or_int4_group32": ([_P, _P, _P, _P], None),
     "or_build_int4": ([_P, _I64, _I64, _P, _P, _P], None),
+    "or_int4_group64": ([_P, _P, _P, _P], None),
+    "or_build_int4_g": ([_P, _I64, _I64, ctypes.c_int, _P, _P, _P], None),
+    "or_linear_fwd_int4_g": ([_P, _P, _P, ctypes.c_int, _P, _P, _I64, _I64, _I64, _P, _I64, _P], None),
     "or_sf_offset": ([_I64, _I64, _I64], _I64),
     "or_sf_bytes": ([_I64, _I64], _I64),
     "or_nvfp4_global_scale": ([_F], _F),
@@ -167,14 +170,28 @@ def int4_group32(r):
     return q, int(s[0]), int(j[0])
 
 
-def build_int4(R):
-    """R [N, K] fp32 -> (codes [N, K/2] u8, scales [N, K/32] fp16 bits u16, frac [N, K/32] u8)."""
+def int4_group64(r):
+    r = _c(r, np.float32)
+    assert r.shape == (64,)
+    q = np.empty(64, np.int8)
+    s = np.empty(1, np.uint16)
+    j = np.empty(1, np.uint8)
+    lib().or_int4_group64(_p(r), _p(q), _p(s), _p(j))
+    return q, int(s[0]), int(j[0])
+
+
+def build_int4(R, group=32):
+    """R [N, K] fp32 -> (codes [N, K/2] u8, scales [N, K/group] fp16 bits u16, frac [N, K/group] u8),
+    group 32 or 64."""
     R = _c(R, np.float32)
     N, K = R.shape
     codes = np.empty((N, K // 2), np.uint8)
-    scales = np.empty((N, K // 32), np.uint16)
-    frac = np.empty((N, K // 32), np.uint8)
-    lib().or_build_int4(_p(R), N, K, _p(codes), _p(scales), _p(frac))
+    scales = np.empty((N, K // group), np.uint16)
+    frac = np.empty((N, K // group), np.uint8)
+    if group == 32:
+        lib().or_build_int4(_p(R), N, K, _p(codes), _p(scales), _p(frac))
+    else:
+        lib().or_build_int4_g(_p(R), N, K, int(group), _p(codes), _p(scales), _p(frac))
     return codes, scales, frac
 
 
@@ -254,7 +271,7 @@ def linear_fwd_nvfp4(xc, xsf, g_x, wc, wsf, g_w, t, U_bits, M, N, K, rows=None):
     return y
 
 
-def linear_fwd_int4(xrot, codes, scales, t, U_bits, M, N, K, rows=None):
+def linear_fwd_int4(xrot, codes, scales, t, U_bits, M, N, K, rows=None, group=32):
     rows = np.arange(M, dtype=np.int64) if rows is None else _c(rows, np.int64)
     y = np.empty((len(rows), N), np.float64)
     xrot = _c(xrot, np.float32)
@@ -262,8 +279,12 @@ def linear_fwd_int4(xrot, codes, scales, t, U_bits, M, N, K, rows=None):
     scales = _c(scales, np.uint16)
     t = None if t is None else _c(t, np.float64)
     U = None if U_bits is None else _c(U_bits, np.uint16)
-    lib().or_linear_fwd_int4(_p(xrot), _p(codes), _p(scales), _p(t), _p(U), M, N, K,
-                             _p(rows), len(rows), _p(y))
+    if group == 32:
+        lib().or_linear_fwd_int4(_p(xrot), _p(codes), _p(scales), _p(t), _p(U), M, N, K,
+                                 _p(rows), len(rows), _p(y))
+    else:
+        lib().or_linear_fwd_int4_g(_p(xrot), _p(codes), _p(scales), int(group), _p(t), _p(U), M, N, K,
+                                   _p(rows), len(rows), _p(y))
     return y
 
 
@@ -271,11 +292,12 @@ def linear_fwd_int4(xrot, codes, scales, t, U_bits, M, N, K, rows=None):
 
 FMT_INT4 = 1
 FMT_NVFP4 = 2
+FMT_INT4_G64 = 3
 
 
 def reconstruct_bf16(fmt, codes, scales, g_w, U_bits, D_bits, N, K, residual_only=False):
     codes = _c(codes, np.uint8)
-    scales = _c(scales, np.uint16 if fmt == FMT_INT4 else np.uint8)
+    scales = _c(scales, np.uint8 if fmt == FMT_NVFP4 else np.uint16)
     U = _c(U_bits, np.uint16)
     D = _c(D_bits, np.uint16)
     W = np.empty((N, K), np.uint16)

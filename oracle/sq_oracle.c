@@ -347,6 +347,74 @@ void or_int4_group32(const float *r, int8_t *q_out, uint16_t *s_out, uint8_t *j_
 }
 
 /*
+ * One group of 64 rotated residual values: the group-64 variant the same
+ * paragraph names beside group-32 ("int4 group-32/64 scales").  The same sweep
+ * over the 64 values (a = max|r_i| over all 64); the pages give no order for
+ * the squared-error sum, and the reading taken here is the group-32 rule per
+ * half: each 32-value half is summed by the xor butterfly above (strides 16, 8,
+ * 4, 2, 1), then the two half sums are added (first half + second half).
+ */
+void or_int4_group64(const float *r, int8_t *q_out, uint16_t *s_out, uint8_t *j_out)
+{
+    float a = 0.0f;
+    for (int i = 0; i < 64; i++) {
+        float m = fabsf(r[i]);
+        if (m > a)
+            a = m;
+    }
+    float best = INFINITY;
+    int best_j = -1;
+    for (int j = 0; j < 26; j++) {
+        float f = or_int4_fraction(j);
+        float fa = f * a;
+        float s7 = fa / 7.0f;
+        uint16_t sh = or_f32_to_f16(s7);
+        float s = or_f16_to_f32(sh);
+        int8_t q[64];
+        float p[64];
+        if (s == 0.0f) {
+            for (int i = 0; i < 64; i++) {
+                q[i] = 0;
+                p[i] = r[i] * r[i];
+            }
+        } else {
+            float inv = 1.0f / s;
+            for (int i = 0; i < 64; i++) {
+                float v = r[i] * inv;
+                float rq = nearbyintf(v);
+                if (rq > 7.0f)
+                    rq = 7.0f;
+                if (rq < -7.0f)
+                    rq = -7.0f;
+                q[i] = (int8_t)rq;
+                float qs = rq * s;              /* exact: <= 14 significant bits */
+                float e = r[i] - qs;
+                p[i] = e * e;
+            }
+        }
+        float half[2];
+        for (int h = 0; h < 2; h++) {
+            float *ph = p + 32 * h;
+            for (int d = 16; d >= 1; d >>= 1) {
+                float nxt[32];
+                for (int i = 0; i < 32; i++)
+                    nxt[i] = ph[i] + ph[i ^ d];
+                memcpy(ph, nxt, sizeof(nxt));
+            }
+            half[h] = ph[0];
+        }
+        float mse = half[0] + half[1];
+        if (best_j < 0 || mse < best) {
+            best = mse;
+            best_j = j;
+            memcpy(q_out, q, 64);
+            *s_out = sh;
+        }
+    }
+    *j_out = (uint8_t)best_j;
+}
+
+/*
  * int4 builder: rotate R [N, K] fp32 row-blockwise, then run the group codec
  * on every 32 consecutive rotated values of a row.  codes [N, K/2]: element
  * 2k in the low nibble, 4-bit two's complement; scales [N, K/32] fp16 bits;
@@ -375,6 +443,43 @@ void or_build_int4(const float *R, int64_t N, int64_t K,
                     uint8_t lo = (uint8_t)q[i] & 0xFu;
                     uint8_t hi = (uint8_t)q[i + 1] & 0xFu;
                     codes[n * (K / 2) + (b + 32 * g + i) / 2] = (uint8_t)(lo | (hi << 4));
+                }
+            }
+        }
+    }
+}
+
+/*
+ * The same builder for a group size of 32 or 64: scales and frac are
+ * [N, K/group].  group 32 is or_build_int4.
+ */
+void or_build_int4_g(const float *R, int64_t N, int64_t K, int group,
+                     uint8_t *codes, uint16_t *scales, uint8_t *frac)
+{
+    if (group == 32) {
+        or_build_int4(R, N, K, codes, scales, frac);
+        return;
+    }
+#pragma omp parallel for schedule(static)
+    for (int64_t n = 0; n < N; n++) {
+        for (int64_t b = 0; b < K; b += 256) {
+            float v[256];
+            for (int i = 0; i < 256; i++)
+                v[i] = R[n * K + b + i];
+            or_fwht256(v);
+            for (int g = 0; g < 4; g++) {
+                int8_t q[64];
+                uint16_t s;
+                uint8_t j;
+                or_int4_group64(v + 64 * g, q, &s, &j);
+                int64_t gi = n * (K / 64) + (b / 64) + g;
+                scales[gi] = s;
+                if (frac)
+                    frac[gi] = j;
+                for (int i = 0; i < 64; i += 2) {
+                    uint8_t lo = (uint8_t)q[i] & 0xFu;
+                    uint8_t hi = (uint8_t)q[i + 1] & 0xFu;
+                    codes[n * (K / 2) + (b + 64 * g + i) / 2] = (uint8_t)(lo | (hi << 4));
                 }
             }
         }
@@ -588,10 +693,10 @@ void or_linear_fwd_nvfp4(const uint8_t *xc, const uint8_t *xsf, float g_x,
  *   y[m,n] = sum_k xb wb + sum_r t[m,r] U[n,r].
  * xrot is the fp32 rotated x [M, K]; codes/scales as or_build_int4 writes.
  */
-void or_linear_fwd_int4(const float *xrot, const uint8_t *codes, const uint16_t *scales,
-                        const double *t, const uint16_t *U,
-                        int64_t M, int64_t N, int64_t K,
-                        const int64_t *rows, int64_t n_rows, double *y)
+void or_linear_fwd_int4_g(const float *xrot, const uint8_t *codes, const uint16_t *scales, int group,
+                          const double *t, const uint16_t *U,
+                          int64_t M, int64_t N, int64_t K,
+                          const int64_t *rows, int64_t n_rows, double *y)
 {
     (void)M;
     double *xb = (double *)malloc((size_t)(n_rows * K) * sizeof(double));
@@ -605,7 +710,7 @@ void or_linear_fwd_int4(const float *xrot, const uint8_t *codes, const uint16_t 
             uint8_t byte = codes[n * (K / 2) + k / 2];
             int nib = (k & 1) ? (byte >> 4) : (byte & 0xF);
             int q = nib >= 8 ? nib - 16 : nib;
-            float s = or_f16_to_f32(scales[n * (K / 32) + k / 32]);
+            float s = or_f16_to_f32(scales[n * (K / group) + k / group]);
             float d = (float)q * s;                     /* exact */
             wb[k] = (double)or_bf16_to_f32(or_f32_to_bf16(d));
         }
@@ -624,6 +729,15 @@ void or_linear_fwd_int4(const float *xrot, const uint8_t *codes, const uint16_t 
     free(xb);
 }
 
+/* group 32 (scales [N, K/32]) */
+void or_linear_fwd_int4(const float *xrot, const uint8_t *codes, const uint16_t *scales,
+                        const double *t, const uint16_t *U,
+                        int64_t M, int64_t N, int64_t K,
+                        const int64_t *rows, int64_t n_rows, double *y)
+{
+    or_linear_fwd_int4_g(xrot, codes, scales, 32, t, U, M, N, K, rows, n_rows, y);
+}
+
 /* ------------------------------------------------------------------------ */
 /* O9: bf16 reconstruct of W from the payload                                */
 /* ------------------------------------------------------------------------ */
@@ -635,7 +749,8 @@ void or_linear_fwd_int4(const float *xrot, const uint8_t *codes, const uint16_t 
  *   h = inverse_H256 of d over each 256-block of the row (= the same FWHT),
  *   L = fmaf chain over r = 0..31 of U[n,r] * D[k,r], starting from 0.
  * residual_only drops L: W = bf16(h).
- * fmt: 1 = int4 g32 (scales fp16 [N, K/32]), 2 = NVFP4 (sf tiled, g_w).
+ * fmt: 1 = int4 g32 (scales fp16 [N, K/32]), 2 = NVFP4 (sf tiled, g_w),
+ * 3 = int4 g64 (scales fp16 [N, K/64]).
  */
 void or_reconstruct_bf16(int fmt, const uint8_t *codes, const void *scales, float g_w,
                          const uint16_t *U, const uint16_t *D,
@@ -650,9 +765,10 @@ void or_reconstruct_bf16(int fmt, const uint8_t *codes, const void *scales, floa
                 int64_t k = b + i;
                 uint8_t byte = codes[n * (K / 2) + k / 2];
                 uint8_t nib = (k & 1) ? (byte >> 4) : (byte & 0xF);
-                if (fmt == 1) {
+                if (fmt == 1 || fmt == 3) {
+                    const int64_t G = fmt == 3 ? 64 : 32;
                     int q = nib >= 8 ? (int)nib - 16 : (int)nib;
-                    float s = or_f16_to_f32(((const uint16_t *)scales)[n * (K / 32) + k / 32]);
+                    float s = or_f16_to_f32(((const uint16_t *)scales)[n * (K / G) + k / G]);
                     v[i] = (float)q * s;
                 } else {
                     float dec = or_ue4m3_to_f32(((const uint8_t *)scales)[or_sf_offset(n, k / 16, C)]);
