@@ -4,7 +4,8 @@
 One step = one pass of the whole hot path over one synthetic layer of the
 chosen shape (default the headline 4480 x 16384 x 6144, M x N x K):
   sq_build_int4, sq_build_nvfp4, sq_linear_fwd (NVFP4, incl. the activation
-  prologue), sq_linear_fwd (int4), sq_reconstruct_bf16 (both payloads).
+  prologue), sq_linear_fwd (int4), sq_reconstruct_bf16 (both payloads), and the
+  int4 group-64 variant's build, forward and reconstruct.
 Every op is timed with CUDA events on the launching stream after an L2 flush
 (a 256 MB write outside the op's events); the NVFP4 forward is the headline
 metric (TFLOP/s = 2 M N K / time of the whole sq_linear_fwd call).  The GEMM
@@ -84,6 +85,9 @@ def op_work(M, N, K):
         "fwd_int4": ("TFLOP/s", 2.0 * M * N * K),
         "reconstruct_nvfp4": ("GB/s", NK * (0.5 + 1 / 16 + 2)),
         "reconstruct_int4": ("GB/s", NK * (0.5 + 2 / 32 + 2)),
+        "build_int4_g64": ("GB/s", NK * (4 + 0.5 + 2 / 64 + 1 / 64)),
+        "fwd_int4_g64": ("TFLOP/s", 2.0 * M * N * K),
+        "reconstruct_int4_g64": ("GB/s", NK * (0.5 + 2 / 64 + 2)),
         "gemm_nvfp4": ("TFLOP/s", 2.0 * M * N * K),
         "gemm_int4": ("TFLOP/s", 2.0 * M * N * K),
     }
@@ -92,6 +96,7 @@ def op_work(M, N, K):
 LAUNCHES_PER_STEP = {   # our kernels per op (memsets excluded)
     "build_int4": 1, "build_nvfp4": 2, "fwd_nvfp4": 5, "fwd_int4": 5,
     "reconstruct_nvfp4": 1, "reconstruct_int4": 1,
+    "build_int4_g64": 1, "fwd_int4_g64": 5, "reconstruct_int4_g64": 1,
 }
 
 
@@ -225,6 +230,17 @@ def cpu_sample(d, M_s: int, N_s: int):
     t0 = time.perf_counter()
     oracle.reconstruct_bf16(1, c4, s4, 0.0, U, D, N_s, K)
     t["reconstruct_int4"] = time.perf_counter() - t0
+    t0 = time.perf_counter()
+    c6, s6, _ = oracle.build_int4(R, group=64)
+    t["build_int4_g64"] = time.perf_counter() - t0
+    t0 = time.perf_counter()
+    xr = oracle.rotate_rows_bf16(x)
+    _, _, _, tt3 = oracle.act_quant_nvfp4(x, D)
+    oracle.linear_fwd_int4(xr, c6, s6, tt3, U, M_s, N_s, K, group=64)
+    t["fwd_int4_g64"] = time.perf_counter() - t0
+    t0 = time.perf_counter()
+    oracle.reconstruct_bf16(oracle.FMT_INT4_G64, c6, s6, 0.0, U, D, N_s, K)
+    t["reconstruct_int4_g64"] = time.perf_counter() - t0
     return t, oracle.num_threads()
 
 
@@ -282,7 +298,8 @@ def workload_config(cfg, args):
                     f"seed {cfg.seed}, {cfg.dist} residual" + (f", {cfg.hot_channels} hot channels"
                                                               if cfg.hot_channels else ""),
         "name": cfg.name, "M": cfg.M, "N": cfg.N, "K": cfg.K, "rank": 32,
-        "codecs": ["nvfp4 (e2m1, ue4m3 block-16, fp32 global)", "int4 group-32 MSE-swept"],
+        "codecs": ["nvfp4 (e2m1, ue4m3 block-16, fp32 global)", "int4 group-32 MSE-swept",
+                   "int4 group-64 MSE-swept"],
         "l2": "flushed (256 MB write) before every op, outside its events",
         "parallelism": f"replicas x{args.gpus}",
     }
@@ -312,6 +329,9 @@ def run_sq(args, cfg, d, rank, world, local_rank):
     nv = sq.Weight(sq.SQ_FMT_NVFP4, N, K, torch.empty((N, K // 2), dtype=torch.uint8, device=dev),
                    torch.empty(sq.sq_sf_bytes(N, K), dtype=torch.uint8, device=dev),
                    torch.empty(1, dtype=torch.float32, device=dev), U, D)
+    i6 = sq.Weight(sq.SQ_FMT_INT4_G64, N, K, torch.empty((N, K // 2), dtype=torch.uint8, device=dev),
+                   torch.empty((N, K // 64), dtype=torch.float16, device=dev), None, U, D,
+                   torch.empty((N, K // 64), dtype=torch.uint8, device=dev))
     ws_b = sq.workspace(sq.SQ_OP_BUILD_NVFP4, 0, N, K, dev)
     ws_nv = sq.workspace(sq.SQ_OP_LINEAR_FWD_NVFP4, M, N, K, dev)
     ws_i4 = sq.workspace(sq.SQ_OP_LINEAR_FWD_INT4, M, N, K, dev)
@@ -328,6 +348,9 @@ def run_sq(args, cfg, d, rank, world, local_rank):
         ("fwd_int4", lambda: sq.sq_linear_fwd(i4, x, y_i4, ws=ws_i4)),
         ("reconstruct_nvfp4", lambda: sq.sq_reconstruct_bf16(nv, W)),
         ("reconstruct_int4", lambda: sq.sq_reconstruct_bf16(i4, W)),
+        ("build_int4_g64", lambda: sq.sq_build_int4(R, i6.codes, i6.scales, i6.frac_idx, group=64)),
+        ("fwd_int4_g64", lambda: sq.sq_linear_fwd(i6, x, y_i4, ws=ws_i4)),
+        ("reconstruct_int4_g64", lambda: sq.sq_reconstruct_bf16(i6, W)),
     ]
     names = [n for n, _ in ops]
     gemm_of = {"fwd_nvfp4": "gemm_nvfp4", "fwd_int4": "gemm_int4"}

@@ -24,6 +24,7 @@ LIB_PATH = os.environ.get("SQ_LIBSQ_PATH") or os.path.join(_HERE, "libsq.so")
 SQ_OK = 0
 SQ_FMT_INT4_G32 = 1
 SQ_FMT_NVFP4 = 2
+SQ_FMT_INT4_G64 = 3
 SQ_OP_BUILD_INT4 = 1
 SQ_OP_BUILD_NVFP4 = 2
 SQ_OP_ACT_QUANT_NVFP4 = 3
@@ -215,11 +216,11 @@ class Weight:
     N: int
     K: int
     codes: torch.Tensor                  # uint8 [N, K/2]
-    scales: torch.Tensor                 # int4: float16 [N, K/32]; NVFP4: uint8 tiled
+    scales: torch.Tensor                 # int4: float16 [N, K/group]; NVFP4: uint8 tiled
     g_w: torch.Tensor | None = None      # float32 [1] (NVFP4)
     lora_up: torch.Tensor | None = None  # bf16 [N, 32]
     lora_down: torch.Tensor | None = None  # bf16 [K, 32]
-    frac_idx: torch.Tensor | None = None  # uint8 [N, K/32] (int4)
+    frac_idx: torch.Tensor | None = None  # uint8 [N, K/group] (int4)
 
     def as_c(self) -> sq_weight:
         return sq_weight(self.fmt, self.N, self.K, _ptr(self.codes), _ptr(self.scales), _ptr(self.g_w),
@@ -231,14 +232,15 @@ def workspace(op: int, M: int, N: int, K: int, device=None) -> torch.Tensor:
     return torch.empty(n, dtype=torch.uint8, device=device or "cuda")
 
 
-def build_int4(R: torch.Tensor, lora_up=None, lora_down=None, stream=None) -> Weight:
+def build_int4(R: torch.Tensor, lora_up=None, lora_down=None, group: int = 32, stream=None) -> Weight:
     N, K = R.shape
     dev = R.device
     codes = torch.empty((N, K // 2), dtype=torch.uint8, device=dev)
-    scales = torch.empty((N, K // 32), dtype=torch.float16, device=dev)
-    frac = torch.empty((N, K // 32), dtype=torch.uint8, device=dev)
-    sq_build_int4(R, codes, scales, frac, stream=stream)
-    return Weight(SQ_FMT_INT4_G32, N, K, codes, scales, None, lora_up, lora_down, frac)
+    scales = torch.empty((N, K // group), dtype=torch.float16, device=dev)
+    frac = torch.empty((N, K // group), dtype=torch.uint8, device=dev)
+    sq_build_int4(R, codes, scales, frac, group=group, stream=stream)
+    fmt = SQ_FMT_INT4_G64 if group == 64 else SQ_FMT_INT4_G32
+    return Weight(fmt, N, K, codes, scales, None, lora_up, lora_down, frac)
 
 
 def build_nvfp4(R: torch.Tensor, lora_up=None, lora_down=None, ws=None, stream=None) -> Weight:

@@ -139,7 +139,7 @@ sq_status check_weight(const sq_weight *w)
 {
     if (!w || !w->codes || !w->scales)
         return SQ_ERR_NULL;
-    if (w->fmt != SQ_FMT_INT4_G32 && w->fmt != SQ_FMT_NVFP4)
+    if (w->fmt != SQ_FMT_INT4_G32 && w->fmt != SQ_FMT_NVFP4 && w->fmt != SQ_FMT_INT4_G64)
         return SQ_ERR_ARG;
     if (w->fmt == SQ_FMT_NVFP4 && !w->g_w)
         return SQ_ERR_NULL;
@@ -214,7 +214,7 @@ sq_status sq_build_int4(const float *R, int64_t N, int64_t K, int32_t group, uin
 {
     if (!R || !codes || !scales)
         return SQ_ERR_NULL;
-    if (group != 32 || !shape_ok_nk(N, K))
+    if ((group != 32 && group != 64) || !shape_ok_nk(N, K))
         return SQ_ERR_SHAPE;
     if (!aligned(R, 16) || !aligned(codes, 16) || !aligned(scales, 16) || !aligned(frac_idx, 16))
         return SQ_ERR_ALIGN;
@@ -223,7 +223,7 @@ sq_status sq_build_int4(const float *R, int64_t N, int64_t K, int32_t group, uin
     if (st != SQ_OK)
         return st;
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-    SQ_CUDA(sq::launch_int4_build(R, N, K, codes, scales, frac_idx, sms, s), "int4 build");
+    SQ_CUDA(sq::launch_int4_build(R, N, K, group, codes, scales, frac_idx, sms, s), "int4 build");
     return SQ_OK;
 }
 
@@ -358,7 +358,8 @@ sq_status sq_linear_fwd(const sq_weight *w, const uint16_t *x, int64_t M, float 
         uint16_t *xb = reinterpret_cast<uint16_t *>(ws_at(ws, L.a));
         uint16_t *wb = reinterpret_cast<uint16_t *>(ws_at(ws, L.b));
         SQ_CUDA(sq::launch_rotate_bf16(x, M, K, xb, sms, s), "rotate x");
-        SQ_CUDA(sq::launch_dequant_int4(w->codes, reinterpret_cast<const uint16_t *>(w->scales), N, K, wb, sms, s),
+        SQ_CUDA(sq::launch_dequant_int4(w->codes, reinterpret_cast<const uint16_t *>(w->scales),
+                                        w->fmt == SQ_FMT_INT4_G64 ? 64 : 32, N, K, wb, sms, s),
                 "dequant");
         if (lora) {
             SQ_CUDA(sq::launch_act_pass1(x, M, K, w->lora_down, nullptr, t32, status, sms, s), "low-rank input");

@@ -28,16 +28,17 @@ cudaError_t launch_nvfp4_quant_f32(const float *in, int64_t rows, int64_t K, con
 cudaError_t launch_nvfp4_quant_bf16(const uint16_t *in, int64_t rows, int64_t K, const uint32_t *amax,
                                     const float *g_static, float *g_out, uint8_t *codes, uint8_t *sf,
                                     const LowrankOut &lr, int sms, cudaStream_t s);
-cudaError_t launch_int4_build(const float *R, int64_t N, int64_t K, uint8_t *codes, uint16_t *scales,
+cudaError_t launch_int4_build(const float *R, int64_t N, int64_t K, int group, uint8_t *codes, uint16_t *scales,
                               uint8_t *frac, int sms, cudaStream_t s);
 cudaError_t launch_rotate_bf16(const uint16_t *x, int64_t M, int64_t K, uint16_t *xb, int sms, cudaStream_t s);
-cudaError_t launch_dequant_int4(const uint8_t *codes, const uint16_t *scales, int64_t N, int64_t K, uint16_t *wb,
-                                int sms, cudaStream_t s);
+cudaError_t launch_dequant_int4(const uint8_t *codes, const uint16_t *scales, int group, int64_t N, int64_t K,
+                                uint16_t *wb, int sms, cudaStream_t s);
 cudaError_t launch_act_pass1(const uint16_t *x, int64_t M, int64_t K, const uint16_t *D, uint32_t *amax,
                              float *t32, uint32_t *status, int sms, cudaStream_t s);
 cudaError_t launch_lowrank_finish(const float *t32, int64_t M, const float *g_x, const float *g_w,
                                   uint16_t *tsplit, const uint16_t *U, int64_t N, uint16_t *udup, int sms,
                                   cudaStream_t s);
+// fmt: 1 int4 group 32, 2 NVFP4, 3 int4 group 64
 cudaError_t launch_reconstruct(int fmt, const uint8_t *codes, const void *scales, const float *g_w,
                                const uint16_t *U, const uint16_t *D, int64_t N, int64_t K, int with_lowrank,
                                uint16_t *W, int sms, cudaStream_t s);

@@ -286,11 +286,14 @@ __global__ void __launch_bounds__(kStreamThreads) nvfp4_quant_kernel(const __gri
 }
 
 // ---------------------------------------------------------------------------
-// int4 group-32 builder.  With the 8-lane Hadamard layout every lane holds one
-// whole group of 32 rotated values and sweeps the 26 scale fractions in
-// registers (group index = 8 * block + lane % 8).
+// int4 builder, group 32 or 64.  With the 8-lane Hadamard layout every lane
+// holds 32 consecutive rotated values: one whole group of 32 (group index
+// 8 * block + lane % 8), or one half of a group of 64 whose other half sits in
+// the neighbouring lane (lane ^ 1; group index 4 * block + (lane % 8) / 2).
+// Each lane sweeps the 26 scale fractions in registers; for group 64 the two
+// lanes of a pair share the absmax and add their half errors.
 // ---------------------------------------------------------------------------
-// sum of RN((r_i - q_i s)^2) over the group, as lane 0 of an xor butterfly over
+// sum of RN((r_i - q_i s)^2) over 32 values, as lane 0 of an xor butterfly over
 // strides 16, 8, 4, 2, 1; rp holds the 32 rotated values as pairs (r_2j, r_2j+1).
 // q = clamp(rint(r inv), -7, 7): |r inv| <= 14, so adding and subtracting
 // 1.5 * 2^23 rounds to the nearest integer, ties to even, exactly like rint (and
@@ -336,20 +339,26 @@ __constant__ float kFrac[26] = {
     78.0f / 100, 80.0f / 100, 82.0f / 100, 84.0f / 100, 86.0f / 100, 88.0f / 100, 90.0f / 100,
     92.0f / 100, 94.0f / 100, 96.0f / 100, 98.0f / 100, 100.0f / 100};
 
+template <int G>
 __global__ void __launch_bounds__(kStreamThreads, 2) int4_build_kernel(const __grid_constant__ CUtensorMap tm,
                                                                     int64_t blocks, uint8_t *__restrict__ codes,
                                                                     uint16_t *__restrict__ scales,
                                                                     uint8_t *__restrict__ frac)
 {
+    static_assert(G == 32 || G == 64, "group 32 or 64");
     const int lane = threadIdx.x & 31;
     stream_blocks<float>(&tm, blocks, nullptr, [&](int64_t b, float (&r)[32], bool valid) {
         fwht256_l32(r, lane);
-        if (!valid)
+        // group 64: both lanes of a pair run the sweep (shuffles), so no lane leaves before it;
+        // blocks past the tensor are zero-filled and only their stores are skipped
+        if (G == 32 && !valid)
             return;
         float a = 0.0f;
 #pragma unroll
         for (int i = 0; i < 32; i += 2)
             a = fmax3(a, fabsf(r[i]), fabsf(r[i + 1]));
+        if (G == 64)
+            a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, 1));
         uint64_t rp[16];
 #pragma unroll
         for (int j = 0; j < 16; ++j)
@@ -363,7 +372,9 @@ __global__ void __launch_bounds__(kStreamThreads, 2) int4_build_kernel(const __g
             const __half hs = __float2half_rn(__fdiv_rn(__fmul_rn(f, a), 7.0f));
             const float s = __half2float(hs);
             const float inv = s == 0.0f ? 0.0f : __frcp_rn(s);
-            const float mse = group_sq_error(rp, s, inv);
+            float mse = group_sq_error(rp, s, inv);
+            if (G == 64)                               // first half + second half (addition commutes)
+                mse = __fadd_rn(mse, __shfl_xor_sync(0xffffffffu, mse, 1));
             if (j == 0 || mse < best) {
                 best = mse;
                 best_j = j;
@@ -371,6 +382,8 @@ __global__ void __launch_bounds__(kStreamThreads, 2) int4_build_kernel(const __g
                 best_h = __half_as_ushort(hs);
             }
         }
+        if (!valid)
+            return;
         // codes for the winning scale (same arithmetic as in the sweep)
         const float inv = best_s == 0.0f ? 0.0f : __frcp_rn(best_s);
         uint32_t word[4] = {0u, 0u, 0u, 0u};
@@ -385,11 +398,14 @@ __global__ void __launch_bounds__(kStreamThreads, 2) int4_build_kernel(const __g
             }
             word[i >> 3] |= (((uint32_t)q0 & 0xFu) | (((uint32_t)q1 & 0xFu) << 4)) << (4 * (i & 7));
         }
-        const int64_t gidx = 8 * b + (lane & 7);     // flat group index
-        reinterpret_cast<uint4 *>(codes)[gidx] = make_uint4(word[0], word[1], word[2], word[3]);
-        scales[gidx] = best_h;
-        if (frac)
-            frac[gidx] = (uint8_t)best_j;
+        const int64_t hidx = 8 * b + (lane & 7);     // flat index of this lane's 32 values
+        reinterpret_cast<uint4 *>(codes)[hidx] = make_uint4(word[0], word[1], word[2], word[3]);
+        if (G == 32 || (lane & 1) == 0) {
+            const int64_t gidx = G == 32 ? hidx : hidx >> 1;
+            scales[gidx] = best_h;
+            if (frac)
+                frac[gidx] = (uint8_t)best_j;
+        }
     });
 }
 
@@ -417,16 +433,18 @@ __global__ void __launch_bounds__(kStreamThreads) rotate_bf16_kernel(const __gri
 }
 
 // ---------------------------------------------------------------------------
-// int4 "dequant-first": wb[n, k] = bf16(q s), 8 values per thread
+// int4 "dequant-first": wb[n, k] = bf16(q s), 8 values per thread, group G
 // ---------------------------------------------------------------------------
+template <int G>
 __global__ void __launch_bounds__(256) dequant_int4_kernel(const uint32_t *__restrict__ codes,
                                                            const uint16_t *__restrict__ scales,
                                                            int64_t total8, uint4 *__restrict__ wb)
 {
+    constexpr int kWordsLog2 = G == 64 ? 3 : 2;      // 8-value code words per group
     for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < total8;
          i += (int64_t)gridDim.x * blockDim.x) {
         const uint32_t c = __ldg(codes + i);
-        const float s = __half2float(__ushort_as_half(__ldg(scales + (i >> 2))));  // 4 words per group
+        const float s = __half2float(__ushort_as_half(__ldg(scales + (i >> kWordsLog2))));
         uint32_t o[4];
 #pragma unroll
         for (int p = 0; p < 4; ++p) {
@@ -788,8 +806,14 @@ __device__ __forceinline__ void cp_async4(uint32_t dst, const void *src, uint32_
     asm volatile("cp.async.ca.shared.global [%0], [%1], 4, %2;" ::"r"(dst), "l"(src), "r"(src_bytes) : "memory");
 }
 
+__device__ __forceinline__ void cp_async8(uint32_t dst, const void *src, uint32_t src_bytes)
+{
+    asm volatile("cp.async.ca.shared.global [%0], [%1], 8, %2;" ::"r"(dst), "l"(src), "r"(src_bytes) : "memory");
+}
+
 // Stage tile (kb, rows n0..n0+63) into one buffer: codes [64][128 B], scales
-// [64][16 B] (int4: the 8 fp16 group scales; NVFP4: the 16 ue4m3 block scales,
+// [64][16 B] (int4 group 32: the 8 fp16 group scales; int4 group 64: the 4 fp16
+// group scales in the first 8 bytes; NVFP4: the 16 ue4m3 block scales,
 // gathered from the tiled layout 4 bytes at a time), lora_up [64][64 B].
 // Rows past N are zero filled.
 template <int FMT, bool LOWRANK>
@@ -812,6 +836,13 @@ __device__ __forceinline__ void rec_stage(uint32_t buf, const uint8_t *codes, co
                                        : reinterpret_cast<const uint8_t *>(scales);
             cp_async16(sbuf + 16 * tid, src, n < N ? 16u : 0u);
         }
+    } else if (FMT == 3) {
+        if (tid < kRecRows) {                        // 4 scales = 8 bytes, 8-byte aligned (K % 256 == 0)
+            const int64_t n = n0 + tid;
+            const uint8_t *src = n < N ? reinterpret_cast<const uint8_t *>(scales) + (n * (K / 64) + kb * 4) * 2
+                                       : reinterpret_cast<const uint8_t *>(scales);
+            cp_async8(sbuf + 16 * tid, src, n < N ? 8u : 0u);
+        }
     } else {
         const int r = tid >> 2, j = tid & 3;
         const int64_t n = n0 + r;
@@ -828,15 +859,16 @@ __device__ __forceinline__ void rec_stage(uint32_t buf, const uint8_t *codes, co
     }
 }
 
-// 32 payload values of staged row r, group q (values 32q..32q+31 of the block)
+// 32 payload values of staged row r, values 32q..32q+31 of the block (one int4
+// group of 32, half of a group of 64, or two NVFP4 blocks)
 template <int FMT>
 __device__ __forceinline__ void rec_decode(const uint8_t *stage, int r, int q, float g, float (&v)[32])
 {
     const uint4 c = *reinterpret_cast<const uint4 *>(stage + r * 128 + 16 * q);
     const uint32_t w[4] = {c.x, c.y, c.z, c.w};
     const uint8_t *sc = stage + kRecCodeBytes + 16 * r;
-    if (FMT == 1) {
-        const float s = __half2float(*reinterpret_cast<const __half *>(sc + 2 * q));
+    if (FMT == 1 || FMT == 3) {
+        const float s = __half2float(*reinterpret_cast<const __half *>(sc + 2 * (FMT == 3 ? q >> 1 : q)));
 #pragma unroll
         for (int i = 0; i < 32; ++i) {
             int qq = (int)((w[i >> 3] >> (4 * (i & 7))) & 0xFu);
@@ -1019,9 +1051,10 @@ static bool stream_map(CUtensorMap *tm, const T *in, int64_t rows, int64_t K)
                      32, (uint64_t)(rows * K / 32), 32, 256, f32 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B);
 }
 
-// shared-memory opt-in, once per device and kernel
-template <typename T, typename Kern>
-static cudaError_t stream_attr(Kern k)
+// shared-memory opt-in, once per device and kernel (keyed on the kernel itself:
+// kernels with the same signature must not share the flag)
+template <typename T, auto k>
+static cudaError_t stream_attr()
 {
     constexpr int kMaxDev = 64;
     static bool done[kMaxDev];
@@ -1049,7 +1082,7 @@ static cudaError_t launch_absmax_rot(const T *in, int64_t rows, int64_t K, uint3
     CUtensorMap tm;
     if (!stream_map(&tm, in, rows, K))
         return cudaErrorInvalidValue;
-    cudaError_t e = stream_attr<T>(absmax_rot_kernel<T>);
+    cudaError_t e = stream_attr<T, absmax_rot_kernel<T>>();
     if (e != cudaSuccess)
         return e;
     const int64_t blocks = rows * (K / kHad);
@@ -1066,7 +1099,7 @@ static cudaError_t launch_nvfp4_quant(const T *in, int64_t rows, int64_t K, cons
     CUtensorMap tm;
     if (!stream_map(&tm, in, rows, K))
         return cudaErrorInvalidValue;
-    cudaError_t e = stream_attr<T>(nvfp4_quant_kernel<T>);
+    cudaError_t e = stream_attr<T, nvfp4_quant_kernel<T>>();
     if (e != cudaSuccess)
         return e;
     const int64_t rows_pad = (rows + 127) / 128 * 128;
@@ -1110,18 +1143,26 @@ cudaError_t launch_nvfp4_quant_bf16(const uint16_t *in, int64_t rows, int64_t K,
     return launch_nvfp4_quant(in, rows, K, amax, g_static, g_out, codes, sf, lr, sms, s);
 }
 
-cudaError_t launch_int4_build(const float *R, int64_t N, int64_t K, uint8_t *codes, uint16_t *scales,
+cudaError_t launch_int4_build(const float *R, int64_t N, int64_t K, int group, uint8_t *codes, uint16_t *scales,
                               uint8_t *frac, int sms, cudaStream_t s)
 {
     CUtensorMap tm;
     if (!stream_map(&tm, R, N, K))
         return cudaErrorInvalidValue;
-    cudaError_t e = stream_attr<float>(int4_build_kernel);
+    cudaError_t e = stream_attr<float, int4_build_kernel<32>>();
     if (e != cudaSuccess)
         return e;
     const int64_t blocks = N * K / kHad;
-    int4_build_kernel<<<stream_grid(blocks, sms, 2), kStreamThreads, StreamCfg<float>::kSmem, s>>>(tm, blocks, codes,
-                                                                                                   scales, frac);
+    if (group == 64) {
+        e = stream_attr<float, int4_build_kernel<64>>();
+        if (e != cudaSuccess)
+            return e;
+        int4_build_kernel<64><<<stream_grid(blocks, sms, 2), kStreamThreads, StreamCfg<float>::kSmem, s>>>(
+            tm, blocks, codes, scales, frac);
+    } else {
+        int4_build_kernel<32><<<stream_grid(blocks, sms, 2), kStreamThreads, StreamCfg<float>::kSmem, s>>>(
+            tm, blocks, codes, scales, frac);
+    }
     return cudaGetLastError();
 }
 
@@ -1130,7 +1171,7 @@ cudaError_t launch_rotate_bf16(const uint16_t *x, int64_t M, int64_t K, uint16_t
     CUtensorMap tm;
     if (!stream_map(&tm, x, M, K))
         return cudaErrorInvalidValue;
-    cudaError_t e = stream_attr<uint16_t>(rotate_bf16_kernel);
+    cudaError_t e = stream_attr<uint16_t, rotate_bf16_kernel>();
     if (e != cudaSuccess)
         return e;
     const int64_t blocks = M * (K / kHad);
@@ -1138,12 +1179,16 @@ cudaError_t launch_rotate_bf16(const uint16_t *x, int64_t M, int64_t K, uint16_t
     return cudaGetLastError();
 }
 
-cudaError_t launch_dequant_int4(const uint8_t *codes, const uint16_t *scales, int64_t N, int64_t K,
+cudaError_t launch_dequant_int4(const uint8_t *codes, const uint16_t *scales, int group, int64_t N, int64_t K,
                                 uint16_t *wb, int sms, cudaStream_t s)
 {
     const int64_t total8 = N * K / 8;
-    dequant_int4_kernel<<<grid_for(total8, 256, sms, 8), 256, 0, s>>>(
-        reinterpret_cast<const uint32_t *>(codes), scales, total8, reinterpret_cast<uint4 *>(wb));
+    if (group == 64)
+        dequant_int4_kernel<64><<<grid_for(total8, 256, sms, 8), 256, 0, s>>>(
+            reinterpret_cast<const uint32_t *>(codes), scales, total8, reinterpret_cast<uint4 *>(wb));
+    else
+        dequant_int4_kernel<32><<<grid_for(total8, 256, sms, 8), 256, 0, s>>>(
+            reinterpret_cast<const uint32_t *>(codes), scales, total8, reinterpret_cast<uint4 *>(wb));
     return cudaGetLastError();
 }
 
@@ -1219,6 +1264,9 @@ cudaError_t launch_reconstruct(int fmt, const uint8_t *codes, const void *scales
         if (e == cudaSuccess)
             e = cudaFuncSetAttribute(reconstruct_kernel<2, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                      kRecSmemLowrank);
+        if (e == cudaSuccess)
+            e = cudaFuncSetAttribute(reconstruct_kernel<3, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                     kRecSmemLowrank);
         if (e != cudaSuccess)
             return e;
         attr_done[dev] = true;
@@ -1232,6 +1280,11 @@ cudaError_t launch_reconstruct(int fmt, const uint8_t *codes, const void *scales
             reconstruct_kernel<2, true><<<grid, 256, smem, s>>>(codes, scales, g_w, U, D, N, K, W);
         else
             reconstruct_kernel<2, false><<<grid, 256, smem, s>>>(codes, scales, g_w, U, D, N, K, W);
+    } else if (fmt == 3) {
+        if (with_lowrank)
+            reconstruct_kernel<3, true><<<grid, 256, smem, s>>>(codes, scales, g_w, U, D, N, K, W);
+        else
+            reconstruct_kernel<3, false><<<grid, 256, smem, s>>>(codes, scales, g_w, U, D, N, K, W);
     } else {
         if (with_lowrank)
             reconstruct_kernel<1, true><<<grid, 256, smem, s>>>(codes, scales, g_w, U, D, N, K, W);

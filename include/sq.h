@@ -53,7 +53,7 @@ extern "C" {
 typedef enum {
     SQ_OK = 0,
     SQ_ERR_NULL = 1,       /* a required pointer is NULL                          */
-    SQ_ERR_SHAPE = 2,      /* K % 256, N % 128, M < 1, group != 32, or too large  */
+    SQ_ERR_SHAPE = 2,      /* K % 256, N % 128, M < 1, group not 32/64, too large */
     SQ_ERR_ALIGN = 3,      /* pointer not 16-byte (workspace: 256-byte) aligned   */
     SQ_ERR_WORKSPACE = 4,  /* workspace smaller than sq_workspace_bytes()         */
     SQ_ERR_DEVICE = 5,     /* current device is not sm_100 (B200 class)          */
@@ -64,7 +64,8 @@ typedef enum {
 
 typedef enum {
     SQ_FMT_INT4_G32 = 1,   /* int4 codes [N, K/2], fp16 scales [N, K/32]          */
-    SQ_FMT_NVFP4 = 2       /* e2m1 codes [N, K/2], ue4m3 tiled scales, fp32 g_w   */
+    SQ_FMT_NVFP4 = 2,      /* e2m1 codes [N, K/2], ue4m3 tiled scales, fp32 g_w   */
+    SQ_FMT_INT4_G64 = 3    /* int4 codes [N, K/2], fp16 scales [N, K/64]          */
 } sq_format;
 
 /* operations for sq_workspace_bytes() */
@@ -83,12 +84,12 @@ typedef enum {
 
 /*
  * A built weight.  All pointers are device pointers owned by the caller.
- *   fmt        SQ_FMT_INT4_G32 or SQ_FMT_NVFP4
+ *   fmt        SQ_FMT_INT4_G32, SQ_FMT_INT4_G64 or SQ_FMT_NVFP4
  *   N, K       output / input features
  *   codes      [N, K/2] uint8, value 2k in the low nibble of byte k
  *              (int4: 4-bit two's complement in [-7, 7]; NVFP4: e2m1)
- *   scales     int4: fp16 bits [N, K/32]; NVFP4: ue4m3 bytes in the tiled
- *              layout, sq_sf_bytes(N, K) bytes
+ *   scales     int4: fp16 bits [N, K/32] (group 32) or [N, K/64] (group 64);
+ *              NVFP4: ue4m3 bytes in the tiled layout, sq_sf_bytes(N, K) bytes
  *   g_w        NVFP4 only: 1 float, the per-tensor global scale
  *   lora_up    bf16 [N, 32], or NULL for no low-rank branch
  *   lora_down  bf16 [K, 32], or NULL for no low-rank branch
@@ -130,16 +131,19 @@ SQ_API size_t sq_sf_bytes(int64_t rows, int64_t K);
 SQ_API size_t sq_workspace_bytes(int op, int64_t M, int64_t N, int64_t K);
 
 /*
- * int4 group-32 builder (SquareQ README, "Residual codecs": int4 group-32
- * scales with MSE-swept fractions).  For each row of R [N, K] fp32 (device):
- * rotate every 256-block with H256, then for each group of 32 rotated values
- * r_i with a = max|r_i| try the fractions f_j = (50 + 2j)/100, j = 0..25:
+ * int4 builder (SquareQ README, "Residual codecs": int4 group-32/64 scales
+ * with MSE-swept fractions).  For each row of R [N, K] fp32 (device): rotate
+ * every 256-block with H256, then for each group of `group` (32 or 64)
+ * rotated values r_i with a = max|r_i| try the fractions f_j = (50 + 2j)/100,
+ * j = 0..25:
  *   s_j = fp16(RN(RN(f_j a) / 7)),  q_i = clamp(rint(RN(r_i RN(1/s_j))), -7, 7),
  *   error_j = sum over an xor butterfly (strides 16,8,4,2,1) of RN((r_i - q_i s_j)^2)
- * (a scale of 0 gives q = 0 and error r_i^2); keep the smallest error, the
- * smaller j on ties.  Outputs (device): codes [N, K/2], scales fp16 bits
- * [N, K/32], frac_idx [N, K/32] winning j (may be NULL).  group must be 32.
- * Rotated values must stay below 458000 in magnitude (fp16 scale range).
+ * for each 32 consecutive values (group 64: the two 32-value sums added,
+ * RN(first + second)); a scale of 0 gives q = 0 and error r_i^2.  Keep the
+ * smallest error, the smaller j on ties.  Outputs (device): codes [N, K/2],
+ * scales fp16 bits [N, K/group], frac_idx [N, K/group] winning j (may be
+ * NULL).  The weight is then SQ_FMT_INT4_G32 or SQ_FMT_INT4_G64.  Rotated
+ * values must stay below 458000 in magnitude (fp16 scale range).
  */
 SQ_API sq_status sq_build_int4(const float *R, int64_t N, int64_t K, int32_t group,
                         uint8_t *codes, uint16_t *scales, uint8_t *frac_idx,
@@ -183,7 +187,8 @@ SQ_API sq_status sq_act_quant_nvfp4(const uint16_t *x, int64_t M, int64_t K,
  *          tensor-core GEMM (tcgen05, fp32 accumulation in tensor memory),
  *          y = g_x g_w acc + t lora_up^T.
  *   int4:  "dequant-first": xb = bf16(H x), wb = bf16(q s), y = xb wb^T +
- *          t lora_up^T on bf16 tensor cores (fp32 accumulation).
+ *          t lora_up^T on bf16 tensor cores (fp32 accumulation); either
+ *          group size (SQ_FMT_INT4_G32 / _G64).
  * The low-rank term is accumulated on the tensor cores in the same
  * accumulator.  Accuracy: max|y - y_exact| / max|y_exact| <= 2e-3 against the
  * exact result on the same quantised operands.  flags: SQ_ACT_STATIC_SCALE
@@ -232,7 +237,7 @@ SQ_API sq_status sq_linear_fwd_noalloc(const sq_weight *w, const uint16_t *x, in
 /*
  * bf16 reconstruct of W for the backward pass (SquareQ README: "the bwd-side
  * bf16 reconstruct from the same payload").  For each element
- *   d = q s (int4) or RN(RN(e2m1 value(sf)) g_w) (NVFP4),
+ *   d = q s (int4, either group size) or RN(RN(e2m1 value(sf)) g_w) (NVFP4),
  *   h = H256 applied to each 256-block of d along K,
  *   L = fmaf(U[n,31], D[k,31], ... fmaf(U[n,0], D[k,0], 0)),
  *   W[n, k] = bf16(RN(L + h))          (bf16(h) with SQ_RECON_RESIDUAL_ONLY

@@ -66,7 +66,8 @@ def test_build_int4_validation():
     assert _int4(codes=None) == SQ_ERR_NULL
     assert _int4(K=300) == SQ_ERR_SHAPE
     assert _int4(N=100) == SQ_ERR_SHAPE
-    assert _int4(group=64) == SQ_ERR_SHAPE
+    assert _int4(group=16) == SQ_ERR_SHAPE
+    assert _int4(group=128) == SQ_ERR_SHAPE
     assert _int4(R=MIS) == SQ_ERR_ALIGN
     assert _int4(frac=MIS) == SQ_ERR_ALIGN
 
@@ -122,6 +123,9 @@ def test_reconstruct_validation():
 @pytest.mark.skipif(torch.cuda.is_available(), reason="checks the no-device path")
 def test_valid_call_without_device_reports_device_error():
     assert _int4() == SQ_ERR_DEVICE
+    assert _int4(group=64) == SQ_ERR_DEVICE            # group 64 passes validation
+    assert sq.lib().sq_reconstruct_bf16(ctypes.byref(_w(fmt=sq.SQ_FMT_INT4_G64, g_w=None)), A, 0, None) \
+        == SQ_ERR_DEVICE
     assert sq.lib().sq_reconstruct_bf16(ctypes.byref(_w()), A, 0, None) == SQ_ERR_DEVICE
 
 
