@@ -69,6 +69,10 @@ _SIGS = {
     "or_linear_fwd_nvfp4": ([_P, _P, _F, _P, _P, _F, _P, _P, _I64, _I64, _I64, _P, _I64, _P], None),
     "or_linear_fwd_int4": ([_P, _P, _P, _P, _P, _I64, _I64, _I64, _P, _I64, _P], None),
     "or_reconstruct_bf16": ([ctypes.c_int, _P, _P, _F, _P, _P, _I64, _I64, ctypes.c_int, _P], None),
+    "or_int8_row": ([_P, _I64, _P, _P, _P], None),
+    "or_build_int8": ([_P, _I64, _I64, _P, _P, _P], None),
+    "or_linear_fwd_int8": ([_P, _P, _P, _P, _P, _I64, _I64, _I64, _P, _I64, _P], None),
+    "or_lowrank_input": ([_P, _I64, _I64, _P, ctypes.c_int, _P], None),
 }
 
 
@@ -288,16 +292,66 @@ def linear_fwd_int4(xrot, codes, scales, t, U_bits, M, N, K, rows=None, group=32
     return y
 
 
+# ---- v3.1 int8 per-row codec (rank-16 low-rank branch) ---------------------
+
+RANK_INT8 = 16
+
+
+def int8_row(r):
+    """One rotated row (K % 256 == 0) -> (codes int8 [K], scale float32, winning j)."""
+    r = _c(r, np.float32)
+    K = r.shape[0]
+    q = np.empty(K, np.int8)
+    s = np.empty(1, np.float32)
+    j = np.empty(1, np.uint8)
+    lib().or_int8_row(_p(r), K, _p(q), _p(s), _p(j))
+    return q, np.float32(s[0]), int(j[0])
+
+
+def build_int8(R):
+    """R [N, K] fp32 -> (codes int8 [N, K], scales float32 [N], frac uint8 [N])."""
+    R = _c(R, np.float32)
+    N, K = R.shape
+    codes = np.empty((N, K), np.int8)
+    scales = np.empty(N, np.float32)
+    frac = np.empty(N, np.uint8)
+    lib().or_build_int8(_p(R), N, K, _p(codes), _p(scales), _p(frac))
+    return codes, scales, frac
+
+
+def lowrank_input(x_bits, lora_down_bits):
+    """t = x lora_down in fp64, [M, rank] (rank = lora_down's columns)."""
+    x = _c(x_bits, np.uint16)
+    D = _c(lora_down_bits, np.uint16)
+    M, K = x.shape
+    rank = D.shape[1]
+    t = np.empty((M, rank), np.float64)
+    lib().or_lowrank_input(_p(x), M, K, _p(D), rank, _p(t))
+    return t
+
+
+def linear_fwd_int8(xrot, codes, scales, t, U_bits, M, N, K, rows=None):
+    """y rows of the int8 forward, fp64 [n_rows, N]; t [M, 16] fp64 and U [N, 16] bf16 bits, or None."""
+    rows = np.arange(M, dtype=np.int64) if rows is None else _c(rows, np.int64)
+    y = np.empty((len(rows), N), np.float64)
+    t = None if t is None else _c(t, np.float64)
+    U = None if U_bits is None else _c(U_bits, np.uint16)
+    lib().or_linear_fwd_int8(_p(_c(xrot, np.float32)), _p(_c(codes, np.int8)), _p(_c(scales, np.float32)),
+                             _p(t), _p(U), M, N, K, _p(rows), len(rows), _p(y))
+    return y
+
+
 # ---- O9 reconstruct -------------------------------------------------------
 
 FMT_INT4 = 1
 FMT_NVFP4 = 2
 FMT_INT4_G64 = 3
+FMT_INT8_ROW = 4
 
 
 def reconstruct_bf16(fmt, codes, scales, g_w, U_bits, D_bits, N, K, residual_only=False):
-    codes = _c(codes, np.uint8)
-    scales = _c(scales, np.uint8 if fmt == FMT_NVFP4 else np.uint16)
+    codes = _c(codes, np.int8 if fmt == FMT_INT8_ROW else np.uint8)
+    scales = _c(scales, {FMT_NVFP4: np.uint8, FMT_INT8_ROW: np.float32}.get(fmt, np.uint16))
     U = _c(U_bits, np.uint16)
     D = _c(D_bits, np.uint16)
     W = np.empty((N, K), np.uint16)

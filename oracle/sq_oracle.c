@@ -11,10 +11,12 @@
  *     W = lora_up . lora_down^T + inverse_H256( dequant( residual ) )
  *
  * with a block-diagonal normalised Hadamard-256 over the input dim
- * ("Rotation" paragraph), an int4 group-32 codec with MSE-swept scale
+ * ("Rotation" paragraph), an int4 group-32/64 codec with MSE-swept scale
  * fractions or an NVFP4 codec (e2m1 codes, ue4m3 block-16 scales in the
  * cuBLASLt tiled layout, fp32 per-tensor global scale) ("Residual codecs"
- * paragraph), and a rank-32 bf16 low-rank branch ("Low-rank branch").
+ * paragraph), and a rank-32 bf16 low-rank branch ("Low-rank branch"); plus
+ * the v3.1 int8 mode (int8 per-row MSE-swept codes of the rotated residual,
+ * rank-16 low-rank branch; section "v3.1 -- int8-residual mode").
  *
  * Arithmetic rules (the pages fix none of them; these are the readings that
  * make bit-exact parity well defined):
@@ -739,6 +741,181 @@ void or_linear_fwd_int4(const float *xrot, const uint8_t *codes, const uint16_t 
 }
 
 /* ------------------------------------------------------------------------ */
+/* v3.1 int8 per-row codec (rank-16 low-rank branch)                         */
+/* ------------------------------------------------------------------------ */
+
+/*
+ * The squared-error sum of one row of K values p[0..K-1] (K % 256 == 0), in
+ * the order fixed for the int8 codec: inside each 256-block, every 32-value
+ * group is summed by the xor butterfly of the int4 codec (strides 16, 8, 4, 2,
+ * 1; element 0), the block's 8 group sums by an xor butterfly over the group
+ * index (strides 4, 2, 1; group 0), and the blocks are added in order from
+ * block 0: E = ((B_0 + B_1) + B_2) + ...  The pages print no order; this is
+ * the reading (one level more than the int4 group rule, then a plain running
+ * sum over the row).
+ */
+static float int8_row_error(const float *p_in, int64_t K)
+{
+    float E = 0.0f;
+    for (int64_t b = 0; b < K; b += 256) {
+        float g[8];
+        for (int k = 0; k < 8; k++) {
+            float p[32];
+            memcpy(p, p_in + b + 32 * k, sizeof(p));
+            for (int d = 16; d >= 1; d >>= 1) {
+                float nxt[32];
+                for (int i = 0; i < 32; i++)
+                    nxt[i] = p[i] + p[i ^ d];
+                memcpy(p, nxt, sizeof(p));
+            }
+            g[k] = p[0];
+        }
+        for (int d = 4; d >= 1; d >>= 1) {
+            float nxt[8];
+            for (int k = 0; k < 8; k++)
+                nxt[k] = g[k] + g[k ^ d];
+            memcpy(g, nxt, sizeof(g));
+        }
+        E = (b == 0) ? g[0] : E + g[0];
+    }
+    return E;
+}
+
+/*
+ * One row of K rotated residual values (SquareQ README, "v3.1 -- int8-residual
+ * mode": int8 per-row, MSE-swept, of the H256-rotated rank-16 residual).
+ * a = max|r_k| over the row; for each fraction f_j of the int4 sweep
+ * (j = 0..25) the fp32 scale is s = RN(RN(f_j a) / 127) and the codes
+ * q_k = clamp(rint_even(RN(r_k RN(1/s))), -127, 127); the error of value k is
+ * e_k = fmaf(-q_k, s, r_k) (r - q s with one rounding: q s is not exact in
+ * fp32 any more) and p_k = RN(e_k^2), summed by int8_row_error.  A scale of 0
+ * gives q = 0 and p_k = RN(r_k^2).  The smallest error wins, the smaller j on a
+ * tie.  Readings: the scale is kept in fp32 (one per row, so its bytes do not
+ * matter), the code range is symmetric (-128 is never used), the fraction grid
+ * is the int4 codec's.
+ */
+void or_int8_row(const float *r, int64_t K, int8_t *q_out, float *s_out, uint8_t *j_out)
+{
+    float a = 0.0f;
+    for (int64_t k = 0; k < K; k++) {
+        float m = fabsf(r[k]);
+        if (m > a)
+            a = m;
+    }
+    float *p = (float *)malloc((size_t)K * sizeof(float));
+    int8_t *q = (int8_t *)malloc((size_t)K);
+    float best = INFINITY;
+    int best_j = -1;
+    for (int j = 0; j < 26; j++) {
+        float f = or_int4_fraction(j);
+        float fa = f * a;
+        float s = fa / 127.0f;
+        if (s == 0.0f) {
+            for (int64_t k = 0; k < K; k++) {
+                q[k] = 0;
+                p[k] = r[k] * r[k];
+            }
+        } else {
+            float inv = 1.0f / s;
+            for (int64_t k = 0; k < K; k++) {
+                float v = r[k] * inv;
+                float rq = nearbyintf(v);
+                if (rq > 127.0f)
+                    rq = 127.0f;
+                if (rq < -127.0f)
+                    rq = -127.0f;
+                q[k] = (int8_t)rq;
+                float e = fmaf(-rq, s, r[k]);
+                p[k] = e * e;
+            }
+        }
+        float E = int8_row_error(p, K);
+        if (best_j < 0 || E < best) {
+            best = E;
+            best_j = j;
+            memcpy(q_out, q, (size_t)K);
+            *s_out = s;
+        }
+    }
+    *j_out = (uint8_t)best_j;
+    free(p);
+    free(q);
+}
+
+/*
+ * int8 builder: rotate each row of R [N, K] block-wise with H256, then the row
+ * codec.  codes [N, K] int8, scales [N] fp32, frac [N] (may be NULL).
+ */
+void or_build_int8(const float *R, int64_t N, int64_t K, int8_t *codes, float *scales, uint8_t *frac)
+{
+#pragma omp parallel for schedule(dynamic)
+    for (int64_t n = 0; n < N; n++) {
+        float *row = (float *)malloc((size_t)K * sizeof(float));
+        for (int64_t b = 0; b < K; b += 256) {
+            memcpy(row + b, R + n * K + b, 256 * sizeof(float));
+            or_fwht256(row + b);
+        }
+        uint8_t j;
+        or_int8_row(row, K, codes + n * K, scales + n, &j);
+        if (frac)
+            frac[n] = j;
+        free(row);
+    }
+}
+
+/*
+ * int8 forward ("dequant-first", as the int4 codec), fp64 on the exact operands:
+ *   xb = bf16(H(x)),  wb[n,k] = bf16(RN(q[n,k] * s[n])),
+ *   y[m,n] = sum_k xb wb + sum_{r<16} t[m,r] U[n,r]
+ * with the rank-16 branch: t [M, 16] fp64 = x lora_down, U [N, 16] bf16.
+ */
+void or_linear_fwd_int8(const float *xrot, const int8_t *codes, const float *scales,
+                        const double *t, const uint16_t *U,
+                        int64_t M, int64_t N, int64_t K,
+                        const int64_t *rows, int64_t n_rows, double *y)
+{
+    (void)M;
+    double *xb = (double *)malloc((size_t)(n_rows * K) * sizeof(double));
+    for (int64_t i = 0; i < n_rows; i++)
+        for (int64_t k = 0; k < K; k++)
+            xb[i * K + k] = (double)or_bf16_to_f32(or_f32_to_bf16(xrot[rows[i] * K + k]));
+#pragma omp parallel for schedule(static)
+    for (int64_t n = 0; n < N; n++) {
+        double *wb = (double *)malloc((size_t)K * sizeof(double));
+        for (int64_t k = 0; k < K; k++) {
+            float d = (float)codes[n * K + k] * scales[n];
+            wb[k] = (double)or_bf16_to_f32(or_f32_to_bf16(d));
+        }
+        for (int64_t i = 0; i < n_rows; i++) {
+            int64_t m = rows[i];
+            double acc = 0.0;
+            for (int64_t k = 0; k < K; k++)
+                acc += xb[i * K + k] * wb[k];
+            if (t)
+                for (int r = 0; r < 16; r++)
+                    acc += t[m * 16 + r] * (double)or_bf16_to_f32(U[n * 16 + r]);
+            y[i * N + n] = acc;
+        }
+        free(wb);
+    }
+    free(xb);
+}
+
+/* low-rank input t[m, r] = sum_k x[m, k] lora_down[k, r] in fp64, rank columns */
+void or_lowrank_input(const uint16_t *x, int64_t M, int64_t K, const uint16_t *lora_down, int rank, double *t)
+{
+#pragma omp parallel for schedule(static)
+    for (int64_t m = 0; m < M; m++) {
+        for (int rr = 0; rr < rank; rr++) {
+            double acc = 0.0;
+            for (int64_t k = 0; k < K; k++)
+                acc += (double)or_bf16_to_f32(x[m * K + k]) * (double)or_bf16_to_f32(lora_down[k * rank + rr]);
+            t[m * rank + rr] = acc;
+        }
+    }
+}
+
+/* ------------------------------------------------------------------------ */
 /* O9: bf16 reconstruct of W from the payload                                */
 /* ------------------------------------------------------------------------ */
 
@@ -750,19 +927,26 @@ void or_linear_fwd_int4(const float *xrot, const uint8_t *codes, const uint16_t 
  *   L = fmaf chain over r = 0..31 of U[n,r] * D[k,r], starting from 0.
  * residual_only drops L: W = bf16(h).
  * fmt: 1 = int4 g32 (scales fp16 [N, K/32]), 2 = NVFP4 (sf tiled, g_w),
- * 3 = int4 g64 (scales fp16 [N, K/64]).
+ * 3 = int4 g64 (scales fp16 [N, K/64]), 4 = int8 per row (codes int8 [N, K],
+ * scales fp32 [N], d = RN(q * s), low-rank rank 16: U [N, 16], D [K, 16], the
+ * fmaf chain over r = 0..15).
  */
 void or_reconstruct_bf16(int fmt, const uint8_t *codes, const void *scales, float g_w,
                          const uint16_t *U, const uint16_t *D,
                          int64_t N, int64_t K, int residual_only, uint16_t *W)
 {
     int64_t C = K / 16;
+    const int rank = fmt == 4 ? 16 : 32;
 #pragma omp parallel for schedule(static)
     for (int64_t n = 0; n < N; n++) {
         for (int64_t b = 0; b < K; b += 256) {
             float v[256];
             for (int i = 0; i < 256; i++) {
                 int64_t k = b + i;
+                if (fmt == 4) {
+                    v[i] = (float)((const int8_t *)codes)[n * K + k] * ((const float *)scales)[n];
+                    continue;
+                }
                 uint8_t byte = codes[n * (K / 2) + k / 2];
                 uint8_t nib = (k & 1) ? (byte >> 4) : (byte & 0xF);
                 if (fmt == 1 || fmt == 3) {
@@ -783,8 +967,8 @@ void or_reconstruct_bf16(int fmt, const uint8_t *codes, const void *scales, floa
                 float out = v[i];
                 if (!residual_only) {
                     float L = 0.0f;
-                    for (int r = 0; r < 32; r++)
-                        L = fmaf(or_bf16_to_f32(U[n * 32 + r]), or_bf16_to_f32(D[k * 32 + r]), L);
+                    for (int r = 0; r < rank; r++)
+                        L = fmaf(or_bf16_to_f32(U[n * rank + r]), or_bf16_to_f32(D[k * rank + r]), L);
                     out = L + v[i];
                 }
                 W[n * K + k] = or_f32_to_bf16(out);
