@@ -5,7 +5,8 @@ One step = one pass of the whole hot path over one synthetic layer of the
 chosen shape (default the headline 4480 x 16384 x 6144, M x N x K):
   sq_build_int4, sq_build_nvfp4, sq_linear_fwd (NVFP4, incl. the activation
   prologue), sq_linear_fwd (int4), sq_reconstruct_bf16 (both payloads), and the
-  int4 group-64 variant's build, forward and reconstruct.
+  build, forward and reconstruct of the int4 group-64 variant and of the int8
+  per-row mode (rank-16 low-rank branch).
 Every op is timed with CUDA events on the launching stream after an L2 flush
 (a 256 MB write outside the op's events); the NVFP4 forward is the headline
 metric (TFLOP/s = 2 M N K / time of the whole sq_linear_fwd call).  The GEMM
@@ -88,6 +89,9 @@ def op_work(M, N, K):
         "build_int4_g64": ("GB/s", NK * (4 + 0.5 + 2 / 64 + 1 / 64)),
         "fwd_int4_g64": ("TFLOP/s", 2.0 * M * N * K),
         "reconstruct_int4_g64": ("GB/s", NK * (0.5 + 2 / 64 + 2)),
+        "build_int8": ("GB/s", NK * (4 + 1) + N * 5),
+        "fwd_int8": ("TFLOP/s", 2.0 * M * N * K),
+        "reconstruct_int8": ("GB/s", NK * (1 + 2) + N * 4),
         "gemm_nvfp4": ("TFLOP/s", 2.0 * M * N * K),
         "gemm_int4": ("TFLOP/s", 2.0 * M * N * K),
     }
@@ -97,6 +101,7 @@ LAUNCHES_PER_STEP = {   # our kernels per op (memsets excluded)
     "build_int4": 1, "build_nvfp4": 2, "fwd_nvfp4": 5, "fwd_int4": 5,
     "reconstruct_nvfp4": 1, "reconstruct_int4": 1,
     "build_int4_g64": 1, "fwd_int4_g64": 5, "reconstruct_int4_g64": 1,
+    "build_int8": 1, "fwd_int8": 7, "reconstruct_int8": 1,
 }
 
 
@@ -241,6 +246,18 @@ def cpu_sample(d, M_s: int, N_s: int):
     t0 = time.perf_counter()
     oracle.reconstruct_bf16(oracle.FMT_INT4_G64, c6, s6, 0.0, U, D, N_s, K)
     t["reconstruct_int4_g64"] = time.perf_counter() - t0
+    U16, D16 = np.ascontiguousarray(U[:, :16]), np.ascontiguousarray(D[:, :16])
+    t0 = time.perf_counter()
+    c8, s8, _ = oracle.build_int8(R)
+    t["build_int8"] = time.perf_counter() - t0
+    t0 = time.perf_counter()
+    xr = oracle.rotate_rows_bf16(x)
+    tt4 = oracle.lowrank_input(x, D16)
+    oracle.linear_fwd_int8(xr, c8, s8, tt4, U16, M_s, N_s, K)
+    t["fwd_int8"] = time.perf_counter() - t0
+    t0 = time.perf_counter()
+    oracle.reconstruct_bf16(oracle.FMT_INT8_ROW, c8, s8, 0.0, U16, D16, N_s, K)
+    t["reconstruct_int8"] = time.perf_counter() - t0
     return t, oracle.num_threads()
 
 
@@ -299,7 +316,7 @@ def workload_config(cfg, args):
                                                               if cfg.hot_channels else ""),
         "name": cfg.name, "M": cfg.M, "N": cfg.N, "K": cfg.K, "rank": 32,
         "codecs": ["nvfp4 (e2m1, ue4m3 block-16, fp32 global)", "int4 group-32 MSE-swept",
-                   "int4 group-64 MSE-swept"],
+                   "int4 group-64 MSE-swept", "int8 per-row MSE-swept, rank-16 low-rank branch"],
         "l2": "flushed (256 MB write) before every op, outside its events",
         "parallelism": f"replicas x{args.gpus}",
     }
@@ -332,6 +349,11 @@ def run_sq(args, cfg, d, rank, world, local_rank):
     i6 = sq.Weight(sq.SQ_FMT_INT4_G64, N, K, torch.empty((N, K // 2), dtype=torch.uint8, device=dev),
                    torch.empty((N, K // 64), dtype=torch.float16, device=dev), None, U, D,
                    torch.empty((N, K // 64), dtype=torch.uint8, device=dev))
+    U16, D16 = U[:, :16].contiguous(), D[:, :16].contiguous()
+    i8 = sq.Weight(sq.SQ_FMT_INT8_ROW, N, K, torch.empty((N, K), dtype=torch.int8, device=dev),
+                   torch.empty(N, dtype=torch.float32, device=dev), None, U16, D16,
+                   torch.empty(N, dtype=torch.uint8, device=dev))
+    ws_i8 = sq.workspace(sq.SQ_OP_LINEAR_FWD_INT8, M, N, K, dev)
     ws_b = sq.workspace(sq.SQ_OP_BUILD_NVFP4, 0, N, K, dev)
     ws_nv = sq.workspace(sq.SQ_OP_LINEAR_FWD_NVFP4, M, N, K, dev)
     ws_i4 = sq.workspace(sq.SQ_OP_LINEAR_FWD_INT4, M, N, K, dev)
@@ -351,6 +373,9 @@ def run_sq(args, cfg, d, rank, world, local_rank):
         ("build_int4_g64", lambda: sq.sq_build_int4(R, i6.codes, i6.scales, i6.frac_idx, group=64)),
         ("fwd_int4_g64", lambda: sq.sq_linear_fwd(i6, x, y_i4, ws=ws_i4)),
         ("reconstruct_int4_g64", lambda: sq.sq_reconstruct_bf16(i6, W)),
+        ("build_int8", lambda: sq.sq_build_int8(R, i8.codes, i8.scales, i8.frac_idx)),
+        ("fwd_int8", lambda: sq.sq_linear_fwd(i8, x, y_i4, ws=ws_i8)),
+        ("reconstruct_int8", lambda: sq.sq_reconstruct_bf16(i8, W)),
     ]
     names = [n for n, _ in ops]
     gemm_of = {"fwd_nvfp4": "gemm_nvfp4", "fwd_int4": "gemm_int4"}
@@ -380,6 +405,7 @@ def run_sq(args, cfg, d, rank, world, local_rank):
     torch.cuda.synchronize()
     sq.sq_check_device_status(ws_nv)
     sq.sq_check_device_status(ws_i4)
+    sq.sq_check_device_status(ws_i8)
 
     keys = names + list(gemm_of.values())
     evs = [{k: (torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for k in keys}

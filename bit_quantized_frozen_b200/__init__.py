@@ -25,19 +25,24 @@ SQ_OK = 0
 SQ_FMT_INT4_G32 = 1
 SQ_FMT_NVFP4 = 2
 SQ_FMT_INT4_G64 = 3
+SQ_FMT_INT8_ROW = 4
 SQ_OP_BUILD_INT4 = 1
 SQ_OP_BUILD_NVFP4 = 2
 SQ_OP_ACT_QUANT_NVFP4 = 3
 SQ_OP_LINEAR_FWD_NVFP4 = 4
 SQ_OP_LINEAR_FWD_INT4 = 5
 SQ_OP_RECONSTRUCT = 6
+SQ_OP_LINEAR_FWD_INT8 = 7
+SQ_OP_BUILD_INT8 = 8
+RANK_INT8 = 16
 SQ_ACT_STATIC_SCALE = 0x1
 SQ_RECON_RESIDUAL_ONLY = 0x2
 RANK = 32
 
 EXPORTED = [
     "sq_status_str", "sq_abi_version", "sq_last_error_detail", "sq_sf_bytes", "sq_workspace_bytes",
-    "sq_build_int4", "sq_build_nvfp4", "sq_act_quant_nvfp4", "sq_linear_fwd", "sq_reconstruct_bf16",
+    "sq_build_int4", "sq_build_int8", "sq_build_nvfp4", "sq_act_quant_nvfp4", "sq_linear_fwd",
+    "sq_reconstruct_bf16",
     "sq_check_device_status", "sq_set_gemm_events", "sq_linear_fwd_noalloc",
 ]
 
@@ -73,6 +78,7 @@ _SIGS = {
     "sq_sf_bytes": ([_I64, _I64], ctypes.c_size_t),
     "sq_workspace_bytes": ([ctypes.c_int, _I64, _I64, _I64], ctypes.c_size_t),
     "sq_build_int4": ([_P, _I64, _I64, ctypes.c_int32, _P, _P, _P, _P], ctypes.c_int),
+    "sq_build_int8": ([_P, _I64, _I64, _P, _P, _P, _P], ctypes.c_int),
     "sq_build_nvfp4": ([_P, _I64, _I64, _P, _P, _P, _P, ctypes.c_size_t, _P], ctypes.c_int),
     "sq_act_quant_nvfp4": ([_P, _I64, _I64, _P, _P, _P, _P, _P, ctypes.c_uint32, _P, ctypes.c_size_t, _P],
                            ctypes.c_int),
@@ -156,6 +162,12 @@ def sq_build_int4(R, codes, scales, frac_idx=None, group: int = 32, stream=None)
                                                 _stream(stream)))
 
 
+def sq_build_int8(R, codes, scales, frac_idx=None, stream=None):
+    N, K = R.shape
+    _check("sq_build_int8", lib().sq_build_int8(_ptr(R), N, K, _ptr(codes), _ptr(scales), _ptr(frac_idx),
+                                                _stream(stream)))
+
+
 def sq_build_nvfp4(R, codes, sf_tiled, g_w, ws, stream=None):
     N, K = R.shape
     _check("sq_build_nvfp4", lib().sq_build_nvfp4(_ptr(R), N, K, _ptr(codes), _ptr(sf_tiled), _ptr(g_w), _ptr(ws),
@@ -215,12 +227,12 @@ class Weight:
     fmt: int
     N: int
     K: int
-    codes: torch.Tensor                  # uint8 [N, K/2]
-    scales: torch.Tensor                 # int4: float16 [N, K/group]; NVFP4: uint8 tiled
+    codes: torch.Tensor                  # uint8 [N, K/2] (int8 format: int8 [N, K])
+    scales: torch.Tensor                 # int4: float16 [N, K/group]; NVFP4: uint8 tiled; int8: float32 [N]
     g_w: torch.Tensor | None = None      # float32 [1] (NVFP4)
-    lora_up: torch.Tensor | None = None  # bf16 [N, 32]
-    lora_down: torch.Tensor | None = None  # bf16 [K, 32]
-    frac_idx: torch.Tensor | None = None  # uint8 [N, K/group] (int4)
+    lora_up: torch.Tensor | None = None  # bf16 [N, 32] (int8 format: [N, 16])
+    lora_down: torch.Tensor | None = None  # bf16 [K, 32] (int8 format: [K, 16])
+    frac_idx: torch.Tensor | None = None  # uint8 [N, K/group] (int4), [N] (int8)
 
     def as_c(self) -> sq_weight:
         return sq_weight(self.fmt, self.N, self.K, _ptr(self.codes), _ptr(self.scales), _ptr(self.g_w),
@@ -243,6 +255,17 @@ def build_int4(R: torch.Tensor, lora_up=None, lora_down=None, group: int = 32, s
     return Weight(fmt, N, K, codes, scales, None, lora_up, lora_down, frac)
 
 
+def build_int8(R: torch.Tensor, lora_up=None, lora_down=None, stream=None) -> Weight:
+    """int8 per-row weight; lora_up [N, 16] / lora_down [K, 16] (rank 16) or None."""
+    N, K = R.shape
+    dev = R.device
+    codes = torch.empty((N, K), dtype=torch.int8, device=dev)
+    scales = torch.empty(N, dtype=torch.float32, device=dev)
+    frac = torch.empty(N, dtype=torch.uint8, device=dev)
+    sq_build_int8(R, codes, scales, frac, stream=stream)
+    return Weight(SQ_FMT_INT8_ROW, N, K, codes, scales, None, lora_up, lora_down, frac)
+
+
 def build_nvfp4(R: torch.Tensor, lora_up=None, lora_down=None, ws=None, stream=None) -> Weight:
     N, K = R.shape
     dev = R.device
@@ -257,7 +280,7 @@ def build_nvfp4(R: torch.Tensor, lora_up=None, lora_down=None, ws=None, stream=N
 def linear_fwd(w: Weight, x: torch.Tensor, ws=None, g_x=None, flags: int = 0, stream=None) -> torch.Tensor:
     M = x.shape[0]
     y = torch.empty((M, w.N), dtype=torch.float32, device=x.device)
-    op = SQ_OP_LINEAR_FWD_NVFP4 if w.fmt == SQ_FMT_NVFP4 else SQ_OP_LINEAR_FWD_INT4
+    op = {SQ_FMT_NVFP4: SQ_OP_LINEAR_FWD_NVFP4, SQ_FMT_INT8_ROW: SQ_OP_LINEAR_FWD_INT8}.get(w.fmt, SQ_OP_LINEAR_FWD_INT4)
     ws = ws if ws is not None else workspace(op, M, w.N, w.K, x.device)
     sq_linear_fwd(w, x, y, g_x=g_x, flags=flags, ws=ws, stream=stream)
     return y

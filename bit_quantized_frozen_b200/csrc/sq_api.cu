@@ -69,6 +69,7 @@ size_t round_up(size_t v, size_t a)
 constexpr int64_t kMaxM = int64_t(1) << 24;
 constexpr int64_t kMaxN = int64_t(1) << 20;
 constexpr int64_t kMaxK = int64_t(1) << 17;
+constexpr int64_t kMaxKInt8 = 16384;          // the int8 builder keeps one rotated row in shared memory
 
 bool shape_ok_nk(int64_t N, int64_t K)
 {
@@ -86,7 +87,7 @@ constexpr size_t kHeader = 256;
 constexpr size_t kAlign = 1024;
 
 struct FwdLayout {
-    size_t a = 0, a_sf = 0, b = 0, t32 = 0, tsplit = 0, udup = 0, total = 0;
+    size_t a = 0, a_sf = 0, b = 0, t32 = 0, tsplit = 0, udup = 0, d32 = 0, u32 = 0, total = 0;
 };
 
 FwdLayout fwd_layout(int fmt, int64_t M, int64_t N, int64_t K)
@@ -109,6 +110,10 @@ FwdLayout fwd_layout(int fmt, int64_t M, int64_t N, int64_t K)
     L.t32 = take((size_t)M * 32 * 4);
     L.tsplit = take((size_t)M * 64 * 2);
     L.udup = take((size_t)N * 64 * 2);
+    if (fmt == SQ_FMT_INT8_ROW) {                 // rank-16 factors widened to rank 32
+        L.d32 = take((size_t)K * 32 * 2);
+        L.u32 = take((size_t)N * 32 * 2);
+    }
     L.total = round_up(off, kAlign);
     return L;
 }
@@ -139,11 +144,12 @@ sq_status check_weight(const sq_weight *w)
 {
     if (!w || !w->codes || !w->scales)
         return SQ_ERR_NULL;
-    if (w->fmt != SQ_FMT_INT4_G32 && w->fmt != SQ_FMT_NVFP4 && w->fmt != SQ_FMT_INT4_G64)
+    if (w->fmt != SQ_FMT_INT4_G32 && w->fmt != SQ_FMT_NVFP4 && w->fmt != SQ_FMT_INT4_G64 &&
+        w->fmt != SQ_FMT_INT8_ROW)
         return SQ_ERR_ARG;
     if (w->fmt == SQ_FMT_NVFP4 && !w->g_w)
         return SQ_ERR_NULL;
-    if (!shape_ok_nk(w->N, w->K))
+    if (!shape_ok_nk(w->N, w->K) || (w->fmt == SQ_FMT_INT8_ROW && w->K > kMaxKInt8))
         return SQ_ERR_SHAPE;
     if (!aligned(w->codes, 16) || !aligned(w->scales, 16) || !aligned(w->g_w, 4) ||
         !aligned(w->lora_up, 16) || !aligned(w->lora_down, 16))
@@ -204,6 +210,10 @@ size_t sq_workspace_bytes(int op, int64_t M, int64_t N, int64_t K)
         return fwd_layout(SQ_FMT_NVFP4, M, N, K).total;
     case SQ_OP_LINEAR_FWD_INT4:
         return fwd_layout(SQ_FMT_INT4_G32, M, N, K).total;
+    case SQ_OP_LINEAR_FWD_INT8:
+        return fwd_layout(SQ_FMT_INT8_ROW, M, N, K).total;
+    case SQ_OP_BUILD_INT8:
+        return kHeader;
     default:
         return 0;
     }
@@ -224,6 +234,24 @@ sq_status sq_build_int4(const float *R, int64_t N, int64_t K, int32_t group, uin
         return st;
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     SQ_CUDA(sq::launch_int4_build(R, N, K, group, codes, scales, frac_idx, sms, s), "int4 build");
+    return SQ_OK;
+}
+
+sq_status sq_build_int8(const float *R, int64_t N, int64_t K, int8_t *codes, float *scales, uint8_t *frac_idx,
+                        void *stream)
+{
+    if (!R || !codes || !scales)
+        return SQ_ERR_NULL;
+    if (!shape_ok_nk(N, K) || K > kMaxKInt8)
+        return SQ_ERR_SHAPE;
+    if (!aligned(R, 16) || !aligned(codes, 16) || !aligned(scales, 4))
+        return SQ_ERR_ALIGN;
+    int sms = 0;
+    sq_status st = check_device(&sms);
+    if (st != SQ_OK)
+        return st;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    SQ_CUDA(sq::launch_int8_build(R, N, K, codes, scales, frac_idx, sms, s), "int8 build");
     return SQ_OK;
 }
 
@@ -358,12 +386,26 @@ sq_status sq_linear_fwd(const sq_weight *w, const uint16_t *x, int64_t M, float 
         uint16_t *xb = reinterpret_cast<uint16_t *>(ws_at(ws, L.a));
         uint16_t *wb = reinterpret_cast<uint16_t *>(ws_at(ws, L.b));
         SQ_CUDA(sq::launch_rotate_bf16(x, M, K, xb, sms, s), "rotate x");
-        SQ_CUDA(sq::launch_dequant_int4(w->codes, reinterpret_cast<const uint16_t *>(w->scales),
-                                        w->fmt == SQ_FMT_INT4_G64 ? 64 : 32, N, K, wb, sms, s),
-                "dequant");
+        if (w->fmt == SQ_FMT_INT8_ROW)
+            SQ_CUDA(sq::launch_dequant_int8(reinterpret_cast<const int8_t *>(w->codes),
+                                            reinterpret_cast<const float *>(w->scales), N, K, wb, sms, s),
+                    "dequant");
+        else
+            SQ_CUDA(sq::launch_dequant_int4(w->codes, reinterpret_cast<const uint16_t *>(w->scales),
+                                            w->fmt == SQ_FMT_INT4_G64 ? 64 : 32, N, K, wb, sms, s),
+                    "dequant");
         if (lora) {
-            SQ_CUDA(sq::launch_act_pass1(x, M, K, w->lora_down, nullptr, t32, status, sms, s), "low-rank input");
-            SQ_CUDA(sq::launch_lowrank_finish(t32, M, nullptr, nullptr, tsplit, w->lora_up, N, udup, sms, s),
+            const uint16_t *Dw = w->lora_down, *Uw = w->lora_up;
+            if (w->fmt == SQ_FMT_INT8_ROW) {          // rank 16: zero columns 16..31
+                uint16_t *d32 = reinterpret_cast<uint16_t *>(ws_at(ws, L.d32));
+                uint16_t *u32 = reinterpret_cast<uint16_t *>(ws_at(ws, L.u32));
+                SQ_CUDA(sq::launch_widen_rank16(w->lora_down, K, d32, sms, s), "widen lora_down");
+                SQ_CUDA(sq::launch_widen_rank16(w->lora_up, N, u32, sms, s), "widen lora_up");
+                Dw = d32;
+                Uw = u32;
+            }
+            SQ_CUDA(sq::launch_act_pass1(x, M, K, Dw, nullptr, t32, status, sms, s), "low-rank input");
+            SQ_CUDA(sq::launch_lowrank_finish(t32, M, nullptr, nullptr, tsplit, Uw, N, udup, sms, s),
                     "low-rank operands");
         }
         g.fp4 = 0;
@@ -389,7 +431,9 @@ sq_status sq_linear_fwd_noalloc(const sq_weight *w, const uint16_t *x, int64_t M
         return st;
     if (!shape_ok_mk(M, w->K))
         return SQ_ERR_SHAPE;
-    const int op = w->fmt == SQ_FMT_NVFP4 ? SQ_OP_LINEAR_FWD_NVFP4 : SQ_OP_LINEAR_FWD_INT4;
+    const int op = w->fmt == SQ_FMT_NVFP4      ? SQ_OP_LINEAR_FWD_NVFP4
+                   : w->fmt == SQ_FMT_INT8_ROW ? SQ_OP_LINEAR_FWD_INT8
+                                               : SQ_OP_LINEAR_FWD_INT4;
     const size_t need = sq_workspace_bytes(op, M, w->N, w->K);
     if (need > kNoAllocScratchBytes) {
         snprintf(g_detail, sizeof(g_detail),

@@ -30,6 +30,12 @@ cudaError_t launch_nvfp4_quant_bf16(const uint16_t *in, int64_t rows, int64_t K,
                                     const LowrankOut &lr, int sms, cudaStream_t s);
 cudaError_t launch_int4_build(const float *R, int64_t N, int64_t K, int group, uint8_t *codes, uint16_t *scales,
                               uint8_t *frac, int sms, cudaStream_t s);
+// int8 per-row builder (K <= 16384), its dequant, and the rank-16 -> rank-32 widening
+cudaError_t launch_int8_build(const float *R, int64_t N, int64_t K, int8_t *codes, float *scales, uint8_t *frac,
+                              int sms, cudaStream_t s);
+cudaError_t launch_dequant_int8(const int8_t *codes, const float *scales, int64_t N, int64_t K, uint16_t *wb, int sms,
+                                cudaStream_t s);
+cudaError_t launch_widen_rank16(const uint16_t *src, int64_t rows, uint16_t *dst, int sms, cudaStream_t s);
 cudaError_t launch_rotate_bf16(const uint16_t *x, int64_t M, int64_t K, uint16_t *xb, int sms, cudaStream_t s);
 cudaError_t launch_dequant_int4(const uint8_t *codes, const uint16_t *scales, int group, int64_t N, int64_t K,
                                 uint16_t *wb, int sms, cudaStream_t s);
@@ -38,7 +44,7 @@ cudaError_t launch_act_pass1(const uint16_t *x, int64_t M, int64_t K, const uint
 cudaError_t launch_lowrank_finish(const float *t32, int64_t M, const float *g_x, const float *g_w,
                                   uint16_t *tsplit, const uint16_t *U, int64_t N, uint16_t *udup, int sms,
                                   cudaStream_t s);
-// fmt: 1 int4 group 32, 2 NVFP4, 3 int4 group 64
+// fmt: 1 int4 group 32, 2 NVFP4, 3 int4 group 64, 4 int8 per row (rank 16)
 cudaError_t launch_reconstruct(int fmt, const uint8_t *codes, const void *scales, const float *g_w,
                                const uint16_t *U, const uint16_t *D, int64_t N, int64_t K, int with_lowrank,
                                uint16_t *W, int sms, cudaStream_t s);

@@ -295,10 +295,11 @@ __global__ void __launch_bounds__(kStreamThreads) nvfp4_quant_kernel(const __gri
 // ---------------------------------------------------------------------------
 // sum of RN((r_i - q_i s)^2) over 32 values, as lane 0 of an xor butterfly over
 // strides 16, 8, 4, 2, 1; rp holds the 32 rotated values as pairs (r_2j, r_2j+1).
-// q = clamp(rint(r inv), -7, 7): |r inv| <= 14, so adding and subtracting
-// 1.5 * 2^23 rounds to the nearest integer, ties to even, exactly like rint (and
-// on the FMA pipe, not the conversion unit).  q s is exact (<= 14 significant
-// bits), so fma(-q, s, r) rounds like r - q s.
+// q = clamp(rint(r inv), -QMAX, QMAX): |r inv| <= 2 QMAX < 2^22, so adding and
+// subtracting 1.5 * 2^23 rounds to the nearest integer, ties to even, exactly
+// like rint (and on the FMA pipe, not the conversion unit).  The error is
+// fma(-q, s, r): r - q s with one rounding (for int4, q s is exact anyway).
+template <int QMAX = 7>
 __device__ __forceinline__ float group_sq_error(const uint64_t (&rp)[16], float s, float inv)
 {
     uint64_t p[16];
@@ -314,8 +315,8 @@ __device__ __forceinline__ float group_sq_error(const uint64_t (&rp)[16], float 
         for (int j = 0; j < 16; ++j) {
             float t0, t1;
             f2_unpack(f2_add(f2_mul(rp[j], inv2), rnd), t0, t1);
-            t0 = fminf(fmaxf(t0, kRound - 7.0f), kRound + 7.0f);
-            t1 = fminf(fmaxf(t1, kRound - 7.0f), kRound + 7.0f);
+            t0 = fminf(fmaxf(t0, kRound - (float)QMAX), kRound + (float)QMAX);
+            t1 = fminf(fmaxf(t1, kRound - (float)QMAX), kRound + (float)QMAX);
             const uint64_t q = f2_sub(f2_pack(t0, t1), rnd);
             const uint64_t e = f2_fma(q, nsn, rp[j]);
             p[j] = f2_mul(e, e);
@@ -372,7 +373,7 @@ __global__ void __launch_bounds__(kStreamThreads, 2) int4_build_kernel(const __g
             const __half hs = __float2half_rn(__fdiv_rn(__fmul_rn(f, a), 7.0f));
             const float s = __half2float(hs);
             const float inv = s == 0.0f ? 0.0f : __frcp_rn(s);
-            float mse = group_sq_error(rp, s, inv);
+            float mse = group_sq_error<7>(rp, s, inv);
             if (G == 64)                               // first half + second half (addition commutes)
                 mse = __fadd_rn(mse, __shfl_xor_sync(0xffffffffu, mse, 1));
             if (j == 0 || mse < best) {
@@ -407,6 +408,199 @@ __global__ void __launch_bounds__(kStreamThreads, 2) int4_build_kernel(const __g
                 frac[gidx] = (uint8_t)best_j;
         }
     });
+}
+
+// ---------------------------------------------------------------------------
+// int8 per-row builder (v3.1 int8-residual mode).  One CTA of 256 threads per
+// row at a time (persistent over rows).  The row is copied into shared memory
+// (16-byte chunk c of each lane's 128-byte piece at slot c ^ lane%8, so the 8
+// lanes of a block read 8 different bank groups), rotated in place by 8-lane
+// groups (group i takes blocks i, i + 32, ...), and its absmax reduced.  Each
+// group then sweeps the 26 scales over its blocks with the values in
+// registers: per block, the 32-value butterfly in each lane and a butterfly
+// over the 8 lanes (strides 4, 2, 1) give the block's error, stored per
+// (fraction, block); 26 threads then add the blocks of their fraction in
+// order, and the smallest sum (first on ties) picks the scale.  Finally each
+// group quantises its blocks and writes 32 int8 codes per lane.
+// ---------------------------------------------------------------------------
+constexpr int kI8Threads = 256;
+constexpr int kI8MaxK = 16384;
+
+__host__ __device__ constexpr int i8_smem_bytes(int K)
+{
+    return K * 4 + kFracCount * (K / kHad) * 4 + 2 * kFracCount * 4 + 64;
+}
+
+__device__ __forceinline__ int i8_slot(int block, int q, int c)   // float4 index in the shared row
+{
+    return block * 64 + q * 8 + (c ^ q);
+}
+
+__global__ void __launch_bounds__(kI8Threads) int8_build_kernel(const float *__restrict__ R, int64_t N, int K,
+                                                                int8_t *__restrict__ codes,
+                                                                float *__restrict__ scales,
+                                                                uint8_t *__restrict__ frac)
+{
+    extern __shared__ __align__(16) uint8_t i8_smem[];
+    float4 *row = reinterpret_cast<float4 *>(i8_smem);                        // K floats, swizzled
+    float *berr = reinterpret_cast<float *>(i8_smem + K * 4);                  // [26][nb] block errors
+    float *stab = berr + kFracCount * (K / kHad);                              // [26] scales, [26] errors
+    float *etab = stab + kFracCount;
+    float *red = etab + kFracCount;                                            // [8] warp maxima, choice
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int q = lane & 7;
+    const int grp = tid >> 3;                                                  // 8-lane group, 0..31
+    const int nb = K / kHad;
+    const int iters = (nb + 31) / 32;                                          // blocks per group (max)
+
+    for (int64_t n = blockIdx.x; n < N; n += gridDim.x) {
+        // copy the row (float4 f of the row -> block f/64, lane (f/8)%8, chunk f%8)
+        const float4 *src = reinterpret_cast<const float4 *>(R + n * K);
+        for (int f = tid; f < K / 4; f += kI8Threads)
+            row[i8_slot(f >> 6, (f >> 3) & 7, f & 7)] = __ldg(src + f);
+        __syncthreads();
+        // rotate in place, absmax
+        float a = 0.0f;
+        for (int it = 0; it < iters; ++it) {
+            const int b = grp + 32 * it;
+            const bool valid = b < nb;                 // the whole warp runs the shuffles
+            float v[32];
+#pragma unroll
+            for (int c = 0; c < 8; ++c) {
+                const float4 x = valid ? row[i8_slot(b, q, c)] : make_float4(0.f, 0.f, 0.f, 0.f);
+                v[4 * c] = x.x; v[4 * c + 1] = x.y; v[4 * c + 2] = x.z; v[4 * c + 3] = x.w;
+            }
+            fwht256_l32(v, lane);
+            if (valid) {
+#pragma unroll
+                for (int c = 0; c < 8; ++c)
+                    row[i8_slot(b, q, c)] = make_float4(v[4 * c], v[4 * c + 1], v[4 * c + 2], v[4 * c + 3]);
+#pragma unroll
+                for (int i = 0; i < 32; i += 2)
+                    a = fmax3(a, fabsf(v[i]), fabsf(v[i + 1]));
+            }
+        }
+#pragma unroll
+        for (int x = 16; x >= 1; x >>= 1)
+            a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, x));
+        if (lane == 0)
+            red[warp] = a;
+        __syncthreads();
+        if (tid < kFracCount) {
+            float m = 0.0f;
+            for (int w = 0; w < kI8Threads / 32; ++w)
+                m = fmaxf(m, red[w]);
+            stab[tid] = __fdiv_rn(__fmul_rn(kFrac[tid], m), 127.0f);
+        }
+        __syncthreads();
+        // sweep: per block and fraction, the block's error
+        for (int it = 0; it < iters; ++it) {
+            const int b = grp + 32 * it;
+            const bool valid = b < nb;
+            uint64_t rp[16];
+#pragma unroll
+            for (int c = 0; c < 8; ++c) {
+                const float4 x = valid ? row[i8_slot(b, q, c)] : make_float4(0.f, 0.f, 0.f, 0.f);
+                rp[2 * c] = f2_pack(x.x, x.y);
+                rp[2 * c + 1] = f2_pack(x.z, x.w);
+            }
+#pragma unroll 1
+            for (int j = 0; j < kFracCount; ++j) {
+                const float sj = stab[j];
+                const float inv = sj == 0.0f ? 0.0f : __frcp_rn(sj);
+                float e = group_sq_error<127>(rp, sj, inv);
+                e = __fadd_rn(e, __shfl_xor_sync(0xffffffffu, e, 4));
+                e = __fadd_rn(e, __shfl_xor_sync(0xffffffffu, e, 2));
+                e = __fadd_rn(e, __shfl_xor_sync(0xffffffffu, e, 1));
+                if (valid && q == 0)
+                    berr[j * nb + b] = e;
+            }
+        }
+        __syncthreads();
+        if (tid < kFracCount) {                        // blocks in order, per fraction
+            float E = berr[tid * nb];
+            for (int b = 1; b < nb; ++b)
+                E = __fadd_rn(E, berr[tid * nb + b]);
+            etab[tid] = E;
+        }
+        __syncthreads();
+        int best_j = 0;
+        {
+            float best = etab[0];
+            for (int j = 1; j < kFracCount; ++j)
+                if (etab[j] < best) {
+                    best = etab[j];
+                    best_j = j;
+                }
+        }
+        const float s = stab[best_j];
+        const float inv = s == 0.0f ? 0.0f : __frcp_rn(s);
+        // codes
+        for (int it = 0; it < iters; ++it) {
+            const int b = grp + 32 * it;
+            if (b >= nb)
+                break;
+            uint32_t w[8];
+#pragma unroll
+            for (int c = 0; c < 8; ++c) {
+                const float4 x = row[i8_slot(b, q, c)];
+                const float xv[4] = {x.x, x.y, x.z, x.w};
+                uint32_t word = 0;
+#pragma unroll
+                for (int k = 0; k < 4; ++k) {
+                    int qi = 0;
+                    if (s != 0.0f)
+                        qi = (int)fminf(fmaxf(rintf(__fmul_rn(xv[k], inv)), -127.0f), 127.0f);
+                    word |= ((uint32_t)qi & 0xFFu) << (8 * k);
+                }
+                w[c] = word;
+            }
+            uint4 *dst = reinterpret_cast<uint4 *>(codes + n * K + (int64_t)b * kHad + 32 * q);
+            dst[0] = make_uint4(w[0], w[1], w[2], w[3]);
+            dst[1] = make_uint4(w[4], w[5], w[6], w[7]);
+        }
+        if (tid == 0) {
+            scales[n] = s;
+            if (frac)
+                frac[n] = (uint8_t)best_j;
+        }
+        __syncthreads();                               // the shared row is free for the next one
+    }
+}
+
+// int8 "dequant-first": wb[n, k] = bf16(RN(q s_n)), 16 values per thread
+__global__ void __launch_bounds__(256) dequant_int8_kernel(const uint4 *__restrict__ codes,
+                                                           const float *__restrict__ scales, int64_t K,
+                                                           int64_t total16, uint4 *__restrict__ wb)
+{
+    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < total16;
+         i += (int64_t)gridDim.x * blockDim.x) {
+        const uint4 c = __ldg(codes + i);
+        const float s = __ldg(scales + (i * 16) / K);
+        const uint32_t w[4] = {c.x, c.y, c.z, c.w};
+        uint32_t o[8];
+#pragma unroll
+        for (int p = 0; p < 8; ++p) {
+            const int q0 = (int)(int8_t)((w[p >> 1] >> (16 * (p & 1))) & 0xFFu);
+            const int q1 = (int)(int8_t)((w[p >> 1] >> (16 * (p & 1) + 8)) & 0xFFu);
+            o[p] = f32_to_bf16_bits(__fmul_rn((float)q0, s)) | (f32_to_bf16_bits(__fmul_rn((float)q1, s)) << 16);
+        }
+        wb[2 * i] = make_uint4(o[0], o[1], o[2], o[3]);
+        wb[2 * i + 1] = make_uint4(o[4], o[5], o[6], o[7]);
+    }
+}
+
+// rank-16 low-rank factors widened to rank 32 with zero columns 16..31, so the
+// rank-32 forward machinery (t = x lora_down, the low-rank MMA step) adds
+// exactly the rank-16 term: src [rows, 16] bf16 -> dst [rows, 32] bf16
+__global__ void __launch_bounds__(256) widen_rank16_kernel(const uint4 *__restrict__ src, int64_t rows,
+                                                           uint4 *__restrict__ dst)
+{
+    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < rows * 4;
+         i += (int64_t)gridDim.x * blockDim.x) {
+        const int64_t r = i >> 2, c = i & 3;       // 16-byte chunk c of dst row r
+        dst[i] = c < 2 ? __ldg(src + 2 * r + c) : make_uint4(0u, 0u, 0u, 0u);
+    }
 }
 
 // ---------------------------------------------------------------------------
@@ -763,25 +957,35 @@ __global__ void __launch_bounds__(256) lowrank_finish_kernel(const float *__rest
 // next tile's codes, scales and lora_up rows in shared memory by cp.async
 // while the current one is computed, and keeping lora_down for the current kb
 // in registers.
-// Phase 1: each lane decodes 32 payload values of a row (one int4 group, or
-//   two NVFP4 blocks), runs the 8-lane Hadamard transform and writes h into a
+// Phase 1: each lane decodes 32 payload values of a row (an int4 group or half
+//   group, two NVFP4 blocks, or 32 int8 codes), runs the 8-lane Hadamard
+//   transform and writes h into a
 //   shared fp32 tile (float4 f of a row stored at f ^ (f >> 3) -- conflict free
 //   for both phases).
 // Phase 2: thread t owns columns 2(t%128), 2(t%128)+1 and rows 32(t/128)..+31.
 //   lora_down for its two columns stays in registers; lora_up rows are
-//   broadcast from shared memory; each output's rank-32 fmaf chain runs in
-//   order r = 0..31 from 0, two columns at a time with fma.rn.f32x2 (two
+//   broadcast from shared memory; each output's fmaf chain runs in order
+//   r = 0..rank-1 from 0 (rank 32, or 16 for int8), two columns at a time with
+//   fma.rn.f32x2 (two
 //   independent fmaf, bit-identical to the scalar chain); W = bf16(RN(L + h)).
 // ---------------------------------------------------------------------------
 constexpr int kRecRows = 64;
-constexpr int kRecCodeBytes = kRecRows * kHad / 2;        // 8 KB
-constexpr int kRecScaleBytes = kRecRows * 16;             // 1 KB (8 fp16 or 16 ue4m3 per row)
-constexpr int kRecUBytes = kRecRows * kRank * 2;          // 4 KB
-constexpr int kRecStageBytes = kRecCodeBytes + kRecScaleBytes + kRecUBytes;
+constexpr int kRecScaleBytes = kRecRows * 16;             // 1 KB (8 fp16, 4 fp16, 16 ue4m3 or 1 fp32 per row)
 constexpr int kRecHBytes = kRecRows * kHad * 4;           // 64 KB
-constexpr int kRecUsBytes = kRecRows * kRank * 4;         // 8 KB
-constexpr int kRecSmemLowrank = kRecHBytes + kRecUsBytes + 2 * kRecStageBytes;   // 98 KB
-constexpr int kRecSmemResidual = 2 * kRecStageBytes;
+
+// per payload format (1 int4 g32, 2 NVFP4, 3 int4 g64: 4-bit codes, rank 32;
+// 4 int8 per row: 8-bit codes, rank 16)
+template <int FMT>
+struct RecCfg {
+    static constexpr int kRank = FMT == 4 ? 16 : 32;
+    static constexpr int kCodeRow = FMT == 4 ? kHad : kHad / 2;             // code bytes per row and block
+    static constexpr int kCodeBytes = kRecRows * kCodeRow;                    // 8 or 16 KB
+    static constexpr int kUBytes = kRecRows * kRank * 2;                      // 4 or 2 KB
+    static constexpr int kStageBytes = kCodeBytes + kRecScaleBytes + kUBytes;
+    static constexpr int kUsBytes = kRecRows * kRank * 4;
+    static constexpr int kSmemLowrank = kRecHBytes + kUsBytes + 2 * kStageBytes;   // 98 or 106 KB
+    static constexpr int kSmemResidual = 2 * kStageBytes;
+};
 
 __device__ __forceinline__ uint64_t pack2(float lo, float hi)
 {
@@ -811,24 +1015,28 @@ __device__ __forceinline__ void cp_async8(uint32_t dst, const void *src, uint32_
     asm volatile("cp.async.ca.shared.global [%0], [%1], 8, %2;" ::"r"(dst), "l"(src), "r"(src_bytes) : "memory");
 }
 
-// Stage tile (kb, rows n0..n0+63) into one buffer: codes [64][128 B], scales
-// [64][16 B] (int4 group 32: the 8 fp16 group scales; int4 group 64: the 4 fp16
-// group scales in the first 8 bytes; NVFP4: the 16 ue4m3 block scales,
-// gathered from the tiled layout 4 bytes at a time), lora_up [64][64 B].
-// Rows past N are zero filled.
+// Stage tile (kb, rows n0..n0+63) into one buffer: codes [64][128 B] (4-bit
+// formats) or [64][256 B] (int8), scales [64][16 B] (int4 group 32: the 8 fp16
+// group scales; int4 group 64: the 4 fp16 group scales in the first 8 bytes;
+// NVFP4: the 16 ue4m3 block scales, gathered from the tiled layout 4 bytes at
+// a time; int8: the row's fp32 scale in the first 4 bytes), lora_up
+// [64][2 * rank B].  Rows past N are zero filled.
 template <int FMT, bool LOWRANK>
 __device__ __forceinline__ void rec_stage(uint32_t buf, const uint8_t *codes, const void *scales, const uint16_t *U,
                                           int64_t N, int64_t K, int64_t kb, int64_t n0, int tid)
 {
+    using Cfg = RecCfg<FMT>;
+    constexpr int kChunksPerRow = Cfg::kCodeRow / 16;
 #pragma unroll
-    for (int i = 0; i < 2; ++i) {
+    for (int i = 0; i < kRecRows * kChunksPerRow / 256; ++i) {
         const int e = tid + 256 * i;
-        const int r = e >> 3, c = e & 7;
+        const int r = e / kChunksPerRow, c = e % kChunksPerRow;
         const int64_t n = n0 + r;
-        const uint8_t *src = n < N ? codes + n * (K / 2) + kb * (kHad / 2) + 16 * c : codes;
-        cp_async16(buf + r * 128 + 16 * c, src, n < N ? 16u : 0u);
+        const uint8_t *src =
+            n < N ? codes + n * (K * Cfg::kCodeRow / kHad) + kb * Cfg::kCodeRow + 16 * c : codes;
+        cp_async16(buf + r * Cfg::kCodeRow + 16 * c, src, n < N ? 16u : 0u);
     }
-    const uint32_t sbuf = buf + kRecCodeBytes;
+    const uint32_t sbuf = buf + Cfg::kCodeBytes;
     if (FMT == 1) {
         if (tid < kRecRows) {
             const int64_t n = n0 + tid;
@@ -843,6 +1051,13 @@ __device__ __forceinline__ void rec_stage(uint32_t buf, const uint8_t *codes, co
                                        : reinterpret_cast<const uint8_t *>(scales);
             cp_async8(sbuf + 16 * tid, src, n < N ? 8u : 0u);
         }
+    } else if (FMT == 4) {
+        if (tid < kRecRows) {
+            const int64_t n = n0 + tid;
+            const uint8_t *src = n < N ? reinterpret_cast<const uint8_t *>(scales) + n * 4
+                                       : reinterpret_cast<const uint8_t *>(scales);
+            cp_async4(sbuf + 16 * tid, src, n < N ? 4u : 0u);
+        }
     } else {
         const int r = tid >> 2, j = tid & 3;
         const int64_t n = n0 + r;
@@ -852,21 +1067,38 @@ __device__ __forceinline__ void rec_stage(uint32_t buf, const uint8_t *codes, co
         cp_async4(sbuf + 16 * r + 4 * j, src, n < N ? 4u : 0u);
     }
     if (LOWRANK) {
-        const int r = tid >> 2, c = tid & 3;
-        const int64_t n = n0 + r;
-        const uint16_t *src = n < N ? U + n * kRank + 8 * c : U;
-        cp_async16(buf + kRecCodeBytes + kRecScaleBytes + r * 64 + 16 * c, src, n < N ? 16u : 0u);
+        constexpr int kUChunks = Cfg::kRank / 8;     // 16-byte chunks of a lora_up row
+        if (tid < kRecRows * kUChunks) {
+            const int r = tid / kUChunks, c = tid % kUChunks;
+            const int64_t n = n0 + r;
+            const uint16_t *src = n < N ? U + n * Cfg::kRank + 8 * c : U;
+            cp_async16(buf + Cfg::kCodeBytes + kRecScaleBytes + r * (2 * Cfg::kRank) + 16 * c, src,
+                       n < N ? 16u : 0u);
+        }
     }
 }
 
 // 32 payload values of staged row r, values 32q..32q+31 of the block (one int4
-// group of 32, half of a group of 64, or two NVFP4 blocks)
+// group of 32, half of a group of 64, two NVFP4 blocks, or 32 int8 codes)
 template <int FMT>
 __device__ __forceinline__ void rec_decode(const uint8_t *stage, int r, int q, float g, float (&v)[32])
 {
-    const uint4 c = *reinterpret_cast<const uint4 *>(stage + r * 128 + 16 * q);
+    using Cfg = RecCfg<FMT>;
+    const uint8_t *sc = stage + Cfg::kCodeBytes + 16 * r;
+    if (FMT == 4) {
+        const float s = *reinterpret_cast<const float *>(sc);
+        const uint4 c0 = *reinterpret_cast<const uint4 *>(stage + r * Cfg::kCodeRow + 32 * q);
+        const uint4 c1 = *reinterpret_cast<const uint4 *>(stage + r * Cfg::kCodeRow + 32 * q + 16);
+        const uint32_t w[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
+#pragma unroll
+        for (int i = 0; i < 32; ++i) {
+            const int qi = (int)(int8_t)((w[i >> 2] >> (8 * (i & 3))) & 0xFFu);
+            v[i] = __fmul_rn((float)qi, s);
+        }
+        return;
+    }
+    const uint4 c = *reinterpret_cast<const uint4 *>(stage + r * Cfg::kCodeRow + 16 * q);
     const uint32_t w[4] = {c.x, c.y, c.z, c.w};
-    const uint8_t *sc = stage + kRecCodeBytes + 16 * r;
     if (FMT == 1 || FMT == 3) {
         const float s = __half2float(*reinterpret_cast<const __half *>(sc + 2 * (FMT == 3 ? q >> 1 : q)));
 #pragma unroll
@@ -896,10 +1128,12 @@ __global__ void __launch_bounds__(256, LOWRANK ? 2 : 3) reconstruct_kernel(const
                                                              const uint16_t *__restrict__ D, int64_t N, int64_t K,
                                                              uint16_t *__restrict__ W)
 {
+    using Cfg = RecCfg<FMT>;
+    constexpr int kR = Cfg::kRank;
     extern __shared__ __align__(128) uint8_t rec_smem[];
     float *h = reinterpret_cast<float *>(rec_smem);                                // [64][256] swizzled
-    float *us = reinterpret_cast<float *>(rec_smem + kRecHBytes);                  // [64][32] lora_up, fp32
-    uint8_t *stage0 = rec_smem + (LOWRANK ? kRecHBytes + kRecUsBytes : 0);
+    float *us = reinterpret_cast<float *>(rec_smem + kRecHBytes);                  // [64][rank] lora_up, fp32
+    uint8_t *stage0 = rec_smem + (LOWRANK ? kRecHBytes + Cfg::kUsBytes : 0);
     const int tid = threadIdx.x;
     const int lane = tid & 31, warp = tid >> 5;
     const float g = FMT == 2 ? *g_w : 0.0f;
@@ -917,21 +1151,21 @@ __global__ void __launch_bounds__(256, LOWRANK ? 2 : 3) reconstruct_kernel(const
     const int rbase = 32 * (tid >> 7);
     const int f = cp >> 1;                           // float4 of h holding columns 2cp, 2cp+1
     const int fo = 2 * (cp & 1);
-    uint64_t d2[kRank];
+    uint64_t d2[kR];
     int64_t cur_kb = -1;
 
 #pragma unroll 1
     for (int64_t t = t_begin, i = 0; t < t_end; ++t, ++i) {
         const int buf = (int)(i & 1);
         if (t + 1 < t_end)
-            rec_stage<FMT, LOWRANK>(sbase + (buf ^ 1) * kRecStageBytes, codes, scales, U, N, K, (t + 1) / NT,
+            rec_stage<FMT, LOWRANK>(sbase + (buf ^ 1) * Cfg::kStageBytes, codes, scales, U, N, K, (t + 1) / NT,
                                     ((t + 1) % NT) * kRecRows, tid);
         cp_async_commit();
         cp_async_wait<1>();
         __syncthreads();                             // tile t staged; previous tile's phase 2 done
         const int64_t kb = t / NT;
         const int64_t n0 = (t % NT) * kRecRows;
-        const uint8_t *st = stage0 + buf * kRecStageBytes;
+        const uint8_t *st = stage0 + buf * Cfg::kStageBytes;
 
         // phase 1: h = H(d)
 #pragma unroll 1
@@ -969,19 +1203,19 @@ __global__ void __launch_bounds__(256, LOWRANK ? 2 : 3) reconstruct_kernel(const
             continue;
         }
         {
-            const uint16_t *ust = reinterpret_cast<const uint16_t *>(st + kRecCodeBytes + kRecScaleBytes);
+            const uint16_t *ust = reinterpret_cast<const uint16_t *>(st + Cfg::kCodeBytes + kRecScaleBytes);
 #pragma unroll
-            for (int j = 0; j < kRecRows * kRank / 256; ++j) {
+            for (int j = 0; j < kRecRows * kR / 256; ++j) {
                 us[tid + 256 * j] = bf16_bits_to_f32(ust[tid + 256 * j]);
             }
         }
         if (kb != cur_kb) {                          // lora_down of this thread's two columns
             cur_kb = kb;
             const int64_t k0 = kb * kHad + 2 * cp;
-            const uint4 *dr0 = reinterpret_cast<const uint4 *>(D + k0 * kRank);
-            const uint4 *dr1 = reinterpret_cast<const uint4 *>(D + (k0 + 1) * kRank);
+            const uint4 *dr0 = reinterpret_cast<const uint4 *>(D + k0 * kR);
+            const uint4 *dr1 = reinterpret_cast<const uint4 *>(D + (k0 + 1) * kR);
 #pragma unroll
-            for (int k = 0; k < 4; ++k) {
+            for (int k = 0; k < kR / 8; ++k) {
                 const uint4 a = __ldg(dr0 + k), b = __ldg(dr1 + k);
                 const uint32_t wa[4] = {a.x, a.y, a.z, a.w}, wb[4] = {b.x, b.y, b.z, b.w};
 #pragma unroll
@@ -999,11 +1233,11 @@ __global__ void __launch_bounds__(256, LOWRANK ? 2 : 3) reconstruct_kernel(const
         for (int r0 = rbase; r0 < rbase + 32; r0 += 4) {
             uint64_t acc[4] = {0ull, 0ull, 0ull, 0ull};
 #pragma unroll
-            for (int rr = 0; rr < kRank; rr += 4) {
+            for (int rr = 0; rr < kR; rr += 4) {
                 float4 u4[4];
 #pragma unroll
                 for (int j = 0; j < 4; ++j)
-                    u4[j] = *reinterpret_cast<const float4 *>(us + (r0 + j) * kRank + rr);
+                    u4[j] = *reinterpret_cast<const float4 *>(us + (r0 + j) * kR + rr);
 #pragma unroll
                 for (int j = 0; j < 4; ++j) {
                     fma2(acc[j], pack2(u4[j].x, u4[j].x), d2[rr]);
@@ -1166,6 +1400,52 @@ cudaError_t launch_int4_build(const float *R, int64_t N, int64_t K, int group, u
     return cudaGetLastError();
 }
 
+cudaError_t launch_int8_build(const float *R, int64_t N, int64_t K, int8_t *codes, float *scales, uint8_t *frac,
+                              int sms, cudaStream_t s)
+{
+    if (K > kI8MaxK)
+        return cudaErrorInvalidValue;
+    constexpr int kMaxDev = 64;
+    static bool attr_done[kMaxDev];
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDev)
+        return cudaErrorInvalidDevice;
+    if (!attr_done[dev]) {
+        cudaError_t e = cudaFuncSetAttribute(int8_build_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             i8_smem_bytes(kI8MaxK));
+        if (e != cudaSuccess)
+            return e;
+        attr_done[dev] = true;
+    }
+    // persistent CTAs over rows: only as many as are resident at once (registers and
+    // shared memory), so that no CTA waits for a whole earlier CTA's share of rows
+    const int smem = i8_smem_bytes((int)K);
+    int per_sm = 0;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, int8_build_kernel, kI8Threads, smem) != cudaSuccess ||
+        per_sm < 1)
+        per_sm = 1;
+    const int64_t want = (int64_t)sms * per_sm;
+    const unsigned grid = (unsigned)(N < want ? N : want);
+    int8_build_kernel<<<grid, kI8Threads, smem, s>>>(R, N, (int)K, codes, scales, frac);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_dequant_int8(const int8_t *codes, const float *scales, int64_t N, int64_t K, uint16_t *wb, int sms,
+                                cudaStream_t s)
+{
+    const int64_t total16 = N * K / 16;
+    dequant_int8_kernel<<<grid_for(total16, 256, sms, 8), 256, 0, s>>>(reinterpret_cast<const uint4 *>(codes), scales,
+                                                                      K, total16, reinterpret_cast<uint4 *>(wb));
+    return cudaGetLastError();
+}
+
+cudaError_t launch_widen_rank16(const uint16_t *src, int64_t rows, uint16_t *dst, int sms, cudaStream_t s)
+{
+    widen_rank16_kernel<<<grid_for(rows * 4, 256, sms, 4), 256, 0, s>>>(reinterpret_cast<const uint4 *>(src), rows,
+                                                                       reinterpret_cast<uint4 *>(dst));
+    return cudaGetLastError();
+}
+
 cudaError_t launch_rotate_bf16(const uint16_t *x, int64_t M, int64_t K, uint16_t *xb, int sms, cudaStream_t s)
 {
     CUtensorMap tm;
@@ -1249,24 +1529,20 @@ cudaError_t launch_lowrank_finish(const float *t32, int64_t M, const float *g_x,
     return cudaGetLastError();
 }
 
-cudaError_t launch_reconstruct(int fmt, const uint8_t *codes, const void *scales, const float *g_w,
-                               const uint16_t *U, const uint16_t *D, int64_t N, int64_t K, int with_lowrank,
-                               uint16_t *W, int sms, cudaStream_t s)
+template <int FMT>
+static cudaError_t launch_reconstruct_fmt(const uint8_t *codes, const void *scales, const float *g_w,
+                                          const uint16_t *U, const uint16_t *D, int64_t N, int64_t K,
+                                          int with_lowrank, uint16_t *W, int sms, cudaStream_t s)
 {
+    using Cfg = RecCfg<FMT>;
     constexpr int kMaxDev = 64;
     static bool attr_done[kMaxDev];
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDev)
         return cudaErrorInvalidDevice;
     if (!attr_done[dev]) {
-        cudaError_t e = cudaFuncSetAttribute(reconstruct_kernel<1, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                             kRecSmemLowrank);
-        if (e == cudaSuccess)
-            e = cudaFuncSetAttribute(reconstruct_kernel<2, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                     kRecSmemLowrank);
-        if (e == cudaSuccess)
-            e = cudaFuncSetAttribute(reconstruct_kernel<3, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                     kRecSmemLowrank);
+        cudaError_t e = cudaFuncSetAttribute(reconstruct_kernel<FMT, true>,
+                                             cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::kSmemLowrank);
         if (e != cudaSuccess)
             return e;
         attr_done[dev] = true;
@@ -1274,24 +1550,23 @@ cudaError_t launch_reconstruct(int fmt, const uint8_t *codes, const void *scales
     const int64_t tiles = (K / kHad) * ((N + kRecRows - 1) / kRecRows);
     const int64_t per_sm = with_lowrank ? 2 : 3;            // resident CTAs per SM (registers, shared memory)
     const unsigned grid = (unsigned)(tiles < per_sm * sms ? tiles : per_sm * sms);
-    const int smem = with_lowrank ? kRecSmemLowrank : kRecSmemResidual;
-    if (fmt == 2) {
-        if (with_lowrank)
-            reconstruct_kernel<2, true><<<grid, 256, smem, s>>>(codes, scales, g_w, U, D, N, K, W);
-        else
-            reconstruct_kernel<2, false><<<grid, 256, smem, s>>>(codes, scales, g_w, U, D, N, K, W);
-    } else if (fmt == 3) {
-        if (with_lowrank)
-            reconstruct_kernel<3, true><<<grid, 256, smem, s>>>(codes, scales, g_w, U, D, N, K, W);
-        else
-            reconstruct_kernel<3, false><<<grid, 256, smem, s>>>(codes, scales, g_w, U, D, N, K, W);
-    } else {
-        if (with_lowrank)
-            reconstruct_kernel<1, true><<<grid, 256, smem, s>>>(codes, scales, g_w, U, D, N, K, W);
-        else
-            reconstruct_kernel<1, false><<<grid, 256, smem, s>>>(codes, scales, g_w, U, D, N, K, W);
-    }
+    if (with_lowrank)
+        reconstruct_kernel<FMT, true><<<grid, 256, Cfg::kSmemLowrank, s>>>(codes, scales, g_w, U, D, N, K, W);
+    else
+        reconstruct_kernel<FMT, false><<<grid, 256, Cfg::kSmemResidual, s>>>(codes, scales, g_w, U, D, N, K, W);
     return cudaGetLastError();
+}
+
+cudaError_t launch_reconstruct(int fmt, const uint8_t *codes, const void *scales, const float *g_w,
+                               const uint16_t *U, const uint16_t *D, int64_t N, int64_t K, int with_lowrank,
+                               uint16_t *W, int sms, cudaStream_t s)
+{
+    switch (fmt) {
+    case 2: return launch_reconstruct_fmt<2>(codes, scales, g_w, U, D, N, K, with_lowrank, W, sms, s);
+    case 3: return launch_reconstruct_fmt<3>(codes, scales, g_w, U, D, N, K, with_lowrank, W, sms, s);
+    case 4: return launch_reconstruct_fmt<4>(codes, scales, g_w, U, D, N, K, with_lowrank, W, sms, s);
+    default: return launch_reconstruct_fmt<1>(codes, scales, g_w, U, D, N, K, with_lowrank, W, sms, s);
+    }
 }
 
 }  // namespace sq

@@ -16,12 +16,14 @@ Operations:
   act_quant_nolowrank  sq_act_quant_nvfp4 without t (absmax pass + quantisation)
   fwd_nvfp4            sq_linear_fwd, NVFP4 weight
   fwd_int4             sq_linear_fwd, int4 group-32 weight
+  fwd_int8             sq_linear_fwd, int8 per-row weight (rank-16 low-rank branch)
   build_nvfp4          sq_build_nvfp4
   build_int4           sq_build_int4, group 32
   build_int4_g64       sq_build_int4, group 64
-  recon_nvfp4 / recon_int4 / recon_int4_g64
+  build_int8           sq_build_int8
+  recon_nvfp4 / recon_int4 / recon_int4_g64 / recon_int8
                        sq_reconstruct_bf16 with the low-rank term
-  recon_nvfp4_resid / recon_int4_resid
+  recon_nvfp4_resid / recon_int4_resid / recon_int8_resid
                        sq_reconstruct_bf16 with SQ_RECON_RESIDUAL_ONLY
   gemm_nvfp4 / gemm_int4
                        the tensor-core GEMM launch inside sq_linear_fwd, timed by
@@ -50,9 +52,9 @@ import synth_inputs as si  # noqa: E402
 
 FLUSH_BYTES = 256 << 20
 
-OPS = ["act_quant", "act_quant_nolowrank", "fwd_nvfp4", "fwd_int4", "build_nvfp4", "build_int4",
-       "build_int4_g64", "recon_nvfp4", "recon_int4", "recon_int4_g64", "recon_nvfp4_resid", "recon_int4_resid",
-       "gemm_nvfp4", "gemm_int4"]
+OPS = ["act_quant", "act_quant_nolowrank", "fwd_nvfp4", "fwd_int4", "fwd_int8", "build_nvfp4", "build_int4",
+       "build_int4_g64", "build_int8", "recon_nvfp4", "recon_int4", "recon_int4_g64", "recon_int8",
+       "recon_nvfp4_resid", "recon_int4_resid", "recon_int8_resid", "gemm_nvfp4", "gemm_int4"]
 
 
 def work(op, M, N, K):
@@ -68,6 +70,10 @@ def work(op, M, N, K):
         return "GB/s", NK * (4 + 0.5 + 3 / 32)
     if op == "build_int4_g64":
         return "GB/s", NK * (4 + 0.5 + 3 / 64)
+    if op == "build_int8":
+        return "GB/s", NK * (4 + 1) + N * 5
+    if op.startswith("recon_int8"):
+        return "GB/s", NK * (1 + 2) + N * 4
     scale = {"nvfp4": 1 / 16, "int4": 2 / 32, "int4_g64": 2 / 64}[op.split("_", 1)[1].replace("_resid", "")]
     return "GB/s", NK * (0.5 + scale + 2)
 
@@ -131,6 +137,8 @@ def main():
     w4 = sq.build_int4(R, U, D)
     w6 = sq.build_int4(R, U, D, group=64)
     wn = sq.build_nvfp4(R, U, D)
+    w8 = sq.build_int8(R, U[:, :16].contiguous(), D[:, :16].contiguous())
+    ws_8 = sq.workspace(sq.SQ_OP_LINEAR_FWD_INT8, M, N, K, dev)
     ws_b = sq.workspace(sq.SQ_OP_BUILD_NVFP4, 0, N, K, dev)
     ws_a = sq.workspace(sq.SQ_OP_ACT_QUANT_NVFP4, M, 0, K, dev)
     ws_n = sq.workspace(sq.SQ_OP_LINEAR_FWD_NVFP4, M, N, K, dev)
@@ -145,12 +153,17 @@ def main():
     s4, f4 = torch.empty_like(w4.scales), torch.empty_like(w4.frac_idx)
     s6, f6 = torch.empty_like(w6.scales), torch.empty_like(w6.frac_idx)
     cn, sfn, gn = torch.empty_like(wn.codes), torch.empty_like(wn.scales), torch.empty_like(wn.g_w)
+    c8, s8, f8 = torch.empty_like(w8.codes), torch.empty_like(w8.scales), torch.empty_like(w8.frac_idx)
     RES = sq.SQ_RECON_RESIDUAL_ONLY
     calls = {
         "act_quant": lambda: sq.sq_act_quant_nvfp4(x, xc, xsf, gx, D, t, ws=ws_a),
         "act_quant_nolowrank": lambda: sq.sq_act_quant_nvfp4(x, xc, xsf, gx, ws=ws_a),
         "fwd_nvfp4": lambda: sq.sq_linear_fwd(wn, x, y, g_x=gx, ws=ws_n),
         "fwd_int4": lambda: sq.sq_linear_fwd(w4, x, y, ws=ws_i),
+        "fwd_int8": lambda: sq.sq_linear_fwd(w8, x, y, ws=ws_8),
+        "build_int8": lambda: sq.sq_build_int8(R, c8, s8, f8),
+        "recon_int8": lambda: sq.sq_reconstruct_bf16(w8, W),
+        "recon_int8_resid": lambda: sq.sq_reconstruct_bf16(w8, W, RES),
         "build_nvfp4": lambda: sq.sq_build_nvfp4(R, cn, sfn, gn, ws_b),
         "build_int4": lambda: sq.sq_build_int4(R, c4, s4, f4),
         "build_int4_g64": lambda: sq.sq_build_int4(R, c4, s6, f6, group=64),

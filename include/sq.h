@@ -65,7 +65,8 @@ typedef enum {
 typedef enum {
     SQ_FMT_INT4_G32 = 1,   /* int4 codes [N, K/2], fp16 scales [N, K/32]          */
     SQ_FMT_NVFP4 = 2,      /* e2m1 codes [N, K/2], ue4m3 tiled scales, fp32 g_w   */
-    SQ_FMT_INT4_G64 = 3    /* int4 codes [N, K/2], fp16 scales [N, K/64]          */
+    SQ_FMT_INT4_G64 = 3,   /* int4 codes [N, K/2], fp16 scales [N, K/64]          */
+    SQ_FMT_INT8_ROW = 4    /* int8 codes [N, K], fp32 scales [N], rank-16 low rank */
 } sq_format;
 
 /* operations for sq_workspace_bytes() */
@@ -75,7 +76,9 @@ typedef enum {
     SQ_OP_ACT_QUANT_NVFP4 = 3,
     SQ_OP_LINEAR_FWD_NVFP4 = 4,
     SQ_OP_LINEAR_FWD_INT4 = 5,
-    SQ_OP_RECONSTRUCT = 6
+    SQ_OP_RECONSTRUCT = 6,
+    SQ_OP_LINEAR_FWD_INT8 = 7,
+    SQ_OP_BUILD_INT8 = 8
 } sq_op;
 
 /* flags */
@@ -84,15 +87,19 @@ typedef enum {
 
 /*
  * A built weight.  All pointers are device pointers owned by the caller.
- *   fmt        SQ_FMT_INT4_G32, SQ_FMT_INT4_G64 or SQ_FMT_NVFP4
- *   N, K       output / input features
- *   codes      [N, K/2] uint8, value 2k in the low nibble of byte k
- *              (int4: 4-bit two's complement in [-7, 7]; NVFP4: e2m1)
+ *   fmt        SQ_FMT_INT4_G32, SQ_FMT_INT4_G64, SQ_FMT_NVFP4 or SQ_FMT_INT8_ROW
+ *   N, K       output / input features (SQ_FMT_INT8_ROW: K <= 16384)
+ *   codes      4-bit formats: [N, K/2] uint8, value 2k in the low nibble of
+ *              byte k (int4: 4-bit two's complement in [-7, 7]; NVFP4: e2m1);
+ *              SQ_FMT_INT8_ROW: [N, K] int8 in [-127, 127]
  *   scales     int4: fp16 bits [N, K/32] (group 32) or [N, K/64] (group 64);
- *              NVFP4: ue4m3 bytes in the tiled layout, sq_sf_bytes(N, K) bytes
+ *              NVFP4: ue4m3 bytes in the tiled layout, sq_sf_bytes(N, K) bytes;
+ *              SQ_FMT_INT8_ROW: fp32 [N], one per row
  *   g_w        NVFP4 only: 1 float, the per-tensor global scale
- *   lora_up    bf16 [N, 32], or NULL for no low-rank branch
- *   lora_down  bf16 [K, 32], or NULL for no low-rank branch
+ *   lora_up    bf16 [N, 32] ([N, 16] for SQ_FMT_INT8_ROW), or NULL for no
+ *              low-rank branch
+ *   lora_down  bf16 [K, 32] ([K, 16] for SQ_FMT_INT8_ROW), or NULL for no
+ *              low-rank branch
  */
 typedef struct {
     int32_t fmt;
@@ -150,6 +157,25 @@ SQ_API sq_status sq_build_int4(const float *R, int64_t N, int64_t K, int32_t gro
                         void *stream);
 
 /*
+ * int8 per-row builder (SquareQ README, "v3.1 -- int8-residual mode": int8
+ * per-row, MSE-swept, of the H256-rotated rank-16 residual).  For each row of
+ * R [N, K] fp32 (device, K <= 16384): rotate every 256-block with H256; with
+ * a = max|r_k| over the row try the fractions f_j = (50 + 2j)/100,
+ * j = 0..25, of the int4 sweep:
+ *   s_j = RN(RN(f_j a) / 127) (fp32),  q_k = clamp(rint(RN(r_k RN(1/s_j))), -127, 127),
+ *   error_j = sum of RN(fmaf(-q_k, s_j, r_k)^2): per 256-block, each 32-value
+ *             group by the xor butterfly (strides 16, 8, 4, 2, 1), the 8 group
+ *             sums by a butterfly over the group index (strides 4, 2, 1), then
+ *             the blocks added in order from block 0
+ * (a scale of 0 gives q = 0 and error r_k^2); keep the smallest error, the
+ * smaller j on ties.  Outputs (device): codes [N, K] int8, scales [N] fp32,
+ * frac_idx [N] winning j (may be NULL).  The weight is SQ_FMT_INT8_ROW, whose
+ * low-rank branch has rank 16.
+ */
+SQ_API sq_status sq_build_int8(const float *R, int64_t N, int64_t K, int8_t *codes, float *scales,
+                               uint8_t *frac_idx, void *stream);
+
+/*
  * NVFP4 builder (SquareQ README, "Residual codecs": e2m1 + ue4m3 block-16
  * scales in the tiled layout + per-tensor global scale).  Pass 1 rotates R
  * [N, K] fp32 (device) and takes A = max|H R|; g_w = RN(A / 2688), i.e.
@@ -189,6 +215,8 @@ SQ_API sq_status sq_act_quant_nvfp4(const uint16_t *x, int64_t M, int64_t K,
  *   int4:  "dequant-first": xb = bf16(H x), wb = bf16(q s), y = xb wb^T +
  *          t lora_up^T on bf16 tensor cores (fp32 accumulation); either
  *          group size (SQ_FMT_INT4_G32 / _G64).
+ *   int8:  the same with wb = bf16(RN(q s_row)) and the rank-16 branch
+ *          (SQ_FMT_INT8_ROW; workspace op SQ_OP_LINEAR_FWD_INT8).
  * The low-rank term is accumulated on the tensor cores in the same
  * accumulator.  Accuracy: max|y - y_exact| / max|y_exact| <= 2e-3 against the
  * exact result on the same quantised operands.  flags: SQ_ACT_STATIC_SCALE
@@ -237,9 +265,11 @@ SQ_API sq_status sq_linear_fwd_noalloc(const sq_weight *w, const uint16_t *x, in
 /*
  * bf16 reconstruct of W for the backward pass (SquareQ README: "the bwd-side
  * bf16 reconstruct from the same payload").  For each element
- *   d = q s (int4, either group size) or RN(RN(e2m1 value(sf)) g_w) (NVFP4),
+ *   d = q s (int4, either group size), RN(q s_row) (int8) or
+ *       RN(RN(e2m1 value(sf)) g_w) (NVFP4),
  *   h = H256 applied to each 256-block of d along K,
- *   L = fmaf(U[n,31], D[k,31], ... fmaf(U[n,0], D[k,0], 0)),
+ *   L = fmaf(U[n,R-1], D[k,R-1], ... fmaf(U[n,0], D[k,0], 0)), R the rank
+ *       (32; 16 for SQ_FMT_INT8_ROW),
  *   W[n, k] = bf16(RN(L + h))          (bf16(h) with SQ_RECON_RESIDUAL_ONLY
  *                                       or NULL low-rank pointers).
  * W_out: [N, K] bf16 (device).

@@ -52,6 +52,8 @@ def test_size_helpers():
     assert ws >= 64 * 256 + sq.sq_sf_bytes(64, 512) + 64 * 32 * 4 + 64 * 128 + 256 * 128
     wsi = sq.sq_workspace_bytes(sq.SQ_OP_LINEAR_FWD_INT4, 64, 256, 512)
     assert wsi >= 64 * 512 * 2 + 256 * 512 * 2
+    # int8: the int4 layout plus the rank-16 factors widened to rank 32
+    assert sq.sq_workspace_bytes(sq.SQ_OP_LINEAR_FWD_INT8, 64, 256, 512) >= wsi + (512 + 256) * 64
     assert sq.sq_workspace_bytes(99, 1, 1, 1) == 0
     assert sq.status_str(0) == "ok"
     assert sq.status_str(2) == "unsupported shape"
@@ -70,6 +72,17 @@ def test_build_int4_validation():
     assert _int4(group=128) == SQ_ERR_SHAPE
     assert _int4(R=MIS) == SQ_ERR_ALIGN
     assert _int4(frac=MIS) == SQ_ERR_ALIGN
+
+
+def test_build_int8_validation():
+    L = sq.lib()
+    assert L.sq_build_int8(None, 256, 512, A, A, None, None) == SQ_ERR_NULL
+    assert L.sq_build_int8(A, 256, 512, None, A, None, None) == SQ_ERR_NULL
+    assert L.sq_build_int8(A, 256, 300, A, A, None, None) == SQ_ERR_SHAPE
+    assert L.sq_build_int8(A, 256, 16384 + 256, A, A, None, None) == SQ_ERR_SHAPE   # one rotated row in smem
+    assert L.sq_build_int8(A, 100, 512, A, A, None, None) == SQ_ERR_SHAPE
+    assert L.sq_build_int8(MIS, 256, 512, A, A, None, None) == SQ_ERR_ALIGN
+    assert L.sq_build_int8(A, 256, 512, A, A + 2, None, None) == SQ_ERR_ALIGN
 
 
 def test_build_nvfp4_validation():
@@ -102,6 +115,7 @@ def test_linear_fwd_validation():
     assert fwd(_w(codes=None)) == SQ_ERR_NULL
     assert fwd(_w(g_w=None)) == SQ_ERR_NULL
     assert fwd(_w(fmt=7)) == SQ_ERR_ARG
+    assert fwd(_w(fmt=sq.SQ_FMT_INT8_ROW, K=16384 + 256, g_w=None)) == SQ_ERR_SHAPE
     assert fwd(_w(N=192)) == SQ_ERR_SHAPE
     assert fwd(_w(), M=0) == SQ_ERR_SHAPE
     assert fwd(_w(), y=MIS) == SQ_ERR_ALIGN
@@ -124,6 +138,9 @@ def test_reconstruct_validation():
 def test_valid_call_without_device_reports_device_error():
     assert _int4() == SQ_ERR_DEVICE
     assert _int4(group=64) == SQ_ERR_DEVICE            # group 64 passes validation
+    assert sq.lib().sq_build_int8(A, 256, 512, A, A, None, None) == SQ_ERR_DEVICE
+    assert sq.lib().sq_reconstruct_bf16(ctypes.byref(_w(fmt=sq.SQ_FMT_INT8_ROW, g_w=None)), A, 0, None) \
+        == SQ_ERR_DEVICE
     assert sq.lib().sq_reconstruct_bf16(ctypes.byref(_w(fmt=sq.SQ_FMT_INT4_G64, g_w=None)), A, 0, None) \
         == SQ_ERR_DEVICE
     assert sq.lib().sq_reconstruct_bf16(ctypes.byref(_w()), A, 0, None) == SQ_ERR_DEVICE
