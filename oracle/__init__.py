@@ -73,6 +73,7 @@ _SIGS = {
     "or_build_int8": ([_P, _I64, _I64, _P, _P, _P], None),
     "or_linear_fwd_int8": ([_P, _P, _P, _P, _P, _I64, _I64, _I64, _P, _I64, _P], None),
     "or_lowrank_input": ([_P, _I64, _I64, _P, ctypes.c_int, _P], None),
+    "or_linear_bwd_dx": ([_P, _P, _I64, _I64, _I64, _P, _I64, _P], None),
 }
 
 
@@ -358,3 +359,17 @@ def reconstruct_bf16(fmt, codes, scales, g_w, U_bits, D_bits, N, K, residual_onl
     lib().or_reconstruct_bf16(int(fmt), _p(codes), _p(scales), float(np.float32(g_w)),
                               _p(U), _p(D), N, K, 1 if residual_only else 0, _p(W))
     return W
+
+
+# ---- backward of the input ------------------------------------------------
+
+def linear_bwd_dx(dy_bits, W_bits, rows=None):
+    """dx = dy W in fp64 [n_rows, K]: dy [M, N] bf16 bits, W [N, K] bf16 bits (the reconstruct)."""
+    dy = _c(dy_bits, np.uint16)
+    W = _c(W_bits, np.uint16)
+    M, N = dy.shape
+    K = W.shape[1]
+    rows = np.arange(M, dtype=np.int64) if rows is None else _c(rows, np.int64)
+    dx = np.empty((len(rows), K), np.float64)
+    lib().or_linear_bwd_dx(_p(dy), _p(W), M, N, K, _p(rows), len(rows), _p(dx))
+    return dx

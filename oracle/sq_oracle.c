@@ -976,3 +976,33 @@ void or_reconstruct_bf16(int fmt, const uint8_t *codes, const void *scales, floa
         }
     }
 }
+
+/* ------------------------------------------------------------------------ */
+/* Backward of the input: dx = dy W on the bf16 reconstruct                  */
+/* ------------------------------------------------------------------------ */
+
+/*
+ * dx[m, k] = sum_n dy[m, n] W[n, k] in fp64 on the exact bf16 operands
+ * (SquareQ README, "End-to-end": the backward rebuilds bf16 W from the payload
+ * and runs the normal bf16 GEMM).  dy [M, N] and W [N, K] are bf16 bits (W as
+ * or_reconstruct_bf16 writes it); only the rows listed in `rows` are
+ * evaluated; dx is [n_rows, K].
+ */
+void or_linear_bwd_dx(const uint16_t *dy, const uint16_t *W, int64_t M, int64_t N, int64_t K,
+                      const int64_t *rows, int64_t n_rows, double *dx)
+{
+    (void)M;
+#pragma omp parallel for schedule(static)
+    for (int64_t i = 0; i < n_rows; i++) {
+        double *acc = (double *)calloc((size_t)K, sizeof(double));
+        for (int64_t n = 0; n < N; n++) {
+            double a = (double)or_bf16_to_f32(dy[rows[i] * N + n]);
+            if (a == 0.0)
+                continue;
+            for (int64_t k = 0; k < K; k++)
+                acc[k] += a * (double)or_bf16_to_f32(W[n * K + k]);
+        }
+        memcpy(dx + i * K, acc, (size_t)K * sizeof(double));
+        free(acc);
+    }
+}

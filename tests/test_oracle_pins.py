@@ -455,3 +455,22 @@ def test_reconstruct_lowrank_chain_and_fidelity(oracle_mod):
                                                              residual_only=True)).astype(np.float64)
         cos_r = (Wr * d["R"]).sum() / np.linalg.norm(Wr) / np.linalg.norm(d["R"])
         assert cos_r > 0.98
+
+
+# --------------------------------------------------------------------------
+# backward of the input ("End-to-end": bf16 reconstruct, then the bf16 GEMM)
+# --------------------------------------------------------------------------
+
+def test_bwd_dx_equals_decoded_gemm(oracle_mod):
+    M, K, N = 12, 512, 136
+    d = si.make_inputs(M, K, N, 33)
+    c, s, _ = oracle_mod.build_int4(d["R"])
+    W = oracle_mod.reconstruct_bf16(oracle_mod.FMT_INT4, c, s, 0.0, d["U"], d["D"], N, K)
+    rng = np.random.default_rng(34)
+    dy = si.to_bf16_bits(rng.standard_normal((M, N)).astype(np.float32))
+    dy[3, :] = 0
+    dx = oracle_mod.linear_bwd_dx(dy, W)
+    want = si.bf16_bits_to_f32(dy).astype(np.float64) @ si.bf16_bits_to_f32(W).astype(np.float64)
+    assert np.allclose(dx, want, rtol=1e-12, atol=1e-12 * np.abs(want).max())
+    rows = np.array([0, 5, 11], np.int64)
+    assert np.array_equal(oracle_mod.linear_bwd_dx(dy, W, rows), dx[rows])
