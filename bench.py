@@ -6,7 +6,8 @@ chosen shape (default the headline 4480 x 16384 x 6144, M x N x K):
   sq_build_int4, sq_build_nvfp4, sq_linear_fwd (NVFP4, incl. the activation
   prologue), sq_linear_fwd (int4), sq_reconstruct_bf16 (both payloads), and the
   build, forward and reconstruct of the int4 group-64 variant and of the int8
-  per-row mode (rank-16 low-rank branch).
+  per-row mode (rank-16 low-rank branch), and the input backward dx = dy W
+  (transposed bf16 reconstruct + bf16 GEMM) on the NVFP4 payload.
 Every op is timed with CUDA events on the launching stream after an L2 flush
 (a 256 MB write outside the op's events); the NVFP4 forward is the headline
 metric (TFLOP/s = 2 M N K / time of the whole sq_linear_fwd call).  The GEMM
@@ -92,8 +93,10 @@ def op_work(M, N, K):
         "build_int8": ("GB/s", NK * (4 + 1) + N * 5),
         "fwd_int8": ("TFLOP/s", 2.0 * M * N * K),
         "reconstruct_int8": ("GB/s", NK * (1 + 2) + N * 4),
+        "bwd_dx_nvfp4": ("TFLOP/s", 2.0 * M * N * K),
         "gemm_nvfp4": ("TFLOP/s", 2.0 * M * N * K),
         "gemm_int4": ("TFLOP/s", 2.0 * M * N * K),
+        "gemm_bwd_dx": ("TFLOP/s", 2.0 * M * N * K),
     }
 
 
@@ -102,6 +105,7 @@ LAUNCHES_PER_STEP = {   # our kernels per op (memsets excluded)
     "reconstruct_nvfp4": 1, "reconstruct_int4": 1,
     "build_int4_g64": 1, "fwd_int4_g64": 5, "reconstruct_int4_g64": 1,
     "build_int8": 1, "fwd_int8": 7, "reconstruct_int8": 1,
+    "bwd_dx_nvfp4": 2,
 }
 
 
@@ -354,6 +358,9 @@ def run_sq(args, cfg, d, rank, world, local_rank):
                    torch.empty(N, dtype=torch.float32, device=dev), None, U16, D16,
                    torch.empty(N, dtype=torch.uint8, device=dev))
     ws_i8 = sq.workspace(sq.SQ_OP_LINEAR_FWD_INT8, M, N, K, dev)
+    ws_dx = sq.workspace(sq.SQ_OP_LINEAR_BWD_DX, M, N, K, dev)
+    dy = torch.randn((M, N), device=dev, generator=torch.Generator(device=dev).manual_seed(cfg.seed)).to(torch.bfloat16)
+    dx = torch.empty((M, K), dtype=torch.float32, device=dev)
     ws_b = sq.workspace(sq.SQ_OP_BUILD_NVFP4, 0, N, K, dev)
     ws_nv = sq.workspace(sq.SQ_OP_LINEAR_FWD_NVFP4, M, N, K, dev)
     ws_i4 = sq.workspace(sq.SQ_OP_LINEAR_FWD_INT4, M, N, K, dev)
@@ -376,9 +383,10 @@ def run_sq(args, cfg, d, rank, world, local_rank):
         ("build_int8", lambda: sq.sq_build_int8(R, i8.codes, i8.scales, i8.frac_idx)),
         ("fwd_int8", lambda: sq.sq_linear_fwd(i8, x, y_i4, ws=ws_i8)),
         ("reconstruct_int8", lambda: sq.sq_reconstruct_bf16(i8, W)),
+        ("bwd_dx_nvfp4", lambda: sq.sq_linear_bwd_dx(nv, dy, dx, ws_dx)),
     ]
     names = [n for n, _ in ops]
-    gemm_of = {"fwd_nvfp4": "gemm_nvfp4", "fwd_int4": "gemm_int4"}
+    gemm_of = {"fwd_nvfp4": "gemm_nvfp4", "fwd_int4": "gemm_int4", "bwd_dx_nvfp4": "gemm_bwd_dx"}
 
     # The GEMM kernel's own events are recorded on even steps only: an event between
     # the activation quantisation and the GEMM launch would stop the GEMM's set-up
@@ -500,8 +508,9 @@ def summarise(args, cfg, per_op, outer_ms, clocks, e2e, world, cpu):
         if unit == "GB/s":
             frac, peak = rate / peaks["hbm_gbs"], "hbm"
         else:
-            peak_v = fp4_peak if "nvfp4" in k else peaks["bf16_tflops"]
-            frac, peak = rate / peak_v, "fp4 tensor" if "nvfp4" in k else "bf16 tensor"
+            fp4 = k in ("fwd_nvfp4", "gemm_nvfp4")      # the backward's GEMM runs in bf16
+            peak_v = fp4_peak if fp4 else peaks["bf16_tflops"]
+            frac, peak = rate / peak_v, "fp4 tensor" if fp4 else "bf16 tensor"
         ops[k] = {"ms": ms, unit: rate, "frac": frac, "of": f"{peak} ({peak_src})"}
     fwd_tflops = 2.0 * M * N * K / (per_op["fwd_nvfp4"] * 1e-3) / 1e12
     gemm_tflops = 2.0 * M * N * K / (per_op["gemm_nvfp4"] * 1e-3) / 1e12

@@ -37,13 +37,15 @@ SQ_OP_BUILD_INT8 = 8
 RANK_INT8 = 16
 SQ_ACT_STATIC_SCALE = 0x1
 SQ_RECON_RESIDUAL_ONLY = 0x2
+SQ_RECON_TRANSPOSED = 0x4
+SQ_OP_LINEAR_BWD_DX = 9
 RANK = 32
 
 EXPORTED = [
     "sq_status_str", "sq_abi_version", "sq_last_error_detail", "sq_sf_bytes", "sq_workspace_bytes",
     "sq_build_int4", "sq_build_int8", "sq_build_nvfp4", "sq_act_quant_nvfp4", "sq_linear_fwd",
     "sq_reconstruct_bf16",
-    "sq_check_device_status", "sq_set_gemm_events", "sq_linear_fwd_noalloc",
+    "sq_check_device_status", "sq_set_gemm_events", "sq_linear_fwd_noalloc", "sq_linear_bwd_dx",
 ]
 
 
@@ -87,6 +89,7 @@ _SIGS = {
     "sq_linear_fwd_noalloc": ([ctypes.POINTER(sq_weight), _P, _I64, _P, _P, ctypes.c_uint32,
                                ctypes.POINTER(ctypes.c_void_p), _P], ctypes.c_int),
     "sq_reconstruct_bf16": ([ctypes.POINTER(sq_weight), _P, ctypes.c_uint32, _P], ctypes.c_int),
+    "sq_linear_bwd_dx": ([ctypes.POINTER(sq_weight), _P, _I64, _P, _P, ctypes.c_size_t, _P], ctypes.c_int),
     "sq_check_device_status": ([_P, _P], ctypes.c_int),
     "sq_set_gemm_events": ([_P, _P], ctypes.c_int),
 }
@@ -204,6 +207,13 @@ def sq_reconstruct_bf16(w: "Weight", W_out, flags: int = 0, stream=None):
     _check("sq_reconstruct_bf16", lib().sq_reconstruct_bf16(ctypes.byref(cw), _ptr(W_out), flags, _stream(stream)))
 
 
+def sq_linear_bwd_dx(w: "Weight", dy, dx, ws, stream=None):
+    M = dy.shape[0]
+    cw = w.as_c()
+    _check("sq_linear_bwd_dx", lib().sq_linear_bwd_dx(ctypes.byref(cw), _ptr(dy), M, _ptr(dx), _ptr(ws),
+                                                      _numel_bytes(ws), _stream(stream)))
+
+
 def sq_check_device_status(ws, stream=None):
     _check("sq_check_device_status", lib().sq_check_device_status(_ptr(ws), _stream(stream)))
 
@@ -286,7 +296,18 @@ def linear_fwd(w: Weight, x: torch.Tensor, ws=None, g_x=None, flags: int = 0, st
     return y
 
 
-def reconstruct_bf16(w: Weight, residual_only: bool = False, stream=None) -> torch.Tensor:
-    W = torch.empty((w.N, w.K), dtype=torch.bfloat16, device=w.codes.device)
-    sq_reconstruct_bf16(w, W, SQ_RECON_RESIDUAL_ONLY if residual_only else 0, stream=stream)
+def reconstruct_bf16(w: Weight, residual_only: bool = False, transposed: bool = False, stream=None) -> torch.Tensor:
+    shape = (w.K, w.N) if transposed else (w.N, w.K)
+    W = torch.empty(shape, dtype=torch.bfloat16, device=w.codes.device)
+    flags = (SQ_RECON_RESIDUAL_ONLY if residual_only else 0) | (SQ_RECON_TRANSPOSED if transposed else 0)
+    sq_reconstruct_bf16(w, W, flags, stream=stream)
     return W
+
+
+def linear_bwd_dx(w: Weight, dy: torch.Tensor, ws=None, stream=None) -> torch.Tensor:
+    """dx = dy W (dy [M, N] bf16) as fp32 [M, K]."""
+    M = dy.shape[0]
+    dx = torch.empty((M, w.K), dtype=torch.float32, device=dy.device)
+    ws = ws if ws is not None else workspace(SQ_OP_LINEAR_BWD_DX, M, w.N, w.K, dy.device)
+    sq_linear_bwd_dx(w, dy, dx, ws, stream=stream)
+    return dx

@@ -214,6 +214,8 @@ size_t sq_workspace_bytes(int op, int64_t M, int64_t N, int64_t K)
         return fwd_layout(SQ_FMT_INT8_ROW, M, N, K).total;
     case SQ_OP_BUILD_INT8:
         return kHeader;
+    case SQ_OP_LINEAR_BWD_DX:
+        return kAlign + round_up((size_t)N * (size_t)K * 2, kAlign);
     default:
         return 0;
     }
@@ -465,7 +467,7 @@ sq_status sq_reconstruct_bf16(const sq_weight *w, uint16_t *W_out, uint32_t flag
         return st;
     if (!W_out)
         return SQ_ERR_NULL;
-    if (flags & ~SQ_RECON_RESIDUAL_ONLY)
+    if (flags & ~(SQ_RECON_RESIDUAL_ONLY | SQ_RECON_TRANSPOSED))
         return SQ_ERR_ARG;
     if (!aligned(W_out, 16))
         return SQ_ERR_ALIGN;
@@ -474,10 +476,56 @@ sq_status sq_reconstruct_bf16(const sq_weight *w, uint16_t *W_out, uint32_t flag
     if (st != SQ_OK)
         return st;
     const int with_lowrank = (!(flags & SQ_RECON_RESIDUAL_ONLY) && w->lora_up && w->lora_down) ? 1 : 0;
+    const int transposed = (flags & SQ_RECON_TRANSPOSED) ? 1 : 0;
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     SQ_CUDA(sq::launch_reconstruct(w->fmt, w->codes, w->scales, w->g_w, w->lora_up, w->lora_down, w->N, w->K,
-                                   with_lowrank, W_out, sms, s),
+                                   with_lowrank, transposed, W_out, sms, s),
             "reconstruct");
+    return SQ_OK;
+}
+
+sq_status sq_linear_bwd_dx(const sq_weight *w, const uint16_t *dy, int64_t M, float *dx, void *ws, size_t ws_bytes,
+                           void *stream)
+{
+    sq_status st = check_weight(w);
+    if (st != SQ_OK)
+        return st;
+    if (!dy || !dx || !ws)
+        return SQ_ERR_NULL;
+    const int64_t N = w->N, K = w->K;
+    if (M < 1 || M > kMaxM)
+        return SQ_ERR_SHAPE;
+    if (!aligned(dy, 16) || !aligned(dx, 16) || !aligned(ws, 256))
+        return SQ_ERR_ALIGN;
+    if (ws_bytes < sq_workspace_bytes(SQ_OP_LINEAR_BWD_DX, M, N, K))
+        return SQ_ERR_WORKSPACE;
+    int sms = 0;
+    st = check_device(&sms);
+    if (st != SQ_OK)
+        return st;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    uint32_t *status = reinterpret_cast<uint32_t *>(ws_at(ws, 0));
+    uint16_t *wt = reinterpret_cast<uint16_t *>(ws_at(ws, kAlign));      // W^T [K, N] bf16
+    const int with_lowrank = (w->lora_up && w->lora_down) ? 1 : 0;
+    SQ_CUDA(cudaMemsetAsync(status, 0, 8, s), "memset");
+    SQ_CUDA(sq::launch_reconstruct(w->fmt, w->codes, w->scales, w->g_w, w->lora_up, w->lora_down, N, K,
+                                   with_lowrank, 1, wt, sms, s),
+            "transposed reconstruct");
+    sq::GemmLaunch g;
+    memset(&g, 0, sizeof(g));
+    g.fp4 = 0;
+    g.a = dy;             // [M, N]: the reduction runs over N
+    g.b = wt;             // [K, N]
+    g.y = dx;             // [M, K]
+    g.status = status;
+    g.M = M;
+    g.N = K;
+    g.K = N;
+    if (g_gemm_ev0)
+        SQ_CUDA(cudaEventRecord(g_gemm_ev0, s), "event record");
+    SQ_CUDA(sq::launch_gemm(g, sms, s), "gemm");
+    if (g_gemm_ev1)
+        SQ_CUDA(cudaEventRecord(g_gemm_ev1, s), "event record");
     return SQ_OK;
 }
 

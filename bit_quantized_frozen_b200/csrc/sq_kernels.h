@@ -47,7 +47,7 @@ cudaError_t launch_lowrank_finish(const float *t32, int64_t M, const float *g_x,
 // fmt: 1 int4 group 32, 2 NVFP4, 3 int4 group 64, 4 int8 per row (rank 16)
 cudaError_t launch_reconstruct(int fmt, const uint8_t *codes, const void *scales, const float *g_w,
                                const uint16_t *U, const uint16_t *D, int64_t N, int64_t K, int with_lowrank,
-                               uint16_t *W, int sms, cudaStream_t s);
+                               int transposed, uint16_t *W, int sms, cudaStream_t s);
 
 // forward GEMM y = beta (A B^T + tsplit udup^T), see sq_gemm.cu
 struct GemmLaunch {

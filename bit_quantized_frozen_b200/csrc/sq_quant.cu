@@ -962,7 +962,8 @@ __global__ void __launch_bounds__(256) lowrank_finish_kernel(const float *__rest
 //   transform and writes h into a
 //   shared fp32 tile (float4 f of a row stored at f ^ (f >> 3) -- conflict free
 //   for both phases).
-// Phase 2: thread t owns columns 2(t%128), 2(t%128)+1 and rows 32(t/128)..+31.
+// Phase 2 (with the low-rank term, or for the transposed output W^T [K, N]):
+//   thread t owns columns 2(t%128), 2(t%128)+1 and rows 32(t/128)..+31.
 //   lora_down for its two columns stays in registers; lora_up rows are
 //   broadcast from shared memory; each output's fmaf chain runs in order
 //   r = 0..rank-1 from 0 (rank 32, or 16 for int8), two columns at a time with
@@ -1120,8 +1121,8 @@ __device__ __forceinline__ void rec_decode(const uint8_t *stage, int r, int q, f
     }
 }
 
-template <int FMT, bool LOWRANK>
-__global__ void __launch_bounds__(256, LOWRANK ? 2 : 3) reconstruct_kernel(const uint8_t *__restrict__ codes,
+template <int FMT, bool LOWRANK, bool TRANS>
+__global__ void __launch_bounds__(256, (LOWRANK || TRANS) ? 2 : 3) reconstruct_kernel(const uint8_t *__restrict__ codes,
                                                              const void *__restrict__ scales,
                                                              const float *__restrict__ g_w,
                                                              const uint16_t *__restrict__ U,
@@ -1133,7 +1134,8 @@ __global__ void __launch_bounds__(256, LOWRANK ? 2 : 3) reconstruct_kernel(const
     extern __shared__ __align__(128) uint8_t rec_smem[];
     float *h = reinterpret_cast<float *>(rec_smem);                                // [64][256] swizzled
     float *us = reinterpret_cast<float *>(rec_smem + kRecHBytes);                  // [64][rank] lora_up, fp32
-    uint8_t *stage0 = rec_smem + (LOWRANK ? kRecHBytes + Cfg::kUsBytes : 0);
+    constexpr bool kTile = LOWRANK || TRANS;      // h goes through the shared tile (phase 2 writes W)
+    uint8_t *stage0 = rec_smem + (kTile ? kRecHBytes + Cfg::kUsBytes : 0);
     const int tid = threadIdx.x;
     const int lane = tid & 31, warp = tid >> 5;
     const float g = FMT == 2 ? *g_w : 0.0f;
@@ -1175,7 +1177,7 @@ __global__ void __launch_bounds__(256, LOWRANK ? 2 : 3) reconstruct_kernel(const
             float v[32];
             rec_decode<FMT>(st, r, q, g, v);
             fwht256_l32(v, lane);
-            if (!LOWRANK) {                          // residual only: straight to W
+            if (!kTile) {                            // residual only, row-major: straight to W
                 const int64_t n = n0 + r;
                 if (n < N) {
                     uint4 *o = reinterpret_cast<uint4 *>(W + n * K + kb * kHad + 32 * q);
@@ -1198,18 +1200,18 @@ __global__ void __launch_bounds__(256, LOWRANK ? 2 : 3) reconstruct_kernel(const
                 }
             }
         }
-        if (!LOWRANK) {
+        if (!kTile) {
             __syncthreads();                         // stage buffer free before the next prefetch lands
             continue;
         }
-        {
+        if (LOWRANK) {
             const uint16_t *ust = reinterpret_cast<const uint16_t *>(st + Cfg::kCodeBytes + kRecScaleBytes);
 #pragma unroll
             for (int j = 0; j < kRecRows * kR / 256; ++j) {
                 us[tid + 256 * j] = bf16_bits_to_f32(ust[tid + 256 * j]);
             }
         }
-        if (kb != cur_kb) {                          // lora_down of this thread's two columns
+        if (LOWRANK && kb != cur_kb) {               // lora_down of this thread's two columns
             cur_kb = kb;
             const int64_t k0 = kb * kHad + 2 * cp;
             const uint4 *dr0 = reinterpret_cast<const uint4 *>(D + k0 * kR);
@@ -1229,11 +1231,13 @@ __global__ void __launch_bounds__(256, LOWRANK ? 2 : 3) reconstruct_kernel(const
 
         // phase 2
         const int64_t k0 = kb * kHad + 2 * cp;
-#pragma unroll 1
+        uint32_t tw0[16], tw1[16];                   // TRANS: columns k0, k0 + 1 of the 32 rows, bf16 pairs
+        constexpr int kUnroll = TRANS ? 8 : 1;       // register-indexed pieces need constant indices
+#pragma unroll kUnroll
         for (int r0 = rbase; r0 < rbase + 32; r0 += 4) {
             uint64_t acc[4] = {0ull, 0ull, 0ull, 0ull};
 #pragma unroll
-            for (int rr = 0; rr < kR; rr += 4) {
+            for (int rr = 0; rr < (LOWRANK ? kR : 0); rr += 4) {
                 float4 u4[4];
 #pragma unroll
                 for (int j = 0; j < 4; ++j)
@@ -1250,14 +1254,38 @@ __global__ void __launch_bounds__(256, LOWRANK ? 2 : 3) reconstruct_kernel(const
             for (int j = 0; j < 4; ++j) {
                 const int r = r0 + j;
                 const int64_t n = n0 + r;
-                if (n >= N)
-                    continue;
                 const float2 hv = *reinterpret_cast<const float2 *>(h + r * kHad + 4 * (f ^ (f >> 3)) + fo);
                 float L0, L1;
                 unpack2(acc[j], L0, L1);
-                const uint32_t o = f32_to_bf16_bits(__fadd_rn(L0, hv.x)) |
-                                   (f32_to_bf16_bits(__fadd_rn(L1, hv.y)) << 16);
-                *reinterpret_cast<uint32_t *>(W + n * K + k0) = o;
+                // with the low-rank term W = bf16(RN(L + h)); residual only: bf16(h)
+                const uint32_t b0 = f32_to_bf16_bits(LOWRANK ? __fadd_rn(L0, hv.x) : hv.x);
+                const uint32_t b1 = f32_to_bf16_bits(LOWRANK ? __fadd_rn(L1, hv.y) : hv.y);
+                if (TRANS) {
+                    const int slot = (r - rbase) >> 1, hi = (r - rbase) & 1;
+                    tw0[slot] = hi ? (tw0[slot] | (b0 << 16)) : b0;
+                    tw1[slot] = hi ? (tw1[slot] | (b1 << 16)) : b1;
+                } else if (n < N) {
+                    *reinterpret_cast<uint32_t *>(W + n * K + k0) = b0 | (b1 << 16);
+                }
+            }
+        }
+        if (TRANS) {                                 // W^T [K, N]: rows k0, k0 + 1, columns n0 + rbase .. + 31
+            const int64_t nb0 = n0 + rbase;
+            if (nb0 + 32 <= N) {
+                uint4 *o0 = reinterpret_cast<uint4 *>(W + k0 * N + nb0);
+                uint4 *o1 = reinterpret_cast<uint4 *>(W + (k0 + 1) * N + nb0);
+#pragma unroll
+                for (int c = 0; c < 4; ++c) {
+                    o0[c] = make_uint4(tw0[4 * c], tw0[4 * c + 1], tw0[4 * c + 2], tw0[4 * c + 3]);
+                    o1[c] = make_uint4(tw1[4 * c], tw1[4 * c + 1], tw1[4 * c + 2], tw1[4 * c + 3]);
+                }
+            } else {
+#pragma unroll
+                for (int i = 0; i < 32; ++i)
+                    if (nb0 + i < N) {
+                        W[k0 * N + nb0 + i] = (uint16_t)(tw0[i >> 1] >> (16 * (i & 1)));
+                        W[(k0 + 1) * N + nb0 + i] = (uint16_t)(tw1[i >> 1] >> (16 * (i & 1)));
+                    }
             }
         }
     }
@@ -1529,43 +1557,54 @@ cudaError_t launch_lowrank_finish(const float *t32, int64_t M, const float *g_x,
     return cudaGetLastError();
 }
 
-template <int FMT>
-static cudaError_t launch_reconstruct_fmt(const uint8_t *codes, const void *scales, const float *g_w,
-                                          const uint16_t *U, const uint16_t *D, int64_t N, int64_t K,
-                                          int with_lowrank, uint16_t *W, int sms, cudaStream_t s)
+template <int FMT, bool LOWRANK, bool TRANS>
+static cudaError_t launch_reconstruct_v(const uint8_t *codes, const void *scales, const float *g_w,
+                                        const uint16_t *U, const uint16_t *D, int64_t N, int64_t K, uint16_t *W,
+                                        int sms, cudaStream_t s)
 {
     using Cfg = RecCfg<FMT>;
+    constexpr bool kTile = LOWRANK || TRANS;
+    constexpr int kSmem = kTile ? Cfg::kSmemLowrank : Cfg::kSmemResidual;
     constexpr int kMaxDev = 64;
     static bool attr_done[kMaxDev];
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDev)
         return cudaErrorInvalidDevice;
-    if (!attr_done[dev]) {
-        cudaError_t e = cudaFuncSetAttribute(reconstruct_kernel<FMT, true>,
-                                             cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::kSmemLowrank);
+    if (kTile && !attr_done[dev]) {
+        cudaError_t e = cudaFuncSetAttribute(reconstruct_kernel<FMT, LOWRANK, TRANS>,
+                                             cudaFuncAttributeMaxDynamicSharedMemorySize, kSmem);
         if (e != cudaSuccess)
             return e;
         attr_done[dev] = true;
     }
     const int64_t tiles = (K / kHad) * ((N + kRecRows - 1) / kRecRows);
-    const int64_t per_sm = with_lowrank ? 2 : 3;            // resident CTAs per SM (registers, shared memory)
+    const int64_t per_sm = kTile ? 2 : 3;                   // resident CTAs per SM (registers, shared memory)
     const unsigned grid = (unsigned)(tiles < per_sm * sms ? tiles : per_sm * sms);
-    if (with_lowrank)
-        reconstruct_kernel<FMT, true><<<grid, 256, Cfg::kSmemLowrank, s>>>(codes, scales, g_w, U, D, N, K, W);
-    else
-        reconstruct_kernel<FMT, false><<<grid, 256, Cfg::kSmemResidual, s>>>(codes, scales, g_w, U, D, N, K, W);
+    reconstruct_kernel<FMT, LOWRANK, TRANS><<<grid, 256, kSmem, s>>>(codes, scales, g_w, U, D, N, K, W);
     return cudaGetLastError();
+}
+
+template <int FMT>
+static cudaError_t launch_reconstruct_fmt(const uint8_t *codes, const void *scales, const float *g_w,
+                                          const uint16_t *U, const uint16_t *D, int64_t N, int64_t K,
+                                          int with_lowrank, int transposed, uint16_t *W, int sms, cudaStream_t s)
+{
+    if (transposed)
+        return with_lowrank ? launch_reconstruct_v<FMT, true, true>(codes, scales, g_w, U, D, N, K, W, sms, s)
+                            : launch_reconstruct_v<FMT, false, true>(codes, scales, g_w, U, D, N, K, W, sms, s);
+    return with_lowrank ? launch_reconstruct_v<FMT, true, false>(codes, scales, g_w, U, D, N, K, W, sms, s)
+                        : launch_reconstruct_v<FMT, false, false>(codes, scales, g_w, U, D, N, K, W, sms, s);
 }
 
 cudaError_t launch_reconstruct(int fmt, const uint8_t *codes, const void *scales, const float *g_w,
                                const uint16_t *U, const uint16_t *D, int64_t N, int64_t K, int with_lowrank,
-                               uint16_t *W, int sms, cudaStream_t s)
+                               int transposed, uint16_t *W, int sms, cudaStream_t s)
 {
     switch (fmt) {
-    case 2: return launch_reconstruct_fmt<2>(codes, scales, g_w, U, D, N, K, with_lowrank, W, sms, s);
-    case 3: return launch_reconstruct_fmt<3>(codes, scales, g_w, U, D, N, K, with_lowrank, W, sms, s);
-    case 4: return launch_reconstruct_fmt<4>(codes, scales, g_w, U, D, N, K, with_lowrank, W, sms, s);
-    default: return launch_reconstruct_fmt<1>(codes, scales, g_w, U, D, N, K, with_lowrank, W, sms, s);
+    case 2: return launch_reconstruct_fmt<2>(codes, scales, g_w, U, D, N, K, with_lowrank, transposed, W, sms, s);
+    case 3: return launch_reconstruct_fmt<3>(codes, scales, g_w, U, D, N, K, with_lowrank, transposed, W, sms, s);
+    case 4: return launch_reconstruct_fmt<4>(codes, scales, g_w, U, D, N, K, with_lowrank, transposed, W, sms, s);
+    default: return launch_reconstruct_fmt<1>(codes, scales, g_w, U, D, N, K, with_lowrank, transposed, W, sms, s);
     }
 }
 

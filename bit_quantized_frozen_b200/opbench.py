@@ -25,9 +25,12 @@ Operations:
                        sq_reconstruct_bf16 with the low-rank term
   recon_nvfp4_resid / recon_int4_resid / recon_int8_resid
                        sq_reconstruct_bf16 with SQ_RECON_RESIDUAL_ONLY
-  gemm_nvfp4 / gemm_int4
-                       the tensor-core GEMM launch inside sq_linear_fwd, timed by
-                       the events the library records around it (sq_set_gemm_events)
+  recon_nvfp4_t        sq_reconstruct_bf16 with SQ_RECON_TRANSPOSED (W^T)
+  bwd_dx_nvfp4         sq_linear_bwd_dx (transposed reconstruct + bf16 GEMM)
+  gemm_nvfp4 / gemm_int4 / gemm_bwd_dx
+                       the tensor-core GEMM launch inside sq_linear_fwd /
+                       sq_linear_bwd_dx, timed by the events the library records
+                       around it (sq_set_gemm_events)
 """
 from __future__ import annotations
 
@@ -54,7 +57,8 @@ FLUSH_BYTES = 256 << 20
 
 OPS = ["act_quant", "act_quant_nolowrank", "fwd_nvfp4", "fwd_int4", "fwd_int8", "build_nvfp4", "build_int4",
        "build_int4_g64", "build_int8", "recon_nvfp4", "recon_int4", "recon_int4_g64", "recon_int8",
-       "recon_nvfp4_resid", "recon_int4_resid", "recon_int8_resid", "gemm_nvfp4", "gemm_int4"]
+       "recon_nvfp4_resid", "recon_int4_resid", "recon_int8_resid", "recon_nvfp4_t", "gemm_nvfp4", "gemm_int4",
+       "bwd_dx_nvfp4", "gemm_bwd_dx"]
 
 
 def work(op, M, N, K):
@@ -62,7 +66,7 @@ def work(op, M, N, K):
     NK, MK = N * K, M * K
     if op.startswith("act_quant"):
         return "GB/s", MK * (2 + 0.5 + 1 / 16) + (M * 32 * 4 if op == "act_quant" else 0)
-    if op.startswith("fwd") or op.startswith("gemm"):
+    if op.startswith("fwd") or op.startswith("gemm") or op.startswith("bwd"):
         return "TFLOP/s", 2.0 * M * N * K
     if op == "build_nvfp4":
         return "GB/s", NK * (4 + 0.5 + 1 / 16)
@@ -74,7 +78,8 @@ def work(op, M, N, K):
         return "GB/s", NK * (4 + 1) + N * 5
     if op.startswith("recon_int8"):
         return "GB/s", NK * (1 + 2) + N * 4
-    scale = {"nvfp4": 1 / 16, "int4": 2 / 32, "int4_g64": 2 / 64}[op.split("_", 1)[1].replace("_resid", "")]
+    scale = {"nvfp4": 1 / 16, "int4": 2 / 32, "int4_g64": 2 / 64}[
+        op.split("_", 1)[1].replace("_resid", "").replace("_t", "")]
     return "GB/s", NK * (0.5 + scale + 2)
 
 
@@ -149,6 +154,10 @@ def main():
     t = torch.empty((M, 32), dtype=torch.float32, device=dev)
     y = torch.empty((M, N), dtype=torch.float32, device=dev)
     W = torch.empty((N, K), dtype=torch.bfloat16, device=dev)
+    Wt = torch.empty((K, N), dtype=torch.bfloat16, device=dev)
+    dy = torch.randn((M, N), device=dev, generator=torch.Generator(device=dev).manual_seed(cfg.seed)).to(torch.bfloat16)
+    dx = torch.empty((M, K), dtype=torch.float32, device=dev)
+    ws_dx = sq.workspace(sq.SQ_OP_LINEAR_BWD_DX, M, N, K, dev)
     c4 = torch.empty_like(w4.codes)
     s4, f4 = torch.empty_like(w4.scales), torch.empty_like(w4.frac_idx)
     s6, f6 = torch.empty_like(w6.scales), torch.empty_like(w6.frac_idx)
@@ -172,6 +181,9 @@ def main():
         "recon_int4_g64": lambda: sq.sq_reconstruct_bf16(w6, W),
         "recon_nvfp4_resid": lambda: sq.sq_reconstruct_bf16(wn, W, RES),
         "recon_int4_resid": lambda: sq.sq_reconstruct_bf16(w4, W, RES),
+        "recon_nvfp4_t": lambda: sq.sq_reconstruct_bf16(wn, Wt, sq.SQ_RECON_TRANSPOSED),
+        "bwd_dx_nvfp4": lambda: sq.sq_linear_bwd_dx(wn, dy, dx, ws_dx),
+        "gemm_bwd_dx": lambda: sq.sq_linear_bwd_dx(wn, dy, dx, ws_dx),
         "gemm_nvfp4": lambda: sq.sq_linear_fwd(wn, x, y, g_x=gx, ws=ws_n),
         "gemm_int4": lambda: sq.sq_linear_fwd(w4, x, y, ws=ws_i),
     }

@@ -78,12 +78,14 @@ typedef enum {
     SQ_OP_LINEAR_FWD_INT4 = 5,
     SQ_OP_RECONSTRUCT = 6,
     SQ_OP_LINEAR_FWD_INT8 = 7,
-    SQ_OP_BUILD_INT8 = 8
+    SQ_OP_BUILD_INT8 = 8,
+    SQ_OP_LINEAR_BWD_DX = 9
 } sq_op;
 
 /* flags */
 #define SQ_ACT_STATIC_SCALE    0x1u  /* sq_act_quant_nvfp4 / sq_linear_fwd: *g_x is an input */
 #define SQ_RECON_RESIDUAL_ONLY 0x2u  /* sq_reconstruct_bf16: drop the low-rank term        */
+#define SQ_RECON_TRANSPOSED    0x4u  /* sq_reconstruct_bf16: write W^T [K, N] instead of W  */
 
 /*
  * A built weight.  All pointers are device pointers owned by the caller.
@@ -272,16 +274,31 @@ SQ_API sq_status sq_linear_fwd_noalloc(const sq_weight *w, const uint16_t *x, in
  *       (32; 16 for SQ_FMT_INT8_ROW),
  *   W[n, k] = bf16(RN(L + h))          (bf16(h) with SQ_RECON_RESIDUAL_ONLY
  *                                       or NULL low-rank pointers).
- * W_out: [N, K] bf16 (device).
+ * W_out: [N, K] bf16 (device), or with SQ_RECON_TRANSPOSED the same values as
+ * W^T [K, N] (the layout the backward GEMM reads).
  */
 SQ_API sq_status sq_reconstruct_bf16(const sq_weight *w, uint16_t *W_out, uint32_t flags,
                               void *stream);
 
 /*
+ * Backward of the layer's input: dx = dy W, dy [M, N] bf16 (device), dx [M, K]
+ * fp32 (device), W the bf16 reconstruct of the weight (low-rank term
+ * included when the weight has one).  The SquareQ README runs the backward as
+ * "the bwd-side bf16 reconstruct from the same payload" followed by the normal
+ * bf16 GEMM ("End-to-end" paragraph); here the reconstruct writes W^T into
+ * the workspace and the library's bf16 tensor-core GEMM (fp32 accumulation in
+ * tensor memory) reduces over N.  Accuracy: max|dx - dx_exact| /
+ * max|dx_exact| <= 2e-3 against dy W on the same bf16 operands.  ws:
+ * sq_workspace_bytes(SQ_OP_LINEAR_BWD_DX, M, N, K) bytes (holds W^T).
+ */
+SQ_API sq_status sq_linear_bwd_dx(const sq_weight *w, const uint16_t *dy, int64_t M, float *dx, void *ws,
+                                  size_t ws_bytes, void *stream);
+
+/*
  * Optional instrumentation for timing the tensor-core GEMM on its own: when
- * both handles are non-NULL, every later sq_linear_fwd call made by this host
- * thread records start_event immediately before and stop_event immediately
- * after its GEMM launch, on the call's stream.  The handles are cudaEvent_t
+ * both handles are non-NULL, every later sq_linear_fwd or sq_linear_bwd_dx call
+ * made by this host thread records start_event immediately before and
+ * stop_event immediately after its GEMM launch, on the call's stream.  The handles are cudaEvent_t
  * values passed as void*, created and owned by the caller; (NULL, NULL) turns
  * recording off.  No work is added or skipped.
  */

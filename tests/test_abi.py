@@ -126,11 +126,24 @@ def test_linear_fwd_validation():
     assert fwd(_w(), fl=0x40) == SQ_ERR_ARG
 
 
+def test_bwd_dx_validation():
+    L = sq.lib()
+    big = 1 << 34
+    bwd = lambda w, dy=A, M=8, dx=A, ws=A, wsb=big: L.sq_linear_bwd_dx(ctypes.byref(w), dy, M, dx, ws, wsb, None)
+    assert bwd(_w(), dy=None) == SQ_ERR_NULL
+    assert bwd(_w(), M=0) == SQ_ERR_SHAPE
+    assert bwd(_w(N=200)) == SQ_ERR_SHAPE
+    assert bwd(_w(), dx=MIS) == SQ_ERR_ALIGN
+    assert bwd(_w(), wsb=1000) == SQ_ERR_WORKSPACE
+    assert sq.sq_workspace_bytes(sq.SQ_OP_LINEAR_BWD_DX, 8, 256, 512) >= 256 * 512 * 2
+
+
 def test_reconstruct_validation():
     L = sq.lib()
     assert L.sq_reconstruct_bf16(ctypes.byref(_w()), None, 0, None) == SQ_ERR_NULL
     assert L.sq_reconstruct_bf16(ctypes.byref(_w()), MIS, 0, None) == SQ_ERR_ALIGN
     assert L.sq_reconstruct_bf16(ctypes.byref(_w()), A, 0x10, None) == SQ_ERR_ARG
+    assert L.sq_reconstruct_bf16(ctypes.byref(_w()), A, 0x8, None) == SQ_ERR_ARG
     assert L.sq_reconstruct_bf16(ctypes.byref(_w(U=MIS)), A, 0, None) == SQ_ERR_ALIGN
 
 
