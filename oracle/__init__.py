@@ -74,6 +74,8 @@ _SIGS = {
     "or_linear_fwd_int8": ([_P, _P, _P, _P, _P, _I64, _I64, _I64, _P, _I64, _P], None),
     "or_lowrank_input": ([_P, _I64, _I64, _P, ctypes.c_int, _P], None),
     "or_linear_bwd_dx": ([_P, _P, _I64, _I64, _I64, _P, _I64, _P], None),
+    "or_svd_residual": ([_P, _P, _P, _I64, _I64, _P], None),
+    "or_f32_to_bf16_n": ([_P, _I64, _P], None),
 }
 
 
@@ -373,3 +375,32 @@ def linear_bwd_dx(dy_bits, W_bits, rows=None):
     dx = np.empty((len(rows), K), np.float64)
     lib().or_linear_bwd_dx(_p(dy), _p(W), M, N, K, _p(rows), len(rows), _p(dx))
     return dx
+
+
+# ---- SVD init of the low-rank branch ("Low-rank branch: rank-32 SVD of the weight") ----
+
+def svd_residual(W, up_bits, down_bits):
+    """R = RN(W - L), L the rank-32 fmaf chain of bf16 up [N, 32] and down [K, 32] (as the reconstruct)."""
+    W = _c(W, np.float32)
+    N, K = W.shape
+    R = np.empty((N, K), np.float32)
+    lib().or_svd_residual(_p(W), _p(_c(up_bits, np.uint16)), _p(_c(down_bits, np.uint16)), N, K, _p(R))
+    return R
+
+
+def svd_init(W, rank=32):
+    """Truncated SVD of W [N, K] (fp64 LAPACK through numpy: a library step) ->
+    (lora_up bf16 bits [N, rank], lora_down bf16 bits [K, rank], R fp32 [N, K], sigma fp64 [rank]).
+    The singular values are split evenly: up = U sqrt(sigma), down = V sqrt(sigma), each rounded
+    to bf16 once (round to nearest even); R = RN(W - L) with the fmaf chain of svd_residual."""
+    W = _c(W, np.float32)
+    U, S, Vt = np.linalg.svd(W.astype(np.float64), full_matrices=False)
+    sq = np.sqrt(S[:rank])
+    up = (U[:, :rank] * sq).astype(np.float32)
+    down = (Vt[:rank].T * sq).astype(np.float32)
+    up_b = np.empty(up.shape, np.uint16)
+    down_b = np.empty(down.shape, np.uint16)
+    for src, dst in ((up, up_b), (down, down_b)):
+        src = np.ascontiguousarray(src)
+        lib().or_f32_to_bf16_n(_p(src), src.size, _p(dst))
+    return up_b, down_b, svd_residual(W, up_b, down_b), S[:rank]

@@ -111,6 +111,13 @@ float or_bf16_to_f32(uint16_t h)
     return v;
 }
 
+/* bf16 of n values (the routine above, element by element) */
+void or_f32_to_bf16_n(const float *v, int64_t n, uint16_t *out)
+{
+    for (int64_t i = 0; i < n; i++)
+        out[i] = or_f32_to_bf16(v[i]);
+}
+
 /* IEEE binary16: 10 fraction bits, emin = -14, largest finite 65504. */
 uint16_t or_f32_to_f16(float v)
 {
@@ -1004,5 +1011,29 @@ void or_linear_bwd_dx(const uint16_t *dy, const uint16_t *W, int64_t M, int64_t 
         }
         memcpy(dx + i * K, acc, (size_t)K * sizeof(double));
         free(acc);
+    }
+}
+
+/* ------------------------------------------------------------------------ */
+/* SVD init: residual of the rank-32 branch                                 */
+/* ------------------------------------------------------------------------ */
+
+/*
+ * R[n, k] = RN(W[n, k] - L[n, k]) with L the rank-32 fmaf chain over r = 0..31
+ * of up[n, r] * down[k, r] from 0 -- the same L the bf16 reconstruct adds back
+ * (SquareQ README, "Low-rank branch: rank-32 SVD of the weight": the residual
+ * is the weight minus the low-rank branch).  W, R fp32 [N, K]; up [N, 32],
+ * down [K, 32] bf16 bits.
+ */
+void or_svd_residual(const float *W, const uint16_t *up, const uint16_t *down, int64_t N, int64_t K, float *R)
+{
+#pragma omp parallel for schedule(static)
+    for (int64_t n = 0; n < N; n++) {
+        for (int64_t k = 0; k < K; k++) {
+            float L = 0.0f;
+            for (int r = 0; r < 32; r++)
+                L = fmaf(or_bf16_to_f32(up[n * 32 + r]), or_bf16_to_f32(down[k * 32 + r]), L);
+            R[n * K + k] = W[n * K + k] - L;
+        }
     }
 }
