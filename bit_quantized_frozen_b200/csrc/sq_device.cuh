@@ -335,6 +335,38 @@ __device__ __forceinline__ uint32_t f32_to_bf16_bits(float v)
     return (uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(v));
 }
 
+// bf16(lo) | bf16(hi) << 16, both round to nearest even, in one conversion
+// instruction (cvt.rn.bf16x2.f32 puts its first source in the upper half)
+__device__ __forceinline__ uint32_t f32x2_to_bf16x2_bits(float lo, float hi)
+{
+    uint32_t r;
+    asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
+    return r;
+}
+
+// Integer codes to exact floats without the int-to-float conversion unit:
+// 2^23 + u (0 <= u < 2^23) is the float whose bit pattern is 0x4B000000 | u,
+// so a small integer is recovered by one exact subtraction.
+//   int4 (4-bit two's complement nibble n):  q = (n ^ 8) - 8
+//   int8 (byte b, two's complement):         q = (b ^ 0x80) - 128
+// v[i] = q of nibble i of w (nibble 0 = low bits)
+__device__ __forceinline__ void int4x8_to_f32(uint32_t w, float (&v)[8])
+{
+    const uint32_t x = w ^ 0x88888888u;
+#pragma unroll
+    for (int i = 0; i < 8; ++i)
+        v[i] = __fsub_rn(__uint_as_float(0x4B000000u | ((x >> (4 * i)) & 0xFu)), 8388616.0f);
+}
+
+// v[i] = q of byte i of w (byte 0 = low bits)
+__device__ __forceinline__ void int8x4_to_f32(uint32_t w, float (&v)[4])
+{
+    const uint32_t x = w ^ 0x80808080u;
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+        v[i] = __fsub_rn(__uint_as_float(__byte_perm(x, 0x4B000000u, 0x7650u + i)), 8388736.0f);
+}
+
 // tiled scale-factor byte offset, C = K/16 scale columns
 __device__ __forceinline__ int64_t sf_offset(int64_t r, int64_t c, int64_t C)
 {

@@ -580,10 +580,11 @@ __global__ void __launch_bounds__(256) dequant_int8_kernel(const uint4 *__restri
         const uint32_t w[4] = {c.x, c.y, c.z, c.w};
         uint32_t o[8];
 #pragma unroll
-        for (int p = 0; p < 8; ++p) {
-            const int q0 = (int)(int8_t)((w[p >> 1] >> (16 * (p & 1))) & 0xFFu);
-            const int q1 = (int)(int8_t)((w[p >> 1] >> (16 * (p & 1) + 8)) & 0xFFu);
-            o[p] = f32_to_bf16_bits(__fmul_rn((float)q0, s)) | (f32_to_bf16_bits(__fmul_rn((float)q1, s)) << 16);
+        for (int j = 0; j < 4; ++j) {
+            float q[4];
+            int8x4_to_f32(w[j], q);
+            o[2 * j] = f32x2_to_bf16x2_bits(__fmul_rn(q[0], s), __fmul_rn(q[1], s));
+            o[2 * j + 1] = f32x2_to_bf16x2_bits(__fmul_rn(q[2], s), __fmul_rn(q[3], s));
         }
         wb[2 * i] = make_uint4(o[0], o[1], o[2], o[3]);
         wb[2 * i + 1] = make_uint4(o[4], o[5], o[6], o[7]);
@@ -620,7 +621,7 @@ __global__ void __launch_bounds__(kStreamThreads) rotate_bf16_kernel(const __gri
             uint32_t w[4];
 #pragma unroll
             for (int j = 0; j < 4; ++j)
-                w[j] = f32_to_bf16_bits(v[8 * i + 2 * j]) | (f32_to_bf16_bits(v[8 * i + 2 * j + 1]) << 16);
+                w[j] = f32x2_to_bf16x2_bits(v[8 * i + 2 * j], v[8 * i + 2 * j + 1]);
             o[i] = make_uint4(w[0], w[1], w[2], w[3]);
         }
     });
@@ -639,15 +640,12 @@ __global__ void __launch_bounds__(256) dequant_int4_kernel(const uint32_t *__res
          i += (int64_t)gridDim.x * blockDim.x) {
         const uint32_t c = __ldg(codes + i);
         const float s = __half2float(__ushort_as_half(__ldg(scales + (i >> kWordsLog2))));
+        float q[8];
+        int4x8_to_f32(c, q);
         uint32_t o[4];
 #pragma unroll
-        for (int p = 0; p < 4; ++p) {
-            int q0 = (int)((c >> (8 * p)) & 0xFu);
-            int q1 = (int)((c >> (8 * p + 4)) & 0xFu);
-            q0 = q0 >= 8 ? q0 - 16 : q0;
-            q1 = q1 >= 8 ? q1 - 16 : q1;
-            o[p] = f32_to_bf16_bits(__fmul_rn((float)q0, s)) | (f32_to_bf16_bits(__fmul_rn((float)q1, s)) << 16);
-        }
+        for (int p = 0; p < 4; ++p)
+            o[p] = f32x2_to_bf16x2_bits(__fmul_rn(q[2 * p], s), __fmul_rn(q[2 * p + 1], s));
         wb[i] = make_uint4(o[0], o[1], o[2], o[3]);
     }
 }
@@ -1092,9 +1090,12 @@ __device__ __forceinline__ void rec_decode(const uint8_t *stage, int r, int q, f
         const uint4 c1 = *reinterpret_cast<const uint4 *>(stage + r * Cfg::kCodeRow + 32 * q + 16);
         const uint32_t w[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
 #pragma unroll
-        for (int i = 0; i < 32; ++i) {
-            const int qi = (int)(int8_t)((w[i >> 2] >> (8 * (i & 3))) & 0xFFu);
-            v[i] = __fmul_rn((float)qi, s);
+        for (int j = 0; j < 8; ++j) {
+            float q[4];
+            int8x4_to_f32(w[j], q);
+#pragma unroll
+            for (int t = 0; t < 4; ++t)
+                v[4 * j + t] = __fmul_rn(q[t], s);
         }
         return;
     }
@@ -1103,10 +1104,12 @@ __device__ __forceinline__ void rec_decode(const uint8_t *stage, int r, int q, f
     if (FMT == 1 || FMT == 3) {
         const float s = __half2float(*reinterpret_cast<const __half *>(sc + 2 * (FMT == 3 ? q >> 1 : q)));
 #pragma unroll
-        for (int i = 0; i < 32; ++i) {
-            int qq = (int)((w[i >> 3] >> (4 * (i & 7))) & 0xFu);
-            qq = qq >= 8 ? qq - 16 : qq;
-            v[i] = __fmul_rn((float)qq, s);
+        for (int j = 0; j < 4; ++j) {
+            float q[8];
+            int4x8_to_f32(w[j], q);
+#pragma unroll
+            for (int t = 0; t < 8; ++t)
+                v[8 * j + t] = __fmul_rn(q[t], s);
         }
     } else {
         const uint32_t sf2 = *reinterpret_cast<const uint16_t *>(sc + 2 * q);
@@ -1186,8 +1189,7 @@ __global__ void __launch_bounds__(256, (LOWRANK || TRANS) ? 2 : 3) reconstruct_k
                         uint32_t ww[4];
 #pragma unroll
                         for (int j = 0; j < 4; ++j)
-                            ww[j] = f32_to_bf16_bits(v[8 * k + 2 * j]) |
-                                    (f32_to_bf16_bits(v[8 * k + 2 * j + 1]) << 16);
+                            ww[j] = f32x2_to_bf16x2_bits(v[8 * k + 2 * j], v[8 * k + 2 * j + 1]);
                         o[k] = make_uint4(ww[0], ww[1], ww[2], ww[3]);
                     }
                 }
@@ -1258,14 +1260,15 @@ __global__ void __launch_bounds__(256, (LOWRANK || TRANS) ? 2 : 3) reconstruct_k
                 float L0, L1;
                 unpack2(acc[j], L0, L1);
                 // with the low-rank term W = bf16(RN(L + h)); residual only: bf16(h)
-                const uint32_t b0 = f32_to_bf16_bits(LOWRANK ? __fadd_rn(L0, hv.x) : hv.x);
-                const uint32_t b1 = f32_to_bf16_bits(LOWRANK ? __fadd_rn(L1, hv.y) : hv.y);
+                const float o0 = LOWRANK ? __fadd_rn(L0, hv.x) : hv.x;
+                const float o1 = LOWRANK ? __fadd_rn(L1, hv.y) : hv.y;
                 if (TRANS) {
+                    const uint32_t b0 = f32_to_bf16_bits(o0), b1 = f32_to_bf16_bits(o1);
                     const int slot = (r - rbase) >> 1, hi = (r - rbase) & 1;
                     tw0[slot] = hi ? (tw0[slot] | (b0 << 16)) : b0;
                     tw1[slot] = hi ? (tw1[slot] | (b1 << 16)) : b1;
                 } else if (n < N) {
-                    *reinterpret_cast<uint32_t *>(W + n * K + k0) = b0 | (b1 << 16);
+                    *reinterpret_cast<uint32_t *>(W + n * K + k0) = f32x2_to_bf16x2_bits(o0, o1);
                 }
             }
         }
