@@ -46,6 +46,7 @@ EXPORTED = [
     "sq_build_int4", "sq_build_int8", "sq_build_nvfp4", "sq_act_quant_nvfp4", "sq_linear_fwd",
     "sq_reconstruct_bf16",
     "sq_check_device_status", "sq_set_gemm_events", "sq_linear_fwd_noalloc", "sq_linear_bwd_dx",
+    "sq_selftest_wait_timeout",
 ]
 
 
@@ -91,6 +92,7 @@ _SIGS = {
     "sq_reconstruct_bf16": ([ctypes.POINTER(sq_weight), _P, ctypes.c_uint32, _P], ctypes.c_int),
     "sq_linear_bwd_dx": ([ctypes.POINTER(sq_weight), _P, _I64, _P, _P, ctypes.c_size_t, _P], ctypes.c_int),
     "sq_check_device_status": ([_P, _P], ctypes.c_int),
+    "sq_selftest_wait_timeout": ([_P, ctypes.c_uint32, _P], ctypes.c_int),
     "sq_set_gemm_events": ([_P, _P], ctypes.c_int),
 }
 _lib = None
@@ -212,6 +214,10 @@ def sq_linear_bwd_dx(w: "Weight", dy, dx, ws, stream=None):
     cw = w.as_c()
     _check("sq_linear_bwd_dx", lib().sq_linear_bwd_dx(ctypes.byref(cw), _ptr(dy), M, _ptr(dx), _ptr(ws),
                                                       _numel_bytes(ws), _stream(stream)))
+
+
+def sq_selftest_wait_timeout(ws, limit_us: int = 20000, stream=None):
+    _check("sq_selftest_wait_timeout", lib().sq_selftest_wait_timeout(_ptr(ws), int(limit_us), _stream(stream)))
 
 
 def sq_check_device_status(ws, stream=None):

@@ -10,8 +10,26 @@
 
 #include "sq.h"
 #include "sq_kernels.h"
+#include "sq_ptx.cuh"
 
 static __device__ __align__(256) uint8_t g_noalloc_scratch[size_t(32) << 20];
+
+// One thread waits on an mbarrier that nothing ever arrives on, with the
+// bounded wait every kernel of the library uses; it must give up after
+// limit_ns, set the status word and return.
+static __global__ void selftest_wait_kernel(uint32_t *status, unsigned long long limit_ns)
+{
+    __shared__ __align__(8) uint64_t bar;
+    __shared__ uint32_t abort_flag;
+    if (threadIdx.x == 0) {
+        sq::mbar_init(sq::smem_u32(&bar), 1);
+        abort_flag = 0u;
+        sq::fence_mbar_init();
+    }
+    __syncthreads();
+    if (threadIdx.x == 0)
+        (void)sq::mbar_wait(sq::smem_u32(&bar), 0u, &abort_flag, status, limit_ns);
+}
 
 namespace {
 
@@ -535,6 +553,26 @@ sq_status sq_set_gemm_events(void *start_event, void *stop_event)
         return SQ_ERR_NULL;
     g_gemm_ev0 = reinterpret_cast<cudaEvent_t>(start_event);
     g_gemm_ev1 = reinterpret_cast<cudaEvent_t>(stop_event);
+    return SQ_OK;
+}
+
+sq_status sq_selftest_wait_timeout(void *ws, uint32_t limit_us, void *stream)
+{
+    if (!ws)
+        return SQ_ERR_NULL;
+    if (!aligned(ws, 256))
+        return SQ_ERR_ALIGN;
+    if (limit_us < 1 || limit_us > 1000000)
+        return SQ_ERR_ARG;
+    int sms = 0;
+    sq_status st = check_device(&sms);
+    if (st != SQ_OK)
+        return st;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    uint32_t *status = reinterpret_cast<uint32_t *>(ws);
+    SQ_CUDA(cudaMemsetAsync(status, 0, 4, s), "memset");
+    selftest_wait_kernel<<<1, 32, 0, s>>>(status, 1000ull * limit_us);
+    SQ_CUDA(cudaGetLastError(), "self-test launch");
     return SQ_OK;
 }
 

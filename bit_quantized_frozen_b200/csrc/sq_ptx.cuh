@@ -55,9 +55,10 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity)
 }
 
 // Wait for the phase with the given parity to complete.  Gives up after
-// kWaitLimitNs, or as soon as another role of the CTA has given up.
+// limit_ns (kWaitLimitNs by default), or as soon as another role of the CTA
+// has given up.
 __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile uint32_t *abort_flag,
-                                          uint32_t *status)
+                                          uint32_t *status, unsigned long long limit_ns = kWaitLimitNs)
 {
     if (mbar_try_wait(bar, parity))
         return true;
@@ -68,7 +69,7 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatil
         if ((it & 255u) == 0) {
             if (*abort_flag)
                 return false;
-            if (global_ns() - t0 > kWaitLimitNs) {
+            if (global_ns() - t0 > limit_ns) {
                 *abort_flag = 1u;
                 if (status)
                     atomicOr(status, 1u);

@@ -312,6 +312,18 @@ SQ_API sq_status sq_set_gemm_events(void *start_event, void *stop_event);
  */
 SQ_API sq_status sq_check_device_status(void *ws, void *stream);
 
+/*
+ * Self-test of the failure detection every kernel relies on: all waits in the
+ * library are bounded; a kernel that gives up a wait sets the status word of
+ * its workspace and returns (no trap), and sq_check_device_status reports
+ * SQ_ERR_TIMEOUT.  This call launches one kernel whose wait can never be
+ * satisfied, with a limit of limit_us microseconds (1 .. 1000000), on `stream`:
+ * afterwards sq_check_device_status(ws, stream) must return SQ_ERR_TIMEOUT and
+ * the context stays usable.  ws: at least 256 bytes of device memory (only
+ * the status word is written).
+ */
+SQ_API sq_status sq_selftest_wait_timeout(void *ws, uint32_t limit_us, void *stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -159,6 +159,14 @@ def test_valid_call_without_device_reports_device_error():
     assert sq.lib().sq_reconstruct_bf16(ctypes.byref(_w()), A, 0, None) == SQ_ERR_DEVICE
 
 
+def test_selftest_validation():
+    L = sq.lib()
+    assert L.sq_selftest_wait_timeout(None, 100, None) == SQ_ERR_NULL
+    assert L.sq_selftest_wait_timeout(MIS, 100, None) == SQ_ERR_ALIGN
+    assert L.sq_selftest_wait_timeout(A, 0, None) == SQ_ERR_ARG
+    assert L.sq_selftest_wait_timeout(A, 2000000, None) == SQ_ERR_ARG
+
+
 def test_binding_raises_with_status():
     with pytest.raises(sq.SqError) as e:
         sq._check("sq_build_int4", SQ_ERR_SHAPE)
