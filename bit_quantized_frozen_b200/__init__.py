@@ -39,6 +39,7 @@ SQ_ACT_STATIC_SCALE = 0x1
 SQ_RECON_RESIDUAL_ONLY = 0x2
 SQ_RECON_TRANSPOSED = 0x4
 SQ_OP_LINEAR_BWD_DX = 9
+SQ_OP_SVD_INIT = 10
 RANK = 32
 
 EXPORTED = [
@@ -46,7 +47,7 @@ EXPORTED = [
     "sq_build_int4", "sq_build_int8", "sq_build_nvfp4", "sq_act_quant_nvfp4", "sq_linear_fwd",
     "sq_reconstruct_bf16",
     "sq_check_device_status", "sq_set_gemm_events", "sq_linear_fwd_noalloc", "sq_linear_bwd_dx",
-    "sq_selftest_wait_timeout",
+    "sq_selftest_wait_timeout", "sq_svd_init",
 ]
 
 
@@ -82,6 +83,7 @@ _SIGS = {
     "sq_workspace_bytes": ([ctypes.c_int, _I64, _I64, _I64], ctypes.c_size_t),
     "sq_build_int4": ([_P, _I64, _I64, ctypes.c_int32, _P, _P, _P, _P], ctypes.c_int),
     "sq_build_int8": ([_P, _I64, _I64, _P, _P, _P, _P], ctypes.c_int),
+    "sq_svd_init": ([_P, _I64, _I64, _P, ctypes.c_int32, _P, _P, _P, _P, ctypes.c_size_t, _P], ctypes.c_int),
     "sq_build_nvfp4": ([_P, _I64, _I64, _P, _P, _P, _P, ctypes.c_size_t, _P], ctypes.c_int),
     "sq_act_quant_nvfp4": ([_P, _I64, _I64, _P, _P, _P, _P, _P, ctypes.c_uint32, _P, ctypes.c_size_t, _P],
                            ctypes.c_int),
@@ -165,6 +167,12 @@ def sq_build_int4(R, codes, scales, frac_idx=None, group: int = 32, stream=None)
     N, K = R.shape
     _check("sq_build_int4", lib().sq_build_int4(_ptr(R), N, K, group, _ptr(codes), _ptr(scales), _ptr(frac_idx),
                                                 _stream(stream)))
+
+
+def sq_svd_init(W, omega, iters, lora_up, lora_down, R, ws, stream=None):
+    N, K = W.shape
+    _check("sq_svd_init", lib().sq_svd_init(_ptr(W), N, K, _ptr(omega), int(iters), _ptr(lora_up), _ptr(lora_down),
+                                            _ptr(R), _ptr(ws), _numel_bytes(ws), _stream(stream)))
 
 
 def sq_build_int8(R, codes, scales, frac_idx=None, stream=None):
@@ -291,6 +299,18 @@ def build_nvfp4(R: torch.Tensor, lora_up=None, lora_down=None, ws=None, stream=N
     ws = ws if ws is not None else workspace(SQ_OP_BUILD_NVFP4, 0, N, K, dev)
     sq_build_nvfp4(R, codes, sf, g, ws, stream=stream)
     return Weight(SQ_FMT_NVFP4, N, K, codes, sf, g, lora_up, lora_down)
+
+
+def svd_init(W: torch.Tensor, omega: torch.Tensor, iters: int = 8, stream=None):
+    """(lora_up bf16 [N, 32], lora_down bf16 [K, 32], R fp32 [N, K]) of W [N, K] fp32."""
+    N, K = W.shape
+    dev = W.device
+    up = torch.empty((N, RANK), dtype=torch.bfloat16, device=dev)
+    down = torch.empty((K, RANK), dtype=torch.bfloat16, device=dev)
+    R = torch.empty((N, K), dtype=torch.float32, device=dev)
+    ws = workspace(SQ_OP_SVD_INIT, 0, N, K, dev)
+    sq_svd_init(W, omega, iters, up, down, R, ws, stream=stream)
+    return up, down, R
 
 
 def linear_fwd(w: Weight, x: torch.Tensor, ws=None, g_x=None, flags: int = 0, stream=None) -> torch.Tensor:

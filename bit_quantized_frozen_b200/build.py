@@ -10,7 +10,7 @@ ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(PKG, "libsq.so")
-SOURCES = ["sq_api.cu", "sq_quant.cu", "sq_gemm.cu"]
+SOURCES = ["sq_api.cu", "sq_quant.cu", "sq_gemm.cu", "sq_svd.cu"]
 HEADERS = ["sq_device.cuh", "sq_ptx.cuh", "sq_kernels.h"]
 
 NVCC_FLAGS = [

@@ -234,6 +234,8 @@ size_t sq_workspace_bytes(int op, int64_t M, int64_t N, int64_t K)
         return kHeader;
     case SQ_OP_LINEAR_BWD_DX:
         return kAlign + round_up((size_t)N * (size_t)K * 2, kAlign);
+    case SQ_OP_SVD_INIT:
+        return sq::svd_workspace_bytes(N, K);
     default:
         return 0;
     }
@@ -272,6 +274,34 @@ sq_status sq_build_int8(const float *R, int64_t N, int64_t K, int8_t *codes, flo
         return st;
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     SQ_CUDA(sq::launch_int8_build(R, N, K, codes, scales, frac_idx, sms, s), "int8 build");
+    return SQ_OK;
+}
+
+sq_status sq_svd_init(const float *W, int64_t N, int64_t K, const float *omega, int32_t iters, uint16_t *lora_up,
+                      uint16_t *lora_down, float *R, void *ws, size_t ws_bytes, void *stream)
+{
+    if (!W || !omega || !lora_up || !lora_down || !R || !ws)
+        return SQ_ERR_NULL;
+    if (!shape_ok_nk(N, K))
+        return SQ_ERR_SHAPE;
+    if (iters < 1 || iters > 100)
+        return SQ_ERR_ARG;
+    if (!aligned(W, 16) || !aligned(omega, 16) || !aligned(lora_up, 16) || !aligned(lora_down, 16) ||
+        !aligned(R, 16) || !aligned(ws, 256))
+        return SQ_ERR_ALIGN;
+    if (ws_bytes < sq_workspace_bytes(SQ_OP_SVD_INIT, 0, N, K))
+        return SQ_ERR_WORKSPACE;
+    int sms = 0;
+    sq_status st = check_device(&sms);
+    if (st != SQ_OK)
+        return st;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    const char *stage = "svd init";
+    const cudaError_t e = sq::launch_svd_init(W, N, K, omega, iters, lora_up, lora_down, R, ws, sms, s, &stage);
+    if (e != cudaSuccess) {
+        set_detail(stage, e);
+        return SQ_ERR_CUDA;
+    }
     return SQ_OK;
 }
 

@@ -1,0 +1,138 @@
+"""SVD init of the rank-32 low-rank branch (SquareQ README, "Low-rank branch: rank-32
+SVD of the weight, always on, bf16") through the C ABI against the CPU oracle.
+
+The oracle takes the exact truncated SVD (fp64 LAPACK); the GPU runs subspace
+iteration from a seeded start block.  The test weights have a spectral gap at 32
+(sigma_32 / sigma_33 >= 3, checked), so the rank-32 product L = up down^T is unique
+and the iteration error, (sigma_33 / sigma_32)^(2 iters) <= 3^-16, is negligible.
+Compared:
+- L against the oracle's within ||dL||_F / ||L||_F <= 2 * 2^-9: each factor is rounded
+  to bf16 once (relative error <= 2^-9 per entry), which bounds the difference of two
+  correctly rounded factorisations of the same L to first order;
+- the residual bit for bit against the oracle's R = RN(W - L) on the GPU's own factors;
+- the residual's norm against the optimal one (Eckart-Young).
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import synth_inputs as si
+from sqcase import bits16, first_mismatch, host, to_dev
+
+pytestmark = pytest.mark.gpu
+
+L_TOL = 2 * 2.0 ** -9
+
+
+@pytest.fixture(scope="module")
+def sq():
+    import bit_quantized_frozen_b200 as m
+    assert torch.cuda.is_available(), "GPU tests need a CUDA device"
+    m.lib()
+    return m
+
+
+def gap_weight(N, K, seed):
+    """A rank-32 part with singular values 8 .. 2 (geometric) plus the synthetic residual of the
+    layer shape scaled to spectral norm 0.5: a gap of about 4 at index 32."""
+    rng = np.random.default_rng(seed)
+    A = rng.standard_normal((N, 32)) / np.sqrt(N)
+    B = rng.standard_normal((K, 32)) / np.sqrt(K)
+    s = np.geomspace(8.0, 2.0, 32)
+    noise = si.make_inputs(4, K, N, seed)["R"].astype(np.float64)
+    noise *= 0.5 / np.linalg.norm(noise, 2)
+    W = ((A * s) @ B.T + noise).astype(np.float32)
+    S = np.linalg.svd(W.astype(np.float64), compute_uv=False)
+    assert S[31] >= 3 * S[32], "test weight without a spectral gap"
+    return W
+
+
+def omega(K, seed):
+    return np.random.default_rng(seed).standard_normal((K, 32)).astype(np.float32)
+
+
+def run_gpu(sq, W, om, iters=8):
+    up, down, R = sq.svd_init(to_dev(W), to_dev(om), iters)
+    torch.cuda.synchronize()
+    return bits16(up), bits16(down), host(R)
+
+
+def lowrank_product(up, down):
+    return si.bf16_bits_to_f32(up).astype(np.float64) @ si.bf16_bits_to_f32(down).astype(np.float64).T
+
+
+def check_against_oracle(W, up, down, R, rows=None):
+    oup, odown, oR, S = oracle.svd_init(W)
+    L, Lo = lowrank_product(up, down), lowrank_product(oup, odown)
+    err = np.linalg.norm(L - Lo) / np.linalg.norm(Lo)
+    assert err <= L_TOL, f"low-rank product differs by {err:.3e}"
+    sel = slice(None) if rows is None else rows
+    Rw = oracle.svd_residual(W[sel], up[sel], down)
+    assert np.array_equal(R[sel].view(np.uint32), Rw.view(np.uint32)), first_mismatch(R[sel], Rw)
+    assert np.linalg.norm(R) <= np.linalg.norm(oR) * (1 + 1e-2)
+
+
+@pytest.mark.parametrize("shape", [(256, 512), (384, 768), (1024, 256)])
+def test_svd_init_matches_truncated_svd(sq, shape):
+    N, K = shape
+    W = gap_weight(N, K, 100 + N)
+    up, down, R = run_gpu(sq, W, omega(K, 7))
+    check_against_oracle(W, up, down, R)
+
+
+def test_svd_init_singular_values_split_evenly(sq):
+    """up and down carry sigma^(1/2) each: column norms of the factors against the oracle's."""
+    W = gap_weight(256, 512, 110)
+    up, down, _ = run_gpu(sq, W, omega(512, 11))
+    oup, odown, _, S = oracle.svd_init(W)
+    for f, o in ((up, oup), (down, odown)):
+        n = np.linalg.norm(si.bf16_bits_to_f32(f).astype(np.float64), axis=0)
+        no = np.linalg.norm(si.bf16_bits_to_f32(o).astype(np.float64), axis=0)
+        assert np.allclose(n, no, rtol=4e-3)
+        assert np.allclose(n, np.sqrt(S), rtol=4e-3)
+
+
+def test_svd_init_is_deterministic_and_exact_rank(sq):
+    rng = np.random.default_rng(101)
+    W = (rng.standard_normal((256, 32)) @ rng.standard_normal((512, 32)).T / 8).astype(np.float32)
+    a = run_gpu(sq, W, omega(512, 8))
+    b = run_gpu(sq, W, omega(512, 8))
+    for x, y in zip(a, b):
+        assert np.array_equal(x.view(np.uint8), y.view(np.uint8))
+    up, down, R = a
+    assert np.linalg.norm(R) <= 2 * 2.0 ** -8 * np.linalg.norm(W)
+    Rw = oracle.svd_residual(W, up, down)
+    assert np.array_equal(R.view(np.uint32), Rw.view(np.uint32))
+
+
+def test_svd_init_zero_weight(sq):
+    W = np.zeros((128, 256), np.float32)
+    up, down, R = run_gpu(sq, W, omega(256, 9), iters=2)
+    assert not up.any() and not down.any() and not R.view(np.uint32).any()
+
+
+def test_svd_init_residual_in_place(sq):
+    """R may be the weight's own buffer."""
+    W = gap_weight(256, 512, 112)
+    Wd = to_dev(W)
+    up = torch.empty((256, 32), dtype=torch.bfloat16, device="cuda")
+    down = torch.empty((512, 32), dtype=torch.bfloat16, device="cuda")
+    ws = sq.workspace(sq.SQ_OP_SVD_INIT, 0, 256, 512)
+    sq.sq_svd_init(Wd, to_dev(omega(512, 12)), 8, up, down, Wd, ws)
+    torch.cuda.synchronize()
+    Rw = oracle.svd_residual(W, bits16(up), bits16(down))
+    assert np.array_equal(host(Wd).view(np.uint32), Rw.view(np.uint32))
+
+
+def test_svd_init_projection_shape(sq):
+    W = gap_weight(1536, 3072, 102)
+    up, down, R = run_gpu(sq, W, omega(3072, 10))
+    check_against_oracle(W, up, down, R, rows=np.array([0, 7, 777, 1535]))
+
+
+@pytest.mark.slow
+def test_svd_init_large(sq):
+    W = gap_weight(4096, 2048, 103)
+    up, down, R = run_gpu(sq, W, omega(2048, 13))
+    check_against_oracle(W, up, down, R, rows=np.array([0, 1, 2048, 4095]))
