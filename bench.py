@@ -6,8 +6,9 @@ chosen shape (default the headline 4480 x 16384 x 6144, M x N x K):
   sq_build_int4, sq_build_nvfp4, sq_linear_fwd (NVFP4, incl. the activation
   prologue), sq_linear_fwd (int4), sq_reconstruct_bf16 (both payloads), and the
   build, forward and reconstruct of the int4 group-64 variant and of the int8
-  per-row mode (rank-16 low-rank branch), and the input backward dx = dy W
-  (transposed bf16 reconstruct + bf16 GEMM) on the NVFP4 payload.
+  per-row mode (rank-16 low-rank branch), the input backward dx = dy W
+  (transposed bf16 reconstruct + bf16 GEMM) on the NVFP4 payload, and the
+  rank-32 SVD init of W = lora_up lora_down^T + R (sq_svd_init, 8 rounds).
 Every op is timed with CUDA events on the launching stream after an L2 flush
 (a 256 MB write outside the op's events); the NVFP4 forward is the headline
 metric (TFLOP/s = 2 M N K / time of the whole sq_linear_fwd call).  The GEMM
@@ -50,6 +51,9 @@ PAGES_FP4_TFLOPS = {"large_4480x16384x6144": 2 * 4480 * 16384 * 6144 / 1074e-6 /
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 FP4_PER_BF16 = 4.0        # nominal dense FP4 / BF16 tensor ratio (9 / 2.25 PFLOP/s)
 FLUSH_BYTES = 256 << 20   # > 126 MB L2
+# FP32 FMA issue roofline of the SVD init's products: 148 SMs x 128 FMA lanes x 2 flop x 1.965 GHz
+FP32_ALU_TFLOPS = 148 * 128 * 2 * 1.965e9 / 1e12
+SVD_ITERS = 8
 
 
 def parse():
@@ -94,6 +98,7 @@ def op_work(M, N, K):
         "fwd_int8": ("TFLOP/s", 2.0 * M * N * K),
         "reconstruct_int8": ("GB/s", NK * (1 + 2) + N * 4),
         "bwd_dx_nvfp4": ("TFLOP/s", 2.0 * M * N * K),
+        "svd_init": ("TFLOP/s", (4.0 * SVD_ITERS + 2.0) * NK * 32),   # fp32 FMA work (2 products/round + residual)
         "gemm_nvfp4": ("TFLOP/s", 2.0 * M * N * K),
         "gemm_int4": ("TFLOP/s", 2.0 * M * N * K),
         "gemm_bwd_dx": ("TFLOP/s", 2.0 * M * N * K),
@@ -106,6 +111,10 @@ LAUNCHES_PER_STEP = {   # our kernels per op (memsets excluded)
     "build_int4_g64": 1, "fwd_int4_g64": 5, "reconstruct_int4_g64": 1,
     "build_int8": 1, "fwd_int8": 7, "reconstruct_int8": 1,
     "bwd_dx_nvfp4": 2,
+    # start block orth (3) + per round: 2 products, 2 split sums, orth(U) and orth(V) of 3 kernels
+    # per pass (one pass each; the last round two for U and none for V) + Gram, Jacobi, factors,
+    # residual
+    "svd_init": 3 + 10 * SVD_ITERS + 4,
 }
 
 
@@ -262,9 +271,16 @@ def cpu_sample(d, M_s: int, N_s: int):
     t0 = time.perf_counter()
     oracle.reconstruct_bf16(oracle.FMT_INT8_ROW, c8, s8, 0.0, U16, D16, N_s, K)
     t["reconstruct_int8"] = time.perf_counter() - t0
+    n_svd = min(N_s, SVD_SAMPLE_ROWS)
+    Wsvd = (R[:n_svd].astype(np.float64) + si.bf16_bits_to_f32(U[:n_svd]).astype(np.float64)
+            @ si.bf16_bits_to_f32(D).astype(np.float64).T).astype(np.float32)
+    t0 = time.perf_counter()
+    oracle.svd_init(Wsvd)
+    t["svd_init"] = time.perf_counter() - t0
     return t, oracle.num_threads()
 
 
+SVD_SAMPLE_ROWS = 512      # the oracle's SVD init (fp64 LAPACK) runs on the first 512 rows of W
 REF_SAMPLE = (64, 2048)    # reference arm, per step: M_s rows of x, N_s rows of R (all K)
 CPU_SAMPLE = (128, 4096)   # one-off CPU baseline of the GPU arm
 
@@ -368,6 +384,12 @@ def run_sq(args, cfg, d, rank, world, local_rank):
     y_nv = torch.empty((M, N), dtype=torch.float32, device=dev)
     y_i4 = torch.empty((M, N), dtype=torch.float32, device=dev)
     W = torch.empty((N, K), dtype=torch.bfloat16, device=dev)
+    Wsvd = R + U.float() @ D.float().T            # the full weight the SVD init factors (input set-up)
+    omega = torch.randn((K, 32), device=dev, generator=torch.Generator(device=dev).manual_seed(cfg.seed + 1))
+    up_s = torch.empty((N, 32), dtype=torch.bfloat16, device=dev)
+    down_s = torch.empty((K, 32), dtype=torch.bfloat16, device=dev)
+    R_s = torch.empty_like(R)
+    ws_svd = sq.workspace(sq.SQ_OP_SVD_INIT, 0, N, K, dev)
     flush = torch.empty(FLUSH_BYTES // 4, dtype=torch.int32, device=dev)
 
     ops = [
@@ -384,6 +406,7 @@ def run_sq(args, cfg, d, rank, world, local_rank):
         ("fwd_int8", lambda: sq.sq_linear_fwd(i8, x, y_i4, ws=ws_i8)),
         ("reconstruct_int8", lambda: sq.sq_reconstruct_bf16(i8, W)),
         ("bwd_dx_nvfp4", lambda: sq.sq_linear_bwd_dx(nv, dy, dx, ws_dx)),
+        ("svd_init", lambda: sq.sq_svd_init(Wsvd, omega, SVD_ITERS, up_s, down_s, R_s, ws_svd)),
     ]
     names = [n for n, _ in ops]
     gemm_of = {"fwd_nvfp4": "gemm_nvfp4", "fwd_int4": "gemm_int4", "bwd_dx_nvfp4": "gemm_bwd_dx"}
@@ -507,11 +530,14 @@ def summarise(args, cfg, per_op, outer_ms, clocks, e2e, world, cpu):
         rate = amount / (ms * 1e-3) / (1e12 if unit == "TFLOP/s" else 1e9)
         if unit == "GB/s":
             frac, peak = rate / peaks["hbm_gbs"], "hbm"
+        elif k == "svd_init":
+            frac, peak = rate / FP32_ALU_TFLOPS, "fp32 FMA issue"
         else:
             fp4 = k in ("fwd_nvfp4", "gemm_nvfp4")      # the backward's GEMM runs in bf16
             peak_v = fp4_peak if fp4 else peaks["bf16_tflops"]
             frac, peak = rate / peak_v, "fp4 tensor" if fp4 else "bf16 tensor"
-        ops[k] = {"ms": ms, unit: rate, "frac": frac, "of": f"{peak} ({peak_src})"}
+        src = "148 SMs x 128 lanes x 2 flop x 1.965 GHz" if k == "svd_init" else peak_src
+        ops[k] = {"ms": ms, unit: rate, "frac": frac, "of": f"{peak} ({src})"}
     fwd_tflops = 2.0 * M * N * K / (per_op["fwd_nvfp4"] * 1e-3) / 1e12
     gemm_tflops = 2.0 * M * N * K / (per_op["gemm_nvfp4"] * 1e-3) / 1e12
     traffic, traffic_src = profiled_traffic(cfg.name)

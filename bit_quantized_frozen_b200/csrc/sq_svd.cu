@@ -13,7 +13,8 @@
 // With B = the last Z = W^T U, W ~ U B^T.  The Gram B^T B is factored R^T R (Cholesky) and a
 // one-sided Jacobi iteration on the columns of R gives the rotation X with R X = Q S (Q orthogonal,
 // S = the singular values of B), so that W ~ (U X) S (B X S^-1)^T and
-// up = U X S^(1/2), down = B X S^(-1/2).  orth(A) is CholeskyQR applied twice.
+// up = U X S^(1/2), down = B X S^(-1/2).  orth(A) is CholeskyQR: twice for the final U, once for
+// the blocks in between.
 //
 // Work split: the products with W (the only steps that touch [N, K]) and the Grams of the [rows, 32]
 // blocks are grids over all SMs; the 32 x 32 steps (Cholesky, triangular inverse, Jacobi) run in
@@ -31,62 +32,74 @@ namespace sq {
 constexpr int kSvdRank = 32;
 constexpr int kSvdTile = 128;          // rows of W (W V) or columns of W (W^T U) per CTA
 constexpr int kSvdChunk = 32;          // depth of one shared-memory stage of the products
-constexpr int kGramRows = 128;         // rows per partial Gram
+constexpr int kGramRows = 512;         // rows per partial Gram (the last one may be shorter)
+constexpr int kGramSub = 128;          // rows per shared-memory sub-tile of a partial Gram
 constexpr int kJacobiMaxSweeps = 30;
 constexpr double kJacobiSkip = 1e-15;  // pairs whose cosine is below this are left alone
 constexpr double kJacobiTol = 1e-13;   // a sweep whose largest cosine is below this ends the iteration
 constexpr unsigned kFull = 0xffffffffu;
-constexpr int kSvdTargetCtas = 512;    // product grids are split until they reach this many CTAs
+constexpr int kSvdTargetCtas = 1024;   // product grids are split until they reach this many CTAs
+constexpr int kSvdMaxSplits = 16;
 
 // ---------------------------------------------------------------------------
 // Yp[s, n, :] = sum over k in split s of W[n, k] V[k, :], for the 128 rows n of the CTA.
 // Grid (N / 128, S), 128 threads.  Warp w owns outputs 8w..8w+7; lane l rows l, l+32, l+64, l+96.
 // A stage holds 128 rows x 32 columns of W (row pitch 33 words: the 32 lanes' rows fall in 32
-// different banks) and the matching 32 rows of V (read as broadcasts).
+// different banks) and the matching 32 rows of V (read as 16-byte broadcasts).  The next stage is
+// loaded into registers while the current one is multiplied.
 // ---------------------------------------------------------------------------
 __global__ void __launch_bounds__(kSvdTile) svd_wv_kernel(const float *__restrict__ W, int64_t N, int64_t K,
                                                           int64_t k_per_split, const float *__restrict__ V,
                                                           float *__restrict__ Yp)
 {
     __shared__ float Ws[kSvdTile][kSvdChunk + 1];
-    __shared__ float Vs[kSvdChunk][kSvdRank];
+    __shared__ __align__(16) float Vs[kSvdChunk][kSvdRank];
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int64_t n0 = (int64_t)blockIdx.x * kSvdTile;
-    const int64_t kbeg = (int64_t)blockIdx.y * k_per_split;
+    const int64_t kbeg = (int64_t)blockIdx.y * k_per_split, kend = kbeg + k_per_split;
+    const float *wsrc = W + (n0 + warp) * K + lane;    // row warp + 4i, column lane of a stage
+    float wr[kSvdTile / 4], vr[kSvdChunk * kSvdRank / kSvdTile];
+    auto load = [&](int64_t k0) {
+#pragma unroll
+        for (int i = 0; i < kSvdTile / 4; ++i)
+            wr[i] = wsrc[(int64_t)(4 * i) * K + k0];
+#pragma unroll
+        for (int i = 0; i < kSvdChunk * kSvdRank / kSvdTile; ++i)
+            vr[i] = V[k0 * kSvdRank + tid + kSvdTile * i];
+    };
     float acc[4][8];
 #pragma unroll
     for (int j = 0; j < 4; ++j)
 #pragma unroll
         for (int o = 0; o < 8; ++o)
             acc[j][o] = 0.0f;
-    for (int64_t k0 = kbeg; k0 < kbeg + k_per_split; k0 += kSvdChunk) {
-#pragma unroll 8
-        for (int i = 0; i < kSvdTile / 4; ++i) {          // row warp + 4i, column lane
-            const int r = warp + 4 * i;
-            Ws[r][lane] = W[(n0 + r) * K + k0 + lane];
-        }
+    load(kbeg);
+    for (int64_t k0 = kbeg; k0 < kend; k0 += kSvdChunk) {
+        __syncthreads();                               // the previous stage's reads are done
 #pragma unroll
-        for (int i = 0; i < kSvdChunk * kSvdRank / kSvdTile; ++i) {
-            const int e = tid + kSvdTile * i;
-            Vs[e >> 5][e & 31] = V[(k0 + (e >> 5)) * kSvdRank + (e & 31)];
-        }
+        for (int i = 0; i < kSvdTile / 4; ++i)
+            Ws[warp + 4 * i][lane] = wr[i];
+#pragma unroll
+        for (int i = 0; i < kSvdChunk * kSvdRank / kSvdTile; ++i)
+            (&Vs[0][0])[tid + kSvdTile * i] = vr[i];
         __syncthreads();
-#pragma unroll 4
+        if (k0 + kSvdChunk < kend)
+            load(k0 + kSvdChunk);
+#pragma unroll 8
         for (int k = 0; k < kSvdChunk; ++k) {
-            float w[4], v[8];
+            float w[4];
 #pragma unroll
             for (int j = 0; j < 4; ++j)
                 w[j] = Ws[lane + 32 * j][k];
-#pragma unroll
-            for (int o = 0; o < 8; ++o)
-                v[o] = Vs[k][8 * warp + o];
+            const float4 va = *reinterpret_cast<const float4 *>(&Vs[k][8 * warp]);
+            const float4 vb = *reinterpret_cast<const float4 *>(&Vs[k][8 * warp + 4]);
+            const float v[8] = {va.x, va.y, va.z, va.w, vb.x, vb.y, vb.z, vb.w};
 #pragma unroll
             for (int j = 0; j < 4; ++j)
 #pragma unroll
                 for (int o = 0; o < 8; ++o)
                     acc[j][o] = fmaf(w[j], v[o], acc[j][o]);
         }
-        __syncthreads();
     }
     float *out = Yp + (int64_t)blockIdx.y * N * kSvdRank;
 #pragma unroll
@@ -99,49 +112,60 @@ __global__ void __launch_bounds__(kSvdTile) svd_wv_kernel(const float *__restric
 // ---------------------------------------------------------------------------
 // Zp[s, k, :] = sum over rows n of split s of W[n, k] U[n, :], for the 128 columns k of the CTA.
 // Grid (K / 128, S), 128 threads.  Warp w owns outputs 8w..8w+7; lane l columns l, l+32, l+64,
-// l+96.  A stage holds 32 rows x 128 columns of W and the matching 32 rows of U.
+// l+96.  A stage holds 32 rows x 128 columns of W and the matching 32 rows of U; the next stage
+// is loaded into registers while the current one is multiplied.
 // ---------------------------------------------------------------------------
 __global__ void __launch_bounds__(kSvdTile) svd_wtu_kernel(const float *__restrict__ W, int64_t K,
                                                            int64_t n_per_split, const float *__restrict__ U,
                                                            float *__restrict__ Zp)
 {
     __shared__ float Ws[kSvdChunk][kSvdTile];
-    __shared__ float Us[kSvdChunk][kSvdRank];
+    __shared__ __align__(16) float Us[kSvdChunk][kSvdRank];
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int64_t k0 = (int64_t)blockIdx.x * kSvdTile;
-    const int64_t nbeg = (int64_t)blockIdx.y * n_per_split;
+    const int64_t nbeg = (int64_t)blockIdx.y * n_per_split, nend = nbeg + n_per_split;
+    float wr[kSvdChunk], ur[kSvdChunk * kSvdRank / kSvdTile];
+    auto load = [&](int64_t n0) {
+#pragma unroll
+        for (int r = 0; r < kSvdChunk; ++r)
+            wr[r] = W[(n0 + r) * K + k0 + tid];
+#pragma unroll
+        for (int i = 0; i < kSvdChunk * kSvdRank / kSvdTile; ++i)
+            ur[i] = U[n0 * kSvdRank + tid + kSvdTile * i];
+    };
     float acc[4][8];
 #pragma unroll
     for (int j = 0; j < 4; ++j)
 #pragma unroll
         for (int o = 0; o < 8; ++o)
             acc[j][o] = 0.0f;
-    for (int64_t n0 = nbeg; n0 < nbeg + n_per_split; n0 += kSvdChunk) {
-#pragma unroll 8
-        for (int r = 0; r < kSvdChunk; ++r)
-            Ws[r][tid] = W[(n0 + r) * K + k0 + tid];
-#pragma unroll
-        for (int i = 0; i < kSvdChunk * kSvdRank / kSvdTile; ++i) {
-            const int e = tid + kSvdTile * i;
-            Us[e >> 5][e & 31] = U[(n0 + (e >> 5)) * kSvdRank + (e & 31)];
-        }
+    load(nbeg);
+    for (int64_t n0 = nbeg; n0 < nend; n0 += kSvdChunk) {
         __syncthreads();
-#pragma unroll 4
+#pragma unroll
+        for (int r = 0; r < kSvdChunk; ++r)
+            Ws[r][tid] = wr[r];
+#pragma unroll
+        for (int i = 0; i < kSvdChunk * kSvdRank / kSvdTile; ++i)
+            (&Us[0][0])[tid + kSvdTile * i] = ur[i];
+        __syncthreads();
+        if (n0 + kSvdChunk < nend)
+            load(n0 + kSvdChunk);
+#pragma unroll 8
         for (int r = 0; r < kSvdChunk; ++r) {
-            float w[4], u[8];
+            float w[4];
 #pragma unroll
             for (int j = 0; j < 4; ++j)
                 w[j] = Ws[r][lane + 32 * j];
-#pragma unroll
-            for (int o = 0; o < 8; ++o)
-                u[o] = Us[r][8 * warp + o];
+            const float4 ua = *reinterpret_cast<const float4 *>(&Us[r][8 * warp]);
+            const float4 ub = *reinterpret_cast<const float4 *>(&Us[r][8 * warp + 4]);
+            const float u[8] = {ua.x, ua.y, ua.z, ua.w, ub.x, ub.y, ub.z, ub.w};
 #pragma unroll
             for (int j = 0; j < 4; ++j)
 #pragma unroll
                 for (int o = 0; o < 8; ++o)
                     acc[j][o] = fmaf(w[j], u[o], acc[j][o]);
         }
-        __syncthreads();
     }
     float *out = Zp + (int64_t)blockIdx.y * K * kSvdRank;
 #pragma unroll
@@ -165,25 +189,31 @@ __global__ void __launch_bounds__(256) svd_sum_splits_kernel(const float *__rest
 }
 
 // ---------------------------------------------------------------------------
-// partial Grams of A [rows, 32]: Gp[c][i][j] = sum over rows 128c..128c+127 (in order) of
-// a_i a_j, fp64 (each fp32 product is exact in fp64).  Grid rows / 128, 256 threads; thread t
-// owns entries (t / 8, 4 (t % 8) .. +3).
+// partial Grams of A [rows, 32] (rows a multiple of 128): Gp[c][i][j] = sum over rows
+// 512c .. min(512c + 511, rows - 1), in order, of a_i a_j, fp64 (each fp32 product is exact in
+// fp64).  Grid ceil(rows / 512), 256 threads; thread t owns entries (t / 8, 4 (t % 8) .. +3);
+// the rows pass through shared memory 128 at a time.
 // ---------------------------------------------------------------------------
-__global__ void __launch_bounds__(256) svd_gram_kernel(const float *__restrict__ A, double *__restrict__ Gp)
+__global__ void __launch_bounds__(256) svd_gram_kernel(const float *__restrict__ A, int64_t rows,
+                                                       double *__restrict__ Gp)
 {
-    __shared__ float As[kGramRows][kSvdRank + 1];
+    __shared__ float As[kGramSub][kSvdRank + 1];
     const int tid = threadIdx.x;
-    const int64_t r0 = (int64_t)blockIdx.x * kGramRows;
-    for (int e = tid; e < kGramRows * kSvdRank; e += 256)
-        As[e >> 5][e & 31] = A[(r0 + (e >> 5)) * kSvdRank + (e & 31)];
-    __syncthreads();
     const int i = tid >> 3, j0 = 4 * (tid & 7);
+    const int64_t r0 = (int64_t)blockIdx.x * kGramRows;
+    const int64_t r1 = r0 + kGramRows < rows ? r0 + kGramRows : rows;
     double acc[4] = {0.0, 0.0, 0.0, 0.0};
-    for (int r = 0; r < kGramRows; ++r) {
-        const double a = (double)As[r][i];
+    for (int64_t rs = r0; rs < r1; rs += kGramSub) {
+        __syncthreads();                               // the previous sub-tile's reads are done
+        for (int e = tid; e < kGramSub * kSvdRank; e += 256)
+            As[e >> 5][e & 31] = A[rs * kSvdRank + e];
+        __syncthreads();
+        for (int r = 0; r < kGramSub; ++r) {
+            const double a = (double)As[r][i];
 #pragma unroll
-        for (int j = 0; j < 4; ++j)
-            acc[j] = fma(a, (double)As[r][j0 + j], acc[j]);
+            for (int j = 0; j < 4; ++j)
+                acc[j] = fma(a, (double)As[r][j0 + j], acc[j]);
+        }
     }
     double *g = Gp + (int64_t)blockIdx.x * (kSvdRank * kSvdRank) + i * kSvdRank + j0;
 #pragma unroll
@@ -196,18 +226,37 @@ __global__ void __launch_bounds__(256) svd_gram_kernel(const float *__restrict__
 // register index is a compile-time constant (the loops are unrolled), values move between
 // lanes by shuffles only.
 // ---------------------------------------------------------------------------
-// G = sum of the C partial Grams in order; lane c gets column c
-__device__ __forceinline__ void svd_load_gram(const double *__restrict__ Gp, int C, int lane, double (&g)[kSvdRank])
+// G = sum of the C partial Grams in order, by all 256 threads (entry e = t + 256 q, four chains
+// per thread, the loads of four partials in flight), written over partial 0 (each entry is
+// read and written by its own thread only).
+__device__ __forceinline__ void svd_sum_grams(double *__restrict__ Gp, int C)
 {
+    const int t = threadIdx.x;
+    double g[4];
 #pragma unroll
-    for (int i = 0; i < kSvdRank; ++i)
-        g[i] = Gp[i * kSvdRank + lane];
-    for (int c = 1; c < C; ++c) {
-        const double *p = Gp + (int64_t)c * (kSvdRank * kSvdRank) + lane;
+    for (int q = 0; q < 4; ++q)
+        g[q] = Gp[t + 256 * q];
+    int c = 1;
+    for (; c + 4 <= C; c += 4) {
+        double v[4][4];
 #pragma unroll
-        for (int i = 0; i < kSvdRank; ++i)
-            g[i] += p[i * kSvdRank];
+        for (int b = 0; b < 4; ++b)
+#pragma unroll
+            for (int q = 0; q < 4; ++q)
+                v[b][q] = Gp[(int64_t)(c + b) * (kSvdRank * kSvdRank) + t + 256 * q];
+#pragma unroll
+        for (int b = 0; b < 4; ++b)
+#pragma unroll
+            for (int q = 0; q < 4; ++q)
+                g[q] += v[b][q];
     }
+    for (; c < C; ++c)
+#pragma unroll
+        for (int q = 0; q < 4; ++q)
+            g[q] += Gp[(int64_t)c * (kSvdRank * kSvdRank) + t + 256 * q];
+#pragma unroll
+    for (int q = 0; q < 4; ++q)
+        Gp[t + 256 * q] = g[q];
 }
 
 // Cholesky G = R^T R (R upper triangular), right-looking.  In: g = column `lane` of G (destroyed).
@@ -340,13 +389,20 @@ __device__ __forceinline__ void svd_jacobi_warp(double (&r)[kSvdRank], int lane,
 }
 
 // EIG = false: Rinv = (Cholesky factor of G)^-1.  EIG = true: eigen-decomposition of G.
+// 256 threads sum the partial Grams; warp 0 then runs the 32 x 32 step, lane c on column c.
 template <bool EIG>
-__global__ void __launch_bounds__(32) svd_small_kernel(const double *__restrict__ Gp, int C, float *__restrict__ Rinv,
-                                                       double *__restrict__ Xo, double *__restrict__ So)
+__global__ void __launch_bounds__(256) svd_small_kernel(double *__restrict__ Gp, int C, float *__restrict__ Rinv,
+                                                        double *__restrict__ Xo, double *__restrict__ So)
 {
+    svd_sum_grams(Gp, C);
+    __syncthreads();                                   // G (over partial 0) is complete and visible
+    if (threadIdx.x >= 32)
+        return;
     const int lane = threadIdx.x;
     double g[kSvdRank], r[kSvdRank];
-    svd_load_gram(Gp, C, lane, g);
+#pragma unroll
+    for (int i = 0; i < kSvdRank; ++i)
+        g[i] = Gp[i * kSvdRank + lane];
     const uint32_t dead = svd_chol_warp(g, r, lane, EIG ? 0.0 : 1.0);
     if (EIG)
         svd_jacobi_warp(r, lane, Xo, So);
@@ -354,30 +410,36 @@ __global__ void __launch_bounds__(32) svd_small_kernel(const double *__restrict_
         svd_rinv_warp(r, dead, lane, Rinv);
 }
 
-// A[row, :] <- A[row, :] Rinv (Rinv upper triangular, fp32), one row per thread
-__global__ void __launch_bounds__(256) svd_apply_kernel(float *__restrict__ A, int64_t rows,
-                                                        const float *__restrict__ Rinv)
+// A[row, :] <- A[row, :] Rinv (Rinv upper triangular, fp32), one row per thread, 64 rows per CTA
+__global__ void __launch_bounds__(64) svd_apply_kernel(float *__restrict__ A, int64_t rows,
+                                                       const float *__restrict__ Rinv)
 {
     __shared__ float Rs[kSvdRank][kSvdRank];
     for (int e = threadIdx.x; e < kSvdRank * kSvdRank; e += blockDim.x)
-        Rs[e >> 5][e & 31] = Rinv[e];
+        (&Rs[0][0])[e] = Rinv[e];
     __syncthreads();
     const int64_t row = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
     if (row >= rows)
         return;
-    float *a_row = A + row * kSvdRank;
+    float4 *a_row = reinterpret_cast<float4 *>(A + row * kSvdRank);
     float a[kSvdRank];
 #pragma unroll
-    for (int i = 0; i < kSvdRank; ++i)
-        a[i] = a_row[i];
+    for (int i = 0; i < kSvdRank / 4; ++i) {
+        const float4 v = a_row[i];
+        a[4 * i] = v.x; a[4 * i + 1] = v.y; a[4 * i + 2] = v.z; a[4 * i + 3] = v.w;
+    }
+    float o[kSvdRank];
 #pragma unroll
     for (int j = 0; j < kSvdRank; ++j) {
-        float s = 0.0f;
+        float acc = 0.0f;
 #pragma unroll
         for (int i = 0; i <= j; ++i)
-            s = fmaf(a[i], Rs[i][j], s);
-        a_row[j] = s;                                  // a[] keeps the old row
+            acc = fmaf(a[i], Rs[i][j], acc);
+        o[j] = acc;
     }
+#pragma unroll
+    for (int i = 0; i < kSvdRank / 4; ++i)
+        a_row[i] = make_float4(o[4 * i], o[4 * i + 1], o[4 * i + 2], o[4 * i + 3]);
 }
 
 // up[n, :] = bf16(U[n, :] X S^(1/4)) for rows n < N, then down[k, :] = bf16(B[k, :] X S^(-1/4))
@@ -422,37 +484,95 @@ __global__ void __launch_bounds__(256) svd_factors_kernel(const float *__restric
 
 // ---------------------------------------------------------------------------
 // R[n, k] = RN(W[n, k] - L[n, k]), L = fmaf chain over r = 0..31 of up[n, r] down[k, r] from 0
-// (the reconstruct's chain).  Tiles of 64 rows x 256 columns, grid-stride; thread t owns column
-// 256 kb + t of the tile's 64 rows, lora_down of that column in registers, lora_up rows read as
-// shared-memory broadcasts.  R may alias W (each element is read before it is written, by the
-// same thread).
+// (the reconstruct's chain).  Grid (K / 256, m): CTA (kb, j) owns columns 256 kb .. +255 and the
+// 64-row tiles j, j + m, ... .  Thread t owns columns 256 kb + 2 (t % 128) and +1 (both chains
+// advance in one fma.rn.f32x2: two independent fmaf roundings) of rows 32 (t / 128) .. +31 of each
+// tile; lora_down of its two columns is staged once (coalesced, through shared memory) and stays
+// in registers, the tile's lora_up rows are read as 16-byte shared-memory broadcasts.  R may alias
+// W (each element is read before it is written, by the same thread).
 // ---------------------------------------------------------------------------
-__global__ void __launch_bounds__(256) svd_residual_kernel(const float *W, int64_t N, int64_t K,
+__device__ __forceinline__ uint64_t svd_pack2(float lo, float hi)
+{
+    uint64_t r;
+    asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+    return r;
+}
+
+__device__ __forceinline__ void svd_bf16x8(const uint4 v, float (&f)[8])
+{
+    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        f[2 * i] = __uint_as_float(w[i] << 16);
+        f[2 * i + 1] = __uint_as_float(w[i] & 0xFFFF0000u);
+    }
+}
+
+constexpr int kResRows = 8;            // rows of W whose loads a residual thread keeps in flight
+
+__global__ void __launch_bounds__(256, 2) svd_residual_kernel(const float *W, int64_t N, int64_t K,
                                                            const uint16_t *__restrict__ up,
                                                            const uint16_t *__restrict__ down, float *R)
 {
-    __shared__ float us[64][kSvdRank];
+    __shared__ float ds[256][kSvdRank + 1];
+    __shared__ __align__(16) float us[64 * kSvdRank];
     const int tid = threadIdx.x;
-    const int64_t NT = N / 64, T = NT * (K / 256);
-    for (int64_t t = blockIdx.x; t < T; t += gridDim.x) {
-        const int64_t kb = t / NT, n0 = (t % NT) * 64;
-        const int64_t k = kb * 256 + tid;
+    const int cp = tid & 127, rbase = 32 * (tid >> 7);
+    const int64_t k = (int64_t)blockIdx.x * 256 + 2 * cp;
+    const uint4 *dsrc = reinterpret_cast<const uint4 *>(down + (int64_t)blockIdx.x * 256 * kSvdRank);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {                      // 256 columns x 32 bf16 = 1024 16-byte pieces
+        const int e = tid + 256 * i;
+        float f[8];
+        svd_bf16x8(dsrc[e], f);
+#pragma unroll
+        for (int q = 0; q < 8; ++q)
+            ds[e >> 2][8 * (e & 3) + q] = f[q];
+    }
+    __syncthreads();
+    uint64_t d2[kSvdRank];
+#pragma unroll
+    for (int r = 0; r < kSvdRank; ++r)
+        d2[r] = svd_pack2(ds[2 * cp][r], ds[2 * cp + 1][r]);
+    const int64_t NT = N / 64;
+    for (int64_t nt = blockIdx.y; nt < NT; nt += gridDim.y) {
+        const int64_t n0 = nt * 64;
         __syncthreads();                               // the previous tile's reads of us are done
-        for (int e = tid; e < 64 * kSvdRank; e += 256)
-            us[e >> 5][e & 31] = bf16_bits_to_f32(up[(n0 + (e >> 5)) * kSvdRank + (e & 31)]);
-        float d[kSvdRank];
-#pragma unroll
-        for (int r = 0; r < kSvdRank; ++r)
-            d[r] = bf16_bits_to_f32(down[k * kSvdRank + r]);
+        {                                              // 64 rows x 32 bf16 = 256 16-byte pieces
+            float f[8];
+            svd_bf16x8(reinterpret_cast<const uint4 *>(up + n0 * kSvdRank)[tid], f);
+            *reinterpret_cast<float4 *>(&us[8 * tid]) = make_float4(f[0], f[1], f[2], f[3]);
+            *reinterpret_cast<float4 *>(&us[8 * tid + 4]) = make_float4(f[4], f[5], f[6], f[7]);
+        }
         __syncthreads();
-#pragma unroll 2
-        for (int n = 0; n < 64; ++n) {
-            float L = 0.0f;
+        for (int nb = rbase; nb < rbase + 32; nb += kResRows) {
+            float2 w[kResRows];                        // the block's W values, all loads in flight
 #pragma unroll
-            for (int r = 0; r < kSvdRank; ++r)
-                L = fmaf(us[n][r], d[r], L);
-            const int64_t idx = (n0 + n) * K + k;
-            R[idx] = __fsub_rn(W[idx], L);
+            for (int i = 0; i < kResRows; ++i)
+                w[i] = *reinterpret_cast<const float2 *>(W + (n0 + nb + i) * K + k);
+            uint64_t acc[kResRows];
+#pragma unroll
+            for (int i = 0; i < kResRows; ++i)
+                acc[i] = 0ull;
+#pragma unroll
+            for (int r4 = 0; r4 < kSvdRank; r4 += 4) {
+#pragma unroll
+                for (int i = 0; i < kResRows; ++i) {
+                    const float4 u = *reinterpret_cast<const float4 *>(&us[(nb + i) * kSvdRank + r4]);
+                    const float uv[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+                    for (int q = 0; q < 4; ++q)
+                        asm("fma.rn.f32x2 %0, %1, %2, %0;"
+                            : "+l"(acc[i]) : "l"(svd_pack2(uv[q], uv[q])), "l"(d2[r4 + q]));
+                }
+            }
+#pragma unroll
+            for (int i = 0; i < kResRows; ++i) {
+                float L0, L1;
+                asm("mov.b64 {%0, %1}, %2;" : "=f"(L0), "=f"(L1) : "l"(acc[i]));
+                *reinterpret_cast<float2 *>(R + (n0 + nb + i) * K + k) =
+                    make_float2(__fsub_rn(w[i].x, L0), __fsub_rn(w[i].y, L1));
+            }
         }
     }
 }
@@ -474,16 +594,17 @@ size_t svd_workspace_bytes(int64_t N, int64_t K)
 {
     const int64_t rows = max64(N, K);
     return up256((size_t)N * kSvdRank * 4) + up256((size_t)K * kSvdRank * 4) +
-           up256((size_t)8 * rows * kSvdRank * 4) + up256((size_t)(rows / kGramRows) * kSvdRank * kSvdRank * 8) +
+           up256((size_t)kSvdMaxSplits * rows * kSvdRank * 4) +
+           up256((size_t)((rows + kGramRows - 1) / kGramRows) * kSvdRank * kSvdRank * 8) +
            up256(kSvdRank * kSvdRank * 4) + up256(kSvdRank * kSvdRank * 8) + up256(kSvdRank * 8);
 }
 
-// splits s in {1, 2, 4, 8} of the reduction dimension `depth` (each part a multiple of 32 deep)
-// until the grid of `tiles` x s CTAs reaches the target
+// splits s in {1, 2, 4, 8, 16} of the reduction dimension `depth` (each part a multiple of 32
+// deep) until the grid of `tiles` x s CTAs reaches the target
 static int svd_splits(int64_t tiles, int64_t depth)
 {
     int s = 1;
-    while (s < 8 && tiles * s < kSvdTargetCtas && depth % (kSvdChunk * 2 * s) == 0)
+    while (s < kSvdMaxSplits && tiles * s < kSvdTargetCtas && depth % (kSvdChunk * 2 * s) == 0)
         s *= 2;
     return s;
 }
@@ -502,15 +623,17 @@ struct SvdWs {
         }                                                \
     } while (0)
 
-static cudaError_t svd_orth(float *A, int64_t rows, const SvdWs &w, cudaStream_t s, const char **stage)
+// orth(A): CholeskyQR, `passes` times (two for the final U, which must be orthonormal to fp32
+// accuracy; one for the blocks in between, which only carry the subspace to the next product)
+static cudaError_t svd_orth(float *A, int64_t rows, int passes, const SvdWs &w, cudaStream_t s, const char **stage)
 {
-    const int C = (int)(rows / kGramRows);
-    for (int pass = 0; pass < 2; ++pass) {             // CholeskyQR, twice
-        svd_gram_kernel<<<(unsigned)C, 256, 0, s>>>(A, w.Gp);
+    const int C = (int)((rows + kGramRows - 1) / kGramRows);
+    for (int pass = 0; pass < passes; ++pass) {
+        svd_gram_kernel<<<(unsigned)C, 256, 0, s>>>(A, rows, w.Gp);
         SVD_STEP("svd gram");
-        svd_small_kernel<false><<<1, 32, 0, s>>>(w.Gp, C, w.Rinv, nullptr, nullptr);
+        svd_small_kernel<false><<<1, 256, 0, s>>>(w.Gp, C, w.Rinv, nullptr, nullptr);
         SVD_STEP("svd cholesky");
-        svd_apply_kernel<<<(unsigned)((rows + 255) / 256), 256, 0, s>>>(A, rows, w.Rinv);
+        svd_apply_kernel<<<(unsigned)((rows + 63) / 64), 64, 0, s>>>(A, rows, w.Rinv);
         SVD_STEP("svd apply");
     }
     return cudaSuccess;
@@ -537,9 +660,9 @@ cudaError_t launch_svd_init(const float *W, int64_t N, int64_t K, const float *o
     w.V = reinterpret_cast<float *>(p);
     p += up256((size_t)K * kSvdRank * 4);
     w.P = reinterpret_cast<float *>(p);
-    p += up256((size_t)8 * rows * kSvdRank * 4);
+    p += up256((size_t)kSvdMaxSplits * rows * kSvdRank * 4);
     w.Gp = reinterpret_cast<double *>(p);
-    p += up256((size_t)(rows / kGramRows) * kSvdRank * kSvdRank * 8);
+    p += up256((size_t)((rows + kGramRows - 1) / kGramRows) * kSvdRank * kSvdRank * 8);
     w.Rinv = reinterpret_cast<float *>(p);
     p += up256(kSvdRank * kSvdRank * 4);
     w.X = reinterpret_cast<double *>(p);
@@ -550,7 +673,7 @@ cudaError_t launch_svd_init(const float *W, int64_t N, int64_t K, const float *o
     cudaError_t e = cudaMemcpyAsync(w.V, omega, (size_t)K * kSvdRank * 4, cudaMemcpyDeviceToDevice, s);
     if (e != cudaSuccess)
         return e;
-    if ((e = svd_orth(w.V, K, w, s, stage)) != cudaSuccess)
+    if ((e = svd_orth(w.V, K, 1, w, s, stage)) != cudaSuccess)
         return e;
     const int sv = svd_splits(N / kSvdTile, K), sz = svd_splits(K / kSvdTile, N);
     for (int it = 0; it < iters; ++it) {
@@ -558,26 +681,27 @@ cudaError_t launch_svd_init(const float *W, int64_t N, int64_t K, const float *o
         SVD_STEP("svd W V");
         if ((e = svd_sum(w.P, sv, N, w.Y, sms, s, stage)) != cudaSuccess)
             return e;
-        if ((e = svd_orth(w.Y, N, w, s, stage)) != cudaSuccess)
+        if ((e = svd_orth(w.Y, N, it + 1 < iters ? 1 : 2, w, s, stage)) != cudaSuccess)
             return e;
         svd_wtu_kernel<<<dim3((unsigned)(K / kSvdTile), (unsigned)sz), kSvdTile, 0, s>>>(W, K, N / sz, w.Y, w.P);
         SVD_STEP("svd W^T U");
         if ((e = svd_sum(w.P, sz, K, w.V, sms, s, stage)) != cudaSuccess)
             return e;
-        if (it + 1 < iters && (e = svd_orth(w.V, K, w, s, stage)) != cudaSuccess)
+        if (it + 1 < iters && (e = svd_orth(w.V, K, 1, w, s, stage)) != cudaSuccess)
             return e;
     }
     // B = W^T U is in w.V; the eigen-decomposition of its Gram gives the rotation and sigma^2
-    const int CK = (int)(K / kGramRows);
-    svd_gram_kernel<<<(unsigned)CK, 256, 0, s>>>(w.V, w.Gp);
+    const int CK = (int)((K + kGramRows - 1) / kGramRows);
+    svd_gram_kernel<<<(unsigned)CK, 256, 0, s>>>(w.V, K, w.Gp);
     SVD_STEP("svd gram");
-    svd_small_kernel<true><<<1, 32, 0, s>>>(w.Gp, CK, nullptr, w.X, w.S);
+    svd_small_kernel<true><<<1, 256, 0, s>>>(w.Gp, CK, nullptr, w.X, w.S);
     SVD_STEP("svd jacobi");
     svd_factors_kernel<<<(unsigned)((N + K + 255) / 256), 256, 0, s>>>(w.Y, w.V, N, K, w.X, w.S, up, down);
     SVD_STEP("svd factors");
-    const int64_t tiles = (N / 64) * (K / 256);
-    const int64_t grid = tiles < (int64_t)sms * 4 ? tiles : (int64_t)sms * 4;
-    svd_residual_kernel<<<(unsigned)grid, 256, 0, s>>>(W, N, K, up, down, R);
+    const int64_t kbs = K / 256, nts = N / 64;
+    int64_t m = ((int64_t)sms * 2) / kbs;              // one wave of two CTAs per SM
+    m = m < 1 ? 1 : (m > nts ? nts : m);
+    svd_residual_kernel<<<dim3((unsigned)kbs, (unsigned)m), 256, 0, s>>>(W, N, K, up, down, R);
     SVD_STEP("svd residual");
     return cudaSuccess;
 }

@@ -27,6 +27,8 @@ Operations:
                        sq_reconstruct_bf16 with SQ_RECON_RESIDUAL_ONLY
   recon_nvfp4_t        sq_reconstruct_bf16 with SQ_RECON_TRANSPOSED (W^T)
   bwd_dx_nvfp4         sq_linear_bwd_dx (transposed reconstruct + bf16 GEMM)
+  svd_init             sq_svd_init (rank-32 SVD init, 8 rounds of subspace iteration)
+                       of W = lora_up lora_down^T + R
   gemm_nvfp4 / gemm_int4 / gemm_bwd_dx
                        the tensor-core GEMM launch inside sq_linear_fwd /
                        sq_linear_bwd_dx, timed by the events the library records
@@ -58,7 +60,8 @@ FLUSH_BYTES = 256 << 20
 OPS = ["act_quant", "act_quant_nolowrank", "fwd_nvfp4", "fwd_int4", "fwd_int8", "build_nvfp4", "build_int4",
        "build_int4_g64", "build_int8", "recon_nvfp4", "recon_int4", "recon_int4_g64", "recon_int8",
        "recon_nvfp4_resid", "recon_int4_resid", "recon_int8_resid", "recon_nvfp4_t", "gemm_nvfp4", "gemm_int4",
-       "bwd_dx_nvfp4", "gemm_bwd_dx"]
+       "bwd_dx_nvfp4", "gemm_bwd_dx", "svd_init"]
+SVD_ITERS = 8
 
 
 def work(op, M, N, K):
@@ -66,6 +69,8 @@ def work(op, M, N, K):
     NK, MK = N * K, M * K
     if op.startswith("act_quant"):
         return "GB/s", MK * (2 + 0.5 + 1 / 16) + (M * 32 * 4 if op == "act_quant" else 0)
+    if op == "svd_init":   # fp32 FMA work: two products with W per round, then the residual's chain
+        return "TFLOP/s", (4.0 * SVD_ITERS + 2.0) * N * K * 32
     if op.startswith("fwd") or op.startswith("gemm") or op.startswith("bwd"):
         return "TFLOP/s", 2.0 * M * N * K
     if op == "build_nvfp4":
@@ -159,6 +164,13 @@ def main():
     dx = torch.empty((M, K), dtype=torch.float32, device=dev)
     ws_dx = sq.workspace(sq.SQ_OP_LINEAR_BWD_DX, M, N, K, dev)
     c4 = torch.empty_like(w4.codes)
+    if "svd_init" in args.op:
+        Wsvd = R + U.float() @ D.float().T
+        omega = torch.randn((K, 32), device=dev, generator=torch.Generator(device=dev).manual_seed(cfg.seed))
+        up_s = torch.empty((N, 32), dtype=torch.bfloat16, device=dev)
+        down_s = torch.empty((K, 32), dtype=torch.bfloat16, device=dev)
+        R_s = torch.empty_like(R)
+        ws_s = sq.workspace(sq.SQ_OP_SVD_INIT, 0, N, K, dev)
     s4, f4 = torch.empty_like(w4.scales), torch.empty_like(w4.frac_idx)
     s6, f6 = torch.empty_like(w6.scales), torch.empty_like(w6.frac_idx)
     cn, sfn, gn = torch.empty_like(wn.codes), torch.empty_like(wn.scales), torch.empty_like(wn.g_w)
@@ -186,6 +198,7 @@ def main():
         "gemm_bwd_dx": lambda: sq.sq_linear_bwd_dx(wn, dy, dx, ws_dx),
         "gemm_nvfp4": lambda: sq.sq_linear_fwd(wn, x, y, g_x=gx, ws=ws_n),
         "gemm_int4": lambda: sq.sq_linear_fwd(w4, x, y, ws=ws_i),
+        "svd_init": lambda: sq.sq_svd_init(Wsvd, omega, SVD_ITERS, up_s, down_s, R_s, ws_s),
     }
     flush = torch.empty(FLUSH_BYTES // 4, dtype=torch.int32, device=dev)
     torch.cuda.synchronize()

@@ -171,9 +171,10 @@ SQ_API sq_status sq_build_int4(const float *R, int64_t N, int64_t K, int32_t gro
  * `iters` (1..100) rounds of subspace iteration from the caller's start block
  * omega [K, 32] fp32 (device; e.g. seeded N(0, 1) draws): each round one
  * product with W and one with W^T (fp32, fixed summation order), each followed
- * by CholeskyQR twice (fp64 Grams).  With B = W^T U from the last round, the
- * Cholesky factor of B^T B and a one-sided Jacobi iteration on its columns
- * give sigma and the rotation of the factors.  Deterministic for a given shape
+ * by CholeskyQR with fp64 Grams (twice for the final U).  With B = W^T U from
+ * the last round, the Cholesky factor of B^T B and a one-sided Jacobi
+ * iteration on its columns give sigma and the rotation of the factors.
+ * Deterministic for a given shape
  * and omega.  The accuracy of the rank-32 product against the exact truncated
  * SVD improves as (sigma_33 / sigma_32)^(2 iters); R is RN(W - L) of whatever
  * factors result (it absorbs what they miss).

@@ -106,6 +106,23 @@ def test_svd_init_is_deterministic_and_exact_rank(sq):
     assert np.array_equal(R.view(np.uint32), Rw.view(np.uint32))
 
 
+def test_svd_init_ill_conditioned(sq):
+    """Singular values 1e4 .. 1 above the gap (the blocks between the products are orthonormalised
+    once, the final U twice): the product still matches the truncated SVD."""
+    rng = np.random.default_rng(104)
+    N, K = 512, 1024
+    A = np.linalg.qr(rng.standard_normal((N, 40)))[0]
+    B = np.linalg.qr(rng.standard_normal((K, 40)))[0]
+    s = np.concatenate([np.geomspace(1e4, 1.0, 32), np.geomspace(0.2, 0.1, 8)])
+    W = ((A * s) @ B.T).astype(np.float32)
+    up, down, R = run_gpu(sq, W, omega(K, 14))
+    oup, odown, _, _ = oracle.svd_init(W)
+    L, Lo = lowrank_product(up, down), lowrank_product(oup, odown)
+    assert np.linalg.norm(L - Lo) / np.linalg.norm(Lo) <= L_TOL
+    Rw = oracle.svd_residual(W, up, down)
+    assert np.array_equal(R.view(np.uint32), Rw.view(np.uint32))
+
+
 def test_svd_init_zero_weight(sq):
     W = np.zeros((128, 256), np.float32)
     up, down, R = run_gpu(sq, W, omega(256, 9), iters=2)
