@@ -41,6 +41,35 @@ constexpr unsigned kFull = 0xffffffffu;
 constexpr int kSvdTargetCtas = 1024;   // product grids are split until they reach this many CTAs
 constexpr int kSvdMaxSplits = 16;
 
+// two fp32 values as one 64-bit operand of the packed f32x2 instructions, and back
+__device__ __forceinline__ uint64_t svd_pack2(float lo, float hi)
+{
+    uint64_t r;
+    asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+    return r;
+}
+
+__device__ __forceinline__ void svd_unpack2(uint64_t v, float &lo, float &hi)
+{
+    asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+}
+
+// acc[j][p] += w[j] * (v[2p], v[2p+1]) for 4 rows j and 4 output pairs p: 16 fma.rn.f32x2, each two
+// independent fmaf roundings
+__device__ __forceinline__ void svd_fma_4x8(uint64_t (&acc)[4][4], const float (&w)[4], const float4 va,
+                                           const float4 vb)
+{
+    const uint64_t v2[4] = {svd_pack2(va.x, va.y), svd_pack2(va.z, va.w), svd_pack2(vb.x, vb.y),
+                            svd_pack2(vb.z, vb.w)};
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+        const uint64_t w2 = svd_pack2(w[j], w[j]);
+#pragma unroll
+        for (int p = 0; p < 4; ++p)
+            asm("fma.rn.f32x2 %0, %1, %2, %0;" : "+l"(acc[j][p]) : "l"(w2), "l"(v2[p]));
+    }
+}
+
 // ---------------------------------------------------------------------------
 // Yp[s, n, :] = sum over k in split s of W[n, k] V[k, :], for the 128 rows n of the CTA.
 // Grid (N / 128, S), 128 threads.  Warp w owns outputs 8w..8w+7; lane l rows l, l+32, l+64, l+96.
@@ -67,12 +96,12 @@ __global__ void __launch_bounds__(kSvdTile) svd_wv_kernel(const float *__restric
         for (int i = 0; i < kSvdChunk * kSvdRank / kSvdTile; ++i)
             vr[i] = V[k0 * kSvdRank + tid + kSvdTile * i];
     };
-    float acc[4][8];
+    uint64_t acc[4][4];
 #pragma unroll
     for (int j = 0; j < 4; ++j)
 #pragma unroll
-        for (int o = 0; o < 8; ++o)
-            acc[j][o] = 0.0f;
+        for (int p = 0; p < 4; ++p)
+            acc[j][p] = 0ull;
     load(kbeg);
     for (int64_t k0 = kbeg; k0 < kend; k0 += kSvdChunk) {
         __syncthreads();                               // the previous stage's reads are done
@@ -91,22 +120,20 @@ __global__ void __launch_bounds__(kSvdTile) svd_wv_kernel(const float *__restric
 #pragma unroll
             for (int j = 0; j < 4; ++j)
                 w[j] = Ws[lane + 32 * j][k];
-            const float4 va = *reinterpret_cast<const float4 *>(&Vs[k][8 * warp]);
-            const float4 vb = *reinterpret_cast<const float4 *>(&Vs[k][8 * warp + 4]);
-            const float v[8] = {va.x, va.y, va.z, va.w, vb.x, vb.y, vb.z, vb.w};
-#pragma unroll
-            for (int j = 0; j < 4; ++j)
-#pragma unroll
-                for (int o = 0; o < 8; ++o)
-                    acc[j][o] = fmaf(w[j], v[o], acc[j][o]);
+            svd_fma_4x8(acc, w, *reinterpret_cast<const float4 *>(&Vs[k][8 * warp]),
+                        *reinterpret_cast<const float4 *>(&Vs[k][8 * warp + 4]));
         }
     }
     float *out = Yp + (int64_t)blockIdx.y * N * kSvdRank;
 #pragma unroll
     for (int j = 0; j < 4; ++j)
 #pragma unroll
-        for (int o = 0; o < 8; ++o)
-            out[(n0 + lane + 32 * j) * kSvdRank + 8 * warp + o] = acc[j][o];
+        for (int p = 0; p < 4; ++p) {
+            float lo, hi;
+            svd_unpack2(acc[j][p], lo, hi);
+            out[(n0 + lane + 32 * j) * kSvdRank + 8 * warp + 2 * p] = lo;
+            out[(n0 + lane + 32 * j) * kSvdRank + 8 * warp + 2 * p + 1] = hi;
+        }
 }
 
 // ---------------------------------------------------------------------------
@@ -133,12 +160,12 @@ __global__ void __launch_bounds__(kSvdTile) svd_wtu_kernel(const float *__restri
         for (int i = 0; i < kSvdChunk * kSvdRank / kSvdTile; ++i)
             ur[i] = U[n0 * kSvdRank + tid + kSvdTile * i];
     };
-    float acc[4][8];
+    uint64_t acc[4][4];
 #pragma unroll
     for (int j = 0; j < 4; ++j)
 #pragma unroll
-        for (int o = 0; o < 8; ++o)
-            acc[j][o] = 0.0f;
+        for (int p = 0; p < 4; ++p)
+            acc[j][p] = 0ull;
     load(nbeg);
     for (int64_t n0 = nbeg; n0 < nend; n0 += kSvdChunk) {
         __syncthreads();
@@ -157,22 +184,20 @@ __global__ void __launch_bounds__(kSvdTile) svd_wtu_kernel(const float *__restri
 #pragma unroll
             for (int j = 0; j < 4; ++j)
                 w[j] = Ws[r][lane + 32 * j];
-            const float4 ua = *reinterpret_cast<const float4 *>(&Us[r][8 * warp]);
-            const float4 ub = *reinterpret_cast<const float4 *>(&Us[r][8 * warp + 4]);
-            const float u[8] = {ua.x, ua.y, ua.z, ua.w, ub.x, ub.y, ub.z, ub.w};
-#pragma unroll
-            for (int j = 0; j < 4; ++j)
-#pragma unroll
-                for (int o = 0; o < 8; ++o)
-                    acc[j][o] = fmaf(w[j], u[o], acc[j][o]);
+            svd_fma_4x8(acc, w, *reinterpret_cast<const float4 *>(&Us[r][8 * warp]),
+                        *reinterpret_cast<const float4 *>(&Us[r][8 * warp + 4]));
         }
     }
     float *out = Zp + (int64_t)blockIdx.y * K * kSvdRank;
 #pragma unroll
     for (int j = 0; j < 4; ++j)
 #pragma unroll
-        for (int o = 0; o < 8; ++o)
-            out[(k0 + lane + 32 * j) * kSvdRank + 8 * warp + o] = acc[j][o];
+        for (int p = 0; p < 4; ++p) {
+            float lo, hi;
+            svd_unpack2(acc[j][p], lo, hi);
+            out[(k0 + lane + 32 * j) * kSvdRank + 8 * warp + 2 * p] = lo;
+            out[(k0 + lane + 32 * j) * kSvdRank + 8 * warp + 2 * p + 1] = hi;
+        }
 }
 
 // out[i] = P[0][i] + P[1][i] + ... + P[S-1][i] in that order, i < rows * 32
@@ -491,13 +516,6 @@ __global__ void __launch_bounds__(256) svd_factors_kernel(const float *__restric
 // in registers, the tile's lora_up rows are read as 16-byte shared-memory broadcasts.  R may alias
 // W (each element is read before it is written, by the same thread).
 // ---------------------------------------------------------------------------
-__device__ __forceinline__ uint64_t svd_pack2(float lo, float hi)
-{
-    uint64_t r;
-    asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
-    return r;
-}
-
 __device__ __forceinline__ void svd_bf16x8(const uint4 v, float (&f)[8])
 {
     const uint32_t w[4] = {v.x, v.y, v.z, v.w};
@@ -569,7 +587,7 @@ __global__ void __launch_bounds__(256, 2) svd_residual_kernel(const float *W, in
 #pragma unroll
             for (int i = 0; i < kResRows; ++i) {
                 float L0, L1;
-                asm("mov.b64 {%0, %1}, %2;" : "=f"(L0), "=f"(L1) : "l"(acc[i]));
+                svd_unpack2(acc[i], L0, L1);
                 *reinterpret_cast<float2 *>(R + (n0 + nb + i) * K + k) =
                     make_float2(__fsub_rn(w[i].x, L0), __fsub_rn(w[i].y, L1));
             }
