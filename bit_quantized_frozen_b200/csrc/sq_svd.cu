@@ -215,35 +215,63 @@ __global__ void __launch_bounds__(256) svd_sum_splits_kernel(const float *__rest
 
 // ---------------------------------------------------------------------------
 // partial Grams of A [rows, 32] (rows a multiple of 128): Gp[c][i][j] = sum over rows
-// 512c .. min(512c + 511, rows - 1), in order, of a_i a_j, fp64 (each fp32 product is exact in
-// fp64).  Grid ceil(rows / 512), 256 threads; thread t owns entries (t / 8, 4 (t % 8) .. +3);
-// the rows pass through shared memory 128 at a time.
+// 512c .. min(512c + 511, rows - 1) of a_i a_j in fp64 (each fp32 product is exact in fp64).
+// Grid ceil(rows / 512), 256 threads.  Lane l of warp w owns the 4 x 4 block b = 8w + l % 8
+// (entries 4 (b / 8) .. +3 by 4 (b % 8) .. +3) over the rows r with r % 4 == l / 8 of each
+// 128-row shared-memory sub-tile, in order; the four row groups of a block sit in lanes l, l + 8,
+// l + 16, l + 24 and are added by two xor shuffles, ((g0 + g1) + (g2 + g3)) -- a fixed order.
+// Each lane converts 8 fp32 values per row for 16 products.
 // ---------------------------------------------------------------------------
 __global__ void __launch_bounds__(256) svd_gram_kernel(const float *__restrict__ A, int64_t rows,
                                                        double *__restrict__ Gp)
 {
-    __shared__ float As[kGramSub][kSvdRank + 1];
-    const int tid = threadIdx.x;
-    const int i = tid >> 3, j0 = 4 * (tid & 7);
+    __shared__ __align__(16) float As[kGramSub * kSvdRank];
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int b = 8 * warp + (lane & 7), g = lane >> 3;
+    const int bi = 4 * (b >> 3), bj = 4 * (b & 7);
     const int64_t r0 = (int64_t)blockIdx.x * kGramRows;
     const int64_t r1 = r0 + kGramRows < rows ? r0 + kGramRows : rows;
-    double acc[4] = {0.0, 0.0, 0.0, 0.0};
+    double acc[4][4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+#pragma unroll
+        for (int j = 0; j < 4; ++j)
+            acc[i][j] = 0.0;
     for (int64_t rs = r0; rs < r1; rs += kGramSub) {
         __syncthreads();                               // the previous sub-tile's reads are done
-        for (int e = tid; e < kGramSub * kSvdRank; e += 256)
-            As[e >> 5][e & 31] = A[rs * kSvdRank + e];
-        __syncthreads();
-        for (int r = 0; r < kGramSub; ++r) {
-            const double a = (double)As[r][i];
+        const float4 *src = reinterpret_cast<const float4 *>(A + rs * kSvdRank);
 #pragma unroll
-            for (int j = 0; j < 4; ++j)
-                acc[j] = fma(a, (double)As[r][j0 + j], acc[j]);
+        for (int e = 0; e < kGramSub * kSvdRank / 4 / 256; ++e)
+            reinterpret_cast<float4 *>(As)[tid + 256 * e] = src[tid + 256 * e];
+        __syncthreads();
+#pragma unroll 4
+        for (int r = g; r < kGramSub; r += 4) {
+            const float4 x = *reinterpret_cast<const float4 *>(&As[r * kSvdRank + bi]);
+            const float4 y = *reinterpret_cast<const float4 *>(&As[r * kSvdRank + bj]);
+            const double xi[4] = {(double)x.x, (double)x.y, (double)x.z, (double)x.w};
+            const double yj[4] = {(double)y.x, (double)y.y, (double)y.z, (double)y.w};
+#pragma unroll
+            for (int i = 0; i < 4; ++i)
+#pragma unroll
+                for (int j = 0; j < 4; ++j)
+                    acc[i][j] = fma(xi[i], yj[j], acc[i][j]);
         }
     }
-    double *g = Gp + (int64_t)blockIdx.x * (kSvdRank * kSvdRank) + i * kSvdRank + j0;
 #pragma unroll
-    for (int j = 0; j < 4; ++j)
-        g[j] = acc[j];
+    for (int i = 0; i < 4; ++i)
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            acc[i][j] += __shfl_xor_sync(kFull, acc[i][j], 8);
+            acc[i][j] += __shfl_xor_sync(kFull, acc[i][j], 16);
+        }
+    if (g == 0) {
+        double *out = Gp + (int64_t)blockIdx.x * (kSvdRank * kSvdRank);
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+#pragma unroll
+            for (int j = 0; j < 4; ++j)
+                out[(bi + i) * kSvdRank + bj + j] = acc[i][j];
+    }
 }
 
 // ---------------------------------------------------------------------------
@@ -285,11 +313,12 @@ __device__ __forceinline__ void svd_sum_grams(double *__restrict__ Gp, int C)
 }
 
 // Cholesky G = R^T R (R upper triangular), right-looking.  In: g = column `lane` of G (destroyed).
-// Out: r = column `lane` of R (r[i] = R[i][lane], zero below the diagonal).  A pivot that is not
-// positive (a rank-deficient block, e.g. a zero weight) is a bit of the returned mask; its row of
-// R is zero except R[j][j] = dead_diag.
-__device__ __forceinline__ uint32_t svd_chol_warp(double (&g)[kSvdRank], double (&r)[kSvdRank], int lane,
-                                                  double dead_diag)
+// Out: r = column `lane` of R (r[i] = R[i][lane], zero below the diagonal) and inv = 1 / R[lane][lane]
+// (0 for a dead pivot); a pivot d gives R[j][j] = d rsqrt(d) and row j of R = G[j][.] rsqrt(d).  A
+// pivot that is not positive (a rank-deficient block, e.g. a zero weight) is a bit of the returned
+// mask; its row of R is zero except R[j][j] = dead_diag.
+__device__ __forceinline__ uint32_t svd_chol_warp(double (&g)[kSvdRank], double (&r)[kSvdRank], double &inv,
+                                                  int lane, double dead_diag)
 {
     double diag0 = 0.0;                                // G[lane][lane] before any update
 #pragma unroll
@@ -303,12 +332,15 @@ __device__ __forceinline__ uint32_t svd_chol_warp(double (&g)[kSvdRank], double 
         const double d0 = __shfl_sync(kFull, diag0, j);
         const bool dj = !(d > 1e-300 * (1.0 + d0));
         dead |= dj ? (1u << j) : 0u;
-        const double rjj = dj ? dead_diag : sqrt(d);
+        const double ij = dj ? 0.0 : rsqrt(d);
+        const double rjj = dj ? dead_diag : d * ij;
         double rjc = 0.0;
-        if (lane == j)
+        if (lane == j) {
             rjc = rjj;
-        else if (lane > j && !dj)
-            rjc = g[j] / rjj;
+            inv = ij;
+        } else if (lane > j && !dj) {
+            rjc = g[j] * ij;
+        }
         r[j] = rjc;
 #pragma unroll
         for (int i = j + 1; i < kSvdRank; ++i) {       // G[i][lane] -= R[j][i] R[j][lane]
@@ -319,9 +351,10 @@ __device__ __forceinline__ uint32_t svd_chol_warp(double (&g)[kSvdRank], double 
     return dead;
 }
 
-// Rinv = R^-1 (fp32, row-major 32 x 32): lane c solves R x = e_c by back substitution; the rows
-// of dead pivots are zero, so the matching columns of the orthonormalised block are zero.
-__device__ __forceinline__ void svd_rinv_warp(const double (&r)[kSvdRank], uint32_t dead, int lane,
+// Rinv = R^-1 (fp32, row-major 32 x 32): lane c solves R x = e_c by back substitution, dividing by
+// the pivots through their reciprocals (inv of lane i); the rows of dead pivots are zero, so the
+// matching columns of the orthonormalised block are zero.
+__device__ __forceinline__ void svd_rinv_warp(const double (&r)[kSvdRank], double inv, uint32_t dead, int lane,
                                               float *__restrict__ Rinv)
 {
     double x[kSvdRank];
@@ -331,8 +364,8 @@ __device__ __forceinline__ void svd_rinv_warp(const double (&r)[kSvdRank], uint3
 #pragma unroll
         for (int k = i + 1; k < kSvdRank; ++k)
             v = fma(-__shfl_sync(kFull, r[i], k), x[k], v);   // R[i][k] is lane k's r[i]
-        const double rii = __shfl_sync(kFull, r[i], i);
-        x[i] = ((dead >> i) & 1u) ? 0.0 : v / rii;
+        const double ii = __shfl_sync(kFull, inv, i);
+        x[i] = ((dead >> i) & 1u) ? 0.0 : v * ii;
     }
 #pragma unroll
     for (int i = 0; i < kSvdRank; ++i)
@@ -361,22 +394,23 @@ __device__ __forceinline__ void svd_jacobi_warp(double (&r)[kSvdRank], int lane,
                                 : lane == round     ? kSvdRank - 1
                                                     : (2 * round - lane + 2 * (kSvdRank - 1)) % (kSvdRank - 1);
             const bool lower = lane < partner;
-            double a = 0.0, b = 0.0, g = 0.0;
+            double a[2] = {0.0, 0.0}, b[2] = {0.0, 0.0}, g[2] = {0.0, 0.0};   // even / odd i
 #pragma unroll
             for (int i = 0; i < kSvdRank; ++i) {
                 const double p = __shfl_sync(kFull, r[i], partner);
-                a = fma(r[i], r[i], a);
-                b = fma(p, p, b);
-                g = fma(r[i], p, g);
+                a[i & 1] = fma(r[i], r[i], a[i & 1]);
+                b[i & 1] = fma(p, p, b[i & 1]);
+                g[i & 1] = fma(r[i], p, g[i & 1]);
             }
-            const double app = lower ? a : b, aqq = lower ? b : a;
-            const double nrm = sqrt(app) * sqrt(aqq);
+            const double an = a[0] + a[1], bn = b[0] + b[1], gn = g[0] + g[1];
+            const double app = lower ? an : bn, aqq = lower ? bn : an;
+            const double prod = app * aqq, g2 = gn * gn;
             double c = 1.0, s = 0.0;
-            if (fabs(g) > kJacobiSkip * nrm) {
-                off = fmax(off, fabs(g) / nrm);
-                const double z = (aqq - app) / (2.0 * g);
+            if (g2 > kJacobiSkip * kJacobiSkip * prod) {   // cosine of the pair above kJacobiSkip
+                off = fmax(off, g2 / prod);
+                const double z = (aqq - app) / (2.0 * gn);
                 const double t = (z >= 0.0 ? 1.0 : -1.0) / (fabs(z) + sqrt(fma(z, z, 1.0)));
-                c = 1.0 / sqrt(fma(t, t, 1.0));
+                c = rsqrt(fma(t, t, 1.0));
                 s = t * c;
             }
             const double sp = lower ? -s : s;          // own column c x + (-s or +s) partner
@@ -394,7 +428,7 @@ __device__ __forceinline__ void svd_jacobi_warp(double (&r)[kSvdRank], int lane,
 #pragma unroll
         for (int x = 16; x >= 1; x >>= 1)
             off = fmax(off, __shfl_xor_sync(kFull, off, x));
-        if (off <= kJacobiTol)
+        if (off <= kJacobiTol * kJacobiTol)            // off holds squared cosines
             break;
     }
     double s2 = 0.0;
@@ -424,15 +458,15 @@ __global__ void __launch_bounds__(256) svd_small_kernel(double *__restrict__ Gp,
     if (threadIdx.x >= 32)
         return;
     const int lane = threadIdx.x;
-    double g[kSvdRank], r[kSvdRank];
+    double g[kSvdRank], r[kSvdRank], inv = 0.0;
 #pragma unroll
     for (int i = 0; i < kSvdRank; ++i)
         g[i] = Gp[i * kSvdRank + lane];
-    const uint32_t dead = svd_chol_warp(g, r, lane, EIG ? 0.0 : 1.0);
+    const uint32_t dead = svd_chol_warp(g, r, inv, lane, EIG ? 0.0 : 1.0);
     if (EIG)
         svd_jacobi_warp(r, lane, Xo, So);
     else
-        svd_rinv_warp(r, dead, lane, Rinv);
+        svd_rinv_warp(r, inv, dead, lane, Rinv);
 }
 
 // A[row, :] <- A[row, :] Rinv (Rinv upper triangular, fp32), one row per thread, 64 rows per CTA
