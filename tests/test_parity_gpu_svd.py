@@ -123,6 +123,30 @@ def test_svd_init_ill_conditioned(sq):
     assert np.array_equal(R.view(np.uint32), Rw.view(np.uint32))
 
 
+def test_svd_init_ragged_gram_partials(sq):
+    """N = 640 and K = 1280 are not multiples of the 512-row Gram partials (the last partial of
+    each has 128 or 256 rows), and split the products 8 and 4 ways."""
+    W = gap_weight(640, 1280, 105)
+    up, down, R = run_gpu(sq, W, omega(1280, 15))
+    check_against_oracle(W, up, down, R)
+
+
+def test_svd_init_rounds_converge(sq):
+    """iters = 1, 2, 3 from the same start block: the residual is RN(W - L) of the factors bit for
+    bit every time, and the distance of L to the truncated SVD shrinks by at least 4x per round
+    (subspace iteration contracts by (sigma_33 / sigma_32)^2 <= 1/9 per round on this weight)."""
+    W = gap_weight(256, 512, 106)
+    oup, odown, _, _ = oracle.svd_init(W)
+    Lo = lowrank_product(oup, odown)
+    errs = []
+    for iters in (1, 2, 3):
+        up, down, R = run_gpu(sq, W, omega(512, 16), iters=iters)
+        Rw = oracle.svd_residual(W, up, down)
+        assert np.array_equal(R.view(np.uint32), Rw.view(np.uint32))
+        errs.append(np.linalg.norm(lowrank_product(up, down) - Lo) / np.linalg.norm(Lo))
+    assert errs[1] < errs[0] / 4 and errs[2] < errs[1] / 4, errs
+
+
 def test_svd_init_zero_weight(sq):
     W = np.zeros((128, 256), np.float32)
     up, down, R = run_gpu(sq, W, omega(256, 9), iters=2)
