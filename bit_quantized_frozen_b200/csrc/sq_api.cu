@@ -608,10 +608,17 @@ sq_status sq_selftest_wait_timeout(void *ws, uint32_t limit_us, void *stream)
 
 sq_status sq_check_device_status(void *ws, void *stream)
 {
-    if (!ws)
-        return SQ_ERR_NULL;
-    if (!aligned(ws, 256))
+    if (!ws) {                                         // the library's own word (calls without a workspace)
+        int sms = 0;
+        sq_status st = check_device(&sms);
+        if (st != SQ_OK)
+            return st;
+        uint32_t *word = nullptr;
+        SQ_CUDA(sq::library_status_word(&word), "status symbol");
+        ws = word;
+    } else if (!aligned(ws, 256)) {
         return SQ_ERR_ALIGN;
+    }
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     uint32_t word = 0;
     SQ_CUDA(cudaMemcpyAsync(&word, ws, 4, cudaMemcpyDeviceToHost, s), "status read");

@@ -1020,15 +1020,16 @@ __device__ __forceinline__ void cp_async8(uint32_t dst, const void *src, uint32_
 // NVFP4: the 16 ue4m3 block scales, gathered from the tiled layout 4 bytes at
 // a time; int8: the row's fp32 scale in the first 4 bytes), lora_up
 // [64][2 * rank B].  Rows past N are zero filled.
-template <int FMT, bool LOWRANK>
+template <int FMT, bool LOWRANK, int NT = 256>
 __device__ __forceinline__ void rec_stage(uint32_t buf, const uint8_t *codes, const void *scales, const uint16_t *U,
                                           int64_t N, int64_t K, int64_t kb, int64_t n0, int tid)
 {
     using Cfg = RecCfg<FMT>;
     constexpr int kChunksPerRow = Cfg::kCodeRow / 16;
+    static_assert(NT >= kRecRows && (kRecRows * kChunksPerRow) % NT == 0, "staging threads");
 #pragma unroll
-    for (int i = 0; i < kRecRows * kChunksPerRow / 256; ++i) {
-        const int e = tid + 256 * i;
+    for (int i = 0; i < kRecRows * kChunksPerRow / NT; ++i) {
+        const int e = tid + NT * i;
         const int r = e / kChunksPerRow, c = e % kChunksPerRow;
         const int64_t n = n0 + r;
         const uint8_t *src =
@@ -1058,17 +1059,19 @@ __device__ __forceinline__ void rec_stage(uint32_t buf, const uint8_t *codes, co
             cp_async4(sbuf + 16 * tid, src, n < N ? 4u : 0u);
         }
     } else {
-        const int r = tid >> 2, j = tid & 3;
-        const int64_t n = n0 + r;
-        const uint8_t *src = n < N ? reinterpret_cast<const uint8_t *>(scales) +
-                                         sf_offset(n, kb * (kHad / kSfBlock) + 4 * j, K / kSfBlock)
-                                   : reinterpret_cast<const uint8_t *>(scales);
-        cp_async4(sbuf + 16 * r + 4 * j, src, n < N ? 4u : 0u);
+        for (int e = tid; e < 4 * kRecRows; e += NT) {
+            const int r = e >> 2, j = e & 3;
+            const int64_t n = n0 + r;
+            const uint8_t *src = n < N ? reinterpret_cast<const uint8_t *>(scales) +
+                                             sf_offset(n, kb * (kHad / kSfBlock) + 4 * j, K / kSfBlock)
+                                       : reinterpret_cast<const uint8_t *>(scales);
+            cp_async4(sbuf + 16 * r + 4 * j, src, n < N ? 4u : 0u);
+        }
     }
     if (LOWRANK) {
         constexpr int kUChunks = Cfg::kRank / 8;     // 16-byte chunks of a lora_up row
-        if (tid < kRecRows * kUChunks) {
-            const int r = tid / kUChunks, c = tid % kUChunks;
+        for (int e = tid; e < kRecRows * kUChunks; e += NT) {
+            const int r = e / kUChunks, c = e % kUChunks;
             const int64_t n = n0 + r;
             const uint16_t *src = n < N ? U + n * Cfg::kRank + 8 * c : U;
             cp_async16(buf + Cfg::kCodeBytes + kRecScaleBytes + r * (2 * Cfg::kRank) + 16 * c, src,
@@ -1293,6 +1296,240 @@ __global__ void __launch_bounds__(256, (LOWRANK || TRANS) ? 2 : 3) reconstruct_k
         }
     }
     cp_async_wait<0>();
+}
+
+// ---------------------------------------------------------------------------
+// bf16 reconstruct with the low-rank term, warp-specialised (W, or W^T for
+// TRANS).  Same tiles, same arithmetic and same outputs as reconstruct_kernel,
+// but the two phases run in different warps of one CTA per SM and overlap:
+//   warps 0-3 (producer): stage tile i + 2 by cp.async while tile i is
+//     decoded; decode + Hadamard-transform tile i into h[i % 2] (16 rows per
+//     warp), and its lora_up rows into us[i % 2] (fp32);
+//   warps 4-11 (consumer): the rank-r fmaf chains of tile i from h[i % 2] and
+//     us[i % 2] (thread t: columns 2(t%128), +1 and rows 32(t/128)..+31, as in
+//     reconstruct_kernel), W = bf16(RN(L + h)).
+// Hand-offs are mbarriers: stage_full[s] (the producer threads' copies landed,
+// cp.async.mbarrier.arrive.noinc), stage_free[s] (the producer warps are done
+// reading stage s), h_full[b] (h and us of the tile written), h_free[b] (the
+// consumer warps are done with it).  Every wait is bounded; on a timeout the
+// CTA stops, waits for its copies in flight and sets *status.
+// ---------------------------------------------------------------------------
+constexpr int kWsP1Warps = 4;
+constexpr int kWsP2Warps = 8;
+constexpr int kWsP1Threads = 32 * kWsP1Warps;
+constexpr int kWsThreads = 32 * (kWsP1Warps + kWsP2Warps);
+
+template <int FMT>
+struct RecWsCfg {
+    using C = RecCfg<FMT>;
+    static constexpr int kUsOff = 2 * kRecHBytes;                     // h[2] at 0
+    static constexpr int kStageOff = kUsOff + 2 * C::kUsBytes;        // us[2]
+    static constexpr int kBarOff = kStageOff + 2 * C::kStageBytes;    // stage[2]
+    static constexpr int kSmem = kBarOff + 8 * 8 + 16;                // 8 mbarriers, abort flag
+};
+
+__device__ __forceinline__ void cp_async_mbar_arrive_noinc(uint32_t bar)
+{
+    asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(bar) : "memory");
+}
+
+template <int FMT, bool TRANS>
+__global__ void __launch_bounds__(kWsThreads, 1) reconstruct_ws_kernel(const uint8_t *__restrict__ codes,
+                                                                      const void *__restrict__ scales,
+                                                                      const float *__restrict__ g_w,
+                                                                      const uint16_t *__restrict__ U,
+                                                                      const uint16_t *__restrict__ D, int64_t N,
+                                                                      int64_t K, uint16_t *__restrict__ W,
+                                                                      uint32_t *__restrict__ status)
+{
+    using Cfg = RecCfg<FMT>;
+    using L = RecWsCfg<FMT>;
+    constexpr int kR = Cfg::kRank;
+    extern __shared__ __align__(128) uint8_t rec_smem[];
+    uint64_t *bars = reinterpret_cast<uint64_t *>(rec_smem + L::kBarOff);
+    const uint32_t stage_full = smem_u32(bars), stage_free = smem_u32(bars + 2);
+    const uint32_t h_full = smem_u32(bars + 4), h_free = smem_u32(bars + 6);
+    volatile uint32_t *abort_flag = reinterpret_cast<volatile uint32_t *>(bars + 8);
+    const int tid = threadIdx.x;
+    const int lane = tid & 31, warp = tid >> 5;
+    if (tid == 0) {
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(stage_full + 8 * b, kWsP1Threads);
+            mbar_init(stage_free + 8 * b, kWsP1Warps);
+            mbar_init(h_full + 8 * b, kWsP1Warps);
+            mbar_init(h_free + 8 * b, kWsP2Warps);
+        }
+        *abort_flag = 0u;
+        fence_mbar_init();
+    }
+    __syncthreads();
+    const int64_t NT = (N + kRecRows - 1) / kRecRows;
+    const int64_t T = (K / kHad) * NT;
+    const int64_t t_begin = T * blockIdx.x / gridDim.x;
+    const int n_tiles = (int)(T * (blockIdx.x + 1) / gridDim.x - t_begin);
+    if (n_tiles <= 0)
+        return;
+
+    if (warp < kWsP1Warps) {
+        // ------------------------------------------------------------ producer
+        const float g = FMT == 2 ? *g_w : 0.0f;
+        const uint32_t stage0 = smem_u32(rec_smem + L::kStageOff);
+        auto issue = [&](int i) {
+            const int64_t t = t_begin + i;
+            const int sb = i & 1;
+            rec_stage<FMT, true, kWsP1Threads>(stage0 + sb * Cfg::kStageBytes, codes, scales, U, N, K, t / NT,
+                                               (t % NT) * kRecRows, tid);
+            cp_async_mbar_arrive_noinc(stage_full + 8 * sb);
+        };
+        issue(0);
+        if (n_tiles > 1)
+            issue(1);
+        for (int i = 0; i < n_tiles; ++i) {
+            const int sb = i & 1;
+            const uint32_t par = (uint32_t)(i >> 1) & 1u;
+            if (!mbar_wait(stage_full + 8 * sb, par, abort_flag, status))
+                break;
+            if (!mbar_wait(h_free + 8 * sb, par ^ 1u, abort_flag, status))
+                break;
+            const uint8_t *st = rec_smem + L::kStageOff + sb * Cfg::kStageBytes;
+            float *h = reinterpret_cast<float *>(rec_smem + sb * kRecHBytes);
+            float *us = reinterpret_cast<float *>(rec_smem + L::kUsOff + sb * Cfg::kUsBytes);
+#pragma unroll 1
+            for (int pass = 0; pass < kRecRows / (4 * kWsP1Warps); ++pass) {
+                const int r = 4 * kWsP1Warps * pass + 4 * warp + (lane >> 3);
+                const int q = lane & 7;
+                float v[32];
+                rec_decode<FMT>(st, r, q, g, v);
+                fwht256_l32(v, lane);
+                float4 *row = reinterpret_cast<float4 *>(h + r * kHad);
+#pragma unroll
+                for (int k = 0; k < 8; ++k) {
+                    const int ff = 8 * q + k;
+                    row[ff ^ (ff >> 3)] = make_float4(v[4 * k], v[4 * k + 1], v[4 * k + 2], v[4 * k + 3]);
+                }
+            }
+            const uint16_t *ust = reinterpret_cast<const uint16_t *>(st + Cfg::kCodeBytes + kRecScaleBytes);
+#pragma unroll
+            for (int j = 0; j < kRecRows * kR / kWsP1Threads; ++j)
+                us[tid + kWsP1Threads * j] = bf16_bits_to_f32(ust[tid + kWsP1Threads * j]);
+            __syncwarp();
+            if (lane == 0) {
+                mbar_arrive(h_full + 8 * sb);
+                mbar_arrive(stage_free + 8 * sb);
+            }
+            if (i + 2 < n_tiles) {                   // every producer warp is done with stage sb
+                if (!mbar_wait(stage_free + 8 * sb, par, abort_flag, status))
+                    break;
+                issue(i + 2);
+            }
+        }
+        cp_async_wait<0>();                          // no copy lands after the CTA exits
+        return;
+    }
+
+    // ---------------------------------------------------------------- consumer
+    const int ct = tid - kWsP1Threads;
+    const int cp = ct & 127;
+    const int rbase = 32 * (ct >> 7);
+    const int f = cp >> 1;                           // float4 of h holding columns 2cp, 2cp+1
+    const int fo = 2 * (cp & 1);
+    uint64_t d2[kR];
+    int64_t cur_kb = -1;
+#pragma unroll 1
+    for (int i = 0; i < n_tiles; ++i) {
+        const int sb = i & 1;
+        const int64_t t = t_begin + i;
+        const int64_t kb = t / NT;
+        const int64_t n0 = (t % NT) * kRecRows;
+        const int64_t k0 = kb * kHad + 2 * cp;
+        if (kb != cur_kb) {                          // lora_down of this thread's two columns
+            cur_kb = kb;
+            const uint4 *dr0 = reinterpret_cast<const uint4 *>(D + k0 * kR);
+            const uint4 *dr1 = reinterpret_cast<const uint4 *>(D + (k0 + 1) * kR);
+#pragma unroll
+            for (int k = 0; k < kR / 8; ++k) {
+                const uint4 a = __ldg(dr0 + k), b = __ldg(dr1 + k);
+                const uint32_t wa[4] = {a.x, a.y, a.z, a.w}, wb[4] = {b.x, b.y, b.z, b.w};
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                    d2[8 * k + 2 * j] = pack2(bf16_bits_to_f32(wa[j] & 0xFFFFu), bf16_bits_to_f32(wb[j] & 0xFFFFu));
+                    d2[8 * k + 2 * j + 1] = pack2(bf16_bits_to_f32(wa[j] >> 16), bf16_bits_to_f32(wb[j] >> 16));
+                }
+            }
+        }
+        if (!mbar_wait(h_full + 8 * sb, (uint32_t)(i >> 1) & 1u, abort_flag, status))
+            break;
+        const float *h = reinterpret_cast<const float *>(rec_smem + sb * kRecHBytes);
+        const float *us = reinterpret_cast<const float *>(rec_smem + L::kUsOff + sb * Cfg::kUsBytes);
+        uint32_t tw0[16], tw1[16];                   // TRANS: columns k0, k0 + 1 of the 32 rows, bf16 pairs
+        constexpr int kUnroll = TRANS ? 8 : 1;       // register-indexed pieces need constant indices
+#pragma unroll kUnroll
+        for (int r0 = rbase; r0 < rbase + 32; r0 += 4) {
+            uint64_t acc[4] = {0ull, 0ull, 0ull, 0ull};
+#pragma unroll
+            for (int rr = 0; rr < kR; rr += 4) {
+                float4 u4[4];
+#pragma unroll
+                for (int j = 0; j < 4; ++j)
+                    u4[j] = *reinterpret_cast<const float4 *>(us + (r0 + j) * kR + rr);
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                    fma2(acc[j], pack2(u4[j].x, u4[j].x), d2[rr]);
+                    fma2(acc[j], pack2(u4[j].y, u4[j].y), d2[rr + 1]);
+                    fma2(acc[j], pack2(u4[j].z, u4[j].z), d2[rr + 2]);
+                    fma2(acc[j], pack2(u4[j].w, u4[j].w), d2[rr + 3]);
+                }
+            }
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                const int r = r0 + j;
+                const int64_t n = n0 + r;
+                const float2 hv = *reinterpret_cast<const float2 *>(h + r * kHad + 4 * (f ^ (f >> 3)) + fo);
+                float L0, L1;
+                unpack2(acc[j], L0, L1);
+                const float o0 = __fadd_rn(L0, hv.x);  // W = bf16(RN(L + h))
+                const float o1 = __fadd_rn(L1, hv.y);
+                if (TRANS) {
+                    const uint32_t b0 = f32_to_bf16_bits(o0), b1 = f32_to_bf16_bits(o1);
+                    const int slot = (r - rbase) >> 1, hi = (r - rbase) & 1;
+                    tw0[slot] = hi ? (tw0[slot] | (b0 << 16)) : b0;
+                    tw1[slot] = hi ? (tw1[slot] | (b1 << 16)) : b1;
+                } else if (n < N) {
+                    *reinterpret_cast<uint32_t *>(W + n * K + k0) = f32x2_to_bf16x2_bits(o0, o1);
+                }
+            }
+        }
+        __syncwarp();
+        if (lane == 0)
+            mbar_arrive(h_free + 8 * sb);              // h and us of this tile are no longer read
+        if (TRANS) {                                 // W^T [K, N]: rows k0, k0 + 1, columns n0 + rbase .. + 31
+            const int64_t nb0 = n0 + rbase;
+            if (nb0 + 32 <= N) {
+                uint4 *o0 = reinterpret_cast<uint4 *>(W + k0 * N + nb0);
+                uint4 *o1 = reinterpret_cast<uint4 *>(W + (k0 + 1) * N + nb0);
+#pragma unroll
+                for (int c = 0; c < 4; ++c) {
+                    o0[c] = make_uint4(tw0[4 * c], tw0[4 * c + 1], tw0[4 * c + 2], tw0[4 * c + 3]);
+                    o1[c] = make_uint4(tw1[4 * c], tw1[4 * c + 1], tw1[4 * c + 2], tw1[4 * c + 3]);
+                }
+            } else {
+#pragma unroll
+                for (int i2 = 0; i2 < 32; ++i2)
+                    if (nb0 + i2 < N) {
+                        W[k0 * N + nb0 + i2] = (uint16_t)(tw0[i2 >> 1] >> (16 * (i2 & 1)));
+                        W[(k0 + 1) * N + nb0 + i2] = (uint16_t)(tw1[i2 >> 1] >> (16 * (i2 & 1)));
+                    }
+            }
+        }
+    }
+}
+
+// the library's own device status word, for kernels whose call takes no workspace
+__device__ uint32_t g_library_status;
+
+cudaError_t library_status_word(uint32_t **p)
+{
+    return cudaGetSymbolAddress(reinterpret_cast<void **>(p), g_library_status);
 }
 
 // ---------------------------------------------------------------------------
@@ -1587,15 +1824,44 @@ static cudaError_t launch_reconstruct_v(const uint8_t *codes, const void *scales
     return cudaGetLastError();
 }
 
+// the warp-specialised kernel: one CTA of 384 threads per SM
+template <int FMT, bool TRANS>
+static cudaError_t launch_reconstruct_ws(const uint8_t *codes, const void *scales, const float *g_w,
+                                         const uint16_t *U, const uint16_t *D, int64_t N, int64_t K, uint16_t *W,
+                                         int sms, cudaStream_t s)
+{
+    constexpr int kSmem = RecWsCfg<FMT>::kSmem;
+    constexpr int kMaxDev = 64;
+    static bool attr_done[kMaxDev];
+    static uint32_t *status_word[kMaxDev];
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDev)
+        return cudaErrorInvalidDevice;
+    if (!attr_done[dev]) {
+        cudaError_t e = cudaFuncSetAttribute(reconstruct_ws_kernel<FMT, TRANS>,
+                                             cudaFuncAttributeMaxDynamicSharedMemorySize, kSmem);
+        if (e == cudaSuccess)
+            e = library_status_word(&status_word[dev]);
+        if (e != cudaSuccess)
+            return e;
+        attr_done[dev] = true;
+    }
+    const int64_t tiles = (K / kHad) * ((N + kRecRows - 1) / kRecRows);
+    const unsigned grid = (unsigned)(tiles < sms ? tiles : sms);
+    reconstruct_ws_kernel<FMT, TRANS><<<grid, kWsThreads, kSmem, s>>>(codes, scales, g_w, U, D, N, K, W,
+                                                                      status_word[dev]);
+    return cudaGetLastError();
+}
+
 template <int FMT>
 static cudaError_t launch_reconstruct_fmt(const uint8_t *codes, const void *scales, const float *g_w,
                                           const uint16_t *U, const uint16_t *D, int64_t N, int64_t K,
                                           int with_lowrank, int transposed, uint16_t *W, int sms, cudaStream_t s)
 {
     if (transposed)
-        return with_lowrank ? launch_reconstruct_v<FMT, true, true>(codes, scales, g_w, U, D, N, K, W, sms, s)
+        return with_lowrank ? launch_reconstruct_ws<FMT, true>(codes, scales, g_w, U, D, N, K, W, sms, s)
                             : launch_reconstruct_v<FMT, false, true>(codes, scales, g_w, U, D, N, K, W, sms, s);
-    return with_lowrank ? launch_reconstruct_v<FMT, true, false>(codes, scales, g_w, U, D, N, K, W, sms, s)
+    return with_lowrank ? launch_reconstruct_ws<FMT, false>(codes, scales, g_w, U, D, N, K, W, sms, s)
                         : launch_reconstruct_v<FMT, false, false>(codes, scales, g_w, U, D, N, K, W, sms, s);
 }
 

@@ -304,7 +304,11 @@ SQ_API sq_status sq_linear_fwd_noalloc(const sq_weight *w, const uint16_t *x, in
  *   W[n, k] = bf16(RN(L + h))          (bf16(h) with SQ_RECON_RESIDUAL_ONLY
  *                                       or NULL low-rank pointers).
  * W_out: [N, K] bf16 (device), or with SQ_RECON_TRANSPOSED the same values as
- * W^T [K, N] (the layout the backward GEMM reads).
+ * W^T [K, N] (the layout the backward GEMM reads).  With the low-rank term the
+ * kernel's producer and consumer warps hand tiles over through bounded waits;
+ * a wait that gives up (a fault of the library, never expected) stops the
+ * kernel early and sets the library's status word, which
+ * sq_check_device_status(NULL, stream) reports as SQ_ERR_TIMEOUT.
  */
 SQ_API sq_status sq_reconstruct_bf16(const sq_weight *w, uint16_t *W_out, uint32_t flags,
                               void *stream);
@@ -334,10 +338,12 @@ SQ_API sq_status sq_linear_bwd_dx(const sq_weight *w, const uint16_t *dy, int64_
 SQ_API sq_status sq_set_gemm_events(void *start_event, void *stop_event);
 
 /*
- * Read back and clear the device status word that a forward kernel sets when
- * it gives up a bounded wait (SQ_ERR_TIMEOUT); ws is the workspace of the
- * sq_linear_fwd call to check (each such call clears the word when it
- * starts).  This call synchronises `stream` and copies 4 bytes to the host.
+ * Read back and clear the device status word that a kernel sets when it gives
+ * up a bounded wait (SQ_ERR_TIMEOUT); ws is the workspace of the sq_linear_fwd
+ * call to check (each such call clears the word when it starts).  With ws ==
+ * NULL it reads the library's own word on the current device, which the calls
+ * without a workspace (sq_reconstruct_bf16) set instead.  This call
+ * synchronises `stream` and copies 4 bytes to the host.
  */
 SQ_API sq_status sq_check_device_status(void *ws, void *stream);
 
