@@ -170,6 +170,9 @@ def test_valid_call_without_device_reports_device_error():
     assert sq.lib().sq_reconstruct_bf16(ctypes.byref(_w(fmt=sq.SQ_FMT_INT4_G64, g_w=None)), A, 0, None) \
         == SQ_ERR_DEVICE
     assert sq.lib().sq_reconstruct_bf16(ctypes.byref(_w()), A, 0, None) == SQ_ERR_DEVICE
+    # the library's own status word (ws == NULL) needs a device too
+    assert sq.lib().sq_check_device_status(None, None) == SQ_ERR_DEVICE
+    assert sq.lib().sq_check_device_status(MIS, None) == SQ_ERR_ALIGN
 
 
 def test_selftest_validation():

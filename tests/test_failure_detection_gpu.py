@@ -36,3 +36,17 @@ def test_bounded_wait_reports_timeout_and_context_survives():
     xc, xsf, gx, t = oracle.act_quant_nvfp4(d["x"], d["D"])
     ref = oracle.linear_fwd_nvfp4(xc, xsf, gx, wc, wsf, gw, t, d["U"], 64, 256, 512)
     assert norm_err(host(y), ref) <= FWD_TOL
+
+
+def test_library_status_word_clear_after_reconstruct():
+    """sq_reconstruct_bf16 takes no workspace: its pipelined kernel reports a wait that gave up
+    through the library's own status word, read with sq_check_device_status(NULL). After normal
+    reconstructs (W and W^T) the word is clear."""
+    import bit_quantized_frozen_b200 as sq
+    assert torch.cuda.is_available()
+    d = si.make_inputs(8, 512, 384, 72)
+    w = sq.build_nvfp4(to_dev(d["R"]), bf16_dev(d["U"]), bf16_dev(d["D"]))
+    sq.reconstruct_bf16(w)
+    sq.reconstruct_bf16(w, transposed=True)
+    torch.cuda.synchronize()
+    sq.sq_check_device_status(None)
