@@ -177,3 +177,33 @@ def test_svd_init_large(sq):
     W = gap_weight(4096, 2048, 103)
     up, down, R = run_gpu(sq, W, omega(2048, 13))
     check_against_oracle(W, up, down, R, rows=np.array([0, 1, 2048, 4095]))
+
+
+@pytest.mark.slow
+def test_svd_init_bench_shape_properties(sq):
+    """The bench workload's full weight W = U D^T + R (16384 x 6144, no spectral gap, 8 rounds):
+    properties that hold at any size.  R is RN(W - L) bit for bit on sampled rows; the factors'
+    columns are orthogonal with up^T up = down^T down = diag(sigma) in descending order (the even
+    split), up to the bf16 rounding of the factors."""
+    d = si.make_config("large_4480x16384x6144")
+    U = torch.from_numpy(d["U"].view(np.int16)).cuda().view(torch.bfloat16)
+    D = torch.from_numpy(d["D"].view(np.int16)).cuda().view(torch.bfloat16)
+    W = torch.from_numpy(d["R"]).cuda() + U.float() @ D.float().T
+    up, down, R = sq.svd_init(W, to_dev(omega(W.shape[1], 17)), 8)
+    torch.cuda.synchronize()
+    up_b, down_b = bits16(up), bits16(down)
+    rows = np.array([0, 1, 8191, 16383])
+    Wr = W[rows].cpu().numpy()
+    Rr = R[rows].cpu().numpy()
+    Rw = oracle.svd_residual(Wr, up_b[rows], down_b)
+    assert np.array_equal(Rr.view(np.uint32), Rw.view(np.uint32)), first_mismatch(Rr, Rw)
+    for f in (up_b, down_b):
+        F = si.bf16_bits_to_f32(f).astype(np.float64)
+        G = F.T @ F
+        dg = np.sqrt(np.diag(G))
+        assert np.all(np.diff(np.diag(G)) <= 1e-2 * np.diag(G)[:-1])          # descending
+        off = np.abs(G / np.outer(dg, dg) - np.eye(32)).max()
+        assert off <= 1e-2, off
+    su = np.diag(si.bf16_bits_to_f32(up_b).astype(np.float64).T @ si.bf16_bits_to_f32(up_b).astype(np.float64))
+    sd = np.diag(si.bf16_bits_to_f32(down_b).astype(np.float64).T @ si.bf16_bits_to_f32(down_b).astype(np.float64))
+    assert np.allclose(su, sd, rtol=1e-2)
