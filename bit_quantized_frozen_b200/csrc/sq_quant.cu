@@ -428,7 +428,7 @@ constexpr int kI8MaxK = 16384;
 
 __host__ __device__ constexpr int i8_smem_bytes(int K)
 {
-    return K * 4 + kFracCount * (K / kHad) * 4 + 2 * kFracCount * 4 + 64;
+    return K * 4 + kFracCount * (K / kHad) * 4 + 3 * kFracCount * 4 + 64;
 }
 
 __device__ __forceinline__ int i8_slot(int block, int q, int c)   // float4 index in the shared row
@@ -446,7 +446,8 @@ __global__ void __launch_bounds__(kI8Threads) int8_build_kernel(const float *__r
     float *berr = reinterpret_cast<float *>(i8_smem + K * 4);                  // [26][nb] block errors
     float *stab = berr + kFracCount * (K / kHad);                              // [26] scales, [26] errors
     float *etab = stab + kFracCount;
-    float *red = etab + kFracCount;                                            // [8] warp maxima, choice
+    float *itab = etab + kFracCount;                                           // [26] RN(1 / scale)
+    float *red = itab + kFracCount;                                            // [8] warp maxima, choice
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int q = lane & 7;
     const int grp = tid >> 3;                                                  // 8-lane group, 0..31
@@ -490,7 +491,9 @@ __global__ void __launch_bounds__(kI8Threads) int8_build_kernel(const float *__r
             float m = 0.0f;
             for (int w = 0; w < kI8Threads / 32; ++w)
                 m = fmaxf(m, red[w]);
-            stab[tid] = __fdiv_rn(__fmul_rn(kFrac[tid], m), 127.0f);
+            const float sj = __fdiv_rn(__fmul_rn(kFrac[tid], m), 127.0f);
+            stab[tid] = sj;
+            itab[tid] = sj == 0.0f ? 0.0f : __frcp_rn(sj);
         }
         __syncthreads();
         // sweep: per block and fraction, the block's error
@@ -506,8 +509,7 @@ __global__ void __launch_bounds__(kI8Threads) int8_build_kernel(const float *__r
             }
 #pragma unroll 1
             for (int j = 0; j < kFracCount; ++j) {
-                const float sj = stab[j];
-                const float inv = sj == 0.0f ? 0.0f : __frcp_rn(sj);
+                const float sj = stab[j], inv = itab[j];
                 float e = group_sq_error<127>(rp, sj, inv);
                 e = __fadd_rn(e, __shfl_xor_sync(0xffffffffu, e, 4));
                 e = __fadd_rn(e, __shfl_xor_sync(0xffffffffu, e, 2));
