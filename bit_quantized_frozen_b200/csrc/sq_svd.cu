@@ -642,15 +642,6 @@ static int64_t max64(int64_t a, int64_t b)
     return a > b ? a : b;
 }
 
-size_t svd_workspace_bytes(int64_t N, int64_t K)
-{
-    const int64_t rows = max64(N, K);
-    return up256((size_t)N * kSvdRank * 4) + up256((size_t)K * kSvdRank * 4) +
-           up256((size_t)kSvdMaxSplits * rows * kSvdRank * 4) +
-           up256((size_t)((rows + kGramRows - 1) / kGramRows) * kSvdRank * kSvdRank * 8) +
-           up256(kSvdRank * kSvdRank * 4) + up256(kSvdRank * kSvdRank * 8) + up256(kSvdRank * 8);
-}
-
 // splits s in {1, 2, 4, 8, 16} of the reduction dimension `depth` (each part a multiple of 32
 // deep) until the grid of `tiles` x s CTAs reaches the target
 static int svd_splits(int64_t tiles, int64_t depth)
@@ -659,6 +650,21 @@ static int svd_splits(int64_t tiles, int64_t depth)
     while (s < kSvdMaxSplits && tiles * s < kSvdTargetCtas && depth % (kSvdChunk * 2 * s) == 0)
         s *= 2;
     return s;
+}
+
+// rows of the split partials: the larger of the two products' splits x rows
+static int64_t svd_partial_rows(int64_t N, int64_t K)
+{
+    return max64(svd_splits(N / kSvdTile, K) * N, svd_splits(K / kSvdTile, N) * K);
+}
+
+size_t svd_workspace_bytes(int64_t N, int64_t K)
+{
+    const int64_t rows = max64(N, K);
+    return up256((size_t)N * kSvdRank * 4) + up256((size_t)K * kSvdRank * 4) +
+           up256((size_t)svd_partial_rows(N, K) * kSvdRank * 4) +
+           up256((size_t)((rows + kGramRows - 1) / kGramRows) * kSvdRank * kSvdRank * 8) +
+           up256(kSvdRank * kSvdRank * 4) + up256(kSvdRank * kSvdRank * 8) + up256(kSvdRank * 8);
 }
 
 struct SvdWs {
@@ -712,7 +718,7 @@ cudaError_t launch_svd_init(const float *W, int64_t N, int64_t K, const float *o
     w.V = reinterpret_cast<float *>(p);
     p += up256((size_t)K * kSvdRank * 4);
     w.P = reinterpret_cast<float *>(p);
-    p += up256((size_t)kSvdMaxSplits * rows * kSvdRank * 4);
+    p += up256((size_t)svd_partial_rows(N, K) * kSvdRank * 4);
     w.Gp = reinterpret_cast<double *>(p);
     p += up256((size_t)((rows + kGramRows - 1) / kGramRows) * kSvdRank * kSvdRank * 8);
     w.Rinv = reinterpret_cast<float *>(p);
