@@ -96,3 +96,24 @@ def test_bwd_dx_proj_sampled(sq):
     rng = np.random.default_rng(65)
     rows = np.unique(np.concatenate([[0, 1535], rng.choice(1536, 30, replace=False)])).astype(np.int64)
     check_dx(sq, d, "nvfp4", M=1536, rows=rows)
+
+
+@pytest.mark.slow
+def test_bwd_bench_shape_sampled(sq):
+    """The bench workload 4480 x 16384 x 6144 (NVFP4 payload, as the bench times it): W^T bit
+    for bit on sampled rows, dx within tolerance on sampled rows."""
+    d = si.make_config("large_4480x16384x6144")
+    M = d["x"].shape[0]
+    w, Wo = weight_and_oracle_W(sq, d, "nvfp4")
+    Wt = sq.reconstruct_bf16(w, transposed=True)
+    rng = np.random.default_rng(66)
+    dy = si.to_bf16_bits(rng.standard_normal((M, Wo.shape[0])).astype(np.float32))
+    dx = sq.linear_bwd_dx(w, bf16_dev(dy))
+    torch.cuda.synchronize()
+    krows = np.unique(np.concatenate([[0, Wo.shape[1] - 1], rng.choice(Wo.shape[1], 24, replace=False)]))
+    got = bits16(Wt)[krows]
+    want = np.ascontiguousarray(Wo[:, krows].T)
+    assert np.array_equal(got, want), first_mismatch(got, want)
+    rows = np.unique(np.concatenate([[0, M - 1], rng.choice(M, 6, replace=False)])).astype(np.int64)
+    err = norm_err(host(dx)[rows], oracle.linear_bwd_dx(dy, Wo, rows))
+    assert err <= FWD_TOL, f"normalised error {err:.3e}"

@@ -123,3 +123,14 @@ def test_reconstruct_g64(sq, name):
 
 def test_reconstruct_g64_residual_only_ragged(sq):
     check_reconstruct(sq, si.make_inputs(8, 768, 384, 45), residual_only=True)
+
+
+@pytest.mark.slow
+def test_large_g64_sampled(sq):
+    """The bench workload 4480 x 16384 x 6144: builder on sampled rows, forward on sampled
+    outputs, the whole reconstruct bit for bit."""
+    d = inputs("large_4480x16384x6144")
+    N = d["R"].shape[0]
+    check_build(sq, d["R"], sample_rows(N, 48, 46))
+    check_fwd(sq, d, sample_rows(d["x"].shape[0], 6, 47))
+    check_reconstruct(sq, d)
