@@ -74,7 +74,7 @@ _SIGS = {
     "or_linear_fwd_int8": ([_P, _P, _P, _P, _P, _I64, _I64, _I64, _P, _I64, _P], None),
     "or_lowrank_input": ([_P, _I64, _I64, _P, ctypes.c_int, _P], None),
     "or_linear_bwd_dx": ([_P, _P, _I64, _I64, _I64, _P, _I64, _P], None),
-    "or_svd_residual": ([_P, _P, _P, _I64, _I64, _P], None),
+    "or_svd_residual": ([_P, _P, _P, _I64, _I64, ctypes.c_int, _P], None),
     "or_f32_to_bf16_n": ([_P, _I64, _P], None),
 }
 
@@ -380,11 +380,15 @@ def linear_bwd_dx(dy_bits, W_bits, rows=None):
 # ---- SVD init of the low-rank branch ("Low-rank branch: rank-32 SVD of the weight") ----
 
 def svd_residual(W, up_bits, down_bits):
-    """R = RN(W - L), L the rank-32 fmaf chain of bf16 up [N, 32] and down [K, 32] (as the reconstruct)."""
+    """R = RN(W - L), L the fmaf chain over the factors' rank (32, or 16 for the int8 mode) of bf16
+    up [N, rank] and down [K, rank] (as the reconstruct)."""
     W = _c(W, np.float32)
     N, K = W.shape
+    up = _c(up_bits, np.uint16)
+    rank = up.shape[1]
+    assert rank in (16, 32) and _c(down_bits, np.uint16).shape[1] == rank
     R = np.empty((N, K), np.float32)
-    lib().or_svd_residual(_p(W), _p(_c(up_bits, np.uint16)), _p(_c(down_bits, np.uint16)), N, K, _p(R))
+    lib().or_svd_residual(_p(W), _p(up), _p(_c(down_bits, np.uint16)), N, K, rank, _p(R))
     return R
 
 

@@ -1015,24 +1015,25 @@ void or_linear_bwd_dx(const uint16_t *dy, const uint16_t *W, int64_t M, int64_t 
 }
 
 /* ------------------------------------------------------------------------ */
-/* SVD init: residual of the rank-32 branch                                 */
+/* SVD init: residual of the low-rank branch                                */
 /* ------------------------------------------------------------------------ */
 
 /*
- * R[n, k] = RN(W[n, k] - L[n, k]) with L the rank-32 fmaf chain over r = 0..31
- * of up[n, r] * down[k, r] from 0 -- the same L the bf16 reconstruct adds back
+ * R[n, k] = RN(W[n, k] - L[n, k]) with L the fmaf chain over r = 0..rank-1 of
+ * up[n, r] * down[k, r] from 0 -- the same L the bf16 reconstruct adds back
  * (SquareQ README, "Low-rank branch: rank-32 SVD of the weight": the residual
- * is the weight minus the low-rank branch).  W, R fp32 [N, K]; up [N, 32],
- * down [K, 32] bf16 bits.
+ * is the weight minus the low-rank branch; "v3.1 -- int8-residual mode": rank
+ * 16).  W, R fp32 [N, K]; up [N, rank], down [K, rank] bf16 bits; rank 32 or 16.
  */
-void or_svd_residual(const float *W, const uint16_t *up, const uint16_t *down, int64_t N, int64_t K, float *R)
+void or_svd_residual(const float *W, const uint16_t *up, const uint16_t *down, int64_t N, int64_t K, int rank,
+                     float *R)
 {
 #pragma omp parallel for schedule(static)
     for (int64_t n = 0; n < N; n++) {
         for (int64_t k = 0; k < K; k++) {
             float L = 0.0f;
-            for (int r = 0; r < 32; r++)
-                L = fmaf(or_bf16_to_f32(up[n * 32 + r]), or_bf16_to_f32(down[k * 32 + r]), L);
+            for (int r = 0; r < rank; r++)
+                L = fmaf(or_bf16_to_f32(up[n * rank + r]), or_bf16_to_f32(down[k * rank + r]), L);
             R[n * K + k] = W[n * K + k] - L;
         }
     }

@@ -60,3 +60,31 @@ def test_svd_init_exact_rank_32(oracle_mod):
     up, down, R, S = oracle_mod.svd_init(W)
     assert np.linalg.norm(R) <= 2 * 2.0 ** -8 * np.linalg.norm(W)
     assert np.linalg.norm(R) >= 1e-6 * np.linalg.norm(W)      # the bf16 rounding is there
+
+
+def test_svd_init_rank16_is_the_int8_modes_branch(oracle_mod):
+    """Rank 16 (the int8 mode's branch): the factors are the first 16 columns of the rank-32
+    factors (the same singular pairs), the residual's tail energy is that beyond sigma_16, and
+    W - R is the rank-16 fmaf chain that the int8 reconstruct adds back."""
+    W = lowrank_weight(192, 512, 94)
+    up32, down32, _, S32 = oracle_mod.svd_init(W)
+    up, down, R, S = oracle_mod.svd_init(W, rank=16)
+    assert up.shape == (192, 16) and down.shape == (512, 16)
+    assert np.array_equal(up, up32[:, :16]) and np.array_equal(down, down32[:, :16])
+    assert np.array_equal(S, S32[:16])
+    sig = np.linalg.svd(W.astype(np.float64), compute_uv=False)
+    tail = np.sqrt((sig[16:] ** 2).sum())
+    U = si.bf16_bits_to_f32(up).astype(np.float64)
+    D = si.bf16_bits_to_f32(down).astype(np.float64)
+    L = U @ D.T
+    rn = np.linalg.norm(R.astype(np.float64))
+    assert rn >= tail * (1 - 1e-9)
+    assert rn <= np.sqrt(tail ** 2 + (2 * 2.0 ** -8 * np.linalg.norm(L)) ** 2)
+    bound = 16 * 2.0 ** -24 * (np.abs(U) @ np.abs(D).T) + 2.0 ** -24 * np.abs(W)
+    assert np.all(np.abs((W.astype(np.float64) - R) - L) <= bound + 1e-30)
+    # the chain is the int8 reconstruct's: the residual of a zero weight is -L exactly, and zero
+    # codes reconstruct to bf16(L), bit for bit
+    R0 = oracle_mod.svd_residual(np.zeros((192, 512), np.float32), up, down)
+    Wz = oracle_mod.reconstruct_bf16(oracle_mod.FMT_INT8_ROW, np.zeros((192, 512), np.int8),
+                                     np.zeros(192, np.float32), 0.0, up, down, 192, 512)
+    assert np.array_equal(Wz, si.to_bf16_bits(-R0))
