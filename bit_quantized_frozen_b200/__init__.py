@@ -83,7 +83,8 @@ _SIGS = {
     "sq_workspace_bytes": ([ctypes.c_int, _I64, _I64, _I64], ctypes.c_size_t),
     "sq_build_int4": ([_P, _I64, _I64, ctypes.c_int32, _P, _P, _P, _P], ctypes.c_int),
     "sq_build_int8": ([_P, _I64, _I64, _P, _P, _P, _P], ctypes.c_int),
-    "sq_svd_init": ([_P, _I64, _I64, _P, ctypes.c_int32, _P, _P, _P, _P, ctypes.c_size_t, _P], ctypes.c_int),
+    "sq_svd_init": ([_P, _I64, _I64, _P, ctypes.c_int32, ctypes.c_int32, _P, _P, _P, _P, ctypes.c_size_t, _P],
+                    ctypes.c_int),
     "sq_build_nvfp4": ([_P, _I64, _I64, _P, _P, _P, _P, ctypes.c_size_t, _P], ctypes.c_int),
     "sq_act_quant_nvfp4": ([_P, _I64, _I64, _P, _P, _P, _P, _P, ctypes.c_uint32, _P, ctypes.c_size_t, _P],
                            ctypes.c_int),
@@ -170,9 +171,11 @@ def sq_build_int4(R, codes, scales, frac_idx=None, group: int = 32, stream=None)
 
 
 def sq_svd_init(W, omega, iters, lora_up, lora_down, R, ws, stream=None):
+    """The rank (32 or 16) is lora_up's number of columns."""
     N, K = W.shape
-    _check("sq_svd_init", lib().sq_svd_init(_ptr(W), N, K, _ptr(omega), int(iters), _ptr(lora_up), _ptr(lora_down),
-                                            _ptr(R), _ptr(ws), _numel_bytes(ws), _stream(stream)))
+    rank = int(lora_up.shape[1])
+    _check("sq_svd_init", lib().sq_svd_init(_ptr(W), N, K, _ptr(omega), int(iters), rank, _ptr(lora_up),
+                                            _ptr(lora_down), _ptr(R), _ptr(ws), _numel_bytes(ws), _stream(stream)))
 
 
 def sq_build_int8(R, codes, scales, frac_idx=None, stream=None):
@@ -301,12 +304,13 @@ def build_nvfp4(R: torch.Tensor, lora_up=None, lora_down=None, ws=None, stream=N
     return Weight(SQ_FMT_NVFP4, N, K, codes, sf, g, lora_up, lora_down)
 
 
-def svd_init(W: torch.Tensor, omega: torch.Tensor, iters: int = 8, stream=None):
-    """(lora_up bf16 [N, 32], lora_down bf16 [K, 32], R fp32 [N, K]) of W [N, K] fp32."""
+def svd_init(W: torch.Tensor, omega: torch.Tensor, iters: int = 8, rank: int = RANK, stream=None):
+    """(lora_up bf16 [N, rank], lora_down bf16 [K, rank], R fp32 [N, K]) of W [N, K] fp32; rank 32,
+    or 16 (RANK_INT8) for the int8 mode."""
     N, K = W.shape
     dev = W.device
-    up = torch.empty((N, RANK), dtype=torch.bfloat16, device=dev)
-    down = torch.empty((K, RANK), dtype=torch.bfloat16, device=dev)
+    up = torch.empty((N, rank), dtype=torch.bfloat16, device=dev)
+    down = torch.empty((K, rank), dtype=torch.bfloat16, device=dev)
     R = torch.empty((N, K), dtype=torch.float32, device=dev)
     ws = workspace(SQ_OP_SVD_INIT, 0, N, K, dev)
     sq_svd_init(W, omega, iters, up, down, R, ws, stream=stream)

@@ -277,14 +277,14 @@ sq_status sq_build_int8(const float *R, int64_t N, int64_t K, int8_t *codes, flo
     return SQ_OK;
 }
 
-sq_status sq_svd_init(const float *W, int64_t N, int64_t K, const float *omega, int32_t iters, uint16_t *lora_up,
-                      uint16_t *lora_down, float *R, void *ws, size_t ws_bytes, void *stream)
+sq_status sq_svd_init(const float *W, int64_t N, int64_t K, const float *omega, int32_t iters, int32_t rank,
+                      uint16_t *lora_up, uint16_t *lora_down, float *R, void *ws, size_t ws_bytes, void *stream)
 {
     if (!W || !omega || !lora_up || !lora_down || !R || !ws)
         return SQ_ERR_NULL;
     if (!shape_ok_nk(N, K))
         return SQ_ERR_SHAPE;
-    if (iters < 1 || iters > 100)
+    if (iters < 1 || iters > 100 || (rank != 16 && rank != 32))
         return SQ_ERR_ARG;
     if (!aligned(W, 16) || !aligned(omega, 16) || !aligned(lora_up, 16) || !aligned(lora_down, 16) ||
         !aligned(R, 16) || !aligned(ws, 256))
@@ -297,7 +297,8 @@ sq_status sq_svd_init(const float *W, int64_t N, int64_t K, const float *omega, 
         return st;
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     const char *stage = "svd init";
-    const cudaError_t e = sq::launch_svd_init(W, N, K, omega, iters, lora_up, lora_down, R, ws, sms, s, &stage);
+    const cudaError_t e =
+        sq::launch_svd_init(W, N, K, omega, iters, rank, lora_up, lora_down, R, ws, sms, s, &stage);
     if (e != cudaSuccess) {
         set_detail(stage, e);
         return SQ_ERR_CUDA;

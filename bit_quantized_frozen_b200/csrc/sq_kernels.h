@@ -52,11 +52,13 @@ cudaError_t launch_reconstruct(int fmt, const uint8_t *codes, const void *scales
                                const uint16_t *U, const uint16_t *D, int64_t N, int64_t K, int with_lowrank,
                                int transposed, uint16_t *W, int sms, cudaStream_t s);
 
-// SVD init of the rank-32 branch (sq_svd.cu): omega [K, 32] fp32 start block; on an error
-// *stage names the launch that reported it
+// SVD init of the low-rank branch (sq_svd.cu): omega [K, 32] fp32 start block, output rank 32
+// or 16 (up [N, rank], down [K, rank], R with the rank-r chain); on an error *stage names the
+// launch that reported it
 size_t svd_workspace_bytes(int64_t N, int64_t K);
-cudaError_t launch_svd_init(const float *W, int64_t N, int64_t K, const float *omega, int iters, uint16_t *up,
-                            uint16_t *down, float *R, void *ws, int sms, cudaStream_t s, const char **stage);
+cudaError_t launch_svd_init(const float *W, int64_t N, int64_t K, const float *omega, int iters, int rank,
+                            uint16_t *up, uint16_t *down, float *R, void *ws, int sms, cudaStream_t s,
+                            const char **stage);
 
 // forward GEMM y = beta (A B^T + tsplit udup^T), see sq_gemm.cu
 struct GemmLaunch {

@@ -503,7 +503,9 @@ __global__ void __launch_bounds__(64) svd_apply_kernel(float *__restrict__ A, in
 
 // up[n, :] = bf16(U[n, :] X S^(1/4)) for rows n < N, then down[k, :] = bf16(B[k, :] X S^(-1/4))
 // for the next K rows (S = eigenvalues of B^T B = sigma^2, so S^(1/4) = sigma^(1/2)); a zero
-// sigma gives a zero column of down.  One row per thread.
+// sigma gives a zero column of down.  Only the first RO columns (the RO largest sigma) are
+// written: up [N, RO], down [K, RO].  One row per thread.
+template <int RO>
 __global__ void __launch_bounds__(256) svd_factors_kernel(const float *__restrict__ U, const float *__restrict__ B,
                                                           int64_t N, int64_t K, const double *__restrict__ Xd,
                                                           const double *__restrict__ Sd, uint16_t *__restrict__ up,
@@ -525,14 +527,14 @@ __global__ void __launch_bounds__(256) svd_factors_kernel(const float *__restric
         return;
     const bool is_up = row < N;
     const float *src = is_up ? U + row * kSvdRank : B + (row - N) * kSvdRank;
-    uint16_t *dst = is_up ? up + row * kSvdRank : down + (row - N) * kSvdRank;
+    uint16_t *dst = is_up ? up + row * RO : down + (row - N) * RO;
     const float *sc = is_up ? sc_up : sc_down;
     float a[kSvdRank];
 #pragma unroll
     for (int i = 0; i < kSvdRank; ++i)
         a[i] = src[i];
 #pragma unroll
-    for (int j = 0; j < kSvdRank; ++j) {
+    for (int j = 0; j < RO; ++j) {
         float s = 0.0f;
 #pragma unroll
         for (int i = 0; i < kSvdRank; ++i)
@@ -542,8 +544,8 @@ __global__ void __launch_bounds__(256) svd_factors_kernel(const float *__restric
 }
 
 // ---------------------------------------------------------------------------
-// R[n, k] = RN(W[n, k] - L[n, k]), L = fmaf chain over r = 0..31 of up[n, r] down[k, r] from 0
-// (the reconstruct's chain).  Grid (K / 256, m): CTA (kb, j) owns columns 256 kb .. +255 and the
+// R[n, k] = RN(W[n, k] - L[n, k]), L = fmaf chain over r = 0..RO-1 of up[n, r] down[k, r] from 0
+// (the reconstruct's chain; RO = 32, or 16 for the int8 mode).  Grid (K / 256, m): CTA (kb, j) owns columns 256 kb .. +255 and the
 // 64-row tiles j, j + m, ... .  Thread t owns columns 256 kb + 2 (t % 128) and +1 (both chains
 // advance in one fma.rn.f32x2: two independent fmaf roundings) of rows 32 (t / 128) .. +31 of each
 // tile; lora_down of its two columns is staged once (coalesced, through shared memory) and stays
@@ -562,37 +564,39 @@ __device__ __forceinline__ void svd_bf16x8(const uint4 v, float (&f)[8])
 
 constexpr int kResRows = 8;            // rows of W whose loads a residual thread keeps in flight
 
+template <int RO>
 __global__ void __launch_bounds__(256, 2) svd_residual_kernel(const float *W, int64_t N, int64_t K,
                                                            const uint16_t *__restrict__ up,
                                                            const uint16_t *__restrict__ down, float *R)
 {
-    __shared__ float ds[256][kSvdRank + 1];
-    __shared__ __align__(16) float us[64 * kSvdRank];
+    constexpr int kPieces = RO / 8;                    // 16-byte pieces of a factor row
+    __shared__ float ds[256][RO + 1];
+    __shared__ __align__(16) float us[64 * RO];
     const int tid = threadIdx.x;
     const int cp = tid & 127, rbase = 32 * (tid >> 7);
     const int64_t k = (int64_t)blockIdx.x * 256 + 2 * cp;
-    const uint4 *dsrc = reinterpret_cast<const uint4 *>(down + (int64_t)blockIdx.x * 256 * kSvdRank);
+    const uint4 *dsrc = reinterpret_cast<const uint4 *>(down + (int64_t)blockIdx.x * 256 * RO);
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {                      // 256 columns x 32 bf16 = 1024 16-byte pieces
+    for (int i = 0; i < kPieces; ++i) {                // 256 columns x RO bf16
         const int e = tid + 256 * i;
         float f[8];
         svd_bf16x8(dsrc[e], f);
 #pragma unroll
         for (int q = 0; q < 8; ++q)
-            ds[e >> 2][8 * (e & 3) + q] = f[q];
+            ds[e / kPieces][8 * (e % kPieces) + q] = f[q];
     }
     __syncthreads();
-    uint64_t d2[kSvdRank];
+    uint64_t d2[RO];
 #pragma unroll
-    for (int r = 0; r < kSvdRank; ++r)
+    for (int r = 0; r < RO; ++r)
         d2[r] = svd_pack2(ds[2 * cp][r], ds[2 * cp + 1][r]);
     const int64_t NT = N / 64;
     for (int64_t nt = blockIdx.y; nt < NT; nt += gridDim.y) {
         const int64_t n0 = nt * 64;
         __syncthreads();                               // the previous tile's reads of us are done
-        {                                              // 64 rows x 32 bf16 = 256 16-byte pieces
+        if (tid < 64 * kPieces) {                      // 64 rows x RO bf16
             float f[8];
-            svd_bf16x8(reinterpret_cast<const uint4 *>(up + n0 * kSvdRank)[tid], f);
+            svd_bf16x8(reinterpret_cast<const uint4 *>(up + n0 * RO)[tid], f);
             *reinterpret_cast<float4 *>(&us[8 * tid]) = make_float4(f[0], f[1], f[2], f[3]);
             *reinterpret_cast<float4 *>(&us[8 * tid + 4]) = make_float4(f[4], f[5], f[6], f[7]);
         }
@@ -607,10 +611,10 @@ __global__ void __launch_bounds__(256, 2) svd_residual_kernel(const float *W, in
             for (int i = 0; i < kResRows; ++i)
                 acc[i] = 0ull;
 #pragma unroll
-            for (int r4 = 0; r4 < kSvdRank; r4 += 4) {
+            for (int r4 = 0; r4 < RO; r4 += 4) {
 #pragma unroll
                 for (int i = 0; i < kResRows; ++i) {
-                    const float4 u = *reinterpret_cast<const float4 *>(&us[(nb + i) * kSvdRank + r4]);
+                    const float4 u = *reinterpret_cast<const float4 *>(&us[(nb + i) * RO + r4]);
                     const float uv[4] = {u.x, u.y, u.z, u.w};
 #pragma unroll
                     for (int q = 0; q < 4; ++q)
@@ -707,8 +711,9 @@ static cudaError_t svd_sum(const float *P, int splits, int64_t rows, float *out,
     return cudaSuccess;
 }
 
-cudaError_t launch_svd_init(const float *W, int64_t N, int64_t K, const float *omega, int iters, uint16_t *up,
-                            uint16_t *down, float *R, void *ws, int sms, cudaStream_t s, const char **stage)
+cudaError_t launch_svd_init(const float *W, int64_t N, int64_t K, const float *omega, int iters, int rank,
+                            uint16_t *up, uint16_t *down, float *R, void *ws, int sms, cudaStream_t s,
+                            const char **stage)
 {
     const int64_t rows = max64(N, K);
     uint8_t *p = reinterpret_cast<uint8_t *>(ws);
@@ -754,12 +759,18 @@ cudaError_t launch_svd_init(const float *W, int64_t N, int64_t K, const float *o
     SVD_STEP("svd gram");
     svd_small_kernel<true><<<1, 256, 0, s>>>(w.Gp, CK, nullptr, w.X, w.S);
     SVD_STEP("svd jacobi");
-    svd_factors_kernel<<<(unsigned)((N + K + 255) / 256), 256, 0, s>>>(w.Y, w.V, N, K, w.X, w.S, up, down);
+    if (rank == 16)
+        svd_factors_kernel<16><<<(unsigned)((N + K + 255) / 256), 256, 0, s>>>(w.Y, w.V, N, K, w.X, w.S, up, down);
+    else
+        svd_factors_kernel<32><<<(unsigned)((N + K + 255) / 256), 256, 0, s>>>(w.Y, w.V, N, K, w.X, w.S, up, down);
     SVD_STEP("svd factors");
     const int64_t kbs = K / 256, nts = N / 64;
     int64_t m = ((int64_t)sms * 2) / kbs;              // one wave of two CTAs per SM
     m = m < 1 ? 1 : (m > nts ? nts : m);
-    svd_residual_kernel<<<dim3((unsigned)kbs, (unsigned)m), 256, 0, s>>>(W, N, K, up, down, R);
+    if (rank == 16)
+        svd_residual_kernel<16><<<dim3((unsigned)kbs, (unsigned)m), 256, 0, s>>>(W, N, K, up, down, R);
+    else
+        svd_residual_kernel<32><<<dim3((unsigned)kbs, (unsigned)m), 256, 0, s>>>(W, N, K, up, down, R);
     SVD_STEP("svd residual");
     return cudaSuccess;
 }

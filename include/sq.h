@@ -161,31 +161,32 @@ SQ_API sq_status sq_build_int4(const float *R, int64_t N, int64_t K, int32_t gro
 
 /*
  * SVD init of the low-rank branch (SquareQ README, "Low-rank branch: rank-32
- * SVD of the weight, always on, bf16"): the step before the builders.  From W
- * [N, K] fp32 (device) it writes lora_up = bf16(U sqrt(sigma)) [N, 32],
- * lora_down = bf16(V sqrt(sigma)) [K, 32] for the 32 largest singular values
- * sigma (an even split between the factors), and the residual
- *   R[n, k] = RN(W[n, k] - L[n, k]),  L = fmaf chain of the bf16 factors as in
- *   sq_reconstruct_bf16,
+ * SVD of the weight, always on, bf16"; "v3.1 -- int8-residual mode": rank 16):
+ * the step before the builders.  From W [N, K] fp32 (device) it writes, for
+ * the `rank` (32, or 16 for SQ_FMT_INT8_ROW) largest singular values sigma,
+ * lora_up = bf16(U sqrt(sigma)) [N, rank] and lora_down = bf16(V sqrt(sigma))
+ * [K, rank] (an even split between the factors), and the residual
+ *   R[n, k] = RN(W[n, k] - L[n, k]),  L = fmaf chain of the bf16 factors over
+ *   the rank as in sq_reconstruct_bf16,
  * fp32 [N, K] (device; R may equal W).  The singular subspace is found by
- * `iters` (1..100) rounds of subspace iteration from the caller's start block
- * omega [K, 32] fp32 (device; e.g. seeded N(0, 1) draws): each round one
- * product with W and one with W^T (fp32, fixed summation order), each followed
- * by CholeskyQR with fp64 Grams (twice for the final U).  With B = W^T U from
- * the last round, the Cholesky factor of B^T B and a one-sided Jacobi
- * iteration on its columns give sigma and the rotation of the factors.
- * Deterministic for a given shape
- * and omega.  The accuracy of the rank-32 product against the exact truncated
- * SVD improves as (sigma_33 / sigma_32)^(2 iters); R is RN(W - L) of whatever
- * factors result (it absorbs what they miss).
+ * `iters` (1..100) rounds of subspace iteration on 32 columns from the
+ * caller's start block omega [K, 32] fp32 (device; e.g. seeded N(0, 1)
+ * draws): each round one product with W and one with W^T (fp32, fixed
+ * summation order), each followed by CholeskyQR with fp64 Grams (twice for the
+ * final U).  With B = W^T U from the last round, the Cholesky factor of B^T B
+ * and a one-sided Jacobi iteration on its columns give sigma and the rotation
+ * of the factors.  Deterministic for a given shape and omega.  The accuracy of
+ * the rank-r product against the exact truncated SVD improves as
+ * (sigma_33 / sigma_r)^(2 iters); R is RN(W - L) of whatever factors result
+ * (it absorbs what they miss).
  * ws: sq_workspace_bytes(SQ_OP_SVD_INIT, 0, N, K) bytes, 256-byte aligned,
  * caller-owned.  Errors: SQ_ERR_NULL, SQ_ERR_SHAPE (N, K as for the builders),
- * SQ_ERR_ARG (iters), SQ_ERR_ALIGN (16 bytes; ws 256), SQ_ERR_WORKSPACE, and
- * SQ_ERR_CUDA with sq_last_error_detail() naming the launch that failed.
+ * SQ_ERR_ARG (iters, rank), SQ_ERR_ALIGN (16 bytes; ws 256), SQ_ERR_WORKSPACE,
+ * and SQ_ERR_CUDA with sq_last_error_detail() naming the launch that failed.
  */
 SQ_API sq_status sq_svd_init(const float *W, int64_t N, int64_t K, const float *omega, int32_t iters,
-                             uint16_t *lora_up, uint16_t *lora_down, float *R, void *ws, size_t ws_bytes,
-                             void *stream);
+                             int32_t rank, uint16_t *lora_up, uint16_t *lora_down, float *R, void *ws,
+                             size_t ws_bytes, void *stream);
 
 /*
  * int8 per-row builder (SquareQ README, "v3.1 -- int8-residual mode": int8

@@ -88,11 +88,14 @@ def test_build_int8_validation():
 def test_svd_init_validation():
     L = sq.lib()
     big = 1 << 30
-    svd = lambda W=A, N=256, K=512, om=A, it=4, ws=A, wsb=big: L.sq_svd_init(W, N, K, om, it, A, A, A, ws, wsb, None)
+    svd = lambda W=A, N=256, K=512, om=A, it=4, rk=32, ws=A, wsb=big: \
+        L.sq_svd_init(W, N, K, om, it, rk, A, A, A, ws, wsb, None)
     assert svd(W=None) == SQ_ERR_NULL
     assert svd(K=300) == SQ_ERR_SHAPE
     assert svd(it=0) == SQ_ERR_ARG
     assert svd(it=101) == SQ_ERR_ARG
+    assert svd(rk=8) == SQ_ERR_ARG
+    assert svd(rk=24) == SQ_ERR_ARG
     assert svd(om=MIS) == SQ_ERR_ALIGN
     assert svd(wsb=64) == SQ_ERR_WORKSPACE
     assert sq.sq_workspace_bytes(sq.SQ_OP_SVD_INIT, 0, 256, 512) >= (256 + 512) * 32 * 4

@@ -207,3 +207,56 @@ def test_svd_init_bench_shape_properties(sq):
     su = np.diag(si.bf16_bits_to_f32(up_b).astype(np.float64).T @ si.bf16_bits_to_f32(up_b).astype(np.float64))
     sd = np.diag(si.bf16_bits_to_f32(down_b).astype(np.float64).T @ si.bf16_bits_to_f32(down_b).astype(np.float64))
     assert np.allclose(su, sd, rtol=1e-2)
+
+
+def gap16_weight(N, K, seed):
+    """A rank-32 part with singular values 8 .. 4 then 1 .. 0.5 (a gap of 4 at index 16) plus the
+    synthetic residual scaled to spectral norm 0.1."""
+    rng = np.random.default_rng(seed)
+    A = rng.standard_normal((N, 32)) / np.sqrt(N)
+    B = rng.standard_normal((K, 32)) / np.sqrt(K)
+    s = np.concatenate([np.geomspace(8.0, 4.0, 16), np.geomspace(1.0, 0.5, 16)])
+    noise = si.make_inputs(4, K, N, seed)["R"].astype(np.float64)
+    noise *= 0.1 / np.linalg.norm(noise, 2)
+    W = ((A * s) @ B.T + noise).astype(np.float32)
+    S = np.linalg.svd(W.astype(np.float64), compute_uv=False)
+    assert S[15] >= 3 * S[16], "test weight without a spectral gap at 16"
+    return W
+
+
+@pytest.mark.parametrize("shape", [(256, 512), (1024, 768)])
+def test_svd_init_rank16(sq, shape):
+    """Rank 16 (the int8 mode's branch): factors [N, 16] / [K, 16], the rank-16 product against the
+    oracle's truncated SVD, the residual of the rank-16 chain bit for bit."""
+    N, K = shape
+    W = gap16_weight(N, K, 120 + N)
+    up, down, R = sq.svd_init(to_dev(W), to_dev(omega(K, 18)), 8, rank=16)
+    torch.cuda.synchronize()
+    assert tuple(up.shape) == (N, 16) and tuple(down.shape) == (K, 16)
+    up_b, down_b, Rh = bits16(up), bits16(down), host(R)
+    oup, odown, oR, _ = oracle.svd_init(W, rank=16)
+    L, Lo = lowrank_product(up_b, down_b), lowrank_product(oup, odown)
+    err = np.linalg.norm(L - Lo) / np.linalg.norm(Lo)
+    assert err <= L_TOL, f"rank-16 product differs by {err:.3e}"
+    Rw = oracle.svd_residual(W, up_b, down_b)
+    assert np.array_equal(Rh.view(np.uint32), Rw.view(np.uint32)), first_mismatch(Rh, Rw)
+    assert np.linalg.norm(Rh) <= np.linalg.norm(oR) * (1 + 1e-2)
+
+
+def test_svd_init_then_int8_mode(sq):
+    """The int8 mode end to end from a weight: SVD init at rank 16, the int8 builder on its
+    residual, the reconstruct of W -- every step on the GPU, compared with the oracle run on the
+    GPU's SVD outputs (codes, scales and the bf16 reconstruct bit for bit)."""
+    W = gap16_weight(384, 768, 130)
+    up, down, R = sq.svd_init(to_dev(W), to_dev(omega(768, 19)), 8, rank=16)
+    w = sq.build_int8(R, up, down)
+    Wb = sq.reconstruct_bf16(w)
+    torch.cuda.synchronize()
+    Rh, up_b, down_b = host(R), bits16(up), bits16(down)
+    c, s, _ = oracle.build_int8(Rh)
+    assert np.array_equal(host(w.codes), c) and np.array_equal(host(w.scales).view(np.uint32), s.view(np.uint32))
+    Wo = oracle.reconstruct_bf16(oracle.FMT_INT8_ROW, c, s, 0.0, up_b, down_b, 384, 768)
+    assert np.array_equal(bits16(Wb), Wo), first_mismatch(bits16(Wb), Wo)
+    # the rebuilt weight is close to the original (int8 residual error plus bf16 output rounding)
+    Wf = si.bf16_bits_to_f32(Wo).astype(np.float64)
+    assert np.linalg.norm(Wf - W) <= 4e-3 * np.linalg.norm(W)
