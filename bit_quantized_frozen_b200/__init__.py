@@ -38,6 +38,7 @@ RANK_INT8 = 16
 SQ_ACT_STATIC_SCALE = 0x1
 SQ_RECON_RESIDUAL_ONLY = 0x2
 SQ_RECON_TRANSPOSED = 0x4
+SQ_OUT_BF16 = 0x8
 SQ_OP_LINEAR_BWD_DX = 9
 SQ_OP_SVD_INIT = 10
 RANK = 32
@@ -317,9 +318,13 @@ def svd_init(W: torch.Tensor, omega: torch.Tensor, iters: int = 8, rank: int = R
     return up, down, R
 
 
-def linear_fwd(w: Weight, x: torch.Tensor, ws=None, g_x=None, flags: int = 0, stream=None) -> torch.Tensor:
+def linear_fwd(w: Weight, x: torch.Tensor, ws=None, g_x=None, flags: int = 0, out_bf16: bool = False,
+               stream=None) -> torch.Tensor:
+    """y [M, N] = x W^T: fp32, or bf16 (the same values rounded once) with out_bf16."""
     M = x.shape[0]
-    y = torch.empty((M, w.N), dtype=torch.float32, device=x.device)
+    if out_bf16:
+        flags |= SQ_OUT_BF16
+    y = torch.empty((M, w.N), dtype=torch.bfloat16 if flags & SQ_OUT_BF16 else torch.float32, device=x.device)
     op = {SQ_FMT_NVFP4: SQ_OP_LINEAR_FWD_NVFP4, SQ_FMT_INT8_ROW: SQ_OP_LINEAR_FWD_INT8}.get(w.fmt, SQ_OP_LINEAR_FWD_INT4)
     ws = ws if ws is not None else workspace(op, M, w.N, w.K, x.device)
     sq_linear_fwd(w, x, y, g_x=g_x, flags=flags, ws=ws, stream=stream)

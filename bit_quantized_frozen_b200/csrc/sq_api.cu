@@ -363,7 +363,7 @@ sq_status sq_act_quant_nvfp4(const uint16_t *x, int64_t M, int64_t K, uint8_t *c
     return SQ_OK;
 }
 
-sq_status sq_linear_fwd(const sq_weight *w, const uint16_t *x, int64_t M, float *y, float *g_x, uint32_t flags,
+sq_status sq_linear_fwd(const sq_weight *w, const uint16_t *x, int64_t M, void *y, float *g_x, uint32_t flags,
                         void *ws, size_t ws_bytes, void *stream)
 {
     sq_status st = check_weight(w);
@@ -371,7 +371,7 @@ sq_status sq_linear_fwd(const sq_weight *w, const uint16_t *x, int64_t M, float 
         return st;
     if (!x || !y || !ws)
         return SQ_ERR_NULL;
-    if (flags & ~SQ_ACT_STATIC_SCALE)
+    if (flags & ~(SQ_ACT_STATIC_SCALE | SQ_OUT_BF16))
         return SQ_ERR_ARG;
     const bool stat = (flags & SQ_ACT_STATIC_SCALE) != 0;
     if (stat && (!g_x || w->fmt != SQ_FMT_NVFP4))
@@ -401,6 +401,7 @@ sq_status sq_linear_fwd(const sq_weight *w, const uint16_t *x, int64_t M, float 
     g.N = N;
     g.K = K;
     g.y = y;
+    g.out_bf16 = (flags & SQ_OUT_BF16) ? 1 : 0;
     g.status = status;
     g.tsplit = tsplit;
     g.udup = udup;
@@ -471,7 +472,7 @@ sq_status sq_linear_fwd(const sq_weight *w, const uint16_t *x, int64_t M, float 
     return SQ_OK;
 }
 
-sq_status sq_linear_fwd_noalloc(const sq_weight *w, const uint16_t *x, int64_t M, float *y, float *g_x,
+sq_status sq_linear_fwd_noalloc(const sq_weight *w, const uint16_t *x, int64_t M, void *y, float *g_x,
                                 uint32_t flags, void **scratch_out, void *stream)
 {
     static_assert(sizeof(g_noalloc_scratch) == kNoAllocScratchBytes, "scratch size");

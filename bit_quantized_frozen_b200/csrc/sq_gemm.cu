@@ -84,6 +84,7 @@ struct GemmArgs {
     uint32_t *status;        // device status word
     int M, N, K;
     int lora;                // 1: add the low-rank K-step
+    int out_bf16;            // 1: y is bf16 (RNE of the fp32 result), else fp32
 };
 
 // warp-uniform bounded wait on a local barrier: lane 0 polls, the verdict is broadcast
@@ -107,9 +108,26 @@ __device__ __forceinline__ bool warp_wait_cluster(uint32_t bar, uint32_t parity,
 
 // scale one 32-row x 32-column accumulator chunk into 128B-swizzled staging
 // buffer sb of the warp (the caller made sure the buffer is free)
-__device__ __forceinline__ void stage_chunk(const uint32_t (&r)[32], float beta, uint8_t *staging, int sb, int lane)
+// one warp's 32 rows x 32 columns of y, scaled by beta, into staging buffer sb in the layout of
+// the y tensor map: fp32 rows of 128 bytes with the 128-byte swizzle, or (ybf) bf16 rows of 64
+// bytes with the 64-byte swizzle (16-byte piece j of row r at j ^ ((r >> 1) & 3))
+__device__ __forceinline__ void stage_chunk(const uint32_t (&r)[32], float beta, uint8_t *staging, int sb, int lane,
+                                            bool ybf)
 {
     uint8_t *buf = staging + sb * kStagingBytes;
+    if (ybf) {
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            uint32_t p[4];
+#pragma unroll
+            for (int i = 0; i < 4; ++i)
+                p[i] = f32x2_to_bf16x2_bits(__fmul_rn(__uint_as_float(r[8 * j + 2 * i]), beta),
+                                            __fmul_rn(__uint_as_float(r[8 * j + 2 * i + 1]), beta));
+            *reinterpret_cast<uint4 *>(buf + lane * 64 + ((j ^ ((lane >> 1) & 3)) << 4)) =
+                make_uint4(p[0], p[1], p[2], p[3]);
+        }
+        return;
+    }
 #pragma unroll
     for (int j = 0; j < 8; ++j) {
         float4 o;
@@ -134,12 +152,12 @@ __device__ __forceinline__ void issue_store(uint8_t *staging, int sb, int lane, 
 
 // stage + store a chunk through buffer sb, once at most one earlier store is pending
 __device__ __forceinline__ void store_chunk(const uint32_t (&r)[32], float beta, uint8_t *staging, int sb, int lane,
-                                            const CUtensorMap *tmY, int x, int y)
+                                            const CUtensorMap *tmY, int x, int y, bool ybf)
 {
     if (lane == 0)
         bulk_wait_group_read1();
     __syncwarp();
-    stage_chunk(r, beta, staging, sb, lane);
+    stage_chunk(r, beta, staging, sb, lane, ybf);
     issue_store(staging, sb, lane, tmY, x, y);
 }
 
@@ -428,6 +446,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(GemmCfg<FP4>::kThrea
             beta = b == 0.0f ? 1.0f : b;
         }
         const uint32_t acc_empty_leader = mapa_shared(bar_acc_empty, 0);
+        const bool ybf = args.out_bf16 != 0;
         uint8_t *staging = smem + Cfg::kStagingOff + warp * 2 * kStagingBytes;
         int count = 0;
         for (int tile = cluster_id; tile < tiles; tile += clusters, ++count) {
@@ -455,8 +474,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(GemmCfg<FP4>::kThrea
             tmem_ld_32cols(acc + 32 * ((first + 2) & 7), r2);
             tmem_ld_32cols(acc + 32 * ((first + 3) & 7), r3);
             tmem_wait_ld();
-            stage_chunk(r0, beta, staging, 0, lane);
-            stage_chunk(r1, beta, staging, 1, lane);
+            stage_chunk(r0, beta, staging, 0, lane, ybf);
+            stage_chunk(r1, beta, staging, 1, lane, ybf);
             tmem_ld_32cols(acc + 32 * ((first + 4) & 7), r0);
             tmem_ld_32cols(acc + 32 * ((first + 5) & 7), r1);
             tmem_wait_ld();
@@ -467,17 +486,17 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(GemmCfg<FP4>::kThrea
             if (rows_live) {
                 issue_store(staging, 0, lane, &tmY, n0 + 32 * ((first + 0) & 7), ytop);
                 issue_store(staging, 1, lane, &tmY, n0 + 32 * ((first + 1) & 7), ytop);
-                store_chunk(r2, beta, staging, 0, lane, &tmY, n0 + 32 * ((first + 2) & 7), ytop);
-                store_chunk(r3, beta, staging, 1, lane, &tmY, n0 + 32 * ((first + 3) & 7), ytop);
-                store_chunk(r0, beta, staging, 0, lane, &tmY, n0 + 32 * ((first + 4) & 7), ytop);
-                store_chunk(r1, beta, staging, 1, lane, &tmY, n0 + 32 * ((first + 5) & 7), ytop);
+                store_chunk(r2, beta, staging, 0, lane, &tmY, n0 + 32 * ((first + 2) & 7), ytop, ybf);
+                store_chunk(r3, beta, staging, 1, lane, &tmY, n0 + 32 * ((first + 3) & 7), ytop, ybf);
+                store_chunk(r0, beta, staging, 0, lane, &tmY, n0 + 32 * ((first + 4) & 7), ytop, ybf);
+                store_chunk(r1, beta, staging, 1, lane, &tmY, n0 + 32 * ((first + 5) & 7), ytop, ybf);
             }
             tmem_ld_32cols(acc + 32 * ((first + 6) & 7), r2);
             tmem_ld_32cols(acc + 32 * ((first + 7) & 7), r3);
             tmem_wait_ld();
             if (rows_live) {
-                store_chunk(r2, beta, staging, 0, lane, &tmY, n0 + 32 * ((first + 6) & 7), ytop);
-                store_chunk(r3, beta, staging, 1, lane, &tmY, n0 + 32 * ((first + 7) & 7), ytop);
+                store_chunk(r2, beta, staging, 0, lane, &tmY, n0 + 32 * ((first + 6) & 7), ytop, ybf);
+                store_chunk(r3, beta, staging, 1, lane, &tmY, n0 + 32 * ((first + 7) & 7), ytop, ybf);
             }
         }
         if (lane == 0)
@@ -551,8 +570,12 @@ cudaError_t launch_gemm(const GemmLaunch &g, int sms, cudaStream_t stream)
                     (uint64_t)g.M, 64, 128, CU_TENSOR_MAP_SWIZZLE_128B);
     ok &= make_tmap(&tU, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, lora ? (const void *)g.udup : g.b, 64,
                     (uint64_t)g.N, 64, 128, CU_TENSOR_MAP_SWIZZLE_128B);
-    ok &= make_tmap(&tY, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, g.y, (uint64_t)g.N, (uint64_t)g.M, 32, 32,
-                    CU_TENSOR_MAP_SWIZZLE_128B);
+    if (g.out_bf16)
+        ok &= make_tmap(&tY, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, g.y, (uint64_t)g.N, (uint64_t)g.M, 32, 32,
+                        CU_TENSOR_MAP_SWIZZLE_64B);
+    else
+        ok &= make_tmap(&tY, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, g.y, (uint64_t)g.N, (uint64_t)g.M, 32, 32,
+                        CU_TENSOR_MAP_SWIZZLE_128B);
     if (!ok)
         return cudaErrorInvalidValue;
     GemmArgs a;
@@ -565,6 +588,7 @@ cudaError_t launch_gemm(const GemmLaunch &g, int sms, cudaStream_t stream)
     a.N = (int)g.N;
     a.K = (int)g.K;
     a.lora = lora ? 1 : 0;
+    a.out_bf16 = g.out_bf16 ? 1 : 0;
     const int tiles = (int)(((g.M + BM - 1) / BM) * ((g.N + BN - 1) / BN));
     // persistent grid: as many CTA pairs as can be resident at once (not every SM
     // can pair up inside its GPC), each walking the tile list; queried once per

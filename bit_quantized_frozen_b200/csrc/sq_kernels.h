@@ -71,7 +71,8 @@ struct GemmLaunch {
     const float *g_w;
     const uint16_t *tsplit;  // [M, 64] bf16 or NULL (no low-rank step)
     const uint16_t *udup;    // [N, 64] bf16 or NULL
-    float *y;                // [M, N] fp32
+    void *y;                 // [M, N] fp32, or bf16 with out_bf16
+    int out_bf16;            // 1: y = bf16(RNE) of the fp32 result
     uint32_t *status;        // device status word
     int64_t M, N, K;
 };

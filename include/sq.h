@@ -87,6 +87,7 @@ typedef enum {
 #define SQ_ACT_STATIC_SCALE    0x1u  /* sq_act_quant_nvfp4 / sq_linear_fwd: *g_x is an input */
 #define SQ_RECON_RESIDUAL_ONLY 0x2u  /* sq_reconstruct_bf16: drop the low-rank term        */
 #define SQ_RECON_TRANSPOSED    0x4u  /* sq_reconstruct_bf16: write W^T [K, N] instead of W  */
+#define SQ_OUT_BF16            0x8u  /* sq_linear_fwd(_noalloc): y is bf16 = bf16(y_fp32)   */
 
 /*
  * A built weight.  All pointers are device pointers owned by the caller.
@@ -239,7 +240,9 @@ SQ_API sq_status sq_act_quant_nvfp4(const uint16_t *x, int64_t M, int64_t K,
                              void *ws, size_t ws_bytes, void *stream);
 
 /*
- * Forward y = x W^T, y [M, N] fp32 (device), x [M, K] bf16 (device).
+ * Forward y = x W^T, y [M, N] fp32 (device; with SQ_OUT_BF16 bf16, the
+ * round-to-nearest-even of the same fp32 value, rounded once in the GEMM's
+ * epilogue), x [M, K] bf16 (device).
  * Because H is symmetric, x W^T = H(x) deq(Q)^T + (x lora_down) lora_up^T.
  *   NVFP4: the activation prologue above, then a block-scaled e2m1 x e2m1
  *          tensor-core GEMM (tcgen05, fp32 accumulation in tensor memory),
@@ -251,12 +254,13 @@ SQ_API sq_status sq_act_quant_nvfp4(const uint16_t *x, int64_t M, int64_t K,
  *          (SQ_FMT_INT8_ROW; workspace op SQ_OP_LINEAR_FWD_INT8).
  * The low-rank term is accumulated on the tensor cores in the same
  * accumulator.  Accuracy: max|y - y_exact| / max|y_exact| <= 2e-3 against the
- * exact result on the same quantised operands.  flags: SQ_ACT_STATIC_SCALE
- * (NVFP4; *g_x is then an input, g_x must be non-NULL).  g_x (device, may be
+ * exact result on the same quantised operands (fp32 y; a bf16 y adds its own
+ * rounding, up to 2^-9 of |y|).  flags: SQ_ACT_STATIC_SCALE
+ * (NVFP4; *g_x is then an input, g_x must be non-NULL), SQ_OUT_BF16.  g_x (device, may be
  * NULL unless static) receives the activation global scale.  ws:
  * sq_workspace_bytes(SQ_OP_LINEAR_FWD_NVFP4 or _INT4, M, N, K) bytes.
  */
-SQ_API sq_status sq_linear_fwd(const sq_weight *w, const uint16_t *x, int64_t M, float *y,
+SQ_API sq_status sq_linear_fwd(const sq_weight *w, const uint16_t *x, int64_t M, void *y,
                         float *g_x, uint32_t flags, void *ws, size_t ws_bytes,
                         void *stream);
 
@@ -291,7 +295,7 @@ SQ_API sq_status sq_linear_fwd(const sq_weight *w, const uint16_t *x, int64_t M,
  * device (different streams without an event between them, or several host
  * threads) race on it and give wrong results.  Order them on one stream.
  */
-SQ_API sq_status sq_linear_fwd_noalloc(const sq_weight *w, const uint16_t *x, int64_t M, float *y,
+SQ_API sq_status sq_linear_fwd_noalloc(const sq_weight *w, const uint16_t *x, int64_t M, void *y,
                                        float *g_x, uint32_t flags, void **scratch_out, void *stream);
 
 /*

@@ -138,6 +138,7 @@ def test_linear_fwd_validation():
     assert fwd(_w(), ws=A + 64) == SQ_ERR_ALIGN
     assert fwd(_w(), wsb=100) == SQ_ERR_WORKSPACE
     assert fwd(_w(), fl=sq.SQ_ACT_STATIC_SCALE) == SQ_ERR_NULL          # static scale needs g_x
+    assert fwd(_w(), fl=0x10) == SQ_ERR_ARG                             # unknown flag
     assert fwd(_w(fmt=sq.SQ_FMT_INT4_G32, g_w=None), gx=A, fl=sq.SQ_ACT_STATIC_SCALE) == SQ_ERR_ARG
     assert fwd(_w(), fl=0x40) == SQ_ERR_ARG
 

@@ -217,6 +217,28 @@ def test_linear_fwd_zero_residual_is_lowrank_only(sq, fmt):
     check_fwd(sq, d, fmt)
 
 
+@pytest.mark.parametrize("fmt", [2, 1, 4], ids=["nvfp4", "int4", "int8"])
+@pytest.mark.parametrize("shape", [(300, 1280, 512), (64, 512, 256)])
+def test_linear_fwd_bf16_output(sq, shape, fmt):
+    """SQ_OUT_BF16: y is the round-to-nearest-even of the fp32 output, bit for bit (one rounding
+    of the same value, in the GEMM's epilogue), for every payload format and a ragged M."""
+    M, K, N = shape
+    d = si.make_inputs(M, K, N, 15 + M)
+    if fmt == 4:
+        w = sq.build_int8(to_dev(d["R"]), bf16_dev(np.ascontiguousarray(d["U"][:, :16])),
+                          bf16_dev(np.ascontiguousarray(d["D"][:, :16])))
+    else:
+        w = gpu_weight(sq, d, fmt)
+    x = bf16_dev(d["x"])
+    y32 = sq.linear_fwd(w, x)
+    y16 = sq.linear_fwd(w, x, out_bf16=True)
+    torch.cuda.synchronize()
+    assert y16.dtype == torch.bfloat16 and tuple(y16.shape) == (M, N)
+    want = si.to_bf16_bits(host(y32))
+    got = bits16(y16)
+    assert np.array_equal(got, want), first_mismatch(got, want)
+
+
 def test_linear_fwd_zero_activation(sq):
     d = si.make_inputs(64, 512, 256, 14)
     d["x"][:] = 0
