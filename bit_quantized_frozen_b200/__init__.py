@@ -39,6 +39,7 @@ SQ_ACT_STATIC_SCALE = 0x1
 SQ_RECON_RESIDUAL_ONLY = 0x2
 SQ_RECON_TRANSPOSED = 0x4
 SQ_OUT_BF16 = 0x8
+SQ_CHECK_FINITE = 0x10
 SQ_OP_LINEAR_BWD_DX = 9
 SQ_OP_SVD_INIT = 10
 RANK = 32

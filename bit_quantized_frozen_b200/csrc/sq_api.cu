@@ -191,6 +191,7 @@ const char *sq_status_str(int status)
     case SQ_ERR_CUDA: return "CUDA error";
     case SQ_ERR_ARG: return "bad argument";
     case SQ_ERR_TIMEOUT: return "kernel wait timed out";
+    case SQ_ERR_NONFINITE: return "non-finite input";
     default: return "unknown status";
     }
 }
@@ -335,7 +336,7 @@ sq_status sq_act_quant_nvfp4(const uint16_t *x, int64_t M, int64_t K, uint8_t *c
 {
     if (!x || !codes || !sf_tiled || !g_x || !ws)
         return SQ_ERR_NULL;
-    if (flags & ~SQ_ACT_STATIC_SCALE)
+    if (flags & ~(SQ_ACT_STATIC_SCALE | SQ_CHECK_FINITE))
         return SQ_ERR_ARG;
     if (!shape_ok_mk(M, K))
         return SQ_ERR_SHAPE;
@@ -353,6 +354,8 @@ sq_status sq_act_quant_nvfp4(const uint16_t *x, int64_t M, int64_t K, uint8_t *c
     const bool with_t = lora_down && t;
     uint32_t *amax = reinterpret_cast<uint32_t *>(ws_at(ws, 4));
     SQ_CUDA(cudaMemsetAsync(ws, 0, 8, s), "memset");          // status word + absmax
+    if (flags & SQ_CHECK_FINITE)
+        SQ_CUDA(sq::launch_check_finite_bf16(x, M * K, reinterpret_cast<uint32_t *>(ws), sms, s), "finite check");
     if (!stat || with_t)
         SQ_CUDA(sq::launch_act_pass1(x, M, K, lora_down, stat ? nullptr : amax, with_t ? t : nullptr,
                                              reinterpret_cast<uint32_t *>(ws), sms, s),
@@ -371,7 +374,7 @@ sq_status sq_linear_fwd(const sq_weight *w, const uint16_t *x, int64_t M, void *
         return st;
     if (!x || !y || !ws)
         return SQ_ERR_NULL;
-    if (flags & ~(SQ_ACT_STATIC_SCALE | SQ_OUT_BF16))
+    if (flags & ~(SQ_ACT_STATIC_SCALE | SQ_OUT_BF16 | SQ_CHECK_FINITE))
         return SQ_ERR_ARG;
     const bool stat = (flags & SQ_ACT_STATIC_SCALE) != 0;
     if (stat && (!g_x || w->fmt != SQ_FMT_NVFP4))
@@ -406,6 +409,8 @@ sq_status sq_linear_fwd(const sq_weight *w, const uint16_t *x, int64_t M, void *
     g.tsplit = tsplit;
     g.udup = udup;
     SQ_CUDA(cudaMemsetAsync(status, 0, 8, s), "memset");   // status word + absmax
+    if (flags & SQ_CHECK_FINITE)
+        SQ_CUDA(sq::launch_check_finite_bf16(x, M * K, status, sms, s), "finite check");
     if (w->fmt == SQ_FMT_NVFP4) {
         float *gx = g_x ? g_x : reinterpret_cast<float *>(ws_at(ws, 8));
         uint8_t *xc = ws_at(ws, L.a);
@@ -627,7 +632,7 @@ sq_status sq_check_device_status(void *ws, void *stream)
     SQ_CUDA(cudaStreamSynchronize(s), "status sync");
     if (word != 0) {
         SQ_CUDA(cudaMemsetAsync(ws, 0, 4, s), "status clear");
-        return SQ_ERR_TIMEOUT;
+        return (word & 1u) ? SQ_ERR_TIMEOUT : SQ_ERR_NONFINITE;   // bit 0 timeout, bit 1 non-finite
     }
     return SQ_OK;
 }

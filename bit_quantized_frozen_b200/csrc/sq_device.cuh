@@ -19,7 +19,8 @@ constexpr int kGroup = 32;         // int4 values per fp16 scale
 constexpr int kFracCount = 26;     // int4 scale fractions 0.50, 0.52, ..., 1.00
 
 // device status word bits (first word of every workspace)
-constexpr uint32_t kStatusTimeout = 1u;
+constexpr uint32_t kStatusTimeout = 1u;      // a bounded wait gave up
+constexpr uint32_t kStatusNonfinite = 2u;    // the SQ_CHECK_FINITE scan met a NaN or an infinity
 
 // ---------------------------------------------------------------------------
 // Hadamard-256 over one warp.

@@ -47,6 +47,9 @@ cudaError_t launch_lowrank_finish(const float *t32, int64_t M, const float *g_x,
 // the library's own device status word (set by kernels of calls without a workspace)
 cudaError_t library_status_word(uint32_t **p);
 
+// sets kStatusNonfinite in *status if any of the n bf16 values of x is a NaN or an infinity
+cudaError_t launch_check_finite_bf16(const uint16_t *x, int64_t n, uint32_t *status, int sms, cudaStream_t s);
+
 // fmt: 1 int4 group 32, 2 NVFP4, 3 int4 group 64, 4 int8 per row (rank 16)
 cudaError_t launch_reconstruct(int fmt, const uint8_t *codes, const void *scales, const float *g_w,
                                const uint16_t *U, const uint16_t *D, int64_t N, int64_t K, int with_lowrank,

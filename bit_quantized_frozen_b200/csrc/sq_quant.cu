@@ -1526,6 +1526,35 @@ __global__ void __launch_bounds__(kWsThreads, 1) reconstruct_ws_kernel(const uin
     }
 }
 
+// ---------------------------------------------------------------------------
+// the SQ_CHECK_FINITE scan: n bf16 values (n % 8 == 0), 16 bytes per step; a value whose exponent
+// field is all ones (NaN or infinity) sets kStatusNonfinite, once per warp that meets one
+// ---------------------------------------------------------------------------
+__global__ void __launch_bounds__(256) check_finite_bf16_kernel(const uint4 *__restrict__ x, int64_t n16,
+                                                                uint32_t *__restrict__ status)
+{
+    bool bad = false;
+    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n16; i += (int64_t)gridDim.x * blockDim.x) {
+        const uint4 v = x[i];
+        const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+        for (int j = 0; j < 4; ++j)
+            bad |= ((w[j] & 0x7F80u) == 0x7F80u) | ((w[j] & 0x7F800000u) == 0x7F800000u);
+    }
+    if (__any_sync(0xffffffffu, bad) && (threadIdx.x & 31) == 0)
+        atomicOr(status, kStatusNonfinite);
+}
+
+cudaError_t launch_check_finite_bf16(const uint16_t *x, int64_t n, uint32_t *status, int sms, cudaStream_t s)
+{
+    const int64_t n16 = n / 8;
+    const int64_t blocks = (n16 + 255) / 256;
+    const int64_t grid = blocks < (int64_t)sms * 4 ? blocks : (int64_t)sms * 4;
+    check_finite_bf16_kernel<<<(unsigned)(grid < 1 ? 1 : grid), 256, 0, s>>>(reinterpret_cast<const uint4 *>(x), n16,
+                                                                           status);
+    return cudaGetLastError();
+}
+
 // the library's own device status word, for kernels whose call takes no workspace
 __device__ uint32_t g_library_status;
 

@@ -59,7 +59,8 @@ typedef enum {
     SQ_ERR_DEVICE = 5,     /* current device is not sm_100 (B200 class)          */
     SQ_ERR_CUDA = 6,       /* a CUDA call or launch failed                        */
     SQ_ERR_ARG = 7,        /* bad enum / flag value                               */
-    SQ_ERR_TIMEOUT = 8     /* a kernel gave up a bounded wait (device status word) */
+    SQ_ERR_TIMEOUT = 8,    /* a kernel gave up a bounded wait (device status word) */
+    SQ_ERR_NONFINITE = 9   /* SQ_CHECK_FINITE met a NaN or an infinity (status word) */
 } sq_status;
 
 typedef enum {
@@ -88,6 +89,10 @@ typedef enum {
 #define SQ_RECON_RESIDUAL_ONLY 0x2u  /* sq_reconstruct_bf16: drop the low-rank term        */
 #define SQ_RECON_TRANSPOSED    0x4u  /* sq_reconstruct_bf16: write W^T [K, N] instead of W  */
 #define SQ_OUT_BF16            0x8u  /* sq_linear_fwd(_noalloc): y is bf16 = bf16(y_fp32)   */
+#define SQ_CHECK_FINITE        0x10u /* sq_act_quant_nvfp4 / sq_linear_fwd(_noalloc): scan x
+                                        for NaN and infinities first; a hit sets the status
+                                        word that sq_check_device_status reports as
+                                        SQ_ERR_NONFINITE (the call itself still runs)      */
 
 /*
  * A built weight.  All pointers are device pointers owned by the caller.
@@ -232,7 +237,9 @@ SQ_API sq_status sq_build_nvfp4(const float *R, int64_t N, int64_t K,
  * (device): codes [M, K/2], sf_tiled (sq_sf_bytes(M, K) bytes, padding rows
  * 0), g_x (written unless static).  If lora_down (bf16 [K, 32]) and t are
  * both non-NULL, also t[m, r] = sum_k x[m, k] lora_down[k, r] as fp32 [M, 32]
- * (the low-rank input; fp32 accumulation, order unspecified).
+ * (the low-rank input; fp32 accumulation, order unspecified).  flags:
+ * SQ_ACT_STATIC_SCALE, SQ_CHECK_FINITE (the status word is the first 4 bytes
+ * of ws).
  */
 SQ_API sq_status sq_act_quant_nvfp4(const uint16_t *x, int64_t M, int64_t K,
                              uint8_t *codes, uint8_t *sf_tiled, float *g_x,
@@ -256,8 +263,9 @@ SQ_API sq_status sq_act_quant_nvfp4(const uint16_t *x, int64_t M, int64_t K,
  * accumulator.  Accuracy: max|y - y_exact| / max|y_exact| <= 2e-3 against the
  * exact result on the same quantised operands (fp32 y; a bf16 y adds its own
  * rounding, up to 2^-9 of |y|).  flags: SQ_ACT_STATIC_SCALE
- * (NVFP4; *g_x is then an input, g_x must be non-NULL), SQ_OUT_BF16.  g_x (device, may be
- * NULL unless static) receives the activation global scale.  ws:
+ * (NVFP4; *g_x is then an input, g_x must be non-NULL), SQ_OUT_BF16,
+ * SQ_CHECK_FINITE.  g_x (device, may be NULL unless static) receives the
+ * activation global scale.  ws:
  * sq_workspace_bytes(SQ_OP_LINEAR_FWD_NVFP4 or _INT4, M, N, K) bytes.
  */
 SQ_API sq_status sq_linear_fwd(const sq_weight *w, const uint16_t *x, int64_t M, void *y,
@@ -344,7 +352,9 @@ SQ_API sq_status sq_set_gemm_events(void *start_event, void *stop_event);
 
 /*
  * Read back and clear the device status word that a kernel sets when it gives
- * up a bounded wait (SQ_ERR_TIMEOUT); ws is the workspace of the sq_linear_fwd
+ * up a bounded wait (SQ_ERR_TIMEOUT), or that the SQ_CHECK_FINITE scan sets
+ * on a NaN or an infinity in x (SQ_ERR_NONFINITE; a timeout is reported
+ * first); ws is the workspace of the sq_linear_fwd
  * call to check (each such call clears the word when it starts).  With ws ==
  * NULL it reads the library's own word on the current device, which the calls
  * without a workspace (sq_reconstruct_bf16) set instead.  This call

@@ -138,7 +138,7 @@ def test_linear_fwd_validation():
     assert fwd(_w(), ws=A + 64) == SQ_ERR_ALIGN
     assert fwd(_w(), wsb=100) == SQ_ERR_WORKSPACE
     assert fwd(_w(), fl=sq.SQ_ACT_STATIC_SCALE) == SQ_ERR_NULL          # static scale needs g_x
-    assert fwd(_w(), fl=0x10) == SQ_ERR_ARG                             # unknown flag
+    assert fwd(_w(), fl=0x20) == SQ_ERR_ARG                             # unknown flag
     assert fwd(_w(fmt=sq.SQ_FMT_INT4_G32, g_w=None), gx=A, fl=sq.SQ_ACT_STATIC_SCALE) == SQ_ERR_ARG
     assert fwd(_w(), fl=0x40) == SQ_ERR_ARG
 
@@ -191,3 +191,16 @@ def test_binding_raises_with_status():
     with pytest.raises(sq.SqError) as e:
         sq._check("sq_build_int4", SQ_ERR_SHAPE)
     assert e.value.status == SQ_ERR_SHAPE
+
+
+def test_nonfinite_guard_flag_and_status():
+    L = sq.lib()
+    assert L.sq_status_str(9) == b"non-finite input"
+    big = 1 << 34
+    # the flag passes validation (no device here: the device check answers)
+    fl = sq.SQ_CHECK_FINITE | sq.SQ_OUT_BF16
+    want = SQ_ERR_DEVICE if not torch.cuda.is_available() else None
+    if want is not None:
+        assert L.sq_linear_fwd(ctypes.byref(_w()), A, 8, A, None, fl, A, big, None) == want
+        assert L.sq_act_quant_nvfp4(A, 4, 512, A, A, A, None, None, sq.SQ_CHECK_FINITE, A, big, None) == want
+

@@ -50,3 +50,43 @@ def test_library_status_word_clear_after_reconstruct():
     sq.reconstruct_bf16(w, transposed=True)
     torch.cuda.synchronize()
     sq.sq_check_device_status(None)
+
+
+SQ_ERR_NONFINITE = 9
+
+
+@pytest.mark.parametrize("bad", [float("nan"), float("inf"), -float("inf")], ids=["nan", "inf", "-inf"])
+def test_check_finite_flags_nonfinite_activation(bad):
+    """SQ_CHECK_FINITE scans x before the forward: one NaN or infinity anywhere sets the
+    workspace status word, read back as SQ_ERR_NONFINITE; a clean x, or the same x without the
+    flag, leaves the word clear."""
+    import bit_quantized_frozen_b200 as sq
+    d = si.make_inputs(130, 512, 256, 73)
+    w = sq.build_nvfp4(to_dev(d["R"]), bf16_dev(d["U"]), bf16_dev(d["D"]))
+    ws = sq.workspace(sq.SQ_OP_LINEAR_FWD_NVFP4, 130, 256, 512)
+    x = bf16_dev(d["x"])
+    sq.linear_fwd(w, x, ws=ws, flags=sq.SQ_CHECK_FINITE)
+    sq.sq_check_device_status(ws)                                    # clean input
+    xb = x.clone()
+    xb[129, 511] = bad                                               # the last value of a ragged M
+    sq.linear_fwd(w, xb, ws=ws)
+    sq.sq_check_device_status(ws)                                    # no scan without the flag
+    sq.linear_fwd(w, xb, ws=ws, flags=sq.SQ_CHECK_FINITE)
+    with pytest.raises(sq.SqError) as e:
+        sq.sq_check_device_status(ws)
+    assert e.value.status == SQ_ERR_NONFINITE
+    # the int4 path and the activation quantisation entry take the flag too
+    w4 = sq.build_int4(to_dev(d["R"]), bf16_dev(d["U"]), bf16_dev(d["D"]))
+    ws4 = sq.workspace(sq.SQ_OP_LINEAR_FWD_INT4, 130, 256, 512)
+    sq.linear_fwd(w4, xb, ws=ws4, flags=sq.SQ_CHECK_FINITE)
+    with pytest.raises(sq.SqError) as e:
+        sq.sq_check_device_status(ws4)
+    assert e.value.status == SQ_ERR_NONFINITE
+    wsa = sq.workspace(sq.SQ_OP_ACT_QUANT_NVFP4, 130, 0, 512)
+    codes = torch.empty((130, 256), dtype=torch.uint8, device="cuda")
+    sf = torch.empty(sq.sq_sf_bytes(130, 512), dtype=torch.uint8, device="cuda")
+    gx = torch.empty(1, dtype=torch.float32, device="cuda")
+    sq.sq_act_quant_nvfp4(xb, codes, sf, gx, flags=sq.SQ_CHECK_FINITE, ws=wsa)
+    with pytest.raises(sq.SqError) as e:
+        sq.sq_check_device_status(wsa)
+    assert e.value.status == SQ_ERR_NONFINITE
