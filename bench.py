@@ -4,7 +4,7 @@
 One step = one pass of the whole hot path over one synthetic layer of the
 chosen shape (default the headline 4480 x 16384 x 6144, M x N x K):
   sq_build_int4, sq_build_nvfp4, sq_linear_fwd (NVFP4, incl. the activation
-  prologue), sq_linear_fwd (int4), sq_reconstruct_bf16 (both payloads), and the
+  prologue; fp32 y, and bf16 y with SQ_OUT_BF16), sq_linear_fwd (int4), sq_reconstruct_bf16 (both payloads), and the
   build, forward and reconstruct of the int4 group-64 variant and of the int8
   per-row mode (rank-16 low-rank branch), the input backward dx = dy W
   (transposed bf16 reconstruct + bf16 GEMM) on the NVFP4 payload, and the
@@ -88,6 +88,7 @@ def op_work(M, N, K):
         "build_int4": ("GB/s", NK * (4 + 0.5 + 2 / 32 + 1 / 32)),
         "build_nvfp4": ("GB/s", NK * (4 + 0.5 + 1 / 16)),
         "fwd_nvfp4": ("TFLOP/s", 2.0 * M * N * K),
+        "fwd_nvfp4_bf16out": ("TFLOP/s", 2.0 * M * N * K),
         "fwd_int4": ("TFLOP/s", 2.0 * M * N * K),
         "reconstruct_nvfp4": ("GB/s", NK * (0.5 + 1 / 16 + 2)),
         "reconstruct_int4": ("GB/s", NK * (0.5 + 2 / 32 + 2)),
@@ -106,7 +107,7 @@ def op_work(M, N, K):
 
 
 LAUNCHES_PER_STEP = {   # our kernels per op (memsets excluded)
-    "build_int4": 1, "build_nvfp4": 2, "fwd_nvfp4": 5, "fwd_int4": 5,
+    "build_int4": 1, "build_nvfp4": 2, "fwd_nvfp4": 3, "fwd_nvfp4_bf16out": 3, "fwd_int4": 5,
     "reconstruct_nvfp4": 1, "reconstruct_int4": 1,
     "build_int4_g64": 1, "fwd_int4_g64": 5, "reconstruct_int4_g64": 1,
     "build_int8": 1, "fwd_int8": 7, "reconstruct_int8": 1,
@@ -383,6 +384,7 @@ def run_sq(args, cfg, d, rank, world, local_rank):
     g_x = torch.empty(1, dtype=torch.float32, device=dev)
     y_nv = torch.empty((M, N), dtype=torch.float32, device=dev)
     y_i4 = torch.empty((M, N), dtype=torch.float32, device=dev)
+    y_bf = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
     W = torch.empty((N, K), dtype=torch.bfloat16, device=dev)
     Wsvd = R + U.float() @ D.float().T            # the full weight the SVD init factors (input set-up)
     omega = torch.randn((K, 32), device=dev, generator=torch.Generator(device=dev).manual_seed(cfg.seed + 1))
@@ -396,6 +398,7 @@ def run_sq(args, cfg, d, rank, world, local_rank):
         ("build_int4", lambda: sq.sq_build_int4(R, i4.codes, i4.scales, i4.frac_idx)),
         ("build_nvfp4", lambda: sq.sq_build_nvfp4(R, nv.codes, nv.scales, nv.g_w, ws_b)),
         ("fwd_nvfp4", lambda: sq.sq_linear_fwd(nv, x, y_nv, g_x=g_x, ws=ws_nv)),
+        ("fwd_nvfp4_bf16out", lambda: sq.sq_linear_fwd(nv, x, y_bf, g_x=g_x, flags=sq.SQ_OUT_BF16, ws=ws_nv)),
         ("fwd_int4", lambda: sq.sq_linear_fwd(i4, x, y_i4, ws=ws_i4)),
         ("reconstruct_nvfp4", lambda: sq.sq_reconstruct_bf16(nv, W)),
         ("reconstruct_int4", lambda: sq.sq_reconstruct_bf16(i4, W)),
@@ -533,7 +536,7 @@ def summarise(args, cfg, per_op, outer_ms, clocks, e2e, world, cpu):
         elif k == "svd_init":
             frac, peak = rate / FP32_ALU_TFLOPS, "fp32 FMA issue"
         else:
-            fp4 = k in ("fwd_nvfp4", "gemm_nvfp4")      # the backward's GEMM runs in bf16
+            fp4 = k in ("fwd_nvfp4", "fwd_nvfp4_bf16out", "gemm_nvfp4")   # the backward's GEMM runs in bf16
             peak_v = fp4_peak if fp4 else peaks["bf16_tflops"]
             frac, peak = rate / peak_v, "fp4 tensor" if fp4 else "bf16 tensor"
         src = "148 SMs x 128 lanes x 2 flop x 1.965 GHz" if k == "svd_init" else peak_src
