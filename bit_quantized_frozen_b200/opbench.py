@@ -33,6 +33,13 @@ Operations:
                        the tensor-core GEMM launch inside sq_linear_fwd /
                        sq_linear_bwd_dx, timed by the events the library records
                        around it (sq_set_gemm_events)
+
+    python -m bit_quantized_frozen_b200.opbench --stack 28
+
+times the builders on the builder stack of the down-projection shape instead: 28 residual
+weights [6144, 16384] fp32 (seeds 4000 + i), each uploaded into one reused device buffer
+(the upload untimed) and built with sq_build_int4 (group 32), sq_build_nvfp4 and
+sq_build_int8; one JSON line per builder with the whole stack's algorithmic GB/s.
 """
 from __future__ import annotations
 
@@ -128,6 +135,54 @@ class Clocks:
                 "samples": len(vals)}
 
 
+def run_stack(n_weights: int):
+    """The builder stack: n residuals of the down-projection shape through one device buffer."""
+    N, K = 6144, 16384
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    R = torch.empty((N, K), dtype=torch.float32, device=dev)
+    host = torch.empty((N, K), dtype=torch.float32).pin_memory()
+    c4 = torch.empty((N, K // 2), dtype=torch.uint8, device=dev)
+    s4 = torch.empty((N, K // 32), dtype=torch.float16, device=dev)
+    f4 = torch.empty((N, K // 32), dtype=torch.uint8, device=dev)
+    cn = torch.empty((N, K // 2), dtype=torch.uint8, device=dev)
+    sfn = torch.empty(sq.sq_sf_bytes(N, K), dtype=torch.uint8, device=dev)
+    gn = torch.empty(1, dtype=torch.float32, device=dev)
+    ws_b = sq.workspace(sq.SQ_OP_BUILD_NVFP4, 0, N, K, dev)
+    c8 = torch.empty((N, K), dtype=torch.int8, device=dev)
+    s8 = torch.empty(N, dtype=torch.float32, device=dev)
+    f8 = torch.empty(N, dtype=torch.uint8, device=dev)
+    builders = {
+        "build_int4": (lambda: sq.sq_build_int4(R, c4, s4, f4), N * K * (4 + 0.5 + 3 / 32)),
+        "build_nvfp4": (lambda: sq.sq_build_nvfp4(R, cn, sfn, gn, ws_b), N * K * (4 + 0.5 + 1 / 16)),
+        "build_int8": (lambda: sq.sq_build_int8(R, c8, s8, f8), N * K * (4 + 1) + N * 5),
+    }
+    ms = {k: [] for k in builders}
+    for i in range(n_weights):
+        host.copy_(torch.from_numpy(si.make_stack_residual(i, N, K)))
+        R.copy_(host, non_blocking=True)                 # the upload is not timed
+        torch.cuda.synchronize()
+        if i == 0:                                       # one untimed pass: module load, attributes
+            for fn, _ in builders.values():
+                fn()
+            torch.cuda.synchronize()
+        evs = {}
+        for k, (fn, _) in builders.items():
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record()
+            fn()
+            b.record()
+            evs[k] = (a, b)
+        torch.cuda.synchronize()
+        for k, (a, b) in evs.items():
+            ms[k].append(a.elapsed_time(b))
+    for k, (_, nbytes) in builders.items():
+        total = sum(ms[k])
+        print(json.dumps({"op": k + "_stack", "weights": n_weights, "shape": [N, K], "ms_total": total,
+                          "ms_per_weight_mean": statistics.mean(ms[k]), "ms_per_weight_max": max(ms[k]),
+                          "GB/s": nbytes * n_weights / (total * 1e-3) / 1e9}), flush=True)
+
+
 def main():
     p = argparse.ArgumentParser()
     p.add_argument("--config", default="large_4480x16384x6144", choices=sorted(si.CONFIGS))
@@ -135,7 +190,11 @@ def main():
     p.add_argument("--reps", type=int, default=20)
     p.add_argument("--warmup", type=int, default=3)
     p.add_argument("--clocks", action="store_true", help="sample SM clocks and power during the timed calls")
+    p.add_argument("--stack", type=int, default=0, help="time the builders on this many stack weights instead")
     args = p.parse_args()
+    if args.stack:
+        run_stack(args.stack)
+        return
     cfg = si.CONFIGS[args.config]
     M, N, K = cfg.M, cfg.N, cfg.K
     d = si.make_config(cfg.name)
