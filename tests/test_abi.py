@@ -204,3 +204,63 @@ def test_nonfinite_guard_flag_and_status():
         assert L.sq_linear_fwd(ctypes.byref(_w()), A, 8, A, None, fl, A, big, None) == want
         assert L.sq_act_quant_nvfp4(A, 4, 512, A, A, A, None, None, sq.SQ_CHECK_FINITE, A, big, None) == want
 
+
+
+C_PROGRAM = r"""
+#include "sq.h"
+#include <stdio.h>
+#include <string.h>
+
+/* every entry point, by address: the header is plain C and the library exports them all */
+typedef void (*fnptr)(void);
+static const fnptr entries[] = {
+    (fnptr)sq_status_str, (fnptr)sq_abi_version, (fnptr)sq_last_error_detail, (fnptr)sq_sf_bytes,
+    (fnptr)sq_workspace_bytes, (fnptr)sq_build_int4, (fnptr)sq_svd_init, (fnptr)sq_build_int8,
+    (fnptr)sq_build_nvfp4, (fnptr)sq_act_quant_nvfp4, (fnptr)sq_linear_fwd, (fnptr)sq_linear_fwd_noalloc,
+    (fnptr)sq_reconstruct_bf16, (fnptr)sq_linear_bwd_dx, (fnptr)sq_set_gemm_events,
+    (fnptr)sq_check_device_status, (fnptr)sq_selftest_wait_timeout,
+};
+
+int main(void)
+{
+    sq_weight w;
+    size_t i;
+    for (i = 0; i < sizeof(entries) / sizeof(entries[0]); ++i)
+        if (!entries[i])
+            return 1;
+    memset(&w, 0, sizeof(w));
+    w.fmt = SQ_FMT_NVFP4;
+    w.N = 256;
+    w.K = 512;
+    /* host-side validation only: no device is touched */
+    if (sq_linear_fwd(&w, NULL, 8, NULL, NULL, 0, NULL, 0, NULL) != SQ_ERR_NULL)
+        return 2;
+    if (sq_build_int4(NULL, 256, 512, 32, NULL, NULL, NULL, NULL) != SQ_ERR_NULL)
+        return 3;
+    if (sq_sf_bytes(130, 512) != 256 * 32)
+        return 4;
+    printf("%d %s\n", sq_abi_version(), sq_status_str(SQ_ERR_NONFINITE));
+    return 0;
+}
+"""
+
+
+def test_header_is_plain_c_and_links(tmp_path):
+    """include/sq.h compiles as strict C99 (-pedantic, warnings as errors), a C program links
+    against libsq.so, takes the address of every entry point and runs the host-side checks."""
+    import shutil
+    import subprocess
+    if shutil.which("gcc") is None:
+        pytest.skip("no C compiler")
+    src = tmp_path / "use_sq.c"
+    exe = tmp_path / "use_sq"
+    src.write_text(C_PROGRAM)
+    libdir = os.path.dirname(sq.LIB_PATH)
+    subprocess.run(["gcc", "-std=c99", "-Wall", "-Wextra", "-Werror", "-pedantic", "-I",
+                    os.path.join(ROOT, "include"), str(src), "-L", libdir, "-lsq", "-Wl,-rpath," + libdir,
+                    "-o", str(exe)], check=True)
+    out = subprocess.run([str(exe)], check=True, capture_output=True, text=True).stdout
+    assert out.split() == ["1", "non-finite", "input"]
+    text = open(HEADER).read()
+    assert len(header_functions()) == C_PROGRAM.count("(fnptr)sq_")
+    assert "namespace" not in text and "torch" not in text
