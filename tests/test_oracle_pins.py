@@ -428,6 +428,37 @@ def test_reconstruct_on_grid_is_explicit_hadamard(oracle_mod):
     assert np.array_equal(W, si.to_bf16_bits(h.astype(np.float32)))
 
 
+def test_reconstruct_nvfp4_on_grid_is_explicit_hadamard(oracle_mod):
+    """NVFP4 payload on a grid where every step is exact in fp32: e2m1 codes times ue4m3 scales in
+    [1, 2) times g_w = 3 * 2^-8 are integer multiples of 3 * 2^-12 below 2^11 of them, so the fp32
+    Hadamard sums are exact and W = bf16(H applied to the decoded values) is computable by the
+    explicit matrix.  Pins the decode value(e2m1) * value(sf) * g_w, the tiled scale lookup and the
+    inverse rotation; residual_only must give the same W whatever the low-rank factors hold."""
+    N, K = 3, 512
+    C = K // 16
+    rng = np.random.default_rng(32)
+    nib = rng.integers(0, 16, (N, K)).astype(np.uint8)
+    codes = (nib[:, 0::2] | (nib[:, 1::2] << 4)).astype(np.uint8)
+    sfc = rng.integers(0x38, 0x40, (N, C)).astype(np.uint8)       # values 1 + m/8
+    sf = np.zeros(128 * C, np.uint8)
+    r = np.arange(N)[:, None]
+    c = np.arange(C)[None, :]
+    sf[((r // 128) * (C // 4) + c // 4) * 512 + (r % 32) * 16 + ((r % 128) // 32) * 4 + (c % 4)] = sfc
+    g = np.float32(3 * 2.0 ** -8)
+    d = E2M1[nib] * np.repeat(1 + (sfc & 7) / 8.0, 16, axis=1) * float(g)
+    H = sylvester()
+    h = np.concatenate([d[:, b:b + 256] @ H.T for b in (0, 256)], 1)
+    want = si.to_bf16_bits(h.astype(np.float32))
+    zeroU = np.zeros((N, 32), np.uint16)
+    zeroD = np.zeros((K, 32), np.uint16)
+    W = oracle_mod.reconstruct_bf16(oracle_mod.FMT_NVFP4, codes, sf, g, zeroU, zeroD, N, K)
+    assert np.array_equal(W, want)
+    U = si.to_bf16_bits(rng.standard_normal((N, 32)).astype(np.float32))
+    D = si.to_bf16_bits(rng.standard_normal((K, 32)).astype(np.float32))
+    Wr = oracle_mod.reconstruct_bf16(oracle_mod.FMT_NVFP4, codes, sf, g, U, D, N, K, residual_only=True)
+    assert np.array_equal(Wr, want)
+
+
 def test_reconstruct_lowrank_chain_and_fidelity(oracle_mod):
     N, K = 64, 512
     d = si.make_inputs(8, K, N, 31)

@@ -52,6 +52,17 @@ def test_g64_exact_roundtrip_on_grid(oracle_mod):
         assert j == 25
 
 
+def test_g64_ties_go_to_smaller_fraction(oracle_mod):
+    # all-zero group: every fraction has zero error -> j = 0, s = 0
+    q, s, j = oracle_mod.int4_group64(np.zeros(64, np.float32))
+    assert j == 0 and s == 0 and not q.any()
+    # a = 7 * 2^-24: j = 0 (f = 0.5) rounds the scale to fp16 0 (error = sum r^2); every j >= 1
+    # gives s = 2^-24 (fp16 bits 0x0001) and zero error, a 25-way tie -> the smallest, j = 1
+    r = np.full(64, 7 * 2.0 ** -24, np.float32)
+    q, s, j = oracle_mod.int4_group64(r)
+    assert j == 1 and s == 1 and np.all(q == 7)
+
+
 def test_g64_of_two_equal_halves_is_g32(oracle_mod):
     """Two copies of a group-32 input: same max, every candidate error exactly doubles
     (the two half sums are equal, and x + x is exact), so the same scale, fraction and
