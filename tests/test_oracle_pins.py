@@ -354,6 +354,26 @@ def _decode_nvfp4(codes, sf, rows, K):
     return E2M1[nib] * np.repeat(s, 16, axis=1)
 
 
+def test_build_nvfp4_global_scale_is_of_the_rotated_tensor(oracle_mod):
+    """Rows of R are scaled Sylvester rows, so the rotated tensor is exactly one-hot: c at (0, 5)
+    and c/4 at (1, 256 + 200), while R itself peaks at c/16.  The global scale must come from the
+    rotated tensor, g_w = RN(c / 2688) = 2^-10, and both peaks decode back exactly (e2m1 6 times
+    ue4m3 448, resp. 112, times g_w); every other value is 0."""
+    N, K = 2, 512
+    H16 = np.rint(sylvester() * 16)                         # the +-1 Sylvester matrix
+    c = 2688.0 * 2.0 ** -10
+    R = np.zeros((N, K), np.float32)
+    R[0, :256] = (c / 16) * H16[5]
+    R[1, 256:] = (c / 64) * H16[200]
+    assert np.abs(R).max() == c / 16
+    codes, sf, g = oracle_mod.build_nvfp4(R)
+    assert g == np.float32(2.0 ** -10)
+    want = np.zeros((N, K))
+    want[0, 5] = c
+    want[1, 256 + 200] = c / 4
+    assert np.array_equal(_decode_nvfp4(codes, sf, N, K) * float(g), want)
+
+
 def test_act_quant_lowrank_input_matches_matmul(oracle_mod):
     d = si.make_inputs(40, 512, 128, 7)
     codes, sf, g, t = oracle_mod.act_quant_nvfp4(d["x"], d["D"])
