@@ -101,6 +101,31 @@ MUTANTS = {
     # backward of the input
     "bwd_dy_column": (C, "double a = (double)or_bf16_to_f32(dy[rows[i] * N + n]);",
                       "double a = (double)or_bf16_to_f32(dy[rows[i] * N + (N - 1 - n)]);", 0),
+    # decoders, rotation of whole rows, absmax and rounding inside the codecs
+    "e2m1_decode_table": (C, "{0.0f, 0.5f, 1.0f, 1.5f, 2.0f, 3.0f, 4.0f, 6.0f};",
+                          "{0.0f, 0.5f, 1.0f, 1.5f, 2.0f, 3.0f, 4.0f, 5.0f};", 0),
+    "ue4m3_decode_bias": (C, "return (float)ldexp(8.0 + m, e - 7 - 3);", "return (float)ldexp(8.0 + m, e - 8 - 3);", 0),
+    "f16_decode_bias": (C, "v = ldexp(1024.0 + m, e - 15 - 10);", "v = ldexp(1024.0 + m, e - 14 - 10);", 0),
+    "rotate_first_block_only": (C, "v[i] = in[r * K + b + i];", "v[i] = in[r * K + i];", 0),
+    "int4_build_skips_rotation": (C, "            or_fwht256(v);\n            for (int g = 0; g < 8; g++) {",
+                                  "            for (int g = 0; g < 8; g++) {", 0),
+    "int4_scale_index": (C, "int64_t gi = n * (K / 32) + (b / 32) + g;", "int64_t gi = n * (K / 32) + g;", 0),
+    "int4_amax_half": (C, "for (int i = 0; i < 32; i++) {\n        float m = fabsf(r[i]);",
+                       "for (int i = 0; i < 16; i++) {\n        float m = fabsf(r[i]);", 0),
+    "int4_truncates": (C, "float rq = nearbyintf(v);", "float rq = truncf(v);", 0),
+    "g64_amax_half": (C, "for (int i = 0; i < 64; i++) {\n        float m = fabsf(r[i]);",
+                      "for (int i = 0; i < 32; i++) {\n        float m = fabsf(r[i]);", 0),
+    "g64_truncates": (C, "float rq = nearbyintf(v);", "float rq = truncf(v);", 1),
+    "nvfp4_absmax_unrotated": (C, "float A = absmax_f32(rot_scratch, N * K);", "float A = absmax_f32(R, N * K);", 0),
+    "nvfp4_sf_byte": (C, "sf_tiled[or_sf_offset(r, c, C)] = sf;", "sf_tiled[or_sf_offset(r, c, C) ^ 1] = sf;", 0),
+    "int8_build_skips_rotation": (C, "            or_fwht256(row + b);\n", "", 0),
+    "int8_amax_first_block": (C, "for (int64_t k = 0; k < K; k++) {\n        float m = fabsf(r[k]);",
+                              "for (int64_t k = 0; k < 256; k++) {\n        float m = fabsf(r[k]);", 0),
+    "int8_truncates": (C, "float rq = nearbyintf(v);", "float rq = truncf(v);", 2),
+    "lowrank_input_transposed": (C, "(double)or_bf16_to_f32(lora_down[k * rank + rr]);",
+                                 "(double)or_bf16_to_f32(lora_down[rr * K + k]);", 0),
+    "fwd_int8_row_scale": (C, "float d = (float)codes[n * K + k] * scales[n];",
+                           "float d = (float)codes[n * K + k] * scales[0];", 0),
     # SVD init ("Low-rank branch: rank-32 SVD of the weight")
     "svd_residual_sign": (C, "R[n * K + k] = W[n * K + k] - L;", "R[n * K + k] = W[n * K + k] + L;", 0),
     "svd_residual_index": (C, "L = fmaf(or_bf16_to_f32(up[n * rank + r]), or_bf16_to_f32(down[k * rank + r]), L);",
