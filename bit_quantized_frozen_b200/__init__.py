@@ -152,6 +152,39 @@ def _numel_bytes(t) -> int:
     return t.numel() * t.element_size()
 
 
+def _need(fn: str, name: str, t, nbytes: int):
+    """Raise before the call if tensor t holds fewer bytes than the entry point reads or writes
+    through it.  The C entry points take bare pointers and cannot see a buffer's end, so a short
+    tensor would be overrun on the device.  None (a NULL argument) and raw integer addresses are
+    passed through unchecked; the library validates the rest (shapes, alignment, flags)."""
+    if t is None or isinstance(t, int):
+        return
+    have = _numel_bytes(t)
+    if have < nbytes:
+        raise ValueError(f"{fn}: {name} holds {have} bytes, the call needs {nbytes}")
+
+
+def _need_weight(fn: str, w: "Weight"):
+    """The payload and low-rank factors of a built weight, sized by its format."""
+    N, K = int(w.N), int(w.K)
+    if N <= 0 or K <= 0:
+        return                                   # the library rejects the shape
+    if w.fmt == SQ_FMT_INT8_ROW:
+        _need(fn, "codes", w.codes, N * K)
+        _need(fn, "scales", w.scales, 4 * N)
+        rank = RANK_INT8
+    else:
+        _need(fn, "codes", w.codes, N * K // 2)
+        if w.fmt == SQ_FMT_NVFP4:
+            _need(fn, "scales", w.scales, sq_sf_bytes(N, K))
+            _need(fn, "g_w", w.g_w, 4)
+        elif w.fmt in (SQ_FMT_INT4_G32, SQ_FMT_INT4_G64):
+            _need(fn, "scales", w.scales, 2 * N * (K // (64 if w.fmt == SQ_FMT_INT4_G64 else 32)))
+        rank = RANK
+    _need(fn, "lora_up", w.lora_up, 2 * N * rank)
+    _need(fn, "lora_down", w.lora_down, 2 * K * rank)
+
+
 # ---- C entry points ----------------------------------------------------------
 
 def sq_abi_version() -> int:
@@ -168,6 +201,12 @@ def sq_workspace_bytes(op: int, M: int, N: int, K: int) -> int:
 
 def sq_build_int4(R, codes, scales, frac_idx=None, group: int = 32, stream=None):
     N, K = R.shape
+    if group in (32, 64):
+        fn, G = "sq_build_int4", N * (K // group)
+        _need(fn, "R", R, 4 * N * K)
+        _need(fn, "codes", codes, N * K // 2)
+        _need(fn, "scales", scales, 2 * G)
+        _need(fn, "frac_idx", frac_idx, G)
     _check("sq_build_int4", lib().sq_build_int4(_ptr(R), N, K, group, _ptr(codes), _ptr(scales), _ptr(frac_idx),
                                                 _stream(stream)))
 
@@ -176,31 +215,64 @@ def sq_svd_init(W, omega, iters, lora_up, lora_down, R, ws, stream=None):
     """The rank (32 or 16) is lora_up's number of columns."""
     N, K = W.shape
     rank = int(lora_up.shape[1])
+    fn = "sq_svd_init"
+    _need(fn, "W", W, 4 * N * K)
+    _need(fn, "omega", omega, 4 * K * RANK)
+    _need(fn, "lora_up", lora_up, 2 * N * rank)
+    _need(fn, "lora_down", lora_down, 2 * K * rank)
+    _need(fn, "R", R, 4 * N * K)
     _check("sq_svd_init", lib().sq_svd_init(_ptr(W), N, K, _ptr(omega), int(iters), rank, _ptr(lora_up),
                                             _ptr(lora_down), _ptr(R), _ptr(ws), _numel_bytes(ws), _stream(stream)))
 
 
 def sq_build_int8(R, codes, scales, frac_idx=None, stream=None):
     N, K = R.shape
+    fn = "sq_build_int8"
+    _need(fn, "R", R, 4 * N * K)
+    _need(fn, "codes", codes, N * K)
+    _need(fn, "scales", scales, 4 * N)
+    _need(fn, "frac_idx", frac_idx, N)
     _check("sq_build_int8", lib().sq_build_int8(_ptr(R), N, K, _ptr(codes), _ptr(scales), _ptr(frac_idx),
                                                 _stream(stream)))
 
 
 def sq_build_nvfp4(R, codes, sf_tiled, g_w, ws, stream=None):
     N, K = R.shape
+    fn = "sq_build_nvfp4"
+    _need(fn, "R", R, 4 * N * K)
+    _need(fn, "codes", codes, N * K // 2)
+    _need(fn, "sf_tiled", sf_tiled, sq_sf_bytes(N, K) if N > 0 and K > 0 else 0)
+    _need(fn, "g_w", g_w, 4)
     _check("sq_build_nvfp4", lib().sq_build_nvfp4(_ptr(R), N, K, _ptr(codes), _ptr(sf_tiled), _ptr(g_w), _ptr(ws),
                                                   _numel_bytes(ws), _stream(stream)))
 
 
 def sq_act_quant_nvfp4(x, codes, sf_tiled, g_x, lora_down=None, t=None, flags: int = 0, ws=None, stream=None):
     M, K = x.shape
+    fn = "sq_act_quant_nvfp4"
+    _need(fn, "x", x, 2 * M * K)
+    _need(fn, "codes", codes, M * K // 2)
+    _need(fn, "sf_tiled", sf_tiled, sq_sf_bytes(M, K) if M > 0 and K > 0 else 0)
+    _need(fn, "g_x", g_x, 4)
+    if lora_down is not None and t is not None:
+        _need(fn, "lora_down", lora_down, 2 * K * RANK)
+        _need(fn, "t", t, 4 * M * RANK)
     _check("sq_act_quant_nvfp4",
            lib().sq_act_quant_nvfp4(_ptr(x), M, K, _ptr(codes), _ptr(sf_tiled), _ptr(g_x), _ptr(lora_down), _ptr(t),
                                     flags, _ptr(ws), 0 if ws is None else _numel_bytes(ws), _stream(stream)))
 
 
+def _need_fwd(fn: str, w: "Weight", x, y, g_x, flags: int):
+    M = x.shape[0]
+    _need_weight(fn, w)
+    _need(fn, "x", x, 2 * M * int(w.K))
+    _need(fn, "y", y, M * int(w.N) * (2 if flags & SQ_OUT_BF16 else 4))
+    _need(fn, "g_x", g_x, 4)
+
+
 def sq_linear_fwd(w: "Weight", x, y, g_x=None, flags: int = 0, ws=None, stream=None):
     M = x.shape[0]
+    _need_fwd("sq_linear_fwd", w, x, y, g_x, flags)
     cw = w.as_c()
     _check("sq_linear_fwd", lib().sq_linear_fwd(ctypes.byref(cw), _ptr(x), M, _ptr(y), _ptr(g_x), flags, _ptr(ws),
                                                 0 if ws is None else _numel_bytes(ws), _stream(stream)))
@@ -210,6 +282,7 @@ def sq_linear_fwd_noalloc(w: "Weight", x, y, g_x=None, flags: int = 0, stream=No
     """sq_linear_fwd on libsq's static per-device scratch (no workspace);
     returns the scratch's device address (for sq_check_device_status)."""
     M = x.shape[0]
+    _need_fwd("sq_linear_fwd_noalloc", w, x, y, g_x, flags)
     cw = w.as_c()
     scratch = ctypes.c_void_p()
     _check("sq_linear_fwd_noalloc", lib().sq_linear_fwd_noalloc(ctypes.byref(cw), _ptr(x), M, _ptr(y), _ptr(g_x),
@@ -218,12 +291,18 @@ def sq_linear_fwd_noalloc(w: "Weight", x, y, g_x=None, flags: int = 0, stream=No
 
 
 def sq_reconstruct_bf16(w: "Weight", W_out, flags: int = 0, stream=None):
+    _need_weight("sq_reconstruct_bf16", w)
+    _need("sq_reconstruct_bf16", "W_out", W_out, 2 * int(w.N) * int(w.K))
     cw = w.as_c()
     _check("sq_reconstruct_bf16", lib().sq_reconstruct_bf16(ctypes.byref(cw), _ptr(W_out), flags, _stream(stream)))
 
 
 def sq_linear_bwd_dx(w: "Weight", dy, dx, ws, stream=None):
     M = dy.shape[0]
+    fn = "sq_linear_bwd_dx"
+    _need_weight(fn, w)
+    _need(fn, "dy", dy, 2 * M * int(w.N))
+    _need(fn, "dx", dx, 4 * M * int(w.K))
     cw = w.as_c()
     _check("sq_linear_bwd_dx", lib().sq_linear_bwd_dx(ctypes.byref(cw), _ptr(dy), M, _ptr(dx), _ptr(ws),
                                                       _numel_bytes(ws), _stream(stream)))
