@@ -10,8 +10,10 @@ Every routine follows the SquareQ README, section "SquareQ v3 -- W4
 (Hadamard-256 + low-rank + int4 / NVFP4)"; the C source states, routine by
 routine, which paragraph it follows and the reading taken where the page is
 silent.  Parity status: every routine here is pinned by the ``-m "not gpu"``
-tests in ``tests/test_oracle_pins.py`` (closed forms, invariants, library
-conversions, brute force); none is "parity unpinned".
+tests in ``tests/test_oracle_pins*.py`` (closed forms, invariants, library
+conversions, brute force); none is "parity unpinned".  ``tests/test_oracle_mutants.py``
+plants single mistakes in a scratch copy of this package and checks that a pin
+fails for each.
 """
 from __future__ import annotations
 
