@@ -190,11 +190,21 @@ def physical_gpu_index(local_rank: int) -> int:
 GEMM_SOURCES = ["bit_quantized_frozen_b200/csrc/sq_gemm.cu", "bit_quantized_frozen_b200/csrc/sq_ptx.cuh"]
 
 
-def gemm_source_hash() -> str:
+def code_only(text: str) -> str:
+    """C/C++ source without its comments, trailing blanks and empty lines."""
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    text = re.sub(r"//[^\n]*", "", text)
+    return "\n".join(ln.rstrip() for ln in text.splitlines() if ln.strip())
+
+
+def gemm_source_hash(read=None) -> str:
+    """First 16 hex digits of sha256 over the GEMM's sources with comments removed: an edit of a
+    comment keeps the ncu counters, any change of code drops them.  read(rel) returns a source's
+    text (default: the file in this tree)."""
+    read = read or (lambda rel: open(os.path.join(ROOT, rel)).read())
     h = hashlib.sha256()
     for rel in GEMM_SOURCES:
-        with open(os.path.join(ROOT, rel), "rb") as f:
-            h.update(f.read())
+        h.update(code_only(read(rel)).encode())
     return h.hexdigest()[:16]
 
 

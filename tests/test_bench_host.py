@@ -64,3 +64,14 @@ def test_traffic_only_for_the_profiled_source(monkeypatch):
     assert bench.profiled_traffic("no_such_workload") == (None, "no capture for this workload")
     monkeypatch.setattr(bench, "gemm_source_hash", lambda: "0" * 16)
     assert bench.profiled_traffic(bench.HEADLINE) == (None, "kernel changed since the ncu capture")
+
+
+def test_traffic_hash_ignores_comments_only():
+    src = {rel: open(f"{bench.ROOT}/{rel}").read() for rel in bench.GEMM_SOURCES}
+    base = bench.gemm_source_hash(src.__getitem__)
+    assert base == bench.gemm_source_hash()
+    first = bench.GEMM_SOURCES[0]
+    commented = dict(src, **{first: "// a new comment\n/* and a\n   block */\n" + src[first] + "\n\n// tail\n"})
+    assert bench.gemm_source_hash(commented.__getitem__) == base
+    edited = dict(src, **{first: src[first].replace("kStages", "kStages ", 1) + "\nstatic int extra;\n"})
+    assert bench.gemm_source_hash(edited.__getitem__) != base
