@@ -10,8 +10,9 @@
 //               = [U | U]; one extra kind::f16 K-step into the same accumulator
 //               adds (t / beta) U^T, so the epilogue only scales by beta.
 //
-// (SquareQ README, "Op-level parity of the full FP4 forward": block-scaled
-// GEMM + epilogue; "Residual codecs": int4 "dequant-first".)
+// (SquareQ README: the op-level parity paragraph of the FP4 forward names the
+// block-scaled GEMM and its epilogue; the "Residual codecs" paragraph makes the
+// int4 codec dequant-first.)
 //
 // CTA tile 128 x 256, one CTA per SM, 6 warps (+4 scale warps on the NVFP4 path):
 //   warps 0-3  epilogue: tcgen05.ld of their 32 accumulator lanes, scale,

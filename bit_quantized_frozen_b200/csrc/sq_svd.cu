@@ -1,5 +1,5 @@
-// sq_svd.cu -- SVD init of the rank-32 low-rank branch (SquareQ README,
-// "Low-rank branch: rank-32 SVD of the weight, always on, bf16"):
+// sq_svd.cu -- SVD init of the rank-32 low-rank branch (SquareQ README, the
+// "Low-rank branch" paragraph: a bf16 branch of rank 32 from the weight's SVD):
 //
 //   W [N, K] fp32  ->  lora_up   = bf16(U sqrt(sigma))  [N, 32]
 //                      lora_down = bf16(V sqrt(sigma))  [K, 32]

@@ -147,8 +147,8 @@ SQ_API size_t sq_sf_bytes(int64_t rows, int64_t K);
 SQ_API size_t sq_workspace_bytes(int op, int64_t M, int64_t N, int64_t K);
 
 /*
- * int4 builder (SquareQ README, "Residual codecs": int4 group-32/64 scales
- * with MSE-swept fractions).  For each row of R [N, K] fp32 (device): rotate
+ * int4 builder (SquareQ README, "Residual codecs": int4 codes with one scale
+ * per group of 32 or 64 values, its fraction of the absmax chosen by MSE).  For each row of R [N, K] fp32 (device): rotate
  * every 256-block with H256, then for each group of `group` (32 or 64)
  * rotated values r_i with a = max|r_i| try the fractions f_j = (50 + 2j)/100,
  * j = 0..25:
@@ -166,8 +166,8 @@ SQ_API sq_status sq_build_int4(const float *R, int64_t N, int64_t K, int32_t gro
                         void *stream);
 
 /*
- * SVD init of the low-rank branch (SquareQ README, "Low-rank branch: rank-32
- * SVD of the weight, always on, bf16"; "v3.1 -- int8-residual mode": rank 16):
+ * SVD init of the low-rank branch (SquareQ README, "Low-rank branch": a
+ * rank-32 bf16 branch from the weight's SVD; "v3.1 -- int8-residual mode": rank 16):
  * the step before the builders.  From W [N, K] fp32 (device) it writes, for
  * the `rank` (32, or 16 for SQ_FMT_INT8_ROW) largest singular values sigma,
  * lora_up = bf16(U sqrt(sigma)) [N, rank] and lora_down = bf16(V sqrt(sigma))
@@ -195,8 +195,8 @@ SQ_API sq_status sq_svd_init(const float *W, int64_t N, int64_t K, const float *
                              size_t ws_bytes, void *stream);
 
 /*
- * int8 per-row builder (SquareQ README, "v3.1 -- int8-residual mode": int8
- * per-row, MSE-swept, of the H256-rotated rank-16 residual).  For each row of
+ * int8 per-row builder (SquareQ README, "v3.1 -- int8-residual mode": the
+ * rotated residual of a rank-16 branch in int8, one MSE-chosen scale per row).  For each row of
  * R [N, K] fp32 (device, K <= 16384): rotate every 256-block with H256; with
  * a = max|r_k| over the row try the fractions f_j = (50 + 2j)/100,
  * j = 0..25, of the int4 sweep:
@@ -214,8 +214,8 @@ SQ_API sq_status sq_build_int8(const float *R, int64_t N, int64_t K, int8_t *cod
                                uint8_t *frac_idx, void *stream);
 
 /*
- * NVFP4 builder (SquareQ README, "Residual codecs": e2m1 + ue4m3 block-16
- * scales in the tiled layout + per-tensor global scale).  Pass 1 rotates R
+ * NVFP4 builder (SquareQ README, "Residual codecs": e2m1 codes, one ue4m3
+ * scale per 16 values in the tiled order, one fp32 scale for the tensor).  Pass 1 rotates R
  * [N, K] fp32 (device) and takes A = max|H R|; g_w = RN(A / 2688), i.e.
  * A / (6 * 448).  Pass 2 rotates again and, per 16 values with b = max|r|:
  *   sf = ue4m3(RN(b / RN(6 g_w))),  code_i = e2m1(RN(r_i RN(1 / RN(value(sf) g_w))))
@@ -230,8 +230,8 @@ SQ_API sq_status sq_build_nvfp4(const float *R, int64_t N, int64_t K,
 
 /*
  * Activation quantisation, the prologue of the NVFP4 forward (SquareQ README,
- * "Op-level parity of the full FP4 forward": H256-rotate + block-quant + tiled
- * scales).  x [M, K] bf16 (device) is rotated; g_x = RN(max|H x| / 2688)
+ * the op-level parity paragraph of the FP4 forward: the Hadamard rotation, block
+ * quantisation and tiled scales of x, fused in front of the GEMM).  x [M, K] bf16 (device) is rotated; g_x = RN(max|H x| / 2688)
  * unless SQ_ACT_STATIC_SCALE is set, in which case *g_x (device) is read as
  * given.  Then the same block-16 step as sq_build_nvfp4 with g_x.  Outputs
  * (device): codes [M, K/2], sf_tiled (sq_sf_bytes(M, K) bytes, padding rows
@@ -247,7 +247,11 @@ SQ_API sq_status sq_act_quant_nvfp4(const uint16_t *x, int64_t M, int64_t K,
                              void *ws, size_t ws_bytes, void *stream);
 
 /*
- * Forward y = x W^T, y [M, N] fp32 (device; with SQ_OUT_BF16 bf16, the
+ * Forward y = x W^T (SquareQ README, the op-level parity paragraph of the FP4
+ * forward: rotation, block quantisation and tiled scales of x, the
+ * GEMM and its epilogue; "Residual codecs": the int4 codec runs dequant-first;
+ * "v3.1 -- int8-residual mode" for int8).
+ * y [M, N] fp32 (device; with SQ_OUT_BF16 bf16, the
  * round-to-nearest-even of the same fp32 value, rounded once in the GEMM's
  * epilogue), x [M, K] bf16 (device).
  * Because H is symmetric, x W^T = H(x) deq(Q)^T + (x lora_down) lora_up^T.
@@ -307,8 +311,8 @@ SQ_API sq_status sq_linear_fwd_noalloc(const sq_weight *w, const uint16_t *x, in
                                        float *g_x, uint32_t flags, void **scratch_out, void *stream);
 
 /*
- * bf16 reconstruct of W for the backward pass (SquareQ README: "the bwd-side
- * bf16 reconstruct from the same payload").  For each element
+ * bf16 reconstruct of W for the backward pass (SquareQ README, the op-level parity
+ * paragraph: the backward rebuilds W in bf16 from the forward's payload).  For each element
  *   d = q s (int4, either group size), RN(q s_row) (int8) or
  *       RN(RN(e2m1 value(sf)) g_w) (NVFP4),
  *   h = H256 applied to each 256-block of d along K,
@@ -329,9 +333,9 @@ SQ_API sq_status sq_reconstruct_bf16(const sq_weight *w, uint16_t *W_out, uint32
 /*
  * Backward of the layer's input: dx = dy W, dy [M, N] bf16 (device), dx [M, K]
  * fp32 (device), W the bf16 reconstruct of the weight (low-rank term
- * included when the weight has one).  The SquareQ README runs the backward as
- * "the bwd-side bf16 reconstruct from the same payload" followed by the normal
- * bf16 GEMM ("End-to-end" paragraph); here the reconstruct writes W^T into
+ * included when the weight has one).  In the SquareQ README the backward
+ * rebuilds W in bf16 from the forward's payload and then runs an ordinary bf16
+ * GEMM ("End-to-end" paragraph); here the reconstruct writes W^T into
  * the workspace and the library's bf16 tensor-core GEMM (fp32 accumulation in
  * tensor memory) reduces over N.  Accuracy: max|dx - dx_exact| /
  * max|dx_exact| <= 2e-3 against dy W on the same bf16 operands.  ws:

@@ -379,7 +379,7 @@ def linear_bwd_dx(dy_bits, W_bits, rows=None):
     return dx
 
 
-# ---- SVD init of the low-rank branch ("Low-rank branch: rank-32 SVD of the weight") ----
+# ---- SVD init of the low-rank branch (SquareQ README, "Low-rank branch" paragraph) ----
 
 def svd_residual(W, up_bits, down_bits):
     """R = RN(W - L), L the fmaf chain over the factors' rank (32, or 16 for the int8 mode) of bf16

@@ -12,8 +12,8 @@
  *
  * with a block-diagonal normalised Hadamard-256 over the input dim
  * ("Rotation" paragraph), an int4 group-32/64 codec with MSE-swept scale
- * fractions or an NVFP4 codec (e2m1 codes, ue4m3 block-16 scales in the
- * cuBLASLt tiled layout, fp32 per-tensor global scale) ("Residual codecs"
+ * fractions or an NVFP4 codec (e2m1 codes; one ue4m3 scale per 16 values,
+ * stored in cuBLASLt's tiled order; one fp32 scale for the tensor) ("Residual codecs"
  * paragraph), and a rank-32 bf16 low-rank branch ("Low-rank branch"); plus
  * the v3.1 int8 mode (int8 per-row MSE-swept codes of the rotated residual,
  * rank-16 low-rank branch; section "v3.1 -- int8-residual mode").
@@ -357,7 +357,7 @@ void or_int4_group32(const float *r, int8_t *q_out, uint16_t *s_out, uint8_t *j_
 
 /*
  * One group of 64 rotated residual values: the group-64 variant the same
- * paragraph names beside group-32 ("int4 group-32/64 scales").  The same sweep
+ * paragraph allows beside group 32.  The same sweep
  * over the 64 values (a = max|r_i| over all 64); the pages give no order for
  * the squared-error sum, and the reading taken here is the group-32 rule per
  * half: each 32-value half is summed by the xor butterfly above (strides 16, 8,
@@ -501,8 +501,8 @@ void or_build_int4_g(const float *R, int64_t N, int64_t K, int group,
 
 /*
  * Byte offset of scale (row r, scale column c) in the tiled layout, C = K/16
- * scale columns per row (a multiple of 4).  The pages name "the cuBLASLt tiled
- * layout" without printing it; this is the publicly documented 1D
+ * scale columns per row (a multiple of 4).  The pages name cuBLASLt's tiled scale
+ * layout without printing it; this is the publicly documented 1D
  * block-scaling layout: 128-row x 4-column tiles of 512 bytes, tiles ordered
  * along the scale columns first, and inside a tile row r%32 picks a 16-byte
  * line, (r%128)/32 a 4-byte word in it and c%4 the byte.
@@ -526,7 +526,8 @@ float or_nvfp4_global_scale(float A)
 
 /*
  * One block of 16 rotated values with global scale g (SquareQ README,
- * "Residual codecs": e2m1 + ue4m3 block-16 scales + per-tensor global scale).
+ * "Residual codecs": e2m1 codes, a ue4m3 scale per 16 values and one fp32
+ * scale for the tensor).
  * b = max|r|, sf = ue4m3(RN(b / RN(6 g))); with den = RN(value(sf) * g) the
  * codes are e2m1(RN(r_i * RN(1/den))).  sf == 0 or g == 0 gives all-zero
  * codes.  codes8 gets 8 bytes, element 2k in the low nibble.
@@ -642,8 +643,8 @@ void or_act_quant_nvfp4(const uint16_t *x, int64_t M, int64_t K, int static_g,
 /*
  * Since W = U D^T + H(deq(Q)) and H is symmetric, y = x W^T =
  * H(x) deq(Q)^T + (x D) U^T: the rotation moves onto the activation
- * (SquareQ README, "Op-level parity of the full FP4 forward": rotate, block
- * quant, tiled scales, GEMM, epilogue).
+ * (SquareQ README, the op-level parity paragraph of the FP4 forward: rotation,
+ * block quantisation and tiled scales of x, then the GEMM and its epilogue).
  *
  * NVFP4 forward, fp64 on the exact decoded operands:
  *   y[m,n] = g_x g_w sum_k e2m1(xc[m,k]) sf_x(m,k/16) e2m1(wc[n,k]) sf_w(n,k/16)
@@ -790,7 +791,8 @@ static float int8_row_error(const float *p_in, int64_t K)
 
 /*
  * One row of K rotated residual values (SquareQ README, "v3.1 -- int8-residual
- * mode": int8 per-row, MSE-swept, of the H256-rotated rank-16 residual).
+ * mode": the rotated residual of a rank-16 branch in int8, one MSE-chosen
+ * scale per row).
  * a = max|r_k| over the row; for each fraction f_j of the int4 sweep
  * (j = 0..25) the fp32 scale is s = RN(RN(f_j a) / 127) and the codes
  * q_k = clamp(rint_even(RN(r_k RN(1/s))), -127, 127); the error of value k is
@@ -927,8 +929,8 @@ void or_lowrank_input(const uint16_t *x, int64_t M, int64_t K, const uint16_t *l
 /* ------------------------------------------------------------------------ */
 
 /*
- * W[n,k] = bf16( RN( L[n,k] + h[n,k] ) ) (SquareQ README, "the bwd-side bf16
- * reconstruct from the same payload"), where
+ * W[n,k] = bf16( RN( L[n,k] + h[n,k] ) ) (SquareQ README, the op-level parity
+ * paragraph: the backward's bf16 reconstruct from the forward's payload), where
  *   d = q * s (int4, exact) or RN(RN(e2m1 * value(sf)) * g_w) (NVFP4),
  *   h = inverse_H256 of d over each 256-block of the row (= the same FWHT),
  *   L = fmaf chain over r = 0..31 of U[n,r] * D[k,r], starting from 0.
@@ -1021,8 +1023,8 @@ void or_linear_bwd_dx(const uint16_t *dy, const uint16_t *W, int64_t M, int64_t 
 /*
  * R[n, k] = RN(W[n, k] - L[n, k]) with L the fmaf chain over r = 0..rank-1 of
  * up[n, r] * down[k, r] from 0 -- the same L the bf16 reconstruct adds back
- * (SquareQ README, "Low-rank branch: rank-32 SVD of the weight": the residual
- * is the weight minus the low-rank branch; "v3.1 -- int8-residual mode": rank
+ * (SquareQ README, "Low-rank branch" paragraph: the branch comes from the
+ * weight's SVD, and the residual is what is left of the weight; "v3.1 -- int8-residual mode": rank
  * 16).  W, R fp32 [N, K]; up [N, rank], down [K, rank] bf16 bits; rank 32 or 16.
  */
 void or_svd_residual(const float *W, const uint16_t *up, const uint16_t *down, int64_t N, int64_t K, int rank,

@@ -126,7 +126,7 @@ MUTANTS = {
                                  "(double)or_bf16_to_f32(lora_down[rr * K + k]);", 0),
     "fwd_int8_row_scale": (C, "float d = (float)codes[n * K + k] * scales[n];",
                            "float d = (float)codes[n * K + k] * scales[0];", 0),
-    # SVD init ("Low-rank branch: rank-32 SVD of the weight")
+    # SVD init (the "Low-rank branch" paragraph)
     "svd_residual_sign": (C, "R[n * K + k] = W[n * K + k] - L;", "R[n * K + k] = W[n * K + k] + L;", 0),
     "svd_residual_index": (C, "L = fmaf(or_bf16_to_f32(up[n * rank + r]), or_bf16_to_f32(down[k * rank + r]), L);",
                            "L = fmaf(or_bf16_to_f32(up[n * rank + r]), or_bf16_to_f32(down[k * rank + (rank - 1 - r)]), L);", 0),

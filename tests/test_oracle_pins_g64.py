@@ -1,5 +1,5 @@
-"""Pins of the oracle's int4 group-64 codec (SquareQ README, "Residual codecs":
-"int4 group-32/64 scales with MSE-swept fractions").
+"""Pins of the oracle's int4 group-64 codec (SquareQ README, "Residual codecs"
+paragraph: int4 scales per group of 32 or 64 values, the fraction chosen by MSE).
 
 Reading pinned here: the same 26-fraction sweep as group 32 over 64 values
 (a = max over all 64), with the squared-error sum taken as the group-32 xor

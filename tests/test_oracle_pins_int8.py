@@ -1,5 +1,5 @@
 """Pins of the oracle's int8 per-row codec (SquareQ README, "v3.1 -- int8-residual
-mode": int8 per-row, MSE-swept, of the H256-rotated rank-16 residual).
+mode": the rotated residual of a rank-16 branch in int8, one MSE-chosen scale per row).
 
 Readings pinned here: the int4 fraction grid f_j = (50 + 2j)/100, an fp32 row scale
 s = RN(RN(f_j a) / 127), codes clamp(rint(RN(r RN(1/s))), -127, 127), the error

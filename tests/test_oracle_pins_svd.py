@@ -1,5 +1,5 @@
 """Pins of the oracle's SVD init of the low-rank branch (SquareQ README, "Low-rank
-branch: rank-32 SVD of the weight, always on, bf16").
+branch" paragraph: a rank-32 bf16 branch taken from the weight's SVD).
 
 Readings pinned here: the rank-32 truncated SVD, singular values split evenly between
 the factors (up = U sqrt(sigma), down = V sqrt(sigma), each rounded to bf16 once), and

@@ -1,4 +1,4 @@
-"""int4 group-64 (SquareQ README, "Residual codecs": "int4 group-32/64 scales")
+"""int4 group-64 (SquareQ README, "Residual codecs" paragraph: groups of 32 or 64)
 through the C ABI against the CPU oracle on the same seeded inputs.
 
 The builder's codes, fp16 scales and winning fraction indices are compared bit

@@ -1,5 +1,5 @@
-"""SVD init of the rank-32 low-rank branch (SquareQ README, "Low-rank branch: rank-32
-SVD of the weight, always on, bf16") through the C ABI against the CPU oracle.
+"""SVD init of the rank-32 low-rank branch (SquareQ README, "Low-rank branch"
+paragraph) through the C ABI against the CPU oracle.
 
 The oracle takes the exact truncated SVD (fp64 LAPACK); the GPU runs subspace
 iteration from a seeded start block.  The test weights have a spectral gap at 32
