@@ -6,7 +6,6 @@ arm (the CPU oracle) runs and prints on rank 0 alone.
 """
 import json
 import os
-import socket
 import subprocess
 import sys
 
@@ -18,16 +17,9 @@ import torch.multiprocessing as mp
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 
 
-def _free_port() -> int:
-    with socket.socket() as s:
-        s.bind(("127.0.0.1", 0))
-        return s.getsockname()[1]
-
-
-def _rank_main(rank, world, port, out):
-    os.environ["MASTER_ADDR"] = "127.0.0.1"
-    os.environ["MASTER_PORT"] = str(port)
-    dist.init_process_group("gloo", rank=rank, world_size=world)
+def _rank_main(rank, world, store_path, out):
+    # a file rendezvous: no TCP port to race for
+    dist.init_process_group("gloo", init_method=f"file://{store_path}", rank=rank, world_size=world)
     try:
         sys.path.insert(0, ROOT)
         import bench
@@ -37,11 +29,10 @@ def _rank_main(rank, world, port, out):
         dist.destroy_process_group()
 
 
-def test_max_over_ranks_gloo_two_ranks():
-    port = _free_port()
+def test_max_over_ranks_gloo_two_ranks(tmp_path):
     with mp.Manager() as mgr:
         out = mgr.dict()
-        mp.spawn(_rank_main, args=(2, port, out), nprocs=2, join=True)
+        mp.spawn(_rank_main, args=(2, str(tmp_path / "store"), out), nprocs=2, join=True)
         res = dict(out)
     assert res[0] == res[1] == [1.0, 10.0, 5.0, 0.5]
 
@@ -53,9 +44,10 @@ def test_max_over_ranks_single_rank_is_identity():
 
 
 def test_reference_arm_under_torchrun_two_ranks():
-    port = _free_port()
-    cmd = [sys.executable, "-m", "torch.distributed.run", "--nnodes=1", "--nproc-per-node", "2",
-           "--master-addr", "127.0.0.1", "--master-port", str(port), os.path.join(ROOT, "bench.py"),
+    # --standalone binds the rendezvous store to a port of its own choosing: no window between
+    # picking a free port here and torchrun binding it
+    cmd = [sys.executable, "-m", "torch.distributed.run", "--standalone", "--local-addr", "127.0.0.1",
+           "--nproc-per-node", "2", os.path.join(ROOT, "bench.py"),
            "--impl", "reference", "--gpus", "2", "--steps", "1", "--warmup", "0", "--config", "tiny_64x256x512"]
     env = dict(os.environ, OMP_NUM_THREADS="2")
     r = subprocess.run(cmd, cwd=ROOT, env=env, capture_output=True, text=True, timeout=300)
