@@ -30,7 +30,7 @@ def _rank_main(rank, world, store_path, out):
 
 
 def test_max_over_ranks_gloo_two_ranks(tmp_path):
-    with mp.Manager() as mgr:
+    with mp.get_context("spawn").Manager() as mgr:       # no fork of a multi-threaded process
         out = mgr.dict()
         mp.spawn(_rank_main, args=(2, str(tmp_path / "store"), out), nprocs=2, join=True)
         res = dict(out)
