@@ -100,6 +100,14 @@ def _c(a, dtype):
     return np.ascontiguousarray(a, dtype=dtype)
 
 
+def _rows(rows, M):
+    """The evaluated rows as int64, all of them if None; each must index one of the M rows."""
+    rows = np.arange(M, dtype=np.int64) if rows is None else _c(rows, np.int64)
+    if rows.size and (rows.min() < 0 or rows.max() >= M):
+        raise IndexError(f"rows must lie in [0, {M})")
+    return rows
+
+
 def num_threads() -> int:
     return lib().or_num_threads()
 
@@ -270,7 +278,7 @@ def act_quant_nvfp4(x_bits, lora_down_bits=None, static_g=None):
 # ---- O7/O8 forward --------------------------------------------------------
 
 def linear_fwd_nvfp4(xc, xsf, g_x, wc, wsf, g_w, t, U_bits, M, N, K, rows=None):
-    rows = np.arange(M, dtype=np.int64) if rows is None else _c(rows, np.int64)
+    rows = _rows(rows, M)
     y = np.empty((len(rows), N), np.float64)
     xc, xsf, wc, wsf = (_c(a, np.uint8) for a in (xc, xsf, wc, wsf))
     t = None if t is None else _c(t, np.float64)
@@ -281,7 +289,7 @@ def linear_fwd_nvfp4(xc, xsf, g_x, wc, wsf, g_w, t, U_bits, M, N, K, rows=None):
 
 
 def linear_fwd_int4(xrot, codes, scales, t, U_bits, M, N, K, rows=None, group=32):
-    rows = np.arange(M, dtype=np.int64) if rows is None else _c(rows, np.int64)
+    rows = _rows(rows, M)
     y = np.empty((len(rows), N), np.float64)
     xrot = _c(xrot, np.float32)
     codes = _c(codes, np.uint8)
@@ -337,7 +345,7 @@ def lowrank_input(x_bits, lora_down_bits):
 
 def linear_fwd_int8(xrot, codes, scales, t, U_bits, M, N, K, rows=None):
     """y rows of the int8 forward, fp64 [n_rows, N]; t [M, 16] fp64 and U [N, 16] bf16 bits, or None."""
-    rows = np.arange(M, dtype=np.int64) if rows is None else _c(rows, np.int64)
+    rows = _rows(rows, M)
     y = np.empty((len(rows), N), np.float64)
     t = None if t is None else _c(t, np.float64)
     U = None if U_bits is None else _c(U_bits, np.uint16)
@@ -373,7 +381,7 @@ def linear_bwd_dx(dy_bits, W_bits, rows=None):
     W = _c(W_bits, np.uint16)
     M, N = dy.shape
     K = W.shape[1]
-    rows = np.arange(M, dtype=np.int64) if rows is None else _c(rows, np.int64)
+    rows = _rows(rows, M)
     dx = np.empty((len(rows), K), np.float64)
     lib().or_linear_bwd_dx(_p(dy), _p(W), M, N, K, _p(rows), len(rows), _p(dx))
     return dx

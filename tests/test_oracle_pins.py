@@ -425,6 +425,9 @@ def test_int4_forward_equals_decoded_gemm(oracle_mod):
     U = si.bf16_bits_to_f32(d["U"]).astype(np.float64)
     want = xb @ wb.T + t @ U.T
     assert np.allclose(y, want, rtol=1e-12, atol=1e-12 * np.abs(want).max())
+    rows = np.array([5, 0, 23])                      # a row subset evaluates exactly those rows
+    ys = oracle_mod.linear_fwd_int4(xr, codes, scales, t, d["U"], M, N, K, rows)
+    assert np.array_equal(ys, y[rows])
     x = si.bf16_bits_to_f32(d["x"]).astype(np.float64)
     Wtrue = U @ si.bf16_bits_to_f32(d["D"]).astype(np.float64).T + d["R"].astype(np.float64)
     ref = x @ Wtrue.T

@@ -106,6 +106,9 @@ def test_int8_forward_equals_decoded_gemm(oracle_mod):
     assert np.allclose(t, x @ D, rtol=1e-12, atol=1e-12 * np.abs(x @ D).max())
     want = xb @ wb.T + t @ U.T
     assert np.allclose(y, want, rtol=1e-12, atol=1e-12 * np.abs(want).max())
+    rows = np.array([5, 0, 19])                      # a row subset evaluates exactly those rows
+    ys = oracle_mod.linear_fwd_int8(xr, codes, scales, t, U16, M, N, K, rows)
+    assert np.array_equal(ys, y[rows])
     Wtrue = U @ D.T + d["R"].astype(np.float64)
     ref = x @ Wtrue.T
     cos = (y * ref).sum() / np.linalg.norm(y) / np.linalg.norm(ref)
