@@ -126,11 +126,23 @@ MUTANTS = {
                                  "(double)or_bf16_to_f32(lora_down[rr * K + k]);", 0),
     "fwd_int8_row_scale": (C, "float d = (float)codes[n * K + k] * scales[n];",
                            "float d = (float)codes[n * K + k] * scales[0];", 0),
+    # row subsets of the sampled forwards and backward, and the backward's zero skip
+    "fwd_nvfp4_x_scale_row": (C, "(double)or_ue4m3_to_f32(xsf[or_sf_offset(m, k / 16, C)]);",
+                              "(double)or_ue4m3_to_f32(xsf[or_sf_offset(i, k / 16, C)]);", 0),
+    "fwd_int4_x_row": (C, "xb[i * K + k] = (double)or_bf16_to_f32(or_f32_to_bf16(xrot[rows[i] * K + k]));",
+                       "xb[i * K + k] = (double)or_bf16_to_f32(or_f32_to_bf16(xrot[i * K + k]));", 0),
+    "fwd_int8_x_row": (C, "xb[i * K + k] = (double)or_bf16_to_f32(or_f32_to_bf16(xrot[rows[i] * K + k]));",
+                       "xb[i * K + k] = (double)or_bf16_to_f32(or_f32_to_bf16(xrot[i * K + k]));", 1),
+    "bwd_dy_row": (C, "double a = (double)or_bf16_to_f32(dy[rows[i] * N + n]);",
+                   "double a = (double)or_bf16_to_f32(dy[i * N + n]);", 0),
+    "bwd_skips_nonzero": (C, "if (a == 0.0)\n                continue;", "if (a != 0.0)\n                continue;", 0),
     # SVD init (the "Low-rank branch" paragraph)
     "svd_residual_sign": (C, "R[n * K + k] = W[n * K + k] - L;", "R[n * K + k] = W[n * K + k] + L;", 0),
     "svd_residual_index": (C, "L = fmaf(or_bf16_to_f32(up[n * rank + r]), or_bf16_to_f32(down[k * rank + r]), L);",
                            "L = fmaf(or_bf16_to_f32(up[n * rank + r]), or_bf16_to_f32(down[k * rank + (rank - 1 - r)]), L);", 0),
     "svd_sigma_not_split": (PY, "sq = np.sqrt(S[:rank])", "sq = S[:rank]", 0),
+    "svd_down_not_split": (PY, "down = (Vt[:rank].T * sq).astype(np.float32)",
+                           "down = (Vt[:rank].T * 1.0).astype(np.float32)", 0),
     "svd_skips_top_vector": (PY, "up = (U[:, :rank] * sq).astype(np.float32)",
                              "up = (U[:, 1:rank + 1] * sq).astype(np.float32)", 0),
 }
