@@ -291,7 +291,8 @@ def cpu_sample(d, M_s: int, N_s: int):
     return t, oracle.num_threads()
 
 
-SVD_SAMPLE_ROWS = 512      # the oracle's SVD init (fp64 LAPACK) runs on the first 512 rows of W
+SVD_SAMPLE_ROWS = 64       # the oracle's SVD init runs on the first 64 rows of W (its 64-vector
+                           # subspace then spans the sample's row space: two rounds)
 REF_SAMPLE = (64, 2048)    # reference arm, per step: M_s rows of x, N_s rows of R (all K)
 CPU_SAMPLE = (128, 4096)   # one-off CPU baseline of the GPU arm
 

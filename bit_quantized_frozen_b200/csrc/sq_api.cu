@@ -5,6 +5,7 @@
 #include <cuda_runtime.h>
 
 #include <atomic>
+#include <mutex>
 #include <cstdio>
 #include <cstring>
 
@@ -13,6 +14,35 @@
 #include "sq_ptx.cuh"
 
 static __device__ __align__(256) uint8_t g_noalloc_scratch[size_t(32) << 20];
+
+namespace sq {
+typedef CUresult (*PFN_ctxGetCurrent)(CUcontext *);
+typedef CUresult (*PFN_ctxGetId)(CUcontext, unsigned long long *);
+
+unsigned long long current_context_id()
+{
+    static PFN_ctxGetCurrent get_current = nullptr;
+    static PFN_ctxGetId get_id = nullptr;
+    if (!get_current || !get_id) {
+        void *p = nullptr, *q = nullptr;
+        cudaDriverEntryPointQueryResult r1, r2;
+        if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &r1) != cudaSuccess ||
+            r1 != cudaDriverEntryPointSuccess ||
+            cudaGetDriverEntryPoint("cuCtxGetId", &q, cudaEnableDefault, &r2) != cudaSuccess ||
+            r2 != cudaDriverEntryPointSuccess)
+            return 0;
+        get_current = reinterpret_cast<PFN_ctxGetCurrent>(p);
+        get_id = reinterpret_cast<PFN_ctxGetId>(q);
+    }
+    CUcontext c = nullptr;
+    unsigned long long id = 0;
+    if (get_current(&c) != CUDA_SUCCESS || !c || get_id(c, &id) != CUDA_SUCCESS)
+        return 0;
+    return id;
+}
+
+}  // namespace sq
+
 
 // One thread waits on an mbarrier that nothing ever arrives on, with the
 // bounded wait every kernel of the library uses; it must give up after
@@ -153,10 +183,20 @@ uint8_t *ws_at(void *ws, size_t off)
 // Static scratch of sq_linear_fwd_noalloc --------------------------------------
 // A fixed 32 MiB forward workspace that lives in the module's own device
 // memory (one copy per device, created when the module's device code is
-// loaded, released with the context), so that the call needs no allocation.
-// Its device address is looked up once per device, with that device current.
+// loaded into a context, released with the context), so that the call needs
+// no allocation.  Its device address is looked up with the device current,
+// once per device and context: the address is kept together with the ID of
+// the context it was looked up in, and looked up again when the current
+// context has another ID (after cudaDeviceReset, or once the primary context
+// was released and created again, the module is loaded anew and the array may
+// sit elsewhere).
 constexpr size_t kNoAllocScratchBytes = size_t(32) << 20;
-std::atomic<void *> g_noalloc_scratch_ptr[kMaxDevices];
+struct ScratchSlot {
+    void *ptr = nullptr;
+    unsigned long long ctx = 0;
+};
+ScratchSlot g_noalloc_scratch_slot[kMaxDevices];
+std::mutex g_noalloc_mutex;
 
 sq_status check_weight(const sq_weight *w)
 {
@@ -505,10 +545,18 @@ sq_status sq_linear_fwd_noalloc(const sq_weight *w, const uint16_t *x, int64_t M
         return st;
     int dev = 0;
     SQ_CUDA(cudaGetDevice(&dev), "cudaGetDevice");
-    void *scratch = g_noalloc_scratch_ptr[dev].load(std::memory_order_acquire);
-    if (!scratch) {                  // first call on this device: look the scratch up (device is current)
-        SQ_CUDA(cudaGetSymbolAddress(&scratch, g_noalloc_scratch), "cudaGetSymbolAddress(static scratch)");
-        g_noalloc_scratch_ptr[dev].store(scratch, std::memory_order_release);
+    void *scratch = nullptr;
+    {
+        // first call on this device and context: look the scratch up (the device is current)
+        const unsigned long long ctx = sq::current_context_id();
+        std::lock_guard<std::mutex> lock(g_noalloc_mutex);
+        ScratchSlot &slot = g_noalloc_scratch_slot[dev];
+        if (!slot.ptr || ctx == 0 || slot.ctx != ctx) {
+            slot.ptr = nullptr;
+            SQ_CUDA(cudaGetSymbolAddress(&slot.ptr, g_noalloc_scratch), "cudaGetSymbolAddress(static scratch)");
+            slot.ctx = ctx;
+        }
+        scratch = slot.ptr;
     }
     if (scratch_out)
         *scratch_out = scratch;

@@ -82,6 +82,12 @@ struct GemmLaunch {
 
 cudaError_t launch_gemm(const GemmLaunch &g, int sms, cudaStream_t stream);
 
+// ID of the current CUDA context (unique for the life of the process; a context created
+// after cudaDeviceReset gets a new one), 0 if it cannot be read.  Per-device caches of
+// symbol addresses and function attributes are keyed on it: a new context loads the
+// library's device code again, so those have to be looked up or set again.
+unsigned long long current_context_id();
+
 // 2D row-major tensor map [rows, inner] of esize-byte elements, box [box_rows, box_inner]
 bool make_tmap(CUtensorMap *m, CUtensorMapDataType dt, int esize, const void *base, uint64_t inner,
                uint64_t rows, uint32_t box_inner, uint32_t box_rows, CUtensorMapSwizzle sw);

@@ -1584,21 +1584,22 @@ static bool stream_map(CUtensorMap *tm, const T *in, int64_t rows, int64_t K)
                      32, (uint64_t)(rows * K / 32), 32, 256, f32 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B);
 }
 
-// shared-memory opt-in, once per device and kernel (keyed on the kernel itself:
-// kernels with the same signature must not share the flag)
+// shared-memory opt-in, once per device, context and kernel (keyed on the kernel
+// itself: kernels with the same signature must not share the flag)
 template <typename T, auto k>
 static cudaError_t stream_attr()
 {
     constexpr int kMaxDev = 64;
-    static bool done[kMaxDev];
+    static unsigned long long done_ctx[kMaxDev];
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDev)
         return cudaErrorInvalidDevice;
-    if (done[dev])
+    const unsigned long long ctx = current_context_id();
+    if (ctx != 0 && done_ctx[dev] == ctx)
         return cudaSuccess;
     cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, StreamCfg<T>::kSmem);
     if (e == cudaSuccess)
-        done[dev] = true;
+        done_ctx[dev] = ctx;
     return e;
 }
 
@@ -1705,16 +1706,17 @@ cudaError_t launch_int8_build(const float *R, int64_t N, int64_t K, int8_t *code
     if (K > kI8MaxK)
         return cudaErrorInvalidValue;
     constexpr int kMaxDev = 64;
-    static bool attr_done[kMaxDev];
+    static unsigned long long attr_ctx[kMaxDev];
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDev)
         return cudaErrorInvalidDevice;
-    if (!attr_done[dev]) {
+    const unsigned long long ctx = current_context_id();
+    if (ctx == 0 || attr_ctx[dev] != ctx) {
         cudaError_t e = cudaFuncSetAttribute(int8_build_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                              i8_smem_bytes(kI8MaxK));
         if (e != cudaSuccess)
             return e;
-        attr_done[dev] = true;
+        attr_ctx[dev] = ctx;
     }
     // persistent CTAs over rows: only as many as are resident at once (registers and
     // shared memory), so that no CTA waits for a whole earlier CTA's share of rows
@@ -1775,15 +1777,16 @@ cudaError_t launch_act_pass1(const uint16_t *x, int64_t M, int64_t K, const uint
                              float *t32, uint32_t *status, int sms, cudaStream_t s)
 {
     constexpr int kMaxDev = 64;
-    static bool attr_done[kMaxDev];
+    static unsigned long long attr_ctx[kMaxDev];
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDev)
         return cudaErrorInvalidDevice;
-    if (!attr_done[dev]) {
+    const unsigned long long ctx = current_context_id();
+    if (ctx == 0 || attr_ctx[dev] != ctx) {
         cudaError_t e = cudaFuncSetAttribute(act_pass1_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kP1Smem);
         if (e != cudaSuccess)
             return e;
-        attr_done[dev] = true;
+        attr_ctx[dev] = ctx;
     }
     CUtensorMap tmx, tmd;
     memset(&tmd, 0, sizeof(tmd));
@@ -1837,16 +1840,17 @@ static cudaError_t launch_reconstruct_v(const uint8_t *codes, const void *scales
     constexpr bool kTile = LOWRANK || TRANS;
     constexpr int kSmem = kTile ? Cfg::kSmemLowrank : Cfg::kSmemResidual;
     constexpr int kMaxDev = 64;
-    static bool attr_done[kMaxDev];
+    static unsigned long long attr_ctx[kMaxDev];
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDev)
         return cudaErrorInvalidDevice;
-    if (kTile && !attr_done[dev]) {
+    const unsigned long long ctx = current_context_id();
+    if (kTile && (ctx == 0 || attr_ctx[dev] != ctx)) {
         cudaError_t e = cudaFuncSetAttribute(reconstruct_kernel<FMT, LOWRANK, TRANS>,
                                              cudaFuncAttributeMaxDynamicSharedMemorySize, kSmem);
         if (e != cudaSuccess)
             return e;
-        attr_done[dev] = true;
+        attr_ctx[dev] = ctx;
     }
     const int64_t tiles = (K / kHad) * ((N + kRecRows - 1) / kRecRows);
     const int64_t per_sm = kTile ? 2 : 3;                   // resident CTAs per SM (registers, shared memory)
@@ -1863,19 +1867,20 @@ static cudaError_t launch_reconstruct_ws(const uint8_t *codes, const void *scale
 {
     constexpr int kSmem = RecWsCfg<FMT>::kSmem;
     constexpr int kMaxDev = 64;
-    static bool attr_done[kMaxDev];
+    static unsigned long long attr_ctx[kMaxDev];
     static uint32_t *status_word[kMaxDev];
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDev)
         return cudaErrorInvalidDevice;
-    if (!attr_done[dev]) {
+    const unsigned long long ctx = current_context_id();
+    if (ctx == 0 || attr_ctx[dev] != ctx) {
         cudaError_t e = cudaFuncSetAttribute(reconstruct_ws_kernel<FMT, TRANS>,
                                              cudaFuncAttributeMaxDynamicSharedMemorySize, kSmem);
         if (e == cudaSuccess)
             e = library_status_word(&status_word[dev]);
         if (e != cudaSuccess)
             return e;
-        attr_done[dev] = true;
+        attr_ctx[dev] = ctx;
     }
     const int64_t tiles = (K / kHad) * ((N + kRecRows - 1) / kRecRows);
     const unsigned grid = (unsigned)(tiles < sms ? tiles : sms);

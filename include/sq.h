@@ -299,7 +299,11 @@ SQ_API sq_status sq_linear_fwd(const sq_weight *w, const uint16_t *x, int64_t M,
  *
  * The first call on each device looks up the scratch's address
  * (cudaGetSymbolAddress, with that device current), which may load libsq's
- * device code; make that first call before any stream capture.  Nothing has
+ * device code; make that first call before any stream capture.  The address
+ * is kept with the ID of the CUDA context it was looked up in and looked up
+ * again in a new context (after cudaDeviceReset, or after the primary context
+ * was released and created again), so a call never uses an address from a
+ * context that no longer exists.  Nothing has
  * to start at zero: each call clears the status word and the absmax
  * accumulator at the start of its own stream work, like sq_linear_fwd.
  *

@@ -78,6 +78,9 @@ _SIGS = {
     "or_linear_bwd_dx": ([_P, _P, _I64, _I64, _I64, _P, _I64, _P], None),
     "or_svd_residual": ([_P, _P, _P, _I64, _I64, ctypes.c_int, _P], None),
     "or_f32_to_bf16_n": ([_P, _I64, _P], None),
+    "or_f64_to_bf16": ([ctypes.c_double], ctypes.c_uint16),
+    "or_svd_top": ([_P, _I64, _I64, ctypes.c_int, ctypes.c_int, _P, _P, _P], ctypes.c_int),
+    "or_svd_init": ([_P, _I64, _I64, ctypes.c_int, ctypes.c_int, _P, _P, _P, _P], ctypes.c_int),
 }
 
 
@@ -402,19 +405,38 @@ def svd_residual(W, up_bits, down_bits):
     return R
 
 
-def svd_init(W, rank=32):
-    """Truncated SVD of W [N, K] (fp64 LAPACK through numpy: a library step) ->
-    (lora_up bf16 bits [N, rank], lora_down bf16 bits [K, rank], R fp32 [N, K], sigma fp64 [rank]).
-    The singular values are split evenly: up = U sqrt(sigma), down = V sqrt(sigma), each rounded
-    to bf16 once (round to nearest even); R = RN(W - L) with the fmaf chain of svd_residual."""
+SVD_MAX_ITER = 500
+
+
+def f64_to_bf16(v) -> int:
+    """bf16 bits of a float64, rounded once (nearest, ties to even)."""
+    return int(lib().or_f64_to_bf16(float(v)))
+
+
+def svd_top(W, rank=32, max_iter=SVD_MAX_ITER):
+    """Leading singular triplets of W [N, K] by the oracle's fp64 subspace iteration with a
+    one-sided Jacobi Rayleigh-Ritz step (sq_oracle.c, or_svd_top) -> (sigma [rank], u [N, rank],
+    v [K, rank], iterations)."""
     W = _c(W, np.float32)
-    U, S, Vt = np.linalg.svd(W.astype(np.float64), full_matrices=False)
-    sq = np.sqrt(S[:rank])
-    up = (U[:, :rank] * sq).astype(np.float32)
-    down = (Vt[:rank].T * sq).astype(np.float32)
-    up_b = np.empty(up.shape, np.uint16)
-    down_b = np.empty(down.shape, np.uint16)
-    for src, dst in ((up, up_b), (down, down_b)):
-        src = np.ascontiguousarray(src)
-        lib().or_f32_to_bf16_n(_p(src), src.size, _p(dst))
-    return up_b, down_b, svd_residual(W, up_b, down_b), S[:rank]
+    N, K = W.shape
+    s = np.empty(rank, np.float64)
+    u = np.empty((N, rank), np.float64)
+    v = np.empty((K, rank), np.float64)
+    it = lib().or_svd_top(_p(W), N, K, int(rank), int(max_iter), _p(s), _p(u), _p(v))
+    return s, u, v, it
+
+
+def svd_init(W, rank=32, max_iter=SVD_MAX_ITER):
+    """Truncated SVD of W [N, K] in scalar C (sq_oracle.c, or_svd_init) ->
+    (lora_up bf16 bits [N, rank], lora_down bf16 bits [K, rank], R fp32 [N, K], sigma fp64 [rank]).
+    The singular values are split evenly: up = u sqrt(sigma), down = v sqrt(sigma), each rounded
+    from fp64 to bf16 once (nearest, ties to even); R = RN(W - L) with the fmaf chain of
+    svd_residual."""
+    W = _c(W, np.float32)
+    N, K = W.shape
+    up = np.empty((N, rank), np.uint16)
+    down = np.empty((K, rank), np.uint16)
+    R = np.empty((N, K), np.float32)
+    s = np.empty(rank, np.float64)
+    lib().or_svd_init(_p(W), N, K, int(rank), int(max_iter), _p(up), _p(down), _p(R), _p(s))
+    return up, down, R, s

@@ -1040,3 +1040,300 @@ void or_svd_residual(const float *W, const uint16_t *up, const uint16_t *down, i
         }
     }
 }
+
+/* ------------------------------------------------------------------------ */
+/* SVD init: the rank-32 (or rank-16) truncated SVD of the weight            */
+/* ------------------------------------------------------------------------ */
+
+/*
+ * bf16 of an fp64 value, rounded once (round to nearest, ties to even) on the
+ * bf16 grid: 7 fraction bits, fp32's exponent range, overflow to infinity.
+ * Going through fp32 first would round twice, which differs whenever the fp32
+ * value lands on a bf16 midpoint that the fp64 value is not on.
+ */
+uint16_t or_f64_to_bf16(double v)
+{
+    uint16_t sign = signbit(v) ? 0x8000u : 0u;
+    if (isnan(v))
+        return (uint16_t)(sign | 0x7FC0u);
+    if (isinf(v))
+        return (uint16_t)(sign | 0x7F80u);
+    double r = round_to_grid(fabs(v), 7, -126);      /* a / spacing is exact for any double */
+    if (r >= ldexp(1.0, 128))
+        return (uint16_t)(sign | 0x7F80u);
+    float rf = (float)r;                               /* exact: r is on the bf16 grid */
+    uint32_t rb;
+    memcpy(&rb, &rf, 4);
+    return (uint16_t)(sign | (rb >> 16));
+}
+
+/* start block of the subspace iteration: a 64-bit linear congruential
+ * sequence (Knuth's MMIX multiplier and increment), top 53 bits as a uniform
+ * value in [-1, 1) */
+static double lcg_uniform(uint64_t *s)
+{
+    *s = *s * 6364136223846793005ull + 1442695040888963407ull;
+    return (double)(*s >> 11) * ldexp(1.0, -52) - 1.0;
+}
+
+static double dot_f64(const double *a, const double *b, int64_t n)
+{
+    double s = 0.0;
+    for (int64_t i = 0; i < n; i++)
+        s += a[i] * b[i];
+    return s;
+}
+
+/*
+ * Orthonormalise the p vectors (each `len` long, stored one after another) by
+ * modified Gram-Schmidt, applied twice.  A vector that has (next to) nothing
+ * left after the projections is replaced by a fresh start vector and
+ * projected again, so the result always has p orthonormal columns.
+ */
+static void orthonormalise(double *A, int64_t len, int p, uint64_t *seed)
+{
+    for (int j = 0; j < p; j++) {
+        double *a = A + (int64_t)j * len;
+        for (int attempt = 0; attempt < 4; attempt++) {
+            double before = sqrt(dot_f64(a, a, len));
+            for (int pass = 0; pass < 2; pass++)
+                for (int i = 0; i < j; i++) {
+                    const double *q = A + (int64_t)i * len;
+                    double c = dot_f64(q, a, len);
+                    for (int64_t t = 0; t < len; t++)
+                        a[t] -= c * q[t];
+                }
+            double nrm = sqrt(dot_f64(a, a, len));
+            if (nrm > 0.0 && nrm > 1e-10 * before) {
+                for (int64_t t = 0; t < len; t++)
+                    a[t] /= nrm;
+                break;
+            }
+            for (int64_t t = 0; t < len; t++)
+                a[t] = lcg_uniform(seed);
+        }
+    }
+}
+
+/*
+ * One-sided Jacobi (Hestenes): rotate pairs of the p columns of B (each `len`
+ * long, stored one after another) until every pair is orthogonal to within
+ * tol, applying the same rotations to the columns of J (p x p, starts as I).
+ * A pair (i, j) with a_ii = |b_i|^2, a_jj = |b_j|^2, a_ij = b_i . b_j is
+ * rotated by the angle that zeroes a_ij: zeta = (a_jj - a_ii) / (2 a_ij),
+ * t = sign(zeta) / (|zeta| + sqrt(1 + zeta^2)), c = 1 / sqrt(1 + t^2), s = c t,
+ * b_i <- c b_i - s b_j, b_j <- s b_i + c b_j.  Pairs are visited row by row.
+ */
+static void jacobi_onesided(double *B, int64_t len, int p, double *J, double tol)
+{
+    for (int sweep = 0; sweep < 100; sweep++) {
+        int rotated = 0;
+        for (int i = 0; i < p - 1; i++)
+            for (int j = i + 1; j < p; j++) {
+                double *bi = B + (int64_t)i * len, *bj = B + (int64_t)j * len;
+                double aii = dot_f64(bi, bi, len), ajj = dot_f64(bj, bj, len), aij = dot_f64(bi, bj, len);
+                if (aii == 0.0 || ajj == 0.0 || fabs(aij) <= tol * sqrt(aii * ajj))
+                    continue;
+                double zeta = (ajj - aii) / (2.0 * aij);
+                double t = copysign(1.0, zeta) / (fabs(zeta) + sqrt(1.0 + zeta * zeta));
+                double c = 1.0 / sqrt(1.0 + t * t), s = c * t;
+                for (int64_t e = 0; e < len; e++) {
+                    double x = bi[e], y = bj[e];
+                    bi[e] = c * x - s * y;
+                    bj[e] = s * x + c * y;
+                }
+                double *ji = J + (int64_t)i * p, *jj = J + (int64_t)j * p;
+                for (int e = 0; e < p; e++) {
+                    double x = ji[e], y = jj[e];
+                    ji[e] = c * x - s * y;
+                    jj[e] = s * x + c * y;
+                }
+                rotated++;
+            }
+        if (!rotated)
+            return;
+    }
+}
+
+/* Z[j][n] = sum_k W[n][k] V[j][k]  (vectors V[j] of length K, Z[j] of length N) */
+static void mul_w(const float *W, int64_t N, int64_t K, const double *V, int p, double *Z)
+{
+#pragma omp parallel for schedule(static)
+    for (int64_t n = 0; n < N; n++)
+        for (int j = 0; j < p; j++) {
+            const float *w = W + n * K;
+            const double *v = V + (int64_t)j * K;
+            double s = 0.0;
+            for (int64_t k = 0; k < K; k++)
+                s += (double)w[k] * v[k];
+            Z[(int64_t)j * N + n] = s;
+        }
+}
+
+/* Y[j][k] = sum_n W[n][k] U[j][n], each sum taken over n in order */
+static void mul_wt(const float *W, int64_t N, int64_t K, const double *U, int p, double *Y)
+{
+    const int64_t kblk = 256;
+#pragma omp parallel for schedule(static)
+    for (int64_t k0 = 0; k0 < K; k0 += kblk) {
+        int64_t k1 = k0 + kblk < K ? k0 + kblk : K;
+        for (int j = 0; j < p; j++)
+            for (int64_t k = k0; k < k1; k++)
+                Y[(int64_t)j * K + k] = 0.0;
+        for (int64_t n = 0; n < N; n++) {
+            const float *w = W + n * K;
+            for (int j = 0; j < p; j++) {
+                double u = U[(int64_t)j * N + n];
+                double *y = Y + (int64_t)j * K;
+                for (int64_t k = k0; k < k1; k++)
+                    y[k] += (double)w[k] * u;
+            }
+        }
+    }
+}
+
+/*
+ * Leading singular triplets of W [N, K] fp32 (SquareQ README, "Low-rank
+ * branch" paragraph: the branch is taken from the weight's SVD).  Block
+ * subspace iteration in fp64 with p = min(64, N, K) vectors:
+ *     V <- orthonormal start block [K, p]
+ *     repeat:  B = W V;  one-sided Jacobi on B's columns (B J = U S, the
+ *              Rayleigh-Ritz step: the SVD of W restricted to span V);
+ *              U = B J / S, V <- V J, sorted by S descending;
+ *              Y = W^T U;  stop when |y_i - s_i v_i| <= 1e-13 s_0 for every
+ *              i < rank (the triplets are singular triplets of W to that
+ *              residual);  else V <- orthonormalised Y.
+ * With p = min(N, K) one step spans W's whole row space, so the result is
+ * the full SVD's leading part.  Outputs: sigma[rank] descending, u [N, rank]
+ * and v [K, rank] (row-major), each pair's sign fixed so that its largest |v|
+ * entry (first one on a tie) is positive.  Returns the number of iterations.
+ */
+int or_svd_top(const float *W, int64_t N, int64_t K, int rank, int max_iter, double *sigma, double *u_out,
+               double *v_out)
+{
+    int p = 64;
+    if (p > N)
+        p = (int)N;
+    if (p > K)
+        p = (int)K;
+    const int stride = rank;                /* row stride of u_out, v_out */
+    if (rank > p)
+        rank = p;                           /* triplets beyond min(N, K) are zero */
+    double *V = (double *)malloc(sizeof(double) * (size_t)(K * p));
+    double *B = (double *)malloc(sizeof(double) * (size_t)(N * p));
+    double *Y = (double *)malloc(sizeof(double) * (size_t)(K * p));
+    double *J = (double *)malloc(sizeof(double) * (size_t)(p * p));
+    double *VJ = (double *)malloc(sizeof(double) * (size_t)(K * p));
+    double *S = (double *)malloc(sizeof(double) * (size_t)p);
+    int *ord = (int *)malloc(sizeof(int) * (size_t)p);
+    uint64_t seed = 0x5EEDull;
+    for (int64_t i = 0; i < K * p; i++)
+        V[i] = lcg_uniform(&seed);
+    orthonormalise(V, K, p, &seed);
+    const double jtol = 1e-15 * sqrt((double)N);
+    int it;
+    for (it = 1;; it++) {
+        mul_w(W, N, K, V, p, B);
+        for (int i = 0; i < p * p; i++)
+            J[i] = (i / p == i % p) ? 1.0 : 0.0;
+        jacobi_onesided(B, N, p, J, jtol);
+        /* V J, column norms of B J, U = B J / S (stored back into B) */
+        for (int j = 0; j < p; j++) {
+            double *vj = VJ + (int64_t)j * K;
+            for (int64_t k = 0; k < K; k++) {
+                double s = 0.0;
+                for (int i = 0; i < p; i++)
+                    s += V[(int64_t)i * K + k] * J[(int64_t)j * p + i];
+                vj[k] = s;
+            }
+            double *b = B + (int64_t)j * N;
+            S[j] = sqrt(dot_f64(b, b, N));
+            for (int64_t n = 0; n < N; n++)
+                b[n] = S[j] > 0.0 ? b[n] / S[j] : 0.0;
+        }
+        /* order by S descending (stable) */
+        for (int j = 0; j < p; j++)
+            ord[j] = j;
+        for (int a = 1; a < p; a++)
+            for (int b2 = a; b2 > 0 && S[ord[b2]] > S[ord[b2 - 1]]; b2--) {
+                int t = ord[b2];
+                ord[b2] = ord[b2 - 1];
+                ord[b2 - 1] = t;
+            }
+        mul_wt(W, N, K, B, p, Y);
+        double s0 = S[ord[0]], worst = 0.0;
+        for (int i = 0; i < rank; i++) {
+            const double *y = Y + (int64_t)ord[i] * K, *vj = VJ + (int64_t)ord[i] * K;
+            double r2 = 0.0;
+            for (int64_t k = 0; k < K; k++) {
+                double d = y[k] - S[ord[i]] * vj[k];
+                r2 += d * d;
+            }
+            if (sqrt(r2) > worst)
+                worst = sqrt(r2);
+        }
+        if (s0 == 0.0 || worst <= 1e-13 * s0 || it >= max_iter)
+            break;
+        memcpy(V, Y, sizeof(double) * (size_t)(K * p));
+        orthonormalise(V, K, p, &seed);
+    }
+    for (int i = 0; i < rank; i++) {
+        const double *ui = B + (int64_t)ord[i] * N, *vi = VJ + (int64_t)ord[i] * K;
+        int64_t big = 0;
+        for (int64_t k = 1; k < K; k++)
+            if (fabs(vi[k]) > fabs(vi[big]))
+                big = k;
+        double sg = vi[big] < 0.0 ? -1.0 : 1.0;
+        sigma[i] = S[ord[i]];
+        for (int64_t n = 0; n < N; n++)
+            u_out[n * stride + i] = sg * ui[n];
+        for (int64_t k = 0; k < K; k++)
+            v_out[k * stride + i] = sg * vi[k];
+    }
+    for (int i = rank; i < stride; i++) {
+        sigma[i] = 0.0;
+        for (int64_t n = 0; n < N; n++)
+            u_out[n * stride + i] = 0.0;
+        for (int64_t k = 0; k < K; k++)
+            v_out[k * stride + i] = 0.0;
+    }
+    free(V);
+    free(B);
+    free(Y);
+    free(J);
+    free(VJ);
+    free(S);
+    free(ord);
+    return it;
+}
+
+/*
+ * SVD init of the low-rank branch: the leading 32 singular triplets
+ * (or_svd_top), of which the first `rank` (32, or 16 for the int8 mode's
+ * branch: its 16 leading pairs) make the factors, the singular values split
+ * evenly between them,
+ *     up[n, i] = bf16(u[n, i] sqrt(sigma_i)),  down[k, i] = bf16(v[k, i] sqrt(sigma_i)),
+ * each rounded from fp64 to bf16 once, and R = RN(W - L) with L the
+ * reconstruct's fmaf chain over the rank (or_svd_residual).  Returns the
+ * iteration count.
+ */
+int or_svd_init(const float *W, int64_t N, int64_t K, int rank, int max_iter, uint16_t *up, uint16_t *down,
+                float *R, double *sigma)
+{
+    double *u = (double *)malloc(sizeof(double) * (size_t)(N * 32));
+    double *v = (double *)malloc(sizeof(double) * (size_t)(K * 32));
+    double s32[32];
+    int it = or_svd_top(W, N, K, 32, max_iter, s32, u, v);
+    for (int i = 0; i < rank; i++) {
+        sigma[i] = s32[i];
+        double rs = sqrt(sigma[i]);
+        for (int64_t n = 0; n < N; n++)
+            up[n * rank + i] = or_f64_to_bf16(u[n * 32 + i] * rs);
+        for (int64_t k = 0; k < K; k++)
+            down[k * rank + i] = or_f64_to_bf16(v[k * 32 + i] * rs);
+    }
+    free(u);
+    free(v);
+    or_svd_residual(W, up, down, N, K, rank, R);
+    return it;
+}

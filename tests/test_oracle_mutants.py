@@ -140,11 +140,17 @@ MUTANTS = {
     "svd_residual_sign": (C, "R[n * K + k] = W[n * K + k] - L;", "R[n * K + k] = W[n * K + k] + L;", 0),
     "svd_residual_index": (C, "L = fmaf(or_bf16_to_f32(up[n * rank + r]), or_bf16_to_f32(down[k * rank + r]), L);",
                            "L = fmaf(or_bf16_to_f32(up[n * rank + r]), or_bf16_to_f32(down[k * rank + (rank - 1 - r)]), L);", 0),
-    "svd_sigma_not_split": (PY, "sq = np.sqrt(S[:rank])", "sq = S[:rank]", 0),
-    "svd_down_not_split": (PY, "down = (Vt[:rank].T * sq).astype(np.float32)",
-                           "down = (Vt[:rank].T * 1.0).astype(np.float32)", 0),
-    "svd_skips_top_vector": (PY, "up = (U[:, :rank] * sq).astype(np.float32)",
-                             "up = (U[:, 1:rank + 1] * sq).astype(np.float32)", 0),
+    "svd_sigma_not_split": (C, "double rs = sqrt(sigma[i]);", "double rs = sigma[i];", 0),
+    "svd_down_not_split": (C, "down[k * rank + i] = or_f64_to_bf16(v[k * 32 + i] * rs);",
+                           "down[k * rank + i] = or_f64_to_bf16(v[k * 32 + i]);", 0),
+    "svd_skips_top_vector": (C, "const double *ui = B + (int64_t)ord[i] * N, *vi = VJ + (int64_t)ord[i] * K;",
+                             "const double *ui = B + (int64_t)ord[i + 1] * N, *vi = VJ + (int64_t)ord[i + 1] * K;", 0),
+    "svd_rounds_through_f32": (C, "up[n * rank + i] = or_f64_to_bf16(u[n * 32 + i] * rs);",
+                               "up[n * rank + i] = or_f32_to_bf16((float)(u[n * 32 + i] * rs));", 0),
+    "svd_jacobi_rotation_sign": (C, "bi[e] = c * x - s * y;", "bi[e] = c * x + s * y;", 0),
+    "svd_sorted_ascending": (C, "S[ord[b2]] > S[ord[b2 - 1]]", "S[ord[b2]] < S[ord[b2 - 1]]", 0),
+    "svd_stops_early": (C, "worst <= 1e-13 * s0", "worst <= 1e-3 * s0", 0),
+    "f64_bf16_fraction_bits": (C, "round_to_grid(fabs(v), 7, -126)", "round_to_grid(fabs(v), 6, -126)", 0),
 }
 
 

@@ -1,7 +1,8 @@
 """SVD init of the rank-32 low-rank branch (SquareQ README, "Low-rank branch"
 paragraph) through the C ABI against the CPU oracle.
 
-The oracle takes the exact truncated SVD (fp64 LAPACK); the GPU runs subspace
+The oracle takes the truncated SVD in scalar C (fp64 subspace iteration run to a 1e-13
+residual, one-sided Jacobi Rayleigh-Ritz steps); the GPU runs 8 rounds of subspace
 iteration from a seeded start block.  The test weights have a spectral gap at 32
 (sigma_32 / sigma_33 >= 3, checked), so the rank-32 product L = up down^T is unique
 and the iteration error, (sigma_33 / sigma_32)^(2 iters) <= 3^-16, is negligible.

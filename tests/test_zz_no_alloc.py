@@ -63,6 +63,68 @@ def test_noalloc_matches_workspace_forward(sq, name, fmt):
     sq.sq_check_device_status(scratch[1])
 
 
+VARIANTS = {
+    # id: (format, flag name or None, pass g_x)
+    "nvfp4-no-gx": (2, None, False),
+    "nvfp4-bf16-out": (2, "SQ_OUT_BF16", True),
+    "nvfp4-static-scale": (2, "SQ_ACT_STATIC_SCALE", True),
+    "int4-g64": (3, None, False),
+    "int8-row": (4, None, False),
+}
+
+
+@pytest.mark.gpu
+@pytest.mark.parametrize("variant", list(VARIANTS))
+def test_noalloc_variants_match_workspace_forward(sq, variant):
+    """The other layouts the static scratch is carved into: the NVFP4 forward without a g_x
+    pointer (the scale then lives inside the scratch), with bf16 output, with a static activation
+    scale; the group-64 int4 and the int8 per-row formats (the latter with its widened rank-16
+    factors).  Each against sq_linear_fwd with a caller workspace on the same inputs, two calls in
+    a row, bit for bit (the same kernels run on the same values), and the scratch's status word
+    read back clean."""
+    assert torch.cuda.is_available(), "GPU tests need a CUDA device"
+    fmt, flag, pass_g = VARIANTS[variant]
+    flags = getattr(sq, flag) if flag else 0
+    d = si.make_config("tiny_64x256x512")
+    M, K = d["x"].shape
+    N = d["R"].shape[0]
+    R, U, D = to_dev(d["R"]), bf16_dev(d["U"]), bf16_dev(d["D"])
+    if fmt == 2:
+        w = sq.build_nvfp4(R, U, D)
+    elif fmt == 3:
+        w = sq.build_int4(R, U, D, group=64)
+    else:
+        w = sq.build_int8(R, U[:, :16].contiguous(), D[:, :16].contiguous())
+    x = bf16_dev(d["x"])
+    ydt = torch.bfloat16 if flags & sq.SQ_OUT_BF16 else torch.float32
+    static = torch.tensor([0.0123], dtype=torch.float32, device="cuda")
+
+    def g_in():
+        if flags & sq.SQ_ACT_STATIC_SCALE:
+            return static.clone()
+        return torch.full((1,), -1.0, dtype=torch.float32, device="cuda") if pass_g else None
+
+    y_ref = torch.empty((M, N), dtype=ydt, device="cuda")
+    op = {2: sq.SQ_OP_LINEAR_FWD_NVFP4, 4: sq.SQ_OP_LINEAR_FWD_INT8}.get(fmt, sq.SQ_OP_LINEAR_FWD_INT4)
+    g_ref = g_in()
+    sq.sq_linear_fwd(w, x, y_ref, g_x=g_ref, flags=flags, ws=sq.workspace(op, M, N, K))
+    torch.cuda.synchronize()
+    ref = y_ref.view(torch.int16 if ydt == torch.bfloat16 else torch.int32).cpu().numpy()
+    assert np.all(np.isfinite(y_ref.float().cpu().numpy())) and y_ref.float().abs().max().item() > 0
+    scratch = []
+    for call in range(2):
+        y = torch.full((M, N), float("nan"), dtype=ydt, device="cuda")
+        g = g_in()
+        scratch.append(sq.sq_linear_fwd_noalloc(w, x, y, g_x=g, flags=flags))
+        torch.cuda.synchronize()
+        got = y.view(torch.int16 if ydt == torch.bfloat16 else torch.int32).cpu().numpy()
+        assert np.array_equal(got, ref), f"{variant}, call {call}: output differs from the workspace forward"
+        if g is not None:
+            assert host(g)[0] == host(g_ref)[0], f"{variant}, call {call}: g_x differs"
+        sq.sq_check_device_status(scratch[-1])
+    assert scratch[0] and scratch[0] == scratch[1]
+
+
 def test_noalloc_rejects_shape_beyond_scratch(sq):
     # NVFP4 at N = 16384, K = 6144 fits M = 8462 rows, not 8463: refused before
     # any device work (the weight pointers are never touched).
