@@ -155,7 +155,7 @@ FwdLayout fwd_layout(int fmt, int64_t M, int64_t N, int64_t K)
         L.a = take((size_t)M * (size_t)K * 2);
         L.b = take((size_t)N * (size_t)K * 2);
     }
-    L.t32 = take((size_t)M * 32 * 4);
+    L.t32 = take((size_t)sq::act_t_parts(M, K) * (size_t)M * 32 * 4);   // partial tiles of t
     L.tsplit = take((size_t)M * 64 * 2);
     L.udup = take((size_t)N * 64 * 2);
     if (fmt == SQ_FMT_INT8_ROW) {                 // rank-16 factors widened to rank 32
@@ -263,8 +263,11 @@ size_t sq_workspace_bytes(int op, int64_t M, int64_t N, int64_t K)
         return kHeader;
     case SQ_OP_BUILD_NVFP4:
         return kHeader;
-    case SQ_OP_ACT_QUANT_NVFP4:
-        return kHeader;
+    case SQ_OP_ACT_QUANT_NVFP4: {
+        // the partial tiles of t = x lora_down when K is split over several CTAs
+        const int parts = sq::act_t_parts(M, K);
+        return parts > 1 ? kAlign + round_up((size_t)parts * (size_t)M * 32 * 4, kAlign) : kHeader;
+    }
     case SQ_OP_LINEAR_FWD_NVFP4:
         return fwd_layout(SQ_FMT_NVFP4, M, N, K).total;
     case SQ_OP_LINEAR_FWD_INT4:
@@ -392,16 +395,24 @@ sq_status sq_act_quant_nvfp4(const uint16_t *x, int64_t M, int64_t K, uint8_t *c
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     const bool stat = (flags & SQ_ACT_STATIC_SCALE) != 0;
     const bool with_t = lora_down && t;
+    const int parts = sq::act_t_parts(M, K);
+    float *t_part = !with_t ? nullptr : parts > 1 ? reinterpret_cast<float *>(ws_at(ws, kAlign)) : t;
     uint32_t *amax = reinterpret_cast<uint32_t *>(ws_at(ws, 4));
     SQ_CUDA(cudaMemsetAsync(ws, 0, 8, s), "memset");          // status word + absmax
     if (flags & SQ_CHECK_FINITE)
         SQ_CUDA(sq::launch_check_finite_bf16(x, M * K, reinterpret_cast<uint32_t *>(ws), sms, s), "finite check");
     if (!stat || with_t)
-        SQ_CUDA(sq::launch_act_pass1(x, M, K, lora_down, stat ? nullptr : amax, with_t ? t : nullptr,
-                                             reinterpret_cast<uint32_t *>(ws), sms, s),
+        SQ_CUDA(sq::launch_act_pass1(x, M, K, lora_down, stat ? nullptr : amax, t_part,
+                                     reinterpret_cast<uint32_t *>(ws), sms, s),
                 "activation pass 1");
+    sq::LowrankOut lr;                                          // t = the sum of the partial tiles
+    if (with_t && parts > 1) {
+        lr.t_part = t_part;
+        lr.parts = parts;
+        lr.t_out = t;
+    }
     SQ_CUDA(sq::launch_nvfp4_quant_bf16(x, M, K, amax, stat ? g_x : nullptr, stat ? nullptr : g_x, codes, sf_tiled,
-                                        sq::LowrankOut{}, sms, s),
+                                        lr, reinterpret_cast<uint32_t *>(ws), sms, s),
             "nvfp4 quant");
     return SQ_OK;
 }
@@ -462,7 +473,8 @@ sq_status sq_linear_fwd(const sq_weight *w, const uint16_t *x, int64_t M, void *
         // the quantisation also writes the low-rank operands (g_x is known by then)
         sq::LowrankOut lr;
         if (lora) {
-            lr.t32 = t32;
+            lr.t_part = t32;
+            lr.parts = sq::act_t_parts(M, K);
             lr.g_w = w->g_w;
             lr.tsplit = tsplit;
             lr.U = w->lora_up;
@@ -470,7 +482,7 @@ sq_status sq_linear_fwd(const sq_weight *w, const uint16_t *x, int64_t M, void *
             lr.udup = udup;
         }
         SQ_CUDA(sq::launch_nvfp4_quant_bf16(x, M, K, amax, stat ? gx : nullptr, stat ? nullptr : gx, xc, xsf, lr,
-                                            sms, s),
+                                            status, sms, s),
                 "nvfp4 act quant + low-rank operands");
         g.fp4 = 1;
         g.a = xc;
@@ -502,7 +514,8 @@ sq_status sq_linear_fwd(const sq_weight *w, const uint16_t *x, int64_t M, void *
                 Uw = u32;
             }
             SQ_CUDA(sq::launch_act_pass1(x, M, K, Dw, nullptr, t32, status, sms, s), "low-rank input");
-            SQ_CUDA(sq::launch_lowrank_finish(t32, M, nullptr, nullptr, tsplit, Uw, N, udup, sms, s),
+            SQ_CUDA(sq::launch_lowrank_finish(t32, sq::act_t_parts(M, K), M, nullptr, nullptr, tsplit, Uw, N, udup,
+                                              sms, s),
                     "low-rank operands");
         }
         g.fp4 = 0;

@@ -228,6 +228,100 @@ __device__ __forceinline__ void fwht256_l32s_unscaled(float (&v)[32], int lane)
         f2_unpack(p[j], v[2 * j], v[2 * j + 1]);
 }
 
+// ---------------------------------------------------------------------------
+// Hadamard-256 over 4 lanes, without the final 1/16 (fwht256_q4_from_s2: the
+// strides from 2 on, for pairs whose stride-1 butterfly is done).
+//
+// Layout: the four quarters q = 0..3 of a 256-block sit in lanes 8q + r of a
+// warp (r = 0..7 picks one of eight blocks), and quarter q holds elements
+// 64q .. 64q+63 as pairs p[j] = (v[2j], v[2j+1]).  Stride 1 pairs the two
+// values of a pair, strides 2 .. 32 pair whole pairs inside the lane (packed
+// f32x2 arithmetic), strides 64 and 128 pair lane q with lane q ^ 1 (lane ^ 8)
+// and q ^ 2 (lane ^ 16).  The same butterflies with the same operands in the
+// same order of strides as the sequential transform, so every element equals
+// the sequential result (before its 1/16) bit for bit.
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ void fwht256_q4_from_s2(uint64_t (&p)[32], int lane)
+{
+#pragma unroll
+    for (int hp = 1; hp <= 16; hp <<= 1)          // strides 2 .. 32
+#pragma unroll
+        for (int j = 0; j < 32; ++j)
+            if ((j & hp) == 0) {
+                const uint64_t a = p[j], b = p[j + hp];
+                p[j] = f2_add(a, b);
+                p[j + hp] = f2_sub(a, b);
+            }
+#pragma unroll
+    for (int x = 8; x <= 16; x <<= 1) {           // strides 64, 128, across lanes
+        // lower lane: own + partner, upper lane: partner - own, one fma with +-1 each
+        const float sg = (lane & x) == 0 ? 1.0f : -1.0f;
+        const uint64_t sg2 = f2_pack(sg, sg);
+#pragma unroll
+        for (int j = 0; j < 32; ++j) {
+            float lo, hi;
+            f2_unpack(p[j], lo, hi);
+            const uint64_t o = f2_pack(__shfl_xor_sync(0xffffffffu, lo, x), __shfl_xor_sync(0xffffffffu, hi, x));
+            p[j] = f2_fma(sg2, p[j], o);
+        }
+    }
+}
+
+__device__ __forceinline__ void fwht256_q4_unscaled(uint64_t (&p)[32], int lane)
+{
+#pragma unroll
+    for (int j = 0; j < 32; ++j) {               // stride 1, inside each pair
+        float a, b;
+        f2_unpack(p[j], a, b);
+        p[j] = f2_pack(__fadd_rn(a, b), __fsub_rn(a, b));
+    }
+    fwht256_q4_from_s2(p, lane);
+}
+
+// 64 bf16 values (one 128-byte row R of a box of 64 columns stored with the
+// 128-byte swizzle: 16-byte piece i of the row at i ^ (R % 8)) as fp32 pairs.
+// Eight lanes reading the same piece of eight consecutive rows hit eight
+// different bank groups.
+__device__ __forceinline__ void load_row64_bf16_sw128(const uint8_t *box, int R, uint64_t (&p)[32])
+{
+    const uint8_t *row = box + R * 128;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+        const uint4 a = *reinterpret_cast<const uint4 *>(row + 16 * (i ^ (R & 7)));
+        const uint32_t w[4] = {a.x, a.y, a.z, a.w};
+#pragma unroll
+        for (int j = 0; j < 4; ++j)
+            p[4 * i + j] = f2_pack(__uint_as_float(w[j] << 16), __uint_as_float(w[j] & 0xFFFF0000u));
+    }
+}
+
+// The same row with the stride-1 butterfly folded into the widening (mixed
+// bf16 + fp32 arithmetic: one rounding each, like the fp32 butterfly on the
+// exactly widened values): pair j becomes (RN(v[2j] + v[2j+1]),
+// RN(v[2j+1] - v[2j])), i.e. the second value NEGATED.  Every later stride
+// pairs values of equal parity, so the odd values stay exactly negated through
+// the transform (round to nearest is symmetric); callers undo the sign where it
+// matters (a maximum of |v| does not care).
+__device__ __forceinline__ void load_row64_bf16_sw128_s1(const uint8_t *box, int R, uint64_t (&p)[32])
+{
+    const uint8_t *row = box + R * 128;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+        const uint4 a = *reinterpret_cast<const uint4 *>(row + 16 * (i ^ (R & 7)));
+        const uint32_t w[4] = {a.x, a.y, a.z, a.w};
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            const float lo = __uint_as_float(w[j] << 16);
+            float sum, ndiff;
+            asm("{\n\t.reg .b16 h0, h1;\n\tmov.b32 {h0, h1}, %2;\n\t"
+                "add.rn.f32.bf16 %0, h1, %3;\n\t"
+                "sub.rn.f32.bf16 %1, h1, %3;\n\t}"
+                : "=f"(sum), "=f"(ndiff) : "r"(w[j]), "f"(lo));
+            p[4 * i + j] = f2_pack(sum, ndiff);
+        }
+    }
+}
+
 // max(a, b, c) in one instruction (sm_100)
 __device__ __forceinline__ float fmax3(float a, float b, float c)
 {

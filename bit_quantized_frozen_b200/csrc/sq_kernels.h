@@ -7,16 +7,24 @@
 
 namespace sq {
 
-// low-rank operands of the NVFP4 forward, written by the activation quant
-// kernel after its blocks (t32 == nullptr: nothing to write)
+// low-rank operands of the NVFP4 forward (and the final t of the activation
+// quantiser), written by the activation quant kernel before its blocks
+// (t_part == nullptr: nothing to write)
 struct LowrankOut {
-    const float *t32 = nullptr;      // [M, 32] fp32, t = x lora_down
+    const float *t_part = nullptr;   // [parts, M, 32] fp32 partial tiles of t = x lora_down (summed in order)
+    int parts = 1;
+    float *t_out = nullptr;          // [M, 32] fp32 t, or NULL
     const float *g_w = nullptr;      // weight global scale (beta = g_x g_w)
-    uint16_t *tsplit = nullptr;      // [M, 64] bf16
+    uint16_t *tsplit = nullptr;      // [M, 64] bf16, or NULL
     const uint16_t *U = nullptr;     // lora_up [N, 32] bf16
     int64_t N = 0;
-    uint16_t *udup = nullptr;        // [N, 64] bf16
+    uint16_t *udup = nullptr;        // [N, 64] bf16, or NULL
 };
+
+// K split of the activation pass that computes t = x lora_down: the pass
+// writes this many partial [M, 32] tiles (1: t itself), a function of the
+// shape only, so t is the same on every device for a given shape
+int act_t_parts(int64_t M, int64_t K);
 
 cudaError_t launch_absmax_rot_f32(const float *in, int64_t rows, int64_t K, uint32_t *amax, int sms,
                                   cudaStream_t s);
@@ -27,7 +35,7 @@ cudaError_t launch_nvfp4_quant_f32(const float *in, int64_t rows, int64_t K, con
                                    cudaStream_t s);
 cudaError_t launch_nvfp4_quant_bf16(const uint16_t *in, int64_t rows, int64_t K, const uint32_t *amax,
                                     const float *g_static, float *g_out, uint8_t *codes, uint8_t *sf,
-                                    const LowrankOut &lr, int sms, cudaStream_t s);
+                                    const LowrankOut &lr, uint32_t *status, int sms, cudaStream_t s);
 cudaError_t launch_int4_build(const float *R, int64_t N, int64_t K, int group, uint8_t *codes, uint16_t *scales,
                               uint8_t *frac, int sms, cudaStream_t s);
 // int8 per-row builder (K <= 16384), its dequant, and the rank-16 -> rank-32 widening
@@ -39,9 +47,10 @@ cudaError_t launch_widen_rank16(const uint16_t *src, int64_t rows, uint16_t *dst
 cudaError_t launch_rotate_bf16(const uint16_t *x, int64_t M, int64_t K, uint16_t *xb, int sms, cudaStream_t s);
 cudaError_t launch_dequant_int4(const uint8_t *codes, const uint16_t *scales, int group, int64_t N, int64_t K,
                                 uint16_t *wb, int sms, cudaStream_t s);
+// t_part: act_t_parts(M, K) partial tiles [parts, M, 32] (NULL: no t)
 cudaError_t launch_act_pass1(const uint16_t *x, int64_t M, int64_t K, const uint16_t *D, uint32_t *amax,
-                             float *t32, uint32_t *status, int sms, cudaStream_t s);
-cudaError_t launch_lowrank_finish(const float *t32, int64_t M, const float *g_x, const float *g_w,
+                             float *t_part, uint32_t *status, int sms, cudaStream_t s);
+cudaError_t launch_lowrank_finish(const float *t_part, int parts, int64_t M, const float *g_x, const float *g_w,
                                   uint16_t *tsplit, const uint16_t *U, int64_t N, uint16_t *udup, int sms,
                                   cudaStream_t s);
 // the library's own device status word (set by kernels of calls without a workspace)

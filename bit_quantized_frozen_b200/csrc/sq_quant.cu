@@ -172,15 +172,29 @@ __device__ __forceinline__ float lowrank_beta(float g_x, const float *g_w)
     return b == 0.0f ? 1.0f : b;
 }
 
-// unit i < M*8: t[m, 4c..4c+3] -> both halves of tsplit[m] (m = i/8, c = i%8);
+// unit i < M*8: t[m, 4c..4c+3] = the sum of the `parts` partial t tiles in
+// order (tp[j] = t_part + j*M*32), written to t_out (when non-NULL) and split
+// into both halves of tsplit[m] (when non-NULL) (m = i/8, c = i%8);
 // unit i >= M*8: 16-byte chunk c of U[n] -> both halves of udup[n] (n, c from i - M*8)
-__device__ __forceinline__ void lowrank_unit(int64_t i, int64_t nT, const float *__restrict__ t32, float beta,
-                                             uint16_t *__restrict__ tsplit, const uint16_t *__restrict__ U,
-                                             uint16_t *__restrict__ udup)
+__device__ __forceinline__ void lowrank_unit(int64_t i, int64_t nT, const float *__restrict__ t_part, int parts,
+                                             float *__restrict__ t_out, float beta, uint16_t *__restrict__ tsplit,
+                                             const uint16_t *__restrict__ U, uint16_t *__restrict__ udup)
 {
     if (i < nT) {
         const int64_t m = i >> 3, c = i & 7;
-        const float4 t4 = *reinterpret_cast<const float4 *>(t32 + m * kRank + 4 * c);
+        const int64_t M = nT >> 3;
+        float4 t4 = *reinterpret_cast<const float4 *>(t_part + m * kRank + 4 * c);
+        for (int j = 1; j < parts; ++j) {
+            const float4 a = *reinterpret_cast<const float4 *>(t_part + (j * M + m) * kRank + 4 * c);
+            t4.x = __fadd_rn(t4.x, a.x);
+            t4.y = __fadd_rn(t4.y, a.y);
+            t4.z = __fadd_rn(t4.z, a.z);
+            t4.w = __fadd_rn(t4.w, a.w);
+        }
+        if (t_out)
+            *reinterpret_cast<float4 *>(t_out + m * kRank + 4 * c) = t4;
+        if (!tsplit)
+            return;
         const float tv[4] = {t4.x, t4.y, t4.z, t4.w};
         uint32_t hi[4], lo[4];
 #pragma unroll
@@ -192,7 +206,7 @@ __device__ __forceinline__ void lowrank_unit(int64_t i, int64_t nT, const float 
         *reinterpret_cast<uint2 *>(tsplit + m * 64 + 4 * c) = make_uint2(hi[0] | (hi[1] << 16), hi[2] | (hi[3] << 16));
         *reinterpret_cast<uint2 *>(tsplit + m * 64 + 32 + 4 * c) =
             make_uint2(lo[0] | (lo[1] << 16), lo[2] | (lo[3] << 16));
-    } else {
+    } else if (udup) {
         const int64_t j = i - nT;
         const int64_t n = j >> 2, c = j & 3;
         const uint4 u = *reinterpret_cast<const uint4 *>(U + n * kRank + 8 * c);
@@ -234,13 +248,13 @@ __global__ void __launch_bounds__(kStreamThreads) nvfp4_quant_kernel(const __gri
         sixg = __fmul_rn(6.0f, g);
         if (g_out && blockIdx.x == 0 && c == 0)
             *g_out = g;
-        if (!lr.t32)
+        if (!lr.t_part)
             return;
         const float beta = lowrank_beta(g, lr.g_w);
-        const int64_t nT = rows * 8, total = nT + lr.N * 4;
+        const int64_t nT = rows * 8, total = nT + (lr.udup ? lr.N * 4 : 0);
         const int64_t stride = (int64_t)gridDim.x * (32 * kStreamConsumers);
         for (int64_t i = (int64_t)blockIdx.x * (32 * kStreamConsumers) + c; i < total; i += stride)
-            lowrank_unit(i, nT, lr.t32, beta, lr.tsplit, lr.U, lr.udup);
+            lowrank_unit(i, nT, lr.t_part, lr.parts, lr.t_out, beta, lr.tsplit, lr.U, lr.udup);
     };
     stream_blocks<T>(&tm, rows_pad * kb_per_row, nullptr, [&](int64_t b, float (&v)[32], bool valid) {
         fwht256_l32(v, lane);
@@ -654,29 +668,43 @@ __global__ void __launch_bounds__(256) dequant_int4_kernel(const uint32_t *__res
 
 // ---------------------------------------------------------------------------
 // Activation pass 1: one read of x for two results.
-//   amax (optional): max |H x| over the whole tensor (the activation global
-//                    scale's input), from the 8-lane Hadamard transform;
-//   t32 (optional):  t = x . lora_down, fp32 [M, 32], on mma.sync bf16 tensor
-//                    cores (fp32 accumulation, summed in a fixed order, so t
-//                    is deterministic for a given shape and SM count).
-// A CTA owns 32 rows and a range of 256-column chunks; when there are few row
-// tiles, K is split over a cluster of `split` CTAs (one per range) whose
-// partial t tiles are summed in rank order by rank 0 through distributed
-// shared memory.  One producer warp streams each chunk -- the x tile (32 x 256,
-// four TMA boxes of 64 columns, 128-byte swizzle) and the lora_down tile
-// (256 x 32, one box, 64-byte swizzle) -- into a 3-deep ring with mbarriers;
-// every consumer warp transforms 4 rows and runs 4 of the chunk's 16 k-steps
-// for one 16-row half of the tile, then releases the stage on its own.
+//   amax (optional):   max |H x| over the whole tensor (the activation global
+//                      scale's input), from the 4-lane Hadamard transform;
+//   t_part (optional): t = x . lora_down on the tcgen05 tensor cores (fp32
+//                      accumulation in tensor memory), as `split` partial
+//                      [M, 32] tiles, one per range of K, which the consumer
+//                      adds in order (t is deterministic for a given shape).
+// A CTA owns 128 rows (the MMA's M) and one of `split` ranges of 256-column
+// chunks (blockIdx.x = tile * split + range).  One producer warp streams each
+// chunk -- the x tile (128 x 256, four TMA boxes of 64 columns, 128-byte
+// swizzle) and the lora_down tile (256 x 32, one box, 64-byte swizzle) --
+// into a 2-deep ring; sixteen consumer warps each transform eight rows
+// (fwht256_q4_unscaled) and release the stage as soon as their rows are in
+// registers; one thread issues the chunk's 16 MMAs (M = 128, N = 32, K = 16)
+// straight from the stage.
 // ---------------------------------------------------------------------------
-constexpr int kP1Rows = 32;
-constexpr int kP1XBytes = kP1Rows * kHad * 2;      // 16 KB
-constexpr int kP1DBytes = kHad * kRank * 2;        // 16 KB
+constexpr int kP1Rows = 128;
+constexpr int kP1BoxBytes = kP1Rows * 128;          // 128 rows x 64 bf16
+constexpr int kP1XBytes = 4 * kP1BoxBytes;          // 64 KB
+constexpr int kP1DBytes = kHad * kRank * 2;         // 16 KB
 constexpr int kP1BufBytes = kP1XBytes + kP1DBytes;
-constexpr int kP1Stages = 3;
-constexpr int kP1Consumers = 8;
+constexpr int kP1Stages = 2;
+constexpr int kP1Consumers = 16;                    // 8 rows each
 constexpr int kP1Threads = 32 * (kP1Consumers + 2);   // + TMA producer warp + MMA warp
 constexpr int kP1Smem = kP1Stages * kP1BufBytes + 1024 + 256;   // ring, 1 KB alignment, barriers
-constexpr int kP1MaxSplit = 8;
+constexpr int kP1MaxSplit = 16;
+constexpr int kP1SplitSms = 148;                    // K split sized for one CTA per SM of a B200
+
+int act_t_parts(int64_t M, int64_t K)
+{
+    const int64_t tiles = (M + kP1Rows - 1) / kP1Rows;
+    const int64_t nkb = K / kHad;
+    int64_t split = kP1SplitSms / (tiles < 1 ? 1 : tiles);
+    split = split < 1 ? 1 : split;
+    split = split > kP1MaxSplit ? kP1MaxSplit : split;
+    split = split > nkb ? nkb : split;
+    return (int)split;
+}
 
 __device__ __forceinline__ void cp_async16(uint32_t dst, const void *src, uint32_t src_bytes)
 {
@@ -694,50 +722,16 @@ __device__ __forceinline__ void cp_async_wait()
     asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
 }
 
-__device__ __forceinline__ void ldmatrix_x4(uint32_t addr, uint32_t (&r)[4])
+// barrier over the first `threads` threads of the CTA (named barrier 1)
+__device__ __forceinline__ void bar_sync_named(uint32_t threads)
 {
-    asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0, %1, %2, %3}, [%4];"
-                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]) : "r"(addr));
+    asm volatile("bar.sync 1, %0;" ::"r"(threads) : "memory");
 }
 
-__device__ __forceinline__ void ldmatrix_x4_trans(uint32_t addr, uint32_t (&r)[4])
-{
-    asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0, %1, %2, %3}, [%4];"
-                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]) : "r"(addr));
-}
-
-__device__ __forceinline__ void mma_bf16_16816(float (&c)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1)
-{
-    asm volatile("mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 "
-                 "{%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, {%0, %1, %2, %3};\n"
-                 : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
-                 : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
-}
-
-// x stage: 16-byte chunk c (0..31) of row r -- box c / 8, 128-byte swizzle
-__device__ __forceinline__ uint32_t p1_xoff(int r, int c)
-{
-    return (uint32_t)((c >> 3) * 4096 + r * 128 + 16 * ((c & 7) ^ (r & 7)));
-}
-
-// lora_down stage: 16-byte chunk c (0..3) of k-row k -- 64-byte swizzle
-__device__ __forceinline__ uint32_t p1_doff(int k, int c)
-{
-    return (uint32_t)(k * 64 + 16 * (c ^ ((k >> 1) & 3)));
-}
-
-__device__ __forceinline__ float ld_shared_cluster_f32(uint32_t addr)
-{
-    float v;
-    asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(v) : "r"(addr) : "memory");
-    return v;
-}
-
-// t = x . lora_down on the tensor cores: one thread issues, per chunk, 16 MMAs
-// (M = 128, N = 32, K = 16, bf16 -> fp32 in tensor memory).  A is the x stage
-// (K-major, 128B swizzle); only rows 0..31 are the tile's, the MMA's other 96
-// rows read the rest of the stage and their results are never read.  B is the
-// lora_down stage, N-major (32 values of a k-row are one 64-byte swizzled row).
+// t = x . lora_down on the tensor cores: per chunk 16 MMAs (M = 128, N = 32,
+// K = 16, bf16 -> fp32 in tensor memory).  A is the x stage (K-major, 128B
+// swizzle, four boxes of 128 rows); B is the lora_down stage, N-major (32
+// values of a k-row are one 64-byte swizzled row).
 constexpr uint32_t kP1Idesc = (1u << 4) | (1u << 7) | (1u << 10) | (1u << 16) | ((uint32_t)(kRank >> 3) << 17) |
                               ((uint32_t)(128 >> 4) << 24);
 __device__ __forceinline__ uint64_t p1_bdesc(uint32_t saddr)
@@ -746,12 +740,13 @@ __device__ __forceinline__ uint64_t p1_bdesc(uint32_t saddr)
            ((uint64_t)1u << 46) | ((uint64_t)4u << 61);
 }
 
-__global__ void __launch_bounds__(kP1Threads, 2) act_pass1_kernel(const __grid_constant__ CUtensorMap tmx,
+__global__ void __launch_bounds__(kP1Threads, 1) act_pass1_kernel(const __grid_constant__ CUtensorMap tmx,
                                                                   const __grid_constant__ CUtensorMap tmd,
                                                                   int64_t M, int64_t K, uint32_t *__restrict__ amax,
-                                                                  float *__restrict__ t32, int split,
+                                                                  float *__restrict__ t_part, int split,
                                                                   uint32_t *__restrict__ status)
 {
+    float *const t32 = t_part;                        // non-NULL: this CTA writes partial tile j of t
     extern __shared__ uint8_t p1_raw[];
     uint8_t *p1_smem =
         reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(p1_raw) + 1023) & ~uintptr_t(1023));
@@ -763,7 +758,7 @@ __global__ void __launch_bounds__(kP1Threads, 2) act_pass1_kernel(const __grid_c
     const int tid = threadIdx.x;
     const int lane = tid & 31;
     const int warp = tid >> 5;
-    const int j = (int)(blockIdx.x % (unsigned)split);       // cluster rank (clusters run along x)
+    const int j = (int)(blockIdx.x % (unsigned)split);       // range of K chunks
     const int64_t m0 = (int64_t)(blockIdx.x / (unsigned)split) * kP1Rows;
     const int nkb = (int)(K / kHad);
     const int kb0 = (int)((int64_t)j * nkb / split);
@@ -804,7 +799,7 @@ __global__ void __launch_bounds__(kP1Threads, 2) act_pass1_kernel(const __grid_c
                 const int kb = kb0 + c;
 #pragma unroll
                 for (int b = 0; b < 4; ++b)
-                    tma_load_2d(xs + 4096 * b, &tmx, kb * kHad + 64 * b, (int32_t)m0, full + 8 * st);
+                    tma_load_2d(xs + kP1BoxBytes * b, &tmx, kb * kHad + 64 * b, (int32_t)m0, full + 8 * st);
                 if (t32)
                     tma_load_2d(xs + kP1XBytes, &tmd, 0, kb * kHad, full + 8 * st);
             }
@@ -825,7 +820,7 @@ __global__ void __launch_bounds__(kP1Threads, 2) act_pass1_kernel(const __grid_c
                 const uint64_t da = sdesc_sw128(xs), db = p1_bdesc(xs + kP1XBytes);
 #pragma unroll
                 for (int ks = 0; ks < 16; ++ks)           // k-step: columns 16ks..16ks+15 of the chunk
-                    mma_bf16(tmem_base, da + (uint64_t)((ks >> 2) * 256 + (ks & 3) * 2),
+                    mma_bf16(tmem_base, da + (uint64_t)((ks >> 2) * (kP1BoxBytes >> 4) + (ks & 3) * 2),
                              db + (uint64_t)(ks * 64), kP1Idesc, (c > 0 || ks > 0) ? 1u : 0u);
                 tc_commit(empty + 8 * st);
             }
@@ -833,6 +828,9 @@ __global__ void __launch_bounds__(kP1Threads, 2) act_pass1_kernel(const __grid_c
         }
         __syncwarp();
     } else if (amax) {                                // consumers: Hadamard absmax
+        // lane (q, r) = (lane / 8, lane % 8) holds quarter q of row 8 warp + r: 64 values of box q
+        const int q = lane >> 3;
+        const int R = 8 * warp + (lane & 7);
         for (int c = 0; c < nch; ++c) {
             const int st = c % kP1Stages;
             const uint32_t ph = (uint32_t)(c / kP1Stages) & 1u;
@@ -841,43 +839,34 @@ __global__ void __launch_bounds__(kP1Threads, 2) act_pass1_kernel(const __grid_c
                 ok = mbar_wait(full + 8 * st, ph, abort_flag, status) ? 1 : 0;
             if (__shfl_sync(0xffffffffu, ok, 0) == 0)
                 break;
-            // lane q of row r takes 16 bytes (8 values, columns 64b + 8q..) of each of the
-            // four boxes: the 8 lanes of a row read 8 different bank slots
-            const int r = 4 * warp + (lane >> 3);
-            const int q = lane & 7;
-            const uint8_t *rowp = p1_smem + st * kP1BufBytes + r * 128 + 16 * (q ^ (r & 7));
-            float v[32];
-#pragma unroll
-            for (int b = 0; b < 4; ++b) {
-                const uint4 a = *reinterpret_cast<const uint4 *>(rowp + 4096 * b);
-                const uint32_t w[4] = {a.x, a.y, a.z, a.w};
-#pragma unroll
-                for (int jj = 0; jj < 4; ++jj) {
-                    v[8 * b + 2 * jj] = __uint_as_float(w[jj] << 16);
-                    v[8 * b + 2 * jj + 1] = __uint_as_float(w[jj] & 0xFFFF0000u);
-                }
-            }
+            uint64_t p[32];
+            load_row64_bf16_sw128_s1(p1_smem + st * kP1BufBytes + q * kP1BoxBytes, R, p);
             __syncwarp();
             if (lane == 0)
-                mbar_arrive(empty + 8 * st);              // the stage's x is in registers
-            fwht256_l32s_unscaled(v, lane);
+                mbar_arrive(empty + 8 * st);              // the stage's rows are in registers
+            fwht256_q4_from_s2(p, lane);                  // odd values negated: the maximum of |v| is unchanged
 #pragma unroll
-            for (int i = 0; i < 32; i += 2)
-                m = fmax3(m, fabsf(v[i]), fabsf(v[i + 1]));
+            for (int i = 0; i < 32; ++i) {
+                float lo, hi;
+                f2_unpack(p[i], lo, hi);
+                m = fmax3(m, fabsf(lo), fabsf(hi));
+            }
         }
     }
     __syncthreads();                                  // every role's loop is done
 
-    // t rows 0..31 of this CTA: tensor-memory lanes 0..31, read by warp 0 once every MMA finished
-    uint32_t tr[32];
-    if (t32 && warp == 0) {
+    // t rows of this CTA: warp w < 4 reads tensor-memory lanes 32w..32w+31 once every MMA
+    // finished and stores its rows of partial tile j (row m0 + 32w + lane, 128 contiguous bytes)
+    __shared__ float wmax[kP1Consumers + 2];
+    if (t32 && warp < 4) {
+        uint32_t tr[32];
         int ok = 1;
         if (lane == 0)
             ok = mbar_wait(done, 0, abort_flag, status) ? 1 : 0;
         ok = __shfl_sync(0xffffffffu, ok, 0);
         tc_fence_after();
         if (ok) {
-            tmem_ld_32cols(tmem_base, tr);
+            tmem_ld_32cols(tmem_base + ((uint32_t)(32 * warp) << 16), tr);
             tmem_wait_ld();
         } else {
 #pragma unroll
@@ -885,59 +874,226 @@ __global__ void __launch_bounds__(kP1Threads, 2) act_pass1_kernel(const __grid_c
                 tr[i] = 0u;
         }
         tc_fence_before();
+        const int64_t row = m0 + 32 * warp + lane;
+        if (row < M) {
+            float4 *o = reinterpret_cast<float4 *>(t32 + ((int64_t)j * M + row) * kRank);
+#pragma unroll
+            for (int i = 0; i < 32; i += 4)
+                o[i / 4] = make_float4(__uint_as_float(tr[i]), __uint_as_float(tr[i + 1]),
+                                       __uint_as_float(tr[i + 2]), __uint_as_float(tr[i + 3]));
+        }
     }
-    __syncthreads();                                  // ring idle and tensor memory read
-    if (t32 && warp == kP1Consumers + 1)
-        tmem_dealloc(tmem_base, 32);
-
     if (amax) {
         m = __fmul_rn(m, 0.0625f);                    // the transform's 1/16, once (exact for a max)
 #pragma unroll
         for (int xx = 16; xx >= 1; xx >>= 1)
             m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, xx));
     }
-    float *tcta = reinterpret_cast<float *>(p1_smem);          // [32][32] this CTA's t tile
-    float *wmax = tcta + kP1Rows * kRank;                       // [10]
-    if (t32 && warp == 0) {
-#pragma unroll
-        for (int i = 0; i < 32; i += 4)                  // once per CTA: bank conflicts do not matter
-            *reinterpret_cast<float4 *>(tcta + lane * kRank + i) =
-                make_float4(__uint_as_float(tr[i]), __uint_as_float(tr[i + 1]), __uint_as_float(tr[i + 2]),
-                            __uint_as_float(tr[i + 3]));
-    }
     if (lane == 0)
         wmax[warp] = m;
-    __syncthreads();
+    __syncthreads();                                  // tensor memory read, maxima stored
+    if (t32 && warp == kP1Consumers + 1)
+        tmem_dealloc(tmem_base, 32);
     if (amax && tid == 0) {
         float b = 0.0f;
         for (int w = 0; w < kP1Consumers; ++w)
             b = fmaxf(b, wmax[w]);
         atomic_max_nonneg(amax, b);
     }
-    if (!t32)
+}
+
+// ---------------------------------------------------------------------------
+// Activation pass 2: NVFP4 block quantisation of H x with the global scale g
+// into codes [M, K/2] and the tiled scales (rows_pad = M rounded up to 128;
+// rows past M are zero and only their scale bytes are written, as 0, which
+// fills the tiled layout's padding).  g comes from *g_static when non-NULL,
+// else RN(A / 2688) from *amax, and is stored to *g_out (when non-NULL) by
+// thread 0 of block 0.  The forward's low-rank operands (LowrankOut) are
+// written first, while the first chunks load.
+// Work unit: 64 rows x one 256-column chunk, four TMA boxes of 64 x 64 bf16
+// (128-byte swizzle) in a 3-deep ring; consumer warp w takes rows 8w..8w+7 in
+// the 4-lane layout, so each lane owns four whole 16-value scale blocks and
+// writes 32 code bytes and 4 scale bytes.  The reciprocals RN(1 / RN(value(sf)
+// g)) depend only on the scale code: a table of the 126 finite non-zero codes
+// is built once per CTA.
+// ---------------------------------------------------------------------------
+constexpr int kAQRows = 64;
+constexpr int kAQBoxBytes = kAQRows * 128;          // 64 rows x 64 bf16
+constexpr int kAQBytes = 4 * kAQBoxBytes;           // 32 KB
+constexpr int kAQStages = 3;
+constexpr int kAQConsumers = 8;
+constexpr int kAQThreads = 32 * (kAQConsumers + 1);
+constexpr int kAQSmem = kAQStages * kAQBytes + 1024 + 256 + 128 * 4;   // ring, alignment, barriers, table
+
+__global__ void __launch_bounds__(kAQThreads, 2) act_quant_kernel(const __grid_constant__ CUtensorMap tmx,
+                                                                  int64_t M, int64_t rows_pad, int64_t K,
+                                                                  const uint32_t *__restrict__ amax,
+                                                                  const float *__restrict__ g_static,
+                                                                  float *__restrict__ g_out,
+                                                                  uint8_t *__restrict__ codes,
+                                                                  uint8_t *__restrict__ sf, LowrankOut lr,
+                                                                  uint32_t *__restrict__ status)
+{
+    extern __shared__ uint8_t aq_raw[];
+    uint8_t *aq_smem =
+        reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(aq_raw) + 1023) & ~uintptr_t(1023));
+    uint64_t *bars = reinterpret_cast<uint64_t *>(aq_smem + kAQStages * kAQBytes);
+    const uint32_t full = smem_u32(bars), empty = smem_u32(bars + kAQStages);
+    volatile uint32_t *abort_flag = reinterpret_cast<uint32_t *>(bars + 2 * kAQStages);
+    float *inv_tab = reinterpret_cast<float *>(aq_smem + kAQStages * kAQBytes + 256);
+    const int tid = threadIdx.x;
+    const int lane = tid & 31;
+    const int warp = tid >> 5;
+    grid_dep_launch();                                // the GEMM may start its set-up
+    if (tid == 0) {
+        for (int st = 0; st < kAQStages; ++st) {
+            mbar_init(full + 8 * st, 1);
+            mbar_init(empty + 8 * st, kAQConsumers);
+        }
+        *abort_flag = 0u;
+        fence_mbar_init();
+    }
+    __syncthreads();
+    const int64_t nkb = K / kHad;
+    const int64_t units = rows_pad / kAQRows * nkb;
+    if (warp == kAQConsumers) {                       // TMA producer: x does not depend on pass 1
+        if (lane == 0) {
+            prefetch_tmap(&tmx);
+            int it = 0;
+            for (int64_t u = blockIdx.x; u < units; u += gridDim.x, ++it) {
+                const int st = it % kAQStages;
+                const uint32_t ph = (uint32_t)(it / kAQStages) & 1u;
+                if (!mbar_wait(empty + 8 * st, ph ^ 1u, abort_flag, status))
+                    break;
+                const int64_t rt = u / nkb, kb = u - rt * nkb;
+                mbar_arrive_expect_tx(full + 8 * st, kAQBytes);
+                const uint32_t xs = smem_u32(aq_smem + st * kAQBytes);
+#pragma unroll
+                for (int b = 0; b < 4; ++b)
+                    tma_load_2d(xs + kAQBoxBytes * b, &tmx, (int32_t)(kb * kHad + 64 * b), (int32_t)(rt * kAQRows),
+                                full + 8 * st);
+            }
+        }
+        __syncwarp();
         return;
-    if (split > 1)
-        cluster_sync();                               // every rank's tile is complete
-    if (j == 0) {
-        const uint32_t tl = (uint32_t)__cvta_generic_to_shared(tcta);
-        for (int e = tid; e < kP1Rows * kRank; e += kP1Threads) {
-            const int64_t row = m0 + (e >> 5);
-            float v = tcta[e];
-            for (int rk = 1; rk < split; ++rk)
-                v = __fadd_rn(v, ld_shared_cluster_f32(mapa_shared(tl + 4 * e, (uint32_t)rk)));
-            if (row < M)
-                t32[row * kRank + (e & 31)] = v;
+    }
+    // ---- consumers: the global scale, the reciprocal table, the low-rank operands
+    grid_dep_wait();                                  // amax and t of pass 1 are final
+    const float g = g_static ? *g_static : __fdiv_rn(__uint_as_float(*amax), 2688.0f);
+    const float sixg = __fmul_rn(6.0f, g);
+    if (g_out && blockIdx.x == 0 && tid == 0)
+        *g_out = g;
+    // inv_tab[c] = RN(1 / RN(value(c) g)) for the finite non-zero codes 1..126;
+    // entry 127 (not a finite code) counts the entries whose /16 would round
+    if (tid < 128)
+        inv_tab[tid] = 0.0f;
+    bar_sync_named(32 * kAQConsumers);
+    if (tid >= 1 && tid <= 126 && g != 0.0f) {
+        const float inv = __frcp_rn(__fmul_rn(ue4m3_value((uint32_t)tid), g));
+        inv_tab[tid] = inv;
+        if (__fmul_rn(__fmul_rn(inv, 0.0625f), 16.0f) != inv)
+            atomicAdd(&inv_tab[127], 1.0f);
+    }
+    if (lr.t_part) {
+        const float beta = lowrank_beta(g, lr.g_w);
+        const int64_t nT = M * 8, total = nT + (lr.udup ? lr.N * 4 : 0);
+        const int64_t stride = (int64_t)gridDim.x * (32 * kAQConsumers);
+        for (int64_t i = (int64_t)blockIdx.x * (32 * kAQConsumers) + tid; i < total; i += stride)
+            lowrank_unit(i, nT, lr.t_part, lr.parts, lr.t_out, beta, lr.tsplit, lr.U, lr.udup);
+    }
+    bar_sync_named(32 * kAQConsumers);                // the table is complete
+    // With A >= 2^-100 (the codec's precondition) and every table entry still exact
+    // after a further /16, RN(RN(v / 16) inv) = RN(v (inv / 16)) for every value that
+    // can give a non-zero code (v / 16 is then a normal number), and both are a zero of
+    // the same sign otherwise: one multiply per value instead of two.
+    const bool fold16 = g >= 0x1p-100f / 2688.0f && inv_tab[127] == 0.0f;
+    const int q = lane >> 3;
+    const int R = 8 * warp + (lane & 7);
+    const uint32_t C = (uint32_t)(K / kSfBlock);
+    const uint32_t nkb32 = (uint32_t)nkb;
+    const uint32_t step_rt = gridDim.x / nkb32, step_kb = gridDim.x % nkb32;
+    uint32_t rt = blockIdx.x / nkb32, kb = blockIdx.x % nkb32;
+    int it = 0;
+    for (int64_t u = blockIdx.x; u < units; u += gridDim.x, ++it) {
+        const int st = it % kAQStages;
+        const uint32_t ph = (uint32_t)(it / kAQStages) & 1u;
+        int ok = 1;
+        if (lane == 0)
+            ok = mbar_wait(full + 8 * st, ph, abort_flag, status) ? 1 : 0;
+        if (__shfl_sync(0xffffffffu, ok, 0) == 0)
+            break;
+        uint64_t p[32];
+        load_row64_bf16_sw128_s1(aq_smem + st * kAQBytes + q * kAQBoxBytes, R, p);
+        __syncwarp();
+        if (lane == 0)
+            mbar_arrive(empty + 8 * st);
+        fwht256_q4_from_s2(p, lane);                  // p[j] = (v[2j], -v[2j+1]), unscaled
+        const uint32_t row = rt * kAQRows + (uint32_t)R;
+        uint32_t word[8];
+        uint32_t sfw = 0;
+#pragma unroll
+        for (int b = 0; b < 4; ++b) {                 // scale block b: values 16b .. 16b+15 of the quarter
+            float a[16];
+#pragma unroll
+            for (int i = 0; i < 8; ++i)
+                f2_unpack(p[8 * b + i], a[2 * i], a[2 * i + 1]);
+            const float m0 = fmax3(fabsf(a[0]), fabsf(a[1]), fabsf(a[2]));
+            const float m1 = fmax3(fabsf(a[3]), fabsf(a[4]), fabsf(a[5]));
+            const float m2 = fmax3(fabsf(a[6]), fabsf(a[7]), fabsf(a[8]));
+            const float m3 = fmax3(fabsf(a[9]), fabsf(a[10]), fabsf(a[11]));
+            const float m4 = fmax3(fabsf(a[12]), fabsf(a[13]), fabsf(a[14]));
+            const float bmax = fmax3(fmax3(m0, m1, m2), fmax3(m3, m4, fabsf(a[15])), 0.0f);
+            uint32_t code = 0, w0 = 0, w1 = 0;
+            if (g != 0.0f) {
+                // max |v / 16| = max |v| / 16 exactly (rounding is monotonic)
+                code = to_ue4m3(__fdiv_rn(__fmul_rn(bmax, 0.0625f), sixg));
+                if (code != 0) {
+                    const float inv = inv_tab[code];
+                    float sv[16];
+                    if (fold16) {
+                        const float i16 = __fmul_rn(inv, 0.0625f);
+                        const uint64_t inv2 = f2_pack(i16, -i16);      // odd values are negated
+#pragma unroll
+                        for (int i = 0; i < 8; ++i)
+                            f2_unpack(f2_mul(p[8 * b + i], inv2), sv[2 * i], sv[2 * i + 1]);
+                    } else {
+                        const uint64_t inv2 = f2_pack(inv, -inv), s16 = f2_pack(0.0625f, 0.0625f);
+#pragma unroll
+                        for (int i = 0; i < 8; ++i)
+                            f2_unpack(f2_mul(f2_mul(p[8 * b + i], s16), inv2), sv[2 * i], sv[2 * i + 1]);
+                    }
+                    w0 = to_e2m1x4(sv[0], sv[1], sv[2], sv[3]) | (to_e2m1x4(sv[4], sv[5], sv[6], sv[7]) << 16);
+                    w1 = to_e2m1x4(sv[8], sv[9], sv[10], sv[11]) |
+                         (to_e2m1x4(sv[12], sv[13], sv[14], sv[15]) << 16);
+                }
+            }
+            word[2 * b] = w0;
+            word[2 * b + 1] = w1;
+            sfw |= code << (8 * b);
+        }
+        if ((int64_t)row < M) {
+            uint4 *o = reinterpret_cast<uint4 *>(codes + (size_t)row * (size_t)(K / 2) + kb * (kHad / 2) + 32 * q);
+            o[0] = make_uint4(word[0], word[1], word[2], word[3]);
+            o[1] = make_uint4(word[4], word[5], word[6], word[7]);
+        }
+        // scale columns 4q .. 4q+3 of the chunk are four adjacent bytes of the tiled layout
+        const uint32_t c4 = kb * (kHad / kSfBlock) / 4 + q;       // (column / 4) of the first of the four
+        const size_t off = ((size_t)(row >> 7) * (C >> 2) + c4) * 512 + (row & 31) * 16 + ((row & 127) >> 5) * 4;
+        *reinterpret_cast<uint32_t *>(sf + off) = sfw;
+        kb += step_kb;
+        rt += step_rt;
+        if (kb >= nkb32) {
+            kb -= nkb32;
+            ++rt;
         }
     }
-    if (split > 1)
-        cluster_sync();                               // ranks > 0 keep their tiles until rank 0 is done
 }
 
 // ---------------------------------------------------------------------------
 // low-rank operands as a kernel of their own (the int4 forward; see
 // lowrank_unit).  g_x NULL means beta = 1.
 // ---------------------------------------------------------------------------
-__global__ void __launch_bounds__(256) lowrank_finish_kernel(const float *__restrict__ t32, int64_t M,
+__global__ void __launch_bounds__(256) lowrank_finish_kernel(const float *__restrict__ t_part, int parts, int64_t M,
                                                              const float *__restrict__ g_x,
                                                              const float *__restrict__ g_w,
                                                              uint16_t *__restrict__ tsplit,
@@ -948,7 +1104,7 @@ __global__ void __launch_bounds__(256) lowrank_finish_kernel(const float *__rest
     const int64_t nT = M * 8;
     for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < nT + N * 4;
          i += (int64_t)gridDim.x * blockDim.x)
-        lowrank_unit(i, nT, t32, beta, tsplit, U, udup);
+        lowrank_unit(i, nT, t_part, parts, nullptr, beta, tsplit, U, udup);
 }
 
 // ---------------------------------------------------------------------------
@@ -1672,9 +1828,40 @@ cudaError_t launch_nvfp4_quant_f32(const float *in, int64_t rows, int64_t K, con
 
 cudaError_t launch_nvfp4_quant_bf16(const uint16_t *in, int64_t rows, int64_t K, const uint32_t *amax,
                                     const float *g_static, float *g_out, uint8_t *codes, uint8_t *sf,
-                                    const LowrankOut &lr, int sms, cudaStream_t s)
+                                    const LowrankOut &lr, uint32_t *status, int sms, cudaStream_t s)
 {
-    return launch_nvfp4_quant(in, rows, K, amax, g_static, g_out, codes, sf, lr, sms, s);
+    constexpr int kMaxDev = 64;
+    static unsigned long long attr_ctx[kMaxDev];
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDev)
+        return cudaErrorInvalidDevice;
+    const unsigned long long ctx = current_context_id();
+    if (ctx == 0 || attr_ctx[dev] != ctx) {
+        cudaError_t e = cudaFuncSetAttribute(act_quant_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kAQSmem);
+        if (e != cudaSuccess)
+            return e;
+        attr_ctx[dev] = ctx;
+    }
+    CUtensorMap tmx;
+    if (!make_tmap(&tmx, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, in, (uint64_t)K, (uint64_t)rows, 64, kAQRows,
+                   CU_TENSOR_MAP_SWIZZLE_128B))
+        return cudaErrorInvalidValue;
+    const int64_t rows_pad = (rows + 127) / 128 * 128;
+    const int64_t units = rows_pad / kAQRows * (K / kHad);
+    const int64_t cap = 2LL * sms;                   // two CTAs per SM
+    // dependent launch: the CTAs start (and stream x) while pass 1 drains
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)(units < cap ? units : cap));
+    cfg.blockDim = dim3(kAQThreads);
+    cfg.dynamicSmemBytes = kAQSmem;
+    cfg.stream = s;
+    cudaLaunchAttribute at[1];
+    at[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    at[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = at;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, act_quant_kernel, tmx, rows, rows_pad, K, amax, g_static, g_out, codes, sf, lr,
+                              status);
 }
 
 cudaError_t launch_int4_build(const float *R, int64_t N, int64_t K, int group, uint8_t *codes, uint16_t *scales,
@@ -1774,8 +1961,9 @@ cudaError_t launch_dequant_int4(const uint8_t *codes, const uint16_t *scales, in
 }
 
 cudaError_t launch_act_pass1(const uint16_t *x, int64_t M, int64_t K, const uint16_t *D, uint32_t *amax,
-                             float *t32, uint32_t *status, int sms, cudaStream_t s)
+                             float *t_part, uint32_t *status, int sms, cudaStream_t s)
 {
+    (void)sms;
     constexpr int kMaxDev = 64;
     static unsigned long long attr_ctx[kMaxDev];
     int dev = 0;
@@ -1793,41 +1981,22 @@ cudaError_t launch_act_pass1(const uint16_t *x, int64_t M, int64_t K, const uint
     if (!make_tmap(&tmx, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, x, (uint64_t)K, (uint64_t)M, 64, kP1Rows,
                    CU_TENSOR_MAP_SWIZZLE_128B))
         return cudaErrorInvalidValue;
-    if (t32 && !make_tmap(&tmd, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, D, (uint64_t)kRank, (uint64_t)K, kRank, kHad,
-                          CU_TENSOR_MAP_SWIZZLE_64B))
+    if (t_part && !make_tmap(&tmd, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, D, (uint64_t)kRank, (uint64_t)K, kRank, kHad,
+                             CU_TENSOR_MAP_SWIZZLE_64B))
         return cudaErrorInvalidValue;
     const int64_t tiles = (M + kP1Rows - 1) / kP1Rows;
-    const int nkb = (int)(K / kHad);
-    int64_t split = (2LL * sms) / tiles;              // two CTAs per SM
-    split = split < 1 ? 1 : split;
-    split = split > kP1MaxSplit ? kP1MaxSplit : split;
-    split = split > nkb ? nkb : split;
-    const unsigned grid = (unsigned)(tiles * split);
-    if (split == 1) {
-        act_pass1_kernel<<<grid, kP1Threads, kP1Smem, s>>>(tmx, tmd, M, K, amax, t32, 1, status);
-        return cudaGetLastError();
-    }
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(grid);
-    cfg.blockDim = dim3(kP1Threads);
-    cfg.dynamicSmemBytes = kP1Smem;
-    cfg.stream = s;
-    cudaLaunchAttribute at[1];
-    at[0].id = cudaLaunchAttributeClusterDimension;
-    at[0].val.clusterDim.x = (unsigned)split;
-    at[0].val.clusterDim.y = 1;
-    at[0].val.clusterDim.z = 1;
-    cfg.attrs = at;
-    cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, act_pass1_kernel, tmx, tmd, M, K, amax, t32, (int)split, status);
+    const int split = act_t_parts(M, K);
+    act_pass1_kernel<<<(unsigned)(tiles * split), kP1Threads, kP1Smem, s>>>(tmx, tmd, M, K, amax, t_part, split,
+                                                                            status);
+    return cudaGetLastError();
 }
 
-cudaError_t launch_lowrank_finish(const float *t32, int64_t M, const float *g_x, const float *g_w,
+cudaError_t launch_lowrank_finish(const float *t_part, int parts, int64_t M, const float *g_x, const float *g_w,
                                   uint16_t *tsplit, const uint16_t *U, int64_t N, uint16_t *udup, int sms,
                                   cudaStream_t s)
 {
-    lowrank_finish_kernel<<<grid_for(M * 8 + N * 4, 256, sms, 4), 256, 0, s>>>(t32, M, g_x, g_w, tsplit, U, N,
-                                                                                  udup);
+    lowrank_finish_kernel<<<grid_for(M * 8 + N * 4, 256, sms, 4), 256, 0, s>>>(t_part, parts, M, g_x, g_w, tsplit,
+                                                                                  U, N, udup);
     return cudaGetLastError();
 }
 

@@ -237,7 +237,10 @@ SQ_API sq_status sq_build_nvfp4(const float *R, int64_t N, int64_t K,
  * (device): codes [M, K/2], sf_tiled (sq_sf_bytes(M, K) bytes, padding rows
  * 0), g_x (written unless static).  If lora_down (bf16 [K, 32]) and t are
  * both non-NULL, also t[m, r] = sum_k x[m, k] lora_down[k, r] as fp32 [M, 32]
- * (the low-rank input; fp32 accumulation, order unspecified).  flags:
+ * (the low-rank input; fp32 accumulation, order unspecified but fixed for a
+ * given M and K, so t is the same on every run).  ws: sq_workspace_bytes(
+ * SQ_OP_ACT_QUANT_NVFP4, M, 0, K) bytes (the status word, the absmax and,
+ * when K is split over several CTAs, their partial t tiles).  flags:
  * SQ_ACT_STATIC_SCALE, SQ_CHECK_FINITE (the status word is the first 4 bytes
  * of ws).
  */
@@ -293,7 +296,7 @@ SQ_API sq_status sq_linear_fwd(const sq_weight *w, const uint16_t *x, int64_t M,
  * Limit: sq_workspace_bytes(SQ_OP_LINEAR_FWD_NVFP4 or _INT4, M, N, K) must
  * be at most 33554432 (32 MiB); larger shapes return SQ_ERR_WORKSPACE before
  * any work, with the sizes in sq_last_error_detail().  (NVFP4 at N = 16384,
- * K = 6144 fits M up to 8462 rows; the int4 forward, which keeps a bf16 copy
+ * K = 6144 fits M up to 8191 rows; the int4 forward, which keeps a bf16 copy
  * of W in the workspace, fits N x K up to about 16 M values, e.g. M = 1536
  * at N = K = 3072.)
  *

@@ -126,16 +126,16 @@ def test_noalloc_variants_match_workspace_forward(sq, variant):
 
 
 def test_noalloc_rejects_shape_beyond_scratch(sq):
-    # NVFP4 at N = 16384, K = 6144 fits M = 8462 rows, not 8463: refused before
+    # NVFP4 at N = 16384, K = 6144 fits M = 8191 rows, not 8192: refused before
     # any device work (the weight pointers are never touched).
     fake = 1 << 20
     w = sq.sq_weight(sq.SQ_FMT_NVFP4, 16384, 6144, fake, fake, fake, fake, fake)
-    assert sq.sq_workspace_bytes(sq.SQ_OP_LINEAR_FWD_NVFP4, 8463, 16384, 6144) > SCRATCH_BYTES
-    assert sq.sq_workspace_bytes(sq.SQ_OP_LINEAR_FWD_NVFP4, 8462, 16384, 6144) <= SCRATCH_BYTES
+    assert sq.sq_workspace_bytes(sq.SQ_OP_LINEAR_FWD_NVFP4, 8192, 16384, 6144) > SCRATCH_BYTES
+    assert sq.sq_workspace_bytes(sq.SQ_OP_LINEAR_FWD_NVFP4, 8191, 16384, 6144) <= SCRATCH_BYTES
     import ctypes
     out = ctypes.c_void_p(123)
-    st = sq.lib().sq_linear_fwd_noalloc(ctypes.byref(w), fake, 8463, fake, None, 0, ctypes.byref(out), None)
+    st = sq.lib().sq_linear_fwd_noalloc(ctypes.byref(w), fake, 8192, fake, None, 0, ctypes.byref(out), None)
     assert sq.status_str(st) == "workspace too small"
     assert out.value is None
     detail = sq.lib().sq_last_error_detail().decode()
-    assert "33554432" in detail and "M=8463" in detail
+    assert "33554432" in detail and "M=8192" in detail
