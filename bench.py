@@ -53,6 +53,13 @@ FP4_PER_BF16 = 4.0        # nominal dense FP4 / BF16 tensor ratio (9 / 2.25 PFLO
 FLUSH_BYTES = 256 << 20   # > 126 MB L2
 # FP32 FMA issue roofline of the SVD init's products: 148 SMs x 128 FMA lanes x 2 flop x 1.965 GHz
 FP32_ALU_TFLOPS = 148 * 128 * 2 * 1.965e9 / 1e12
+ALU_GOPS = 148 * 128 * 1.965e9 / 1e9    # FP32 lane-operations per second at the maximum SM clock
+# algorithmic FP32 lane-operations per element of the [N, K] operand for the ALU-bound kernels:
+# the builders' 26-trial sweep (multiply, round, clamp, error, square, sum: 8 per trial) plus the
+# Hadamard transform (8), the reconstruct's rank-r fmaf chain plus the transform
+ALU_OPS = {"build_int4": 26 * 8 + 8, "build_int4_g64": 26 * 8 + 8, "build_int8": 26 * 8 + 8,
+           "reconstruct_nvfp4": 32 + 8, "reconstruct_int4": 32 + 8, "reconstruct_int4_g64": 32 + 8,
+           "reconstruct_int8": 16 + 8}
 SVD_ITERS = 8
 
 
@@ -66,6 +73,7 @@ def parse():
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--no-e2e", action="store_true")
     p.add_argument("--no-clocks", action="store_true")
+    p.add_argument("--no-extra", action="store_true", help="skip the other configurations and the builder stack")
     return p.parse_args()
 
 
@@ -100,6 +108,10 @@ def op_work(M, N, K):
         "reconstruct_int8": ("GB/s", NK * (1 + 2) + N * 4),
         "bwd_dx_nvfp4": ("TFLOP/s", 2.0 * M * N * K),
         "svd_init": ("TFLOP/s", (4.0 * SVD_ITERS + 2.0) * NK * 32),   # fp32 FMA work (2 products/round + residual)
+        "act_quant_nvfp4": ("GB/s", MK * (2 + 0.5 + 1 / 16) + M * 32 * 4),
+        "act_pass1": ("GB/s", MK * 2 + M * 32 * 4),            # x read once (absmax and t)
+        "act_pass2": ("GB/s", MK * (2 + 0.5 + 1 / 16)),        # x again, codes and scales
+        "reconstruct_nvfp4_resid": ("GB/s", NK * (0.5 + 1 / 16 + 2)),
         "gemm_nvfp4": ("TFLOP/s", 2.0 * M * N * K),
         "gemm_int4": ("TFLOP/s", 2.0 * M * N * K),
         "gemm_bwd_dx": ("TFLOP/s", 2.0 * M * N * K),
@@ -108,6 +120,7 @@ def op_work(M, N, K):
 
 LAUNCHES_PER_STEP = {   # our kernels per op (memsets excluded)
     "build_int4": 1, "build_nvfp4": 2, "fwd_nvfp4": 3, "fwd_nvfp4_bf16out": 3, "fwd_int4": 5,
+    "act_quant_nvfp4": 2, "reconstruct_nvfp4_resid": 1,
     "reconstruct_nvfp4": 1, "reconstruct_int4": 1,
     "build_int4_g64": 1, "fwd_int4_g64": 5, "reconstruct_int4_g64": 1,
     "build_int8": 1, "fwd_int8": 7, "reconstruct_int8": 1,
@@ -314,7 +327,7 @@ def run_reference(args, cfg, d):
         t, cores = cpu_sample(d, M_s, N_s)
         times.append(t)
     wall = time.perf_counter() - t_start
-    fwd = statistics.mean(t["fwd_nvfp4"] for t in times)
+    fwd = statistics.median(t["fwd_nvfp4"] for t in times)
     value = flops / fwd / 1e12
     line = {
         "impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": args.gpus,
@@ -325,7 +338,7 @@ def run_reference(args, cfg, d):
         "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
                          "sample": cpu_sample_desc(cfg, M_s, N_s)},
         "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
-        "ops_s": {k: statistics.mean(t[k] for t in times) for k in times[0]},
+        "ops_s": {k: statistics.median(t[k] for t in times) for k in times[0]},
     }
     print(json.dumps(line), flush=True)
 
@@ -349,7 +362,8 @@ def workload_config(cfg, args):
         "name": cfg.name, "M": cfg.M, "N": cfg.N, "K": cfg.K, "rank": 32,
         "codecs": ["nvfp4 (e2m1, ue4m3 block-16, fp32 global)", "int4 group-32 MSE-swept",
                    "int4 group-64 MSE-swept", "int8 per-row MSE-swept, rank-16 low-rank branch"],
-        "l2": "flushed (256 MB write) before every op, outside its events",
+        "l2": "flushed before every op, outside its events: a 256 MB write, then a read of another "
+              "256 MB buffer (none of the op's inputs in L2, and no dirty lines left to write back)",
         "parallelism": f"replicas x{args.gpus}",
     }
 
@@ -357,6 +371,62 @@ def workload_config(cfg, args):
 # ---------------------------------------------------------------------------
 # the CUDA path
 # ---------------------------------------------------------------------------
+
+class L2Flush:
+    """Before every timed op: write a buffer larger than L2, then read another one, so the op
+    finds none of its inputs in L2 and no dirty lines of the flush still to be written back."""
+
+    def __init__(self, dev):
+        import torch
+        self.w = torch.empty(FLUSH_BYTES // 4, dtype=torch.int32, device=dev)
+        self.r = torch.zeros(FLUSH_BYTES // 4, dtype=torch.int32, device=dev)
+        self.out = torch.empty((), dtype=torch.int32, device=dev)
+
+    def __call__(self):
+        import torch
+        self.w.fill_(1)
+        torch.amax(self.r, dim=0, out=self.out)
+
+
+def time_ops(ops, flush, steps, warmup, stage_of=None):
+    """Median milliseconds of each (name, fn) over `steps` runs after `warmup`, each run after an
+    L2 flush, timed with CUDA events on the current stream.  stage_of[name] = [(key, stage)]
+    also times those library launches with the stage events, on separate runs."""
+    import torch
+    import bit_quantized_frozen_b200 as sq
+    stage_of = stage_of or {}
+    for _ in range(warmup):
+        for _, fn in ops:
+            flush()
+            fn()
+    times = {}
+    for name, fn in ops:
+        keys = [k for k, _ in stage_of.get(name, [])]
+        rec = {name: []} | {k: [] for k in keys}
+        for it in range(steps * (2 if keys else 1)):
+            inst = keys and it % 2 == 1
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            sev = {}
+            if inst:
+                for k, st in stage_of[name]:
+                    sev[k] = (torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+                    sq.sq_set_stage_events(st, *sev[k])
+            flush()
+            a.record()
+            fn()
+            b.record()
+            if inst:
+                for k, st in stage_of[name]:
+                    sq.sq_set_stage_events(st, None, None)
+            torch.cuda.synchronize()
+            if inst:
+                for k in keys:
+                    rec[k].append(sev[k][0].elapsed_time(sev[k][1]))
+            else:
+                rec[name].append(a.elapsed_time(b))
+        for k, v in rec.items():
+            times[k] = statistics.median(v)
+    return times
 
 def run_sq(args, cfg, d, rank, world, local_rank):
     import torch
@@ -403,7 +473,11 @@ def run_sq(args, cfg, d, rank, world, local_rank):
     down_s = torch.empty((K, 32), dtype=torch.bfloat16, device=dev)
     R_s = torch.empty_like(R)
     ws_svd = sq.workspace(sq.SQ_OP_SVD_INIT, 0, N, K, dev)
-    flush = torch.empty(FLUSH_BYTES // 4, dtype=torch.int32, device=dev)
+    a_codes = torch.empty((M, K // 2), dtype=torch.uint8, device=dev)
+    a_sf = torch.empty(sq.sq_sf_bytes(M, K), dtype=torch.uint8, device=dev)
+    a_t = torch.empty((M, 32), dtype=torch.float32, device=dev)
+    ws_aq = sq.workspace(sq.SQ_OP_ACT_QUANT_NVFP4, M, 0, K, dev)
+    flush = L2Flush(dev)
 
     ops = [
         ("build_int4", lambda: sq.sq_build_int4(R, i4.codes, i4.scales, i4.frac_idx)),
@@ -421,29 +495,37 @@ def run_sq(args, cfg, d, rank, world, local_rank):
         ("reconstruct_int8", lambda: sq.sq_reconstruct_bf16(i8, W)),
         ("bwd_dx_nvfp4", lambda: sq.sq_linear_bwd_dx(nv, dy, dx, ws_dx)),
         ("svd_init", lambda: sq.sq_svd_init(Wsvd, omega, SVD_ITERS, up_s, down_s, R_s, ws_svd)),
+        ("act_quant_nvfp4", lambda: sq.sq_act_quant_nvfp4(x, a_codes, a_sf, g_x, lora_down=D, t=a_t, ws=ws_aq)),
+        ("reconstruct_nvfp4_resid", lambda: sq.sq_reconstruct_bf16(nv, W, sq.SQ_RECON_RESIDUAL_ONLY)),
     ]
     names = [n for n, _ in ops]
-    gemm_of = {"fwd_nvfp4": "gemm_nvfp4", "fwd_int4": "gemm_int4", "bwd_dx_nvfp4": "gemm_bwd_dx"}
+    # launches timed on their own by the library's stage events (even steps; the op itself on odd
+    # steps, because an event between two launches stops the second from overlapping the first)
+    stages_of = {"fwd_nvfp4": [("gemm_nvfp4", sq.SQ_STAGE_GEMM)], "fwd_int4": [("gemm_int4", sq.SQ_STAGE_GEMM)],
+                 "bwd_dx_nvfp4": [("gemm_bwd_dx", sq.SQ_STAGE_GEMM)],
+                 "act_quant_nvfp4": [("act_pass1", sq.SQ_STAGE_ACT_PASS1), ("act_pass2", sq.SQ_STAGE_ACT_QUANT)]}
+    gemm_of = {op: [k for k, _ in st] for op, st in stages_of.items()}
 
     # The GEMM kernel's own events are recorded on even steps only: an event between
     # the activation quantisation and the GEMM launch would stop the GEMM's set-up
     # from overlapping the quantisation, so the forward is timed on the odd steps.
     def run_step(evs, instrument_gemm=False):
         for name, fn in ops:
-            flush.fill_(1)
+            flush()
             if evs is None:
                 fn()
                 continue
             a, b = evs[name]
-            gemm = instrument_gemm and name in gemm_of
-            if gemm:
-                ga, gb = evs[gemm_of[name]]
-                sq.sq_set_gemm_events(ga, gb)
+            inst = instrument_gemm and name in stages_of
+            if inst:
+                for key, stage in stages_of[name]:
+                    sq.sq_set_stage_events(stage, *evs[key])
             a.record()
             fn()
             b.record()
-            if gemm:
-                sq.sq_set_gemm_events(None, None)
+            if inst:
+                for key, stage in stages_of[name]:
+                    sq.sq_set_stage_events(stage, None, None)
 
     for _ in range(args.warmup):
         run_step(None)
@@ -452,7 +534,8 @@ def run_sq(args, cfg, d, rank, world, local_rank):
     sq.sq_check_device_status(ws_i4)
     sq.sq_check_device_status(ws_i8)
 
-    keys = names + list(gemm_of.values())
+    stage_keys = [k for v in gemm_of.values() for k in v]
+    keys = names + stage_keys
     evs = [{k: (torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for k in keys}
            for _ in range(args.steps)]
     outer = (torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
@@ -476,10 +559,10 @@ def run_sq(args, cfg, d, rank, world, local_rank):
     sq.sq_check_device_status(ws_i4)
 
     even = evs[0::2]
-    odd = evs[1::2] or evs                     # a single step: the forward carries the GEMM events
-    per_op = {k: statistics.mean(e[k][0].elapsed_time(e[k][1])
-                                 for e in (even if k in gemm_of.values() else odd if k in gemm_of else evs))
-              for k in keys}   # ms
+    odd = evs[1::2] or evs                     # a single step: the op carries the stage events
+    per_op = {k: statistics.median(e[k][0].elapsed_time(e[k][1])
+                                   for e in (even if k in stage_keys else odd if k in gemm_of else evs))
+              for k in keys}   # ms, median over the steps
     outer_ms = outer[0].elapsed_time(outer[1]) / max(args.steps, 1)
     vals = max_over_ranks([per_op[k] for k in keys] + [outer_ms], world, dev)
     per_op = dict(zip(keys, vals[:-1]))
@@ -533,10 +616,9 @@ def run_sq(args, cfg, d, rank, world, local_rank):
     return per_op, outer_ms, clocks, e2e
 
 
-def summarise(args, cfg, per_op, outer_ms, clocks, e2e, world, cpu):
-    peaks, peak_src = load_peaks()
+def rate_entries(per_op, M, N, K, peaks, peak_src):
+    """{op: {ms, rate, frac of its roofline, alu (the ALU-bound kernels)}} for median times."""
     fp4_peak = peaks["bf16_tflops"] * FP4_PER_BF16
-    M, N, K = cfg.M, cfg.N, cfg.K
     work = op_work(M, N, K)
     ops = {}
     for k, ms in per_op.items():
@@ -552,6 +634,18 @@ def summarise(args, cfg, per_op, outer_ms, clocks, e2e, world, cpu):
             frac, peak = rate / peak_v, "fp4 tensor" if fp4 else "bf16 tensor"
         src = "148 SMs x 128 lanes x 2 flop x 1.965 GHz" if k == "svd_init" else peak_src
         ops[k] = {"ms": ms, unit: rate, "frac": frac, "of": f"{peak} ({src})"}
+        if k in ALU_OPS:
+            gops = ALU_OPS[k] * N * K / (ms * 1e-3) / 1e9
+            ops[k]["alu"] = {"Gop/s": gops, "frac": gops / ALU_GOPS, "ops_per_element": ALU_OPS[k],
+                             "of": "fp32 lane-op issue, 148 SMs x 128 lanes x 1.965 GHz (unit counts, max clock)"}
+    return ops
+
+
+def summarise(args, cfg, per_op, outer_ms, clocks, e2e, world, cpu, extra=None):
+    peaks, peak_src = load_peaks()
+    fp4_peak = peaks["bf16_tflops"] * FP4_PER_BF16
+    M, N, K = cfg.M, cfg.N, cfg.K
+    ops = rate_entries(per_op, M, N, K, peaks, peak_src)
     fwd_tflops = 2.0 * M * N * K / (per_op["fwd_nvfp4"] * 1e-3) / 1e12
     gemm_tflops = 2.0 * M * N * K / (per_op["gemm_nvfp4"] * 1e-3) / 1e12
     traffic, traffic_src = profiled_traffic(cfg.name)
@@ -592,7 +686,113 @@ def summarise(args, cfg, per_op, outer_ms, clocks, e2e, world, cpu):
         "e2e": e2e,
         "cpu_baseline": cpu,
     }
+    if extra:
+        for name, times in extra.get("per_config", {}).items():
+            c = si.CONFIGS[name]
+            line.setdefault("per_config", {})[name] = {
+                "M": c.M, "N": c.N, "K": c.K, "ops": rate_entries(times, c.M, c.N, c.K, peaks, peak_src)}
+        if "stack" in extra:
+            line["builder_stack"] = extra["stack"]
     return line
+
+
+PER_CONFIG = ["tiny_64x256x512", "proj_1536x3072x3072", "qkv_1536x9216x3072", "large_4480x6144x6144",
+              "down_4480x6144x16384"]
+
+
+def run_configs(headline, dev):
+    """The forward, activation quantiser, builders and reconstructs on every other configuration,
+    5 timed runs each (median) after 2 warm-up runs, L2 flushed before each."""
+    import torch
+    import bit_quantized_frozen_b200 as sq
+    flush = L2Flush(dev)
+    out = {}
+    for name in PER_CONFIG:
+        if name == headline:
+            continue
+        cfg = si.CONFIGS[name]
+        d = si.make_config(name)
+        M, N, K = cfg.M, cfg.N, cfg.K
+        to_bf16 = lambda a: torch.from_numpy(a.view(np.int16)).to(dev).view(torch.bfloat16)
+        R, x, U, D = torch.from_numpy(d["R"]).to(dev), to_bf16(d["x"]), to_bf16(d["U"]), to_bf16(d["D"])
+        nv = sq.Weight(sq.SQ_FMT_NVFP4, N, K, torch.empty((N, K // 2), dtype=torch.uint8, device=dev),
+                       torch.empty(sq.sq_sf_bytes(N, K), dtype=torch.uint8, device=dev),
+                       torch.empty(1, dtype=torch.float32, device=dev), U, D)
+        i4 = sq.Weight(sq.SQ_FMT_INT4_G32, N, K, torch.empty((N, K // 2), dtype=torch.uint8, device=dev),
+                       torch.empty((N, K // 32), dtype=torch.float16, device=dev), None, U, D,
+                       torch.empty((N, K // 32), dtype=torch.uint8, device=dev))
+        ws_b = sq.workspace(sq.SQ_OP_BUILD_NVFP4, 0, N, K, dev)
+        ws_nv = sq.workspace(sq.SQ_OP_LINEAR_FWD_NVFP4, M, N, K, dev)
+        ws_i4 = sq.workspace(sq.SQ_OP_LINEAR_FWD_INT4, M, N, K, dev)
+        ws_aq = sq.workspace(sq.SQ_OP_ACT_QUANT_NVFP4, M, 0, K, dev)
+        y = torch.empty((M, N), dtype=torch.float32, device=dev)
+        W = torch.empty((N, K), dtype=torch.bfloat16, device=dev)
+        g_x = torch.empty(1, dtype=torch.float32, device=dev)
+        a_codes = torch.empty((M, K // 2), dtype=torch.uint8, device=dev)
+        a_sf = torch.empty(sq.sq_sf_bytes(M, K), dtype=torch.uint8, device=dev)
+        a_t = torch.empty((M, 32), dtype=torch.float32, device=dev)
+        ops = [
+            ("build_nvfp4", lambda: sq.sq_build_nvfp4(R, nv.codes, nv.scales, nv.g_w, ws_b)),
+            ("build_int4", lambda: sq.sq_build_int4(R, i4.codes, i4.scales, i4.frac_idx)),
+            ("act_quant_nvfp4", lambda: sq.sq_act_quant_nvfp4(x, a_codes, a_sf, g_x, lora_down=D, t=a_t, ws=ws_aq)),
+            ("fwd_nvfp4", lambda: sq.sq_linear_fwd(nv, x, y, g_x=g_x, ws=ws_nv)),
+            ("fwd_int4", lambda: sq.sq_linear_fwd(i4, x, y, ws=ws_i4)),
+            ("reconstruct_nvfp4", lambda: sq.sq_reconstruct_bf16(nv, W)),
+            ("reconstruct_nvfp4_resid", lambda: sq.sq_reconstruct_bf16(nv, W, sq.SQ_RECON_RESIDUAL_ONLY)),
+        ]
+        stage_of = {"fwd_nvfp4": [("gemm_nvfp4", sq.SQ_STAGE_GEMM)],
+                    "act_quant_nvfp4": [("act_pass1", sq.SQ_STAGE_ACT_PASS1), ("act_pass2", sq.SQ_STAGE_ACT_QUANT)]}
+        out[name] = time_ops(ops, flush, steps=5, warmup=2, stage_of=stage_of)
+        sq.sq_check_device_status(ws_nv)
+        del R, x, U, D, nv, i4, ws_b, ws_nv, ws_i4, ws_aq, y, W, a_codes, a_sf, a_t, ops
+        torch.cuda.empty_cache()
+    return out
+
+
+def run_stack(dev, count=si.STACK_COUNT):
+    """The down-projection shape's builder stack: `count` residual weights [6144, 16384] fp32 drawn
+    one after another into one device buffer (untimed), each built by the three builders (timed,
+    L2 flushed before each build)."""
+    import torch
+    import bit_quantized_frozen_b200 as sq
+    N, K = 6144, 16384
+    flush = L2Flush(dev)
+    Rb = torch.empty((N, K), dtype=torch.float32, device=dev)
+    c4 = torch.empty((N, K // 2), dtype=torch.uint8, device=dev)
+    s4 = torch.empty((N, K // 32), dtype=torch.float16, device=dev)
+    f4 = torch.empty((N, K // 32), dtype=torch.uint8, device=dev)
+    cn = torch.empty((N, K // 2), dtype=torch.uint8, device=dev)
+    sn = torch.empty(sq.sq_sf_bytes(N, K), dtype=torch.uint8, device=dev)
+    gn = torch.empty(1, dtype=torch.float32, device=dev)
+    ws_b = sq.workspace(sq.SQ_OP_BUILD_NVFP4, 0, N, K, dev)
+    c8 = torch.empty((N, K), dtype=torch.int8, device=dev)
+    s8 = torch.empty(N, dtype=torch.float32, device=dev)
+    f8 = torch.empty(N, dtype=torch.uint8, device=dev)
+    builders = [("build_int4", lambda: sq.sq_build_int4(Rb, c4, s4, f4), 4 + 0.5 + 2 / 32 + 1 / 32),
+                ("build_nvfp4", lambda: sq.sq_build_nvfp4(Rb, cn, sn, gn, ws_b), 4 + 0.5 + 1 / 16),
+                ("build_int8", lambda: sq.sq_build_int8(Rb, c8, s8, f8), 4 + 1)]
+    ev = {b: [] for b, _, _ in builders}
+    for i in range(count):
+        si.make_stack_residual_device(i, Rb, N, K)
+        for b, fn, _ in builders:
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            flush()
+            e0.record()
+            fn()
+            e1.record()
+            ev[b].append((e0, e1))
+    torch.cuda.synchronize()
+    res = {"weights": count, "shape": [N, K],
+           "inputs": "seeded Student-t(4) residuals (std 1/sqrt(K)), drawn on the device per weight into "
+                     "one buffer, untimed; L2 flushed before each build"}
+    for b, _, bpe in builders:
+        ms = [a.elapsed_time(e) for a, e in ev[b]]
+        tot = sum(ms)
+        res[b] = {"total_ms": tot, "ms_per_weight_median": statistics.median(ms),
+                  "GB/s": count * N * K * bpe / (tot * 1e-3) / 1e9}
+    del Rb, c4, s4, f4, cn, sn, gn, ws_b, c8, s8, f8
+    torch.cuda.empty_cache()
+    return res
 
 
 def main():
@@ -614,6 +814,10 @@ def main():
                                              device_id=torch.device("cuda", local_rank))
     d = si.make_config(cfg.name)
     per_op, outer_ms, clocks, e2e = run_sq(args, cfg, d, rank, world, local_rank)
+    extra = None
+    if rank == 0 and world == 1 and not args.no_extra:
+        dev = torch.device("cuda", local_rank)
+        extra = {"per_config": run_configs(cfg.name, dev), "stack": run_stack(dev)}
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         M_s, N_s = CPU_SAMPLE
@@ -621,7 +825,7 @@ def main():
         cpu = {"value": 2.0 * M_s * N_s * cfg.K / t["fwd_nvfp4"] / 1e12, "unit": "TFLOP/s", "cores": cores,
                "kind": "oracle", "sample": cpu_sample_desc(cfg, M_s, N_s), "ops_s": t}
     if rank == 0:
-        print(json.dumps(summarise(args, cfg, per_op, outer_ms, clocks, e2e, world, cpu)), flush=True)
+        print(json.dumps(summarise(args, cfg, per_op, outer_ms, clocks, e2e, world, cpu, extra)), flush=True)
     if world > 1:
         torch.distributed.barrier()
         torch.distributed.destroy_process_group()

@@ -39,6 +39,9 @@ SQ_ACT_STATIC_SCALE = 0x1
 SQ_RECON_RESIDUAL_ONLY = 0x2
 SQ_RECON_TRANSPOSED = 0x4
 SQ_OUT_BF16 = 0x8
+SQ_STAGE_GEMM = 0                     # sq_set_stage_events
+SQ_STAGE_ACT_PASS1 = 1
+SQ_STAGE_ACT_QUANT = 2
 SQ_CHECK_FINITE = 0x10
 SQ_OP_LINEAR_BWD_DX = 9
 SQ_OP_SVD_INIT = 10
@@ -48,7 +51,7 @@ EXPORTED = [
     "sq_status_str", "sq_abi_version", "sq_last_error_detail", "sq_sf_bytes", "sq_workspace_bytes",
     "sq_build_int4", "sq_build_int8", "sq_build_nvfp4", "sq_act_quant_nvfp4", "sq_linear_fwd",
     "sq_reconstruct_bf16",
-    "sq_check_device_status", "sq_set_gemm_events", "sq_linear_fwd_noalloc", "sq_linear_bwd_dx",
+    "sq_check_device_status", "sq_set_gemm_events", "sq_set_stage_events", "sq_linear_fwd_noalloc", "sq_linear_bwd_dx",
     "sq_selftest_wait_timeout", "sq_svd_init",
 ]
 
@@ -99,6 +102,7 @@ _SIGS = {
     "sq_check_device_status": ([_P, _P], ctypes.c_int),
     "sq_selftest_wait_timeout": ([_P, ctypes.c_uint32, _P], ctypes.c_int),
     "sq_set_gemm_events": ([_P, _P], ctypes.c_int),
+    "sq_set_stage_events": ([ctypes.c_int32, _P, _P], ctypes.c_int),
 }
 _lib = None
 
@@ -316,16 +320,24 @@ def sq_check_device_status(ws, stream=None):
     _check("sq_check_device_status", lib().sq_check_device_status(_ptr(ws), _stream(stream)))
 
 
+def _event_handle(ev):
+    if ev is None:
+        return None
+    if ev.cuda_event == 0:              # torch creates the CUDA event lazily
+        ev.record()
+    return ev.cuda_event
+
+
 def sq_set_gemm_events(start_event=None, stop_event=None):
     """Record these torch.cuda.Event objects around the GEMM launch of later
     sq_linear_fwd calls on this thread (None, None turns it off)."""
-    def handle(ev):
-        if ev is None:
-            return None
-        if ev.cuda_event == 0:          # torch creates the CUDA event lazily
-            ev.record()
-        return ev.cuda_event
-    _check("sq_set_gemm_events", lib().sq_set_gemm_events(handle(start_event), handle(stop_event)))
+    _check("sq_set_gemm_events", lib().sq_set_gemm_events(_event_handle(start_event), _event_handle(stop_event)))
+
+
+def sq_set_stage_events(stage: int, start_event=None, stop_event=None):
+    """The same for SQ_STAGE_GEMM, SQ_STAGE_ACT_PASS1 or SQ_STAGE_ACT_QUANT."""
+    _check("sq_set_stage_events",
+           lib().sq_set_stage_events(int(stage), _event_handle(start_event), _event_handle(stop_event)))
 
 
 # ---- a built weight and allocating helpers (torch provides the memory) --------

@@ -68,8 +68,15 @@ int g_sms[kMaxDevices];          // 0 = not yet queried
 int g_cc_ok[kMaxDevices];        // 0 unknown, 1 sm_100, -1 other
 
 thread_local char g_detail[256] = "";
-thread_local cudaEvent_t g_gemm_ev0 = nullptr;   // sq_set_gemm_events
-thread_local cudaEvent_t g_gemm_ev1 = nullptr;
+// sq_set_stage_events: [stage][0 = before the launch, 1 = after]
+thread_local cudaEvent_t g_stage_ev[SQ_STAGE_COUNT][2] = {};
+
+// record stage event `which` (0 before, 1 after) on stream s, when the caller set one
+cudaError_t stage_event(int stage, int which, cudaStream_t s)
+{
+    cudaEvent_t e = g_stage_ev[stage][which];
+    return e ? cudaEventRecord(e, s) : cudaSuccess;
+}
 
 void set_detail(const char *what, cudaError_t e)
 {
@@ -401,19 +408,24 @@ sq_status sq_act_quant_nvfp4(const uint16_t *x, int64_t M, int64_t K, uint8_t *c
     SQ_CUDA(cudaMemsetAsync(ws, 0, 8, s), "memset");          // status word + absmax
     if (flags & SQ_CHECK_FINITE)
         SQ_CUDA(sq::launch_check_finite_bf16(x, M * K, reinterpret_cast<uint32_t *>(ws), sms, s), "finite check");
-    if (!stat || with_t)
+    if (!stat || with_t) {
+        SQ_CUDA(stage_event(SQ_STAGE_ACT_PASS1, 0, s), "event record");
         SQ_CUDA(sq::launch_act_pass1(x, M, K, lora_down, stat ? nullptr : amax, t_part,
                                      reinterpret_cast<uint32_t *>(ws), sms, s),
                 "activation pass 1");
+        SQ_CUDA(stage_event(SQ_STAGE_ACT_PASS1, 1, s), "event record");
+    }
     sq::LowrankOut lr;                                          // t = the sum of the partial tiles
     if (with_t && parts > 1) {
         lr.t_part = t_part;
         lr.parts = parts;
         lr.t_out = t;
     }
+    SQ_CUDA(stage_event(SQ_STAGE_ACT_QUANT, 0, s), "event record");
     SQ_CUDA(sq::launch_nvfp4_quant_bf16(x, M, K, amax, stat ? g_x : nullptr, stat ? nullptr : g_x, codes, sf_tiled,
                                         lr, reinterpret_cast<uint32_t *>(ws), sms, s),
             "nvfp4 quant");
+    SQ_CUDA(stage_event(SQ_STAGE_ACT_QUANT, 1, s), "event record");
     return SQ_OK;
 }
 
@@ -467,9 +479,12 @@ sq_status sq_linear_fwd(const sq_weight *w, const uint16_t *x, int64_t M, void *
         uint8_t *xc = ws_at(ws, L.a);
         uint8_t *xsf = ws_at(ws, L.a_sf);
         // one read of x for the absmax and the low-rank input, one for the quantisation
-        if (!stat || lora)
+        if (!stat || lora) {
+            SQ_CUDA(stage_event(SQ_STAGE_ACT_PASS1, 0, s), "event record");
             SQ_CUDA(sq::launch_act_pass1(x, M, K, w->lora_down, stat ? nullptr : amax, t32, status, sms, s),
                     "activation pass 1");
+            SQ_CUDA(stage_event(SQ_STAGE_ACT_PASS1, 1, s), "event record");
+        }
         // the quantisation also writes the low-rank operands (g_x is known by then)
         sq::LowrankOut lr;
         if (lora) {
@@ -481,9 +496,11 @@ sq_status sq_linear_fwd(const sq_weight *w, const uint16_t *x, int64_t M, void *
             lr.N = N;
             lr.udup = udup;
         }
+        SQ_CUDA(stage_event(SQ_STAGE_ACT_QUANT, 0, s), "event record");
         SQ_CUDA(sq::launch_nvfp4_quant_bf16(x, M, K, amax, stat ? gx : nullptr, stat ? nullptr : gx, xc, xsf, lr,
                                             status, sms, s),
                 "nvfp4 act quant + low-rank operands");
+        SQ_CUDA(stage_event(SQ_STAGE_ACT_QUANT, 1, s), "event record");
         g.fp4 = 1;
         g.a = xc;
         g.b = w->codes;
@@ -522,11 +539,9 @@ sq_status sq_linear_fwd(const sq_weight *w, const uint16_t *x, int64_t M, void *
         g.a = xb;
         g.b = wb;
     }
-    if (g_gemm_ev0)
-        SQ_CUDA(cudaEventRecord(g_gemm_ev0, s), "event record");
+    SQ_CUDA(stage_event(SQ_STAGE_GEMM, 0, s), "event record");
     SQ_CUDA(sq::launch_gemm(g, sms, s), "gemm");
-    if (g_gemm_ev1)
-        SQ_CUDA(cudaEventRecord(g_gemm_ev1, s), "event record");
+    SQ_CUDA(stage_event(SQ_STAGE_GEMM, 1, s), "event record");
     return SQ_OK;
 }
 
@@ -637,21 +652,26 @@ sq_status sq_linear_bwd_dx(const sq_weight *w, const uint16_t *dy, int64_t M, fl
     g.M = M;
     g.N = K;
     g.K = N;
-    if (g_gemm_ev0)
-        SQ_CUDA(cudaEventRecord(g_gemm_ev0, s), "event record");
+    SQ_CUDA(stage_event(SQ_STAGE_GEMM, 0, s), "event record");
     SQ_CUDA(sq::launch_gemm(g, sms, s), "gemm");
-    if (g_gemm_ev1)
-        SQ_CUDA(cudaEventRecord(g_gemm_ev1, s), "event record");
+    SQ_CUDA(stage_event(SQ_STAGE_GEMM, 1, s), "event record");
+    return SQ_OK;
+}
+
+sq_status sq_set_stage_events(int32_t stage, void *start_event, void *stop_event)
+{
+    if (stage < 0 || stage >= SQ_STAGE_COUNT)
+        return SQ_ERR_ARG;
+    if ((start_event == nullptr) != (stop_event == nullptr))
+        return SQ_ERR_NULL;
+    g_stage_ev[stage][0] = reinterpret_cast<cudaEvent_t>(start_event);
+    g_stage_ev[stage][1] = reinterpret_cast<cudaEvent_t>(stop_event);
     return SQ_OK;
 }
 
 sq_status sq_set_gemm_events(void *start_event, void *stop_event)
 {
-    if ((start_event == nullptr) != (stop_event == nullptr))
-        return SQ_ERR_NULL;
-    g_gemm_ev0 = reinterpret_cast<cudaEvent_t>(start_event);
-    g_gemm_ev1 = reinterpret_cast<cudaEvent_t>(stop_event);
-    return SQ_OK;
+    return sq_set_stage_events(SQ_STAGE_GEMM, start_event, stop_event);
 }
 
 sq_status sq_selftest_wait_timeout(void *ws, uint32_t limit_us, void *stream)

@@ -296,12 +296,10 @@ __device__ __forceinline__ void load_row64_bf16_sw128(const uint8_t *box, int R,
 }
 
 // The same row with the stride-1 butterfly folded into the widening (mixed
-// bf16 + fp32 arithmetic: one rounding each, like the fp32 butterfly on the
+// bf16 / fp32 arithmetic, one rounding each, like the fp32 butterfly on the
 // exactly widened values): pair j becomes (RN(v[2j] + v[2j+1]),
-// RN(v[2j+1] - v[2j])), i.e. the second value NEGATED.  Every later stride
-// pairs values of equal parity, so the odd values stay exactly negated through
-// the transform (round to nearest is symmetric); callers undo the sign where it
-// matters (a maximum of |v| does not care).
+// RN(v[2j] - v[2j+1])), the difference as fma(v[2j+1], -1, v[2j]) -- the same
+// bits as the fp32 subtraction, zero signs included.
 __device__ __forceinline__ void load_row64_bf16_sw128_s1(const uint8_t *box, int R, uint64_t (&p)[32])
 {
     const uint8_t *row = box + R * 128;
@@ -312,12 +310,12 @@ __device__ __forceinline__ void load_row64_bf16_sw128_s1(const uint8_t *box, int
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
             const float lo = __uint_as_float(w[j] << 16);
-            float sum, ndiff;
-            asm("{\n\t.reg .b16 h0, h1;\n\tmov.b32 {h0, h1}, %2;\n\t"
+            float sum, diff;
+            asm("{\n\t.reg .b16 h0, h1, m1;\n\tmov.b32 {h0, h1}, %2;\n\tmov.b16 m1, 0xBF80;\n\t"
                 "add.rn.f32.bf16 %0, h1, %3;\n\t"
-                "sub.rn.f32.bf16 %1, h1, %3;\n\t}"
-                : "=f"(sum), "=f"(ndiff) : "r"(w[j]), "f"(lo));
-            p[4 * i + j] = f2_pack(sum, ndiff);
+                "fma.rn.f32.bf16 %1, h1, m1, %3;\n\t}"
+                : "=f"(sum), "=f"(diff) : "r"(w[j]), "f"(lo));
+            p[4 * i + j] = f2_pack(sum, diff);
         }
     }
 }

@@ -844,7 +844,7 @@ __global__ void __launch_bounds__(kP1Threads, 1) act_pass1_kernel(const __grid_c
             __syncwarp();
             if (lane == 0)
                 mbar_arrive(empty + 8 * st);              // the stage's rows are in registers
-            fwht256_q4_from_s2(p, lane);                  // odd values negated: the maximum of |v| is unchanged
+            fwht256_q4_from_s2(p, lane);
 #pragma unroll
             for (int i = 0; i < 32; ++i) {
                 float lo, hi;
@@ -1027,7 +1027,7 @@ __global__ void __launch_bounds__(kAQThreads, 2) act_quant_kernel(const __grid_c
         __syncwarp();
         if (lane == 0)
             mbar_arrive(empty + 8 * st);
-        fwht256_q4_from_s2(p, lane);                  // p[j] = (v[2j], -v[2j+1]), unscaled
+        fwht256_q4_from_s2(p, lane);                  // unscaled: v[j] * 16
         const uint32_t row = rt * kAQRows + (uint32_t)R;
         uint32_t word[8];
         uint32_t sfw = 0;
@@ -1052,12 +1052,12 @@ __global__ void __launch_bounds__(kAQThreads, 2) act_quant_kernel(const __grid_c
                     float sv[16];
                     if (fold16) {
                         const float i16 = __fmul_rn(inv, 0.0625f);
-                        const uint64_t inv2 = f2_pack(i16, -i16);      // odd values are negated
+                        const uint64_t inv2 = f2_pack(i16, i16);
 #pragma unroll
                         for (int i = 0; i < 8; ++i)
                             f2_unpack(f2_mul(p[8 * b + i], inv2), sv[2 * i], sv[2 * i + 1]);
                     } else {
-                        const uint64_t inv2 = f2_pack(inv, -inv), s16 = f2_pack(0.0625f, 0.0625f);
+                        const uint64_t inv2 = f2_pack(inv, inv), s16 = f2_pack(0.0625f, 0.0625f);
 #pragma unroll
                         for (int i = 0; i < 8; ++i)
                             f2_unpack(f2_mul(f2_mul(p[8 * b + i], s16), inv2), sv[2 * i], sv[2 * i + 1]);

@@ -362,6 +362,21 @@ SQ_API sq_status sq_linear_bwd_dx(const sq_weight *w, const uint16_t *dy, int64_
 SQ_API sq_status sq_set_gemm_events(void *start_event, void *stop_event);
 
 /*
+ * The same instrumentation for any of the launches below (SQ_STAGE_GEMM is
+ * what sq_set_gemm_events sets): SQ_STAGE_ACT_PASS1 brackets the activation
+ * pass that takes max|H x| and t = x lora_down (sq_act_quant_nvfp4 and the
+ * NVFP4 sq_linear_fwd), SQ_STAGE_ACT_QUANT the pass that quantises H x.  An
+ * event between two launches keeps the second one from starting its set-up
+ * early (the launches overlap otherwise), so a timed call is a little slower
+ * than an untimed one.  Returns SQ_ERR_ARG for an unknown stage.
+ */
+#define SQ_STAGE_GEMM       0
+#define SQ_STAGE_ACT_PASS1  1
+#define SQ_STAGE_ACT_QUANT  2
+#define SQ_STAGE_COUNT      3
+SQ_API sq_status sq_set_stage_events(int32_t stage, void *start_event, void *stop_event);
+
+/*
  * Read back and clear the device status word that a kernel sets when it gives
  * up a bounded wait (SQ_ERR_TIMEOUT), or that the SQ_CHECK_FINITE scan sets
  * on a NaN or an infinity in x (SQ_ERR_NONFINITE; a timeout is reported

@@ -131,3 +131,15 @@ def make_stack_residual(i: int, N: int = 6144, K: int = 16384) -> np.ndarray:
     """Residual i of the 28-weight builder stack (down-projection shape, Student-t)."""
     rng = np.random.Generator(np.random.PCG64(stack_seed(i)))
     return _residual(rng, N, K, "student")
+
+
+def make_stack_residual_device(i: int, out, N: int = 6144, K: int = 16384):
+    """The same distribution drawn on a CUDA device into `out` (fp32 [N, K]) with torch's seeded
+    generator (seed stack_seed(i)): z / sqrt(Gamma(2) / 2) / sqrt(2 K), a Student-t(4) scaled to
+    std 1/sqrt(K).  A different stream from make_stack_residual, for timing only (numpy takes
+    seconds per weight)."""
+    g = torch.Generator(device=out.device).manual_seed(stack_seed(i))
+    torch.randn((N, K), generator=g, device=out.device, out=out)
+    chi = torch._standard_gamma(torch.full((N, K), 2.0, device=out.device), generator=g)
+    out.div_(chi.mul_(0.5).sqrt_()).mul_(float(1.0 / np.sqrt(2.0 * K)))
+    return out

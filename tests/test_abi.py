@@ -217,7 +217,7 @@ static const fnptr entries[] = {
     (fnptr)sq_status_str, (fnptr)sq_abi_version, (fnptr)sq_last_error_detail, (fnptr)sq_sf_bytes,
     (fnptr)sq_workspace_bytes, (fnptr)sq_build_int4, (fnptr)sq_svd_init, (fnptr)sq_build_int8,
     (fnptr)sq_build_nvfp4, (fnptr)sq_act_quant_nvfp4, (fnptr)sq_linear_fwd, (fnptr)sq_linear_fwd_noalloc,
-    (fnptr)sq_reconstruct_bf16, (fnptr)sq_linear_bwd_dx, (fnptr)sq_set_gemm_events,
+    (fnptr)sq_reconstruct_bf16, (fnptr)sq_linear_bwd_dx, (fnptr)sq_set_gemm_events, (fnptr)sq_set_stage_events,
     (fnptr)sq_check_device_status, (fnptr)sq_selftest_wait_timeout,
 };
 

@@ -306,12 +306,42 @@ def test_large_builders_sampled(sq, name):
     check_nvfp4_build(sq, d["R"], rows)
 
 
+def last_tile_rows(M, count, seed):
+    """Rows of the last 256-row GEMM tile (the half-empty one when M % 256 == 128)."""
+    lo = (M - 1) // 256 * 256
+    rng = np.random.default_rng(seed)
+    return rng.choice(np.arange(lo, M), size=min(count, M - lo), replace=False)
+
+
 @pytest.mark.parametrize("fmt", [2, 1], ids=["nvfp4", "int4"])
 @pytest.mark.parametrize("name", LARGE)
 def test_large_forward_sampled(sq, name, fmt):
+    """64 sampled rows of the full-size forward, 8 of them from the last 256-row tile."""
     d = inputs(name)
     M = d["x"].shape[0]
-    check_fwd(sq, d, fmt, sample_rows(M, 6, 22))
+    rows = np.unique(np.concatenate([sample_rows(M, 56, 22), last_tile_rows(M, 8, 25)])).astype(np.int64)
+    assert len(rows) >= 64 and rows.max() >= (M - 1) // 256 * 256
+    check_fwd(sq, d, fmt, rows)
+
+
+@pytest.mark.parametrize("name", LARGE)
+def test_large_act_quant_bit_exact(sq, name):
+    """The activation quantisation at M = 4480 in full: every code, every tiled scale byte
+    (padding included) and g_x bit for bit, t within 1e-5 of the fp64 sum."""
+    d = inputs(name)
+    check_act_quant(sq, d["x"], d["D"])
+
+
+@pytest.mark.parametrize("M", [9472, 9600], ids=["split-k", "unsplit"])
+def test_act_quant_unsplit_first_pass(sq, M):
+    """M = 9600 has 75 tiles of 128 rows, more than half the SMs, so the pass that takes the
+    absmax and t runs without splitting K (t written in one piece); M = 9472 (74 tiles) still splits
+    K in two.  Both bit-exact against the oracle, t within 1e-5."""
+    rng = np.random.default_rng(26)
+    K = 512
+    x = si.to_bf16_bits(rng.standard_normal((M, K), dtype=np.float32) * np.float32(1.5))
+    D = si.to_bf16_bits(rng.standard_normal((K, 32), dtype=np.float32) * np.float32(0.02))
+    check_act_quant(sq, x, D)
 
 
 @pytest.mark.parametrize("name", LARGE)
