@@ -48,7 +48,7 @@ SQ_OP_SVD_INIT = 10
 RANK = 32
 
 EXPORTED = [
-    "sq_status_str", "sq_abi_version", "sq_last_error_detail", "sq_sf_bytes", "sq_workspace_bytes",
+    "sq_status_str", "sq_abi_version", "sq_debug_checks", "sq_selftest_index_check", "sq_last_error_detail", "sq_sf_bytes", "sq_workspace_bytes",
     "sq_build_int4", "sq_build_int8", "sq_build_nvfp4", "sq_act_quant_nvfp4", "sq_linear_fwd",
     "sq_reconstruct_bf16",
     "sq_check_device_status", "sq_set_gemm_events", "sq_set_stage_events", "sq_linear_fwd_noalloc", "sq_linear_bwd_dx",
@@ -83,6 +83,8 @@ _I64 = ctypes.c_int64
 _SIGS = {
     "sq_status_str": ([ctypes.c_int], ctypes.c_char_p),
     "sq_abi_version": ([], ctypes.c_int),
+    "sq_debug_checks": ([], ctypes.c_int),
+    "sq_selftest_index_check": ([_P, _P], ctypes.c_int),
     "sq_last_error_detail": ([], ctypes.c_char_p),
     "sq_sf_bytes": ([_I64, _I64], ctypes.c_size_t),
     "sq_workspace_bytes": ([ctypes.c_int, _I64, _I64, _I64], ctypes.c_size_t),
@@ -310,6 +312,15 @@ def sq_linear_bwd_dx(w: "Weight", dy, dx, ws, stream=None):
     cw = w.as_c()
     _check("sq_linear_bwd_dx", lib().sq_linear_bwd_dx(ctypes.byref(cw), _ptr(dy), M, _ptr(dx), _ptr(ws),
                                                       _numel_bytes(ws), _stream(stream)))
+
+
+def sq_debug_checks() -> int:
+    """1 if the loaded library was built with the device-side index checks (libsq_debug.so)."""
+    return lib().sq_debug_checks()
+
+
+def sq_selftest_index_check(ws, stream=None):
+    _check("sq_selftest_index_check", lib().sq_selftest_index_check(_ptr(ws), _stream(stream)))
 
 
 def sq_selftest_wait_timeout(ws, limit_us: int = 20000, stream=None):

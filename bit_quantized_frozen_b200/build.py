@@ -10,6 +10,9 @@ ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(PKG, "libsq.so")
+# the same library with the device-side index checks on (-DSQ_DEBUG_CHECKS): every checked store
+# tests its index against its buffer, skips it when outside and reports SQ_ERR_INDEX
+LIB_DEBUG = os.path.join(PKG, "libsq_debug.so")
 SOURCES = ["sq_api.cu", "sq_quant.cu", "sq_gemm.cu", "sq_svd.cu"]
 HEADERS = ["sq_device.cuh", "sq_ptx.cuh", "sq_kernels.h"]
 
@@ -26,34 +29,39 @@ def nvcc() -> str:
     return cand if os.path.exists(cand) else "nvcc"
 
 
-def _stale() -> bool:
-    if not os.path.exists(LIB):
+def _stale(lib: str = LIB) -> bool:
+    if not os.path.exists(lib):
         return True
-    t = os.path.getmtime(LIB)
+    t = os.path.getmtime(lib)
     deps = [os.path.join(CSRC, f) for f in SOURCES + HEADERS] + [os.path.join(INCLUDE, "sq.h")]
     return any(os.path.getmtime(d) > t for d in deps)
 
 
-def build(force: bool = False, verbose: bool = False, extra: list[str] | None = None) -> str:
-    if not force and not _stale():
-        return LIB
+def build(force: bool = False, verbose: bool = False, extra: list[str] | None = None,
+          debug_checks: bool = False) -> str:
+    lib = LIB_DEBUG if debug_checks else LIB
+    if not force and not _stale(lib):
+        return lib
+    if debug_checks:
+        extra = list(extra or []) + ["-DSQ_DEBUG_CHECKS"]
     objs = []
     for src in SOURCES:
-        obj = os.path.join(CSRC, src.replace(".cu", ".o"))
+        obj = os.path.join(CSRC, src.replace(".cu", ".debug.o" if debug_checks else ".o"))
         cmd = [nvcc(), *NVCC_FLAGS, *(extra or []), "-I", INCLUDE, "-c", os.path.join(CSRC, src), "-o", obj]
         if verbose:
             print(" ".join(cmd), file=sys.stderr)
         subprocess.run(cmd, check=True)
         objs.append(obj)
-    tmp = LIB + ".tmp"
+    tmp = lib + ".tmp"
     subprocess.run([nvcc(), "-shared", "-gencode", "arch=compute_100a,code=sm_100a", "-o", tmp, *objs,
                     "-cudart", "static"], check=True)
-    os.replace(tmp, LIB)
+    os.replace(tmp, lib)
     for o in objs:
         os.remove(o)
-    return LIB
+    return lib
 
 
 if __name__ == "__main__":
     build(force="--force" in sys.argv, verbose=True,
-          extra=["-Xptxas", "-v"] if "--ptxas-v" in sys.argv else None)
+          extra=["-Xptxas", "-v"] if "--ptxas-v" in sys.argv else None,
+          debug_checks="--debug-checks" in sys.argv)

@@ -10,6 +10,7 @@
 #include <cstring>
 
 #include "sq.h"
+#include "sq_device.cuh"
 #include "sq_kernels.h"
 #include "sq_ptx.cuh"
 
@@ -43,6 +44,18 @@ unsigned long long current_context_id()
 
 }  // namespace sq
 
+
+// One thread checks the index one past `bound` with the device-side index check
+// of the debug builds: the check fails, the access it guards (never made) is
+// skipped, and the status word gets the index bit.
+static __global__ void selftest_index_kernel(uint32_t *status, uint32_t bound)
+{
+    if (threadIdx.x == 0) {
+        const uint32_t idx = bound;
+        if (sq::dcheck(idx < bound, status))
+            status[1] = idx;                          // unreachable: the check fails
+    }
+}
 
 // One thread waits on an mbarrier that nothing ever arrives on, with the
 // bounded wait every kernel of the library uses; it must give up after
@@ -239,6 +252,7 @@ const char *sq_status_str(int status)
     case SQ_ERR_ARG: return "bad argument";
     case SQ_ERR_TIMEOUT: return "kernel wait timed out";
     case SQ_ERR_NONFINITE: return "non-finite input";
+    case SQ_ERR_INDEX: return "device index check failed";
     default: return "unknown status";
     }
 }
@@ -246,6 +260,15 @@ const char *sq_status_str(int status)
 int sq_abi_version(void)
 {
     return 1;
+}
+
+int sq_debug_checks(void)
+{
+#ifdef SQ_DEBUG_CHECKS
+    return 1;
+#else
+    return 0;
+#endif
 }
 
 const char *sq_last_error_detail(void)
@@ -694,6 +717,24 @@ sq_status sq_selftest_wait_timeout(void *ws, uint32_t limit_us, void *stream)
     return SQ_OK;
 }
 
+sq_status sq_selftest_index_check(void *ws, void *stream)
+{
+    if (!ws)
+        return SQ_ERR_NULL;
+    if (!aligned(ws, 256))
+        return SQ_ERR_ALIGN;
+    int sms = 0;
+    sq_status st = check_device(&sms);
+    if (st != SQ_OK)
+        return st;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    uint32_t *status = reinterpret_cast<uint32_t *>(ws);
+    SQ_CUDA(cudaMemsetAsync(status, 0, 4, s), "memset");
+    selftest_index_kernel<<<1, 32, 0, s>>>(status, 256u);
+    SQ_CUDA(cudaGetLastError(), "self-test launch");
+    return SQ_OK;
+}
+
 sq_status sq_check_device_status(void *ws, void *stream)
 {
     if (!ws) {                                         // the library's own word (calls without a workspace)
@@ -713,7 +754,8 @@ sq_status sq_check_device_status(void *ws, void *stream)
     SQ_CUDA(cudaStreamSynchronize(s), "status sync");
     if (word != 0) {
         SQ_CUDA(cudaMemsetAsync(ws, 0, 4, s), "status clear");
-        return (word & 1u) ? SQ_ERR_TIMEOUT : SQ_ERR_NONFINITE;   // bit 0 timeout, bit 1 non-finite
+        // bit 0 timeout, bit 2 failed index check, bit 1 non-finite input
+        return (word & 1u) ? SQ_ERR_TIMEOUT : (word & sq::kStatusIndex) ? SQ_ERR_INDEX : SQ_ERR_NONFINITE;
     }
     return SQ_OK;
 }

@@ -21,6 +21,24 @@ constexpr int kFracCount = 26;     // int4 scale fractions 0.50, 0.52, ..., 1.00
 // device status word bits (first word of every workspace)
 constexpr uint32_t kStatusTimeout = 1u;      // a bounded wait gave up
 constexpr uint32_t kStatusNonfinite = 2u;    // the SQ_CHECK_FINITE scan met a NaN or an infinity
+constexpr uint32_t kStatusIndex = 4u;        // a device-side index check failed (the access was skipped)
+
+// Device-side index check: true if ok; otherwise sets kStatusIndex in *status
+// (when non-NULL) and returns false so the caller skips the access.  Kernels
+// call it through SQ_DCHECK, which is the check itself in a build with
+// SQ_DEBUG_CHECKS and the constant true otherwise.
+__device__ __forceinline__ bool dcheck(bool ok, uint32_t *status)
+{
+    if (!ok && status)
+        atomicOr(status, kStatusIndex);
+    return ok;
+}
+
+#ifdef SQ_DEBUG_CHECKS
+#define SQ_DCHECK(cond, status) (::sq::dcheck((cond), (status)))
+#else
+#define SQ_DCHECK(cond, status) (true)
+#endif
 
 // ---------------------------------------------------------------------------
 // Hadamard-256 over one warp.

@@ -1,18 +1,27 @@
-// sq_quant.cu -- HBM-bound kernels of the SquareQ W4 layer: Hadamard-256
-// rotation + absmax, NVFP4 block quantisation into the tiled scale layout,
-// the int4 group-32 builder with its scale-fraction sweep, the bf16
-// activation rotation and int4 dequant of the "dequant-first" forward, the
-// low-rank input t = x . lora_down, and the bf16 reconstruct.
+// sq_quant.cu -- the non-GEMM kernels of the SquareQ W4 layer: the NVFP4
+// builder (Hadamard-256 + tensor absmax, then block quantisation into the
+// tiled scale layout), the int4 and int8 builders with their scale-fraction
+// sweeps, the activation prologue of the NVFP4 forward (absmax + t on tcgen05,
+// then quantisation), the bf16 rotation and dequant of the "dequant-first"
+// int4 / int8 forwards, the low-rank operands, and the bf16 reconstructs.
 //
-// All kernels are grid-stride loops over warp-sized tasks, launched with a
-// grid that is a multiple of the SM count; loads and stores are contiguous per
-// warp.  They follow the SquareQ README, section "SquareQ v3 -- W4", as stated
-// operation by operation in include/sq.h.
+// What bounds each: the builders' passes and the residual-only reconstruct
+// stream HBM; the int4 / int8 builders are bound by the FP32 / ALU issue of
+// their 26-trial sweeps; the reconstruct with the low-rank term by the FMA
+// pipe (its rank-r fmaf chain); the activation passes by the L1 data pipe
+// (Hadamard shuffles) and the FP32 pipe.  Persistent grids are sized from the
+// SM count; loads and stores are contiguous per warp or go through TMA.  They
+// follow the SquareQ README, section "SquareQ v3 -- W4", as stated operation
+// by operation in include/sq.h.
 #include "sq_kernels.h"
 #include "sq_device.cuh"
 #include "sq_ptx.cuh"
 
 namespace sq {
+
+// the library's own device status word, for kernels whose call takes no
+// workspace (timeouts of bounded waits, failed index checks of debug builds)
+__device__ uint32_t g_library_status;
 
 // ---------------------------------------------------------------------------
 // Block streamer.  The input ([rows, K], K % 256 == 0) is viewed as a 2-D
@@ -290,11 +299,12 @@ __global__ void __launch_bounds__(kStreamThreads) nvfp4_quant_kernel(const __gri
             word[2 * h + 1] = w1;
             sfc[h] = code;
         }
-        if (row < rows)
+        if (row < rows && SQ_DCHECK(row * (K / 2) + kb * (kHad / 2) + 16 * q + 16 <= rows * (K / 2), &g_library_status))
             *reinterpret_cast<uint4 *>(codes + row * (K / 2) + kb * (kHad / 2) + 16 * q) =
                 make_uint4(word[0], word[1], word[2], word[3]);
         // scale columns 2q, 2q+1 of the block are adjacent bytes of the tiled layout
-        *reinterpret_cast<uint16_t *>(sf + sf_offset(row, kb * (kHad / kSfBlock) + 2 * q, C)) =
+        if (SQ_DCHECK(sf_offset(row, kb * (kHad / kSfBlock) + 2 * q, C) + 2 <= rows_pad * C, &g_library_status))
+            *reinterpret_cast<uint16_t *>(sf + sf_offset(row, kb * (kHad / kSfBlock) + 2 * q, C)) =
             (uint16_t)(sfc[0] | (sfc[1] << 8));
     }, lowrank);
 }
@@ -414,6 +424,8 @@ __global__ void __launch_bounds__(kStreamThreads, 2) int4_build_kernel(const __g
             word[i >> 3] |= (((uint32_t)q0 & 0xFu) | (((uint32_t)q1 & 0xFu) << 4)) << (4 * (i & 7));
         }
         const int64_t hidx = 8 * b + (lane & 7);     // flat index of this lane's 32 values
+        if (!SQ_DCHECK(hidx < 8 * blocks, &g_library_status))
+            return;
         reinterpret_cast<uint4 *>(codes)[hidx] = make_uint4(word[0], word[1], word[2], word[3]);
         if (G == 32 || (lane & 1) == 0) {
             const int64_t gidx = G == 32 ? hidx : hidx >> 1;
@@ -571,6 +583,8 @@ __global__ void __launch_bounds__(kI8Threads) int8_build_kernel(const float *__r
                 }
                 w[c] = word;
             }
+            if (!SQ_DCHECK(n < N && (int64_t)b * kHad + 32 * q + 32 <= K, &g_library_status))
+                continue;
             uint4 *dst = reinterpret_cast<uint4 *>(codes + n * K + (int64_t)b * kHad + 32 * q);
             dst[0] = make_uint4(w[0], w[1], w[2], w[3]);
             dst[1] = make_uint4(w[4], w[5], w[6], w[7]);
@@ -876,6 +890,8 @@ __global__ void __launch_bounds__(kP1Threads, 1) act_pass1_kernel(const __grid_c
         tc_fence_before();
         const int64_t row = m0 + 32 * warp + lane;
         if (row < M) {
+            if (!SQ_DCHECK(j < split, status))
+                return;
             float4 *o = reinterpret_cast<float4 *>(t32 + ((int64_t)j * M + row) * kRank);
 #pragma unroll
             for (int i = 0; i < 32; i += 4)
@@ -1071,7 +1087,7 @@ __global__ void __launch_bounds__(kAQThreads, 2) act_quant_kernel(const __grid_c
             word[2 * b + 1] = w1;
             sfw |= code << (8 * b);
         }
-        if ((int64_t)row < M) {
+        if ((int64_t)row < M && SQ_DCHECK(kb * (kHad / 2) + 32 * q + 32 <= K / 2, status)) {
             uint4 *o = reinterpret_cast<uint4 *>(codes + (size_t)row * (size_t)(K / 2) + kb * (kHad / 2) + 32 * q);
             o[0] = make_uint4(word[0], word[1], word[2], word[3]);
             o[1] = make_uint4(word[4], word[5], word[6], word[7]);
@@ -1079,7 +1095,8 @@ __global__ void __launch_bounds__(kAQThreads, 2) act_quant_kernel(const __grid_c
         // scale columns 4q .. 4q+3 of the chunk are four adjacent bytes of the tiled layout
         const uint32_t c4 = kb * (kHad / kSfBlock) / 4 + q;       // (column / 4) of the first of the four
         const size_t off = ((size_t)(row >> 7) * (C >> 2) + c4) * 512 + (row & 31) * 16 + ((row & 127) >> 5) * 4;
-        *reinterpret_cast<uint32_t *>(sf + off) = sfw;
+        if (SQ_DCHECK(off + 4 <= (size_t)rows_pad * C, status))
+            *reinterpret_cast<uint32_t *>(sf + off) = sfw;
         kb += step_kb;
         rt += step_rt;
         if (kb >= nkb32) {
@@ -1108,23 +1125,19 @@ __global__ void __launch_bounds__(256) lowrank_finish_kernel(const float *__rest
 }
 
 // ---------------------------------------------------------------------------
-// bf16 reconstruct.  Tile = one 256-column block kb x 64 rows.  Persistent
-// CTAs of 256 threads walk a contiguous range of tiles (kb-major), staging the
-// next tile's codes, scales and lora_up rows in shared memory by cp.async
-// while the current one is computed, and keeping lora_down for the current kb
-// in registers.
+// bf16 reconstruct without the low-rank term (SQ_RECON_RESIDUAL_ONLY, or a
+// weight without factors).  Tile = one 256-column block kb x 64 rows.
+// Persistent CTAs of 256 threads walk a contiguous range of tiles (kb-major),
+// staging the next tile's codes and scales in shared memory by cp.async while
+// the current one is computed.
 // Phase 1: each lane decodes 32 payload values of a row (an int4 group or half
 //   group, two NVFP4 blocks, or 32 int8 codes), runs the 8-lane Hadamard
-//   transform and writes h into a
-//   shared fp32 tile (float4 f of a row stored at f ^ (f >> 3) -- conflict free
-//   for both phases).
-// Phase 2 (with the low-rank term, or for the transposed output W^T [K, N]):
-//   thread t owns columns 2(t%128), 2(t%128)+1 and rows 32(t/128)..+31.
-//   lora_down for its two columns stays in registers; lora_up rows are
-//   broadcast from shared memory; each output's fmaf chain runs in order
-//   r = 0..rank-1 from 0 (rank 32, or 16 for int8), two columns at a time with
-//   fma.rn.f32x2 (two
-//   independent fmaf, bit-identical to the scalar chain); W = bf16(RN(L + h)).
+//   transform and writes bf16(h) to W, or (for the transposed output W^T
+//   [K, N]) h into a shared fp32 tile (float4 f of a row stored at f ^ (f >> 3)
+//   -- conflict free for both phases).
+// Phase 2 (W^T only): thread t owns columns 2(t%128), 2(t%128)+1 and rows
+//   32(t/128)..+31 of the tile and writes them as two 64-byte row pieces of W^T.
+// The low-rank reconstruct is reconstruct_ws_kernel below.
 // ---------------------------------------------------------------------------
 constexpr int kRecRows = 64;
 constexpr int kRecScaleBytes = kRecRows * 16;             // 1 KB (8 fp16, 4 fp16, 16 ue4m3 or 1 fp32 per row)
@@ -1140,7 +1153,7 @@ struct RecCfg {
     static constexpr int kUBytes = kRecRows * kRank * 2;                      // 4 or 2 KB
     static constexpr int kStageBytes = kCodeBytes + kRecScaleBytes + kUBytes;
     static constexpr int kUsBytes = kRecRows * kRank * 4;
-    static constexpr int kSmemLowrank = kRecHBytes + kUsBytes + 2 * kStageBytes;   // 98 or 106 KB
+    static constexpr int kSmemTiled = kRecHBytes + 2 * kStageBytes;             // h tile + two stages (W^T)
     static constexpr int kSmemResidual = 2 * kStageBytes;
 };
 
@@ -1285,21 +1298,17 @@ __device__ __forceinline__ void rec_decode(const uint8_t *stage, int r, int q, f
     }
 }
 
-template <int FMT, bool LOWRANK, bool TRANS>
-__global__ void __launch_bounds__(256, (LOWRANK || TRANS) ? 2 : 3) reconstruct_kernel(const uint8_t *__restrict__ codes,
-                                                             const void *__restrict__ scales,
-                                                             const float *__restrict__ g_w,
-                                                             const uint16_t *__restrict__ U,
-                                                             const uint16_t *__restrict__ D, int64_t N, int64_t K,
-                                                             uint16_t *__restrict__ W)
+template <int FMT, bool TRANS>
+__global__ void __launch_bounds__(256, TRANS ? 2 : 3) reconstruct_kernel(const uint8_t *__restrict__ codes,
+                                                                      const void *__restrict__ scales,
+                                                                      const float *__restrict__ g_w,
+                                                                      const uint16_t *__restrict__ U, int64_t N,
+                                                                      int64_t K, uint16_t *__restrict__ W)
 {
     using Cfg = RecCfg<FMT>;
-    constexpr int kR = Cfg::kRank;
     extern __shared__ __align__(128) uint8_t rec_smem[];
     float *h = reinterpret_cast<float *>(rec_smem);                                // [64][256] swizzled
-    float *us = reinterpret_cast<float *>(rec_smem + kRecHBytes);                  // [64][rank] lora_up, fp32
-    constexpr bool kTile = LOWRANK || TRANS;      // h goes through the shared tile (phase 2 writes W)
-    uint8_t *stage0 = rec_smem + (kTile ? kRecHBytes + Cfg::kUsBytes : 0);
+    uint8_t *stage0 = rec_smem + (TRANS ? kRecHBytes : 0);
     const int tid = threadIdx.x;
     const int lane = tid & 31, warp = tid >> 5;
     const float g = FMT == 2 ? *g_w : 0.0f;
@@ -1310,22 +1319,20 @@ __global__ void __launch_bounds__(256, (LOWRANK || TRANS) ? 2 : 3) reconstruct_k
     if (t_begin >= t_end)
         return;
     const uint32_t sbase = smem_u32(stage0);
-    rec_stage<FMT, LOWRANK>(sbase, codes, scales, U, N, K, t_begin / NT, (t_begin % NT) * kRecRows, tid);
+    rec_stage<FMT, false>(sbase, codes, scales, U, N, K, t_begin / NT, (t_begin % NT) * kRecRows, tid);
     cp_async_commit();
 
-    const int cp = tid & 127;                        // phase 2: column pair
+    const int cp = tid & 127;                        // phase 2 (W^T): column pair
     const int rbase = 32 * (tid >> 7);
     const int f = cp >> 1;                           // float4 of h holding columns 2cp, 2cp+1
     const int fo = 2 * (cp & 1);
-    uint64_t d2[kR];
-    int64_t cur_kb = -1;
 
 #pragma unroll 1
     for (int64_t t = t_begin, i = 0; t < t_end; ++t, ++i) {
         const int buf = (int)(i & 1);
         if (t + 1 < t_end)
-            rec_stage<FMT, LOWRANK>(sbase + (buf ^ 1) * Cfg::kStageBytes, codes, scales, U, N, K, (t + 1) / NT,
-                                    ((t + 1) % NT) * kRecRows, tid);
+            rec_stage<FMT, false>(sbase + (buf ^ 1) * Cfg::kStageBytes, codes, scales, U, N, K, (t + 1) / NT,
+                                  ((t + 1) % NT) * kRecRows, tid);
         cp_async_commit();
         cp_async_wait<1>();
         __syncthreads();                             // tile t staged; previous tile's phase 2 done
@@ -1341,9 +1348,9 @@ __global__ void __launch_bounds__(256, (LOWRANK || TRANS) ? 2 : 3) reconstruct_k
             float v[32];
             rec_decode<FMT>(st, r, q, g, v);
             fwht256_l32(v, lane);
-            if (!kTile) {                            // residual only, row-major: straight to W
+            if (!TRANS) {                            // row-major: straight to W
                 const int64_t n = n0 + r;
-                if (n < N) {
+                if (n < N && SQ_DCHECK(kb * kHad + 32 * q + 32 <= K, &g_library_status)) {
                     uint4 *o = reinterpret_cast<uint4 *>(W + n * K + kb * kHad + 32 * q);
 #pragma unroll
                     for (int k = 0; k < 4; ++k) {
@@ -1363,94 +1370,42 @@ __global__ void __launch_bounds__(256, (LOWRANK || TRANS) ? 2 : 3) reconstruct_k
                 }
             }
         }
-        if (!kTile) {
+        if (!TRANS) {
             __syncthreads();                         // stage buffer free before the next prefetch lands
             continue;
         }
-        if (LOWRANK) {
-            const uint16_t *ust = reinterpret_cast<const uint16_t *>(st + Cfg::kCodeBytes + kRecScaleBytes);
-#pragma unroll
-            for (int j = 0; j < kRecRows * kR / 256; ++j) {
-                us[tid + 256 * j] = bf16_bits_to_f32(ust[tid + 256 * j]);
-            }
-        }
-        if (LOWRANK && kb != cur_kb) {               // lora_down of this thread's two columns
-            cur_kb = kb;
-            const int64_t k0 = kb * kHad + 2 * cp;
-            const uint4 *dr0 = reinterpret_cast<const uint4 *>(D + k0 * kR);
-            const uint4 *dr1 = reinterpret_cast<const uint4 *>(D + (k0 + 1) * kR);
-#pragma unroll
-            for (int k = 0; k < kR / 8; ++k) {
-                const uint4 a = __ldg(dr0 + k), b = __ldg(dr1 + k);
-                const uint32_t wa[4] = {a.x, a.y, a.z, a.w}, wb[4] = {b.x, b.y, b.z, b.w};
-#pragma unroll
-                for (int j = 0; j < 4; ++j) {
-                    d2[8 * k + 2 * j] = pack2(bf16_bits_to_f32(wa[j] & 0xFFFFu), bf16_bits_to_f32(wb[j] & 0xFFFFu));
-                    d2[8 * k + 2 * j + 1] = pack2(bf16_bits_to_f32(wa[j] >> 16), bf16_bits_to_f32(wb[j] >> 16));
-                }
-            }
-        }
-        __syncthreads();                             // h and us complete
+        __syncthreads();                             // h complete
 
-        // phase 2
+        // phase 2 (W^T [K, N]): rows k0, k0 + 1, columns n0 + rbase .. + 31
         const int64_t k0 = kb * kHad + 2 * cp;
-        uint32_t tw0[16], tw1[16];                   // TRANS: columns k0, k0 + 1 of the 32 rows, bf16 pairs
-        constexpr int kUnroll = TRANS ? 8 : 1;       // register-indexed pieces need constant indices
-#pragma unroll kUnroll
-        for (int r0 = rbase; r0 < rbase + 32; r0 += 4) {
-            uint64_t acc[4] = {0ull, 0ull, 0ull, 0ull};
+        uint32_t tw0[16], tw1[16];                   // columns k0, k0 + 1 of the 32 rows, bf16 pairs
 #pragma unroll
-            for (int rr = 0; rr < (LOWRANK ? kR : 0); rr += 4) {
-                float4 u4[4];
-#pragma unroll
-                for (int j = 0; j < 4; ++j)
-                    u4[j] = *reinterpret_cast<const float4 *>(us + (r0 + j) * kR + rr);
-#pragma unroll
-                for (int j = 0; j < 4; ++j) {
-                    fma2(acc[j], pack2(u4[j].x, u4[j].x), d2[rr]);
-                    fma2(acc[j], pack2(u4[j].y, u4[j].y), d2[rr + 1]);
-                    fma2(acc[j], pack2(u4[j].z, u4[j].z), d2[rr + 2]);
-                    fma2(acc[j], pack2(u4[j].w, u4[j].w), d2[rr + 3]);
-                }
-            }
-#pragma unroll
-            for (int j = 0; j < 4; ++j) {
-                const int r = r0 + j;
-                const int64_t n = n0 + r;
-                const float2 hv = *reinterpret_cast<const float2 *>(h + r * kHad + 4 * (f ^ (f >> 3)) + fo);
-                float L0, L1;
-                unpack2(acc[j], L0, L1);
-                // with the low-rank term W = bf16(RN(L + h)); residual only: bf16(h)
-                const float o0 = LOWRANK ? __fadd_rn(L0, hv.x) : hv.x;
-                const float o1 = LOWRANK ? __fadd_rn(L1, hv.y) : hv.y;
-                if (TRANS) {
-                    const uint32_t b0 = f32_to_bf16_bits(o0), b1 = f32_to_bf16_bits(o1);
-                    const int slot = (r - rbase) >> 1, hi = (r - rbase) & 1;
-                    tw0[slot] = hi ? (tw0[slot] | (b0 << 16)) : b0;
-                    tw1[slot] = hi ? (tw1[slot] | (b1 << 16)) : b1;
-                } else if (n < N) {
-                    *reinterpret_cast<uint32_t *>(W + n * K + k0) = f32x2_to_bf16x2_bits(o0, o1);
-                }
-            }
+        for (int rr = 0; rr < 32; ++rr) {
+            const int r = rbase + rr;
+            const float2 hv = *reinterpret_cast<const float2 *>(h + r * kHad + 4 * (f ^ (f >> 3)) + fo);
+            const uint32_t b0 = f32_to_bf16_bits(hv.x), b1 = f32_to_bf16_bits(hv.y);
+            const int slot = rr >> 1, hi = rr & 1;
+            tw0[slot] = hi ? (tw0[slot] | (b0 << 16)) : b0;
+            tw1[slot] = hi ? (tw1[slot] | (b1 << 16)) : b1;
         }
-        if (TRANS) {                                 // W^T [K, N]: rows k0, k0 + 1, columns n0 + rbase .. + 31
-            const int64_t nb0 = n0 + rbase;
-            if (nb0 + 32 <= N) {
-                uint4 *o0 = reinterpret_cast<uint4 *>(W + k0 * N + nb0);
-                uint4 *o1 = reinterpret_cast<uint4 *>(W + (k0 + 1) * N + nb0);
+        const int64_t nb0 = n0 + rbase;
+        if (!SQ_DCHECK(k0 + 1 < K, &g_library_status))
+            continue;
+        if (nb0 + 32 <= N) {
+            uint4 *o0 = reinterpret_cast<uint4 *>(W + k0 * N + nb0);
+            uint4 *o1 = reinterpret_cast<uint4 *>(W + (k0 + 1) * N + nb0);
 #pragma unroll
-                for (int c = 0; c < 4; ++c) {
-                    o0[c] = make_uint4(tw0[4 * c], tw0[4 * c + 1], tw0[4 * c + 2], tw0[4 * c + 3]);
-                    o1[c] = make_uint4(tw1[4 * c], tw1[4 * c + 1], tw1[4 * c + 2], tw1[4 * c + 3]);
-                }
-            } else {
-#pragma unroll
-                for (int i = 0; i < 32; ++i)
-                    if (nb0 + i < N) {
-                        W[k0 * N + nb0 + i] = (uint16_t)(tw0[i >> 1] >> (16 * (i & 1)));
-                        W[(k0 + 1) * N + nb0 + i] = (uint16_t)(tw1[i >> 1] >> (16 * (i & 1)));
-                    }
+            for (int c = 0; c < 4; ++c) {
+                o0[c] = make_uint4(tw0[4 * c], tw0[4 * c + 1], tw0[4 * c + 2], tw0[4 * c + 3]);
+                o1[c] = make_uint4(tw1[4 * c], tw1[4 * c + 1], tw1[4 * c + 2], tw1[4 * c + 3]);
             }
+        } else {
+#pragma unroll
+            for (int i = 0; i < 32; ++i)
+                if (nb0 + i < N) {
+                    W[k0 * N + nb0 + i] = (uint16_t)(tw0[i >> 1] >> (16 * (i & 1)));
+                    W[(k0 + 1) * N + nb0 + i] = (uint16_t)(tw1[i >> 1] >> (16 * (i & 1)));
+                }
         }
     }
     cp_async_wait<0>();
@@ -1652,7 +1607,7 @@ __global__ void __launch_bounds__(kWsThreads, 1) reconstruct_ws_kernel(const uin
                     const int slot = (r - rbase) >> 1, hi = (r - rbase) & 1;
                     tw0[slot] = hi ? (tw0[slot] | (b0 << 16)) : b0;
                     tw1[slot] = hi ? (tw1[slot] | (b1 << 16)) : b1;
-                } else if (n < N) {
+                } else if (n < N && SQ_DCHECK(k0 + 1 < K, status)) {
                     *reinterpret_cast<uint32_t *>(W + n * K + k0) = f32x2_to_bf16x2_bits(o0, o1);
                 }
             }
@@ -1662,7 +1617,9 @@ __global__ void __launch_bounds__(kWsThreads, 1) reconstruct_ws_kernel(const uin
             mbar_arrive(h_free + 8 * sb);              // h and us of this tile are no longer read
         if (TRANS) {                                 // W^T [K, N]: rows k0, k0 + 1, columns n0 + rbase .. + 31
             const int64_t nb0 = n0 + rbase;
-            if (nb0 + 32 <= N) {
+            if (!SQ_DCHECK(k0 + 1 < K, status)) {
+                // index check failed (debug builds): the stores are skipped
+            } else if (nb0 + 32 <= N) {
                 uint4 *o0 = reinterpret_cast<uint4 *>(W + k0 * N + nb0);
                 uint4 *o1 = reinterpret_cast<uint4 *>(W + (k0 + 1) * N + nb0);
 #pragma unroll
@@ -1710,9 +1667,6 @@ cudaError_t launch_check_finite_bf16(const uint16_t *x, int64_t n, uint32_t *sta
                                                                            status);
     return cudaGetLastError();
 }
-
-// the library's own device status word, for kernels whose call takes no workspace
-__device__ uint32_t g_library_status;
 
 cudaError_t library_status_word(uint32_t **p)
 {
@@ -2000,31 +1954,30 @@ cudaError_t launch_lowrank_finish(const float *t_part, int parts, int64_t M, con
     return cudaGetLastError();
 }
 
-template <int FMT, bool LOWRANK, bool TRANS>
+template <int FMT, bool TRANS>
 static cudaError_t launch_reconstruct_v(const uint8_t *codes, const void *scales, const float *g_w,
-                                        const uint16_t *U, const uint16_t *D, int64_t N, int64_t K, uint16_t *W,
-                                        int sms, cudaStream_t s)
+                                        const uint16_t *U, int64_t N, int64_t K, uint16_t *W, int sms,
+                                        cudaStream_t s)
 {
     using Cfg = RecCfg<FMT>;
-    constexpr bool kTile = LOWRANK || TRANS;
-    constexpr int kSmem = kTile ? Cfg::kSmemLowrank : Cfg::kSmemResidual;
+    constexpr int kSmem = TRANS ? Cfg::kSmemTiled : Cfg::kSmemResidual;
     constexpr int kMaxDev = 64;
     static unsigned long long attr_ctx[kMaxDev];
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDev)
         return cudaErrorInvalidDevice;
     const unsigned long long ctx = current_context_id();
-    if (kTile && (ctx == 0 || attr_ctx[dev] != ctx)) {
-        cudaError_t e = cudaFuncSetAttribute(reconstruct_kernel<FMT, LOWRANK, TRANS>,
+    if (TRANS && (ctx == 0 || attr_ctx[dev] != ctx)) {
+        cudaError_t e = cudaFuncSetAttribute(reconstruct_kernel<FMT, TRANS>,
                                              cudaFuncAttributeMaxDynamicSharedMemorySize, kSmem);
         if (e != cudaSuccess)
             return e;
         attr_ctx[dev] = ctx;
     }
     const int64_t tiles = (K / kHad) * ((N + kRecRows - 1) / kRecRows);
-    const int64_t per_sm = kTile ? 2 : 3;                   // resident CTAs per SM (registers, shared memory)
+    const int64_t per_sm = TRANS ? 2 : 3;                    // resident CTAs per SM (registers, shared memory)
     const unsigned grid = (unsigned)(tiles < per_sm * sms ? tiles : per_sm * sms);
-    reconstruct_kernel<FMT, LOWRANK, TRANS><<<grid, 256, kSmem, s>>>(codes, scales, g_w, U, D, N, K, W);
+    reconstruct_kernel<FMT, TRANS><<<grid, 256, kSmem, s>>>(codes, scales, g_w, U, N, K, W);
     return cudaGetLastError();
 }
 
@@ -2065,9 +2018,9 @@ static cudaError_t launch_reconstruct_fmt(const uint8_t *codes, const void *scal
 {
     if (transposed)
         return with_lowrank ? launch_reconstruct_ws<FMT, true>(codes, scales, g_w, U, D, N, K, W, sms, s)
-                            : launch_reconstruct_v<FMT, false, true>(codes, scales, g_w, U, D, N, K, W, sms, s);
+                            : launch_reconstruct_v<FMT, true>(codes, scales, g_w, U, N, K, W, sms, s);
     return with_lowrank ? launch_reconstruct_ws<FMT, false>(codes, scales, g_w, U, D, N, K, W, sms, s)
-                        : launch_reconstruct_v<FMT, false, false>(codes, scales, g_w, U, D, N, K, W, sms, s);
+                        : launch_reconstruct_v<FMT, false>(codes, scales, g_w, U, N, K, W, sms, s);
 }
 
 cudaError_t launch_reconstruct(int fmt, const uint8_t *codes, const void *scales, const float *g_w,

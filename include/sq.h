@@ -60,7 +60,9 @@ typedef enum {
     SQ_ERR_CUDA = 6,       /* a CUDA call or launch failed                        */
     SQ_ERR_ARG = 7,        /* bad enum / flag value                               */
     SQ_ERR_TIMEOUT = 8,    /* a kernel gave up a bounded wait (device status word) */
-    SQ_ERR_NONFINITE = 9   /* SQ_CHECK_FINITE met a NaN or an infinity (status word) */
+    SQ_ERR_NONFINITE = 9,  /* SQ_CHECK_FINITE met a NaN or an infinity (status word) */
+    SQ_ERR_INDEX = 10      /* a device-side index check failed and its access was
+                              skipped (library built with SQ_DEBUG_CHECKS; status word) */
 } sq_status;
 
 typedef enum {
@@ -126,6 +128,18 @@ SQ_API const char *sq_status_str(int status);
 
 /* ABI version, currently 1. */
 SQ_API int sq_abi_version(void);
+
+/*
+ * 1 if this library was built with SQ_DEBUG_CHECKS, else 0.  In such a build
+ * the kernels that write the layer's outputs (the activation passes, the
+ * NVFP4, int4 and int8 builders, the reconstructs) check every store's index
+ * against the size of the buffer it writes before the store; a store that
+ * would fall outside is skipped and sets bit 2 of the call's device status
+ * word (the workspace's, or the library's own for calls without one), which
+ * sq_check_device_status reports as SQ_ERR_INDEX.  Nothing traps.  The
+ * results of a debug build are the same bits as those of a release build.
+ */
+SQ_API int sq_debug_checks(void);
 
 /*
  * Text of the last failing CUDA call or device check made by this thread
@@ -387,6 +401,16 @@ SQ_API sq_status sq_set_stage_events(int32_t stage, void *start_event, void *sto
  * synchronises `stream` and copies 4 bytes to the host.
  */
 SQ_API sq_status sq_check_device_status(void *ws, void *stream);
+
+/*
+ * Self-test of the device-side index check (any build): one thread checks the
+ * index one past a bound of 256 with the same routine the SQ_DEBUG_CHECKS
+ * kernels use.  The check fails, the (never made) access is skipped and bit 2
+ * of the status word at ws is set; sq_check_device_status(ws, stream) then
+ * returns SQ_ERR_INDEX and the context stays usable.  ws: at least 256 bytes
+ * of device memory (only the first word is used), 256-byte aligned.
+ */
+SQ_API sq_status sq_selftest_index_check(void *ws, void *stream);
 
 /*
  * Self-test of the failure detection every kernel relies on: all waits in the

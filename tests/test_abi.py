@@ -40,6 +40,23 @@ def test_library_exports_every_declared_symbol():
     assert sorted(sq.EXPORTED) == header_functions()
 
 
+def test_debug_library_exports_the_same_symbols():
+    """libsq_debug.so (built with SQ_DEBUG_CHECKS) exports every declared entry point too and says
+    that it is the checked build; the release library says it is not; the index status has a name."""
+    from bit_quantized_frozen_b200 import build as b
+    dbg = b.build(debug_checks=True)
+    D = ctypes.CDLL(dbg)
+    for name in header_functions():
+        assert hasattr(D, name), name
+    D.sq_debug_checks.restype = ctypes.c_int
+    assert D.sq_debug_checks() == 1
+    assert sq.sq_debug_checks() == 0
+    assert sq.status_str(10) == "device index check failed"
+    D.sq_selftest_index_check.restype = ctypes.c_int
+    assert D.sq_selftest_index_check(None, None) == SQ_ERR_NULL
+    assert D.sq_selftest_index_check(ctypes.c_void_p(MIS), None) == SQ_ERR_ALIGN
+
+
 def test_size_helpers():
     assert sq.sq_abi_version() == 1
     assert sq.sq_sf_bytes(1, 256) == 128 * 16
@@ -218,7 +235,8 @@ static const fnptr entries[] = {
     (fnptr)sq_workspace_bytes, (fnptr)sq_build_int4, (fnptr)sq_svd_init, (fnptr)sq_build_int8,
     (fnptr)sq_build_nvfp4, (fnptr)sq_act_quant_nvfp4, (fnptr)sq_linear_fwd, (fnptr)sq_linear_fwd_noalloc,
     (fnptr)sq_reconstruct_bf16, (fnptr)sq_linear_bwd_dx, (fnptr)sq_set_gemm_events, (fnptr)sq_set_stage_events,
-    (fnptr)sq_check_device_status, (fnptr)sq_selftest_wait_timeout,
+    (fnptr)sq_check_device_status, (fnptr)sq_selftest_wait_timeout, (fnptr)sq_debug_checks,
+    (fnptr)sq_selftest_index_check,
 };
 
 int main(void)
