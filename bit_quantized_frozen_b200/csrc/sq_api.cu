@@ -155,8 +155,12 @@ constexpr size_t kHeader = 256;
 constexpr size_t kAlign = 1024;
 
 struct FwdLayout {
-    size_t a = 0, a_sf = 0, b = 0, t32 = 0, tsplit = 0, udup = 0, d32 = 0, u32 = 0, total = 0;
+    size_t a = 0, a_sf = 0, t32 = 0, tsplit = 0, udup = 0, d32 = 0, u32 = 0, ring = 0, ring_ctr = 0, total = 0;
 };
+
+// slots of the int4 / int8 GEMM's W ring: the W tiles in flight (about 74 clusters over
+// m_tiles of them each) plus room for the writers to run ahead
+constexpr int kRingSlots = 8;
 
 FwdLayout fwd_layout(int fmt, int64_t M, int64_t N, int64_t K)
 {
@@ -172,8 +176,10 @@ FwdLayout fwd_layout(int fmt, int64_t M, int64_t N, int64_t K)
         L.a = take((size_t)M * (size_t)K / 2);
         L.a_sf = take(sq_sf_bytes(M, K));
     } else {
-        L.a = take((size_t)M * (size_t)K * 2);
-        L.b = take((size_t)N * (size_t)K * 2);
+        L.a = take((size_t)M * (size_t)K * 2);    // bf16(H x)
+        // the GEMM's ring of dequantised 256-row W tiles, and its counters
+        L.ring = take((size_t)kRingSlots * 256 * (size_t)K * 2);
+        L.ring_ctr = take((size_t)2 * kRingSlots * 4);
     }
     L.t32 = take((size_t)sq::act_t_parts(M, K) * (size_t)M * 32 * 4);   // partial tiles of t
     L.tsplit = take((size_t)M * 64 * 2);
@@ -495,6 +501,8 @@ sq_status sq_linear_fwd(const sq_weight *w, const uint16_t *x, int64_t M, void *
     g.tsplit = tsplit;
     g.udup = udup;
     SQ_CUDA(cudaMemsetAsync(status, 0, 8, s), "memset");   // status word + absmax
+    if (w->fmt != SQ_FMT_NVFP4)       // the W ring's counters (before every kernel of the call)
+        SQ_CUDA(cudaMemsetAsync(ws_at(ws, L.ring_ctr), 0, (size_t)2 * kRingSlots * 4, s), "memset");
     if (flags & SQ_CHECK_FINITE)
         SQ_CUDA(sq::launch_check_finite_bf16(x, M * K, status, sms, s), "finite check");
     if (w->fmt == SQ_FMT_NVFP4) {
@@ -524,7 +532,7 @@ sq_status sq_linear_fwd(const sq_weight *w, const uint16_t *x, int64_t M, void *
                                             status, sms, s),
                 "nvfp4 act quant + low-rank operands");
         SQ_CUDA(stage_event(SQ_STAGE_ACT_QUANT, 1, s), "event record");
-        g.fp4 = 1;
+        g.mode = sq::kGemmNvfp4;
         g.a = xc;
         g.b = w->codes;
         g.sfa = xsf;
@@ -532,17 +540,9 @@ sq_status sq_linear_fwd(const sq_weight *w, const uint16_t *x, int64_t M, void *
         g.g_x = gx;
         g.g_w = w->g_w;
     } else {
+        // dequant-first: the GEMM makes bf16(q s) from the payload in shared memory
         uint16_t *xb = reinterpret_cast<uint16_t *>(ws_at(ws, L.a));
-        uint16_t *wb = reinterpret_cast<uint16_t *>(ws_at(ws, L.b));
         SQ_CUDA(sq::launch_rotate_bf16(x, M, K, xb, sms, s), "rotate x");
-        if (w->fmt == SQ_FMT_INT8_ROW)
-            SQ_CUDA(sq::launch_dequant_int8(reinterpret_cast<const int8_t *>(w->codes),
-                                            reinterpret_cast<const float *>(w->scales), N, K, wb, sms, s),
-                    "dequant");
-        else
-            SQ_CUDA(sq::launch_dequant_int4(w->codes, reinterpret_cast<const uint16_t *>(w->scales),
-                                            w->fmt == SQ_FMT_INT4_G64 ? 64 : 32, N, K, wb, sms, s),
-                    "dequant");
         if (lora) {
             const uint16_t *Dw = w->lora_down, *Uw = w->lora_up;
             if (w->fmt == SQ_FMT_INT8_ROW) {          // rank 16: zero columns 16..31
@@ -558,9 +558,15 @@ sq_status sq_linear_fwd(const sq_weight *w, const uint16_t *x, int64_t M, void *
                                               sms, s),
                     "low-rank operands");
         }
-        g.fp4 = 0;
+        g.mode = w->fmt == SQ_FMT_INT8_ROW ? sq::kGemmInt8
+                 : w->fmt == SQ_FMT_INT4_G64 ? sq::kGemmInt4G64
+                                             : sq::kGemmInt4G32;
         g.a = xb;
-        g.b = wb;
+        g.b = w->codes;
+        g.b_scales = w->scales;
+        g.wring = reinterpret_cast<uint16_t *>(ws_at(ws, L.ring));
+        g.ring_ctr = reinterpret_cast<uint32_t *>(ws_at(ws, L.ring_ctr));
+        g.ring_slots = kRingSlots;
     }
     SQ_CUDA(stage_event(SQ_STAGE_GEMM, 0, s), "event record");
     SQ_CUDA(sq::launch_gemm(g, sms, s), "gemm");
@@ -667,7 +673,7 @@ sq_status sq_linear_bwd_dx(const sq_weight *w, const uint16_t *dy, int64_t M, fl
             "transposed reconstruct");
     sq::GemmLaunch g;
     memset(&g, 0, sizeof(g));
-    g.fp4 = 0;
+    g.mode = sq::kGemmBf16;
     g.a = dy;             // [M, N]: the reduction runs over N
     g.b = wt;             // [K, N]
     g.y = dx;             // [M, K]

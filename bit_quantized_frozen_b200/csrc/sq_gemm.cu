@@ -5,7 +5,12 @@
 //   NVFP4 path: A = e2m1 activation codes [M, K/2] with ue4m3 block-16 scales,
 //               B = e2m1 weight codes [N, K/2] with ue4m3 scales (tiled layout),
 //               block-scaled MMA (kind::mxf4nvf4.block16), beta = g_x * g_w.
-//   int4 path:  A = bf16(H x) [M, K], B = bf16(q s) [N, K], kind::f16, beta = 1.
+//   int4 / int8 path: A = bf16(H x) [M, K] by TMA; B = bf16(q s) by TMA from a
+//               ring of R slots of 256 rows in global memory (L2-resident),
+//               which the kernel's own dequantising warps fill from the 4- or
+//               8-bit payload, each 256-row tile of W once (not once per M
+//               tile); kind::f16, beta = 1.
+//   bf16 path:  A and B bf16 by TMA (the input gradient's GEMM).
 //   Low-rank:   Tsplit [M, 64] = [hi | lo] bf16 split of t / beta, Udup [N, 64]
 //               = [U | U]; one extra kind::f16 K-step into the same accumulator
 //               adds (t / beta) U^T, so the epilogue only scales by beta.
@@ -14,7 +19,8 @@
 // block-scaled GEMM and its epilogue; the "Residual codecs" paragraph makes the
 // int4 codec dequant-first.)
 //
-// CTA tile 128 x 256, one CTA per SM, 6 warps (+4 scale warps on the NVFP4 path):
+// CTA tile 128 x 256, one CTA per SM, 6 warps (+4 scale warps on the NVFP4 path,
+// +4 dequantising warps on the int4 / int8 paths):
 //   warps 0-3  epilogue: tcgen05.ld of their 32 accumulator lanes, scale,
 //              128B-swizzled staging in shared memory, TMA store;
 //   warp 4     TMA producer (tiles of A, B, the scale factors, the low-rank
@@ -22,7 +28,11 @@
 //   warp 5     tensor-memory allocator and the single MMA-issuing thread;
 //   warps 6-9  (NVFP4) move each MMA's ue4m3 scale factors from shared memory
 //              into tensor memory with tcgen05.st, one 32-lane sub-partition
-//              per warp, so the tensor pipe spends no cycles on copies.
+//              per warp, so the tensor pipe spends no cycles on copies;
+//              (int4 / int8) write this CTA's share of each W tile its cluster
+//              multiplies into the ring (see "W ring" below), from the start of
+//              the kernel (they read only the weight payload, not the outputs of
+//              the preceding kernels).
 // Tensor memory (512 columns): two accumulator slots at columns 0 and 64
 // that overlap in columns 64..255, and four 48-column scale-factor buffers at
 // 320..511 (NVFP4: four stages of scale factors between the scale warps and
@@ -51,7 +61,8 @@ constexpr int kSfbBytes = 2 * kSfaBytes;       // both 128-row halves of B (ever
 constexpr int kEpiWarps = 4;
 constexpr int kStagingBytes = 32 * 128;        // one warp's 32 rows x 32 fp32
 constexpr uint32_t kTmemCols = 512;
-constexpr uint32_t kAccSlot1 = 64;             // accumulator slots [0, 256) and [64, 320)
+constexpr uint32_t kAccSlot1 = 64;             // NVFP4: accumulator slots [0, 256) and [64, 320)
+constexpr uint32_t kAccSlot1Full = 256;        // bf16 / int4 / int8: slots [0, 256) and [256, 512)
 constexpr int kOverlapChunks = 6;              // 32-column chunks shared by the two slots
 constexpr uint32_t kSfCol = 320;               // ring of four scale-factor buffers, one stage (4 MMAs) each
 constexpr uint32_t kSfBufCols = 48;            // SFB for MMA k at +8k (256 rows), SFA at +32+4k (128 rows)
@@ -63,18 +74,21 @@ constexpr uint32_t kIdescBf16 = (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)
 constexpr uint32_t kIdescNvfp4 = (1u << 7) | (1u << 10) | ((uint32_t)(BN >> 3) << 17) |
                                  ((uint32_t)(BM >> 4) << 24);          // e2m1 x e2m1, ue4m3 scales
 
-template <bool FP4>
+template <int MODE>
 struct GemmCfg {
+    static constexpr bool FP4 = MODE == kGemmNvfp4;
+    static constexpr bool DQ = MODE == kGemmInt4G32 || MODE == kGemmInt4G64 || MODE == kGemmInt8;
     static constexpr int kStages = FP4 ? 5 : 6;
     static constexpr int kScaleWarps = FP4 ? 4 : 0;              // warps 6..9 fill the scale-factor buffers
-    static constexpr int kThreads = 32 * (6 + kScaleWarps);
+    static constexpr int kDqWarps = DQ ? 4 : 0;                  // warps 6..9 fill the W ring
+    static constexpr int kThreads = 32 * (6 + kScaleWarps + kDqWarps);
     static constexpr int kStageBytes = kABytes + kBBytes + (FP4 ? kSfaBytes + kSfbBytes : 0);
     static constexpr int kKPerStage = FP4 ? 256 : 64;            // K values per stage
     static constexpr int kStagingOff = kStages * kStageBytes;
     static constexpr int kBarOff = kStagingOff + kEpiWarps * 2 * kStagingBytes;
-    // full[s], empty[s], sfdata[s], acc_full[2], acc_empty, drain
-    static constexpr int kNumBars = 3 * kStages + 4;
-    static constexpr int kSmemBytes = kBarOff + 8 * kNumBars + 16 + 1024;   // + holder, flag, alignment
+    // full[s], empty[s], sfdata[s], acc_full[2], acc_empty[2], drain
+    static constexpr int kNumBars = 3 * kStages + 5;
+    static constexpr int kSmemBytes = kBarOff + 8 * kNumBars + 16 + 1024;   // + holder, flag, verdict, alignment
 };
 
 struct GemmArgs {
@@ -82,6 +96,12 @@ struct GemmArgs {
     const uint8_t *sfb;      // NVFP4: tiled weight scales
     const float *g_x;        // NVFP4: activation global scale (device)
     const float *g_w;        // NVFP4: weight global scale (device)
+    const uint8_t *bq;       // int4 / int8: weight codes ([N, K/2] or [N, K])
+    const void *bscale;      // int4: fp16 group scales [N, K/G]; int8: fp32 row scales [N]
+    uint16_t *wring;         // int4 / int8: W ring, [ring_slots * 256, K] bf16
+    uint32_t *ring_ready;    // [ring_slots] shares written (2 per tile: both CTAs), zero at launch
+    uint32_t *ring_done;     // [ring_slots] tiles whose B loads have all landed, zero at launch
+    int ring_slots;
     uint32_t *status;        // device status word
     int M, N, K;
     int lora;                // 1: add the low-rank K-step
@@ -162,13 +182,132 @@ __device__ __forceinline__ void store_chunk(const uint32_t (&r)[32], float beta,
     issue_store(staging, sb, lane, tmY, x, y);
 }
 
-template <bool FP4>
-__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(GemmCfg<FP4>::kThreads, 1)
+// ---------------------------------------------------------------------------
+// W ring (int4 / int8 paths).  Every one of the m_tiles clusters that multiply
+// W tile nt (256 rows of W) writes 1/m_tiles of its rows as bf16(q s) into slot
+// nt % R of a ring in global memory and counts its share in ring_ready[slot]
+// (release); each of them waits for all 2 m_tiles shares (acquire) before its
+// TMA loads of B from the slot, and counts the tile in ring_done[slot] once its
+// MMAs are done (its epilogue starts), which frees the slot for tile nt + R.  So W is dequantised
+// once per 256-row tile instead of once per (M tile, N tile), the GEMM's B
+// operand moves by TMA as on the bf16 path, and the ring (R x 256 x K bf16,
+// about 3 MB a slot at K = 6144) stays in L2 and in a workspace of fixed size.
+// The values are those of the stand-alone dequantisation:
+//   int4: bf16(q s), rounded once, formed in bf16x2 arithmetic from the split
+//         s = s_hi + s_lo (dq_int4x8);
+//   int8: q s is rounded to fp32 and then to bf16, as the int8 codec defines.
+// (SquareQ README, "Residual codecs": the residual codecs are dequant-first.)
+// Bit for bit the same for every finite scale.
+// ---------------------------------------------------------------------------
+// bf16x2 arithmetic, each lane rounded once (round to nearest even)
+__device__ __forceinline__ uint32_t bf2_sub(uint32_t a, uint32_t b)
+{
+    uint32_t r;
+    asm("sub.rn.bf16x2 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(b));
+    return r;
+}
+
+__device__ __forceinline__ uint32_t bf2_mul(uint32_t a, uint32_t b)
+{
+    uint32_t r;
+    asm("mul.rn.bf16x2 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(b));
+    return r;
+}
+
+__device__ __forceinline__ uint32_t bf2_fma(uint32_t a, uint32_t b, uint32_t c)
+{
+    uint32_t r;
+    asm("fma.rn.bf16x2 %0, %1, %2, %3;" : "=r"(r) : "r"(a), "r"(b), "r"(c));
+    return r;
+}
+
+// eight int4 codes (value i in nibble i) times the scale s = s_hi + s_lo -> 8 bf16
+// values, in bf16x2 arithmetic with no conversion instruction.  s_hi = bf16(s) and
+// s_lo = s - s_hi are both exact in bf16 (an fp16 scale has 11 significant bits), q
+// (the code byte placed under the exponent of 128, minus 136) is exact, q s_lo is
+// exact (at most 7 bits), and one fma forms bf16(q s_hi + q s_lo) = bf16(q s) with a
+// single rounding -- the stand-alone dequantisation's value, zero signs included.
+__device__ __forceinline__ uint4 dq_int4x8(uint32_t w, uint32_t shi2, uint32_t slo2)
+{
+    const uint32_t x = w ^ 0x88888888u;                 // q + 8 in every nibble
+    const uint32_t lo = x & 0x0F0F0F0Fu, hi = (x >> 4) & 0x0F0F0F0Fu;
+    uint32_t o[4];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+        // halves (value 2j, value 2j + 1) = bf16 128 + (q + 8): byte j of lo / hi under 0x43
+        const uint32_t v = (__byte_perm(lo, hi, (4u + j) << 8 | (uint32_t)j) & 0x00FF00FFu) | 0x43004300u;
+        const uint32_t q = bf2_sub(v, 0x43084308u);     // - 136: exact
+        o[j] = bf2_fma(q, shi2, bf2_mul(q, slo2));
+    }
+    return make_uint4(o[0], o[1], o[2], o[3]);
+}
+
+// four int8 codes (value i in byte i) times the fp32 scale pair s2 -> 4 bf16 values (2 words)
+__device__ __forceinline__ void dq_int8x4(uint32_t w, uint64_t s2, uint32_t &o0, uint32_t &o1)
+{
+    const uint32_t x = w ^ 0x80808080u;                 // q + 128 in every byte, under 2^23
+    const uint64_t off = f2_pack(8388736.0f, 8388736.0f);
+    const uint64_t a01 = f2_pack(__uint_as_float(__byte_perm(x, 0x4B000000u, 0x7650u)),
+                                 __uint_as_float(__byte_perm(x, 0x4B000000u, 0x7651u)));
+    const uint64_t a23 = f2_pack(__uint_as_float(__byte_perm(x, 0x4B000000u, 0x7652u)),
+                                 __uint_as_float(__byte_perm(x, 0x4B000000u, 0x7653u)));
+    float p0, p1, p2, p3;
+    f2_unpack(f2_mul(f2_sub(a01, off), s2), p0, p1);
+    f2_unpack(f2_mul(f2_sub(a23, off), s2), p2, p3);
+    o0 = f32x2_to_bf16x2_bits(p0, p1);
+    o1 = f32x2_to_bf16x2_bits(p2, p3);
+}
+
+// the payload of the 8 values 8 kc .. 8 kc + 7 of row n of W, and bf16(q s) of them
+struct DqRaw {
+    uint32_t c0, c1;         // int4: 8 codes in c0; int8: 8 codes in c0, c1
+    uint32_t s;              // int4: fp16 scale bits; int8: fp32 scale bits
+};
+
+template <int MODE>
+__device__ __forceinline__ DqRaw dq_load(const GemmArgs &a, int n, int kc)
+{
+    DqRaw d;
+    if (MODE == kGemmInt8) {
+        const uint2 c = __ldg(reinterpret_cast<const uint2 *>(a.bq + (int64_t)n * a.K) + kc);
+        d.c0 = c.x;
+        d.c1 = c.y;
+        d.s = __ldg(reinterpret_cast<const uint32_t *>(a.bscale) + n);
+    } else {
+        constexpr int gs = MODE == kGemmInt4G32 ? 32 : 64;
+        d.c0 = __ldg(reinterpret_cast<const uint32_t *>(a.bq + (int64_t)n * (a.K / 2)) + kc);
+        d.c1 = 0u;
+        d.s = __ldg(reinterpret_cast<const uint16_t *>(a.bscale) + (int64_t)n * (a.K / gs) + (8 * kc) / gs);
+    }
+    return d;
+}
+
+template <int MODE>
+__device__ __forceinline__ uint4 dq_convert(const DqRaw &d)
+{
+    if (MODE == kGemmInt8) {
+        const float sf = __uint_as_float(d.s);
+        const uint64_t s2 = f2_pack(sf, sf);
+        uint4 o;
+        dq_int8x4(d.c0, s2, o.x, o.y);
+        dq_int8x4(d.c1, s2, o.z, o.w);
+        return o;
+    }
+    const float sf = __half2float(__ushort_as_half((uint16_t)d.s));
+    const uint32_t shi = __bfloat16_as_ushort(__float2bfloat16_rn(sf));
+    const uint32_t slo = __bfloat16_as_ushort(__float2bfloat16_rn(__fsub_rn(sf, __uint_as_float(shi << 16))));
+    return dq_int4x8(d.c0, shi | (shi << 16), slo | (slo << 16));
+}
+
+template <int MODE>
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(GemmCfg<MODE>::kThreads, 1)
     sq_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                    const __grid_constant__ CUtensorMap tmT, const __grid_constant__ CUtensorMap tmU,
                    const __grid_constant__ CUtensorMap tmY, const GemmArgs args)
 {
-    using Cfg = GemmCfg<FP4>;
+    using Cfg = GemmCfg<MODE>;
+    constexpr bool FP4 = Cfg::FP4;
+    constexpr bool DQ = Cfg::DQ;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint64_t *bars = reinterpret_cast<uint64_t *>(smem + Cfg::kBarOff);
@@ -176,8 +315,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(GemmCfg<FP4>::kThrea
     const uint32_t bar_empty = bar_full + 8 * Cfg::kStages;            // each CTA: its stage may be refilled
     const uint32_t bar_sfdata = bar_empty + 8 * Cfg::kStages;          // each CTA: its scale tiles landed
     const uint32_t bar_acc_full = bar_sfdata + 8 * Cfg::kStages;       // each CTA: accumulator ready
-    const uint32_t bar_acc_empty = bar_acc_full + 16;                  // leader: overlap drained in both CTAs
-    const uint32_t bar_drain = bar_acc_empty + 8;                      // leader: every MMA finished
+    // leader: (NVFP4) the overlap drained in both CTAs / (else) slot s drained in both CTAs
+    const uint32_t bar_acc_empty = bar_acc_full + 16;
+    const uint32_t bar_drain = bar_acc_empty + 16;                     // leader: every MMA finished
     uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(bars + Cfg::kNumBars);
     volatile uint32_t *abort_flag = tmem_holder + 1;
 
@@ -188,7 +328,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(GemmCfg<FP4>::kThrea
 
     if (threadIdx.x == 0) {
         for (int st = 0; st < Cfg::kStages; ++st) {
-            // leader's expect_tx (both CTAs' bytes) + every scale warp of both CTAs
+            // leader's expect_tx (both CTAs' bytes) + every scale or dequantising warp of both CTAs
             mbar_init(bar_full + 8 * st, 1 + 2 * Cfg::kScaleWarps);
             mbar_init(bar_empty + 8 * st, 1 + Cfg::kScaleWarps);        // MMA commit + scale warps
             mbar_init(bar_sfdata + 8 * st, 1);
@@ -196,6 +336,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(GemmCfg<FP4>::kThrea
         mbar_init(bar_acc_full, 1);
         mbar_init(bar_acc_full + 8, 1);
         mbar_init(bar_acc_empty, 2 * kEpiWarps);
+        mbar_init(bar_acc_empty + 8, 2 * kEpiWarps);
         mbar_init(bar_drain, 1);
         *abort_flag = 0u;
         fence_mbar_init();
@@ -215,7 +356,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(GemmCfg<FP4>::kThrea
     cluster_sync();                               // barriers of both CTAs initialised, TMEM allocated
     tc_fence_after();
     const uint32_t tmem_base = *tmem_holder;
-    grid_dep_wait();                              // operands written by the preceding kernels are visible
+    // operands written by the preceding kernels are visible after this; the W ring
+    // writers read only the weight payload and start at once
+    if (!(DQ && warp >= 6))
+        grid_dep_wait();
 
     const int m_tiles = (args.M + BM - 1) / BM;
     const int n_tiles = (args.N + BN - 1) / BN;
@@ -240,6 +384,17 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(GemmCfg<FP4>::kThrea
                 const int nh = nt * BN + (int)rank * 128;                 // this CTA's half of B
                 const bool sfa_ok = m0 < m_rows_pad;
                 const bool sfb_hi = (nt * BN + 128) < args.N;
+                // int4 / int8: this CTA's half of W tile nt sits in ring slot nt % R once all
+                // 2 * m_tiles shares of this use of the slot are written
+                const int ring_row = DQ ? (nt % args.ring_slots) * BN + (int)rank * 128 : 0;
+                if (DQ) {
+                    const uint32_t need = (uint32_t)(nt / args.ring_slots + 1) * (uint32_t)m_tiles * 2u;
+                    if (!gwait_geq(args.ring_ready + nt % args.ring_slots, need, abort_flag, args.status)) {
+                        ok = false;
+                        break;
+                    }
+                    fence_proxy_async_global();                // the TMA reads below see those stores
+                }
                 for (int ks = 0; ks < stages_per_tile; ++ks) {
                     if (!mbar_wait(bar_empty + 8 * stage, phase ^ 1u, abort_flag, args.status)) {
                         ok = false;
@@ -278,7 +433,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(GemmCfg<FP4>::kThrea
                                           kSfaBytes, sd);
                         } else {
                             tma_load_2d_pair(sA, &tmA, kk * 64, m0, fb);
-                            tma_load_2d_pair(sB, &tmB, kk * 64, nh, fb);
+                            tma_load_2d_pair(sB, &tmB, kk * 64, DQ ? ring_row : nh, fb);
                         }
                     }
                     if (++stage == Cfg::kStages) {
@@ -315,10 +470,16 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(GemmCfg<FP4>::kThrea
             uint32_t sf = tmem_base + kSfCol;
             bool ok = true;
             for (int tile = cluster_id; tile < tiles && ok; tile += clusters, ++count) {
-                const uint32_t acc = tmem_base + ((count & 1) ? kAccSlot1 : 0u);
-                if (count > 0 &&
-                    !mbar_wait_cluster(bar_acc_empty, (uint32_t)((count - 1) & 1), abort_flag, args.status))
-                    break;
+                const uint32_t acc = tmem_base + ((count & 1) ? (FP4 ? kAccSlot1 : kAccSlot1Full) : 0u);
+                if (FP4) {        // the overlap of the previous tile's slot has been drained
+                    if (count > 0 &&
+                        !mbar_wait_cluster(bar_acc_empty, (uint32_t)((count - 1) & 1), abort_flag, args.status))
+                        break;
+                } else {          // tile count - 2 (same slot) has left tensor memory
+                    if (count >= 2 && !mbar_wait_cluster(bar_acc_empty + 8 * (count & 1),
+                                                         (uint32_t)(((count >> 1) - 1) & 1), abort_flag, args.status))
+                        break;
+                }
                 for (int ks = 0; ks < stages_per_tile; ++ks) {
                     if (!mbar_wait_cluster(bar_full + 8 * stage, phase, abort_flag, args.status)) {
                         ok = false;
@@ -365,7 +526,59 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(GemmCfg<FP4>::kThrea
             (void)mbar_wait(bar_drain, 0, abort_flag, args.status);
         }
         __syncwarp();
-    } else if (warp >= 6) {
+    } else if (DQ && warp >= 6) {
+        // ------------------------------------------------------------ W ring writers (int4 / int8, both CTAs)
+        // For each tile (mt, nt) of the cluster, in order: the cluster writes share mt
+        // of the m_tiles shares (rows 256 mt / m_tiles ..) of W tile nt into ring slot
+        // nt % R, this CTA one half of it, once the slot's previous tile (nt - R) has
+        // been loaded by all of its m_tiles clusters.  The writers run ahead of the
+        // cluster's own MMAs; every wait points at an earlier W tile, so the chain ends.
+        // Only thread 0 waits (bounded) and every writer thread then meets it at named
+        // barrier 1, so the four warps always take the same way out.
+        constexpr int kBatch = 8;                                   // loads in flight per thread
+        const int tid = threadIdx.x - 6 * 32;                      // 0..127
+        const int R = args.ring_slots;
+        const int kc8 = args.K / 8;                                 // 8-value chunks per row
+        volatile uint32_t *verdict = tmem_holder + 2;
+        for (int tile = cluster_id; tile < tiles; tile += clusters) {
+            const int mt = tile % m_tiles, nt = tile / m_tiles;
+            const int slot = nt % R;
+            const int lo = (BN * mt) / m_tiles, hi = (BN * (mt + 1)) / m_tiles;
+            const int mid = lo + (hi - lo) / 2;
+            const int r0 = rank ? mid : lo, r1 = rank ? hi : mid;
+            if (tid == 0)
+                *verdict = gwait_geq(args.ring_done + slot, (uint32_t)(nt / R) * (uint32_t)m_tiles, abort_flag,
+                                     args.status)
+                               ? 1u
+                               : 0u;
+            named_barrier_sync(1, 128);
+            if (*verdict == 0u)
+                break;
+            const int total = (r1 - r0) * kc8;
+            for (int c0 = tid; c0 < total; c0 += kBatch * 128) {
+                DqRaw raw[kBatch];
+#pragma unroll
+                for (int u = 0; u < kBatch; ++u) {
+                    const int c = c0 + 128 * u;
+                    const int rr = r0 + c / kc8, n = nt * BN + rr;
+                    if (c < total && n < args.N)
+                        raw[u] = dq_load<MODE>(args, n, c - (rr - r0) * kc8);
+                }
+#pragma unroll
+                for (int u = 0; u < kBatch; ++u) {
+                    const int c = c0 + 128 * u;
+                    const int rr = r0 + c / kc8, n = nt * BN + rr;
+                    if (c < total)
+                        reinterpret_cast<uint4 *>(args.wring + ((int64_t)slot * BN + rr) * args.K)[c - (rr - r0) * kc8] =
+                            n < args.N ? dq_convert<MODE>(raw[u]) : make_uint4(0u, 0u, 0u, 0u);
+                }
+            }
+            fence_proxy_async_global();                             // for the TMA loads of other SMs
+            named_barrier_sync(1, 128);                             // the four writer warps are done
+            if (tid == 0)
+                red_release_gpu_add(args.ring_ready + slot, 1u);
+        }
+    } else if (FP4 && warp >= 6) {
         // ------------------------------------------------------------ scale warps (NVFP4, both CTAs)
         // Warp w owns tensor-memory lanes 32*(w%4)..+31 of its CTA.  For stage g it
         // copies line `lane` of the four SFA chunks (this CTA's rows 32*j + lane) into 4
@@ -450,6 +663,46 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(GemmCfg<FP4>::kThrea
         const bool ybf = args.out_bf16 != 0;
         uint8_t *staging = smem + Cfg::kStagingOff + warp * 2 * kStagingBytes;
         int count = 0;
+        if constexpr (!FP4) {
+            // Disjoint slots: the MMAs of the next tile run in the other slot, so this
+            // one drains at leisure, chunk by chunk (the load of chunk q + 1 overlaps
+            // the staging and store of chunk q), and is released once all of it has
+            // left tensor memory -- in time for the tile after next.
+            for (int tile = cluster_id; tile < tiles; tile += clusters, ++count) {
+                const int mt = tile % m_tiles, nt = tile / m_tiles;
+                const int m0 = mt * BM + (int)rank * kRowsPerCta;
+                const int n0 = nt * BN;
+                const int slot = count & 1;
+                if (!warp_wait(bar_acc_full + 8 * slot, (uint32_t)((count >> 1) & 1), abort_flag, args.status,
+                               lane))
+                    break;
+                if (DQ && leader && warp == 0 && lane == 0)   // the tile's MMAs are done with its W
+                    red_release_gpu_add(args.ring_done + nt % args.ring_slots, 1u);
+                tc_fence_after();
+                const uint32_t acc = tmem_base + ((uint32_t)(32 * warp) << 16) + (slot ? kAccSlot1Full : 0u);
+                const bool rows_live = m0 + 32 * warp < args.M;   // skip stores wholly below the matrix
+                const int ytop = m0 + 32 * warp;
+                uint32_t ra[32], rb[32];
+                tmem_ld_32cols(acc, ra);
+                tmem_wait_ld();
+#pragma unroll
+                for (int q = 0; q < 8; q += 2) {
+                    tmem_ld_32cols(acc + 32 * (q + 1), rb);
+                    if (rows_live)
+                        store_chunk(ra, beta, staging, 0, lane, &tmY, n0 + 32 * q, ytop, ybf);
+                    tmem_wait_ld();
+                    if (q + 2 < 8)
+                        tmem_ld_32cols(acc + 32 * (q + 2), ra);
+                    if (rows_live)
+                        store_chunk(rb, beta, staging, 1, lane, &tmY, n0 + 32 * (q + 1), ytop, ybf);
+                    tmem_wait_ld();
+                }
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0)
+                    mbar_arrive_cluster(acc_empty_leader + 8 * slot);
+            }
+        } else
         for (int tile = cluster_id; tile < tiles; tile += clusters, ++count) {
             const int mt = tile % m_tiles, nt = tile / m_tiles;
             const int m0 = mt * BM + (int)rank * kRowsPerCta;
@@ -549,10 +802,62 @@ bool make_tmap(CUtensorMap *m, CUtensorMapDataType dt, int esize, const void *ba
     return r == CUDA_SUCCESS;
 }
 
+// persistent grid: as many CTA pairs as can be resident at once (not every SM
+// can pair up inside its GPC), each walking the tile list.  The shared-memory
+// opt-in and the occupancy query run once per CUDA context and kernel (a new
+// context loads the device code again, without the attribute).
+template <int MODE>
+static cudaError_t launch_mode(const CUtensorMap &tA, const CUtensorMap &tB, const CUtensorMap &tT,
+                               const CUtensorMap &tU, const CUtensorMap &tY, const GemmArgs &a, int tiles, int sms,
+                               cudaStream_t stream)
+{
+    using Cfg = GemmCfg<MODE>;
+    constexpr int kMaxDev = 64;
+    static unsigned long long ctx_seen[kMaxDev];
+    static int resident_pairs[kMaxDev];
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDev)
+        return cudaErrorInvalidDevice;
+    const unsigned long long ctx = current_context_id();
+    if (ctx == 0 || ctx_seen[dev] != ctx) {
+        cudaError_t e =
+            cudaFuncSetAttribute(sq_gemm_kernel<MODE>, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::kSmemBytes);
+        if (e != cudaSuccess)
+            return e;
+        cudaLaunchConfig_t q = {};
+        q.gridDim = dim3(2 * (sms / 2));
+        q.blockDim = dim3(Cfg::kThreads);
+        q.dynamicSmemBytes = Cfg::kSmemBytes;
+        int resident = 0;
+        e = cudaOccupancyMaxActiveClusters(&resident, sq_gemm_kernel<MODE>, &q);
+        (void)cudaGetLastError();
+        resident_pairs[dev] = (e == cudaSuccess && resident > 0 && resident < sms / 2) ? resident : sms / 2;
+        ctx_seen[dev] = ctx;
+    }
+    const int pairs = resident_pairs[dev];
+    const int grid = 2 * (tiles < pairs ? tiles : pairs);        // clusters of two CTAs
+    // dependent launch: the set-up (barriers, tensor memory, descriptor prefetch) overlaps
+    // the end of the preceding kernel; the kernel waits for its results before loading
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)grid);
+    cfg.blockDim = dim3(Cfg::kThreads);
+    cfg.dynamicSmemBytes = Cfg::kSmemBytes;
+    cfg.stream = stream;
+    cudaLaunchAttribute at[1];
+    at[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    at[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = at;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, sq_gemm_kernel<MODE>, tA, tB, tT, tU, tY, a);
+}
+
 cudaError_t launch_gemm(const GemmLaunch &g, int sms, cudaStream_t stream)
 {
     CUtensorMap tA, tB, tT, tU, tY;
-    const bool fp4 = g.fp4 != 0;
+    const bool fp4 = g.mode == kGemmNvfp4;
+    const bool dq = g.mode == kGemmInt4G32 || g.mode == kGemmInt4G64 || g.mode == kGemmInt8;
+    if (!fp4 && !dq && g.mode != kGemmBf16)
+        return cudaErrorInvalidValue;
     bool ok = true;
     if (fp4) {
         ok &= make_tmap(&tA, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, g.a, (uint64_t)g.K / 2, (uint64_t)g.M, 128, 128,
@@ -562,15 +867,18 @@ cudaError_t launch_gemm(const GemmLaunch &g, int sms, cudaStream_t stream)
     } else {
         ok &= make_tmap(&tA, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, g.a, (uint64_t)g.K, (uint64_t)g.M, 64, 128,
                         CU_TENSOR_MAP_SWIZZLE_128B);
-        ok &= make_tmap(&tB, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, g.b, (uint64_t)g.K, (uint64_t)g.N, 64, 128,
-                        CU_TENSOR_MAP_SWIZZLE_128B);
+        // (int4 / int8: B comes from the W ring)
+        if (dq && (!g.wring || !g.ring_ctr || g.ring_slots < 1))
+            return cudaErrorInvalidValue;
+        ok &= make_tmap(&tB, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, dq ? (const void *)g.wring : g.b, (uint64_t)g.K,
+                        dq ? (uint64_t)g.ring_slots * BN : (uint64_t)g.N, 64, 128, CU_TENSOR_MAP_SWIZZLE_128B);
     }
     const bool lora = g.tsplit && g.udup;
     // without a low-rank step the maps below are never used; point them at A/B
     ok &= make_tmap(&tT, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, lora ? (const void *)g.tsplit : g.a, 64,
                     (uint64_t)g.M, 64, 128, CU_TENSOR_MAP_SWIZZLE_128B);
-    ok &= make_tmap(&tU, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, lora ? (const void *)g.udup : g.b, 64,
-                    (uint64_t)g.N, 64, 128, CU_TENSOR_MAP_SWIZZLE_128B);
+    ok &= make_tmap(&tU, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, lora ? (const void *)g.udup : g.a, 64,
+                    lora ? (uint64_t)g.N : (uint64_t)g.M, 64, 128, CU_TENSOR_MAP_SWIZZLE_128B);
     if (g.out_bf16)
         ok &= make_tmap(&tY, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, g.y, (uint64_t)g.N, (uint64_t)g.M, 32, 32,
                         CU_TENSOR_MAP_SWIZZLE_64B);
@@ -584,6 +892,12 @@ cudaError_t launch_gemm(const GemmLaunch &g, int sms, cudaStream_t stream)
     a.sfb = g.sfb;
     a.g_x = g.g_x;
     a.g_w = g.g_w;
+    a.bq = dq ? reinterpret_cast<const uint8_t *>(g.b) : nullptr;
+    a.bscale = dq ? g.b_scales : nullptr;
+    a.wring = dq ? g.wring : nullptr;
+    a.ring_ready = dq ? g.ring_ctr : nullptr;
+    a.ring_done = dq ? g.ring_ctr + g.ring_slots : nullptr;
+    a.ring_slots = dq ? g.ring_slots : 1;
     a.status = g.status;
     a.M = (int)g.M;
     a.N = (int)g.N;
@@ -591,49 +905,18 @@ cudaError_t launch_gemm(const GemmLaunch &g, int sms, cudaStream_t stream)
     a.lora = lora ? 1 : 0;
     a.out_bf16 = g.out_bf16 ? 1 : 0;
     const int tiles = (int)(((g.M + BM - 1) / BM) * ((g.N + BN - 1) / BN));
-    // persistent grid: as many CTA pairs as can be resident at once (not every SM
-    // can pair up inside its GPC), each walking the tile list; queried once per
-    // device and kernel, together with the shared-memory opt-in
-    constexpr int kMaxDev = 64;
-    static int resident_pairs[2][kMaxDev];
-    int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDev)
-        return cudaErrorInvalidDevice;
-    int &pairs_cached = resident_pairs[fp4 ? 1 : 0][dev];
-    if (pairs_cached == 0) {
-        cudaLaunchConfig_t cfg = {};
-        cfg.gridDim = dim3(2 * (sms / 2));
-        cfg.blockDim = dim3(fp4 ? GemmCfg<true>::kThreads : GemmCfg<false>::kThreads);
-        cfg.dynamicSmemBytes = fp4 ? GemmCfg<true>::kSmemBytes : GemmCfg<false>::kSmemBytes;
-        int resident = 0;
-        cudaError_t e = fp4 ? cudaFuncSetAttribute(sq_gemm_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                                   GemmCfg<true>::kSmemBytes)
-                            : cudaFuncSetAttribute(sq_gemm_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                                   GemmCfg<false>::kSmemBytes);
-        if (e != cudaSuccess)
-            return e;
-        e = fp4 ? cudaOccupancyMaxActiveClusters(&resident, sq_gemm_kernel<true>, &cfg)
-                : cudaOccupancyMaxActiveClusters(&resident, sq_gemm_kernel<false>, &cfg);
-        (void)cudaGetLastError();
-        pairs_cached = (e == cudaSuccess && resident > 0 && resident < sms / 2) ? resident : sms / 2;
+    switch (g.mode) {
+    case kGemmNvfp4:
+        return launch_mode<kGemmNvfp4>(tA, tB, tT, tU, tY, a, tiles, sms, stream);
+    case kGemmInt4G32:
+        return launch_mode<kGemmInt4G32>(tA, tB, tT, tU, tY, a, tiles, sms, stream);
+    case kGemmInt4G64:
+        return launch_mode<kGemmInt4G64>(tA, tB, tT, tU, tY, a, tiles, sms, stream);
+    case kGemmInt8:
+        return launch_mode<kGemmInt8>(tA, tB, tT, tU, tY, a, tiles, sms, stream);
+    default:
+        return launch_mode<kGemmBf16>(tA, tB, tT, tU, tY, a, tiles, sms, stream);
     }
-    const int pairs = pairs_cached;
-    const int grid = 2 * (tiles < pairs ? tiles : pairs);        // clusters of two CTAs
-    // dependent launch: the set-up (barriers, tensor memory, descriptor prefetch) overlaps
-    // the end of the preceding kernel; the kernel waits for its results before loading
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3((unsigned)grid);
-    cfg.blockDim = dim3(fp4 ? GemmCfg<true>::kThreads : GemmCfg<false>::kThreads);
-    cfg.dynamicSmemBytes = fp4 ? GemmCfg<true>::kSmemBytes : GemmCfg<false>::kSmemBytes;
-    cfg.stream = stream;
-    cudaLaunchAttribute at[1];
-    at[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-    at[0].val.programmaticStreamSerializationAllowed = 1;
-    cfg.attrs = at;
-    cfg.numAttrs = 1;
-    if (fp4)
-        return cudaLaunchKernelEx(&cfg, sq_gemm_kernel<true>, tA, tB, tT, tU, tY, a);
-    return cudaLaunchKernelEx(&cfg, sq_gemm_kernel<false>, tA, tB, tT, tU, tY, a);
 }
 
 }  // namespace sq

@@ -38,15 +38,11 @@ cudaError_t launch_nvfp4_quant_bf16(const uint16_t *in, int64_t rows, int64_t K,
                                     const LowrankOut &lr, uint32_t *status, int sms, cudaStream_t s);
 cudaError_t launch_int4_build(const float *R, int64_t N, int64_t K, int group, uint8_t *codes, uint16_t *scales,
                               uint8_t *frac, int sms, cudaStream_t s);
-// int8 per-row builder (K <= 16384), its dequant, and the rank-16 -> rank-32 widening
+// int8 per-row builder (K <= 16384) and the rank-16 -> rank-32 widening
 cudaError_t launch_int8_build(const float *R, int64_t N, int64_t K, int8_t *codes, float *scales, uint8_t *frac,
                               int sms, cudaStream_t s);
-cudaError_t launch_dequant_int8(const int8_t *codes, const float *scales, int64_t N, int64_t K, uint16_t *wb, int sms,
-                                cudaStream_t s);
 cudaError_t launch_widen_rank16(const uint16_t *src, int64_t rows, uint16_t *dst, int sms, cudaStream_t s);
 cudaError_t launch_rotate_bf16(const uint16_t *x, int64_t M, int64_t K, uint16_t *xb, int sms, cudaStream_t s);
-cudaError_t launch_dequant_int4(const uint8_t *codes, const uint16_t *scales, int group, int64_t N, int64_t K,
-                                uint16_t *wb, int sms, cudaStream_t s);
 // t_part: act_t_parts(M, K) partial tiles [parts, M, 32] (NULL: no t)
 cudaError_t launch_act_pass1(const uint16_t *x, int64_t M, int64_t K, const uint16_t *D, uint32_t *amax,
                              float *t_part, uint32_t *status, int sms, cudaStream_t s);
@@ -73,10 +69,18 @@ cudaError_t launch_svd_init(const float *W, int64_t N, int64_t K, const float *o
                             const char **stage);
 
 // forward GEMM y = beta (A B^T + tsplit udup^T), see sq_gemm.cu
+// B operand of the GEMM: bf16 by TMA, NVFP4 codes + tiled scales by TMA, or
+// int4 / int8 payload turned into bf16(q s) in shared memory by the kernel
+enum GemmMode { kGemmBf16 = 0, kGemmNvfp4 = 1, kGemmInt4G32 = 2, kGemmInt4G64 = 3, kGemmInt8 = 4 };
+
 struct GemmLaunch {
-    int fp4;                 // 1: NVFP4 codes + tiled scales, 0: bf16 operands
-    const void *a;           // [M, K/2] u8 or [M, K] bf16
-    const void *b;           // [N, K/2] u8 or [N, K] bf16
+    int mode;                // GemmMode
+    const void *a;           // [M, K/2] u8 (NVFP4) or [M, K] bf16
+    const void *b;           // [N, K/2] u8 (NVFP4, int4), [N, K] int8 or [N, K] bf16
+    const void *b_scales;    // int4: fp16 [N, K/G]; int8: fp32 [N]
+    uint16_t *wring;         // int4 / int8: W ring [ring_slots * 256, K] bf16 (workspace)
+    uint32_t *ring_ctr;      // int4 / int8: 2 * ring_slots counters, zero before the launch
+    int ring_slots;
     const uint8_t *sfa;      // NVFP4 scales of a (tiled)
     const uint8_t *sfb;      // NVFP4 scales of b (tiled)
     const float *g_x;        // NVFP4: device scalars, beta = g_x * g_w

@@ -218,6 +218,57 @@ __device__ __forceinline__ void fence_proxy_async_smem()
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
 
+// generic-proxy global stores before it are ordered with async-proxy (TMA) accesses after it
+__device__ __forceinline__ void fence_proxy_async_global()
+{
+    asm volatile("fence.proxy.async.global;" ::: "memory");
+}
+
+// gpu-scope release add / acquire load on a global counter
+__device__ __forceinline__ void red_release_gpu_add(uint32_t *p, uint32_t v)
+{
+    asm volatile("red.release.gpu.global.add.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+
+__device__ __forceinline__ uint32_t ld_acquire_gpu(const uint32_t *p)
+{
+    uint32_t v;
+    asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+    return v;
+}
+
+// named barrier among `count` threads (a multiple of 32) of the CTA
+__device__ __forceinline__ void named_barrier_sync(uint32_t id, uint32_t count)
+{
+    asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
+}
+
+// bounded wait until the global counter reaches `target` (acquire); false after
+// kWaitLimitNs or once another role of the CTA has given up
+__device__ __forceinline__ bool gwait_geq(const uint32_t *ctr, uint32_t target, volatile uint32_t *abort_flag,
+                                          uint32_t *status)
+{
+    if (ld_acquire_gpu(ctr) >= target)
+        return true;
+    const unsigned long long t0 = global_ns();
+    for (uint32_t it = 1;; ++it) {
+        __nanosleep(64);
+        if (ld_acquire_gpu(ctr) >= target)
+            return true;
+        if ((it & 63u) == 0) {
+            if (*abort_flag)
+                return false;
+            if (global_ns() - t0 > kWaitLimitNs) {
+                *abort_flag = 1u;
+                if (status)
+                    atomicOr(status, 1u);
+                return false;
+            }
+        }
+    }
+}
+
+
 __device__ __forceinline__ void prefetch_tmap(const void *tmap)
 {
     asm volatile("prefetch.tensormap [%0];" ::"l"((uint64_t)tmap) : "memory");

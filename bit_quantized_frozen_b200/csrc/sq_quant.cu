@@ -598,29 +598,6 @@ __global__ void __launch_bounds__(kI8Threads) int8_build_kernel(const float *__r
     }
 }
 
-// int8 "dequant-first": wb[n, k] = bf16(RN(q s_n)), 16 values per thread
-__global__ void __launch_bounds__(256) dequant_int8_kernel(const uint4 *__restrict__ codes,
-                                                           const float *__restrict__ scales, int64_t K,
-                                                           int64_t total16, uint4 *__restrict__ wb)
-{
-    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < total16;
-         i += (int64_t)gridDim.x * blockDim.x) {
-        const uint4 c = __ldg(codes + i);
-        const float s = __ldg(scales + (i * 16) / K);
-        const uint32_t w[4] = {c.x, c.y, c.z, c.w};
-        uint32_t o[8];
-#pragma unroll
-        for (int j = 0; j < 4; ++j) {
-            float q[4];
-            int8x4_to_f32(w[j], q);
-            o[2 * j] = f32x2_to_bf16x2_bits(__fmul_rn(q[0], s), __fmul_rn(q[1], s));
-            o[2 * j + 1] = f32x2_to_bf16x2_bits(__fmul_rn(q[2], s), __fmul_rn(q[3], s));
-        }
-        wb[2 * i] = make_uint4(o[0], o[1], o[2], o[3]);
-        wb[2 * i + 1] = make_uint4(o[4], o[5], o[6], o[7]);
-    }
-}
-
 // rank-16 low-rank factors widened to rank 32 with zero columns 16..31, so the
 // rank-32 forward machinery (t = x lora_down, the low-rank MMA step) adds
 // exactly the rank-16 term: src [rows, 16] bf16 -> dst [rows, 32] bf16
@@ -655,29 +632,6 @@ __global__ void __launch_bounds__(kStreamThreads) rotate_bf16_kernel(const __gri
             o[i] = make_uint4(w[0], w[1], w[2], w[3]);
         }
     });
-}
-
-// ---------------------------------------------------------------------------
-// int4 "dequant-first": wb[n, k] = bf16(q s), 8 values per thread, group G
-// ---------------------------------------------------------------------------
-template <int G>
-__global__ void __launch_bounds__(256) dequant_int4_kernel(const uint32_t *__restrict__ codes,
-                                                           const uint16_t *__restrict__ scales,
-                                                           int64_t total8, uint4 *__restrict__ wb)
-{
-    constexpr int kWordsLog2 = G == 64 ? 3 : 2;      // 8-value code words per group
-    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < total8;
-         i += (int64_t)gridDim.x * blockDim.x) {
-        const uint32_t c = __ldg(codes + i);
-        const float s = __half2float(__ushort_as_half(__ldg(scales + (i >> kWordsLog2))));
-        float q[8];
-        int4x8_to_f32(c, q);
-        uint32_t o[4];
-#pragma unroll
-        for (int p = 0; p < 4; ++p)
-            o[p] = f32x2_to_bf16x2_bits(__fmul_rn(q[2 * p], s), __fmul_rn(q[2 * p + 1], s));
-        wb[i] = make_uint4(o[0], o[1], o[2], o[3]);
-    }
 }
 
 // ---------------------------------------------------------------------------
@@ -1872,15 +1826,6 @@ cudaError_t launch_int8_build(const float *R, int64_t N, int64_t K, int8_t *code
     return cudaGetLastError();
 }
 
-cudaError_t launch_dequant_int8(const int8_t *codes, const float *scales, int64_t N, int64_t K, uint16_t *wb, int sms,
-                                cudaStream_t s)
-{
-    const int64_t total16 = N * K / 16;
-    dequant_int8_kernel<<<grid_for(total16, 256, sms, 8), 256, 0, s>>>(reinterpret_cast<const uint4 *>(codes), scales,
-                                                                      K, total16, reinterpret_cast<uint4 *>(wb));
-    return cudaGetLastError();
-}
-
 cudaError_t launch_widen_rank16(const uint16_t *src, int64_t rows, uint16_t *dst, int sms, cudaStream_t s)
 {
     widen_rank16_kernel<<<grid_for(rows * 4, 256, sms, 4), 256, 0, s>>>(reinterpret_cast<const uint4 *>(src), rows,
@@ -1898,19 +1843,6 @@ cudaError_t launch_rotate_bf16(const uint16_t *x, int64_t M, int64_t K, uint16_t
         return e;
     const int64_t blocks = M * (K / kHad);
     rotate_bf16_kernel<<<stream_grid(blocks, sms, 3), kStreamThreads, StreamCfg<uint16_t>::kSmem, s>>>(tm, blocks, xb);
-    return cudaGetLastError();
-}
-
-cudaError_t launch_dequant_int4(const uint8_t *codes, const uint16_t *scales, int group, int64_t N, int64_t K,
-                                uint16_t *wb, int sms, cudaStream_t s)
-{
-    const int64_t total8 = N * K / 8;
-    if (group == 64)
-        dequant_int4_kernel<64><<<grid_for(total8, 256, sms, 8), 256, 0, s>>>(
-            reinterpret_cast<const uint32_t *>(codes), scales, total8, reinterpret_cast<uint4 *>(wb));
-    else
-        dequant_int4_kernel<32><<<grid_for(total8, 256, sms, 8), 256, 0, s>>>(
-            reinterpret_cast<const uint32_t *>(codes), scales, total8, reinterpret_cast<uint4 *>(wb));
     return cudaGetLastError();
 }
 

@@ -277,7 +277,10 @@ SQ_API sq_status sq_act_quant_nvfp4(const uint16_t *x, int64_t M, int64_t K,
  *          y = g_x g_w acc + t lora_up^T.
  *   int4:  "dequant-first": xb = bf16(H x), wb = bf16(q s), y = xb wb^T +
  *          t lora_up^T on bf16 tensor cores (fp32 accumulation); either
- *          group size (SQ_FMT_INT4_G32 / _G64).
+ *          group size (SQ_FMT_INT4_G32 / _G64).  wb is never stored whole:
+ *          the GEMM's own warps dequantise each 256-row tile of W once into
+ *          a ring of 8 such tiles in the workspace (8 x 256 x K bf16), from
+ *          which the GEMM loads it, so the workspace does not grow with N.
  *   int8:  the same with wb = bf16(RN(q s_row)) and the rank-16 branch
  *          (SQ_FMT_INT8_ROW; workspace op SQ_OP_LINEAR_FWD_INT8).
  * The low-rank term is accumulated on the tensor cores in the same
@@ -310,9 +313,9 @@ SQ_API sq_status sq_linear_fwd(const sq_weight *w, const uint16_t *x, int64_t M,
  * Limit: sq_workspace_bytes(SQ_OP_LINEAR_FWD_NVFP4 or _INT4, M, N, K) must
  * be at most 33554432 (32 MiB); larger shapes return SQ_ERR_WORKSPACE before
  * any work, with the sizes in sq_last_error_detail().  (NVFP4 at N = 16384,
- * K = 6144 fits M up to 8191 rows; the int4 forward, which keeps a bf16 copy
- * of W in the workspace, fits N x K up to about 16 M values, e.g. M = 1536
- * at N = K = 3072.)
+ * K = 6144 fits M up to 8191 rows; the int4 forward, which needs bf16(H x)
+ * (M K 2 bytes) and its W ring (8 x 256 x K x 2 bytes), fits for example
+ * M = 1536 at N = K = 3072.)
  *
  * The first call on each device looks up the scratch's address
  * (cudaGetSymbolAddress, with that device current), which may load libsq's
