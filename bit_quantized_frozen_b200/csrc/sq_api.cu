@@ -14,7 +14,7 @@
 #include "sq_kernels.h"
 #include "sq_ptx.cuh"
 
-static __device__ __align__(256) uint8_t g_noalloc_scratch[size_t(32) << 20];
+static __device__ __align__(256) uint8_t g_noalloc_scratch[size_t(96) << 20];
 
 namespace sq {
 typedef CUresult (*PFN_ctxGetCurrent)(CUcontext *);
@@ -207,7 +207,7 @@ uint8_t *ws_at(void *ws, size_t off)
     } while (0)
 
 // Static scratch of sq_linear_fwd_noalloc --------------------------------------
-// A fixed 32 MiB forward workspace that lives in the module's own device
+// A fixed 96 MiB forward workspace that lives in the module's own device
 // memory (one copy per device, created when the module's device code is
 // loaded into a context, released with the context), so that the call needs
 // no allocation.  Its device address is looked up with the device current,
@@ -216,7 +216,7 @@ uint8_t *ws_at(void *ws, size_t off)
 // context has another ID (after cudaDeviceReset, or once the primary context
 // was released and created again, the module is loaded anew and the array may
 // sit elsewhere).
-constexpr size_t kNoAllocScratchBytes = size_t(32) << 20;
+constexpr size_t kNoAllocScratchBytes = size_t(96) << 20;
 struct ScratchSlot {
     void *ptr = nullptr;
     unsigned long long ctx = 0;

@@ -258,9 +258,10 @@ __device__ __forceinline__ void dq_int8x4(uint32_t w, uint64_t s2, uint32_t &o0,
     o1 = f32x2_to_bf16x2_bits(p2, p3);
 }
 
-// the payload of the 8 values 8 kc .. 8 kc + 7 of row n of W, and bf16(q s) of them
+// the payload of the 32 values 32 kc .. 32 kc + 31 of row n of W (one group-32 scale,
+// one 16-byte load for int4; two for int8), and bf16(q s) of them (64 bytes)
 struct DqRaw {
-    uint32_t c0, c1;         // int4: 8 codes in c0; int8: 8 codes in c0, c1
+    uint4 c0, c1;            // int4: 32 codes in c0; int8: 32 codes in c0, c1
     uint32_t s;              // int4: fp16 scale bits; int8: fp32 scale bits
 };
 
@@ -269,34 +270,43 @@ __device__ __forceinline__ DqRaw dq_load(const GemmArgs &a, int n, int kc)
 {
     DqRaw d;
     if (MODE == kGemmInt8) {
-        const uint2 c = __ldg(reinterpret_cast<const uint2 *>(a.bq + (int64_t)n * a.K) + kc);
-        d.c0 = c.x;
-        d.c1 = c.y;
+        const uint4 *p = reinterpret_cast<const uint4 *>(a.bq + (int64_t)n * a.K) + 2 * kc;
+        d.c0 = __ldg(p);
+        d.c1 = __ldg(p + 1);
         d.s = __ldg(reinterpret_cast<const uint32_t *>(a.bscale) + n);
     } else {
         constexpr int gs = MODE == kGemmInt4G32 ? 32 : 64;
-        d.c0 = __ldg(reinterpret_cast<const uint32_t *>(a.bq + (int64_t)n * (a.K / 2)) + kc);
-        d.c1 = 0u;
-        d.s = __ldg(reinterpret_cast<const uint16_t *>(a.bscale) + (int64_t)n * (a.K / gs) + (8 * kc) / gs);
+        d.c0 = __ldg(reinterpret_cast<const uint4 *>(a.bq + (int64_t)n * (a.K / 2)) + kc);
+        d.c1 = make_uint4(0u, 0u, 0u, 0u);
+        d.s = __ldg(reinterpret_cast<const uint16_t *>(a.bscale) + (int64_t)n * (a.K / gs) + (32 * kc) / gs);
     }
     return d;
 }
 
 template <int MODE>
-__device__ __forceinline__ uint4 dq_convert(const DqRaw &d)
+__device__ __forceinline__ void dq_convert_store(const DqRaw &d, uint4 *dst)
 {
     if (MODE == kGemmInt8) {
         const float sf = __uint_as_float(d.s);
         const uint64_t s2 = f2_pack(sf, sf);
-        uint4 o;
-        dq_int8x4(d.c0, s2, o.x, o.y);
-        dq_int8x4(d.c1, s2, o.z, o.w);
-        return o;
+        const uint32_t w[8] = {d.c0.x, d.c0.y, d.c0.z, d.c0.w, d.c1.x, d.c1.y, d.c1.z, d.c1.w};
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            uint4 o;
+            dq_int8x4(w[2 * j], s2, o.x, o.y);
+            dq_int8x4(w[2 * j + 1], s2, o.z, o.w);
+            dst[j] = o;
+        }
+        return;
     }
     const float sf = __half2float(__ushort_as_half((uint16_t)d.s));
     const uint32_t shi = __bfloat16_as_ushort(__float2bfloat16_rn(sf));
     const uint32_t slo = __bfloat16_as_ushort(__float2bfloat16_rn(__fsub_rn(sf, __uint_as_float(shi << 16))));
-    return dq_int4x8(d.c0, shi | (shi << 16), slo | (slo << 16));
+    const uint32_t shi2 = shi | (shi << 16), slo2 = slo | (slo << 16);
+    const uint32_t w[4] = {d.c0.x, d.c0.y, d.c0.z, d.c0.w};
+#pragma unroll
+    for (int j = 0; j < 4; ++j)
+        dst[j] = dq_int4x8(w[j], shi2, slo2);
 }
 
 template <int MODE>
@@ -378,6 +388,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(GemmCfg<MODE>::kThre
             int stage = 0;
             uint32_t phase = 0;
             bool ok = true;
+            bool next_ready = false;                                      // (int4 / int8) probed early
             for (int tile = cluster_id; tile < tiles && ok; tile += clusters) {
                 const int mt = tile % m_tiles, nt = tile / m_tiles;
                 const int m0 = mt * BM + (int)rank * kRowsPerCta;         // this CTA's rows of A / y
@@ -389,10 +400,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(GemmCfg<MODE>::kThre
                 const int ring_row = DQ ? (nt % args.ring_slots) * BN + (int)rank * 128 : 0;
                 if (DQ) {
                     const uint32_t need = (uint32_t)(nt / args.ring_slots + 1) * (uint32_t)m_tiles * 2u;
-                    if (!gwait_geq(args.ring_ready + nt % args.ring_slots, need, abort_flag, args.status)) {
+                    if (!next_ready &&
+                        !gwait_geq(args.ring_ready + nt % args.ring_slots, need, abort_flag, args.status)) {
                         ok = false;
                         break;
                     }
+                    next_ready = false;
                     fence_proxy_async_global();                // the TMA reads below see those stores
                 }
                 for (int ks = 0; ks < stages_per_tile; ++ks) {
@@ -435,6 +448,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(GemmCfg<MODE>::kThre
                             tma_load_2d_pair(sA, &tmA, kk * 64, m0, fb);
                             tma_load_2d_pair(sB, &tmB, kk * 64, DQ ? ring_row : nh, fb);
                         }
+                    }
+                    if (DQ && ks == stages_per_tile / 2) {     // one acquire probe for the next tile,
+                        const int nn = (tile + clusters) / m_tiles;   // so its start rarely waits
+                        next_ready = tile + clusters < tiles &&
+                                     ld_acquire_gpu(args.ring_ready + nn % args.ring_slots) >=
+                                         (uint32_t)(nn / args.ring_slots + 1) * (uint32_t)m_tiles * 2u;
                     }
                     if (++stage == Cfg::kStages) {
                         stage = 0;
@@ -535,10 +554,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(GemmCfg<MODE>::kThre
         // cluster's own MMAs; every wait points at an earlier W tile, so the chain ends.
         // Only thread 0 waits (bounded) and every writer thread then meets it at named
         // barrier 1, so the four warps always take the same way out.
-        constexpr int kBatch = 8;                                   // loads in flight per thread
+        constexpr int kBatch = 4;                                   // 32-value chunks in flight per thread
         const int tid = threadIdx.x - 6 * 32;                      // 0..127
         const int R = args.ring_slots;
-        const int kc8 = args.K / 8;                                 // 8-value chunks per row
+        const int kc32 = args.K / 32;                               // 32-value chunks per row
         volatile uint32_t *verdict = tmem_holder + 2;
         for (int tile = cluster_id; tile < tiles; tile += clusters) {
             const int mt = tile % m_tiles, nt = tile / m_tiles;
@@ -554,23 +573,31 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(GemmCfg<MODE>::kThre
             named_barrier_sync(1, 128);
             if (*verdict == 0u)
                 break;
-            const int total = (r1 - r0) * kc8;
+            const int total = (r1 - r0) * kc32;
             for (int c0 = tid; c0 < total; c0 += kBatch * 128) {
                 DqRaw raw[kBatch];
 #pragma unroll
                 for (int u = 0; u < kBatch; ++u) {
                     const int c = c0 + 128 * u;
-                    const int rr = r0 + c / kc8, n = nt * BN + rr;
+                    const int rr = r0 + c / kc32, n = nt * BN + rr;
                     if (c < total && n < args.N)
-                        raw[u] = dq_load<MODE>(args, n, c - (rr - r0) * kc8);
+                        raw[u] = dq_load<MODE>(args, n, c - (rr - r0) * kc32);
                 }
 #pragma unroll
                 for (int u = 0; u < kBatch; ++u) {
                     const int c = c0 + 128 * u;
-                    const int rr = r0 + c / kc8, n = nt * BN + rr;
-                    if (c < total)
-                        reinterpret_cast<uint4 *>(args.wring + ((int64_t)slot * BN + rr) * args.K)[c - (rr - r0) * kc8] =
-                            n < args.N ? dq_convert<MODE>(raw[u]) : make_uint4(0u, 0u, 0u, 0u);
+                    const int rr = r0 + c / kc32, n = nt * BN + rr;
+                    if (c < total) {
+                        uint4 *dst = reinterpret_cast<uint4 *>(args.wring + ((int64_t)slot * BN + rr) * args.K) +
+                                     4 * (c - (rr - r0) * kc32);
+                        if (n < args.N) {
+                            dq_convert_store<MODE>(raw[u], dst);
+                        } else {
+#pragma unroll
+                            for (int j = 0; j < 4; ++j)
+                                dst[j] = make_uint4(0u, 0u, 0u, 0u);
+                        }
+                    }
                 }
             }
             fence_proxy_async_global();                             // for the TMA loads of other SMs

@@ -303,19 +303,19 @@ SQ_API sq_status sq_linear_fwd(const sq_weight *w, const uint16_t *x, int64_t M,
  * without a device allocator of their own, and latency-critical loops where
  * cudaMalloc (which may synchronise the device, and may fail under memory
  * pressure) is not allowed.  Nothing is allocated: the workspace is a fixed
- * 32 MiB scratch array in libsq's own device memory, one per device.
+ * 96 MiB scratch array in libsq's own device memory, one per device.
  *
  * Same arguments, results and accuracy as sq_linear_fwd, minus (ws,
  * ws_bytes).  scratch_out (host, may be NULL) receives the device address of
  * the scratch this call used; pass it to sq_check_device_status to read the
  * call's device status word.
  *
- * Limit: sq_workspace_bytes(SQ_OP_LINEAR_FWD_NVFP4 or _INT4, M, N, K) must
- * be at most 33554432 (32 MiB); larger shapes return SQ_ERR_WORKSPACE before
- * any work, with the sizes in sq_last_error_detail().  (NVFP4 at N = 16384,
- * K = 6144 fits M up to 8191 rows; the int4 forward, which needs bf16(H x)
- * (M K 2 bytes) and its W ring (8 x 256 x K x 2 bytes), fits for example
- * M = 1536 at N = K = 3072.)
+ * Limit: sq_workspace_bytes(SQ_OP_LINEAR_FWD_NVFP4, _INT4 or _INT8, M, N,
+ * K) must be at most 100663296 (96 MiB); larger shapes return
+ * SQ_ERR_WORKSPACE before any work, with the sizes in
+ * sq_last_error_detail().  (At N = 16384, K = 6144: NVFP4 fits M up to
+ * 26544 rows; int4, which needs bf16(H x) (M K 2 bytes) and its W ring
+ * (8 x 256 x K x 2 bytes), fits M up to 5734 rows.)
  *
  * The first call on each device looks up the scratch's address
  * (cudaGetSymbolAddress, with that device current), which may load libsq's

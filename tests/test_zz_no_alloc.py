@@ -12,7 +12,7 @@ import torch
 import synth_inputs as si
 from sqcase import FWD_TOL, bf16_dev, host, norm_err, to_dev
 
-SCRATCH_BYTES = 32 << 20
+SCRATCH_BYTES = 96 << 20
 
 
 @pytest.fixture(scope="module")
@@ -29,7 +29,8 @@ def _weight(sq, d, fmt):
 
 @pytest.mark.gpu
 @pytest.mark.parametrize("name,fmt", [("proj_1536x3072x3072", 2), ("tiny_64x256x512", 2),
-                                      ("tiny_64x256x512", 1)], ids=["proj-nvfp4", "tiny-nvfp4", "tiny-int4"])
+                                      ("tiny_64x256x512", 1), ("large_4480x16384x6144", 1)],
+                         ids=["proj-nvfp4", "tiny-nvfp4", "tiny-int4", "large-int4"])
 def test_noalloc_matches_workspace_forward(sq, name, fmt):
     assert torch.cuda.is_available(), "GPU tests need a CUDA device"
     d = si.make_config(name)
@@ -126,16 +127,18 @@ def test_noalloc_variants_match_workspace_forward(sq, variant):
 
 
 def test_noalloc_rejects_shape_beyond_scratch(sq):
-    # NVFP4 at N = 16384, K = 6144 fits M = 8191 rows, not 8192: refused before
-    # any device work (the weight pointers are never touched).
-    fake = 1 << 20
-    w = sq.sq_weight(sq.SQ_FMT_NVFP4, 16384, 6144, fake, fake, fake, fake, fake)
-    assert sq.sq_workspace_bytes(sq.SQ_OP_LINEAR_FWD_NVFP4, 8192, 16384, 6144) > SCRATCH_BYTES
-    assert sq.sq_workspace_bytes(sq.SQ_OP_LINEAR_FWD_NVFP4, 8191, 16384, 6144) <= SCRATCH_BYTES
+    # int4 at N = 16384, K = 6144 fits M = 5734 rows, not 5735 (NVFP4: 26544, not
+    # 26545): refused before any device work (the weight pointers are never touched).
     import ctypes
-    out = ctypes.c_void_p(123)
-    st = sq.lib().sq_linear_fwd_noalloc(ctypes.byref(w), fake, 8192, fake, None, 0, ctypes.byref(out), None)
-    assert sq.status_str(st) == "workspace too small"
-    assert out.value is None
-    detail = sq.lib().sq_last_error_detail().decode()
-    assert "33554432" in detail and "M=8192" in detail
+    fake = 1 << 20
+    for fmt, op, m_max in ((sq.SQ_FMT_INT4_G32, sq.SQ_OP_LINEAR_FWD_INT4, 5734),
+                           (sq.SQ_FMT_NVFP4, sq.SQ_OP_LINEAR_FWD_NVFP4, 26544)):
+        w = sq.sq_weight(fmt, 16384, 6144, fake, fake, fake, fake, fake)
+        assert sq.sq_workspace_bytes(op, m_max + 1, 16384, 6144) > SCRATCH_BYTES
+        assert sq.sq_workspace_bytes(op, m_max, 16384, 6144) <= SCRATCH_BYTES
+        out = ctypes.c_void_p(123)
+        st = sq.lib().sq_linear_fwd_noalloc(ctypes.byref(w), fake, m_max + 1, fake, None, 0, ctypes.byref(out), None)
+        assert sq.status_str(st) == "workspace too small"
+        assert out.value is None
+        detail = sq.lib().sq_last_error_detail().decode()
+        assert "100663296" in detail and f"M={m_max + 1}" in detail
