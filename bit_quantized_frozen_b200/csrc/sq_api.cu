@@ -158,9 +158,17 @@ struct FwdLayout {
     size_t a = 0, a_sf = 0, t32 = 0, tsplit = 0, udup = 0, d32 = 0, u32 = 0, ring = 0, ring_ctr = 0, total = 0;
 };
 
-// slots of the int4 / int8 GEMM's W ring: the W tiles in flight (about 74 clusters over
-// m_tiles of them each) plus room for the writers to run ahead
-constexpr int kRingSlots = 8;
+// slots of the int4 / int8 GEMM's W ring: the W tiles in flight at once (the GEMM's CTA
+// pairs -- 74 on a B200 -- spread over m_tiles clusters per W tile) plus two for the
+// writers to run ahead, never more than there are W tiles.  Fewer slots would still be
+// correct (every wait points at an earlier W tile) but would make tiles wait in turn.
+constexpr int64_t kGemmPairs = 74;
+int64_t ring_slots(int64_t M, int64_t N)
+{
+    const int64_t m_tiles = (M + 255) / 256, n_tiles = (N + 255) / 256;
+    const int64_t want = (kGemmPairs + m_tiles - 1) / m_tiles + 2;
+    return want < n_tiles ? want : n_tiles;
+}
 
 FwdLayout fwd_layout(int fmt, int64_t M, int64_t N, int64_t K)
 {
@@ -178,8 +186,8 @@ FwdLayout fwd_layout(int fmt, int64_t M, int64_t N, int64_t K)
     } else {
         L.a = take((size_t)M * (size_t)K * 2);    // bf16(H x)
         // the GEMM's ring of dequantised 256-row W tiles, and its counters
-        L.ring = take((size_t)kRingSlots * 256 * (size_t)K * 2);
-        L.ring_ctr = take((size_t)2 * kRingSlots * 4);
+        L.ring = take((size_t)ring_slots(M, N) * 256 * (size_t)K * 2);
+        L.ring_ctr = take((size_t)2 * ring_slots(M, N) * 4);
     }
     L.t32 = take((size_t)sq::act_t_parts(M, K) * (size_t)M * 32 * 4);   // partial tiles of t
     L.tsplit = take((size_t)M * 64 * 2);
@@ -502,7 +510,7 @@ sq_status sq_linear_fwd(const sq_weight *w, const uint16_t *x, int64_t M, void *
     g.udup = udup;
     SQ_CUDA(cudaMemsetAsync(status, 0, 8, s), "memset");   // status word + absmax
     if (w->fmt != SQ_FMT_NVFP4)       // the W ring's counters (before every kernel of the call)
-        SQ_CUDA(cudaMemsetAsync(ws_at(ws, L.ring_ctr), 0, (size_t)2 * kRingSlots * 4, s), "memset");
+        SQ_CUDA(cudaMemsetAsync(ws_at(ws, L.ring_ctr), 0, (size_t)2 * ring_slots(M, N) * 4, s), "memset");
     if (flags & SQ_CHECK_FINITE)
         SQ_CUDA(sq::launch_check_finite_bf16(x, M * K, status, sms, s), "finite check");
     if (w->fmt == SQ_FMT_NVFP4) {
@@ -566,7 +574,7 @@ sq_status sq_linear_fwd(const sq_weight *w, const uint16_t *x, int64_t M, void *
         g.b_scales = w->scales;
         g.wring = reinterpret_cast<uint16_t *>(ws_at(ws, L.ring));
         g.ring_ctr = reinterpret_cast<uint32_t *>(ws_at(ws, L.ring_ctr));
-        g.ring_slots = kRingSlots;
+        g.ring_slots = (int)ring_slots(M, N);
     }
     SQ_CUDA(stage_event(SQ_STAGE_GEMM, 0, s), "event record");
     SQ_CUDA(sq::launch_gemm(g, sms, s), "gemm");

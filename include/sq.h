@@ -277,10 +277,11 @@ SQ_API sq_status sq_act_quant_nvfp4(const uint16_t *x, int64_t M, int64_t K,
  *          y = g_x g_w acc + t lora_up^T.
  *   int4:  "dequant-first": xb = bf16(H x), wb = bf16(q s), y = xb wb^T +
  *          t lora_up^T on bf16 tensor cores (fp32 accumulation); either
- *          group size (SQ_FMT_INT4_G32 / _G64).  wb is never stored whole:
- *          the GEMM's own warps dequantise each 256-row tile of W once into
- *          a ring of 8 such tiles in the workspace (8 x 256 x K bf16), from
- *          which the GEMM loads it, so the workspace does not grow with N.
+ *          group size (SQ_FMT_INT4_G32 / _G64).  The GEMM's own warps
+ *          dequantise each 256-row tile of W once into a ring of R such tiles
+ *          in the workspace (R x 256 x K bf16), from which the GEMM loads it;
+ *          R = min(ceil(N / 256), ceil(74 / ceil(M / 256)) + 2), the tiles in
+ *          flight at once: at M = 4480, 7 tiles whatever N is.
  *   int8:  the same with wb = bf16(RN(q s_row)) and the rank-16 branch
  *          (SQ_FMT_INT8_ROW; workspace op SQ_OP_LINEAR_FWD_INT8).
  * The low-rank term is accumulated on the tensor cores in the same
@@ -315,7 +316,8 @@ SQ_API sq_status sq_linear_fwd(const sq_weight *w, const uint16_t *x, int64_t M,
  * SQ_ERR_WORKSPACE before any work, with the sizes in
  * sq_last_error_detail().  (At N = 16384, K = 6144: NVFP4 fits M up to
  * 26544 rows; int4, which needs bf16(H x) (M K 2 bytes) and its W ring
- * (8 x 256 x K x 2 bytes), fits M up to 5734 rows.)
+ * (R x 256 x K x 2 bytes, see sq_linear_fwd), fits M from 513 to 6536
+ * rows; below 513 rows R grows towards all 64 tiles of W.)
  *
  * The first call on each device looks up the scratch's address
  * (cudaGetSymbolAddress, with that device current), which may load libsq's

@@ -67,13 +67,16 @@ def test_size_helpers():
     ws = sq.sq_workspace_bytes(sq.SQ_OP_LINEAR_FWD_NVFP4, 64, 256, 512)
     # activation codes + scales, fp32 t, [t_hi | t_lo], [U | U]
     assert ws >= 64 * 256 + sq.sq_sf_bytes(64, 512) + 64 * 32 * 4 + 64 * 128 + 256 * 128
-    # int4: bf16(H x), fp32 t, [t_hi | t_lo], [U | U]; no bf16 copy of W (the GEMM makes
-    # bf16(q s) in shared memory), so doubling N adds only the [U | U] rows
+    # int4: bf16(H x), fp32 t, [t_hi | t_lo], [U | U] and the GEMM's ring of dequantised
+    # 256-row W tiles (as many as are in flight: 7 at M = 4480); no bf16 copy of W, so
+    # doubling N adds only the [U | U] rows
     wsi = sq.sq_workspace_bytes(sq.SQ_OP_LINEAR_FWD_INT4, 64, 256, 512)
-    assert wsi >= 64 * 512 * 2 + 64 * 32 * 4 + 64 * 128 + 256 * 128
+    assert wsi >= 64 * 512 * 2 + 64 * 32 * 4 + 64 * 128 + 256 * 128 + 256 * 512 * 2
     for op in (sq.SQ_OP_LINEAR_FWD_INT4, sq.SQ_OP_LINEAR_FWD_INT8):
-        grow = sq.sq_workspace_bytes(op, 64, 4096, 4096) - sq.sq_workspace_bytes(op, 64, 2048, 4096)
+        grow = sq.sq_workspace_bytes(op, 4480, 4096, 4096) - sq.sq_workspace_bytes(op, 4480, 2048, 4096)
         assert 2048 * 128 <= grow <= 2048 * 128 * 2 + 4096
+        ring7 = 7 * 256 * 4096 * 2
+        assert sq.sq_workspace_bytes(op, 4480, 4096, 4096) >= 4480 * 4096 * 2 + ring7
     # int8: the int4 layout plus the rank-16 factors widened to rank 32
     assert sq.sq_workspace_bytes(sq.SQ_OP_LINEAR_FWD_INT8, 64, 256, 512) >= wsi + (512 + 256) * 64
     assert sq.sq_workspace_bytes(99, 1, 1, 1) == 0

@@ -127,11 +127,11 @@ def test_noalloc_variants_match_workspace_forward(sq, variant):
 
 
 def test_noalloc_rejects_shape_beyond_scratch(sq):
-    # int4 at N = 16384, K = 6144 fits M = 5734 rows, not 5735 (NVFP4: 26544, not
+    # int4 at N = 16384, K = 6144 fits M = 6536 rows, not 6537 (NVFP4: 26544, not
     # 26545): refused before any device work (the weight pointers are never touched).
     import ctypes
     fake = 1 << 20
-    for fmt, op, m_max in ((sq.SQ_FMT_INT4_G32, sq.SQ_OP_LINEAR_FWD_INT4, 5734),
+    for fmt, op, m_max in ((sq.SQ_FMT_INT4_G32, sq.SQ_OP_LINEAR_FWD_INT4, 6536),
                            (sq.SQ_FMT_NVFP4, sq.SQ_OP_LINEAR_FWD_NVFP4, 26544)):
         w = sq.sq_weight(fmt, 16384, 6144, fake, fake, fake, fake, fake)
         assert sq.sq_workspace_bytes(op, m_max + 1, 16384, 6144) > SCRATCH_BYTES
