@@ -1386,11 +1386,16 @@ constexpr int kWsP2Warps = 8;
 constexpr int kWsP1Threads = 32 * kWsP1Warps;
 constexpr int kWsThreads = 32 * (kWsP1Warps + kWsP2Warps);
 
+// lora_up of a tile in fp32 for the consumers: [rows][rank] (W^T), or [rank][rows + 4]
+// (W: thread reads of four consecutive rows of one rank are one 16-byte broadcast)
+constexpr int kUsTStride = kRecRows + 4;
+
 template <int FMT>
 struct RecWsCfg {
     using C = RecCfg<FMT>;
+    static constexpr int kUsBytes = C::kRank * kUsTStride * 4 > C::kUsBytes ? C::kRank * kUsTStride * 4 : C::kUsBytes;
     static constexpr int kUsOff = 2 * kRecHBytes;                     // h[2] at 0
-    static constexpr int kStageOff = kUsOff + 2 * C::kUsBytes;        // us[2]
+    static constexpr int kStageOff = kUsOff + 2 * kUsBytes;           // us[2]
     static constexpr int kBarOff = kStageOff + 2 * C::kStageBytes;    // stage[2]
     static constexpr int kSmem = kBarOff + 8 * 8 + 16;                // 8 mbarriers, abort flag
 };
@@ -1460,7 +1465,7 @@ __global__ void __launch_bounds__(kWsThreads, 1) reconstruct_ws_kernel(const uin
                 break;
             const uint8_t *st = rec_smem + L::kStageOff + sb * Cfg::kStageBytes;
             float *h = reinterpret_cast<float *>(rec_smem + sb * kRecHBytes);
-            float *us = reinterpret_cast<float *>(rec_smem + L::kUsOff + sb * Cfg::kUsBytes);
+            float *us = reinterpret_cast<float *>(rec_smem + L::kUsOff + sb * L::kUsBytes);
 #pragma unroll 1
             for (int pass = 0; pass < kRecRows / (4 * kWsP1Warps); ++pass) {
                 const int r = 4 * kWsP1Warps * pass + 4 * warp + (lane >> 3);
@@ -1477,8 +1482,14 @@ __global__ void __launch_bounds__(kWsThreads, 1) reconstruct_ws_kernel(const uin
             }
             const uint16_t *ust = reinterpret_cast<const uint16_t *>(st + Cfg::kCodeBytes + kRecScaleBytes);
 #pragma unroll
-            for (int j = 0; j < kRecRows * kR / kWsP1Threads; ++j)
-                us[tid + kWsP1Threads * j] = bf16_bits_to_f32(ust[tid + kWsP1Threads * j]);
+            for (int j = 0; j < kRecRows * kR / kWsP1Threads; ++j) {
+                const int e = tid + kWsP1Threads * j;          // element (row e / kR, rank e % kR)
+                const float u = bf16_bits_to_f32(ust[e]);
+                if (TRANS)
+                    us[e] = u;
+                else
+                    us[(e % kR) * kUsTStride + e / kR] = u;
+            }
             __syncwarp();
             if (lane == 0) {
                 mbar_arrive(h_full + 8 * sb);
@@ -1495,6 +1506,84 @@ __global__ void __launch_bounds__(kWsThreads, 1) reconstruct_ws_kernel(const uin
     }
 
     // ---------------------------------------------------------------- consumer
+    if (!TRANS) {
+        // W: thread t takes columns k0 = 2 (t % 128), k0 + 1 and rows 32 (t / 128) .. + 31, four
+        // rows at a time.  The packed lanes of an fma run over two rows of one column: the
+        // column's lora_down value is the duplicated operand (duplicated once per 256-column
+        // block, in registers), and the rows' lora_up values come as ready pairs from one
+        // 16-byte broadcast load of the transposed us -- no move per fma.  Each (row, column)
+        // is still its own chain fma(U[n, r], D[k, r], L) for r = 0, 1, .. in order.
+        const int ct = tid - kWsP1Threads;
+        const int cp = ct & 127;
+        const int rbase = 32 * (ct >> 7);
+        const int f = cp >> 1;                       // float4 of h holding columns 2cp, 2cp+1
+        const int fo = 2 * (cp & 1);
+        uint64_t dd0[kR], dd1[kR];                   // (D[k0, r], D[k0, r]) and (D[k0 + 1, r], D[k0 + 1, r])
+        int64_t cur_kb = -1;
+#pragma unroll 1
+        for (int i = 0; i < n_tiles; ++i) {
+            const int sb = i & 1;
+            const int64_t t = t_begin + i;
+            const int64_t kb = t / NT;
+            const int64_t n0 = (t % NT) * kRecRows;
+            const int64_t k0 = kb * kHad + 2 * cp;
+            if (kb != cur_kb) {
+                cur_kb = kb;
+                const uint4 *dr0 = reinterpret_cast<const uint4 *>(D + k0 * kR);
+                const uint4 *dr1 = reinterpret_cast<const uint4 *>(D + (k0 + 1) * kR);
+#pragma unroll
+                for (int k = 0; k < kR / 8; ++k) {
+                    const uint4 a = __ldg(dr0 + k), b = __ldg(dr1 + k);
+                    const uint32_t wa[4] = {a.x, a.y, a.z, a.w}, wb[4] = {b.x, b.y, b.z, b.w};
+#pragma unroll
+                    for (int j = 0; j < 4; ++j) {
+                        const float a0 = bf16_bits_to_f32(wa[j] & 0xFFFFu), a1 = bf16_bits_to_f32(wa[j] >> 16);
+                        const float b0 = bf16_bits_to_f32(wb[j] & 0xFFFFu), b1 = bf16_bits_to_f32(wb[j] >> 16);
+                        dd0[8 * k + 2 * j] = pack2(a0, a0);
+                        dd0[8 * k + 2 * j + 1] = pack2(a1, a1);
+                        dd1[8 * k + 2 * j] = pack2(b0, b0);
+                        dd1[8 * k + 2 * j + 1] = pack2(b1, b1);
+                    }
+                }
+            }
+            if (!mbar_wait(h_full + 8 * sb, (uint32_t)(i >> 1) & 1u, abort_flag, status))
+                break;
+            const float *h = reinterpret_cast<const float *>(rec_smem + sb * kRecHBytes);
+            const float *us = reinterpret_cast<const float *>(rec_smem + L::kUsOff + sb * L::kUsBytes);
+#pragma unroll 2
+            for (int r0 = rbase; r0 < rbase + 32; r0 += 4) {
+                // a01 / a23: rows (r0, r0 + 1) / (r0 + 2, r0 + 3) of column k0; b01 / b23 of k0 + 1
+                uint64_t a01 = 0ull, a23 = 0ull, b01 = 0ull, b23 = 0ull;
+#pragma unroll
+                for (int rr = 0; rr < kR; ++rr) {
+                    const ulonglong2 u = *reinterpret_cast<const ulonglong2 *>(us + rr * kUsTStride + r0);
+                    fma2(a01, u.x, dd0[rr]);
+                    fma2(a23, u.y, dd0[rr]);
+                    fma2(b01, u.x, dd1[rr]);
+                    fma2(b23, u.y, dd1[rr]);
+                }
+                float La[4], Lb[4];
+                unpack2(a01, La[0], La[1]);
+                unpack2(a23, La[2], La[3]);
+                unpack2(b01, Lb[0], Lb[1]);
+                unpack2(b23, Lb[2], Lb[3]);
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                    const int r = r0 + j;
+                    const int64_t n = n0 + r;
+                    const float2 hv = *reinterpret_cast<const float2 *>(h + r * kHad + 4 * (f ^ (f >> 3)) + fo);
+                    const float o0 = __fadd_rn(La[j], hv.x);   // W = bf16(RN(L + h))
+                    const float o1 = __fadd_rn(Lb[j], hv.y);
+                    if (n < N && SQ_DCHECK(k0 + 1 < K, status))
+                        *reinterpret_cast<uint32_t *>(W + n * K + k0) = f32x2_to_bf16x2_bits(o0, o1);
+                }
+            }
+            __syncwarp();
+            if (lane == 0)
+                mbar_arrive(h_free + 8 * sb);          // h and us of this tile are no longer read
+        }
+        return;
+    }
     const int ct = tid - kWsP1Threads;
     const int cp = ct & 127;
     const int rbase = 32 * (ct >> 7);
@@ -1527,7 +1616,7 @@ __global__ void __launch_bounds__(kWsThreads, 1) reconstruct_ws_kernel(const uin
         if (!mbar_wait(h_full + 8 * sb, (uint32_t)(i >> 1) & 1u, abort_flag, status))
             break;
         const float *h = reinterpret_cast<const float *>(rec_smem + sb * kRecHBytes);
-        const float *us = reinterpret_cast<const float *>(rec_smem + L::kUsOff + sb * Cfg::kUsBytes);
+        const float *us = reinterpret_cast<const float *>(rec_smem + L::kUsOff + sb * L::kUsBytes);
         uint32_t tw0[16], tw1[16];                   // TRANS: columns k0, k0 + 1 of the 32 rows, bf16 pairs
         constexpr int kUnroll = TRANS ? 8 : 1;       // register-indexed pieces need constant indices
 #pragma unroll kUnroll

@@ -101,6 +101,14 @@ def test_linear_fwd_g64_edge_shapes(sq, shape):
     check_fwd(sq, si.make_inputs(M, K, N, 200 + M))
 
 
+def test_linear_fwd_g64_ring_slot_reuse(sq):
+    """M = 2560 (10 M tiles) and N = 4096 (16 W tiles): the GEMM's W ring has ceil(74 / 10) + 2
+    = 10 slots, so six slots take a second W tile.  Sampled rows, the last M tile's among them."""
+    d = si.make_inputs(2560, 512, 4096, 244)
+    rows = np.unique(np.concatenate([sample_rows(2560, 40, 45), np.arange(2552, 2560)])).astype(np.int64)
+    check_fwd(sq, d, rows)
+
+
 def test_linear_fwd_g64_without_lowrank(sq):
     check_fwd(sq, si.make_inputs(150, 512, 256, 43), lora=False)
 

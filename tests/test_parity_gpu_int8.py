@@ -111,6 +111,15 @@ def test_linear_fwd_int8_edge_shapes(sq, shape):
     check_fwd(sq, si.make_inputs(M, K, N, 300 + M))
 
 
+def test_linear_fwd_int8_ring_slot_reuse(sq):
+    """M = 2560 (10 M tiles) and N = 4096 (16 W tiles): the GEMM's W ring has
+    ceil(74 / 10) + 2 = 10 slots, so six slots take a second W tile once its ten clusters are
+    done with the first.  Sampled rows, the last M tile's among them."""
+    d = si.make_inputs(2560, 512, 4096, 355)
+    rows = np.unique(np.concatenate([sample_rows(2560, 40, 56), np.arange(2552, 2560)])).astype(np.int64)
+    check_fwd(sq, d, rows)
+
+
 def test_linear_fwd_int8_without_lowrank(sq):
     check_fwd(sq, si.make_inputs(150, 512, 256, 54), lora=False)
 
