@@ -447,7 +447,7 @@ sq_status sq_act_quant_nvfp4(const uint16_t *x, int64_t M, int64_t K, uint8_t *c
         SQ_CUDA(sq::launch_check_finite_bf16(x, M * K, reinterpret_cast<uint32_t *>(ws), sms, s), "finite check");
     if (!stat || with_t) {
         SQ_CUDA(stage_event(SQ_STAGE_ACT_PASS1, 0, s), "event record");
-        SQ_CUDA(sq::launch_act_pass1(x, M, K, lora_down, stat ? nullptr : amax, t_part,
+        SQ_CUDA(sq::launch_act_pass1(x, M, K, lora_down, stat ? nullptr : amax, t_part, nullptr,
                                      reinterpret_cast<uint32_t *>(ws), sms, s),
                 "activation pass 1");
         SQ_CUDA(stage_event(SQ_STAGE_ACT_PASS1, 1, s), "event record");
@@ -520,7 +520,7 @@ sq_status sq_linear_fwd(const sq_weight *w, const uint16_t *x, int64_t M, void *
         // one read of x for the absmax and the low-rank input, one for the quantisation
         if (!stat || lora) {
             SQ_CUDA(stage_event(SQ_STAGE_ACT_PASS1, 0, s), "event record");
-            SQ_CUDA(sq::launch_act_pass1(x, M, K, w->lora_down, stat ? nullptr : amax, t32, status, sms, s),
+            SQ_CUDA(sq::launch_act_pass1(x, M, K, w->lora_down, stat ? nullptr : amax, t32, nullptr, status, sms, s),
                     "activation pass 1");
             SQ_CUDA(stage_event(SQ_STAGE_ACT_PASS1, 1, s), "event record");
         }
@@ -548,24 +548,26 @@ sq_status sq_linear_fwd(const sq_weight *w, const uint16_t *x, int64_t M, void *
         g.g_x = gx;
         g.g_w = w->g_w;
     } else {
-        // dequant-first: the GEMM makes bf16(q s) from the payload in shared memory
+        // dequant-first: one read of x gives xb = bf16(H x) and t = x lora_down; the GEMM
+        // dequantises W itself (its W ring)
         uint16_t *xb = reinterpret_cast<uint16_t *>(ws_at(ws, L.a));
-        SQ_CUDA(sq::launch_rotate_bf16(x, M, K, xb, sms, s), "rotate x");
-        if (lora) {
-            const uint16_t *Dw = w->lora_down, *Uw = w->lora_up;
-            if (w->fmt == SQ_FMT_INT8_ROW) {          // rank 16: zero columns 16..31
-                uint16_t *d32 = reinterpret_cast<uint16_t *>(ws_at(ws, L.d32));
-                uint16_t *u32 = reinterpret_cast<uint16_t *>(ws_at(ws, L.u32));
-                SQ_CUDA(sq::launch_widen_rank16(w->lora_down, K, d32, sms, s), "widen lora_down");
-                SQ_CUDA(sq::launch_widen_rank16(w->lora_up, N, u32, sms, s), "widen lora_up");
-                Dw = d32;
-                Uw = u32;
-            }
-            SQ_CUDA(sq::launch_act_pass1(x, M, K, Dw, nullptr, t32, status, sms, s), "low-rank input");
+        const uint16_t *Dw = w->lora_down, *Uw = w->lora_up;
+        if (lora && w->fmt == SQ_FMT_INT8_ROW) {      // rank 16: zero columns 16..31
+            uint16_t *d32 = reinterpret_cast<uint16_t *>(ws_at(ws, L.d32));
+            uint16_t *u32 = reinterpret_cast<uint16_t *>(ws_at(ws, L.u32));
+            SQ_CUDA(sq::launch_widen_rank16(w->lora_down, K, d32, sms, s), "widen lora_down");
+            SQ_CUDA(sq::launch_widen_rank16(w->lora_up, N, u32, sms, s), "widen lora_up");
+            Dw = d32;
+            Uw = u32;
+        }
+        SQ_CUDA(stage_event(SQ_STAGE_ACT_PASS1, 0, s), "event record");
+        SQ_CUDA(sq::launch_act_pass1(x, M, K, lora ? Dw : nullptr, nullptr, lora ? t32 : nullptr, xb, status, sms, s),
+                "rotate x and low-rank input");
+        SQ_CUDA(stage_event(SQ_STAGE_ACT_PASS1, 1, s), "event record");
+        if (lora)
             SQ_CUDA(sq::launch_lowrank_finish(t32, sq::act_t_parts(M, K), M, nullptr, nullptr, tsplit, Uw, N, udup,
                                               sms, s),
                     "low-rank operands");
-        }
         g.mode = w->fmt == SQ_FMT_INT8_ROW ? sq::kGemmInt8
                  : w->fmt == SQ_FMT_INT4_G64 ? sq::kGemmInt4G64
                                              : sq::kGemmInt4G32;

@@ -42,10 +42,9 @@ cudaError_t launch_int4_build(const float *R, int64_t N, int64_t K, int group, u
 cudaError_t launch_int8_build(const float *R, int64_t N, int64_t K, int8_t *codes, float *scales, uint8_t *frac,
                               int sms, cudaStream_t s);
 cudaError_t launch_widen_rank16(const uint16_t *src, int64_t rows, uint16_t *dst, int sms, cudaStream_t s);
-cudaError_t launch_rotate_bf16(const uint16_t *x, int64_t M, int64_t K, uint16_t *xb, int sms, cudaStream_t s);
 // t_part: act_t_parts(M, K) partial tiles [parts, M, 32] (NULL: no t)
 cudaError_t launch_act_pass1(const uint16_t *x, int64_t M, int64_t K, const uint16_t *D, uint32_t *amax,
-                             float *t_part, uint32_t *status, int sms, cudaStream_t s);
+                             float *t_part, uint16_t *xb, uint32_t *status, int sms, cudaStream_t s);
 cudaError_t launch_lowrank_finish(const float *t_part, int parts, int64_t M, const float *g_x, const float *g_w,
                                   uint16_t *tsplit, const uint16_t *U, int64_t N, uint16_t *udup, int sms,
                                   cudaStream_t s);

@@ -612,32 +612,12 @@ __global__ void __launch_bounds__(256) widen_rank16_kernel(const uint4 *__restri
 }
 
 // ---------------------------------------------------------------------------
-// int4 forward prologue: xb = bf16(H x), [M, K]
-// ---------------------------------------------------------------------------
-__global__ void __launch_bounds__(kStreamThreads) rotate_bf16_kernel(const __grid_constant__ CUtensorMap tm,
-                                                                     int64_t blocks, uint16_t *__restrict__ xb)
-{
-    const int lane = threadIdx.x & 31;
-    stream_blocks<uint16_t>(&tm, blocks, nullptr, [&](int64_t b, float (&v)[32], bool valid) {
-        fwht256_l32(v, lane);
-        if (!valid)
-            return;
-        uint4 *o = reinterpret_cast<uint4 *>(xb + b * kHad + 32 * (lane & 7));
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-            uint32_t w[4];
-#pragma unroll
-            for (int j = 0; j < 4; ++j)
-                w[j] = f32x2_to_bf16x2_bits(v[8 * i + 2 * j], v[8 * i + 2 * j + 1]);
-            o[i] = make_uint4(w[0], w[1], w[2], w[3]);
-        }
-    });
-}
-
-// ---------------------------------------------------------------------------
-// Activation pass 1: one read of x for two results.
+// Activation pass 1: one read of x for up to three results.
 //   amax (optional):   max |H x| over the whole tensor (the activation global
 //                      scale's input), from the 4-lane Hadamard transform;
+//   xb (optional):     bf16(H x) [M, K], the A operand of the int4 / int8
+//                      forward (the same transform, then the exact 1/16 and one
+//                      rounding to bf16);
 //   t_part (optional): t = x . lora_down on the tcgen05 tensor cores (fp32
 //                      accumulation in tensor memory), as `split` partial
 //                      [M, 32] tiles, one per range of K, which the consumer
@@ -712,6 +692,7 @@ __global__ void __launch_bounds__(kP1Threads, 1) act_pass1_kernel(const __grid_c
                                                                   const __grid_constant__ CUtensorMap tmd,
                                                                   int64_t M, int64_t K, uint32_t *__restrict__ amax,
                                                                   float *__restrict__ t_part, int split,
+                                                                  uint16_t *__restrict__ xb,
                                                                   uint32_t *__restrict__ status)
 {
     float *const t32 = t_part;                        // non-NULL: this CTA writes partial tile j of t
@@ -735,7 +716,7 @@ __global__ void __launch_bounds__(kP1Threads, 1) act_pass1_kernel(const __grid_c
     if (tid == 0) {
         for (int st = 0; st < kP1Stages; ++st) {
             mbar_init(full + 8 * st, 1);
-            mbar_init(empty + 8 * st, (amax ? kP1Consumers : 0) + (t32 ? 1 : 0));
+            mbar_init(empty + 8 * st, ((amax || xb) ? kP1Consumers : 0) + (t32 ? 1 : 0));
         }
         mbar_init(done, 1);
         *abort_flag = 0u;
@@ -795,10 +776,11 @@ __global__ void __launch_bounds__(kP1Threads, 1) act_pass1_kernel(const __grid_c
             tc_commit(done);
         }
         __syncwarp();
-    } else if (amax) {                                // consumers: Hadamard absmax
+    } else if (amax || xb) {                          // consumers: Hadamard absmax and / or bf16(H x)
         // lane (q, r) = (lane / 8, lane % 8) holds quarter q of row 8 warp + r: 64 values of box q
         const int q = lane >> 3;
         const int R = 8 * warp + (lane & 7);
+        const bool row_live = m0 + R < M;
         for (int c = 0; c < nch; ++c) {
             const int st = c % kP1Stages;
             const uint32_t ph = (uint32_t)(c / kP1Stages) & 1u;
@@ -813,11 +795,30 @@ __global__ void __launch_bounds__(kP1Threads, 1) act_pass1_kernel(const __grid_c
             if (lane == 0)
                 mbar_arrive(empty + 8 * st);              // the stage's rows are in registers
             fwht256_q4_from_s2(p, lane);
+            if (amax) {
 #pragma unroll
-            for (int i = 0; i < 32; ++i) {
-                float lo, hi;
-                f2_unpack(p[i], lo, hi);
-                m = fmax3(m, fabsf(lo), fabsf(hi));
+                for (int i = 0; i < 32; ++i) {
+                    float lo, hi;
+                    f2_unpack(p[i], lo, hi);
+                    m = fmax3(m, fabsf(lo), fabsf(hi));
+                }
+            }
+            if (xb && row_live) {                     // bf16(H x): elements 64q .. 64q+63 of the block
+                const int64_t col = (int64_t)(kb0 + c) * kHad + 64 * q;
+                if (SQ_DCHECK(col + 64 <= K, status)) {
+                    uint4 *o = reinterpret_cast<uint4 *>(xb + (m0 + R) * K + col);
+#pragma unroll
+                    for (int k = 0; k < 8; ++k) {
+                        uint32_t w4[4];
+#pragma unroll
+                        for (int jj = 0; jj < 4; ++jj) {
+                            float lo, hi;
+                            f2_unpack(p[4 * k + jj], lo, hi);
+                            w4[jj] = f32x2_to_bf16x2_bits(__fmul_rn(lo, 0.0625f), __fmul_rn(hi, 0.0625f));
+                        }
+                        o[k] = make_uint4(w4[0], w4[1], w4[2], w4[3]);
+                    }
+                }
             }
         }
     }
@@ -843,9 +844,7 @@ __global__ void __launch_bounds__(kP1Threads, 1) act_pass1_kernel(const __grid_c
         }
         tc_fence_before();
         const int64_t row = m0 + 32 * warp + lane;
-        if (row < M) {
-            if (!SQ_DCHECK(j < split, status))
-                return;
+        if (row < M && SQ_DCHECK(j < split, status)) {
             float4 *o = reinterpret_cast<float4 *>(t32 + ((int64_t)j * M + row) * kRank);
 #pragma unroll
             for (int i = 0; i < 32; i += 4)
@@ -1922,21 +1921,8 @@ cudaError_t launch_widen_rank16(const uint16_t *src, int64_t rows, uint16_t *dst
     return cudaGetLastError();
 }
 
-cudaError_t launch_rotate_bf16(const uint16_t *x, int64_t M, int64_t K, uint16_t *xb, int sms, cudaStream_t s)
-{
-    CUtensorMap tm;
-    if (!stream_map(&tm, x, M, K))
-        return cudaErrorInvalidValue;
-    cudaError_t e = stream_attr<uint16_t, rotate_bf16_kernel>();
-    if (e != cudaSuccess)
-        return e;
-    const int64_t blocks = M * (K / kHad);
-    rotate_bf16_kernel<<<stream_grid(blocks, sms, 3), kStreamThreads, StreamCfg<uint16_t>::kSmem, s>>>(tm, blocks, xb);
-    return cudaGetLastError();
-}
-
 cudaError_t launch_act_pass1(const uint16_t *x, int64_t M, int64_t K, const uint16_t *D, uint32_t *amax,
-                             float *t_part, uint32_t *status, int sms, cudaStream_t s)
+                             float *t_part, uint16_t *xb, uint32_t *status, int sms, cudaStream_t s)
 {
     (void)sms;
     constexpr int kMaxDev = 64;
@@ -1962,7 +1948,7 @@ cudaError_t launch_act_pass1(const uint16_t *x, int64_t M, int64_t K, const uint
     const int64_t tiles = (M + kP1Rows - 1) / kP1Rows;
     const int split = act_t_parts(M, K);
     act_pass1_kernel<<<(unsigned)(tiles * split), kP1Threads, kP1Smem, s>>>(tmx, tmd, M, K, amax, t_part, split,
-                                                                            status);
+                                                                            xb, status);
     return cudaGetLastError();
 }
 
