@@ -33,14 +33,16 @@
 //              multiplies into the ring (see "W ring" below), from the start of
 //              the kernel (they read only the weight payload, not the outputs of
 //              the preceding kernels).
-// Tensor memory (512 columns): two accumulator slots at columns 0 and 64
-// that overlap in columns 64..255, and four 48-column scale-factor buffers at
-// 320..511 (NVFP4: four stages of scale factors between the scale warps and
-// the MMAs that read them).  The epilogue takes the overlapping 192 columns
-// of a tile first -- four chunks into registers, two of them parked in its
-// staging buffers, then the last two -- and releases the MMA thread, which
-// starts the next tile while the rest drains: accumulator double buffering
-// in 320 columns.
+// Tensor memory (512 columns).  NVFP4: two accumulator slots at columns 0 and
+// 64 that overlap in columns 64..255, and four 48-column scale-factor buffers
+// at 320..511 (four stages of scale factors between the scale warps and the
+// MMAs that read them).  The epilogue takes the overlapping 192 columns of a
+// tile first -- four chunks into registers, two of them parked in its staging
+// buffers, then the last two -- and releases the MMA thread, which starts the
+// next tile while the rest drains: accumulator double buffering in 320
+// columns.  bf16 / int4 / int8 (no scale factors): two disjoint slots, [0, 256)
+// and [256, 512); the epilogue drains its slot chunk by chunk and releases it
+// for the tile after next, so the MMAs never wait for it.
 #include <cuda.h>
 
 #include "sq_device.cuh"
