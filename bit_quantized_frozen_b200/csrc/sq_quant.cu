@@ -1,15 +1,17 @@
 // sq_quant.cu -- the non-GEMM kernels of the SquareQ W4 layer: the NVFP4
 // builder (Hadamard-256 + tensor absmax, then block quantisation into the
 // tiled scale layout), the int4 and int8 builders with their scale-fraction
-// sweeps, the activation prologue of the NVFP4 forward (absmax + t on tcgen05,
-// then quantisation), the bf16 rotation and dequant of the "dequant-first"
-// int4 / int8 forwards, the low-rank operands, and the bf16 reconstructs.
+// sweeps, the activation prologue of the forwards (absmax, bf16(H x) and t on
+// tcgen05 in one read of x, then the NVFP4 quantisation), the low-rank
+// operands, and the bf16 reconstructs.  (The int4 / int8 weight is
+// dequantised inside the GEMM, sq_gemm.cu.)
 //
-// What bounds each: the builders' passes and the residual-only reconstruct
-// stream HBM; the int4 / int8 builders are bound by the FP32 / ALU issue of
-// their 26-trial sweeps; the reconstruct with the low-rank term by the FMA
-// pipe (its rank-r fmaf chain); the activation passes by the L1 data pipe
-// (Hadamard shuffles) and the FP32 pipe.  Persistent grids are sized from the
+// What bounds each: the NVFP4 builder's passes stream HBM; the int4 / int8
+// builders are bound by the FP32 / ALU issue of their 26-trial sweeps; the
+// reconstruct with the low-rank term by the FMA pipe (its rank-r fmaf chain)
+// and the latency of its decode and transform; the activation passes and the
+// residual-only reconstruct by the L1 data pipe (Hadamard shuffles) and the
+// FP32 pipe, below their HBM floors.  Persistent grids are sized from the
 // SM count; loads and stores are contiguous per warp or go through TMA.  They
 // follow the SquareQ README, section "SquareQ v3 -- W4", as stated operation
 // by operation in include/sq.h.
